@@ -1,0 +1,121 @@
+"""Pins for the oracle's block rotations (Hadamard-32 and Kronecker A(x)B).
+
+Checked against explicit matrices built here from their closed forms
+(H_ij = (-1)^popcount(i & j) / sqrt(32); (A(x)B)[8i+k, 8j+l] = A_ij B_kl via
+numpy.kron), orthogonality / invertibility identities, and the fp32 error
+bounds of the stated evaluation orders.
+"""
+import math
+from decimal import Decimal, getcontext
+
+import numpy as np
+
+import oracle
+import synth
+
+
+def _sylvester(n=32):
+    i = np.arange(n)
+    pc = np.vectorize(lambda v: bin(v).count("1"))(i[:, None] & i[None, :])
+    return np.where(pc % 2 == 0, 1.0, -1.0)
+
+
+def test_inv_sqrt32_is_nearest_fp32():
+    getcontext().prec = 60
+    exact = Decimal(1) / Decimal(32).sqrt()
+    c = oracle.inv_sqrt32()
+    lo = np.nextafter(c, np.float32(0))
+    hi = np.nextafter(c, np.float32(1))
+    err = abs(Decimal(float(c)) - exact)
+    assert err <= abs(Decimal(float(lo)) - exact)
+    assert err <= abs(Decimal(float(hi)) - exact)
+
+
+def test_unnormalised_butterfly_is_sylvester_integer_exact():
+    H = _sylvester()
+    cols = np.stack([oracle.fwht32_unnormalised(np.eye(32, dtype=np.float32)[j]) for j in range(32)],
+                    axis=1)
+    assert np.array_equal(cols, H)                   # column j = H e_j, exact integers
+    assert np.array_equal(cols @ cols.T, 32 * np.eye(32))
+
+
+def test_hadamard_orthonormal_in_fp32():
+    Hn = oracle.rotate_blocks(np.eye(32, dtype=np.float32), oracle.ROT_HADAMARD32)
+    # rows of the block-rotated identity are H e_j (H is symmetric)
+    G = Hn.astype(np.float64) @ Hn.astype(np.float64).T
+    assert np.max(np.abs(G - np.eye(32))) < 1e-6
+
+
+def test_hadamard_matches_explicit_matrix():
+    H = _sylvester() / math.sqrt(32.0)
+    x = synth.normal_f32(0, 999, (200, 32))
+    x[:, 3] *= 50.0
+    y = oracle.rotate_blocks(x, oracle.ROT_HADAMARD32).astype(np.float64)
+    ref = x.astype(np.float64) @ H.T
+    # 5 add stages + 1 multiply: relative error per element <= ~6u of sum |x|/sqrt(32)
+    bound = 8 * 2.0 ** -24 * (np.abs(x).astype(np.float64).sum(axis=1, keepdims=True) / math.sqrt(32))
+    assert np.all(np.abs(y - ref) <= bound + 1e-30)
+    # involution: H (H x) = x within fp32 error
+    yy = oracle.rotate_blocks(y.astype(np.float32), oracle.ROT_HADAMARD32).astype(np.float64)
+    assert np.max(np.abs(yy - x) / (np.abs(x).max(axis=1, keepdims=True))) < 1e-5
+
+
+def test_kron_matches_numpy_kron():
+    A, B = synth.kron_factors(0)
+    T = np.kron(A.astype(np.float64), B.astype(np.float64))
+    x = synth.normal_f32(0, 998, (300, 32))
+    y = oracle.rotate_blocks(x, oracle.ROT_KRON_4x8, A, B).astype(np.float64)
+    ref = x.astype(np.float64) @ T.T
+    absT = np.kron(np.abs(A).astype(np.float64), np.abs(B).astype(np.float64))
+    bound = 16 * 2.0 ** -24 * (np.abs(x).astype(np.float64) @ absT.T)
+    assert np.all(np.abs(y - ref) <= bound)
+
+
+def test_kron_identity_factors_is_identity():
+    x = synth.normal_f32(0, 997, (10, 32))
+    y = oracle.rotate_blocks(x, oracle.ROT_KRON_4x8, np.eye(4), np.eye(8))
+    assert np.array_equal(y, x)
+
+
+def test_kron_weight_factors_invert():
+    A, B = synth.kron_factors(0)
+    assert abs(np.linalg.det(A.astype(np.float64))) > 1e-3
+    assert abs(np.linalg.det(B.astype(np.float64))) > 1e-3
+    Ai = oracle.inverse(A)
+    Bi = oracle.inverse(B)
+    I = np.kron(A.astype(np.float64), B.astype(np.float64)) @ np.kron(Ai, Bi)
+    assert np.max(np.abs(I - np.eye(32))) < 1e-12
+    At, Bt = oracle.kron_weight_factors(A, B)
+    assert np.max(np.abs(At.astype(np.float64) - Ai.T)) < 1e-6
+    assert np.max(np.abs(Bt.astype(np.float64) - Bi.T)) < 1e-6
+
+
+def test_rotation_invariance_of_dot_products():
+    """(H x).(H w) = x.w and (T x).(T^-T w) = x.w, evaluated through the oracle's
+    fp32 rotations: catches transposed factors and wrong conventions."""
+    x = synth.normal_f32(0, 996, (64, 32))
+    w = synth.normal_f32(0, 995, (64, 32), 0.02)
+    base = np.sum(x.astype(np.float64) * w.astype(np.float64), axis=1)
+    scale = np.sqrt(np.sum(x.astype(np.float64) ** 2, 1) * np.sum(w.astype(np.float64) ** 2, 1))
+    hx = oracle.rotate_blocks(x, oracle.ROT_HADAMARD32).astype(np.float64)
+    hw = oracle.rotate_blocks(w, oracle.ROT_HADAMARD32).astype(np.float64)
+    assert np.max(np.abs(np.sum(hx * hw, 1) - base) / scale) < 1e-5
+    A, B = synth.kron_factors(0)
+    At, Bt = oracle.kron_weight_factors(A, B)
+    tx = oracle.rotate_blocks(x, oracle.ROT_KRON_4x8, A, B).astype(np.float64)
+    tw = oracle.rotate_blocks(w, oracle.ROT_KRON_4x8, At, Bt).astype(np.float64)
+    assert np.max(np.abs(np.sum(tx * tw, 1) - base) / scale) < 1e-4
+    # and a wrong convention (T^-1 instead of T^-T on w) breaks it
+    Ai, Bi = oracle.inverse(A).astype(np.float32), oracle.inverse(B).astype(np.float32)
+    bad = oracle.rotate_blocks(w, oracle.ROT_KRON_4x8, Ai, Bi).astype(np.float64)
+    assert np.max(np.abs(np.sum(tx * bad, 1) - base) / scale) > 1e-3
+
+
+def test_rotate_quantize_composes_rotation_and_quantisation():
+    xb, _ = synth.activation_bf16(0, 8, 256, 0.02, 20.0)
+    x32 = synth.bf16_bits_to_f32(xb)
+    q, s = oracle.rotate_quantize(xb, oracle.ROT_HADAMARD32)
+    y = oracle.rotate_blocks(x32.reshape(-1, 32), oracle.ROT_HADAMARD32)
+    codes, sc = oracle.quantize_blocks(y)
+    assert np.array_equal(oracle.unpack_codes(q).reshape(-1, 32), codes)
+    assert np.array_equal(s.reshape(-1), sc)
