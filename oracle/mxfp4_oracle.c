@@ -41,7 +41,8 @@
  *    in fp32, then one fp32 multiply by the fp32 value nearest 1/sqrt(32).
  *  - Kronecker: T = A (x) B, A 4x4, B 8x8, one T shared by every block;
  *    y[8i+k] = sum_j A[i][j] * z[8j+k], z[8j+k] = sum_l B[k][l] * x[8j+l],
- *    each sum an fp32 fmaf chain in ascending index order starting from +0.
+ *    each sum in fp32 as the first product (one rounding) followed by fmaf
+ *    steps in ascending index order.
  *    Weights take T^-T = A^-T (x) B^-T (inverses in double, rounded to fp32).
  *  - Packing: byte j of a row holds element 2j in bits 0-3 and element 2j+1
  *    in bits 4-7.
@@ -176,14 +177,14 @@ void oracle_kron32(const float* A, const float* B, const float* x, float* y) {
   float z[32];
   for (int j = 0; j < 4; ++j)
     for (int k = 0; k < 8; ++k) {
-      float acc = 0.0f;
-      for (int l = 0; l < 8; ++l) acc = fmaf(B[k * 8 + l], x[8 * j + l], acc);
+      float acc = B[k * 8 + 0] * x[8 * j + 0];
+      for (int l = 1; l < 8; ++l) acc = fmaf(B[k * 8 + l], x[8 * j + l], acc);
       z[8 * j + k] = acc;
     }
   for (int i = 0; i < 4; ++i)
     for (int k = 0; k < 8; ++k) {
-      float acc = 0.0f;
-      for (int j = 0; j < 4; ++j) acc = fmaf(A[i * 4 + j], z[8 * j + k], acc);
+      float acc = A[i * 4 + 0] * z[8 * 0 + k];
+      for (int j = 1; j < 4; ++j) acc = fmaf(A[i * 4 + j], z[8 * j + k], acc);
       y[8 * i + k] = acc;
     }
 }
