@@ -1,0 +1,445 @@
+"""Benchmark of the MXFP4 W4A4 linear block on B200.
+
+One step = the whole hot path over one batch: for every linear of the
+workload, online block rotation + MXFP4 quantisation of X and the tcgen05
+block-scaled GEMM against pre-quantised weights (bf16 out), through the
+library's public call ``mxfp4_linear``. Default workload: the FLUX-like DiT
+block at batch 1 (3584 tokens): QKV 3072->9216 and MLP-up 3072->12288 on X, and
+MLP-down 12288->3072 on the 3584 x 12288 activation.
+
+Prints ONE JSON line (rank 0). ``value`` = TFLOPS of the whole job (2*M*N*K
+summed over linears and ranks / max-over-ranks device time), inputs resident
+in HBM. ``e2e`` = the same metric through the same public call from host
+buffers (pinned H2D of X, D2H of Y inside the timed region). ``roofline`` =
+the GEMM kernel against the FP4 tensor peak, ``quantize_roofline`` = the
+rotate+quantise kernel against HBM bandwidth, both from CUDA events around
+each kernel launch in an attribution pass over the same steps.
+
+--impl reference times the CPU oracle (the plain C implementation that
+defines the results) on a bounded row sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import synth  # noqa: E402
+
+METRIC = "MXFP4 W4A4 linear TFLOPS & % FP4 peak; quantize GB/s & % HBM peak"
+UNIT = "TFLOPS"
+FP4_OVER_BF16 = 4.0  # nominal dense FP4 : BF16 tensor throughput on B200 (9 : 2.25 PFLOP/s)
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="dit_b1", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p["bf16_tflops_sustained"], "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+def workload_desc(wl) -> str:
+    parts = [f"{l.name} {l.M}x{l.K}->{l.N}" for l in wl.linears]
+    rot = {0: "no rotation", 1: "Hadamard-32", 2: "Kronecker 4x8"}[wl.rotation]
+    return f"{wl.name}: " + ", ".join(parts) + f"; {rot}"
+
+
+# --------------------------------------------------------------------------- CPU oracle
+
+def oracle_sample_time(wl, budget_s: float = 12.0):
+    """Time the oracle (rotate+quantise + exact contraction) on a row sample of
+    every linear; return (TFLOPS extrapolated to the full workload, sample text,
+    seconds spent)."""
+    import oracle
+    A = B = None
+    if wl.rotation == synth.ROT_KRON_4x8:
+        A, B = synth.kron_factors(wl.seed)
+    prepared = []
+    for lin in wl.linears:
+        w = synth.weight_f32(wl.seed, lin.N, lin.K, lin.layer)
+        wq, ws = oracle.prepare_weight(w, wl.rotation, A, B)
+        prepared.append((lin, wq, ws))
+
+    def run(rows):
+        t0 = time.perf_counter()
+        for lin, wq, ws in prepared:
+            r = min(rows, lin.M)
+            x, _ = synth.activation_bf16(wl.seed, r, lin.K, lin.outlier_frac, lin.outlier_factor,
+                                         lin.x_tensor)
+            oracle.linear(x, wq, ws, wl.rotation, A, B)
+        return time.perf_counter() - t0
+
+    rows = 1
+    t = run(rows)
+    while t < budget_s / 8 and rows < min(l.M for l in wl.linears):
+        rows *= 2
+        t = run(rows)
+    sample_flops = sum(2 * min(rows, l.M) * l.N * l.K for l in wl.linears)
+    tflops = sample_flops / t / 1e12
+    sample = (f"{rows} rows of every linear (all N, all K): rotate+quantise of those rows and the "
+              f"exact block-scaled products, {t:.2f} s; extrapolated linearly in rows")
+    return tflops, sample, t
+
+
+def cpu_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+# --------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# --------------------------------------------------------------------------- GPU arm
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+
+    import mxfp4_quantized_linear_block_b200 as mx
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    wl = synth.WORKLOADS[args.workload]
+    peaks = load_peaks()
+    A = B = None
+    if wl.rotation == synth.ROT_KRON_4x8:
+        A, B = synth.kron_factors(wl.seed)
+    Aw, Bw = (mx.kron_weight_factors(A, B) if A is not None else (None, None))
+
+    # ---- inputs: weights prepared on the GPU (offline step, untimed)
+    weights = []
+    for lin in wl.linears:
+        w = torch.from_numpy(synth.weight_f32(wl.seed, lin.N, lin.K, lin.layer)).to(dev)
+        wq, wsf = mx.rotate_quantize(w, wl.rotation, Aw, Bw)
+        del w
+        weights.append((wq, wsf))
+    xs_host = {}
+    for lin in wl.linears:
+        if lin.x_tensor not in xs_host:
+            # each rank takes its own token slice of a weak-scaled batch: same shapes, own draws
+            x, _ = synth.activation_bf16(wl.seed + rank, lin.M, lin.K, lin.outlier_frac,
+                                         lin.outlier_factor, lin.x_tensor)
+            xs_host[lin.x_tensor] = x
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+
+    def make_set():
+        xs = {k: torch.from_numpy(v.view(np.int16)).view(torch.bfloat16).to(dev)
+              for k, v in xs_host.items()}
+        ys = [torch.empty((l.M, l.N), dtype=torch.bfloat16, device=dev) for l in wl.linears]
+        wss = [mx.new_workspace(mx.workspace_bytes(mx.OP_LINEAR, l.M, l.N, l.K), dev)
+               for l in wl.linears]
+        return xs, ys, wss
+
+    def set_bytes(s):
+        xs, ys, wss = s
+        return (sum(t.numel() * t.element_size() for t in xs.values()) +
+                sum(t.numel() * 2 for t in ys) + sum(t.numel() for t in wss))
+
+    w_bytes = sum(wq.numel() + wsf.numel() for wq, wsf in weights)
+    sets = [make_set()]
+    while (len(sets) * set_bytes(sets[0]) + w_bytes) < 3 * l2 and len(sets) < 8:
+        sets.append(make_set())
+    footprint = len(sets) * set_bytes(sets[0]) + w_bytes
+
+    stream = torch.cuda.current_stream(dev)
+
+    def step(i):
+        xs, ys, wss = sets[i % len(sets)]
+        for j, lin in enumerate(wl.linears):
+            wq, wsf = weights[j]
+            mx.linear(xs[lin.x_tensor], wq, wsf, lin.N, wl.rotation, A, B, y=ys[j], ws=wss[j],
+                      stream=stream)
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    def max_over_ranks(v: float) -> float:
+        if world == 1:
+            return v
+        import torch.distributed as dist
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    # ---- warm-up
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+
+    # ---- timed region: K steps through the public call, inputs resident in HBM
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    barrier()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for i in range(args.steps):
+        step(i)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    elapsed = max_over_ranks(ev0.elapsed_time(ev1) * 1e-3)
+    flops_step = wl.flops
+    value = flops_step * args.steps * world / elapsed / 1e12
+    ms_per_step = elapsed / args.steps * 1e3
+    launches = 2 * len(wl.linears) * args.steps
+
+    # status words: no bounded wait expired
+    for s in sets:
+        for ws in s[2]:
+            if mx.poll_status(ws) != mx.OK:
+                raise RuntimeError("a kernel reported a bounded-wait timeout")
+
+    # ---- attribution pass: the same steps as separate quantise / GEMM launches with
+    # CUDA events around each kernel (on the launching stream)
+    qbufs = [(torch.empty((l.M, l.K // 2), dtype=torch.uint8, device=dev),
+              torch.empty(mx.sf_bytes(l.M, l.K), dtype=torch.uint8, device=dev)) for l in wl.linears]
+    gws = mx.new_workspace(mx.workspace_bytes(mx.OP_GEMM, 1, 16, 32), dev)
+    n_lin = len(wl.linears)
+    evs = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+             torch.cuda.Event(enable_timing=True)) for _ in range(n_lin)] for _ in range(args.steps)]
+
+    def step_split(i, rec):
+        xs, ys, _ = sets[i % len(sets)]
+        for j, lin in enumerate(wl.linears):
+            wq, wsf = weights[j]
+            q, sf = qbufs[j]
+            if rec:
+                evs[i][j][0].record(stream)
+            mx.rotate_quantize(xs[lin.x_tensor], wl.rotation, A, B, q=q, sf=sf, stream=stream)
+            if rec:
+                evs[i][j][1].record(stream)
+            mx.gemm(q, sf, wq, wsf, lin.M, lin.N, lin.K, y=ys[j], ws=gws, stream=stream)
+            if rec:
+                evs[i][j][2].record(stream)
+
+    for i in range(args.warmup):
+        step_split(i, False)
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        step_split(i, True)
+    torch.cuda.synchronize()
+    t_q = np.zeros(n_lin)
+    t_g = np.zeros(n_lin)
+    for i in range(args.steps):
+        for j in range(n_lin):
+            a, b, c = evs[i][j]
+            t_q[j] += a.elapsed_time(b) * 1e-3
+            t_g[j] += b.elapsed_time(c) * 1e-3
+    t_q /= args.steps
+    t_g /= args.steps
+    gemm_flops = np.array([l.flops for l in wl.linears], dtype=np.float64)
+    gemm_bytes = np.array([l.M * l.K // 2 + mx.sf_bytes(l.M, l.K) + l.N * l.K // 2 +
+                           mx.sf_bytes(l.N, l.K) + 2 * l.M * l.N for l in wl.linears], np.float64)
+    q_bytes = np.array([2 * l.M * l.K + l.M * l.K // 2 + mx.sf_bytes(l.M, l.K)
+                        for l in wl.linears], np.float64)
+    fp4_peak = peaks["bf16_tflops_sustained"] * FP4_OVER_BF16
+    g_ach = gemm_flops.sum() / t_g.sum() / 1e12
+    q_ach = q_bytes.sum() / t_q.sum() / 1e9
+
+    # ---- end to end: host (pinned) X in, host Y out, inside the timed region
+    e2e = None
+    if args.e2e_steps > 0:
+        xs_pin = {k: torch.from_numpy(v.view(np.int16)).view(torch.bfloat16).pin_memory()
+                  for k, v in xs_host.items()}
+        ys_pin = [torch.empty((l.M, l.N), dtype=torch.bfloat16).pin_memory() for l in wl.linears]
+        xs_d, ys_d, wss_d = sets[0]
+        h2d = sum(t.numel() * 2 for t in xs_pin.values())
+        d2h = sum(t.numel() * 2 for t in ys_pin)
+
+        def e2e_step():
+            for k, t in xs_pin.items():
+                xs_d[k].copy_(t, non_blocking=True)
+            for j, lin in enumerate(wl.linears):
+                wq, wsf = weights[j]
+                mx.linear(xs_d[lin.x_tensor], wq, wsf, lin.N, wl.rotation, A, B, y=ys_d[j],
+                          ws=wss_d[j], stream=stream)
+                ys_pin[j].copy_(ys_d[j], non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        t_e2e = max_over_ranks(a.elapsed_time(b) * 1e-3)
+        e2e = {"value": flops_step * args.e2e_steps * world / t_e2e / 1e12, "unit": UNIT,
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "ms_per_step": t_e2e / args.e2e_steps * 1e3}
+        launches_e2e = 2 * len(wl.linears) * args.e2e_steps
+    else:
+        launches_e2e = 0
+
+    result = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "mxfp4",
+        "dtype_detail": "E2M1 x E2M1 with E8M0 block-32 scales, fp32 accumulate, bf16 out; "
+                        "rotation in fp32",
+        "data": "synthetic (seeded N(0,1) activations with outlier channels, N(0,0.02^2) weights)",
+        "config": {"workload": workload_desc(wl), "tokens_per_gpu": wl.linears[0].M,
+                   "gflop_per_step_per_gpu": flops_step / 1e9, "parallelism": f"replicas x{world} "
+                   "(token-parallel, no collective)",
+                   "l2": f"{len(sets)} rotating input/output sets, footprint "
+                         f"{footprint / 2**20:.0f} MiB >= 3 x L2 ({l2 / 2**20:.0f} MiB)"},
+        "roofline": {"bound": "tensor", "kernel": "mxf4_gemm_kernel (tcgen05 kind::mxf4)",
+                     "achieved": g_ach, "peak": fp4_peak, "unit": "TFLOP/s",
+                     "frac": g_ach / fp4_peak,
+                     "peak_source": f"4 x {peaks['source']} bf16 sustained "
+                                    f"({peaks['bf16_tflops_sustained']} TFLOP/s)",
+                     "per_launch": [{"linear": l.name, "us": t_g[j] * 1e6,
+                                     "tflops": gemm_flops[j] / t_g[j] / 1e12,
+                                     "alg_bytes": int(gemm_bytes[j])}
+                                    for j, l in enumerate(wl.linears)],
+                     "traffic": None},
+        "quantize_roofline": {"bound": "hbm", "kernel": "rotate_quantize_kernel",
+                              "achieved": q_ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                              "frac": q_ach / peaks["hbm_gbs"],
+                              "per_launch_us": [t * 1e6 for t in t_q],
+                              "alg_bytes_per_launch": [int(b) for b in q_bytes],
+                              "traffic": None},
+        "e2e": e2e,
+        "gpu_launches": launches + launches_e2e,
+        "clocks": clk,
+    }
+    return result
+
+
+# --------------------------------------------------------------------------- reference arm
+
+def run_reference(args):
+    wl = synth.WORKLOADS[args.workload]
+    per = max(2.0, 60.0 / max(1, args.steps + args.warmup))
+    vals = []
+    samples = []
+    for i in range(args.warmup + args.steps):
+        v, sample, t = oracle_sample_time(wl, budget_s=per)
+        if i >= args.warmup:
+            vals.append(v)
+            samples.append(sample)
+    value = statistics.median(vals)
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": wl.flops / (value * 1e12) * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "mxfp4",
+        "data": "synthetic", "config": {"workload": workload_desc(wl)},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
+                         "sample": samples[-1]},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        res = run_ours(args, rank, world, local_rank)
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            v, sample, _ = oracle_sample_time(synth.WORKLOADS[args.workload])
+            res["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cpu_cores(),
+                                   "kind": "oracle", "sample": sample}
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,177 @@
+/*
+ * mxfp4.h -- C ABI of libmxfp4, the MXFP4 W4A4 linear block for NVIDIA B200 (sm_100a).
+ *
+ * The layer computes Y = X . W^T in three steps:
+ *   1. an online block-local rotation of every 32-element block of X
+ *      (normalised 32x32 Sylvester Hadamard, "Bridging the Gap Between Promise
+ *      and Performance for Microscaling FP4 Quantization", "Methodologie:
+ *      MR-GPTQ" item 1 and "GPU Kernel Ondersteuning (QuTLASS)"; or a learned
+ *      Kronecker-factored A (x) B transform, "KroQuant: Effiziente Post-
+ *      Training-Quantisierung fuer Diffusion Transformers mittels Kronecker-
+ *      Produkt-Struktur", "Tiefenanalyse");
+ *   2. MXFP4 quantisation: one E8M0 power-of-two scale per 32-element block
+ *      and 4-bit E2M1 elements ("AMD Quark delivers MXFP4 quantization for
+ *      FLUX.1-dev on Instinct MI350 with 1.92x speedup", "What is MXFP4 and
+ *      why does it eliminate dequantization overhead?"; "Bridging the Gap...",
+ *      "Probleemstelling" item 2);
+ *   3. a block-scaled FP4 x FP4 GEMM against pre-quantised MXFP4 weights with
+ *      fp32 accumulation and bf16 (or fp32) output, with no dequantisation to
+ *      bf16 in between (AMD Quark page, opening section).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - All pointers named x, q, sf, aq, asf, bq, bsf, wq, wsf, y, ws are DEVICE
+ *    pointers owned by the caller; the library keeps no reference after the
+ *    call returns and allocates no device memory. kron_a / kron_b are HOST
+ *    pointers (the transform is passed by value to the kernel).
+ *  - Every launch is asynchronous and ordered on `stream` (a cudaStream_t;
+ *    NULL = the legacy default stream).
+ *  - Argument errors are detected on the host before any launch and launch
+ *    nothing: NULL pointer -> MXFP4_ERR_INVALID_ARG; bad sizes ->
+ *    MXFP4_ERR_SHAPE; misaligned pointer or row stride -> MXFP4_ERR_ALIGN;
+ *    workspace too small -> MXFP4_ERR_WORKSPACE; unknown mode / dtype ->
+ *    MXFP4_ERR_UNSUPPORTED. A failed launch returns MXFP4_ERR_CUDA.
+ *    rows == 0 (or M == 0) is a valid empty call: nothing is launched.
+ *  - Packed E2M1 codes ("q" operands): row-major [rows, K/2] bytes; byte j of a
+ *    row holds element 2j in bits 0-3 and element 2j+1 in bits 4-7; bit 3 of a
+ *    code is the sign, codes 0..7 are 0, 0.5, 1, 1.5, 2, 3, 4, 6.
+ *  - E8M0 scale bytes ("sf" operands), byte b meaning 2^(b-127), 0xFF = NaN,
+ *    are stored in the tensor-core scale layout: rows are tiled by 128 and
+ *    32-element blocks by 4 into 512-byte atoms, atoms ordered block-group
+ *    fastest then row tile, and inside an atom (row r, block kb) sits at byte
+ *    (r % 32) * 16 + ((r / 32) % 4) * 4 + kb % 4. The buffer holds
+ *    mxfp4_sf_bytes(rows, K) bytes; padding rows/blocks are written as 0 by the
+ *    quantisers and must be 0 (or any finite scale) in caller-made buffers.
+ *  - Scale rule: e = floor(log2(amax)) - 2 clamped to [-127, 127] (byte
+ *    e + 127) where amax is the block's largest magnitude after rotation;
+ *    elements are round(y * 2^-e) to the nearest E2M1 value, ties to even,
+ *    saturating at +-6; the sign is kept (code 8 for negatives rounding to 0).
+ *    An all-zero block gets byte 0; a block with a non-finite value after
+ *    rotation gets byte 0xFF and all-zero codes.
+ */
+#ifndef MXFP4_H_
+#define MXFP4_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MXFP4_OK = 0,
+  MXFP4_ERR_INVALID_ARG = 1,
+  MXFP4_ERR_SHAPE = 2,
+  MXFP4_ERR_ALIGN = 3,
+  MXFP4_ERR_WORKSPACE = 4,
+  MXFP4_ERR_UNSUPPORTED = 5,
+  MXFP4_ERR_CUDA = 6,
+  MXFP4_ERR_TIMEOUT = 7
+} mxfp4_status;
+
+typedef enum {
+  MXFP4_ROT_NONE = 0,       /* plain MXFP4 quantisation */
+  MXFP4_ROT_HADAMARD32 = 1, /* y = H32 x, H32 = H2^(x5) / sqrt(32) (Sylvester order) */
+  MXFP4_ROT_KRON_4x8 = 2    /* y = (A (x) B) x, A 4x4, B 8x8 */
+} mxfp4_rotation;
+
+typedef enum { MXFP4_DT_BF16 = 0, MXFP4_DT_F32 = 1 } mxfp4_dtype;
+
+typedef enum { MXFP4_OP_QUANTIZE = 0, MXFP4_OP_GEMM = 1, MXFP4_OP_LINEAR = 2 } mxfp4_op;
+
+/* A cudaStream_t, passed as an opaque handle so this header needs no CUDA headers. */
+typedef void* mxfp4_stream_t;
+
+/* Bytes of the scale-factor buffer for a [rows, K] operand:
+ * ceil(rows / 128) * 128 * ceil(K / 128) * 4. K % 32 == 0. Returns 0 on bad sizes. */
+size_t mxfp4_sf_bytes(int64_t rows, int64_t K);
+
+/* Byte offset of the scale of (row, 32-element block kblock) in that buffer, or -1 if out of range. */
+int64_t mxfp4_sf_offset(int64_t row, int64_t kblock, int64_t K);
+
+/* Device workspace that `op` needs for this problem (0 if none). For
+ * MXFP4_OP_LINEAR it holds the quantised activations and a status word. */
+size_t mxfp4_workspace_bytes(int op, int64_t M, int64_t N, int64_t K);
+
+/* Static description of a status code. Never NULL. */
+const char* mxfp4_status_string(mxfp4_status status);
+
+/*
+ * Quantise x[rows, K] (leading dimension ldx elements, bf16 or fp32) to MXFP4
+ * with no rotation: q = packed codes [rows, K/2], sf = scale bytes in the
+ * tensor-core layout (mxfp4_sf_bytes(rows, K) bytes, padding written as 0).
+ * Steps 2 of the layer ("What is MXFP4..." on the AMD Quark page; RTN
+ * quantiser of "Bridging the Gap...", "Probleemstelling").
+ * Requirements: K % 32 == 0, ldx >= K, x 16-byte aligned and ldx * elemsize a
+ * multiple of 16; q and sf 16-byte aligned.
+ */
+mxfp4_status mxfp4_quantize(const void* x, mxfp4_dtype xdt, int64_t rows, int64_t K, int64_t ldx,
+                            uint8_t* q, uint8_t* sf, mxfp4_stream_t stream);
+
+/*
+ * Rotate each 32-element block of x in fp32 (mode), then quantise as
+ * mxfp4_quantize. Hadamard: a five-stage butterfly (strides 1, 2, 4, 8, 16;
+ * (a, b) -> (a + b, a - b)) then one multiply by the fp32 value nearest
+ * 1/sqrt(32) ("Bridging the Gap...", "Methodologie: MR-GPTQ" item 1).
+ * Kronecker: z[8j+k] = sum_l B[k][l] x[8j+l], y[8i+k] = sum_j A[i][j] z[8j+k],
+ * each sum in fp32 as the first product followed by fma steps in ascending
+ * index order ("KroQuant...",
+ * "Tiefenanalyse"). kron_a (16 floats) and kron_b (64 floats) are HOST
+ * pointers, row-major, read during the call; NULL for the other modes. To
+ * prepare weights for the Kronecker mode pass A^-T and B^-T here
+ * (T^-T = A^-T (x) B^-T, "KroQuant...", "Hintergrund": the inverse goes on
+ * the weights).
+ */
+mxfp4_status mxfp4_rotate_quantize(const void* x, mxfp4_dtype xdt, int64_t rows, int64_t K,
+                                   int64_t ldx, mxfp4_rotation mode, const float* kron_a,
+                                   const float* kron_b, uint8_t* q, uint8_t* sf,
+                                   mxfp4_stream_t stream);
+
+/*
+ * Block-scaled GEMM on the tcgen05 tensor cores (kind::mxf4):
+ * y[m][n] = sum_b 2^(asf[m,b] + bsf[n,b] - 254) * sum_{i in b} v(aq[m,i]) v(bq[n,i]),
+ * accumulated in fp32, written as bf16 (round to nearest even) or fp32.
+ * aq/asf: [M, K] operand (activations), bq/bsf: [N, K] operand (weights),
+ * both in the formats above. y: row-major [M, N] with leading dimension ldy
+ * elements. Requirements: K % 32 == 0, N % 16 == 0, ldy >= N, y 16-byte aligned
+ * and ldy * elemsize a multiple of 16; aq, bq, asf, bsf 16-byte aligned.
+ * ws must hold mxfp4_workspace_bytes(MXFP4_OP_GEMM, M, N, K) bytes (at least
+ * 256); its first 16 bytes are the device status word (see mxfp4_poll_status).
+ * ("AMD Quark...", opening section: MXFP4 GEMM with no dequantisation;
+ * "Bridging the Gap...", "GPU Kernel Ondersteuning (QuTLASS)".)
+ */
+mxfp4_status mxfp4_gemm(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq,
+                        const uint8_t* bsf, int64_t M, int64_t N, int64_t K, void* y,
+                        mxfp4_dtype ydt, int64_t ldy, void* ws, size_t ws_bytes,
+                        mxfp4_stream_t stream);
+
+/*
+ * The whole layer: rotate + quantise x (bf16 [M, K], row stride K) into the
+ * workspace, then the block-scaled GEMM with the pre-quantised weights
+ * (wq/wsf: [N, K] operand prepared offline with the matching rotation), bf16
+ * output y[M, N] (row stride N). ws must hold
+ * mxfp4_workspace_bytes(MXFP4_OP_LINEAR, M, N, K) bytes. The two kernels run
+ * back to back on `stream`, the second with programmatic dependent launch so
+ * its set-up overlaps the first one's tail.
+ */
+mxfp4_status mxfp4_linear(const void* x, int64_t M, int64_t K, mxfp4_rotation mode,
+                          const float* kron_a, const float* kron_b, const uint8_t* wq,
+                          const uint8_t* wsf, int64_t N, void* y, void* ws, size_t ws_bytes,
+                          mxfp4_stream_t stream);
+
+/*
+ * Read the device status word at the start of a workspace (synchronises with
+ * the device): MXFP4_OK, or MXFP4_ERR_TIMEOUT if a kernel's bounded wait on a
+ * pipeline barrier ran out (the kernel then stopped early, released its
+ * tensor memory and returned; its output is incomplete). The word is sticky:
+ * kernels only ever set it, this call clears it. Zero the first 16 bytes of a
+ * workspace once when it is allocated.
+ */
+mxfp4_status mxfp4_poll_status(void* ws, mxfp4_status* out);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MXFP4_H_ */

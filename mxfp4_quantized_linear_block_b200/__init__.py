@@ -1,0 +1,203 @@
+"""Python binding of libmxfp4, the MXFP4 W4A4 linear block for B200 (sm_100a).
+
+Argument marshalling only: every step of the layer (rotation, quantisation,
+block-scaled GEMM) runs in the library's CUDA kernels. PyTorch provides device
+memory and the current stream. If ``libmxfp4.so`` is missing the import fails;
+there is no fallback of any kind.
+
+Functions mirror the C ABI in ``include/mxfp4.h``:
+``quantize``, ``rotate_quantize``, ``gemm``, ``linear``, ``poll_status`` and
+the host helpers ``sf_bytes``, ``sf_offset``, ``workspace_bytes``,
+``status_string``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmxfp4.so")
+
+OK, ERR_INVALID_ARG, ERR_SHAPE, ERR_ALIGN, ERR_WORKSPACE, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT = range(8)
+ROT_NONE, ROT_HADAMARD32, ROT_KRON_4x8 = 0, 1, 2
+DT_BF16, DT_F32 = 0, 1
+OP_QUANTIZE, OP_GEMM, OP_LINEAR = 0, 1, 2
+
+EXPORTS = (
+    "mxfp4_sf_bytes", "mxfp4_sf_offset", "mxfp4_workspace_bytes", "mxfp4_status_string",
+    "mxfp4_quantize", "mxfp4_rotate_quantize", "mxfp4_gemm", "mxfp4_linear",
+    "mxfp4_poll_status",
+)
+
+
+class MXFP4Error(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} (status {status})")
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"libmxfp4.so not found at {LIB_PATH}; build it with "
+            "`python -m mxfp4_quantized_linear_block_b200.build` (nvcc, sm_100a)")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+    sig = {
+        "mxfp4_sf_bytes": ([i64, i64], sz),
+        "mxfp4_sf_offset": ([i64, i64, i64], i64),
+        "mxfp4_workspace_bytes": ([i32, i64, i64, i64], sz),
+        "mxfp4_status_string": ([i32], ctypes.c_char_p),
+        "mxfp4_quantize": ([vp, i32, i64, i64, i64, vp, vp, vp], i32),
+        "mxfp4_rotate_quantize": ([vp, i32, i64, i64, i64, i32, vp, vp, vp, vp, vp], i32),
+        "mxfp4_gemm": ([vp, vp, vp, vp, i64, i64, i64, vp, i32, i64, vp, sz, vp], i32),
+        "mxfp4_linear": ([vp, i64, i64, i32, vp, vp, vp, vp, i64, vp, vp, sz, vp], i32),
+        "mxfp4_poll_status": ([vp, vp], i32),
+    }
+    for name, (args, res) in sig.items():
+        f = getattr(lib, name)
+        f.argtypes = args
+        f.restype = res
+    return lib
+
+
+lib = _load()
+
+
+# ---------------------------------------------------------------- host helpers
+
+def sf_bytes(rows: int, K: int) -> int:
+    return lib.mxfp4_sf_bytes(rows, K)
+
+
+def sf_offset(row: int, kblock: int, K: int) -> int:
+    return lib.mxfp4_sf_offset(row, kblock, K)
+
+
+def workspace_bytes(op: int, M: int, N: int, K: int) -> int:
+    return lib.mxfp4_workspace_bytes(op, M, N, K)
+
+
+def status_string(status: int) -> str:
+    return lib.mxfp4_status_string(status).decode()
+
+
+def _check(status: int, where: str) -> None:
+    if status != OK:
+        raise MXFP4Error(status, where)
+
+
+# ---------------------------------------------------------------- device calls
+
+def _torch():
+    import torch
+    return torch
+
+
+def _stream_handle(stream) -> int:
+    torch = _torch()
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _host_f32(a, n: int):
+    """Host float32 copy of a small matrix (Kronecker factor) as a ctypes array."""
+    if a is None:
+        return None
+    try:
+        import numpy as np
+        arr = np.ascontiguousarray(a.detach().cpu().numpy() if hasattr(a, "detach") else a,
+                                   dtype=np.float32).reshape(-1)
+    except Exception as e:  # pragma: no cover
+        raise TypeError(f"Kronecker factor: {e}")
+    if arr.size != n:
+        raise ValueError(f"Kronecker factor must have {n} entries, got {arr.size}")
+    return (ctypes.c_float * n)(*arr.tolist())
+
+
+def _dtype_code(t) -> int:
+    torch = _torch()
+    if t.dtype == torch.bfloat16:
+        return DT_BF16
+    if t.dtype == torch.float32:
+        return DT_F32
+    raise TypeError(f"unsupported dtype {t.dtype} (bf16 or fp32)")
+
+
+def new_workspace(nbytes: int, device=None):
+    """Zero-initialised device workspace (the status word starts cleared)."""
+    torch = _torch()
+    return torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=device or "cuda")
+
+
+def rotate_quantize(x, mode: int = ROT_HADAMARD32, kron_a=None, kron_b=None, q=None, sf=None,
+                    stream=None):
+    """x: [rows, K] bf16/fp32 CUDA tensor (row stride x.stride(0)) ->
+    (q [rows, K/2] uint8 packed E2M1, sf [sf_bytes] uint8 scales in the tensor-core layout)."""
+    torch = _torch()
+    assert x.dim() == 2 and x.stride(1) == 1, "x must be row-major 2-D"
+    rows, K = x.shape
+    if q is None:
+        q = torch.empty((rows, K // 2), dtype=torch.uint8, device=x.device)
+    if sf is None:
+        sf = torch.empty(max(sf_bytes(rows, K), 16), dtype=torch.uint8, device=x.device)
+    a = _host_f32(kron_a, 16) if mode == ROT_KRON_4x8 else None
+    b = _host_f32(kron_b, 64) if mode == ROT_KRON_4x8 else None
+    st = lib.mxfp4_rotate_quantize(x.data_ptr(), _dtype_code(x), rows, K, x.stride(0), mode, a, b,
+                                   q.data_ptr(), sf.data_ptr(), _stream_handle(stream))
+    _check(st, "mxfp4_rotate_quantize")
+    return q, sf
+
+
+def quantize(x, q=None, sf=None, stream=None):
+    """Plain MXFP4 quantisation (no rotation)."""
+    return rotate_quantize(x, ROT_NONE, None, None, q, sf, stream)
+
+
+def gemm(aq, asf, bq, bsf, M: int, N: int, K: int, y=None, out_dtype=None, ws=None, stream=None):
+    """Block-scaled GEMM y[M, N] = A . B^T on the tensor cores (fp32 accumulate)."""
+    torch = _torch()
+    out_dtype = out_dtype or torch.bfloat16
+    if y is None:
+        y = torch.empty((M, N), dtype=out_dtype, device=aq.device)
+    if ws is None:
+        ws = new_workspace(workspace_bytes(OP_GEMM, M, N, K), aq.device)
+    st = lib.mxfp4_gemm(aq.data_ptr(), asf.data_ptr(), bq.data_ptr(), bsf.data_ptr(), M, N, K,
+                        y.data_ptr(), _dtype_code(y), y.stride(0), ws.data_ptr(), ws.numel(),
+                        _stream_handle(stream))
+    _check(st, "mxfp4_gemm")
+    return y
+
+
+def linear(x, wq, wsf, N: int, mode: int = ROT_HADAMARD32, kron_a=None, kron_b=None, y=None,
+           ws=None, stream=None):
+    """The whole layer: y[M, N] (bf16) = MXFP4(rotate(x)) . W^T with pre-quantised W."""
+    torch = _torch()
+    assert x.dim() == 2 and x.is_contiguous() and x.dtype == torch.bfloat16
+    M, K = x.shape
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    if ws is None:
+        ws = new_workspace(workspace_bytes(OP_LINEAR, M, N, K), x.device)
+    a = _host_f32(kron_a, 16) if mode == ROT_KRON_4x8 else None
+    b = _host_f32(kron_b, 64) if mode == ROT_KRON_4x8 else None
+    st = lib.mxfp4_linear(x.data_ptr(), M, K, mode, a, b, wq.data_ptr(), wsf.data_ptr(), N,
+                          y.data_ptr(), ws.data_ptr(), ws.numel(), _stream_handle(stream))
+    _check(st, "mxfp4_linear")
+    return y
+
+
+def poll_status(ws) -> int:
+    out = ctypes.c_int(0)
+    _check(lib.mxfp4_poll_status(ws.data_ptr(), ctypes.byref(out)), "mxfp4_poll_status")
+    return out.value
+
+
+def kron_weight_factors(A, B):
+    """Weight-side factors of the Kronecker mode: (A^-T, B^-T), inverted in float64 on the host
+    (a 4x4 and an 8x8 matrix) and rounded to float32."""
+    import numpy as np
+    A = np.asarray(A, dtype=np.float64)
+    B = np.asarray(B, dtype=np.float64)
+    return (np.linalg.inv(A).T.astype(np.float32).copy(),
+            np.linalg.inv(B).T.astype(np.float32).copy())

@@ -1,0 +1,198 @@
+// abi.cu -- the extern "C" entry points of libmxfp4 (declared in include/mxfp4.h):
+// argument validation, workspace layout and kernel dispatch. No device memory
+// is allocated here; every launch is ordered on the caller's stream.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+
+#include "../../include/mxfp4.h"
+#include "internal.h"
+
+using namespace mxfp4;
+
+namespace {
+
+constexpr size_t kStatusBytes = 256;  // status word region at the start of a workspace
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Valid [rows, K] operand description for the scale layout.
+bool shape_ok(int64_t rows, int64_t K) { return rows >= 0 && K >= 32 && K % 32 == 0; }
+
+// Limits of the kernels' 32-bit index arithmetic.
+bool within_limits(int64_t rows, int64_t K) {
+  const int64_t units = sf_row_tiles(rows) * 128 * sf_katoms(K) * 4;
+  return rows < (1ll << 31) && K < (1ll << 31) && units < (1ll << 32);
+}
+
+mxfp4_status from_cuda(cudaError_t e) { return e == cudaSuccess ? MXFP4_OK : MXFP4_ERR_CUDA; }
+
+mxfp4_status validate_quantize(const void* x, mxfp4_dtype xdt, int64_t rows, int64_t K,
+                               int64_t ldx, const uint8_t* q, const uint8_t* sf) {
+  if (!x || !q || !sf) return MXFP4_ERR_INVALID_ARG;
+  if (xdt != MXFP4_DT_BF16 && xdt != MXFP4_DT_F32) return MXFP4_ERR_UNSUPPORTED;
+  if (!shape_ok(rows, K) || ldx < K || !within_limits(rows, K)) return MXFP4_ERR_SHAPE;
+  const int64_t esize = xdt == MXFP4_DT_F32 ? 4 : 2;
+  if (!aligned16(x) || !aligned16(q) || !aligned16(sf) || (ldx * esize) % 16 != 0)
+    return MXFP4_ERR_ALIGN;
+  return MXFP4_OK;
+}
+
+mxfp4_status validate_gemm(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq,
+                           const uint8_t* bsf, int64_t M, int64_t N, int64_t K, const void* y,
+                           mxfp4_dtype ydt, int64_t ldy) {
+  if (!aq || !asf || !bq || !bsf || !y) return MXFP4_ERR_INVALID_ARG;
+  if (ydt != MXFP4_DT_BF16 && ydt != MXFP4_DT_F32) return MXFP4_ERR_UNSUPPORTED;
+  if (!shape_ok(M, K) || N < 16 || N % 16 != 0 || ldy < N || !within_limits(M, K) ||
+      !within_limits(N, K))
+    return MXFP4_ERR_SHAPE;
+  const int64_t esize = ydt == MXFP4_DT_F32 ? 4 : 2;
+  if (!aligned16(aq) || !aligned16(asf) || !aligned16(bq) || !aligned16(bsf) || !aligned16(y) ||
+      (ldy * esize) % 16 != 0)
+    return MXFP4_ERR_ALIGN;
+  return MXFP4_OK;
+}
+
+bool kron_from_host(const float* a, const float* b, KronCoeffs* out) {
+  if (!a || !b) return false;
+  std::memcpy(out->a, a, sizeof(out->a));
+  std::memcpy(out->b, b, sizeof(out->b));
+  return true;
+}
+
+// Workspace of mxfp4_linear: [status | Xq (M x K/2) | Xsf], each part 256-byte aligned.
+struct LinearWorkspace {
+  size_t q_off, sf_off, total;
+};
+
+LinearWorkspace linear_workspace(int64_t M, int64_t K) {
+  LinearWorkspace w;
+  w.q_off = kStatusBytes;
+  w.sf_off = round_up(w.q_off + (size_t)M * (size_t)(K / 2), 256);
+  w.total = round_up(w.sf_off + mxfp4_sf_bytes(M, K), 256);
+  return w;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t mxfp4_sf_bytes(int64_t rows, int64_t K) {
+  if (!shape_ok(rows, K)) return 0;
+  return (size_t)(sf_row_tiles(rows) * sf_katoms(K) * 512);
+}
+
+int64_t mxfp4_sf_offset(int64_t row, int64_t kblock, int64_t K) {
+  if (K < 32 || K % 32 != 0 || row < 0 || kblock < 0 || kblock >= K / 32) return -1;
+  return ((row / 128) * sf_katoms(K) + kblock / 4) * 512 + (row % 32) * 16 +
+         ((row / 32) % 4) * 4 + (kblock % 4);
+}
+
+size_t mxfp4_workspace_bytes(int op, int64_t M, int64_t N, int64_t K) {
+  (void)N;
+  switch (op) {
+    case MXFP4_OP_QUANTIZE:
+      return 0;
+    case MXFP4_OP_GEMM:
+      return kStatusBytes;
+    case MXFP4_OP_LINEAR:
+      if (!shape_ok(M, K)) return 0;
+      return linear_workspace(M, K).total;
+    default:
+      return 0;
+  }
+}
+
+const char* mxfp4_status_string(mxfp4_status s) {
+  switch (s) {
+    case MXFP4_OK: return "ok";
+    case MXFP4_ERR_INVALID_ARG: return "invalid argument (null pointer)";
+    case MXFP4_ERR_SHAPE: return "unsupported shape";
+    case MXFP4_ERR_ALIGN: return "pointer or row stride not 16-byte aligned";
+    case MXFP4_ERR_WORKSPACE: return "workspace too small";
+    case MXFP4_ERR_UNSUPPORTED: return "unsupported mode or dtype";
+    case MXFP4_ERR_CUDA: return "CUDA launch error";
+    case MXFP4_ERR_TIMEOUT: return "a kernel's bounded wait expired (output incomplete)";
+  }
+  return "unknown status";
+}
+
+mxfp4_status mxfp4_quantize(const void* x, mxfp4_dtype xdt, int64_t rows, int64_t K, int64_t ldx,
+                            uint8_t* q, uint8_t* sf, mxfp4_stream_t stream) {
+  return mxfp4_rotate_quantize(x, xdt, rows, K, ldx, MXFP4_ROT_NONE, nullptr, nullptr, q, sf,
+                               stream);
+}
+
+mxfp4_status mxfp4_rotate_quantize(const void* x, mxfp4_dtype xdt, int64_t rows, int64_t K,
+                                   int64_t ldx, mxfp4_rotation mode, const float* kron_a,
+                                   const float* kron_b, uint8_t* q, uint8_t* sf,
+                                   mxfp4_stream_t stream) {
+  mxfp4_status st = validate_quantize(x, xdt, rows, K, ldx, q, sf);
+  if (st != MXFP4_OK) return st;
+  if (mode != MXFP4_ROT_NONE && mode != MXFP4_ROT_HADAMARD32 && mode != MXFP4_ROT_KRON_4x8)
+    return MXFP4_ERR_UNSUPPORTED;
+  KronCoeffs kc{};
+  if (mode == MXFP4_ROT_KRON_4x8 && !kron_from_host(kron_a, kron_b, &kc))
+    return MXFP4_ERR_INVALID_ARG;
+  if (rows == 0) return MXFP4_OK;
+  return from_cuda(launch_rotate_quantize(x, xdt == MXFP4_DT_F32, rows, K, ldx, (int)mode, &kc, q,
+                                          sf, static_cast<cudaStream_t>(stream)));
+}
+
+mxfp4_status mxfp4_gemm(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq,
+                        const uint8_t* bsf, int64_t M, int64_t N, int64_t K, void* y,
+                        mxfp4_dtype ydt, int64_t ldy, void* ws, size_t ws_bytes,
+                        mxfp4_stream_t stream) {
+  mxfp4_status st = validate_gemm(aq, asf, bq, bsf, M, N, K, y, ydt, ldy);
+  if (st != MXFP4_OK) return st;
+  if (!ws) return MXFP4_ERR_INVALID_ARG;
+  if (!aligned16(ws)) return MXFP4_ERR_ALIGN;
+  if (ws_bytes < mxfp4_workspace_bytes(MXFP4_OP_GEMM, M, N, K)) return MXFP4_ERR_WORKSPACE;
+  if (M == 0) return MXFP4_OK;
+  return from_cuda(launch_gemm(aq, asf, bq, bsf, M, N, K, y, ydt == MXFP4_DT_F32, ldy,
+                               static_cast<int*>(ws), false, static_cast<cudaStream_t>(stream)));
+}
+
+mxfp4_status mxfp4_linear(const void* x, int64_t M, int64_t K, mxfp4_rotation mode,
+                          const float* kron_a, const float* kron_b, const uint8_t* wq,
+                          const uint8_t* wsf, int64_t N, void* y, void* ws, size_t ws_bytes,
+                          mxfp4_stream_t stream) {
+  if (!x || !wq || !wsf || !y || !ws) return MXFP4_ERR_INVALID_ARG;
+  if (mode != MXFP4_ROT_NONE && mode != MXFP4_ROT_HADAMARD32 && mode != MXFP4_ROT_KRON_4x8)
+    return MXFP4_ERR_UNSUPPORTED;
+  if (!shape_ok(M, K) || N < 16 || N % 16 != 0 || !within_limits(M, K) || !within_limits(N, K))
+    return MXFP4_ERR_SHAPE;
+  if (!aligned16(x) || !aligned16(wq) || !aligned16(wsf) || !aligned16(y) || !aligned16(ws) ||
+      (K * 2) % 16 != 0 || (N * 2) % 16 != 0)
+    return MXFP4_ERR_ALIGN;
+  const LinearWorkspace w = linear_workspace(M, K);
+  if (ws_bytes < w.total) return MXFP4_ERR_WORKSPACE;
+  KronCoeffs kc{};
+  if (mode == MXFP4_ROT_KRON_4x8 && !kron_from_host(kron_a, kron_b, &kc))
+    return MXFP4_ERR_INVALID_ARG;
+  if (M == 0) return MXFP4_OK;
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  uint8_t* xq = base + w.q_off;
+  uint8_t* xsf = base + w.sf_off;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_rotate_quantize(x, false, M, K, K, (int)mode, &kc, xq, xsf, s);
+  if (e != cudaSuccess) return MXFP4_ERR_CUDA;
+  return from_cuda(
+      launch_gemm(xq, xsf, wq, wsf, M, N, K, y, false, N, static_cast<int*>(ws), true, s));
+}
+
+mxfp4_status mxfp4_poll_status(void* ws, mxfp4_status* out) {
+  if (!ws || !out) return MXFP4_ERR_INVALID_ARG;
+  int v = 0;
+  if (cudaMemcpy(&v, ws, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return MXFP4_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpy(ws, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
+    return MXFP4_ERR_CUDA;
+  *out = static_cast<mxfp4_status>(v);
+  return MXFP4_OK;
+}
+
+}  // extern "C"

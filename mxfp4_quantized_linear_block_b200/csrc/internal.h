@@ -1,0 +1,33 @@
+// internal.h -- declarations shared by the library's translation units (not installed).
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+namespace mxfp4 {
+
+// Kronecker factors, passed to the kernel by value (constant bank).
+struct KronCoeffs {
+  float a[16];  // A, 4x4 row-major
+  float b[64];  // B, 8x8 row-major
+};
+
+// Rotate (mode 0/1/2) + quantise x[rows, K] (bf16 or fp32) into packed codes q and
+// scale bytes sf (tensor-core layout, padding zeroed). Host-validated arguments.
+cudaError_t launch_rotate_quantize(const void* x, bool x_is_f32, int64_t rows, int64_t K,
+                                   int64_t ldx, int mode, const KronCoeffs* kc, uint8_t* q,
+                                   uint8_t* sf, cudaStream_t stream);
+
+// Block-scaled GEMM y[M, N] = A[M, K] . B[N, K]^T on tcgen05. Host-validated arguments.
+// status: device word set to the timeout code if a bounded wait gives up.
+// pdl: launch with programmatic stream serialization (overlaps the previous kernel's tail).
+cudaError_t launch_gemm(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq,
+                        const uint8_t* bsf, int64_t M, int64_t N, int64_t K, void* y,
+                        bool y_is_f32, int64_t ldy, int* status, bool pdl, cudaStream_t stream);
+
+// Scale-factor layout helpers (host side).
+inline int64_t sf_katoms(int64_t K) { return (K / 32 + 3) / 4; }
+inline int64_t sf_row_tiles(int64_t rows) { return (rows + 127) / 128; }
+
+}  // namespace mxfp4

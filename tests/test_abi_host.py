@@ -1,0 +1,111 @@
+"""The C-ABI library on a machine without a GPU: it loads, exports every symbol
+the header declares, its host helpers agree with the oracle's own layout map,
+and argument errors are reported before anything is launched."""
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+import mxfp4_quantized_linear_block_b200 as mx
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    src = open(os.path.join(ROOT, "include", "mxfp4.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(mxfp4_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_every_declared_symbol_is_exported():
+    names = _declared_functions()
+    assert len(names) >= 9
+    for n in names:
+        assert hasattr(mx.lib, n), n
+    assert set(names) == set(mx.EXPORTS)
+
+
+def test_sf_layout_matches_oracle_map():
+    for rows, K in ((1, 32), (127, 96), (300, 640), (3584, 3072), (16, 14336)):
+        assert mx.sf_bytes(rows, K) == oracle.sf_bytes(rows, K)
+        rng = np.random.default_rng(rows + K)
+        for r, b in zip(rng.integers(0, rows, 200), rng.integers(0, K // 32, 200)):
+            assert mx.sf_offset(int(r), int(b), K) == oracle.sf_offset(int(r), int(b), K)
+    assert mx.sf_offset(0, 3, 64) == -1          # block beyond K
+    assert mx.sf_bytes(10, 33) == 0
+
+
+def test_status_strings():
+    for s in range(8):
+        assert isinstance(mx.status_string(s), str) and mx.status_string(s)
+    assert mx.status_string(99) == "unknown status"
+
+
+def test_workspace_sizes():
+    assert mx.workspace_bytes(mx.OP_QUANTIZE, 10, 16, 64) == 0
+    assert mx.workspace_bytes(mx.OP_GEMM, 10, 16, 64) >= 256
+    M, K = 3584, 3072
+    ws = mx.workspace_bytes(mx.OP_LINEAR, M, 9216, K)
+    assert ws >= 256 + M * K // 2 + mx.sf_bytes(M, K)
+
+
+# Fake device addresses: validation rejects these calls on the host, so nothing is dereferenced.
+P = 1 << 20
+
+
+def test_quantize_argument_errors():
+    L = mx.lib
+    assert L.mxfp4_rotate_quantize(None, 0, 4, 64, 64, 1, None, None, P, P, None) == mx.ERR_INVALID_ARG
+    assert L.mxfp4_rotate_quantize(P, 0, 4, 64, 64, 1, None, None, None, P, None) == mx.ERR_INVALID_ARG
+    assert L.mxfp4_rotate_quantize(P, 0, 4, 48, 64, 1, None, None, P, P, None) == mx.ERR_SHAPE
+    assert L.mxfp4_rotate_quantize(P, 0, 4, 64, 32, 1, None, None, P, P, None) == mx.ERR_SHAPE
+    assert L.mxfp4_rotate_quantize(P, 0, -1, 64, 64, 1, None, None, P, P, None) == mx.ERR_SHAPE
+    assert L.mxfp4_rotate_quantize(P + 8, 0, 4, 64, 64, 1, None, None, P, P, None) == mx.ERR_ALIGN
+    assert L.mxfp4_rotate_quantize(P, 0, 4, 64, 68, 1, None, None, P, P, None) == mx.ERR_ALIGN
+    assert L.mxfp4_rotate_quantize(P, 2, 4, 64, 64, 1, None, None, P, P, None) == mx.ERR_UNSUPPORTED
+    assert L.mxfp4_rotate_quantize(P, 0, 4, 64, 64, 7, None, None, P, P, None) == mx.ERR_UNSUPPORTED
+    # Kronecker mode needs both host factors
+    assert L.mxfp4_rotate_quantize(P, 0, 4, 64, 64, 2, None, None, P, P, None) == mx.ERR_INVALID_ARG
+    # empty input: valid, launches nothing
+    assert L.mxfp4_rotate_quantize(P, 0, 0, 64, 64, 1, None, None, P, P, None) == mx.OK
+    assert L.mxfp4_quantize(P, 1, 0, 64, 64, P, P, None) == mx.OK
+
+
+def test_gemm_argument_errors():
+    L = mx.lib
+    ok = dict(aq=P, asf=P, bq=P, bsf=P, M=4, N=16, K=64, y=P, ydt=0, ldy=16, ws=P, wsb=256)
+
+    def call(**kw):
+        a = {**ok, **kw}
+        return L.mxfp4_gemm(a["aq"], a["asf"], a["bq"], a["bsf"], a["M"], a["N"], a["K"], a["y"],
+                            a["ydt"], a["ldy"], a["ws"], a["wsb"], None)
+
+    assert call(aq=None) == mx.ERR_INVALID_ARG
+    assert call(ws=None) == mx.ERR_INVALID_ARG
+    assert call(N=24) == mx.ERR_SHAPE
+    assert call(K=48) == mx.ERR_SHAPE
+    assert call(ldy=8) == mx.ERR_SHAPE
+    assert call(y=P + 4) == mx.ERR_ALIGN
+    assert call(ldy=20) == mx.ERR_ALIGN
+    assert call(ydt=5) == mx.ERR_UNSUPPORTED
+    assert call(wsb=16) == mx.ERR_WORKSPACE
+    assert call(M=0) == mx.OK
+
+
+def test_linear_argument_errors():
+    L = mx.lib
+    need = mx.workspace_bytes(mx.OP_LINEAR, 8, 32, 64)
+    assert L.mxfp4_linear(P, 8, 64, 1, None, None, P, P, 32, P, P, need - 1, None) == mx.ERR_WORKSPACE
+    assert L.mxfp4_linear(P, 8, 64, 1, None, None, P, P, 24, P, P, need, None) == mx.ERR_SHAPE
+    assert L.mxfp4_linear(P, 8, 64, 9, None, None, P, P, 32, P, P, need, None) == mx.ERR_UNSUPPORTED
+    assert L.mxfp4_linear(P, 8, 64, 2, None, None, P, P, 32, P, P, need, None) == mx.ERR_INVALID_ARG
+    assert L.mxfp4_linear(None, 8, 64, 1, None, None, P, P, 32, P, P, need, None) == mx.ERR_INVALID_ARG
+    assert L.mxfp4_linear(P, 0, 64, 1, None, None, P, P, 32, P, P, need, None) == mx.OK
+
+
+def test_poll_status_null():
+    import ctypes
+    out = ctypes.c_int(0)
+    assert mx.lib.mxfp4_poll_status(None, ctypes.byref(out)) == mx.ERR_INVALID_ARG

@@ -1,0 +1,96 @@
+"""GPU parity of the tcgen05 block-scaled GEMM against the oracle's exact contraction."""
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from gpu_helpers import bf16_dev_to_f64, check_gemm_values, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+def _operand(seed, rows, K, tid, lo=112, hi=138):
+    q = synth.uniform_u8(seed, synth.TID_CODES + tid, (rows, K // 2), 0, 255)
+    s = synth.uniform_u8(seed, synth.TID_SCALES + tid, (rows, K // 32), lo, hi)
+    return q, s
+
+
+def _run(aq, as_, bq, bs, out):
+    import torch
+    import mxfp4_quantized_linear_block_b200 as mx
+    M, K = aq.shape[0], aq.shape[1] * 2
+    N = bq.shape[0]
+    y = mx.gemm(to_dev(aq), to_dev(oracle.sf_to_physical(as_, K)), to_dev(bq),
+                to_dev(oracle.sf_to_physical(bs, K)), M, N, K,
+                out_dtype=torch.float32 if out == "f32" else torch.bfloat16)
+    torch.cuda.synchronize()
+    return y.cpu().numpy().astype(np.float64) if out == "f32" else bf16_dev_to_f64(y)
+
+
+SHAPES = [
+    (1, 16, 32), (2, 16, 64), (64, 128, 256), (127, 144, 96), (128, 256, 256), (129, 272, 288),
+    (300, 384, 512), (256, 512, 1024), (200, 400, 3072), (130, 128, 320),
+]
+
+
+@pytest.mark.parametrize("M,N,K", SHAPES)
+@pytest.mark.parametrize("out", ["bf16", "f32"])
+def test_gemm_shapes(M, N, K, out):
+    aq, as_ = _operand(M * 31 + N * 7 + K, M, K, 0)
+    bq, bs = _operand(M * 31 + N * 7 + K, N, K, 1)
+    y = _run(aq, as_, bq, bs, out)
+    ref, S = oracle.gemm(aq, as_, bq, bs)
+    check_gemm_values(y, ref, S, out, f"gemm {M}x{N}x{K} {out}")
+
+
+def test_gemm_zero_and_single_pair():
+    K = 512
+    aq = np.zeros((130, K // 2), np.uint8)
+    bq = np.zeros((144, K // 2), np.uint8)
+    as_ = synth.uniform_u8(1, 90, (130, K // 32), 100, 150)
+    bs = synth.uniform_u8(1, 91, (144, K // 32), 100, 150)
+    y = _run(aq, as_, bq, bs, "f32")
+    assert not y.any()
+    aq[129, 200] = 13 << 4   # element 401 = -3
+    bq[143, 200] = 3 << 4    # element 401 = 1.5
+    y = _run(aq, as_, bq, bs, "f32")
+    expect = -3 * 1.5 * 2.0 ** (int(as_[129, 401 // 32]) + int(bs[143, 401 // 32]) - 254)
+    assert y[129, 143] == expect
+    y[129, 143] = 0
+    assert not y.any()
+
+
+def test_gemm_wide_scale_range_fp32():
+    """Scales spread over most of the E8M0 range in fp32 output."""
+    M, N, K = 256, 256, 1024
+    aq, as_ = _operand(11, M, K, 2, 70, 180)
+    bq, bs = _operand(11, N, K, 3, 70, 180)
+    y = _run(aq, as_, bq, bs, "f32")
+    ref, S = oracle.gemm(aq, as_, bq, bs)
+    check_gemm_values(y, ref, S, "f32", "wide scales")
+
+
+def _sample_pairs(M, N, BN=256, n_random=4096, seed=0):
+    """(m, n) pairs the oracle computes one by one: the first and last row tile
+    against the first and last column tile, 8 edge rows x every column, every
+    row x 4 edge columns, and n_random seeded random pairs."""
+    rows = np.unique(np.r_[np.arange(min(128, M)), np.arange(max(0, M - 128), M)])
+    cols = np.unique(np.r_[np.arange(min(BN, N)), np.arange(max(0, N - BN), N)])
+    edge_rows = np.unique(np.r_[rows[:4], rows[-4:]])
+    edge_cols = np.unique(np.r_[cols[:2], cols[-2:]])
+    rng = np.random.default_rng(seed)
+    mi = [np.repeat(rows, cols.size), np.repeat(edge_rows, N), np.tile(np.arange(M), edge_cols.size),
+          rng.integers(0, M, n_random)]
+    ni = [np.tile(cols, rows.size), np.tile(np.arange(N), edge_rows.size),
+          np.repeat(edge_cols, M), rng.integers(0, N, n_random)]
+    return np.concatenate(mi).astype(np.int64), np.concatenate(ni).astype(np.int64)
+
+
+@pytest.mark.parametrize("M,N,K", [(3584, 9216, 3072), (3584, 3072, 12288)])
+def test_gemm_full_size_sampled(M, N, K):
+    aq, as_ = _operand(K, M, K, 4)
+    bq, bs = _operand(K, N, K, 5)
+    y = _run(aq, as_, bq, bs, "bf16")
+    mi, ni = _sample_pairs(M, N)
+    ref, S = oracle.gemm_pairs(aq, as_, bq, bs, mi, ni)
+    check_gemm_values(y[mi, ni], ref, S, "bf16", f"gemm {M}x{N}x{K} sampled")

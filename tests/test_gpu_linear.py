@@ -1,0 +1,88 @@
+"""GPU parity of the whole layer (rotate + quantise + block-scaled GEMM, bf16 out)
+on the workload recipes, with pre-quantised weights prepared by the oracle."""
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from gpu_helpers import bf16_dev_to_f64, check_gemm_values, to_dev, to_dev_bf16
+from test_gpu_gemm import _sample_pairs
+
+pytestmark = pytest.mark.gpu
+
+
+def _layer_inputs(wl, lin):
+    x, _ = synth.activation_bf16(wl.seed, lin.M, lin.K, lin.outlier_frac, lin.outlier_factor,
+                                 lin.x_tensor)
+    w = synth.weight_f32(wl.seed, lin.N, lin.K, lin.layer)
+    A = B = None
+    if wl.rotation == oracle.ROT_KRON_4x8:
+        A, B = synth.kron_factors(wl.seed)
+    wq, ws = oracle.prepare_weight(w, wl.rotation, A, B)
+    return x, wq, ws, A, B
+
+
+def _run_linear(x, wq, ws, N, mode, A, B):
+    import torch
+    import mxfp4_quantized_linear_block_b200 as mx
+    K = x.shape[1]
+    y = mx.linear(to_dev_bf16(x), to_dev(wq), to_dev(oracle.sf_to_physical(ws, K)), N, mode, A, B)
+    torch.cuda.synchronize()
+    return bf16_dev_to_f64(y)
+
+
+@pytest.mark.parametrize("name", ["tiny"])
+def test_linear_full_compare(name):
+    wl = synth.WORKLOADS[name]
+    for lin in wl.linears:
+        x, wq, ws, A, B = _layer_inputs(wl, lin)
+        y = _run_linear(x, wq, ws, lin.N, wl.rotation, A, B)
+        ref, S, _, _ = oracle.linear(x, wq, ws, wl.rotation, A, B)
+        check_gemm_values(y, ref, S, "bf16", f"{name}/{lin.name}")
+
+
+@pytest.mark.parametrize("name", ["dit_b1", "kron", "llm_small_m1", "llm_small_m16",
+                                  "llm_small_m128"])
+def test_linear_workloads_sampled(name):
+    wl = synth.WORKLOADS[name]
+    for lin in wl.linears:
+        x, wq, ws, A, B = _layer_inputs(wl, lin)
+        y = _run_linear(x, wq, ws, lin.N, wl.rotation, A, B)
+        xq, xs = oracle.rotate_quantize(x, wl.rotation, A, B)
+        mi, ni = _sample_pairs(lin.M, lin.N, n_random=4096, seed=lin.layer)
+        ref, S = oracle.gemm_pairs(xq, xs, wq, ws, mi, ni)
+        check_gemm_values(y[mi, ni], ref, S, "bf16", f"{name}/{lin.name}")
+
+
+def test_linear_batch16_sampled():
+    wl = synth.WORKLOADS["dit_b16"]
+    lin = wl.linears[0]
+    x, wq, ws, A, B = _layer_inputs(wl, lin)
+    y = _run_linear(x, wq, ws, lin.N, wl.rotation, A, B)
+    xq, xs = oracle.rotate_quantize(x, wl.rotation)
+    mi, ni = _sample_pairs(lin.M, lin.N, n_random=8192, seed=3)
+    ref, S = oracle.gemm_pairs(xq, xs, wq, ws, mi, ni)
+    check_gemm_values(y[mi, ni], ref, S, "bf16", "dit_b16/mlp_up")
+
+
+def test_linear_repeatable():
+    """Two runs give identical bytes (no races between the paired kernels)."""
+    wl = synth.WORKLOADS["dit_b1"]
+    lin = wl.linears[0]
+    x, wq, ws, A, B = _layer_inputs(wl, lin)
+    y1 = _run_linear(x, wq, ws, lin.N, wl.rotation, A, B)
+    y2 = _run_linear(x, wq, ws, lin.N, wl.rotation, A, B)
+    assert np.array_equal(y1, y2)
+
+
+def test_status_word_clear_after_runs():
+    import torch
+    import mxfp4_quantized_linear_block_b200 as mx
+    wl = synth.WORKLOADS["tiny"]
+    lin = wl.linears[0]
+    x, wq, ws, A, B = _layer_inputs(wl, lin)
+    wsp = mx.new_workspace(mx.workspace_bytes(mx.OP_LINEAR, lin.M, lin.N, lin.K))
+    mx.linear(to_dev_bf16(x), to_dev(wq), to_dev(oracle.sf_to_physical(ws, lin.K)), lin.N,
+              wl.rotation, ws=wsp)
+    torch.cuda.synchronize()
+    assert mx.poll_status(wsp) == mx.OK
