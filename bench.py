@@ -45,8 +45,10 @@ FP4_OVER_BF16 = 4.0  # nominal dense FP4 : BF16 tensor throughput on B200 (9 : 2
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--attr-steps", type=int, default=200,
+                    help="steps of the per-kernel attribution pass (capped at --steps)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="dit_b1", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -73,39 +75,58 @@ def workload_desc(wl) -> str:
 
 # --------------------------------------------------------------------------- CPU oracle
 
-def oracle_sample_time(wl, budget_s: float = 12.0):
-    """Time the oracle (rotate+quantise + exact contraction) on a row sample of
-    every linear; return (TFLOPS extrapolated to the full workload, sample text,
-    seconds spent)."""
-    import oracle
-    A = B = None
-    if wl.rotation == synth.ROT_KRON_4x8:
-        A, B = synth.kron_factors(wl.seed)
-    prepared = []
-    for lin in wl.linears:
-        w = synth.weight_f32(wl.seed, lin.N, lin.K, lin.layer)
-        wq, ws = oracle.prepare_weight(w, wl.rotation, A, B)
-        prepared.append((lin, wq, ws))
+class OracleSample:
+    """The CPU oracle (rotate+quantise + exact contraction) timed on a row sample
+    of every linear of a workload; weights are prepared once, outside the timing."""
 
-    def run(rows):
-        t0 = time.perf_counter()
-        for lin, wq, ws in prepared:
+    def __init__(self, wl):
+        import oracle
+        self.oracle = oracle
+        self.wl = wl
+        self.A = self.B = None
+        if wl.rotation == synth.ROT_KRON_4x8:
+            self.A, self.B = synth.kron_factors(wl.seed)
+        self.prepared = []
+        for lin in wl.linears:
+            w = synth.weight_f32(wl.seed, lin.N, lin.K, lin.layer)
+            wq, ws = oracle.prepare_weight(w, wl.rotation, self.A, self.B)
+            self.prepared.append((lin, wq, ws))
+        self.rows = 1
+
+    def _run(self, rows):
+        xs = []
+        for lin, _, _ in self.prepared:
             r = min(rows, lin.M)
-            x, _ = synth.activation_bf16(wl.seed, r, lin.K, lin.outlier_frac, lin.outlier_factor,
-                                         lin.x_tensor)
-            oracle.linear(x, wq, ws, wl.rotation, A, B)
+            x, _ = synth.activation_bf16(self.wl.seed, r, lin.K, lin.outlier_frac,
+                                         lin.outlier_factor, lin.x_tensor)
+            xs.append(x)
+        t0 = time.perf_counter()
+        for (lin, wq, ws), x in zip(self.prepared, xs):
+            self.oracle.linear(x, wq, ws, self.wl.rotation, self.A, self.B)
         return time.perf_counter() - t0
 
-    rows = 1
-    t = run(rows)
-    while t < budget_s / 8 and rows < min(l.M for l in wl.linears):
-        rows *= 2
-        t = run(rows)
-    sample_flops = sum(2 * min(rows, l.M) * l.N * l.K for l in wl.linears)
-    tflops = sample_flops / t / 1e12
-    sample = (f"{rows} rows of every linear (all N, all K): rotate+quantise of those rows and the "
-              f"exact block-scaled products, {t:.2f} s; extrapolated linearly in rows")
-    return tflops, sample, t
+    def calibrate(self, budget_s: float):
+        """Grow the row sample (powers of two) until one run takes about budget_s."""
+        t = self._run(self.rows)
+        while t < budget_s / 2 and self.rows < min(l.M for l in self.wl.linears):
+            self.rows *= 2
+            t = self._run(self.rows)
+        return t
+
+    def measure(self):
+        """One timed run: (TFLOPS extrapolated to the full workload, sample text)."""
+        t = self._run(self.rows)
+        flops = sum(2 * min(self.rows, l.M) * l.N * l.K for l in self.wl.linears)
+        sample = (f"{self.rows} rows of every linear (all N, all K): rotate+quantise of those "
+                  f"rows and the exact block-scaled products in {t:.2f} s, extrapolated "
+                  f"linearly to all rows")
+        return flops / t / 1e12, sample
+
+
+def oracle_sample_time(wl, budget_s: float = 12.0):
+    s = OracleSample(wl)
+    s.calibrate(budget_s)
+    return s.measure()
 
 
 def cpu_cores() -> int:
@@ -245,9 +266,13 @@ def run_ours(args, rank, world, local_rank):
     # ---- timed region: K steps through the public call, inputs resident in HBM
     clocks = ClockSampler(local_rank)
     clocks.start()
+    time.sleep(0.3)  # let the sampler come up before the timed region
     barrier()
     torch.cuda.synchronize()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    # A short GPU sleep ahead of the first event lets the host queue launches ahead of the
+    # device, so the timed steps run back to back (the sleep itself is not timed).
+    torch.cuda._sleep(int(2e7))
     ev0.record(stream)
     for i in range(args.steps):
         step(i)
@@ -273,8 +298,9 @@ def run_ours(args, rank, world, local_rank):
               torch.empty(mx.sf_bytes(l.M, l.K), dtype=torch.uint8, device=dev)) for l in wl.linears]
     gws = mx.new_workspace(mx.workspace_bytes(mx.OP_GEMM, 1, 16, 32), dev)
     n_lin = len(wl.linears)
+    n_attr = max(1, min(args.steps, args.attr_steps))
     evs = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
-             torch.cuda.Event(enable_timing=True)) for _ in range(n_lin)] for _ in range(args.steps)]
+             torch.cuda.Event(enable_timing=True)) for _ in range(n_lin)] for _ in range(n_attr)]
 
     def step_split(i, rec):
         xs, ys, _ = sets[i % len(sets)]
@@ -293,18 +319,19 @@ def run_ours(args, rank, world, local_rank):
     for i in range(args.warmup):
         step_split(i, False)
     torch.cuda.synchronize()
-    for i in range(args.steps):
+    torch.cuda._sleep(int(2e7))
+    for i in range(n_attr):
         step_split(i, True)
     torch.cuda.synchronize()
     t_q = np.zeros(n_lin)
     t_g = np.zeros(n_lin)
-    for i in range(args.steps):
+    for i in range(n_attr):
         for j in range(n_lin):
             a, b, c = evs[i][j]
             t_q[j] += a.elapsed_time(b) * 1e-3
             t_g[j] += b.elapsed_time(c) * 1e-3
-    t_q /= args.steps
-    t_g /= args.steps
+    t_q /= n_attr
+    t_g /= n_attr
     gemm_flops = np.array([l.flops for l in wl.linears], dtype=np.float64)
     gemm_bytes = np.array([l.M * l.K // 2 + mx.sf_bytes(l.M, l.K) + l.N * l.K // 2 +
                            mx.sf_bytes(l.N, l.K) + 2 * l.M * l.N for l in wl.linears], np.float64)
@@ -337,6 +364,7 @@ def run_ours(args, rank, world, local_rank):
         torch.cuda.synchronize()
         barrier()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda._sleep(int(2e7))
         a.record(stream)
         for _ in range(args.e2e_steps):
             e2e_step()
@@ -346,10 +374,8 @@ def run_ours(args, rank, world, local_rank):
         t_e2e = max_over_ranks(a.elapsed_time(b) * 1e-3)
         e2e = {"value": flops_step * args.e2e_steps * world / t_e2e / 1e12, "unit": UNIT,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-               "ms_per_step": t_e2e / args.e2e_steps * 1e3}
-        launches_e2e = 2 * len(wl.linears) * args.e2e_steps
-    else:
-        launches_e2e = 0
+               "ms_per_step": t_e2e / args.e2e_steps * 1e3, "steps": args.e2e_steps,
+               "gpu_launches": 2 * len(wl.linears) * args.e2e_steps}
 
     result = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -380,7 +406,10 @@ def run_ours(args, rank, world, local_rank):
                               "alg_bytes_per_launch": [int(b) for b in q_bytes],
                               "traffic": None},
         "e2e": e2e,
-        "gpu_launches": launches + launches_e2e,
+        "gpu_launches": launches,
+        "attribution": {"steps": n_attr, "gpu_launches": 2 * n_lin * n_attr,
+                        "note": "quantise and GEMM launched separately with CUDA events "
+                                "around each kernel; source of both roofline objects"},
         "clocks": clk,
     }
     return result
@@ -390,14 +419,14 @@ def run_ours(args, rank, world, local_rank):
 
 def run_reference(args):
     wl = synth.WORKLOADS[args.workload]
-    per = max(2.0, 60.0 / max(1, args.steps + args.warmup))
-    vals = []
-    samples = []
+    per = max(1.0, 90.0 / max(1, args.steps + args.warmup))
+    sampler = OracleSample(wl)
+    sampler.calibrate(per)
+    vals, sample = [], ""
     for i in range(args.warmup + args.steps):
-        v, sample, t = oracle_sample_time(wl, budget_s=per)
+        v, sample = sampler.measure()
         if i >= args.warmup:
             vals.append(v)
-            samples.append(sample)
     value = statistics.median(vals)
     return {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1,
@@ -406,7 +435,7 @@ def run_reference(args):
         "scaling": "weak", "vs_baseline": None, "dtype": "mxfp4",
         "data": "synthetic", "config": {"workload": workload_desc(wl)},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
-                         "sample": samples[-1]},
+                         "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
@@ -430,7 +459,7 @@ def main():
     try:
         res = run_ours(args, rank, world, local_rank)
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
-            v, sample, _ = oracle_sample_time(synth.WORKLOADS[args.workload])
+            v, sample = oracle_sample_time(synth.WORKLOADS[args.workload])
             res["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cpu_cores(),
                                    "kind": "oracle", "sample": sample}
         if rank == 0:
