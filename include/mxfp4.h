@@ -160,6 +160,43 @@ mxfp4_status mxfp4_linear(const void* x, int64_t M, int64_t K, mxfp4_rotation mo
                           const uint8_t* wsf, int64_t N, void* y, void* ws, size_t ws_bytes,
                           mxfp4_stream_t stream);
 
+/* Size in bytes of the device scratch array that mxfp4_linear_noalloc uses (per GPU). */
+#define MXFP4_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+
+/*
+ * The same layer as mxfp4_linear, for callers that cannot allocate device
+ * memory when they run it -- for instance an inference engine whose memory
+ * plan is fixed at start-up, a plugin running inside another framework's
+ * enqueue step where allocation is not allowed, or latency-critical code that
+ * must avoid cudaMalloc's implicit device synchronisation. (The pages have no
+ * counterpart: this is an interface choice of this library.)
+ *
+ * The caller passes inputs and outputs exactly as for mxfp4_linear but no
+ * workspace: the quantised activations live in a static device array of
+ * MXFP4_NOALLOC_SCRATCH_BYTES (32 MiB) inside the library, which every GPU
+ * that loads the library keeps until the process exits. Nothing is allocated
+ * per call (no cudaMalloc / cudaFree, no allocating library routine).
+ *  - Limit: 256 + round256(M * K / 2) + round256(mxfp4_sf_bytes(M, K)) must
+ *    not exceed the array (about 62 million activation elements); larger
+ *    problems return MXFP4_ERR_WORKSPACE and launch nothing.
+ *  - status: optional DEVICE pointer to a caller-owned, 4-byte aligned int
+ *    that the caller zeroes; a bounded-wait timeout sets it to
+ *    MXFP4_ERR_TIMEOUT. With NULL the library keeps a status word in its array
+ *    and clears it at the start of each call (the caller cannot read it).
+ *  - The first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    before any stream capture.
+ *  - Every call shares the one array, which keeps the previous call's
+ *    contents (each call rewrites all of the part it reads). Calls whose
+ *    kernels can overlap on the GPU -- different streams, or host threads
+ *    without ordering between them -- race on the array and corrupt each
+ *    other's results; keep them on one stream or otherwise ordered.
+ */
+mxfp4_status mxfp4_linear_noalloc(const void* x, int64_t M, int64_t K, mxfp4_rotation mode,
+                                  const float* kron_a, const float* kron_b, const uint8_t* wq,
+                                  const uint8_t* wsf, int64_t N, void* y, int* status,
+                                  mxfp4_stream_t stream);
+
 /*
  * Read the device status word at the start of a workspace (synchronises with
  * the device): MXFP4_OK, or MXFP4_ERR_TIMEOUT if a kernel's bounded wait on a

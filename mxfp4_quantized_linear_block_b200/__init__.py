@@ -26,7 +26,7 @@ OP_QUANTIZE, OP_GEMM, OP_LINEAR = 0, 1, 2
 EXPORTS = (
     "mxfp4_sf_bytes", "mxfp4_sf_offset", "mxfp4_workspace_bytes", "mxfp4_status_string",
     "mxfp4_quantize", "mxfp4_rotate_quantize", "mxfp4_gemm", "mxfp4_linear",
-    "mxfp4_poll_status",
+    "mxfp4_poll_status", "mxfp4_linear_noalloc",
 )
 
 
@@ -53,6 +53,7 @@ def _load() -> ctypes.CDLL:
         "mxfp4_gemm": ([vp, vp, vp, vp, i64, i64, i64, vp, i32, i64, vp, sz, vp], i32),
         "mxfp4_linear": ([vp, i64, i64, i32, vp, vp, vp, vp, i64, vp, vp, sz, vp], i32),
         "mxfp4_poll_status": ([vp, vp], i32),
+        "mxfp4_linear_noalloc": ([vp, i64, i64, i32, vp, vp, vp, vp, i64, vp, vp, vp], i32),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -184,6 +185,26 @@ def linear(x, wq, wsf, N: int, mode: int = ROT_HADAMARD32, kron_a=None, kron_b=N
     st = lib.mxfp4_linear(x.data_ptr(), M, K, mode, a, b, wq.data_ptr(), wsf.data_ptr(), N,
                           y.data_ptr(), ws.data_ptr(), ws.numel(), _stream_handle(stream))
     _check(st, "mxfp4_linear")
+    return y
+
+
+def linear_noalloc(x, wq, wsf, N: int, mode: int = ROT_HADAMARD32, kron_a=None, kron_b=None,
+                   y=None, status=None, stream=None):
+    """The layer without a workspace, for callers that cannot allocate device memory at
+    call time: the quantised activations go to a fixed 32 MiB array inside the library
+    (see mxfp4_linear_noalloc in include/mxfp4.h for the size limit and the sharing
+    rules). `status`: optional zeroed int32 CUDA tensor that receives a timeout code."""
+    torch = _torch()
+    assert x.dim() == 2 and x.is_contiguous() and x.dtype == torch.bfloat16
+    M, K = x.shape
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    a = _host_f32(kron_a, 16) if mode == ROT_KRON_4x8 else None
+    b = _host_f32(kron_b, 64) if mode == ROT_KRON_4x8 else None
+    st = lib.mxfp4_linear_noalloc(x.data_ptr(), M, K, mode, a, b, wq.data_ptr(), wsf.data_ptr(),
+                                  N, y.data_ptr(), status.data_ptr() if status is not None else None,
+                                  _stream_handle(stream))
+    _check(st, "mxfp4_linear_noalloc")
     return y
 
 
