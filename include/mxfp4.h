@@ -104,7 +104,10 @@ const char* mxfp4_status_string(mxfp4_status status);
  * Steps 2 of the layer ("What is MXFP4..." on the AMD Quark page; RTN
  * quantiser of "Bridging the Gap...", "Probleemstelling").
  * Requirements: K % 32 == 0, ldx >= K, x 16-byte aligned and ldx * elemsize a
- * multiple of 16; q and sf 16-byte aligned.
+ * multiple of 16; q and sf 16-byte aligned. The kernel's input pipeline waits
+ * on its own copies with a time bound; these two calls have no status word, so
+ * an expiry (a copy that never lands) only ends the kernel early, leaving the
+ * output incomplete -- mxfp4_linear reports it through its workspace.
  */
 mxfp4_status mxfp4_quantize(const void* x, mxfp4_dtype xdt, int64_t rows, int64_t K, int64_t ldx,
                             uint8_t* q, uint8_t* sf, mxfp4_stream_t stream);

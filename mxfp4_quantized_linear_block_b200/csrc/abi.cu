@@ -139,7 +139,7 @@ mxfp4_status mxfp4_rotate_quantize(const void* x, mxfp4_dtype xdt, int64_t rows,
     return MXFP4_ERR_INVALID_ARG;
   if (rows == 0) return MXFP4_OK;
   return from_cuda(launch_rotate_quantize(x, xdt == MXFP4_DT_F32, rows, K, ldx, (int)mode, &kc, q,
-                                          sf, static_cast<cudaStream_t>(stream)));
+                                          sf, nullptr, static_cast<cudaStream_t>(stream)));
 }
 
 mxfp4_status mxfp4_gemm(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq,
@@ -178,7 +178,8 @@ mxfp4_status mxfp4_linear(const void* x, int64_t M, int64_t K, mxfp4_rotation mo
   uint8_t* xq = base + w.q_off;
   uint8_t* xsf = base + w.sf_off;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  cudaError_t e = launch_rotate_quantize(x, false, M, K, K, (int)mode, &kc, xq, xsf, s);
+  cudaError_t e =
+      launch_rotate_quantize(x, false, M, K, K, (int)mode, &kc, xq, xsf, static_cast<int*>(ws), s);
   if (e != cudaSuccess) return MXFP4_ERR_CUDA;
   return from_cuda(
       launch_gemm(xq, xsf, wq, wsf, M, N, K, y, false, N, static_cast<int*>(ws), true, s));

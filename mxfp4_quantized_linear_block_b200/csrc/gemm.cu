@@ -341,6 +341,257 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// ---------------------------------------------------------------- CTA-pair kernel
+//
+// Two CTAs of a cluster share one 256 x 256 output tile through
+// tcgen05.mma.cta_group::2 (M = 256, N = 256, K = 64): each CTA loads its own
+// 128 rows of A and its own 128 rows of B, so each SM streams half the operand
+// bytes per MMA that a single-CTA 128 x 256 tile needs. The leader (even rank)
+// issues the MMAs and the scale copies for both; both CTAs run producers and
+// epilogues. Tile loads of both CTAs complete on the leader's stage barrier;
+// the leader's commits arrive on both CTAs' barriers. No load is multicast.
+
+template <uint32_t STAGES>
+struct PairConfig {
+  static constexpr uint32_t BN = 256;                 // N per pair tile
+  static constexpr uint32_t A_STAGE = 128 * BK_BYTES;  // own 128 rows of A
+  static constexpr uint32_t B_STAGE = 128 * BK_BYTES;  // own 128 rows of B
+  static constexpr uint32_t SFA_STAGE = 1024;          // own rows: 2 scale atoms
+  static constexpr uint32_t SFB_STAGE = 2048;          // all 256 rows of B: 2 groups x 2 atoms
+  static constexpr uint32_t STAGE_TX = A_STAGE + B_STAGE + SFA_STAGE + SFB_STAGE;
+  static constexpr uint32_t OFF_A = 0;
+  static constexpr uint32_t OFF_B = OFF_A + STAGES * A_STAGE;
+  static constexpr uint32_t OFF_SFA = OFF_B + STAGES * B_STAGE;
+  static constexpr uint32_t OFF_SFB = OFF_SFA + STAGES * SFA_STAGE;
+  static constexpr uint32_t OFF_BAR = OFF_SFB + STAGES * SFB_STAGE;
+  static constexpr uint32_t NUM_BARS = 2 * STAGES + 3;
+  static constexpr uint32_t OFF_MISC = OFF_BAR + NUM_BARS * 8;
+  static constexpr uint32_t SMEM_BYTES = OFF_MISC + 16 + 1024;
+  static constexpr uint32_t SFA_COL = BN;       // after the 256-column accumulator
+  static constexpr uint32_t SFB_COL = SFA_COL + 8;
+  static constexpr uint32_t TMEM_COLS = 512;
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+};
+
+template <uint32_t STAGES, bool Y_F32>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    mxf4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a,
+                          const __grid_constant__ CUtensorMap tmap_b,
+                          const __grid_constant__ CUtensorMap tmap_sfa,
+                          const __grid_constant__ CUtensorMap tmap_sfb, const Params p) {
+  using C = PairConfig<STAGES>;
+  constexpr uint32_t BN = C::BN;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_addr(smem_raw);
+  const uint32_t pad = ((raw_addr + 1023u) & ~1023u) - raw_addr;
+  uint8_t* smem = smem_raw + pad;
+  const uint32_t sbase = raw_addr + pad;
+
+  const uint32_t warp = threadIdx.x >> 5;
+  const uint32_t lane = threadIdx.x & 31u;
+  const uint32_t rank = cluster_ctarank();  // 0: leader
+  const uint32_t pair = blockIdx.x >> 1;
+  const uint32_t num_pairs = gridDim.x >> 1;
+
+  const uint32_t bar_full = sbase + C::OFF_BAR;        // [STAGES], leader's count both CTAs
+  const uint32_t bar_empty = bar_full + 8 * STAGES;    // [STAGES]
+  const uint32_t bar_tfull = bar_empty + 8 * STAGES;   // accumulator ready
+  const uint32_t bar_tempty = bar_tfull + 8;           // leader: accumulator drained (both CTAs)
+  const uint32_t bar_mma_done = bar_tempty + 8;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+
+  if (threadIdx.x == 0) {
+    for (uint32_t s = 0; s < STAGES; ++s) {
+      mbar_init(bar_full + 8 * s, 1);
+      mbar_init(bar_empty + 8 * s, 1);
+    }
+    mbar_init(bar_tfull, 1);
+    mbar_init(bar_tempty, 2 * kEpiWarps);
+    mbar_init(bar_mma_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tmap(&tmap_a);
+    prefetch_tmap(&tmap_b);
+    prefetch_tmap(&tmap_sfa);
+    prefetch_tmap(&tmap_sfb);
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc_pair(smem_addr(tmem_slot), C::TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // both CTAs' barriers exist before either signals the other
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  griddep_wait();
+
+  const uint32_t n_tiles_total = p.m_tiles * p.n_tiles;  // m_tiles counts 256-row pair tiles
+
+  if (warp == kProducerWarp) {
+    if (elect_one()) {
+      const uint32_t full_at_leader = map_to_rank(bar_full, 0);
+      uint32_t stage = 0, phase = 0, issued = 0;
+      bool ok = true;
+      for (uint32_t tile = pair; tile < n_tiles_total && ok; tile += num_pairs) {
+        const uint32_t mt = tile / p.n_tiles, nt = tile % p.n_tiles;
+        const int32_t m_cta = (int32_t)(mt * 256u + rank * 128u);
+        const int32_t n_cta = (int32_t)(nt * BN + rank * 128u);
+        for (uint32_t kt = 0; kt < p.k_tiles; ++kt) {
+          if (!mbar_wait_bounded(bar_empty + 8 * stage, phase ^ 1u, abort_flag, kWaitLimitNs)) {
+            ok = false;
+            break;
+          }
+          if (rank == 0) mbar_arrive_expect_tx(bar_full + 8 * stage, 2u * C::STAGE_TX);
+          const uint32_t fb = full_at_leader + 8 * stage;
+          tma_load_2d_pair(sbase + C::OFF_A + stage * C::A_STAGE, &tmap_a, fb,
+                           (int32_t)(kt * BK_BYTES), m_cta);
+          tma_load_2d_pair(sbase + C::OFF_B + stage * C::B_STAGE, &tmap_b, fb,
+                           (int32_t)(kt * BK_BYTES), n_cta);
+          // scale atoms: A's are rows of a [row_tiles * k_atoms, 128-word] view, B's a
+          // [row_tiles, k_atoms, 128-word] view (both 128-row groups of the tile)
+          tma_load_2d_pair(sbase + C::OFF_SFA + stage * C::SFA_STAGE, &tmap_sfa, fb, 0,
+                           (int32_t)((uint32_t)(m_cta / 128) * p.k_atoms + 2 * kt));
+          tma_load_3d_pair(sbase + C::OFF_SFB + stage * C::SFB_STAGE, &tmap_sfb, fb, 0,
+                           (int32_t)(2 * kt), (int32_t)(nt * 2u));
+          ++issued;
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) record_timeout(p.status);
+      if (rank == 0) {
+        // Both CTAs' loads into the last stages have landed (they count on these barriers).
+        uint32_t s = stage, ph = phase;
+        for (uint32_t i = 0; i < STAGES && i < issued; ++i) {
+          if (s == 0) {
+            s = STAGES - 1;
+            ph ^= 1u;
+          } else {
+            --s;
+          }
+          volatile int never = 0;
+          mbar_wait_bounded(bar_full + 8 * s, ph, &never, kWaitLimitNs);
+        }
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    if (rank == 0 && elect_one()) {
+      uint32_t stage = 0, phase = 0, acc_phase = 0;
+      bool ok = true;
+      for (uint32_t tile = pair; tile < n_tiles_total && ok; tile += num_pairs) {
+        if (!mbar_wait_bounded(bar_tempty, acc_phase ^ 1u, abort_flag, kWaitLimitNs)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        for (uint32_t kt = 0; kt < p.k_tiles; ++kt) {
+          if (!mbar_wait_bounded(bar_full + 8 * stage, phase, abort_flag, kWaitLimitNs)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sfa_s = sbase + C::OFF_SFA + stage * C::SFA_STAGE;
+          const uint32_t sfb_s = sbase + C::OFF_SFB + stage * C::SFB_STAGE;
+          for (uint32_t a = 0; a < 2; ++a) {
+            tmem_cp_32x128b_warpx4_pair(tmem_base + C::SFA_COL + 4 * a, smem_desc_sf(sfa_s + a * 512));
+            for (uint32_t g = 0; g < 2; ++g)
+              tmem_cp_32x128b_warpx4_pair(tmem_base + C::SFB_COL + 4 * (2 * a + g),
+                                          smem_desc_sf(sfb_s + (g * 2 + a) * 512));
+          }
+          const uint32_t k_left = p.K - kt * 256u;
+          const uint32_t steps = k_left >= 256u ? 4u : (k_left + 63u) / 64u;
+          const uint32_t a_tile = sbase + C::OFF_A + stage * C::A_STAGE;
+          const uint32_t b_tile = sbase + C::OFF_B + stage * C::B_STAGE;
+          for (uint32_t k = 0; k < steps; ++k) {
+            const uint32_t sf_id = (k & 1u) * 2u;
+            mma_mxf4_pair(tmem_base, smem_desc_sw128(a_tile + k * MMA_K_BYTES),
+                          smem_desc_sw128(b_tile + k * MMA_K_BYTES), idesc_mxf4(256, BN, sf_id, sf_id),
+                          tmem_base + C::SFA_COL + 4 * (k >> 1), tmem_base + C::SFB_COL + 8 * (k >> 1),
+                          (kt | k) != 0u);
+          }
+          mma_commit_pair_both(bar_empty + 8 * stage);  // frees the stage in both CTAs
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        mma_commit_pair_both(bar_tfull);  // both halves of the accumulator are ready
+        acc_phase ^= 1u;
+      }
+      if (!ok) record_timeout(p.status);
+      mma_commit_pair_leader(bar_mma_done);
+      volatile int never = 0;
+      mbar_wait_bounded(bar_mma_done, 0, &never, kWaitLimitNs);
+    }
+  } else {
+    const uint32_t quad = warp & 3u;
+    const uint32_t half = (warp - kFirstEpiWarp) / 4u;
+    constexpr uint32_t COLS = BN / 2;
+    constexpr uint32_t CHUNKS = COLS / 32;
+    const uint32_t tempty_at_leader = map_to_rank(bar_tempty, 0);
+    uint32_t acc_phase = 0;
+    for (uint32_t tile = pair; tile < n_tiles_total; tile += num_pairs) {
+      const uint32_t mt = tile / p.n_tiles, nt = tile % p.n_tiles;
+      const bool ok = mbar_wait_bounded(bar_tfull, acc_phase, abort_flag, kWaitLimitNs);
+      if (!__all_sync(0xffffffffu, ok)) {
+        if (lane == 0) record_timeout(p.status);
+        break;
+      }
+      tc_fence_after();
+      uint32_t v[CHUNKS][32];
+      const uint32_t taddr = tmem_base + ((quad * 32u) << 16) + half * COLS;
+#pragma unroll
+      for (uint32_t c = 0; c < CHUNKS; ++c) tmem_ld_32x32b_x32(taddr + 32 * c, v[c]);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(tempty_at_leader);
+
+      const uint32_t row = mt * 256u + rank * 128u + quad * 32u + lane;
+      const uint32_t col0 = nt * BN + half * COLS;
+      if (row < p.M) {
+        if constexpr (Y_F32) {
+          float* yrow = static_cast<float*>(p.y) + (uint64_t)row * p.ldy + col0;
+#pragma unroll
+          for (uint32_t c = 0; c < CHUNKS; ++c)
+#pragma unroll
+            for (uint32_t j = 0; j < 32; j += 4)
+              if (col0 + 32 * c + j < p.N)
+                st_global_v4(yrow + 32 * c + j, v[c][j], v[c][j + 1], v[c][j + 2], v[c][j + 3]);
+        } else {
+          uint16_t* yrow = static_cast<uint16_t*>(p.y) + (uint64_t)row * p.ldy + col0;
+#pragma unroll
+          for (uint32_t c = 0; c < CHUNKS; ++c)
+#pragma unroll
+            for (uint32_t j = 0; j < 32; j += 8)
+              if (col0 + 32 * c + j < p.N)
+                st_global_v4(yrow + 32 * c + j,
+                             pack_bf16x2(__uint_as_float(v[c][j]), __uint_as_float(v[c][j + 1])),
+                             pack_bf16x2(__uint_as_float(v[c][j + 2]), __uint_as_float(v[c][j + 3])),
+                             pack_bf16x2(__uint_as_float(v[c][j + 4]), __uint_as_float(v[c][j + 5])),
+                             pack_bf16x2(__uint_as_float(v[c][j + 6]), __uint_as_float(v[c][j + 7])));
+        }
+      }
+      acc_phase ^= 1u;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // neither CTA leaves while the pair's MMAs or copies may touch it
+  if (warp == kMmaWarp) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
+  }
+}
+
 // ---------------------------------------------------------------- host side
 
 PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
@@ -369,6 +620,98 @@ bool make_operand_map(CUtensorMap* map, const uint8_t* base, uint64_t rows, uint
                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+// Scale atoms of an operand as 128-word (512-byte) rows: 2-D [row_tiles * k_atoms, 128]
+// (box: 2 consecutive atoms) or 3-D [row_tiles, k_atoms, 128] (box: 2 atoms x 2 row tiles).
+bool make_scale_map(CUtensorMap* map, const uint8_t* sf, uint64_t row_tiles, uint64_t k_atoms,
+                    bool three_d) {
+  auto fn = get_encode_fn();
+  if (!fn) return false;
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r;
+  if (three_d) {
+    cuuint64_t dims[3] = {128, k_atoms, row_tiles};
+    cuuint64_t strides[2] = {512, k_atoms * 512};
+    cuuint32_t box[3] = {128, 2, 2};
+    r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<uint8_t*>(sf), dims, strides, box,
+           estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  } else {
+    cuuint64_t dims[2] = {128, row_tiles * k_atoms};
+    cuuint64_t strides[1] = {512};
+    cuuint32_t box[2] = {128, 2};
+    r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint8_t*>(sf), dims, strides, box,
+           estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  }
+  return r == CUDA_SUCCESS;
+}
+
+template <uint32_t STAGES, bool Y_F32>
+cudaError_t launch_pair(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq,
+                        const uint8_t* bsf, int64_t M, int64_t N, int64_t K, void* y, int64_t ldy,
+                        int* status, bool pdl, cudaStream_t stream) {
+  using C = PairConfig<STAGES>;
+  const uint64_t k_atoms = (uint64_t)sf_katoms(K);
+  CUtensorMap ta, tb, tsa, tsb;
+  if (!make_operand_map(&ta, aq, (uint64_t)M, (uint64_t)(K / 2), 128) ||
+      !make_operand_map(&tb, bq, (uint64_t)N, (uint64_t)(K / 2), 128) ||
+      !make_scale_map(&tsa, asf, (uint64_t)sf_row_tiles(M), k_atoms, false) ||
+      !make_scale_map(&tsb, bsf, (uint64_t)sf_row_tiles(N), k_atoms, true))
+    return cudaErrorInvalidValue;
+  auto kern = mxf4_gemm_pair_kernel<STAGES, Y_F32>;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  static bool attr_done[64] = {};
+  static int max_clusters[64] = {};
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!attr_done[dev]) {
+    cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t q{};
+    q.gridDim = dim3(2);
+    q.blockDim = dim3(kThreads);
+    q.dynamicSmemBytes = C::SMEM_BYTES;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &q) != cudaSuccess || n <= 0) {
+      cudaGetLastError();
+      int sms = 148;
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+      n = sms / 2;
+    }
+    max_clusters[dev] = n;
+    attr_done[dev] = true;
+  }
+  Params p{};
+  p.asf = asf;
+  p.bsf = bsf;
+  p.y = y;
+  p.status = status;
+  p.M = (uint32_t)M;
+  p.N = (uint32_t)N;
+  p.K = (uint32_t)K;
+  p.m_tiles = (uint32_t)((M + 255) / 256);
+  p.n_tiles = (uint32_t)((N + C::BN - 1) / C::BN);
+  p.k_tiles = (uint32_t)((K + 255) / 256);
+  p.k_atoms = (uint32_t)k_atoms;
+  p.b_row_tiles = (uint32_t)sf_row_tiles(N);
+  p.ldy = (uint64_t)ldy;
+  const uint32_t tiles = p.m_tiles * p.n_tiles;
+  const uint32_t pairs = tiles < (uint32_t)max_clusters[dev] ? tiles : (uint32_t)max_clusters[dev];
+
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(2 * pairs);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = C::SMEM_BYTES;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, ta, tb, tsa, tsb, p);
 }
 
 template <uint32_t BN, uint32_t STAGES, bool Y_F32>
@@ -428,6 +771,12 @@ cudaError_t launch_cfg(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq,
 cudaError_t launch_gemm(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq,
                         const uint8_t* bsf, int64_t M, int64_t N, int64_t K, void* y,
                         bool y_is_f32, int64_t ldy, int* status, bool pdl, cudaStream_t stream) {
+  // More than one 128-row tile of A: CTA pairs with 256 x 256 tiles.
+  if (M > 128) {
+    if (y_is_f32)
+      return launch_pair<6, true>(aq, asf, bq, bsf, M, N, K, y, ldy, status, pdl, stream);
+    return launch_pair<6, false>(aq, asf, bq, bsf, M, N, K, y, ldy, status, pdl, stream);
+  }
   if (y_is_f32) return launch_cfg<256, 4, true>(aq, asf, bq, bsf, M, N, K, y, ldy, status, pdl, stream);
   return launch_cfg<256, 4, false>(aq, asf, bq, bsf, M, N, K, y, ldy, status, pdl, stream);
 }

@@ -15,9 +15,10 @@ struct KronCoeffs {
 
 // Rotate (mode 0/1/2) + quantise x[rows, K] (bf16 or fp32) into packed codes q and
 // scale bytes sf (tensor-core layout, padding zeroed). Host-validated arguments.
+// status: optional device word set to the timeout code if a bounded wait gives up.
 cudaError_t launch_rotate_quantize(const void* x, bool x_is_f32, int64_t rows, int64_t K,
                                    int64_t ldx, int mode, const KronCoeffs* kc, uint8_t* q,
-                                   uint8_t* sf, cudaStream_t stream);
+                                   uint8_t* sf, int* status, cudaStream_t stream);
 
 // Block-scaled GEMM y[M, N] = A[M, K] . B[N, K]^T on tcgen05. Host-validated arguments.
 // status: device word set to the timeout code if a bounded wait gives up.

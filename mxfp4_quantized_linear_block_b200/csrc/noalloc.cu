@@ -94,7 +94,8 @@ extern "C" mxfp4_status mxfp4_linear_noalloc(const void* x, int64_t M, int64_t K
   }
   uint8_t* xq = scratch + q_off;
   uint8_t* xsf = scratch + sf_off;
-  if (launch_rotate_quantize(x, false, M, K, K, (int)mode, &kc, xq, xsf, s) != cudaSuccess)
+  if (launch_rotate_quantize(x, false, M, K, K, (int)mode, &kc, xq, xsf, status_word, s) !=
+      cudaSuccess)
     return MXFP4_ERR_CUDA;
   if (launch_gemm(xq, xsf, wq, wsf, M, N, K, y, false, N, status_word, true, s) != cudaSuccess)
     return MXFP4_ERR_CUDA;

@@ -1,12 +1,14 @@
 // quantize.cu -- online block rotation + MXFP4 quantisation (HBM-bound).
 //
-// One thread owns one 32-element block of a row. A warp owns 32 consecutive
-// blocks: it loads them with fully coalesced 16-byte loads (lane L reads
-// chunk 32*i + L of the warp's span), transposes them through a swizzled
-// shared-memory buffer so that every thread holds its own block, rotates the
-// block in registers, takes the E8M0 scale from the block amax and writes 16
-// bytes of packed E2M1 codes plus one scale byte in the tensor-core scale
-// layout. Padding rows / blocks of the scale layout are written as 0.
+// Persistent CTAs stream the input through a 4-stage ring of shared-memory
+// tiles filled by TMA (128 rows x 128 bytes per tile, 128-byte swizzle): a
+// tile holds two 32-element blocks of each of 128 bf16 rows (or one block of
+// each of 256 fp32 rows). One thread owns one block: it reads its 64 (128)
+// bytes from the swizzled tile -- bank-conflict free because of the swizzle --
+// rotates the block in registers, takes the E8M0 scale from the block amax and
+// writes 16 bytes of packed E2M1 codes plus one scale byte in the tensor-core
+// scale layout. Padding rows / blocks of the scale layout are written as 0.
+// Bytes in flight are set by the ring (48-96 KB per SM), not by registers.
 //
 // Method: "Bridging the Gap Between Promise and Performance for Microscaling
 // FP4 Quantization" ("Methodologie: MR-GPTQ" item 1: block-wise Hadamard
@@ -22,26 +24,20 @@
 // intrinsic (no contraction, no flush to zero), in the order the C ABI
 // documents, so codes and scales are bit-identical to a sequential fp32
 // evaluation of the same formulas.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include <cstdint>
 
 #include "internal.h"
+#include "sm100.cuh"
 
 namespace mxfp4 {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kWarps = kThreads / 32;
 constexpr float kInvSqrt32 = 0x1.6a09e6p-3f;  // fp32 nearest to 1/sqrt(32)
-
-__device__ __forceinline__ uint4 ld_nc_v4(const uint8_t* p) {
-  uint4 v;
-  asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p));
-  return v;
-}
 
 __device__ __forceinline__ void st_v4(uint8_t* p, uint4 v) {
   asm volatile("st.global.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z),
@@ -49,26 +45,25 @@ __device__ __forceinline__ void st_v4(uint8_t* p, uint4 v) {
                : "memory");
 }
 
-// Chunk swizzle of the per-warp transpose buffer (16-byte units): makes both
-// the coalesced stores and the per-thread block reads bank-conflict free.
-template <int CH>
-__device__ __forceinline__ uint32_t chunk_swizzle(uint32_t t) {
-  return CH == 4 ? ((t >> 1) & 3u) : (t & 7u);
-}
-
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
-// E2M1 pair: element `lo` -> bits 0-3, element `hi` -> bits 4-7; round to nearest
-// even with saturation to +-6 by the hardware conversion, sign bit forced from
-// the input so negatives that round to zero are -0 (code 8).
-__device__ __forceinline__ uint32_t e2m1x2(float lo, float hi) {
-  uint32_t r;
-  asm("{\n\t.reg .b8 t;\n\tcvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\tcvt.u32.u8 %0, t;\n\t}"
-      : "=r"(r)
-      : "f"(hi), "f"(lo));
-  r |= ((__float_as_uint(lo) >> 28) & 0x8u) | ((__float_as_uint(hi) >> 24) & 0x80u);
-  return r;
+// Eight scaled values -> one word of packed E2M1 codes (element 2j in the low
+// nibble of byte j): round to nearest even with saturation to +-6 by the
+// hardware conversion, which keeps the sign of values that round to zero
+// (code 8), as the format rule requires.
+__device__ __forceinline__ uint32_t e2m1x8(float s0, float s1, float s2, float s3, float s4,
+                                           float s5, float s6, float s7) {
+  uint32_t w;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+      : "=r"(w)
+      : "f"(s0), "f"(s1), "f"(s2), "f"(s3), "f"(s4), "f"(s5), "f"(s6), "f"(s7));
+  return w;
 }
 
 __device__ __forceinline__ float max_nan(float a, float b) {
@@ -154,61 +149,106 @@ __device__ __forceinline__ uint32_t quantize_block(const float (&v)[32], uint4& 
   const uint32_t be = mb >> 23;
   const uint32_t byte = (be > 2u ? be : 2u) - 2u;
   const float inv = __uint_as_float((254u - byte) << 23);  // 2^-e, always a normal number
+  const float2 sc = make_float2(inv, inv);
+  float s[32];
+#pragma unroll
+  for (int i = 0; i < 32; i += 2) {
+    const float2 t = __fmul2_rn(make_float2(v[i], v[i + 1]), sc);  // exact: power-of-two scale
+    s[i] = t.x;
+    s[i + 1] = t.y;
+  }
   uint32_t w[4];
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    uint32_t acc = 0;
-#pragma unroll
-    for (int p = 0; p < 4; ++p) {
-      const int i = 8 * q + 2 * p;
-      const float2 s = __fmul2_rn(make_float2(v[i], v[i + 1]), make_float2(inv, inv));
-      acc |= e2m1x2(s.x, s.y) << (8 * p);
-    }
-    w[q] = acc;
-  }
+  for (int q = 0; q < 4; ++q)
+    w[q] = e2m1x8(s[8 * q], s[8 * q + 1], s[8 * q + 2], s[8 * q + 3], s[8 * q + 4], s[8 * q + 5],
+                  s[8 * q + 6], s[8 * q + 7]);
   codes = make_uint4(w[0], w[1], w[2], w[3]);
   return byte;
 }
 
+constexpr uint32_t kStages = 4;
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
+constexpr int kTimeoutCode = 7;                  // MXFP4_ERR_TIMEOUT
+
+template <bool F32_IN>
+struct TileShape {
+  static constexpr uint32_t ROWS = F32_IN ? 256 : 128;  // rows per TMA box
+  static constexpr uint32_t BPR = F32_IN ? 1 : 2;       // 32-element blocks per row per box
+  static constexpr uint32_t STAGE = ROWS * 128;         // bytes per stage (128 bytes per row)
+  static constexpr uint32_t SMEM = kStages * STAGE + 64 + 1024;
+};
+
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr));
+  return v;
+}
+
 template <int MODE, bool F32_IN>
 __global__ void __launch_bounds__(kThreads) rotate_quantize_kernel(
-    const uint8_t* __restrict__ x, uint32_t rows, uint32_t kb_real, uint32_t kb_pad,
-    uint64_t ldx_bytes, uint64_t q_row_bytes, uint32_t n_units, uint32_t n_katoms,
-    const __grid_constant__ KronCoeffs kc, uint8_t* __restrict__ q, uint8_t* __restrict__ sf) {
+    const __grid_constant__ CUtensorMap tmap_x, uint32_t rows, uint32_t rows_pad, uint32_t kb_real,
+    uint32_t k_boxes, uint32_t tiles, uint32_t n_katoms, uint64_t q_row_bytes,
+    const __grid_constant__ KronCoeffs kc, uint8_t* __restrict__ q, uint8_t* __restrict__ sf,
+    int* status) {
+  using namespace sm100;
+  using T = TileShape<F32_IN>;
   constexpr int CH = F32_IN ? 8 : 4;  // 16-byte chunks per 32-element block
-  __shared__ uint4 stage[kWarps][32 * CH];
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_addr(smem_raw);
+  const uint32_t sbase = (raw_addr + 1023u) & ~1023u;  // 128-byte swizzle needs 1024-byte alignment
+  const uint32_t bar_full = sbase + kStages * T::STAGE;
+  volatile int* abort_flag =
+      reinterpret_cast<volatile int*>(smem_raw + (bar_full - raw_addr) + 8 * kStages);
+
   const uint32_t lane = threadIdx.x & 31u, warp = threadIdx.x >> 5;
-  uint4* buf = stage[warp];
+  // thread -> (row inside the tile, block inside the row)
+  const uint32_t r_loc = F32_IN ? warp * 32u + lane : warp * 16u + (lane >> 1);
+  const uint32_t b_loc = F32_IN ? 0u : (lane & 1u);
 
-  for (uint32_t base = blockIdx.x * kThreads + warp * 32u; base < n_units;
-       base += gridDim.x * kThreads) {
-    const uint32_t u = base + lane;
-    const uint32_t r = u / kb_pad;
-    const uint32_t kb = u - r * kb_pad;
-    const bool live = u < n_units && r < rows && kb < kb_real;
-    const unsigned long long src =
-        live ? reinterpret_cast<unsigned long long>(x + (uint64_t)r * ldx_bytes +
-                                                    (uint64_t)kb * (CH * 16))
-             : 0ull;
+  if (threadIdx.x == 0) {
+    for (uint32_t s = 0; s < kStages; ++s) mbar_init(bar_full + 8 * s, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tmap(&tmap_x);
+  }
+  __syncthreads();
 
-    // Coalesced loads of the warp's 32 blocks, then transpose through shared memory.
-    uint4 ld[CH];
-#pragma unroll
-    for (int i = 0; i < CH; ++i) {
-      const uint32_t g = 32u * i + lane, t = g / CH, c = g % CH;
-      const unsigned long long p = __shfl_sync(0xffffffffu, src, t);
-      ld[i] = p ? ld_nc_v4(reinterpret_cast<const uint8_t*>(p) + c * 16) : make_uint4(0, 0, 0, 0);
+  auto issue = [&](uint32_t tile, uint32_t s) {
+    const uint32_t rt = tile / k_boxes, kx = tile - rt * k_boxes;
+    mbar_arrive_expect_tx(bar_full + 8 * s, T::STAGE);
+    tma_load_2d(sbase + s * T::STAGE, &tmap_x, bar_full + 8 * s, (int32_t)(kx * (F32_IN ? 32 : 64)),
+                (int32_t)(rt * T::ROWS));
+  };
+  uint32_t issued = 0;
+  if (threadIdx.x == 0)
+    for (uint32_t j = 0; j < kStages; ++j) {
+      const uint32_t t = blockIdx.x + j * gridDim.x;
+      if (t < tiles) {
+        issue(t, j);
+        ++issued;
+      }
     }
-#pragma unroll
-    for (int i = 0; i < CH; ++i) {
-      const uint32_t g = 32u * i + lane, t = g / CH, c = g % CH;
-      buf[t * CH + (c ^ chunk_swizzle<CH>(t))] = ld[i];
+
+  uint32_t i = 0;
+  for (uint32_t tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++i) {
+    const uint32_t s = i % kStages;
+    const bool ok = mbar_wait_bounded(bar_full + 8 * s, (i / kStages) & 1u, abort_flag, kWaitLimitNs);
+    if (__syncthreads_or(!ok)) {
+      if (threadIdx.x == 0 && status) atomicExch(status, kTimeoutCode);
+      break;
     }
-    __syncwarp();
+    const uint32_t rt = tile / k_boxes, kx = tile - rt * k_boxes;
+    const uint32_t row = rt * T::ROWS + r_loc;
+    const uint32_t kb = kx * T::BPR + b_loc;
+
     float v[32];
+    const uint32_t rbase = sbase + s * T::STAGE + r_loc * 128u;
 #pragma unroll
     for (int c = 0; c < CH; ++c) {
-      const uint4 w = buf[lane * CH + (c ^ chunk_swizzle<CH>(lane))];
+      const uint32_t chunk = ((b_loc * CH + (uint32_t)c) ^ (r_loc & 7u)) << 4;
+      const uint4 w = ld_shared_v4(rbase + chunk);
       if constexpr (F32_IN) {
         v[4 * c + 0] = __uint_as_float(w.x);
         v[4 * c + 1] = __uint_as_float(w.y);
@@ -225,44 +265,98 @@ __global__ void __launch_bounds__(kThreads) rotate_quantize_kernel(
         v[8 * c + 7] = bf16_hi(w.w);
       }
     }
-    __syncwarp();
+    __syncthreads();  // every thread has its block in registers: the stage may be refilled
+    if (threadIdx.x == 0) {
+      const uint32_t next = tile + kStages * gridDim.x;
+      if (next < tiles) {
+        issue(next, s);
+        ++issued;
+      }
+    }
 
-    if (u < n_units) {
+    if (row < rows_pad) {
       uint32_t byte = 0;
-      if (live) {
+      if (row < rows && kb < kb_real) {
         if constexpr (MODE == 1) hadamard32(v);
         if constexpr (MODE == 2) kron32(v, kc);
         uint4 codes;
         byte = quantize_block(v, codes);
-        st_v4(q + (uint64_t)r * q_row_bytes + (uint64_t)kb * 16u, codes);
+        st_v4(q + (uint64_t)row * q_row_bytes + (uint64_t)kb * 16u, codes);
       }
-      const uint64_t off = ((uint64_t)(r >> 7) * n_katoms + (kb >> 2)) * 512u + (r & 31u) * 16u +
-                           ((r >> 5) & 3u) * 4u + (kb & 3u);
+      const uint64_t off = ((uint64_t)(row >> 7) * n_katoms + (kb >> 2)) * 512u +
+                           (row & 31u) * 16u + ((row >> 5) & 3u) * 4u + (kb & 3u);
       sf[off] = static_cast<uint8_t>(byte);
     }
+  }
+  // After an early stop, loads already issued still land in this CTA's shared memory.
+  if (threadIdx.x == 0 && *abort_flag) {
+    volatile int never = 0;
+    for (uint32_t j = i; j < issued; ++j)
+      mbar_wait_bounded(bar_full + 8 * (j % kStages), (j / kStages) & 1u, &never, kWaitLimitNs);
   }
   // Let a dependent kernel (the GEMM of the fused layer) start its set-up; it
   // still waits for this grid's completion before reading q / sf.
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult qr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &qr) ==
+            cudaSuccess &&
+        qr == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
 template <int MODE, bool F32_IN>
 cudaError_t launch_mode(const void* x, int64_t rows, int64_t K, int64_t ldx, const KronCoeffs& kc,
-                        uint8_t* q, uint8_t* sf, cudaStream_t stream) {
+                        uint8_t* q, uint8_t* sf, int* status, cudaStream_t stream) {
+  using T = TileShape<F32_IN>;
+  auto fn = encode_fn();
+  if (!fn) return cudaErrorNotSupported;
+  CUtensorMap map;
+  cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)ldx * (F32_IN ? 4u : 2u)};
+  cuuint32_t box[2] = {F32_IN ? 32u : 64u, T::ROWS};
+  cuuint32_t estr[2] = {1, 1};
+  if (fn(&map, F32_IN ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+         const_cast<void*>(x), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+
+  auto kern = rotate_quantize_kernel<MODE, F32_IN>;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  static int per_sm[64] = {};
+  static int sms[64] = {};
+  if (!per_sm[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, T::SMEM);
+    if (e != cudaSuccess) return e;
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kThreads, T::SMEM) != cudaSuccess ||
+        n <= 0)
+      n = 1;
+    cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev);
+    per_sm[dev] = n;
+  }
   const int64_t kb_real = K / 32;
   const int64_t kb_pad = sf_katoms(K) * 4;
   const int64_t rows_pad = sf_row_tiles(rows) * 128;
-  const int64_t n_units = rows_pad * kb_pad;
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int64_t blocks_needed = (n_units + kThreads - 1) / kThreads;
-  const int64_t cap = (int64_t)sms * 8;  // grid-stride beyond 8 CTAs per SM
-  const int grid = (int)(blocks_needed < cap ? blocks_needed : cap);
-  rotate_quantize_kernel<MODE, F32_IN><<<grid, kThreads, 0, stream>>>(
-      static_cast<const uint8_t*>(x), (uint32_t)rows, (uint32_t)kb_real, (uint32_t)kb_pad,
-      (uint64_t)ldx * (F32_IN ? 4u : 2u), (uint64_t)(K / 2), (uint32_t)n_units,
-      (uint32_t)sf_katoms(K), kc, q, sf);
+  const int64_t k_boxes = kb_pad / T::BPR;
+  const int64_t row_tiles = (rows_pad + T::ROWS - 1) / T::ROWS;
+  const int64_t tiles = row_tiles * k_boxes;
+  const int64_t cap = (int64_t)sms[dev] * per_sm[dev];
+  const int grid = (int)(tiles < cap ? tiles : cap);
+  kern<<<grid, kThreads, T::SMEM, stream>>>(map, (uint32_t)rows, (uint32_t)rows_pad,
+                                             (uint32_t)kb_real, (uint32_t)k_boxes, (uint32_t)tiles,
+                                             (uint32_t)sf_katoms(K), (uint64_t)(K / 2), kc, q, sf,
+                                             status);
   return cudaGetLastError();
 }
 
@@ -270,17 +364,17 @@ cudaError_t launch_mode(const void* x, int64_t rows, int64_t K, int64_t ldx, con
 
 cudaError_t launch_rotate_quantize(const void* x, bool x_is_f32, int64_t rows, int64_t K,
                                    int64_t ldx, int mode, const KronCoeffs* kc, uint8_t* q,
-                                   uint8_t* sf, cudaStream_t stream) {
+                                   uint8_t* sf, int* status, cudaStream_t stream) {
   KronCoeffs k{};
   if (kc) k = *kc;
   if (x_is_f32) {
-    if (mode == 1) return launch_mode<1, true>(x, rows, K, ldx, k, q, sf, stream);
-    if (mode == 2) return launch_mode<2, true>(x, rows, K, ldx, k, q, sf, stream);
-    return launch_mode<0, true>(x, rows, K, ldx, k, q, sf, stream);
+    if (mode == 1) return launch_mode<1, true>(x, rows, K, ldx, k, q, sf, status, stream);
+    if (mode == 2) return launch_mode<2, true>(x, rows, K, ldx, k, q, sf, status, stream);
+    return launch_mode<0, true>(x, rows, K, ldx, k, q, sf, status, stream);
   }
-  if (mode == 1) return launch_mode<1, false>(x, rows, K, ldx, k, q, sf, stream);
-  if (mode == 2) return launch_mode<2, false>(x, rows, K, ldx, k, q, sf, stream);
-  return launch_mode<0, false>(x, rows, K, ldx, k, q, sf, stream);
+  if (mode == 1) return launch_mode<1, false>(x, rows, K, ldx, k, q, sf, status, stream);
+  if (mode == 2) return launch_mode<2, false>(x, rows, K, ldx, k, q, sf, status, stream);
+  return launch_mode<0, false>(x, rows, K, ldx, k, q, sf, status, stream);
 }
 
 }  // namespace mxfp4
