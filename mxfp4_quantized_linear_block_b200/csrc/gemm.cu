@@ -363,7 +363,9 @@ struct PairConfig {
   static constexpr uint32_t OFF_B = OFF_A + STAGES * A_STAGE;
   static constexpr uint32_t OFF_SFA = OFF_B + STAGES * B_STAGE;
   static constexpr uint32_t OFF_SFB = OFF_SFA + STAGES * SFA_STAGE;
-  static constexpr uint32_t OFF_BAR = OFF_SFB + STAGES * SFB_STAGE;
+  static constexpr uint32_t EPI_BUF = 32 * 128;  // per epilogue warp: 32 rows x 128 bytes
+  static constexpr uint32_t OFF_EPI = OFF_SFB + STAGES * SFB_STAGE;
+  static constexpr uint32_t OFF_BAR = OFF_EPI + kEpiWarps * EPI_BUF;
   static constexpr uint32_t NUM_BARS = 2 * STAGES + 3;
   static constexpr uint32_t OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr uint32_t SMEM_BYTES = OFF_MISC + 16 + 1024;
@@ -378,7 +380,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     mxf4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a,
                           const __grid_constant__ CUtensorMap tmap_b,
                           const __grid_constant__ CUtensorMap tmap_sfa,
-                          const __grid_constant__ CUtensorMap tmap_sfb, const Params p) {
+                          const __grid_constant__ CUtensorMap tmap_sfb,
+                          const __grid_constant__ CUtensorMap tmap_y, const Params p) {
   using C = PairConfig<STAGES>;
   constexpr uint32_t BN = C::BN;
   extern __shared__ uint8_t smem_raw[];
@@ -415,6 +418,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     prefetch_tmap(&tmap_b);
     prefetch_tmap(&tmap_sfa);
     prefetch_tmap(&tmap_sfb);
+    prefetch_tmap(&tmap_y);
   }
   if (warp == kMmaWarp) {
     tmem_alloc_pair(smem_addr(tmem_slot), C::TMEM_COLS);
@@ -553,33 +557,43 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(tempty_at_leader);
 
-      const uint32_t row = mt * 256u + rank * 128u + quad * 32u + lane;
-      const uint32_t col0 = nt * BN + half * COLS;
-      if (row < p.M) {
-        if constexpr (Y_F32) {
-          float* yrow = static_cast<float*>(p.y) + (uint64_t)row * p.ldy + col0;
+      // Output: each warp stages 32 rows x 128 bytes at a time in its own shared
+      // buffer (128-byte swizzle, bank-conflict free) and writes it with a TMA
+      // store, which also clips rows >= M and columns >= N.
+      const int32_t row0 = (int32_t)(mt * 256u + rank * 128u + quad * 32u);
+      const int32_t col0 = (int32_t)(nt * BN + half * COLS);
+      const uint32_t buf = sbase + C::OFF_EPI + (warp - kFirstEpiWarp) * C::EPI_BUF;
+      const uint32_t rowoff = buf + lane * 128u;
+      constexpr uint32_t CCOLS = Y_F32 ? 32 : 64;  // columns per 128-byte chunk row
 #pragma unroll
-          for (uint32_t c = 0; c < CHUNKS; ++c)
+      for (uint32_t c = 0; c < COLS / CCOLS; ++c) {
+        if (lane == 0) bulk_wait_read_all();  // the buffer's previous store has read it
+        __syncwarp();
 #pragma unroll
-            for (uint32_t j = 0; j < 32; j += 4)
-              if (col0 + 32 * c + j < p.N)
-                st_global_v4(yrow + 32 * c + j, v[c][j], v[c][j + 1], v[c][j + 2], v[c][j + 3]);
-        } else {
-          uint16_t* yrow = static_cast<uint16_t*>(p.y) + (uint64_t)row * p.ldy + col0;
-#pragma unroll
-          for (uint32_t c = 0; c < CHUNKS; ++c)
-#pragma unroll
-            for (uint32_t j = 0; j < 32; j += 8)
-              if (col0 + 32 * c + j < p.N)
-                st_global_v4(yrow + 32 * c + j,
-                             pack_bf16x2(__uint_as_float(v[c][j]), __uint_as_float(v[c][j + 1])),
-                             pack_bf16x2(__uint_as_float(v[c][j + 2]), __uint_as_float(v[c][j + 3])),
-                             pack_bf16x2(__uint_as_float(v[c][j + 4]), __uint_as_float(v[c][j + 5])),
-                             pack_bf16x2(__uint_as_float(v[c][j + 6]), __uint_as_float(v[c][j + 7])));
+        for (uint32_t j = 0; j < 8; ++j) {
+          const uint32_t addr = rowoff + ((j ^ (lane & 7u)) << 4);
+          if constexpr (Y_F32) {
+            const uint32_t* src = &v[c][4 * j];
+            st_shared_v4(addr, src[0], src[1], src[2], src[3]);
+          } else {
+            const uint32_t* src = &v[(2 * c * 32 + 8 * j) / 32][(8 * j) % 32];
+            st_shared_v4(addr, pack_bf16x2(__uint_as_float(src[0]), __uint_as_float(src[1])),
+                         pack_bf16x2(__uint_as_float(src[2]), __uint_as_float(src[3])),
+                         pack_bf16x2(__uint_as_float(src[4]), __uint_as_float(src[5])),
+                         pack_bf16x2(__uint_as_float(src[6]), __uint_as_float(src[7])));
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&tmap_y, buf, col0 + (int32_t)(c * CCOLS), row0);
+          bulk_commit_group();
         }
       }
       acc_phase ^= 1u;
     }
+    if (lane == 0) bulk_wait_all();  // this warp's output stores are complete
+    __syncwarp();
   }
 
   tc_fence_before();
@@ -648,17 +662,33 @@ bool make_scale_map(CUtensorMap* map, const uint8_t* sf, uint64_t row_tiles, uin
   return r == CUDA_SUCCESS;
 }
 
+// Output map: [M, N] row-major bf16 / fp32, box = 128 bytes of a row x 32 rows, 128-byte swizzle.
+bool make_output_map(CUtensorMap* map, void* y, uint64_t M, uint64_t N, uint64_t ldy, bool f32) {
+  auto fn = get_encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {N, M};
+  cuuint64_t strides[1] = {ldy * (f32 ? 4u : 2u)};
+  cuuint32_t box[2] = {f32 ? 32u : 64u, 32u};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                  y, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 template <uint32_t STAGES, bool Y_F32>
 cudaError_t launch_pair(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq,
                         const uint8_t* bsf, int64_t M, int64_t N, int64_t K, void* y, int64_t ldy,
                         int* status, bool pdl, cudaStream_t stream) {
   using C = PairConfig<STAGES>;
   const uint64_t k_atoms = (uint64_t)sf_katoms(K);
-  CUtensorMap ta, tb, tsa, tsb;
+  CUtensorMap ta, tb, tsa, tsb, ty;
   if (!make_operand_map(&ta, aq, (uint64_t)M, (uint64_t)(K / 2), 128) ||
       !make_operand_map(&tb, bq, (uint64_t)N, (uint64_t)(K / 2), 128) ||
       !make_scale_map(&tsa, asf, (uint64_t)sf_row_tiles(M), k_atoms, false) ||
-      !make_scale_map(&tsb, bsf, (uint64_t)sf_row_tiles(N), k_atoms, true))
+      !make_scale_map(&tsb, bsf, (uint64_t)sf_row_tiles(N), k_atoms, true) ||
+      !make_output_map(&ty, y, (uint64_t)M, (uint64_t)N, (uint64_t)ldy, Y_F32))
     return cudaErrorInvalidValue;
   auto kern = mxf4_gemm_pair_kernel<STAGES, Y_F32>;
   int dev = 0;
@@ -711,7 +741,7 @@ cudaError_t launch_pair(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, kern, ta, tb, tsa, tsb, p);
+  return cudaLaunchKernelEx(&cfg, kern, ta, tb, tsa, tsb, ty, p);
 }
 
 template <uint32_t BN, uint32_t STAGES, bool Y_F32>
@@ -774,8 +804,8 @@ cudaError_t launch_gemm(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq
   // More than one 128-row tile of A: CTA pairs with 256 x 256 tiles.
   if (M > 128) {
     if (y_is_f32)
-      return launch_pair<6, true>(aq, asf, bq, bsf, M, N, K, y, ldy, status, pdl, stream);
-    return launch_pair<6, false>(aq, asf, bq, bsf, M, N, K, y, ldy, status, pdl, stream);
+      return launch_pair<5, true>(aq, asf, bq, bsf, M, N, K, y, ldy, status, pdl, stream);
+    return launch_pair<5, false>(aq, asf, bq, bsf, M, N, K, y, ldy, status, pdl, stream);
   }
   if (y_is_f32) return launch_cfg<256, 4, true>(aq, asf, bq, bsf, M, N, K, y, ldy, status, pdl, stream);
   return launch_cfg<256, 4, false>(aq, asf, bq, bsf, M, N, K, y, ldy, status, pdl, stream);
