@@ -369,9 +369,15 @@ struct PairConfig {
   static constexpr uint32_t NUM_BARS = 2 * STAGES + 3;
   static constexpr uint32_t OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr uint32_t SMEM_BYTES = OFF_MISC + 16 + 1024;
-  static constexpr uint32_t SFA_COL = BN;       // after the 256-column accumulator
+  // Two 256-column accumulators that share 64 columns: tile i uses columns
+  // [ACC_BASE[i % 2], +256). The epilogue drains the shared 64 columns first and
+  // then hands the accumulator back, so the next tile's MMAs overlap the rest of
+  // the drain.
+  static constexpr uint32_t ACC1_COL = 192;
+  static constexpr uint32_t SFA_COL = ACC1_COL + BN;  // 448
   static constexpr uint32_t SFB_COL = SFA_COL + 8;
   static constexpr uint32_t TMEM_COLS = 512;
+  static_assert(SFB_COL + 16 <= TMEM_COLS, "tensor memory budget");
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
@@ -410,7 +416,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       mbar_init(bar_empty + 8 * s, 1);
     }
     mbar_init(bar_tfull, 1);
-    mbar_init(bar_tempty, 2 * kEpiWarps);
+    mbar_init(bar_tempty, 2 * (kEpiWarps / 2));  // the 4 warps draining the shared columns, x2 CTAs
     mbar_init(bar_mma_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -493,6 +499,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           break;
         }
         tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (acc_phase ? C::ACC1_COL : 0u);
         for (uint32_t kt = 0; kt < p.k_tiles; ++kt) {
           if (!mbar_wait_bounded(bar_full + 8 * stage, phase, abort_flag, kWaitLimitNs)) {
             ok = false;
@@ -513,7 +520,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           const uint32_t b_tile = sbase + C::OFF_B + stage * C::B_STAGE;
           for (uint32_t k = 0; k < steps; ++k) {
             const uint32_t sf_id = (k & 1u) * 2u;
-            mma_mxf4_pair(tmem_base, smem_desc_sw128(a_tile + k * MMA_K_BYTES),
+            mma_mxf4_pair(d_tmem, smem_desc_sw128(a_tile + k * MMA_K_BYTES),
                           smem_desc_sw128(b_tile + k * MMA_K_BYTES), idesc_mxf4(256, BN, sf_id, sf_id),
                           tmem_base + C::SFA_COL + 4 * (k >> 1), tmem_base + C::SFB_COL + 8 * (k >> 1),
                           (kt | k) != 0u);
@@ -548,25 +555,44 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
+      // 64-column chunks of this tile's accumulator; chunk `shared` is the one the
+      // other accumulator overlaps. Warps of half 0 drain it first and release the
+      // accumulator; every warp then drains its second chunk.
+      const uint32_t acc_col = acc_phase ? C::ACC1_COL : 0u;
+      const uint32_t shared_chunk = acc_phase ? 0u : 3u;
+      uint32_t ch[2];
+      if (half == 0) {
+        ch[0] = shared_chunk;
+        ch[1] = acc_phase ? 1u : 2u;
+      } else {
+        ch[0] = acc_phase ? 2u : 0u;
+        ch[1] = acc_phase ? 3u : 1u;
+      }
       uint32_t v[CHUNKS][32];
-      const uint32_t taddr = tmem_base + ((quad * 32u) << 16) + half * COLS;
-#pragma unroll
-      for (uint32_t c = 0; c < CHUNKS; ++c) tmem_ld_32x32b_x32(taddr + 32 * c, v[c]);
+      const uint32_t taddr = tmem_base + ((quad * 32u) << 16) + acc_col;
+      tmem_ld_32x32b_x32(taddr + ch[0] * 64u, v[0]);
+      tmem_ld_32x32b_x32(taddr + ch[0] * 64u + 32u, v[1]);
+      if (half == 0) {
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(tempty_at_leader);
+      }
+      tmem_ld_32x32b_x32(taddr + ch[1] * 64u, v[2]);
+      tmem_ld_32x32b_x32(taddr + ch[1] * 64u + 32u, v[3]);
       tmem_ld_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(tempty_at_leader);
 
       // Output: each warp stages 32 rows x 128 bytes at a time in its own shared
       // buffer (128-byte swizzle, bank-conflict free) and writes it with a TMA
       // store, which also clips rows >= M and columns >= N.
       const int32_t row0 = (int32_t)(mt * 256u + rank * 128u + quad * 32u);
-      const int32_t col0 = (int32_t)(nt * BN + half * COLS);
       const uint32_t buf = sbase + C::OFF_EPI + (warp - kFirstEpiWarp) * C::EPI_BUF;
       const uint32_t rowoff = buf + lane * 128u;
       constexpr uint32_t CCOLS = Y_F32 ? 32 : 64;  // columns per 128-byte chunk row
 #pragma unroll
       for (uint32_t c = 0; c < COLS / CCOLS; ++c) {
+        // register group c*CCOLS/32 .. holds tile columns ch[c*CCOLS/64]*64 + (c*CCOLS)%64 ..
+        const int32_t col0 = (int32_t)(nt * BN + ch[(c * CCOLS) / 64] * 64u + (c * CCOLS) % 64u);
         if (lane == 0) bulk_wait_read_all();  // the buffer's previous store has read it
         __syncwarp();
 #pragma unroll
@@ -586,7 +612,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          tma_store_2d(&tmap_y, buf, col0 + (int32_t)(c * CCOLS), row0);
+          tma_store_2d(&tmap_y, buf, col0, row0);
           bulk_commit_group();
         }
       }
