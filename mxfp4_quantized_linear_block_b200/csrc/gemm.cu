@@ -26,6 +26,7 @@
 
 #include <cstdint>
 
+#include "block_quant.cuh"
 #include "internal.h"
 #include "sm100.cuh"
 
@@ -351,6 +352,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 // epilogues. Tile loads of both CTAs complete on the leader's stage barrier;
 // the leader's commits arrive on both CTAs' barriers. No load is multicast.
 
+
 template <uint32_t STAGES>
 struct PairConfig {
   static constexpr uint32_t BN = 256;                 // N per pair tile
@@ -370,9 +372,9 @@ struct PairConfig {
   static constexpr uint32_t OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr uint32_t SMEM_BYTES = OFF_MISC + 16 + 1024;
   // Two 256-column accumulators that share 64 columns: tile i uses columns
-  // [ACC_BASE[i % 2], +256). The epilogue drains the shared 64 columns first and
-  // then hands the accumulator back, so the next tile's MMAs overlap the rest of
-  // the drain.
+  // [0, 256) or [192, 448) alternately. The epilogue drains the shared 64
+  // columns first and then hands the accumulator back, so the next tile's MMAs
+  // overlap the rest of the drain.
   static constexpr uint32_t ACC1_COL = 192;
   static constexpr uint32_t SFA_COL = ACC1_COL + BN;  // 448
   static constexpr uint32_t SFB_COL = SFA_COL + 8;
@@ -405,7 +407,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const uint32_t bar_full = sbase + C::OFF_BAR;        // [STAGES], leader's count both CTAs
   const uint32_t bar_empty = bar_full + 8 * STAGES;    // [STAGES]
   const uint32_t bar_tfull = bar_empty + 8 * STAGES;   // accumulator ready
-  const uint32_t bar_tempty = bar_tfull + 8;           // leader: accumulator drained (both CTAs)
+  const uint32_t bar_tempty = bar_tfull + 8;           // leader: shared columns drained
   const uint32_t bar_mma_done = bar_tempty + 8;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
@@ -436,6 +438,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
+  // Operands may be produced by the kernel launched just before this one.
   griddep_wait();
 
   const uint32_t n_tiles_total = p.m_tiles * p.n_tiles;  // m_tiles counts 256-row pair tiles
@@ -541,23 +544,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       mbar_wait_bounded(bar_mma_done, 0, &never, kWaitLimitNs);
     }
   } else {
+    // Epilogue. Warp w owns TMEM lanes 32 * (w % 4) .. +31 and two of the tile's
+    // four 64-column chunks; the half-0 warps take the chunk the other
+    // accumulator overlaps first and release the accumulator after reading it.
+    // Each chunk goes TMEM -> registers -> bf16/fp32 -> the warp's swizzled
+    // shared buffer -> TMA store (which clips rows >= M and columns >= N).
     const uint32_t quad = warp & 3u;
     const uint32_t half = (warp - kFirstEpiWarp) / 4u;
-    constexpr uint32_t COLS = BN / 2;
-    constexpr uint32_t CHUNKS = COLS / 32;
     const uint32_t tempty_at_leader = map_to_rank(bar_tempty, 0);
+    const uint32_t buf = sbase + C::OFF_EPI + (warp - kFirstEpiWarp) * C::EPI_BUF;
+    const uint32_t rowoff = buf + lane * 128u;
+    constexpr uint32_t CCOLS = Y_F32 ? 32 : 64;  // columns per 128-byte staged row
     uint32_t acc_phase = 0;
     for (uint32_t tile = pair; tile < n_tiles_total; tile += num_pairs) {
       const uint32_t mt = tile / p.n_tiles, nt = tile % p.n_tiles;
       const bool ok = mbar_wait_bounded(bar_tfull, acc_phase, abort_flag, kWaitLimitNs);
-      if (!__all_sync(0xffffffffu, ok)) {
+      if (!__all_sync(0xffffffffu, ok)) {  // leave together so .aligned ops stay convergent
         if (lane == 0) record_timeout(p.status);
         break;
       }
       tc_fence_after();
-      // 64-column chunks of this tile's accumulator; chunk `shared` is the one the
-      // other accumulator overlaps. Warps of half 0 drain it first and release the
-      // accumulator; every warp then drains its second chunk.
       const uint32_t acc_col = acc_phase ? C::ACC1_COL : 0u;
       const uint32_t shared_chunk = acc_phase ? 0u : 3u;
       uint32_t ch[2];
@@ -568,52 +574,44 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         ch[0] = acc_phase ? 2u : 0u;
         ch[1] = acc_phase ? 3u : 1u;
       }
-      uint32_t v[CHUNKS][32];
       const uint32_t taddr = tmem_base + ((quad * 32u) << 16) + acc_col;
-      tmem_ld_32x32b_x32(taddr + ch[0] * 64u, v[0]);
-      tmem_ld_32x32b_x32(taddr + ch[0] * 64u + 32u, v[1]);
-      if (half == 0) {
-        tmem_ld_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(tempty_at_leader);
-      }
-      tmem_ld_32x32b_x32(taddr + ch[1] * 64u, v[2]);
-      tmem_ld_32x32b_x32(taddr + ch[1] * 64u + 32u, v[3]);
-      tmem_ld_wait();
-
-      // Output: each warp stages 32 rows x 128 bytes at a time in its own shared
-      // buffer (128-byte swizzle, bank-conflict free) and writes it with a TMA
-      // store, which also clips rows >= M and columns >= N.
       const int32_t row0 = (int32_t)(mt * 256u + rank * 128u + quad * 32u);
-      const uint32_t buf = sbase + C::OFF_EPI + (warp - kFirstEpiWarp) * C::EPI_BUF;
-      const uint32_t rowoff = buf + lane * 128u;
-      constexpr uint32_t CCOLS = Y_F32 ? 32 : 64;  // columns per 128-byte chunk row
 #pragma unroll
-      for (uint32_t c = 0; c < COLS / CCOLS; ++c) {
-        // register group c*CCOLS/32 .. holds tile columns ch[c*CCOLS/64]*64 + (c*CCOLS)%64 ..
-        const int32_t col0 = (int32_t)(nt * BN + ch[(c * CCOLS) / 64] * 64u + (c * CCOLS) % 64u);
-        if (lane == 0) bulk_wait_read_all();  // the buffer's previous store has read it
-        __syncwarp();
-#pragma unroll
-        for (uint32_t j = 0; j < 8; ++j) {
-          const uint32_t addr = rowoff + ((j ^ (lane & 7u)) << 4);
-          if constexpr (Y_F32) {
-            const uint32_t* src = &v[c][4 * j];
-            st_shared_v4(addr, src[0], src[1], src[2], src[3]);
-          } else {
-            const uint32_t* src = &v[(2 * c * 32 + 8 * j) / 32][(8 * j) % 32];
-            st_shared_v4(addr, pack_bf16x2(__uint_as_float(src[0]), __uint_as_float(src[1])),
-                         pack_bf16x2(__uint_as_float(src[2]), __uint_as_float(src[3])),
-                         pack_bf16x2(__uint_as_float(src[4]), __uint_as_float(src[5])),
-                         pack_bf16x2(__uint_as_float(src[6]), __uint_as_float(src[7])));
-          }
+      for (uint32_t r = 0; r < 2; ++r) {
+        uint32_t v[2][32];
+        tmem_ld_32x32b_x32(taddr + ch[r] * 64u, v[0]);
+        tmem_ld_32x32b_x32(taddr + ch[r] * 64u + 32u, v[1]);
+        tmem_ld_wait();
+        if (r == 0 && half == 0) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster(tempty_at_leader);
         }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          tma_store_2d(&tmap_y, buf, col0, row0);
-          bulk_commit_group();
+#pragma unroll
+        for (uint32_t c = 0; c < 64 / CCOLS; ++c) {
+          const int32_t col0 = (int32_t)(nt * BN + ch[r] * 64u + c * CCOLS);
+          if (lane == 0) bulk_wait_read_all();  // the buffer's previous store has read it
+          __syncwarp();
+#pragma unroll
+          for (uint32_t j = 0; j < 8; ++j) {
+            const uint32_t addr = rowoff + ((j ^ (lane & 7u)) << 4);
+            if constexpr (Y_F32) {
+              const uint32_t* src = &v[c][4 * j];
+              st_shared_v4(addr, src[0], src[1], src[2], src[3]);
+            } else {
+              const uint32_t* src = &v[j / 4][(8 * j) % 32];
+              st_shared_v4(addr, pack_bf16x2(__uint_as_float(src[0]), __uint_as_float(src[1])),
+                           pack_bf16x2(__uint_as_float(src[2]), __uint_as_float(src[3])),
+                           pack_bf16x2(__uint_as_float(src[4]), __uint_as_float(src[5])),
+                           pack_bf16x2(__uint_as_float(src[6]), __uint_as_float(src[7])));
+            }
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tmap_y, buf, col0, row0);
+            bulk_commit_group();
+          }
         }
       }
       acc_phase ^= 1u;

@@ -30,142 +30,16 @@
 
 #include <cstdint>
 
+#include "block_quant.cuh"
 #include "internal.h"
 #include "sm100.cuh"
 
 namespace mxfp4 {
 namespace {
 
+using namespace blockq;
+
 constexpr int kThreads = 256;
-constexpr float kInvSqrt32 = 0x1.6a09e6p-3f;  // fp32 nearest to 1/sqrt(32)
-
-__device__ __forceinline__ void st_v4(uint8_t* p, uint4 v) {
-  asm volatile("st.global.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z),
-               "r"(v.w)
-               : "memory");
-}
-
-__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
-
-// Eight scaled values -> one word of packed E2M1 codes (element 2j in the low
-// nibble of byte j): round to nearest even with saturation to +-6 by the
-// hardware conversion, which keeps the sign of values that round to zero
-// (code 8), as the format rule requires.
-__device__ __forceinline__ uint32_t e2m1x8(float s0, float s1, float s2, float s3, float s4,
-                                           float s5, float s6, float s7) {
-  uint32_t w;
-  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
-      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
-      : "=r"(w)
-      : "f"(s0), "f"(s1), "f"(s2), "f"(s3), "f"(s4), "f"(s5), "f"(s6), "f"(s7));
-  return w;
-}
-
-__device__ __forceinline__ float max_nan(float a, float b) {
-  float d;
-  asm("max.NaN.f32 %0, %1, %2;" : "=f"(d) : "f"(a), "f"(b));
-  return d;
-}
-
-__device__ __forceinline__ float max3_nan(float a, float b, float c) {
-  float d;
-  asm("max.NaN.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
-  return d;
-}
-
-// Normalised Sylvester Hadamard of one block: butterfly stages with strides
-// 1, 2, 4, 8, 16 ((a, b) -> (a + b, a - b)), then one multiply by kInvSqrt32.
-// Stages 1..8 run on packed pairs (v[t], v[t + 16]); stage 16 pairs the two
-// halves of each packed value.
-__device__ __forceinline__ void hadamard32(float (&v)[32]) {
-  float2 P[16];
-#pragma unroll
-  for (int t = 0; t < 16; ++t) P[t] = make_float2(v[t], v[t + 16]);
-#pragma unroll
-  for (int h = 1; h < 16; h <<= 1) {
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      if (i & h) continue;
-      const float2 a = P[i], b = P[i + h];
-      P[i] = __fadd2_rn(a, b);
-      P[i + h] = __fadd2_rn(a, make_float2(-b.x, -b.y));
-    }
-  }
-  const float2 c = make_float2(kInvSqrt32, kInvSqrt32);
-#pragma unroll
-  for (int t = 0; t < 16; ++t) {
-    const float a = P[t].x, b = P[t].y;
-    const float2 s = make_float2(__fadd_rn(a, b), __fsub_rn(a, b));
-    const float2 r = __fmul2_rn(s, c);
-    v[t] = r.x;
-    v[t + 16] = r.y;
-  }
-}
-
-// y = (A (x) B) x: z[8j+k] = sum_l B[k][l] x[8j+l], y[8i+k] = sum_j A[i][j] z[8j+k],
-// each sum a chain that starts with the first product and adds the rest by fma
-// in ascending index order.
-__device__ __forceinline__ void kron32(float (&v)[32], const KronCoeffs& kc) {
-  float z[32];
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      float acc = __fmul_rn(kc.b[k * 8 + 0], v[8 * j + 0]);
-#pragma unroll
-      for (int l = 1; l < 8; ++l) acc = __fmaf_rn(kc.b[k * 8 + l], v[8 * j + l], acc);
-      z[8 * j + k] = acc;
-    }
-  }
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      float acc = __fmul_rn(kc.a[i * 4 + 0], z[k]);
-#pragma unroll
-      for (int j = 1; j < 4; ++j) acc = __fmaf_rn(kc.a[i * 4 + j], z[8 * j + k], acc);
-      v[8 * i + k] = acc;
-    }
-  }
-}
-
-// Quantise one rotated block: returns the E8M0 byte and the 16 code bytes.
-__device__ __forceinline__ uint32_t quantize_block(const float (&v)[32], uint4& codes) {
-  // amax with NaN propagation (a NaN anywhere makes m NaN).
-  float m = max_nan(fabsf(v[0]), fabsf(v[31]));
-#pragma unroll
-  for (int i = 1; i < 31; i += 2) m = max3_nan(m, fabsf(v[i]), fabsf(v[i + 1]));
-  const uint32_t mb = __float_as_uint(m) & 0x7FFFFFFFu;
-  if (mb >= 0x7F800000u) {  // Inf or NaN in the block
-    codes = make_uint4(0u, 0u, 0u, 0u);
-    return 0xFFu;
-  }
-  // e = max(floor(log2 amax) - 2, -127); byte = e + 127 = max(biased_exp, 2) - 2.
-  const uint32_t be = mb >> 23;
-  const uint32_t byte = (be > 2u ? be : 2u) - 2u;
-  const float inv = __uint_as_float((254u - byte) << 23);  // 2^-e, always a normal number
-  const float2 sc = make_float2(inv, inv);
-  float s[32];
-#pragma unroll
-  for (int i = 0; i < 32; i += 2) {
-    const float2 t = __fmul2_rn(make_float2(v[i], v[i + 1]), sc);  // exact: power-of-two scale
-    s[i] = t.x;
-    s[i + 1] = t.y;
-  }
-  uint32_t w[4];
-#pragma unroll
-  for (int q = 0; q < 4; ++q)
-    w[q] = e2m1x8(s[8 * q], s[8 * q + 1], s[8 * q + 2], s[8 * q + 3], s[8 * q + 4], s[8 * q + 5],
-                  s[8 * q + 6], s[8 * q + 7]);
-  codes = make_uint4(w[0], w[1], w[2], w[3]);
-  return byte;
-}
-
 constexpr uint32_t kStages = 4;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 constexpr int kTimeoutCode = 7;                  // MXFP4_ERR_TIMEOUT
@@ -177,14 +51,6 @@ struct TileShape {
   static constexpr uint32_t STAGE = ROWS * 128;         // bytes per stage (128 bytes per row)
   static constexpr uint32_t SMEM = kStages * STAGE + 64 + 1024;
 };
-
-__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
-  uint4 v;
-  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "r"(addr));
-  return v;
-}
 
 template <int MODE, bool F32_IN>
 __global__ void __launch_bounds__(kThreads) rotate_quantize_kernel(
@@ -231,6 +97,9 @@ __global__ void __launch_bounds__(kThreads) rotate_quantize_kernel(
       }
     }
 
+  // tile -> (row tile, k box), advanced incrementally by the grid stride
+  const uint32_t step_rt = gridDim.x / k_boxes, step_kx = gridDim.x - step_rt * k_boxes;
+  uint32_t rt = blockIdx.x / k_boxes, kx = blockIdx.x - rt * k_boxes;
   uint32_t i = 0;
   for (uint32_t tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++i) {
     const uint32_t s = i % kStages;
@@ -239,30 +108,23 @@ __global__ void __launch_bounds__(kThreads) rotate_quantize_kernel(
       if (threadIdx.x == 0 && status) atomicExch(status, kTimeoutCode);
       break;
     }
-    const uint32_t rt = tile / k_boxes, kx = tile - rt * k_boxes;
     const uint32_t row = rt * T::ROWS + r_loc;
     const uint32_t kb = kx * T::BPR + b_loc;
 
-    float v[32];
+    float2 P[16];
     const uint32_t rbase = sbase + s * T::STAGE + r_loc * 128u;
 #pragma unroll
     for (int c = 0; c < CH; ++c) {
       const uint32_t chunk = ((b_loc * CH + (uint32_t)c) ^ (r_loc & 7u)) << 4;
       const uint4 w = ld_shared_v4(rbase + chunk);
       if constexpr (F32_IN) {
-        v[4 * c + 0] = __uint_as_float(w.x);
-        v[4 * c + 1] = __uint_as_float(w.y);
-        v[4 * c + 2] = __uint_as_float(w.z);
-        v[4 * c + 3] = __uint_as_float(w.w);
+        P[2 * c + 0] = make_float2(__uint_as_float(w.x), __uint_as_float(w.y));
+        P[2 * c + 1] = make_float2(__uint_as_float(w.z), __uint_as_float(w.w));
       } else {
-        v[8 * c + 0] = bf16_lo(w.x);
-        v[8 * c + 1] = bf16_hi(w.x);
-        v[8 * c + 2] = bf16_lo(w.y);
-        v[8 * c + 3] = bf16_hi(w.y);
-        v[8 * c + 4] = bf16_lo(w.z);
-        v[8 * c + 5] = bf16_hi(w.z);
-        v[8 * c + 6] = bf16_lo(w.w);
-        v[8 * c + 7] = bf16_hi(w.w);
+        P[4 * c + 0] = make_float2(bf16_lo(w.x), bf16_hi(w.x));
+        P[4 * c + 1] = make_float2(bf16_lo(w.y), bf16_hi(w.y));
+        P[4 * c + 2] = make_float2(bf16_lo(w.z), bf16_hi(w.z));
+        P[4 * c + 3] = make_float2(bf16_lo(w.w), bf16_hi(w.w));
       }
     }
     __syncthreads();  // every thread has its block in registers: the stage may be refilled
@@ -277,15 +139,19 @@ __global__ void __launch_bounds__(kThreads) rotate_quantize_kernel(
     if (row < rows_pad) {
       uint32_t byte = 0;
       if (row < rows && kb < kb_real) {
-        if constexpr (MODE == 1) hadamard32(v);
-        if constexpr (MODE == 2) kron32(v, kc);
+        if constexpr (MODE == 1) hadamard32(P);
+        if constexpr (MODE == 2) kron32(P, kc);
         uint4 codes;
-        byte = quantize_block(v, codes);
+        byte = quantize_block(P, codes);
         st_v4(q + (uint64_t)row * q_row_bytes + (uint64_t)kb * 16u, codes);
       }
-      const uint64_t off = ((uint64_t)(row >> 7) * n_katoms + (kb >> 2)) * 512u +
-                           (row & 31u) * 16u + ((row >> 5) & 3u) * 4u + (kb & 3u);
-      sf[off] = static_cast<uint8_t>(byte);
+      sf[sf_offset(row, kb, n_katoms)] = static_cast<uint8_t>(byte);
+    }
+    kx += step_kx;
+    rt += step_rt;
+    if (kx >= k_boxes) {
+      kx -= k_boxes;
+      ++rt;
     }
   }
   // After an early stop, loads already issued still land in this CTA's shared memory.
