@@ -8,18 +8,21 @@
 // section; "Bridging the Gap Between Promise and Performance for Microscaling
 // FP4 Quantization", "GPU Kernel Ondersteuning (QuTLASS)").
 //
-// Structure (one persistent CTA per SM, 320 threads):
-//   warp 0      TMA producer: A/B tiles (128-byte swizzled, 2-D tensor maps)
-//               and the matching scale atoms (1-D bulk copies) into a ring of
-//               shared-memory stages;
-//   warp 1      allocates tensor memory; one lane copies each stage's scales
-//               into tensor memory (tcgen05.cp) and issues the
-//               tcgen05.mma kind::mxf4 block_scale instructions;
-//   warps 2..9  epilogue: tensor memory -> registers -> bf16/fp32 -> global.
-// Tile: 128 rows of A x BN rows of B, 256 K-elements (128 bytes) per stage,
-// four MMAs of K = 64 per stage. Every barrier wait is bounded in time; on
-// expiry the CTA records MXFP4_ERR_TIMEOUT in the status word, drains its own
-// copies, releases tensor memory and returns.
+// Structure: persistent clusters of two CTAs (one CTA per SM, 320 threads each)
+// share 256 x 256 output tiles through tcgen05.mma.cta_group::2:
+//   warp 0      TMA producer: this CTA's 128 rows of A and 128 rows of B per
+//               stage (128-byte swizzled tiles) and the scale atoms, into a
+//               ring of shared-memory stages;
+//   warp 1      allocates tensor memory; in the leader CTA one lane copies each
+//               stage's scales into tensor memory (tcgen05.cp) and issues the
+//               tcgen05.mma kind::mxf4 block_scale instructions for the pair;
+//   warps 2..9  epilogue: tensor memory -> registers -> bf16/fp32 -> swizzled
+//               shared memory -> TMA store.
+// 256 K-elements (128 bytes) per stage, four MMAs of K = 64 per stage. Every
+// barrier wait is bounded in time; on expiry the CTA records MXFP4_ERR_TIMEOUT
+// in the status word, drains its own copies, releases tensor memory and
+// returns. Problems of at most 128 activation rows go to the weight-streaming
+// kernel in gemm_smallm.cu instead.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
@@ -35,7 +38,6 @@ namespace {
 
 using namespace sm100;
 
-constexpr uint32_t BM = 128;             // rows of A per tile (MMA M)
 constexpr uint32_t BK_BYTES = 128;       // packed bytes of K per stage (256 elements)
 constexpr uint32_t MMA_K_BYTES = 32;     // 64 elements per MMA
 constexpr uint32_t kProducerWarp = 0;
@@ -45,36 +47,6 @@ constexpr uint32_t kEpiWarps = 8;
 constexpr uint32_t kThreads = (kFirstEpiWarp + kEpiWarps) * 32;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 constexpr int kTimeoutCode = 7;                  // MXFP4_ERR_TIMEOUT
-
-template <uint32_t BN, uint32_t STAGES>
-struct Config {
-  static constexpr uint32_t NG = (BN + 127) / 128;  // 128-row scale groups of B per tile
-  static constexpr uint32_t A_STAGE = BM * BK_BYTES;
-  static constexpr uint32_t B_STAGE = BN * BK_BYTES;
-  static constexpr uint32_t SFA_STAGE = 1024;        // 2 atoms x 512 B
-  static constexpr uint32_t SFB_STAGE = NG * 1024;
-  static constexpr uint32_t OFF_A = 0;
-  static constexpr uint32_t OFF_B = OFF_A + STAGES * A_STAGE;
-  static constexpr uint32_t OFF_SFA = OFF_B + STAGES * B_STAGE;
-  static constexpr uint32_t OFF_SFB = OFF_SFA + STAGES * SFA_STAGE;
-  static constexpr uint32_t OFF_BAR = OFF_SFB + STAGES * SFB_STAGE;
-  static constexpr uint32_t ACC = (2 * BN + 8 + 8 * NG <= 512) ? 2 : 1;  // accumulator buffers
-  static constexpr uint32_t NUM_BARS = 2 * STAGES + 2 * ACC + 1;
-  static constexpr uint32_t OFF_MISC = OFF_BAR + NUM_BARS * 8;
-  static constexpr uint32_t SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
-  // tensor memory columns
-  static constexpr uint32_t SFA_COL = ACC * BN;
-  static constexpr uint32_t SFB_COL = SFA_COL + 8;
-  static constexpr uint32_t TMEM_COLS_USED = SFB_COL + 8 * NG;
-  static constexpr uint32_t TMEM_COLS = TMEM_COLS_USED <= 32    ? 32
-                                        : TMEM_COLS_USED <= 64  ? 64
-                                        : TMEM_COLS_USED <= 128 ? 128
-                                        : TMEM_COLS_USED <= 256 ? 256
-                                                                : 512;
-  static_assert(TMEM_COLS_USED <= 512, "tensor memory budget");
-  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-  static_assert(BN % 128 == 0 && BN <= 256, "B tiles cover whole 128-row scale groups");
-};
 
 struct Params {
   const uint8_t* asf;
@@ -99,247 +71,6 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
-}
-
-__device__ __forceinline__ void st_global_v4(void* p, uint32_t a, uint32_t b, uint32_t c,
-                                             uint32_t d) {
-  asm volatile("st.global.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(a), "r"(b), "r"(c), "r"(d)
-               : "memory");
-}
-
-template <uint32_t BN, uint32_t STAGES, bool Y_F32>
-__global__ void __launch_bounds__(kThreads, 1)
-    mxf4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
-                     const __grid_constant__ CUtensorMap tmap_b, const Params p) {
-  using C = Config<BN, STAGES>;
-  extern __shared__ uint8_t smem_raw[];
-  // 1024-byte alignment for the 128-byte swizzle pattern
-  const uint32_t raw_addr = smem_addr(smem_raw);
-  const uint32_t pad = ((raw_addr + 1023u) & ~1023u) - raw_addr;
-  uint8_t* smem = smem_raw + pad;
-  const uint32_t sbase = raw_addr + pad;
-
-  const uint32_t warp = threadIdx.x >> 5;
-  const uint32_t lane = threadIdx.x & 31u;
-
-  const uint32_t bar_full = sbase + C::OFF_BAR;                 // [STAGES]
-  const uint32_t bar_empty = bar_full + 8 * STAGES;             // [STAGES]
-  const uint32_t bar_tfull = bar_empty + 8 * STAGES;            // [ACC]
-  const uint32_t bar_tempty = bar_tfull + 8 * C::ACC;           // [ACC]
-  const uint32_t bar_mma_done = bar_tempty + 8 * C::ACC;        // [1]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
-
-  if (threadIdx.x == 0) {
-    for (uint32_t s = 0; s < STAGES; ++s) {
-      mbar_init(bar_full + 8 * s, 1);
-      mbar_init(bar_empty + 8 * s, 1);
-    }
-    for (uint32_t a = 0; a < C::ACC; ++a) {
-      mbar_init(bar_tfull + 8 * a, 1);
-      mbar_init(bar_tempty + 8 * a, kEpiWarps);
-    }
-    mbar_init(bar_mma_done, 1);
-    *abort_flag = 0;
-    fence_mbar_init();
-    prefetch_tmap(&tmap_a);
-    prefetch_tmap(&tmap_b);
-  }
-  if (warp == kMmaWarp) {
-    tmem_alloc(smem_addr(tmem_slot), C::TMEM_COLS);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem_base = *tmem_slot;
-
-  // Operands may be produced by the kernel launched just before this one.
-  griddep_wait();
-
-  const uint32_t n_tiles_total = p.m_tiles * p.n_tiles;
-
-  if (warp == kProducerWarp) {
-    if (elect_one()) {
-      uint32_t stage = 0, phase = 0, issued = 0;
-      bool ok = true;
-      for (uint32_t tile = blockIdx.x; tile < n_tiles_total && ok; tile += gridDim.x) {
-        const uint32_t mt = tile / p.n_tiles, nt = tile % p.n_tiles;
-        const int32_t m0 = (int32_t)(mt * BM), n0 = (int32_t)(nt * BN);
-        for (uint32_t kt = 0; kt < p.k_tiles; ++kt) {
-          if (!mbar_wait_bounded(bar_empty + 8 * stage, phase ^ 1u, abort_flag, kWaitLimitNs)) {
-            ok = false;
-            break;
-          }
-          const uint32_t atoms = (p.k_atoms - 2 * kt) >= 2 ? 2u : 1u;
-          uint32_t groups = 0;
-          for (uint32_t g = 0; g < C::NG; ++g)
-            if (nt * C::NG + g < p.b_row_tiles) ++groups;
-          // 128-row tiles of B only start on multiples of 128 when BN is, so
-          // scale groups are addressed by absolute 128-row index.
-          const uint32_t tx = C::A_STAGE + C::B_STAGE + atoms * 512u + groups * atoms * 512u;
-          const uint32_t fb = bar_full + 8 * stage;
-          mbar_arrive_expect_tx(fb, tx);
-          tma_load_2d(sbase + C::OFF_A + stage * C::A_STAGE, &tmap_a, fb, (int32_t)(kt * BK_BYTES),
-                      m0);
-          tma_load_2d(sbase + C::OFF_B + stage * C::B_STAGE, &tmap_b, fb, (int32_t)(kt * BK_BYTES),
-                      n0);
-          bulk_load(sbase + C::OFF_SFA + stage * C::SFA_STAGE,
-                    p.asf + ((uint64_t)mt * p.k_atoms + 2 * kt) * 512u, atoms * 512u, fb);
-          for (uint32_t g = 0; g < C::NG; ++g) {
-            const uint32_t rt = (uint32_t)(n0 / 128) + g;
-            if (rt < p.b_row_tiles)
-              bulk_load(sbase + C::OFF_SFB + stage * C::SFB_STAGE + g * 1024u,
-                        p.bsf + ((uint64_t)rt * p.k_atoms + 2 * kt) * 512u, atoms * 512u, fb);
-          }
-          ++issued;
-          if (++stage == STAGES) {
-            stage = 0;
-            phase ^= 1u;
-          }
-        }
-      }
-      if (!ok) record_timeout(p.status);
-      // Drain: the last load into each stage has landed before the CTA may exit.
-      uint32_t s = stage, ph = phase;
-      for (uint32_t i = 0; i < STAGES && i < issued; ++i) {
-        if (s == 0) {
-          s = STAGES - 1;
-          ph ^= 1u;
-        } else {
-          --s;
-        }
-        volatile int never = 0;
-        mbar_wait_bounded(bar_full + 8 * s, ph, &never, kWaitLimitNs);
-      }
-    }
-  } else if (warp == kMmaWarp) {
-    if (elect_one()) {
-      uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
-      bool ok = true;
-      for (uint32_t tile = blockIdx.x; tile < n_tiles_total && ok; tile += gridDim.x) {
-        const uint32_t nt = tile % p.n_tiles;
-        if (!mbar_wait_bounded(bar_tempty + 8 * acc, acc_phase ^ 1u, abort_flag, kWaitLimitNs)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t d_tmem = tmem_base + acc * BN;
-        for (uint32_t kt = 0; kt < p.k_tiles; ++kt) {
-          if (!mbar_wait_bounded(bar_full + 8 * stage, phase, abort_flag, kWaitLimitNs)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t atoms = (p.k_atoms - 2 * kt) >= 2 ? 2u : 1u;
-          // scales -> tensor memory: atom a of A at SFA_COL + 4a; atom a of B's
-          // 128-row group g at SFB_COL + 4 * (NG * a + g)
-          for (uint32_t a = 0; a < atoms; ++a) {
-            tmem_cp_32x128b_warpx4(tmem_base + C::SFA_COL + 4 * a,
-                                   smem_desc_sf(sbase + C::OFF_SFA + stage * C::SFA_STAGE + a * 512));
-            for (uint32_t g = 0; g < C::NG; ++g)
-              if (nt * C::NG + g < p.b_row_tiles)
-                tmem_cp_32x128b_warpx4(
-                    tmem_base + C::SFB_COL + 4 * (C::NG * a + g),
-                    smem_desc_sf(sbase + C::OFF_SFB + stage * C::SFB_STAGE + g * 1024 + a * 512));
-          }
-          // K = 64 per MMA; skip steps that lie wholly beyond K.
-          const uint32_t k_left = p.K - kt * 256u;
-          const uint32_t steps = k_left >= 256u ? 4u : (k_left + 63u) / 64u;
-          const uint32_t a_tile = sbase + C::OFF_A + stage * C::A_STAGE;
-          const uint32_t b_tile = sbase + C::OFF_B + stage * C::B_STAGE;
-          for (uint32_t k = 0; k < steps; ++k) {
-            const uint32_t sf_id = (k & 1u) * 2u;
-            const uint32_t idesc = idesc_mxf4(BM, BN, sf_id, sf_id);
-            mma_mxf4(d_tmem, smem_desc_sw128(a_tile + k * MMA_K_BYTES),
-                     smem_desc_sw128(b_tile + k * MMA_K_BYTES), idesc,
-                     tmem_base + C::SFA_COL + 4 * (k >> 1),
-                     tmem_base + C::SFB_COL + 4 * C::NG * (k >> 1), (kt | k) != 0u);
-          }
-          mma_commit(bar_empty + 8 * stage);  // frees the stage once these MMAs are done
-          if (++stage == STAGES) {
-            stage = 0;
-            phase ^= 1u;
-          }
-        }
-        if (!ok) break;
-        mma_commit(bar_tfull + 8 * acc);  // accumulator ready for the epilogue
-        if (++acc == C::ACC) {
-          acc = 0;
-          acc_phase ^= 1u;
-        }
-      }
-      if (!ok) record_timeout(p.status);
-      // All MMAs issued by this thread are complete before tensor memory is released.
-      mma_commit(bar_mma_done);
-      volatile int never = 0;
-      mbar_wait_bounded(bar_mma_done, 0, &never, kWaitLimitNs);
-    }
-  } else {
-    // Epilogue: warp w reads TMEM lanes 32 * (w % 4) .. +31 (its sub-partition),
-    // columns [half * BN/2, (half + 1) * BN/2): the whole slice goes to registers
-    // first so the accumulator is handed back to the MMA warp as early as possible.
-    const uint32_t quad = warp & 3u;
-    const uint32_t half = (warp - kFirstEpiWarp) / 4u;
-    constexpr uint32_t COLS = BN / 2;
-    constexpr uint32_t CHUNKS = COLS / 32;
-    uint32_t acc = 0, acc_phase = 0;
-    for (uint32_t tile = blockIdx.x; tile < n_tiles_total; tile += gridDim.x) {
-      const uint32_t mt = tile / p.n_tiles, nt = tile % p.n_tiles;
-      const bool ok = mbar_wait_bounded(bar_tfull + 8 * acc, acc_phase, abort_flag, kWaitLimitNs);
-      if (!__all_sync(0xffffffffu, ok)) {  // leave together so .aligned ops stay convergent
-        if (lane == 0) record_timeout(p.status);
-        break;
-      }
-      tc_fence_after();
-      uint32_t v[CHUNKS][32];
-      const uint32_t taddr = tmem_base + ((quad * 32u) << 16) + acc * BN + half * COLS;
-#pragma unroll
-      for (uint32_t c = 0; c < CHUNKS; ++c) tmem_ld_32x32b_x32(taddr + 32 * c, v[c]);
-      tmem_ld_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar_tempty + 8 * acc);  // accumulator may be overwritten now
-
-      const uint32_t row = mt * BM + quad * 32u + lane;
-      const uint32_t col0 = nt * BN + half * COLS;
-      if (row < p.M) {
-        if constexpr (Y_F32) {
-          float* yrow = static_cast<float*>(p.y) + (uint64_t)row * p.ldy + col0;
-#pragma unroll
-          for (uint32_t c = 0; c < CHUNKS; ++c)
-#pragma unroll
-            for (uint32_t j = 0; j < 32; j += 4)
-              if (col0 + 32 * c + j < p.N)
-                st_global_v4(yrow + 32 * c + j, v[c][j], v[c][j + 1], v[c][j + 2], v[c][j + 3]);
-        } else {
-          uint16_t* yrow = static_cast<uint16_t*>(p.y) + (uint64_t)row * p.ldy + col0;
-#pragma unroll
-          for (uint32_t c = 0; c < CHUNKS; ++c)
-#pragma unroll
-            for (uint32_t j = 0; j < 32; j += 8)
-              if (col0 + 32 * c + j < p.N)
-                st_global_v4(yrow + 32 * c + j,
-                             pack_bf16x2(__uint_as_float(v[c][j]), __uint_as_float(v[c][j + 1])),
-                             pack_bf16x2(__uint_as_float(v[c][j + 2]), __uint_as_float(v[c][j + 3])),
-                             pack_bf16x2(__uint_as_float(v[c][j + 4]), __uint_as_float(v[c][j + 5])),
-                             pack_bf16x2(__uint_as_float(v[c][j + 6]), __uint_as_float(v[c][j + 7])));
-        }
-      }
-      if (++acc == C::ACC) {
-        acc = 0;
-        acc_phase ^= 1u;
-      }
-    }
-  }
-
-  tc_fence_before();
-  __syncthreads();
-  if (warp == kMmaWarp) {
-    __syncwarp();
-    tc_fence_after();
-    tmem_dealloc(tmem_base, C::TMEM_COLS);
-  }
 }
 
 // ---------------------------------------------------------------- CTA-pair kernel
@@ -768,71 +499,18 @@ cudaError_t launch_pair(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq
   return cudaLaunchKernelEx(&cfg, kern, ta, tb, tsa, tsb, ty, p);
 }
 
-template <uint32_t BN, uint32_t STAGES, bool Y_F32>
-cudaError_t launch_cfg(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq, const uint8_t* bsf,
-                       int64_t M, int64_t N, int64_t K, void* y, int64_t ldy, int* status, bool pdl,
-                       cudaStream_t stream) {
-  using C = Config<BN, STAGES>;
-  CUtensorMap ta, tb;
-  if (!make_operand_map(&ta, aq, (uint64_t)M, (uint64_t)(K / 2), BM) ||
-      !make_operand_map(&tb, bq, (uint64_t)N, (uint64_t)(K / 2), BN))
-    return cudaErrorInvalidValue;
-  auto kern = mxf4_gemm_kernel<BN, STAGES, Y_F32>;
-  int dev = 0;
-  cudaGetDevice(&dev);
-  static bool attr_done[64] = {};
-  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (!attr_done[dev]) {
-    cudaError_t e =
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    attr_done[dev] = true;
-  }
-  Params p{};
-  p.asf = asf;
-  p.bsf = bsf;
-  p.y = y;
-  p.status = status;
-  p.M = (uint32_t)M;
-  p.N = (uint32_t)N;
-  p.K = (uint32_t)K;
-  p.m_tiles = (uint32_t)((M + BM - 1) / BM);
-  p.n_tiles = (uint32_t)((N + BN - 1) / BN);
-  p.k_tiles = (uint32_t)((K + 255) / 256);
-  p.k_atoms = (uint32_t)sf_katoms(K);
-  p.b_row_tiles = (uint32_t)sf_row_tiles(N);
-  p.ldy = (uint64_t)ldy;
-  int sms = 148;
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const uint32_t tiles = p.m_tiles * p.n_tiles;
-  const uint32_t grid = tiles < (uint32_t)sms ? tiles : (uint32_t)sms;
-
-  cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = C::SMEM_BYTES;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, kern, ta, tb, p);
-}
-
 }  // namespace
 
 cudaError_t launch_gemm(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq,
                         const uint8_t* bsf, int64_t M, int64_t N, int64_t K, void* y,
                         bool y_is_f32, int64_t ldy, int* status, bool pdl, cudaStream_t stream) {
-  // More than one 128-row tile of A: CTA pairs with 256 x 256 tiles.
-  if (M > 128) {
-    if (y_is_f32)
-      return launch_pair<5, true>(aq, asf, bq, bsf, M, N, K, y, ldy, status, pdl, stream);
-    return launch_pair<5, false>(aq, asf, bq, bsf, M, N, K, y, ldy, status, pdl, stream);
-  }
-  if (y_is_f32) return launch_cfg<256, 4, true>(aq, asf, bq, bsf, M, N, K, y, ldy, status, pdl, stream);
-  return launch_cfg<256, 4, false>(aq, asf, bq, bsf, M, N, K, y, ldy, status, pdl, stream);
+  // Few activation rows: stream the weights with the swap-AB split-K kernel.
+  if (M <= 128)
+    return launch_gemm_smallm(aq, asf, bq, bsf, M, N, K, y, y_is_f32, ldy, status, pdl, stream);
+  // Otherwise CTA pairs with 256 x 256 tiles.
+  if (y_is_f32)
+    return launch_pair<5, true>(aq, asf, bq, bsf, M, N, K, y, ldy, status, pdl, stream);
+  return launch_pair<5, false>(aq, asf, bq, bsf, M, N, K, y, ldy, status, pdl, stream);
 }
 
 }  // namespace mxfp4

@@ -27,6 +27,12 @@ cudaError_t launch_gemm(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq
                         const uint8_t* bsf, int64_t M, int64_t N, int64_t K, void* y,
                         bool y_is_f32, int64_t ldy, int* status, bool pdl, cudaStream_t stream);
 
+// Few-row path (M <= 128): swap-AB, K split across the CTAs of a cluster (gemm_smallm.cu).
+cudaError_t launch_gemm_smallm(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq,
+                               const uint8_t* bsf, int64_t M, int64_t N, int64_t K, void* y,
+                               bool y_is_f32, int64_t ldy, int* status, bool pdl,
+                               cudaStream_t stream);
+
 // Scale-factor layout helpers (host side).
 inline int64_t sf_katoms(int64_t K) { return (K / 32 + 3) / 4; }
 inline int64_t sf_row_tiles(int64_t rows) { return (rows + 127) / 128; }

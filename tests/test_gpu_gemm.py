@@ -60,6 +60,45 @@ def test_gemm_zero_and_single_pair():
     assert not y.any()
 
 
+# Few activation rows (M <= 128): the weight-streaming kernel splits K over the
+# CTAs of a thread-block cluster and adds the partials through distributed shared
+# memory. (M, N, K) -> W tiles x K splits: (1,16,4096) 1x8; (5,400,2080) 4x5 with a
+# 32-element K tail; (16,256,8192) 2x8; (17,12288,1024) 96x2; (33,9216,1536) 72x3;
+# (64,2048,3104) 16x7 with a K tail; (100,1024,7168) 8x7; (65,14336,4096) 112x2;
+# (128,4096,14336) 32x8.
+SMALLM_SHAPES = [
+    (1, 16, 4096), (5, 400, 2080), (16, 256, 8192), (17, 12288, 1024), (33, 9216, 1536),
+    (64, 2048, 3104), (100, 1024, 7168), (65, 14336, 4096), (128, 4096, 14336),
+]
+
+
+@pytest.mark.parametrize("M,N,K", SMALLM_SHAPES)
+@pytest.mark.parametrize("out", ["bf16", "f32"])
+def test_gemm_few_rows_split_k(M, N, K, out):
+    aq, as_ = _operand(M * 17 + N + K, M, K, 6)
+    bq, bs = _operand(M * 17 + N + K, N, K, 7)
+    y = _run(aq, as_, bq, bs, out)
+    ref, S = oracle.gemm(aq, as_, bq, bs)
+    check_gemm_values(y, ref, S, out, f"few-row gemm {M}x{N}x{K} {out}")
+
+
+def test_gemm_few_rows_single_pair_in_last_split():
+    """One nonzero product in the K tail, which only the last split of the cluster
+    holds: the cross-CTA sum must carry it to exactly one output, unchanged."""
+    M, N, K = 3, 400, 2080
+    aq = np.zeros((M, K // 2), np.uint8)
+    bq = np.zeros((N, K // 2), np.uint8)
+    as_ = synth.uniform_u8(2, 92, (M, K // 32), 100, 150)
+    bs = synth.uniform_u8(2, 93, (N, K // 32), 100, 150)
+    aq[2, K // 2 - 1] = 7 << 4    # element K-1 = 6
+    bq[399, K // 2 - 1] = 12 << 4  # element K-1 = -2
+    y = _run(aq, as_, bq, bs, "f32")
+    expect = 6 * -2 * 2.0 ** (int(as_[2, K // 32 - 1]) + int(bs[399, K // 32 - 1]) - 254)
+    assert y[2, 399] == expect
+    y[2, 399] = 0
+    assert not y.any()
+
+
 def test_gemm_wide_scale_range_fp32():
     """Scales spread over most of the E8M0 range in fp32 output."""
     M, N, K = 256, 256, 1024
