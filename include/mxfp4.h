@@ -25,7 +25,11 @@
  *    call returns and allocates no device memory. kron_a / kron_b are HOST
  *    pointers (the transform is passed by value to the kernel).
  *  - Every launch is asynchronous and ordered on `stream` (a cudaStream_t;
- *    NULL = the legacy default stream).
+ *    NULL = the legacy default stream). Kernels are launched with programmatic
+ *    dependent launch: one may be scheduled while the kernel before it on the
+ *    stream finishes, and waits for that kernel to complete before it touches
+ *    any memory the two could share. The results are those of plain stream
+ *    order.
  *  - Argument errors are detected on the host before any launch and launch
  *    nothing: NULL pointer -> MXFP4_ERR_INVALID_ARG; bad sizes ->
  *    MXFP4_ERR_SHAPE; misaligned pointer or row stride -> MXFP4_ERR_ALIGN;
@@ -155,8 +159,8 @@ mxfp4_status mxfp4_gemm(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq
  * (wq/wsf: [N, K] operand prepared offline with the matching rotation), bf16
  * output y[M, N] (row stride N). ws must hold
  * mxfp4_workspace_bytes(MXFP4_OP_LINEAR, M, N, K) bytes. The two kernels run
- * back to back on `stream`, the second with programmatic dependent launch so
- * its set-up overlaps the first one's tail.
+ * back to back on `stream`; the GEMM may start loading wq / wsf while the
+ * quantiser is still running, so wq / wsf must not overlap the workspace.
  */
 mxfp4_status mxfp4_linear(const void* x, int64_t M, int64_t K, mxfp4_rotation mode,
                           const float* kron_a, const float* kron_b, const uint8_t* wq,

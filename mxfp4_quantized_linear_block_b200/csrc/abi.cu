@@ -152,6 +152,7 @@ mxfp4_status mxfp4_gemm(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq
   if (!aligned16(ws)) return MXFP4_ERR_ALIGN;
   if (ws_bytes < mxfp4_workspace_bytes(MXFP4_OP_GEMM, M, N, K)) return MXFP4_ERR_WORKSPACE;
   if (M == 0) return MXFP4_OK;
+  // The caller's previous kernel may have written bq / bsf: no early weight loads.
   return from_cuda(launch_gemm(aq, asf, bq, bsf, M, N, K, y, ydt == MXFP4_DT_F32, ldy,
                                static_cast<int*>(ws), false, static_cast<cudaStream_t>(stream)));
 }
@@ -181,6 +182,7 @@ mxfp4_status mxfp4_linear(const void* x, int64_t M, int64_t K, mxfp4_rotation mo
   cudaError_t e =
       launch_rotate_quantize(x, false, M, K, K, (int)mode, &kc, xq, xsf, static_cast<int*>(ws), s);
   if (e != cudaSuccess) return MXFP4_ERR_CUDA;
+  // The kernel just before the GEMM is the quantiser above, which does not write W.
   return from_cuda(
       launch_gemm(xq, xsf, wq, wsf, M, N, K, y, false, N, static_cast<int*>(ws), true, s));
 }

@@ -169,8 +169,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  // Operands may be produced by the kernel launched just before this one.
+  // Operands may be produced by the kernel launched just before this one (programmatic
+  // dependent launch): wait for it, then let the next kernel start its set-up.
   griddep_wait();
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   const uint32_t n_tiles_total = p.m_tiles * p.n_tiles;  // m_tiles counts 256-row pair tiles
 
@@ -435,7 +437,7 @@ bool make_output_map(CUtensorMap* map, void* y, uint64_t M, uint64_t N, uint64_t
 template <uint32_t STAGES, bool Y_F32>
 cudaError_t launch_pair(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq,
                         const uint8_t* bsf, int64_t M, int64_t N, int64_t K, void* y, int64_t ldy,
-                        int* status, bool pdl, cudaStream_t stream) {
+                        int* status, cudaStream_t stream) {
   using C = PairConfig<STAGES>;
   const uint64_t k_atoms = (uint64_t)sf_katoms(K);
   CUtensorMap ta, tb, tsa, tsb, ty;
@@ -495,7 +497,7 @@ cudaError_t launch_pair(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = pdl ? 1 : 0;
+  cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kern, ta, tb, tsa, tsb, ty, p);
 }
 
@@ -503,14 +505,15 @@ cudaError_t launch_pair(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq
 
 cudaError_t launch_gemm(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq,
                         const uint8_t* bsf, int64_t M, int64_t N, int64_t K, void* y,
-                        bool y_is_f32, int64_t ldy, int* status, bool pdl, cudaStream_t stream) {
+                        bool y_is_f32, int64_t ldy, int* status, bool b_early,
+                        cudaStream_t stream) {
   // Few activation rows: stream the weights with the swap-AB split-K kernel.
   if (M <= 128)
-    return launch_gemm_smallm(aq, asf, bq, bsf, M, N, K, y, y_is_f32, ldy, status, pdl, stream);
+    return launch_gemm_smallm(aq, asf, bq, bsf, M, N, K, y, y_is_f32, ldy, status, b_early,
+                              stream);
   // Otherwise CTA pairs with 256 x 256 tiles.
-  if (y_is_f32)
-    return launch_pair<5, true>(aq, asf, bq, bsf, M, N, K, y, ldy, status, pdl, stream);
-  return launch_pair<5, false>(aq, asf, bq, bsf, M, N, K, y, ldy, status, pdl, stream);
+  if (y_is_f32) return launch_pair<5, true>(aq, asf, bq, bsf, M, N, K, y, ldy, status, stream);
+  return launch_pair<5, false>(aq, asf, bq, bsf, M, N, K, y, ldy, status, stream);
 }
 
 }  // namespace mxfp4

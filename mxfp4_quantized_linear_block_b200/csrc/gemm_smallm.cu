@@ -73,6 +73,7 @@ struct SmallParams {
   uint32_t M, N, K;
   uint64_t ldy;
   uint32_t k_tiles, k_atoms, splits, kt_per_split;
+  uint32_t w_early;     // W may be loaded before the previous kernel has finished
 };
 
 __device__ __forceinline__ void record_timeout(int* status) {
@@ -126,10 +127,10 @@ __global__ void __launch_bounds__(kThreads, 2) mxf4_gemm_smallm_kernel(
     fence_proxy_async_smem();
     prefetch_tmap(&tmap_w);
     prefetch_tmap(&tmap_x);
-    // W and its scales never come from the kernel just before this one: the first
-    // stages' W loads go out now, ahead of the set-up below and of the wait for
-    // that kernel. Each stage's barrier expects its X bytes too (issued later).
-    for (uint32_t i = 0; i < pre; ++i) {
+    // When the kernel just before this one does not write W (the layer's own
+    // quantiser), the first stages' W loads go out now, ahead of the set-up below
+    // and of the wait for that kernel. Each stage's barrier expects its X bytes too.
+    for (uint32_t i = 0; i < (p.w_early ? pre : 0u); ++i) {
       const uint32_t kt = kt0 + i;
       const uint32_t atoms = (p.k_atoms - 2 * kt) >= 2 ? 2u : 1u;
       const uint32_t fb = bar_full + 8 * i;
@@ -151,11 +152,21 @@ __global__ void __launch_bounds__(kThreads, 2) mxf4_gemm_smallm_kernel(
 
   if (warp == 0) {
     if (elect_one()) {
-      asm volatile("griddepcontrol.wait;" ::: "memory");  // X may come from the previous kernel
+      // X (and W, unless w_early) may come from the previous kernel: wait for it, then
+      // let the next kernel start its set-up.
+      asm volatile("griddepcontrol.wait;" ::: "memory");
+      asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
       for (uint32_t i = 0; i < pre; ++i) {
         const uint32_t kt = kt0 + i;
         const uint32_t atoms = (p.k_atoms - 2 * kt) >= 2 ? 2u : 1u;
         const uint32_t fb = bar_full + 8 * i;
+        if (!p.w_early) {
+          mbar_arrive_expect_tx(fb, C::A_STAGE + C::B_STAGE + 2u * atoms * 512u);
+          tma_load_2d(sbase + C::OFF_A + i * C::A_STAGE, &tmap_w, fb, (int32_t)(kt * 128u),
+                      (int32_t)(wt * 128u));
+          bulk_load(sbase + C::OFF_SFA + i * C::SF_STAGE,
+                    p.wsf + ((uint64_t)wt * p.k_atoms + 2 * kt) * 512u, atoms * 512u, fb);
+        }
         tma_load_2d(sbase + C::OFF_B + i * C::B_STAGE, &tmap_x, fb, (int32_t)(kt * 128u), 0);
         bulk_load(sbase + C::OFF_SFB + i * C::SF_STAGE, p.xsf + (uint64_t)(2 * kt) * 512u,
                   atoms * 512u, fb);
@@ -361,7 +372,7 @@ Plan make_plan(int64_t M, int64_t N, int64_t K) {
 template <uint32_t NT, bool Y_F32>
 cudaError_t launch_nt(const Plan& pl, const uint8_t* aq, const uint8_t* asf, const uint8_t* bq,
                       const uint8_t* bsf, int64_t M, int64_t N, int64_t K, void* y, int64_t ldy,
-                      int* status, bool pdl, cudaStream_t stream) {
+                      int* status, bool w_early, cudaStream_t stream) {
   using C = SmallConfig<NT>;
   CUtensorMap tw, tx;
   if (!operand_map(&tw, bq, (uint64_t)N, (uint64_t)(K / 2), 128) ||
@@ -391,6 +402,7 @@ cudaError_t launch_nt(const Plan& pl, const uint8_t* aq, const uint8_t* asf, con
   p.k_atoms = (uint32_t)sf_katoms(K);
   p.splits = pl.splits;
   p.kt_per_split = pl.kt_per_split;
+  p.w_early = w_early ? 1u : 0u;
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(pl.units);
   cfg.blockDim = dim3(kThreads);
@@ -404,7 +416,7 @@ cudaError_t launch_nt(const Plan& pl, const uint8_t* aq, const uint8_t* asf, con
   attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = pdl ? 2 : 1;
+  cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, kern, tw, tx, p);
 }
 
@@ -412,13 +424,13 @@ cudaError_t launch_nt(const Plan& pl, const uint8_t* aq, const uint8_t* asf, con
 
 cudaError_t launch_gemm_smallm(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq,
                                const uint8_t* bsf, int64_t M, int64_t N, int64_t K, void* y,
-                               bool y_is_f32, int64_t ldy, int* status, bool pdl,
+                               bool y_is_f32, int64_t ldy, int* status, bool b_early,
                                cudaStream_t stream) {
   const Plan pl = make_plan(M, N, K);
 #define MXFP4_SMALLM(NTV)                                                                        \
   return y_is_f32                                                                                \
-             ? launch_nt<NTV, true>(pl, aq, asf, bq, bsf, M, N, K, y, ldy, status, pdl, stream)  \
-             : launch_nt<NTV, false>(pl, aq, asf, bq, bsf, M, N, K, y, ldy, status, pdl, stream);
+             ? launch_nt<NTV, true>(pl, aq, asf, bq, bsf, M, N, K, y, ldy, status, b_early, stream)  \
+             : launch_nt<NTV, false>(pl, aq, asf, bq, bsf, M, N, K, y, ldy, status, b_early, stream);
   switch (pl.nt) {
     case 16: MXFP4_SMALLM(16)
     case 32: MXFP4_SMALLM(32)

@@ -22,15 +22,19 @@ cudaError_t launch_rotate_quantize(const void* x, bool x_is_f32, int64_t rows, i
 
 // Block-scaled GEMM y[M, N] = A[M, K] . B[N, K]^T on tcgen05. Host-validated arguments.
 // status: device word set to the timeout code if a bounded wait gives up.
-// pdl: launch with programmatic stream serialization (overlaps the previous kernel's tail).
+// Every kernel of the library is launched with programmatic dependent launch: it waits
+// for the previous kernel on the stream before touching memory that kernel may share.
+// b_early: the kernel just before this launch on the stream does not write bq / bsf, so
+// the few-row kernel may start streaming them before that kernel has finished.
 cudaError_t launch_gemm(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq,
                         const uint8_t* bsf, int64_t M, int64_t N, int64_t K, void* y,
-                        bool y_is_f32, int64_t ldy, int* status, bool pdl, cudaStream_t stream);
+                        bool y_is_f32, int64_t ldy, int* status, bool b_early,
+                        cudaStream_t stream);
 
 // Few-row path (M <= 128): swap-AB, K split across the CTAs of a cluster (gemm_smallm.cu).
 cudaError_t launch_gemm_smallm(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq,
                                const uint8_t* bsf, int64_t M, int64_t N, int64_t K, void* y,
-                               bool y_is_f32, int64_t ldy, int* status, bool pdl,
+                               bool y_is_f32, int64_t ldy, int* status, bool b_early,
                                cudaStream_t stream);
 
 // Scale-factor layout helpers (host side).

@@ -97,6 +97,7 @@ extern "C" mxfp4_status mxfp4_linear_noalloc(const void* x, int64_t M, int64_t K
   if (launch_rotate_quantize(x, false, M, K, K, (int)mode, &kc, xq, xsf, status_word, s) !=
       cudaSuccess)
     return MXFP4_ERR_CUDA;
+  // The kernel just before the GEMM is the quantiser above, which does not write W.
   if (launch_gemm(xq, xsf, wq, wsf, M, N, K, y, false, N, status_word, true, s) != cudaSuccess)
     return MXFP4_ERR_CUDA;
   return MXFP4_OK;

@@ -80,6 +80,11 @@ __global__ void __launch_bounds__(kThreads) rotate_quantize_kernel(
     prefetch_tmap(&tmap_x);
   }
   __syncthreads();
+  // Launched with programmatic dependent launch: the kernel before this one may still
+  // be writing x or reading q / sf. Wait for it to finish before the first access,
+  // then let the next kernel start its own set-up.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   auto issue = [&](uint32_t tile, uint32_t s) {
     const uint32_t rt = tile / k_boxes, kx = tile - rt * k_boxes;
@@ -160,9 +165,6 @@ __global__ void __launch_bounds__(kThreads) rotate_quantize_kernel(
     for (uint32_t j = i; j < issued; ++j)
       mbar_wait_bounded(bar_full + 8 * (j % kStages), (j / kStages) & 1u, &never, kWaitLimitNs);
   }
-  // Let a dependent kernel (the GEMM of the fused layer) start its set-up; it
-  // still waits for this grid's completion before reading q / sf.
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -219,11 +221,19 @@ cudaError_t launch_mode(const void* x, int64_t rows, int64_t K, int64_t ldx, con
   const int64_t tiles = row_tiles * k_boxes;
   const int64_t cap = (int64_t)sms[dev] * per_sm[dev];
   const int grid = (int)(tiles < cap ? tiles : cap);
-  kern<<<grid, kThreads, T::SMEM, stream>>>(map, (uint32_t)rows, (uint32_t)rows_pad,
-                                             (uint32_t)kb_real, (uint32_t)k_boxes, (uint32_t)tiles,
-                                             (uint32_t)sf_katoms(K), (uint64_t)(K / 2), kc, q, sf,
-                                             status);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = T::SMEM;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, map, (uint32_t)rows, (uint32_t)rows_pad,
+                            (uint32_t)kb_real, (uint32_t)k_boxes, (uint32_t)tiles,
+                            (uint32_t)sf_katoms(K), (uint64_t)(K / 2), kc, q, sf, status);
 }
 
 }  // namespace
