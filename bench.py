@@ -11,9 +11,11 @@ Prints ONE JSON line (rank 0). ``value`` = TFLOPS of the whole job (2*M*N*K
 summed over linears and ranks / max-over-ranks device time), inputs resident
 in HBM. ``e2e`` = the same metric through the same public call from host
 buffers (pinned H2D of X, D2H of Y inside the timed region). ``roofline`` =
-the GEMM kernel against the FP4 tensor peak, ``quantize_roofline`` = the
-rotate+quantise kernel against HBM bandwidth, both from CUDA events around
-each kernel launch in an attribution pass over the same steps.
+the GEMM kernel (the largest share of every step) against the FP4 tensor peak,
+or against HBM bandwidth when its arithmetic intensity is below the ridge (few
+tokens); ``quantize_roofline`` = the rotate+quantise kernel against HBM
+bandwidth; both from CUDA events around each kernel launch in an attribution
+pass over the same steps.
 
 --impl reference times the CPU oracle (the plain C implementation that
 defines the results) on a bounded row sample of the same workload.
@@ -21,6 +23,7 @@ defines the results) on a bounded row sample of the same workload.
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import os
 import statistics
@@ -40,6 +43,40 @@ import synth  # noqa: E402
 METRIC = "MXFP4 W4A4 linear TFLOPS & % FP4 peak; quantize GB/s & % HBM peak"
 UNIT = "TFLOPS"
 FP4_OVER_BF16 = 4.0  # nominal dense FP4 : BF16 tensor throughput on B200 (9 : 2.25 PFLOP/s)
+PKG = "mxfp4_quantized_linear_block_b200"
+
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the dominant GEMM kernel,
+# one value per linear of the workload in its order, from one ncu capture of this bench
+# (summaries and commands under profiles/). A value is reported only while the kernel's
+# source file still has the SHA-256 it had when the counters were taken.
+# ncu flushes L2 before every pass, so reads are cold; output still dirty in L2 when the
+# kernel ends is written back later and is not counted (hence writes < Y bytes).
+NCU_TRAFFIC = {
+    "dit_b1": {"source": f"{PKG}/csrc/gemm.cu",
+               "sha256": "3375dd2225b170c8bea10ae09bd5825cfe726ef7fc4d86f46d2390450dc9ce4d",
+               "bytes_per_launch": [20924160 + 12758016, 26232064 + 37004032,
+                                    43504896 + 2775552]},
+    "llm_small_m1": {"source": f"{PKG}/csrc/gemm_smallm.cu",
+                     "sha256": "4e2cb66424a7f58bbb686dd0ed5bba39f74382b140c3a691d6a293916c0fb05c",
+                     "bytes_per_launch": [31234304 + 0, 31282944 + 256]},
+}
+NCU_TRAFFIC_QUANTIZE = {
+    "dit_b1": {"source": f"{PKG}/csrc/quantize.cu",
+               "sha256": "daead7a2fa978630267d30cd9dbbba56138ee8ba9de661d3e1cbad8f0f053f49",
+               "bytes_per_launch": [22033920 + 1280, 22033664 + 0, 88095744 + 4947200]},
+}
+
+
+def source_sha256(rel: str) -> str:
+    with open(os.path.join(ROOT, rel), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()
+
+
+def ncu_traffic(workload: str, kernel_src: str, table=None):
+    e = (NCU_TRAFFIC if table is None else table).get(workload)
+    if not e or e["source"] != kernel_src or e["sha256"] != source_sha256(kernel_src):
+        return None
+    return e
 
 
 def parse():
@@ -230,18 +267,24 @@ def run_ours(args, rank, world, local_rank):
         return (sum(t.numel() * t.element_size() for t in xs.values()) +
                 sum(t.numel() * 2 for t in ys) + sum(t.numel() for t in wss))
 
+    # Rotate through input/output sets and, when those are small (few tokens), through
+    # copies of the weights too, so that no step finds its operands in L2.
     w_bytes = sum(wq.numel() + wsf.numel() for wq, wsf in weights)
     sets = [make_set()]
-    while (len(sets) * set_bytes(sets[0]) + w_bytes) < 3 * l2 and len(sets) < 8:
-        sets.append(make_set())
-    footprint = len(sets) * set_bytes(sets[0]) + w_bytes
+    wsets = [weights]
+    while len(sets) * set_bytes(sets[0]) + len(wsets) * w_bytes < 3 * l2:
+        if len(sets) < 8 and set_bytes(sets[0]) >= w_bytes:
+            sets.append(make_set())
+        else:
+            wsets.append([(wq.clone(), wsf.clone()) for wq, wsf in weights])
+    footprint = len(sets) * set_bytes(sets[0]) + len(wsets) * w_bytes
 
     stream = torch.cuda.current_stream(dev)
 
     def step(i):
         xs, ys, wss = sets[i % len(sets)]
         for j, lin in enumerate(wl.linears):
-            wq, wsf = weights[j]
+            wq, wsf = wsets[i % len(wsets)][j]
             mx.linear(xs[lin.x_tensor], wq, wsf, lin.N, wl.rotation, A, B, y=ys[j], ws=wss[j],
                       stream=stream)
 
@@ -305,7 +348,7 @@ def run_ours(args, rank, world, local_rank):
     def step_split(i, rec):
         xs, ys, _ = sets[i % len(sets)]
         for j, lin in enumerate(wl.linears):
-            wq, wsf = weights[j]
+            wq, wsf = wsets[i % len(wsets)][j]
             q, sf = qbufs[j]
             if rec:
                 evs[i][j][0].record(stream)
@@ -338,8 +381,37 @@ def run_ours(args, rank, world, local_rank):
     q_bytes = np.array([2 * l.M * l.K + l.M * l.K // 2 + mx.sf_bytes(l.M, l.K)
                         for l in wl.linears], np.float64)
     fp4_peak = peaks["bf16_tflops_sustained"] * FP4_OVER_BF16
-    g_ach = gemm_flops.sum() / t_g.sum() / 1e12
     q_ach = q_bytes.sum() / t_q.sum() / 1e9
+    # The GEMM dominates every workload's step. It is tensor-bound when its arithmetic
+    # intensity (2MNK over its algorithmic bytes) is above the ridge of the two peaks,
+    # HBM-bound otherwise (few tokens).
+    few_rows = all(l.M <= 128 for l in wl.linears)
+    g_kernel = "mxf4_gemm_smallm_kernel" if few_rows else "mxf4_gemm_pair_kernel"
+    g_src = f"{PKG}/csrc/gemm_smallm.cu" if few_rows else f"{PKG}/csrc/gemm.cu"
+    ridge = fp4_peak * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    intensity = gemm_flops.sum() / gemm_bytes.sum()
+    traffic = ncu_traffic(wl.name, g_src)
+    q_traffic = ncu_traffic(wl.name, f"{PKG}/csrc/quantize.cu", NCU_TRAFFIC_QUANTIZE)
+    if intensity >= ridge:
+        roofline = {"bound": "tensor", "achieved": gemm_flops.sum() / t_g.sum() / 1e12,
+                    "peak": fp4_peak, "unit": "TFLOP/s",
+                    "peak_source": f"4 x {peaks['source']} bf16 sustained "
+                                   f"({peaks['bf16_tflops_sustained']} TFLOP/s)"}
+    else:
+        roofline = {"bound": "hbm", "achieved": gemm_bytes.sum() / t_g.sum() / 1e9,
+                    "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                    "peak_source": f"{peaks['source']} HBM copy bandwidth"}
+    roofline.update({
+        "frac": roofline["achieved"] / roofline["peak"], "kernel": g_kernel,
+        "intensity_flop_per_byte": intensity, "ridge_flop_per_byte": ridge,
+        "per_launch": [{"linear": l.name, "us": t_g[j] * 1e6,
+                        "tflops": gemm_flops[j] / t_g[j] / 1e12,
+                        "gbs": gemm_bytes[j] / t_g[j] / 1e9,
+                        "alg_bytes": int(gemm_bytes[j])} for j, l in enumerate(wl.linears)],
+        "traffic": (float(np.mean(traffic["bytes_per_launch"])) if traffic else None),
+        "traffic_per_launch": (traffic["bytes_per_launch"] if traffic else None),
+        "alg_bytes_per_launch_mean": float(gemm_bytes.mean()),
+    })
 
     # ---- end to end: host (pinned) X in, host Y out, inside the timed region
     e2e = None
@@ -351,23 +423,23 @@ def run_ours(args, rank, world, local_rank):
         h2d = sum(t.numel() * 2 for t in xs_pin.values())
         d2h = sum(t.numel() * 2 for t in ys_pin)
 
-        def e2e_step():
+        def e2e_step(i):
             for k, t in xs_pin.items():
                 xs_d[k].copy_(t, non_blocking=True)
             for j, lin in enumerate(wl.linears):
-                wq, wsf = weights[j]
+                wq, wsf = wsets[i % len(wsets)][j]
                 mx.linear(xs_d[lin.x_tensor], wq, wsf, lin.N, wl.rotation, A, B, y=ys_d[j],
                           ws=wss_d[j], stream=stream)
                 ys_pin[j].copy_(ys_d[j], non_blocking=True)
 
-        e2e_step()
+        e2e_step(0)
         torch.cuda.synchronize()
         barrier()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         torch.cuda._sleep(int(2e7))
         a.record(stream)
-        for _ in range(args.e2e_steps):
-            e2e_step()
+        for i in range(args.e2e_steps):
+            e2e_step(i + 1)
         b.record(stream)
         torch.cuda.synchronize()
         barrier()
@@ -387,24 +459,19 @@ def run_ours(args, rank, world, local_rank):
         "config": {"workload": workload_desc(wl), "tokens_per_gpu": wl.linears[0].M,
                    "gflop_per_step_per_gpu": flops_step / 1e9, "parallelism": f"replicas x{world} "
                    "(token-parallel, no collective)",
-                   "l2": f"{len(sets)} rotating input/output sets, footprint "
-                         f"{footprint / 2**20:.0f} MiB >= 3 x L2 ({l2 / 2**20:.0f} MiB)"},
-        "roofline": {"bound": "tensor", "kernel": "mxf4_gemm_kernel (tcgen05 kind::mxf4)",
-                     "achieved": g_ach, "peak": fp4_peak, "unit": "TFLOP/s",
-                     "frac": g_ach / fp4_peak,
-                     "peak_source": f"4 x {peaks['source']} bf16 sustained "
-                                    f"({peaks['bf16_tflops_sustained']} TFLOP/s)",
-                     "per_launch": [{"linear": l.name, "us": t_g[j] * 1e6,
-                                     "tflops": gemm_flops[j] / t_g[j] / 1e12,
-                                     "alg_bytes": int(gemm_bytes[j])}
-                                    for j, l in enumerate(wl.linears)],
-                     "traffic": None},
+                   "l2": f"{len(sets)} rotating input/output sets and {len(wsets)} weight "
+                         f"copies, footprint {footprint / 2**20:.0f} MiB >= 3 x L2 "
+                         f"({l2 / 2**20:.0f} MiB)"},
+        "roofline": roofline,
         "quantize_roofline": {"bound": "hbm", "kernel": "rotate_quantize_kernel",
                               "achieved": q_ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                               "frac": q_ach / peaks["hbm_gbs"],
                               "per_launch_us": [t * 1e6 for t in t_q],
                               "alg_bytes_per_launch": [int(b) for b in q_bytes],
-                              "traffic": None},
+                              "traffic": (float(np.mean(q_traffic["bytes_per_launch"]))
+                                          if q_traffic else None),
+                              "traffic_per_launch": (q_traffic["bytes_per_launch"]
+                                                     if q_traffic else None)},
         "e2e": e2e,
         "gpu_launches": launches,
         "attribution": {"steps": n_attr, "gpu_launches": 2 * n_lin * n_attr,
