@@ -339,7 +339,8 @@ def run_ours(args, rank, world, local_rank):
     # CUDA events around each kernel (on the launching stream)
     qbufs = [(torch.empty((l.M, l.K // 2), dtype=torch.uint8, device=dev),
               torch.empty(mx.sf_bytes(l.M, l.K), dtype=torch.uint8, device=dev)) for l in wl.linears]
-    gws = mx.new_workspace(mx.workspace_bytes(mx.OP_GEMM, 1, 16, 32), dev)
+    gws = [mx.new_workspace(mx.workspace_bytes(mx.OP_GEMM, l.M, l.N, l.K), dev)
+           for l in wl.linears]
     n_lin = len(wl.linears)
     n_attr = max(1, min(args.steps, args.attr_steps))
     evs = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
@@ -355,7 +356,7 @@ def run_ours(args, rank, world, local_rank):
             mx.rotate_quantize(xs[lin.x_tensor], wl.rotation, A, B, q=q, sf=sf, stream=stream)
             if rec:
                 evs[i][j][1].record(stream)
-            mx.gemm(q, sf, wq, wsf, lin.M, lin.N, lin.K, y=ys[j], ws=gws, stream=stream)
+            mx.gemm(q, sf, wq, wsf, lin.M, lin.N, lin.K, y=ys[j], ws=gws[j], stream=stream)
             if rec:
                 evs[i][j][2].record(stream)
 

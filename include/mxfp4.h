@@ -94,8 +94,11 @@ size_t mxfp4_sf_bytes(int64_t rows, int64_t K);
 /* Byte offset of the scale of (row, 32-element block kblock) in that buffer, or -1 if out of range. */
 int64_t mxfp4_sf_offset(int64_t row, int64_t kblock, int64_t K);
 
-/* Device workspace that `op` needs for this problem (0 if none). For
- * MXFP4_OP_LINEAR it holds the quantised activations and a status word. */
+/* Device workspace that `op` needs for this problem (0 if none). It starts with
+ * a status word; for MXFP4_OP_LINEAR it also holds the quantised activations;
+ * for both GEMM-running ops it ends with the GEMM's scratch (K-split partials
+ * and counters for the last round of output tiles; sized for a 148-SM B200).
+ * Allocate it zeroed: every call that completes leaves the scratch zeroed. */
 size_t mxfp4_workspace_bytes(int op, int64_t M, int64_t N, int64_t K);
 
 /* Static description of a status code. Never NULL. */
@@ -144,7 +147,10 @@ mxfp4_status mxfp4_rotate_quantize(const void* x, mxfp4_dtype xdt, int64_t rows,
  * elements. Requirements: K % 32 == 0, N % 16 == 0, ldy >= N, y 16-byte aligned
  * and ldy * elemsize a multiple of 16; aq, bq, asf, bsf 16-byte aligned.
  * ws must hold mxfp4_workspace_bytes(MXFP4_OP_GEMM, M, N, K) bytes (at least
- * 256); its first 16 bytes are the device status word (see mxfp4_poll_status).
+ * 256), zeroed when allocated; its first 16 bytes are the device status word
+ * (see mxfp4_poll_status). On a GPU whose SM count needs more scratch than
+ * that, the last round of tiles is not split along K (slower; the result
+ * still meets the stated tolerance).
  * ("AMD Quark...", opening section: MXFP4 GEMM with no dequantisation;
  * "Bridging the Gap...", "GPU Kernel Ondersteuning (QuTLASS)".)
  */
@@ -209,8 +215,9 @@ mxfp4_status mxfp4_linear_noalloc(const void* x, int64_t M, int64_t K, mxfp4_rot
  * the device): MXFP4_OK, or MXFP4_ERR_TIMEOUT if a kernel's bounded wait on a
  * pipeline barrier ran out (the kernel then stopped early, released its
  * tensor memory and returned; its output is incomplete). The word is sticky:
- * kernels only ever set it, this call clears it. Zero the first 16 bytes of a
- * workspace once when it is allocated.
+ * kernels only ever set it, this call clears it. Zero the whole workspace once
+ * when it is allocated, and again after a timeout (a kernel that stopped early
+ * can leave GEMM scratch counters set).
  */
 mxfp4_status mxfp4_poll_status(void* ws, mxfp4_status* out);
 

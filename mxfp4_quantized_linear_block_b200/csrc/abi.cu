@@ -63,16 +63,18 @@ bool kron_from_host(const float* a, const float* b, KronCoeffs* out) {
   return true;
 }
 
-// Workspace of mxfp4_linear: [status | Xq (M x K/2) | Xsf], each part 256-byte aligned.
+// Workspace of mxfp4_linear: [status | Xq (M x K/2) | Xsf | GEMM scratch], each part
+// 256-byte aligned.
 struct LinearWorkspace {
-  size_t q_off, sf_off, total;
+  size_t q_off, sf_off, g_off, total;
 };
 
-LinearWorkspace linear_workspace(int64_t M, int64_t K) {
+LinearWorkspace linear_workspace(int64_t M, int64_t N, int64_t K) {
   LinearWorkspace w;
   w.q_off = kStatusBytes;
   w.sf_off = round_up(w.q_off + (size_t)M * (size_t)(K / 2), 256);
-  w.total = round_up(w.sf_off + mxfp4_sf_bytes(M, K), 256);
+  w.g_off = round_up(w.sf_off + mxfp4_sf_bytes(M, K), 256);
+  w.total = round_up(w.g_off + gemm_scratch_bytes(M, N, K), 256);
   return w;
 }
 
@@ -97,10 +99,11 @@ size_t mxfp4_workspace_bytes(int op, int64_t M, int64_t N, int64_t K) {
     case MXFP4_OP_QUANTIZE:
       return 0;
     case MXFP4_OP_GEMM:
-      return kStatusBytes;
+      if (!shape_ok(M, K) || N < 0) return kStatusBytes;
+      return kStatusBytes + round_up(gemm_scratch_bytes(M, N, K), 256);
     case MXFP4_OP_LINEAR:
-      if (!shape_ok(M, K)) return 0;
-      return linear_workspace(M, K).total;
+      if (!shape_ok(M, K) || N < 0) return 0;
+      return linear_workspace(M, N, K).total;
     default:
       return 0;
   }
@@ -154,7 +157,8 @@ mxfp4_status mxfp4_gemm(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq
   if (M == 0) return MXFP4_OK;
   // The caller's previous kernel may have written bq / bsf: no early weight loads.
   return from_cuda(launch_gemm(aq, asf, bq, bsf, M, N, K, y, ydt == MXFP4_DT_F32, ldy,
-                               static_cast<int*>(ws), false, static_cast<cudaStream_t>(stream)));
+                               static_cast<int*>(ws), static_cast<uint8_t*>(ws) + kStatusBytes,
+                               ws_bytes - kStatusBytes, false, static_cast<cudaStream_t>(stream)));
 }
 
 mxfp4_status mxfp4_linear(const void* x, int64_t M, int64_t K, mxfp4_rotation mode,
@@ -169,7 +173,7 @@ mxfp4_status mxfp4_linear(const void* x, int64_t M, int64_t K, mxfp4_rotation mo
   if (!aligned16(x) || !aligned16(wq) || !aligned16(wsf) || !aligned16(y) || !aligned16(ws) ||
       (K * 2) % 16 != 0 || (N * 2) % 16 != 0)
     return MXFP4_ERR_ALIGN;
-  const LinearWorkspace w = linear_workspace(M, K);
+  const LinearWorkspace w = linear_workspace(M, N, K);
   if (ws_bytes < w.total) return MXFP4_ERR_WORKSPACE;
   KronCoeffs kc{};
   if (mode == MXFP4_ROT_KRON_4x8 && !kron_from_host(kron_a, kron_b, &kc))
@@ -183,8 +187,8 @@ mxfp4_status mxfp4_linear(const void* x, int64_t M, int64_t K, mxfp4_rotation mo
       launch_rotate_quantize(x, false, M, K, K, (int)mode, &kc, xq, xsf, static_cast<int*>(ws), s);
   if (e != cudaSuccess) return MXFP4_ERR_CUDA;
   // The kernel just before the GEMM is the quantiser above, which does not write W.
-  return from_cuda(
-      launch_gemm(xq, xsf, wq, wsf, M, N, K, y, false, N, static_cast<int*>(ws), true, s));
+  return from_cuda(launch_gemm(xq, xsf, wq, wsf, M, N, K, y, false, N, static_cast<int*>(ws),
+                               base + w.g_off, ws_bytes - w.g_off, true, s));
 }
 
 mxfp4_status mxfp4_poll_status(void* ws, mxfp4_status* out) {

@@ -59,7 +59,68 @@ struct Params {
   uint32_t k_atoms;        // ceil(K / 128): scale atoms per 128-row group
   uint32_t b_row_tiles;    // ceil(N / 128)
   uint64_t ldy;            // elements
+  // Work units: tiles [0, full_units) whole; each later tile split into split_g K chunks
+  // of kt_per_chunk k-tiles (units full_units + t * split_g + c). Chunk 0 owns the tile.
+  uint32_t full_units, units, split_g, kt_per_chunk;
+  unsigned int* flags;     // [2 * split tiles]: partials stored, owner warps done
+  float* part;             // [split tile][chunk 1..g-1][CTA rank] x 128 x 256 fp32
 };
+
+struct Unit {
+  uint32_t tile, kt0, kt1, chunk;
+  bool split;
+};
+
+__device__ __forceinline__ Unit unit_at(uint32_t u, const Params& p) {
+  Unit w;
+  if (u < p.full_units) {
+    w.tile = u;
+    w.kt0 = 0;
+    w.kt1 = p.k_tiles;
+    w.chunk = 0;
+    w.split = false;
+  } else {
+    const uint32_t v = u - p.full_units;
+    const uint32_t t = v / p.split_g;
+    w.chunk = v - t * p.split_g;
+    w.tile = p.full_units + t;
+    w.kt0 = w.chunk * p.kt_per_chunk;
+    w.kt1 = w.kt0 + p.kt_per_chunk < p.k_tiles ? w.kt0 + p.kt_per_chunk : p.k_tiles;
+    w.split = true;
+  }
+  return w;
+}
+
+// Partial of K chunk c (>= 1) of split tile t for this CTA's 128 rows, at the slot of
+// (32-row quarter `quad`, 4-column group g4, lane): lane-fastest, so a warp's 16-byte
+// accesses for one column group cover 512 consecutive bytes.
+__device__ __forceinline__ float* part_at(const Params& p, uint32_t t, uint32_t c, uint32_t rank,
+                                          uint32_t quad, uint32_t g4, uint32_t lane) {
+  const uint64_t base = ((uint64_t)(t * (p.split_g - 1) + (c - 1)) * 2 + rank) * (128u * 256u);
+  return p.part + base + ((uint64_t)(quad * 64u + g4) * 32u + lane) * 4u;
+}
+
+__device__ __forceinline__ uint32_t ld_acquire_u32(const unsigned int* ptr) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ptr) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Bounded wait until *ptr >= target (stores of the other chunks of a split tile).
+__device__ __forceinline__ bool wait_count(const unsigned int* ptr, uint32_t target) {
+  const uint64_t t0 = global_ns();
+  while (ld_acquire_u32(ptr) < target) {
+    if (global_ns() - t0 > kWaitLimitNs) return false;
+    __nanosleep(100);
+  }
+  return true;
+}
 
 __device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
@@ -174,18 +235,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   griddep_wait();
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
-  const uint32_t n_tiles_total = p.m_tiles * p.n_tiles;  // m_tiles counts 256-row pair tiles
-
   if (warp == kProducerWarp) {
     if (elect_one()) {
       const uint32_t full_at_leader = map_to_rank(bar_full, 0);
       uint32_t stage = 0, phase = 0, issued = 0;
       bool ok = true;
-      for (uint32_t tile = pair; tile < n_tiles_total && ok; tile += num_pairs) {
-        const uint32_t mt = tile / p.n_tiles, nt = tile % p.n_tiles;
+      for (uint32_t u = pair; u < p.units && ok; u += num_pairs) {
+        const Unit w = unit_at(u, p);
+        const uint32_t mt = w.tile / p.n_tiles, nt = w.tile % p.n_tiles;  // 256-row m tiles
         const int32_t m_cta = (int32_t)(mt * 256u + rank * 128u);
         const int32_t n_cta = (int32_t)(nt * BN + rank * 128u);
-        for (uint32_t kt = 0; kt < p.k_tiles; ++kt) {
+        for (uint32_t kt = w.kt0; kt < w.kt1; ++kt) {
           if (!mbar_wait_bounded(bar_empty + 8 * stage, phase ^ 1u, abort_flag, kWaitLimitNs)) {
             ok = false;
             break;
@@ -229,14 +289,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     if (rank == 0 && elect_one()) {
       uint32_t stage = 0, phase = 0, acc_phase = 0;
       bool ok = true;
-      for (uint32_t tile = pair; tile < n_tiles_total && ok; tile += num_pairs) {
+      for (uint32_t u = pair; u < p.units && ok; u += num_pairs) {
+        const Unit w = unit_at(u, p);
         if (!mbar_wait_bounded(bar_tempty, acc_phase ^ 1u, abort_flag, kWaitLimitNs)) {
           ok = false;
           break;
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (acc_phase ? C::ACC1_COL : 0u);
-        for (uint32_t kt = 0; kt < p.k_tiles; ++kt) {
+        for (uint32_t kt = w.kt0; kt < w.kt1; ++kt) {
           if (!mbar_wait_bounded(bar_full + 8 * stage, phase, abort_flag, kWaitLimitNs)) {
             ok = false;
             break;
@@ -259,7 +320,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             mma_mxf4_pair(d_tmem, smem_desc_sw128(a_tile + k * MMA_K_BYTES),
                           smem_desc_sw128(b_tile + k * MMA_K_BYTES), idesc_mxf4(256, BN, sf_id, sf_id),
                           tmem_base + C::SFA_COL + 4 * (k >> 1), tmem_base + C::SFB_COL + 8 * (k >> 1),
-                          (kt | k) != 0u);
+                          (kt != w.kt0 || k != 0u) ? 1u : 0u);
           }
           mma_commit_pair_both(bar_empty + 8 * stage);  // frees the stage in both CTAs
           if (++stage == STAGES) {
@@ -289,14 +350,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const uint32_t rowoff = buf + lane * 128u;
     constexpr uint32_t CCOLS = Y_F32 ? 32 : 64;  // columns per 128-byte staged row
     uint32_t acc_phase = 0;
-    for (uint32_t tile = pair; tile < n_tiles_total; tile += num_pairs) {
-      const uint32_t mt = tile / p.n_tiles, nt = tile % p.n_tiles;
+    for (uint32_t u = pair; u < p.units; u += num_pairs) {
+      const Unit w = unit_at(u, p);
+      const uint32_t mt = w.tile / p.n_tiles, nt = w.tile % p.n_tiles;
+      const uint32_t st = w.tile - p.full_units;  // index among split tiles (if split)
       const bool ok = mbar_wait_bounded(bar_tfull, acc_phase, abort_flag, kWaitLimitNs);
       if (!__all_sync(0xffffffffu, ok)) {  // leave together so .aligned ops stay convergent
         if (lane == 0) record_timeout(p.status);
         break;
       }
       tc_fence_after();
+      // Split tile, chunk 0: the other chunks' partials must be stored before they are added.
+      if (w.split && w.chunk == 0) {
+        bool got = true;
+        if (lane == 0) got = wait_count(p.flags + st, (p.split_g - 1) * 2u * kEpiWarps);
+        got = __shfl_sync(0xffffffffu, got ? 1 : 0, 0) != 0;
+        if (!got && lane == 0) record_timeout(p.status);
+      }
       const uint32_t acc_col = acc_phase ? C::ACC1_COL : 0u;
       const uint32_t shared_chunk = acc_phase ? 0u : 3u;
       uint32_t ch[2];
@@ -319,6 +389,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive_cluster(tempty_at_leader);
+        }
+        if (w.split && w.chunk != 0) {
+          // Another CTA pair owns this tile: store the fp32 partial for it.
+          float* dst = part_at(p, st, w.chunk, rank, quad, ch[r] * 16u, lane);
+#pragma unroll
+          for (uint32_t j = 0; j < 16; ++j) {
+            const uint32_t* src = &v[j / 8][(j % 8) * 4];
+            *reinterpret_cast<float4*>(dst + j * 128u) =
+                make_float4(__uint_as_float(src[0]), __uint_as_float(src[1]),
+                            __uint_as_float(src[2]), __uint_as_float(src[3]));
+          }
+          continue;
+        }
+        if (w.split) {
+          // Owner: add chunks 1, 2, ... in that order to its own chunk-0 sum.
+          for (uint32_t c = 1; c < p.split_g; ++c) {
+            const float* srcp = part_at(p, st, c, rank, quad, ch[r] * 16u, lane);
+#pragma unroll
+            for (uint32_t j = 0; j < 16; ++j) {
+              const float4 q = __ldcg(reinterpret_cast<const float4*>(srcp + j * 128u));
+              uint32_t* d = &v[j / 8][(j % 8) * 4];
+              d[0] = __float_as_uint(__uint_as_float(d[0]) + q.x);
+              d[1] = __float_as_uint(__uint_as_float(d[1]) + q.y);
+              d[2] = __float_as_uint(__uint_as_float(d[2]) + q.z);
+              d[3] = __float_as_uint(__uint_as_float(d[3]) + q.w);
+            }
+          }
         }
 #pragma unroll
         for (uint32_t c = 0; c < 64 / CCOLS; ++c) {
@@ -344,6 +441,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           if (lane == 0) {
             tma_store_2d(&tmap_y, buf, col0, row0);
             bulk_commit_group();
+          }
+        }
+      }
+      if (w.split) {
+        if (w.chunk != 0) {
+          // Publish this warp's part of the partial to the owner.
+          __threadfence();
+          __syncwarp();
+          if (lane == 0) atomicAdd(p.flags + st, 1u);
+        } else {
+          // Owner warps done reading: the last one clears both counters for the next launch.
+          __syncwarp();
+          if (lane == 0) {
+            const uint32_t n_split = (p.units - p.full_units) / p.split_g;
+            unsigned int* done = p.flags + n_split + st;
+            if (atomicAdd(done, 1u) == 2u * kEpiWarps - 1u) {
+              atomicExch(p.flags + st, 0u);
+              atomicExch(done, 0u);
+            }
           }
         }
       }
@@ -434,10 +550,53 @@ bool make_output_map(CUtensorMap* map, void* y, uint64_t M, uint64_t N, uint64_t
   return r == CUDA_SUCCESS;
 }
 
+// Work plan of the persistent pair kernel. Whole 256 x 256 tiles go round-robin over the
+// CTA pairs; when the last round would leave pairs idle, its tiles are split into K
+// chunks (at most 4) so that it finishes in a fraction of a round. Chunk c > 0 leaves an
+// fp32 partial in the scratch; chunk 0 adds them in order. Handing a partial over costs
+// about as long as 4 k-tiles of MMAs, so a chunk gets at least 8 (2048 elements of K).
+constexpr uint32_t kPlanPairs = 74;  // CTA-pair slots of a B200 (148 SMs), for scratch sizing
+constexpr uint32_t kMinChunkKt = 8;
+constexpr uint32_t kMaxSplit = 4;
+
+struct PairPlan {
+  uint32_t tiles, full_units, units, g, kt_per_chunk, n_split;
+  size_t flag_bytes, scratch_bytes;
+};
+
+size_t round256(size_t v) { return (v + 255) / 256 * 256; }
+
+PairPlan pair_plan(int64_t M, int64_t N, int64_t K, uint32_t pairs) {
+  PairPlan pl{};
+  const uint32_t k_tiles = (uint32_t)((K + 255) / 256);
+  pl.tiles = (uint32_t)(((M + 255) / 256) * ((N + 255) / 256));
+  pl.full_units = pl.units = pl.tiles;
+  pl.g = 1;
+  pl.kt_per_chunk = k_tiles;
+  const uint32_t tail = pairs ? pl.tiles % pairs : 0;
+  if (tail == 0) return pl;
+  uint32_t g = pairs / tail;
+  if (g > k_tiles / kMinChunkKt) g = k_tiles / kMinChunkKt;
+  if (g > kMaxSplit) g = kMaxSplit;
+  if (g < 2) return pl;
+  const uint32_t kt = (k_tiles + g - 1) / g;
+  g = (k_tiles + kt - 1) / kt;
+  if (g < 2) return pl;
+  pl.g = g;
+  pl.kt_per_chunk = kt;
+  pl.n_split = tail;
+  pl.full_units = pl.tiles - tail;
+  pl.units = pl.full_units + tail * g;
+  pl.flag_bytes = round256((size_t)2 * tail * sizeof(unsigned int));
+  pl.scratch_bytes = pl.flag_bytes + (size_t)tail * (g - 1) * 2 * 128 * 256 * sizeof(float);
+  return pl;
+}
+
 template <uint32_t STAGES, bool Y_F32>
 cudaError_t launch_pair(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq,
                         const uint8_t* bsf, int64_t M, int64_t N, int64_t K, void* y, int64_t ldy,
-                        int* status, cudaStream_t stream) {
+                        int* status, uint8_t* scratch, size_t scratch_bytes,
+                        cudaStream_t stream) {
   using C = PairConfig<STAGES>;
   const uint64_t k_atoms = (uint64_t)sf_katoms(K);
   CUtensorMap ta, tb, tsa, tsb, ty;
@@ -485,8 +644,17 @@ cudaError_t launch_pair(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq
   p.k_atoms = (uint32_t)k_atoms;
   p.b_row_tiles = (uint32_t)sf_row_tiles(N);
   p.ldy = (uint64_t)ldy;
-  const uint32_t tiles = p.m_tiles * p.n_tiles;
-  const uint32_t pairs = tiles < (uint32_t)max_clusters[dev] ? tiles : (uint32_t)max_clusters[dev];
+  PairPlan pl = pair_plan(M, N, K, (uint32_t)max_clusters[dev]);
+  if (pl.g > 1 && (scratch == nullptr || pl.scratch_bytes > scratch_bytes))
+    pl = pair_plan(M, N, K, 0);  // no room for partials: whole tiles only
+  p.full_units = pl.full_units;
+  p.units = pl.units;
+  p.split_g = pl.g;
+  p.kt_per_chunk = pl.kt_per_chunk;
+  p.flags = pl.g > 1 ? reinterpret_cast<unsigned int*>(scratch) : nullptr;
+  p.part = pl.g > 1 ? reinterpret_cast<float*>(scratch + pl.flag_bytes) : nullptr;
+  const uint32_t pairs =
+      pl.units < (uint32_t)max_clusters[dev] ? pl.units : (uint32_t)max_clusters[dev];
 
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(2 * pairs);
@@ -505,15 +673,23 @@ cudaError_t launch_pair(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq
 
 cudaError_t launch_gemm(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq,
                         const uint8_t* bsf, int64_t M, int64_t N, int64_t K, void* y,
-                        bool y_is_f32, int64_t ldy, int* status, bool b_early,
-                        cudaStream_t stream) {
+                        bool y_is_f32, int64_t ldy, int* status, uint8_t* scratch,
+                        size_t scratch_bytes, bool b_early, cudaStream_t stream) {
   // Few activation rows: stream the weights with the swap-AB split-K kernel.
   if (M <= 128)
     return launch_gemm_smallm(aq, asf, bq, bsf, M, N, K, y, y_is_f32, ldy, status, b_early,
                               stream);
   // Otherwise CTA pairs with 256 x 256 tiles.
-  if (y_is_f32) return launch_pair<5, true>(aq, asf, bq, bsf, M, N, K, y, ldy, status, stream);
-  return launch_pair<5, false>(aq, asf, bq, bsf, M, N, K, y, ldy, status, stream);
+  if (y_is_f32)
+    return launch_pair<5, true>(aq, asf, bq, bsf, M, N, K, y, ldy, status, scratch,
+                                scratch_bytes, stream);
+  return launch_pair<5, false>(aq, asf, bq, bsf, M, N, K, y, ldy, status, scratch, scratch_bytes,
+                               stream);
+}
+
+size_t gemm_scratch_bytes(int64_t M, int64_t N, int64_t K) {
+  if (M <= 128) return 0;
+  return pair_plan(M, N, K, kPlanPairs).scratch_bytes;
 }
 
 }  // namespace mxfp4

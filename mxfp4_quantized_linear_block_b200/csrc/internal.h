@@ -24,12 +24,18 @@ cudaError_t launch_rotate_quantize(const void* x, bool x_is_f32, int64_t rows, i
 // status: device word set to the timeout code if a bounded wait gives up.
 // Every kernel of the library is launched with programmatic dependent launch: it waits
 // for the previous kernel on the stream before touching memory that kernel may share.
+// scratch: scratch_bytes of device memory, zero before its first use and left zero by
+// every launch that completes (K-split partials and counters of the last round's tiles;
+// with less than gemm_scratch_bytes(M, N, K) the tiles are not split).
 // b_early: the kernel just before this launch on the stream does not write bq / bsf, so
 // the few-row kernel may start streaming them before that kernel has finished.
 cudaError_t launch_gemm(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq,
                         const uint8_t* bsf, int64_t M, int64_t N, int64_t K, void* y,
-                        bool y_is_f32, int64_t ldy, int* status, bool b_early,
-                        cudaStream_t stream);
+                        bool y_is_f32, int64_t ldy, int* status, uint8_t* scratch,
+                        size_t scratch_bytes, bool b_early, cudaStream_t stream);
+
+// Scratch that launch_gemm can use for this problem.
+size_t gemm_scratch_bytes(int64_t M, int64_t N, int64_t K);
 
 // Few-row path (M <= 128): swap-AB, K split across the CTAs of a cluster (gemm_smallm.cu).
 cudaError_t launch_gemm_smallm(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq,

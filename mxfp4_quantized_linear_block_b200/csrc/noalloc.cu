@@ -25,7 +25,9 @@ namespace {
 constexpr size_t kScratchBytes = MXFP4_NOALLOC_SCRATCH_BYTES;
 constexpr size_t kStatusBytes = 256;
 
-// Layout: [status word region (256 B) | Xq (M x K/2) | X scales], parts 256-byte aligned.
+// Layout: [status word region (256 B) | Xq (M x K/2) | X scales | GEMM scratch (the rest)],
+// parts 256-byte aligned. The array starts zeroed; the GEMM leaves its scratch counters
+// zeroed after every call that completes.
 static __device__ __align__(256) unsigned char g_linear_scratch[kScratchBytes];
 
 std::mutex g_scratch_mutex;
@@ -98,7 +100,9 @@ extern "C" mxfp4_status mxfp4_linear_noalloc(const void* x, int64_t M, int64_t K
       cudaSuccess)
     return MXFP4_ERR_CUDA;
   // The kernel just before the GEMM is the quantiser above, which does not write W.
-  if (launch_gemm(xq, xsf, wq, wsf, M, N, K, y, false, N, status_word, true, s) != cudaSuccess)
+  // GEMM scratch: what is left of the array (the GEMM splits no tile if it is too small).
+  if (launch_gemm(xq, xsf, wq, wsf, M, N, K, y, false, N, status_word, scratch + need,
+                  kScratchBytes - need, true, s) != cudaSuccess)
     return MXFP4_ERR_CUDA;
   return MXFP4_OK;
 }

@@ -99,6 +99,62 @@ def test_gemm_few_rows_single_pair_in_last_split():
     assert not y.any()
 
 
+# Large-M shapes whose last round of 256x256 tiles is split along K over several CTA
+# pairs (74 pairs on a B200; chunks of at least 8 k-tiles): tiles -> split tiles x K
+# chunks. (512,512,4096) 4 -> 4x2; (768,1024,8192) 12 -> 12x4; (700,784,6176) 12 ragged
+# tiles -> 12x3, chunks of 9, 9 and 7 k-tiles with a 32-element K tail.
+SPLIT_SHAPES = [(512, 512, 4096), (768, 1024, 8192), (700, 784, 6176)]
+
+
+@pytest.mark.parametrize("M,N,K", SPLIT_SHAPES)
+@pytest.mark.parametrize("out", ["bf16", "f32"])
+def test_gemm_split_last_round(M, N, K, out):
+    aq, as_ = _operand(M + 3 * N + K, M, K, 8)
+    bq, bs = _operand(M + 3 * N + K, N, K, 9)
+    y = _run(aq, as_, bq, bs, out)
+    ref, S = oracle.gemm(aq, as_, bq, bs)
+    check_gemm_values(y, ref, S, out, f"split gemm {M}x{N}x{K} {out}")
+
+
+def test_gemm_split_full_rounds_then_tail():
+    """80 tiles on 74 pairs: one round of whole tiles, then 6 tiles in 3 K chunks each.
+    Every element of the last 256-row band (which holds the 6 split tiles) is checked,
+    plus sampled pairs elsewhere."""
+    M, N, K = 2560, 2048, 6144
+    aq, as_ = _operand(5, M, K, 10)
+    bq, bs = _operand(5, N, K, 11)
+    y = _run(aq, as_, bq, bs, "f32")
+    ref, S = oracle.gemm(aq[M - 256:], as_[M - 256:], bq, bs)
+    check_gemm_values(y[M - 256:], ref, S, "f32", "last band")
+    mi, ni = _sample_pairs(M, N, n_random=2048, seed=3)
+    ref, S = oracle.gemm_pairs(aq, as_, bq, bs, mi, ni)
+    check_gemm_values(y[mi, ni], ref, S, "f32", "sampled")
+
+
+def test_gemm_split_repeat_and_scratch_reset():
+    """Back-to-back launches on different inputs through one workspace: each result is
+    right, repeated inputs give identical bits, and the split counters are zero after."""
+    import torch
+    import mxfp4_quantized_linear_block_b200 as mx
+    M, N, K = 768, 1024, 8192
+    ws = mx.new_workspace(mx.workspace_bytes(mx.OP_GEMM, M, N, K))
+    assert ws.numel() > 256 + 12 * 3 * 2 * 128 * 256 * 4  # partials of 12 tiles x 3 chunks
+    outs = []
+    for seed in (21, 22, 21):
+        aq, as_ = _operand(seed, M, K, 12)
+        bq, bs = _operand(seed, N, K, 13)
+        y = mx.gemm(to_dev(aq), to_dev(oracle.sf_to_physical(as_, K)), to_dev(bq),
+                    to_dev(oracle.sf_to_physical(bs, K)), M, N, K,
+                    out_dtype=torch.float32, ws=ws)
+        torch.cuda.synchronize()
+        outs.append(y.cpu().numpy())
+        ref, S = oracle.gemm(aq, as_, bq, bs)
+        check_gemm_values(outs[-1].astype(np.float64), ref, S, "f32", f"seed {seed}")
+    assert np.array_equal(outs[0].view(np.uint32), outs[2].view(np.uint32))
+    assert mx.poll_status(ws) == mx.OK
+    assert not ws[256:512].cpu().numpy().any()  # both counter arrays (2 x 12 words)
+
+
 def test_gemm_wide_scale_range_fp32():
     """Scales spread over most of the E8M0 range in fp32 output."""
     M, N, K = 256, 256, 1024
