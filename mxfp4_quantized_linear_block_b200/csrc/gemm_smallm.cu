@@ -86,6 +86,58 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return r;
 }
 
+// Cross-CTA sum of one W tile's K splits. CTA `sp` of the cluster owns the 4-column
+// groups [sp * 32 / S, (sp + 1) * 32 / S) of the tile's 128 columns, for every token; an
+// item is one (token, group): 4 fp32 values in each split's shared memory. The 128
+// epilogue threads take items tid, tid + 128, ...; IB items at a time, whose loads from
+// all S splits are issued together, then added in split order 0, 1, ..., S-1.
+template <uint32_t NT, bool Y_F32, uint32_t S>
+__device__ __forceinline__ void reduce_store(const SmallParams& p, uint32_t sbase, uint32_t wt,
+                                             uint32_t sp, uint32_t tid) {
+  constexpr uint32_t IB = 16 / S;  // 16 loads in flight per thread
+  const uint32_t g0 = sp * 32u / S, g1 = (sp + 1u) * 32u / S, width = g1 - g0;
+  const uint32_t rows = p.M < NT ? p.M : NT;
+  const uint32_t items = rows * width;
+  for (uint32_t it0 = tid; it0 < items; it0 += 128u * IB) {
+    float4 t[IB][S];
+    uint32_t tok[IB], col[IB];
+#pragma unroll
+    for (uint32_t i = 0; i < IB; ++i) {
+      const uint32_t it = it0 + i * 128u;
+      tok[i] = it / width;
+      const uint32_t g = g0 + (it - tok[i] * width);
+      col[i] = wt * 128u + g * 4u;  // N % 16 == 0: the 4 columns are all in or all out
+      if (it < items) {
+        const uint32_t off = sbase + (tok[i] * 128u + g * 4u) * 4u;
+#pragma unroll
+        for (uint32_t s = 0; s < S; ++s) t[i][s] = ld_shared_cluster_v4(map_to_rank(off, s));
+      }
+    }
+#pragma unroll
+    for (uint32_t i = 0; i < IB; ++i) {
+      if (it0 + i * 128u >= items || col[i] >= p.N) continue;
+      float4 acc = t[i][0];
+#pragma unroll
+      for (uint32_t s = 1; s < S; ++s) {
+        acc.x += t[i][s].x;
+        acc.y += t[i][s].y;
+        acc.z += t[i][s].z;
+        acc.w += t[i][s].w;
+      }
+      if constexpr (Y_F32) {
+        *reinterpret_cast<float4*>(static_cast<float*>(p.y) + (uint64_t)tok[i] * p.ldy + col[i]) =
+            acc;
+      } else {
+        uint2 b;
+        b.x = pack_bf16x2(acc.x, acc.y);
+        b.y = pack_bf16x2(acc.z, acc.w);
+        *reinterpret_cast<uint2*>(static_cast<uint16_t*>(p.y) + (uint64_t)tok[i] * p.ldy +
+                                  col[i]) = b;
+      }
+    }
+  }
+}
+
 template <uint32_t NT, bool Y_F32>
 __global__ void __launch_bounds__(kThreads, 2) mxf4_gemm_smallm_kernel(
     const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
@@ -279,39 +331,16 @@ __global__ void __launch_bounds__(kThreads, 2) mxf4_gemm_smallm_kernel(
     tc_fence_after();
     tmem_dealloc(tmem_base, C::TMEM_COLS);
   } else if (warp >= kFirstEpiWarp) {
-    // This CTA's share of the tile: 4-column groups [g0, g1) of the 32, for tokens m < M.
-    const uint32_t g0 = sp * 32u / S, g1 = (sp + 1u) * 32u / S, width = g1 - g0;
-    const uint32_t rows = p.M < NT ? p.M : NT;
-    const uint32_t items = rows * width;
-    for (uint32_t it = threadIdx.x - kFirstEpiWarp * 32u; it < items; it += 128u) {
-      const uint32_t m = it / width;
-      const uint32_t g = g0 + (it - m * width);
-      const uint32_t off = sbase + (m * 128u + g * 4u) * 4u;
-      float4 part[kMaxSplits];
-#pragma unroll
-      for (uint32_t s = 0; s < kMaxSplits; ++s)
-        if (s < S) part[s] = ld_shared_cluster_v4(map_to_rank(off, s));
-      float4 acc = part[0];
-#pragma unroll
-      for (uint32_t s = 1; s < kMaxSplits; ++s) {
-        if (s < S) {
-          acc.x += part[s].x;
-          acc.y += part[s].y;
-          acc.z += part[s].z;
-          acc.w += part[s].w;
-        }
-      }
-      const uint32_t n = wt * 128u + g * 4u;  // N % 16 == 0: the 4 columns are all in or all out
-      if (n < p.N) {
-        if constexpr (Y_F32) {
-          *reinterpret_cast<float4*>(static_cast<float*>(p.y) + (uint64_t)m * p.ldy + n) = acc;
-        } else {
-          uint2 b;
-          b.x = pack_bf16x2(acc.x, acc.y);
-          b.y = pack_bf16x2(acc.z, acc.w);
-          *reinterpret_cast<uint2*>(static_cast<uint16_t*>(p.y) + (uint64_t)m * p.ldy + n) = b;
-        }
-      }
+    const uint32_t tid = threadIdx.x - kFirstEpiWarp * 32u;
+    switch (S) {
+      case 1: reduce_store<NT, Y_F32, 1>(p, sbase, wt, sp, tid); break;
+      case 2: reduce_store<NT, Y_F32, 2>(p, sbase, wt, sp, tid); break;
+      case 3: reduce_store<NT, Y_F32, 3>(p, sbase, wt, sp, tid); break;
+      case 4: reduce_store<NT, Y_F32, 4>(p, sbase, wt, sp, tid); break;
+      case 5: reduce_store<NT, Y_F32, 5>(p, sbase, wt, sp, tid); break;
+      case 6: reduce_store<NT, Y_F32, 6>(p, sbase, wt, sp, tid); break;
+      case 7: reduce_store<NT, Y_F32, 7>(p, sbase, wt, sp, tid); break;
+      default: reduce_store<NT, Y_F32, 8>(p, sbase, wt, sp, tid); break;
     }
   }
   // No CTA leaves (and releases its shared memory) while a peer may still read it.
