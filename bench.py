@@ -226,6 +226,45 @@ class ClockSampler:
 
 # --------------------------------------------------------------------------- GPU arm
 
+# --------------------------------------------------------------------------- ranks
+#
+# One process per GPU; the layer is token-parallel (weak scaling): every rank runs the
+# same workload shape on its own token slice, with no data-path collective. The process
+# group carries only the barrier around the timed region and the max over ranks.
+
+def rank_inputs(wl, rank: int) -> dict:
+    """Host bf16 activations of one rank: same shapes on every rank, own seeded draws."""
+    xs = {}
+    for lin in wl.linears:
+        if lin.x_tensor not in xs:
+            x, _ = synth.activation_bf16(wl.seed + rank, lin.M, lin.K, lin.outlier_frac,
+                                         lin.outlier_factor, lin.x_tensor)
+            xs[lin.x_tensor] = x
+    return xs
+
+
+def rank_barrier(world: int) -> None:
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def rank_max(v: float, world: int, device) -> float:
+    """Maximum of v over the ranks (each rank's device time of the timed region)."""
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tflops(flops_per_step: float, steps: int, world: int, seconds: float) -> float:
+    """Whole-job throughput: the work of all ranks over the slowest rank's time."""
+    return flops_per_step * steps * world / seconds / 1e12
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
 
@@ -247,13 +286,7 @@ def run_ours(args, rank, world, local_rank):
         wq, wsf = mx.rotate_quantize(w, wl.rotation, Aw, Bw)
         del w
         weights.append((wq, wsf))
-    xs_host = {}
-    for lin in wl.linears:
-        if lin.x_tensor not in xs_host:
-            # each rank takes its own token slice of a weak-scaled batch: same shapes, own draws
-            x, _ = synth.activation_bf16(wl.seed + rank, lin.M, lin.K, lin.outlier_frac,
-                                         lin.outlier_factor, lin.x_tensor)
-            xs_host[lin.x_tensor] = x
+    xs_host = rank_inputs(wl, rank)
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
 
     def make_set():
@@ -291,17 +324,10 @@ def run_ours(args, rank, world, local_rank):
                       stream=s)
 
     def barrier():
-        if world > 1:
-            import torch.distributed as dist
-            dist.barrier()
+        rank_barrier(world)
 
     def max_over_ranks(v: float) -> float:
-        if world == 1:
-            return v
-        import torch.distributed as dist
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return rank_max(v, world, dev)
 
     # ---- warm-up
     for i in range(args.warmup):
@@ -355,7 +381,7 @@ def run_ours(args, rank, world, local_rank):
     clk = clocks.stop()
     elapsed = max_over_ranks(ev0.elapsed_time(ev1) * 1e-3)
     flops_step = wl.flops
-    value = flops_step * args.steps * world / elapsed / 1e12
+    value = job_tflops(flops_step, args.steps, world, elapsed)
     ms_per_step = elapsed / args.steps * 1e3
     launches = 2 * len(wl.linears) * args.steps
 
@@ -475,7 +501,7 @@ def run_ours(args, rank, world, local_rank):
         torch.cuda.synchronize()
         barrier()
         t_e2e = max_over_ranks(a.elapsed_time(b) * 1e-3)
-        e2e = {"value": flops_step * args.e2e_steps * world / t_e2e / 1e12, "unit": UNIT,
+        e2e = {"value": job_tflops(flops_step, args.e2e_steps, world, t_e2e), "unit": UNIT,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "ms_per_step": t_e2e / args.e2e_steps * 1e3, "steps": args.e2e_steps,
                "gpu_launches": 2 * len(wl.linears) * args.e2e_steps}
