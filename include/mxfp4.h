@@ -160,6 +160,37 @@ mxfp4_status mxfp4_gemm(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq
                         mxfp4_stream_t stream);
 
 /*
+ * mxfp4_gemm with a bias: y[m][n] = (fp32 accumulator) + bias[n], one fp32
+ * rounding, then the output conversion. bias: DEVICE fp32 [N], 16-byte
+ * aligned, not NULL. Everything else as mxfp4_gemm. (The bias of the step
+ * after the contraction: "AMD Quark delivers MXFP4 quantization for FLUX.1-dev
+ * on Instinct MI350 with 1.92x speedup", opening section; no formula given.)
+ */
+mxfp4_status mxfp4_gemm_bias(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq,
+                             const uint8_t* bsf, int64_t M, int64_t N, int64_t K,
+                             const float* bias, void* y, mxfp4_dtype ydt, int64_t ldy, void* ws,
+                             size_t ws_bytes, mxfp4_stream_t stream);
+
+/*
+ * mxfp4_gemm whose output is the next layer's MXFP4 activation operand, so no
+ * bf16 copy of Y is written or read between layers ("AMD Quark...", opening
+ * section and "What is MXFP4 and why does it eliminate dequantization
+ * overhead?"): v = (fp32 accumulator) + bias[n] (bias may be NULL), then each
+ * 32-column block of every row is rotated like an activation block (mode,
+ * with kron_a / kron_b as in mxfp4_rotate_quantize) and quantised with the
+ * scale rule and rounding of mxfp4_rotate_quantize, from those fp32 values.
+ * yq: packed codes [M, N/2] (row stride N/2 bytes); ysf: mxfp4_sf_bytes(M, N)
+ * bytes in the tensor-core layout of an [M, N] operand (padding written 0).
+ * Requirements: N % 32 == 0, yq / ysf / bias 16-byte aligned; workspace as
+ * mxfp4_gemm. yq / ysf can be passed as aq / asf of the next mxfp4_gemm*.
+ */
+mxfp4_status mxfp4_gemm_quantize(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq,
+                                 const uint8_t* bsf, int64_t M, int64_t N, int64_t K,
+                                 const float* bias, mxfp4_rotation mode, const float* kron_a,
+                                 const float* kron_b, uint8_t* yq, uint8_t* ysf, void* ws,
+                                 size_t ws_bytes, mxfp4_stream_t stream);
+
+/*
  * The whole layer: rotate + quantise x (bf16 [M, K], row stride K) into the
  * workspace, then the block-scaled GEMM with the pre-quantised weights
  * (wq/wsf: [N, K] operand prepared offline with the matching rotation), bf16

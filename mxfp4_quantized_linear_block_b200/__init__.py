@@ -6,7 +6,8 @@ memory and the current stream. If ``libmxfp4.so`` is missing the import fails;
 there is no fallback of any kind.
 
 Functions mirror the C ABI in ``include/mxfp4.h``:
-``quantize``, ``rotate_quantize``, ``gemm``, ``linear``, ``poll_status`` and
+``quantize``, ``rotate_quantize``, ``gemm``, ``gemm_bias``, ``gemm_quantize``,
+``linear``, ``linear_noalloc``, ``poll_status`` and
 the host helpers ``sf_bytes``, ``sf_offset``, ``workspace_bytes``,
 ``status_string``.
 """
@@ -26,7 +27,7 @@ OP_QUANTIZE, OP_GEMM, OP_LINEAR = 0, 1, 2
 EXPORTS = (
     "mxfp4_sf_bytes", "mxfp4_sf_offset", "mxfp4_workspace_bytes", "mxfp4_status_string",
     "mxfp4_quantize", "mxfp4_rotate_quantize", "mxfp4_gemm", "mxfp4_linear",
-    "mxfp4_poll_status", "mxfp4_linear_noalloc",
+    "mxfp4_poll_status", "mxfp4_linear_noalloc", "mxfp4_gemm_bias", "mxfp4_gemm_quantize",
 )
 
 
@@ -54,6 +55,9 @@ def _load() -> ctypes.CDLL:
         "mxfp4_linear": ([vp, i64, i64, i32, vp, vp, vp, vp, i64, vp, vp, sz, vp], i32),
         "mxfp4_poll_status": ([vp, vp], i32),
         "mxfp4_linear_noalloc": ([vp, i64, i64, i32, vp, vp, vp, vp, i64, vp, vp, vp], i32),
+        "mxfp4_gemm_bias": ([vp, vp, vp, vp, i64, i64, i64, vp, vp, i32, i64, vp, sz, vp], i32),
+        "mxfp4_gemm_quantize": ([vp, vp, vp, vp, i64, i64, i64, vp, i32, vp, vp, vp, vp, vp, sz,
+                                 vp], i32),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -168,6 +172,47 @@ def gemm(aq, asf, bq, bsf, M: int, N: int, K: int, y=None, out_dtype=None, ws=No
                         _stream_handle(stream))
     _check(st, "mxfp4_gemm")
     return y
+
+
+def gemm_bias(aq, asf, bq, bsf, M: int, N: int, K: int, bias, y=None, out_dtype=None, ws=None,
+              stream=None):
+    """y = A . B^T + bias (bias: fp32 CUDA tensor [N], added once in fp32)."""
+    torch = _torch()
+    out_dtype = out_dtype or torch.bfloat16
+    assert bias.dtype == torch.float32 and bias.numel() == N and bias.is_contiguous()
+    if y is None:
+        y = torch.empty((M, N), dtype=out_dtype, device=aq.device)
+    if ws is None:
+        ws = new_workspace(workspace_bytes(OP_GEMM, M, N, K), aq.device)
+    st = lib.mxfp4_gemm_bias(aq.data_ptr(), asf.data_ptr(), bq.data_ptr(), bsf.data_ptr(), M, N,
+                             K, bias.data_ptr(), y.data_ptr(), _dtype_code(y), y.stride(0),
+                             ws.data_ptr(), ws.numel(), _stream_handle(stream))
+    _check(st, "mxfp4_gemm_bias")
+    return y
+
+
+def gemm_quantize(aq, asf, bq, bsf, M: int, N: int, K: int, bias=None,
+                  mode: int = ROT_HADAMARD32, kron_a=None, kron_b=None, yq=None, ysf=None,
+                  ws=None, stream=None):
+    """GEMM whose output is MXFP4, ready as the next layer's activation operand:
+    (A . B^T + bias) with each 32-column block rotated (mode) and quantised.
+    Returns (yq [M, N/2] uint8, ysf [sf_bytes(M, N)] uint8)."""
+    torch = _torch()
+    dev = aq.device
+    if yq is None:
+        yq = torch.empty((M, N // 2), dtype=torch.uint8, device=dev)
+    if ysf is None:
+        ysf = torch.empty(sf_bytes(M, N), dtype=torch.uint8, device=dev)
+    if ws is None:
+        ws = new_workspace(workspace_bytes(OP_GEMM, M, N, K), dev)
+    a = _host_f32(kron_a, 16) if mode == ROT_KRON_4x8 else None
+    b = _host_f32(kron_b, 64) if mode == ROT_KRON_4x8 else None
+    st = lib.mxfp4_gemm_quantize(aq.data_ptr(), asf.data_ptr(), bq.data_ptr(), bsf.data_ptr(), M,
+                                 N, K, bias.data_ptr() if bias is not None else None, mode, a, b,
+                                 yq.data_ptr(), ysf.data_ptr(), ws.data_ptr(), ws.numel(),
+                                 _stream_handle(stream))
+    _check(st, "mxfp4_gemm_quantize")
+    return yq, ysf
 
 
 def linear(x, wq, wsf, N: int, mode: int = ROT_HADAMARD32, kron_a=None, kron_b=None, y=None,

@@ -156,9 +156,57 @@ mxfp4_status mxfp4_gemm(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq
   if (ws_bytes < mxfp4_workspace_bytes(MXFP4_OP_GEMM, M, N, K)) return MXFP4_ERR_WORKSPACE;
   if (M == 0) return MXFP4_OK;
   // The caller's previous kernel may have written bq / bsf: no early weight loads.
-  return from_cuda(launch_gemm(aq, asf, bq, bsf, M, N, K, y, ydt == MXFP4_DT_F32, ldy,
+  Epilogue ep;
+  ep.out = ydt == MXFP4_DT_F32 ? kOutF32 : kOutBf16;
+  return from_cuda(launch_gemm(aq, asf, bq, bsf, M, N, K, y, ep, ldy,
                                static_cast<int*>(ws), static_cast<uint8_t*>(ws) + kStatusBytes,
                                ws_bytes - kStatusBytes, false, static_cast<cudaStream_t>(stream)));
+}
+
+mxfp4_status mxfp4_gemm_bias(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq,
+                             const uint8_t* bsf, int64_t M, int64_t N, int64_t K,
+                             const float* bias, void* y, mxfp4_dtype ydt, int64_t ldy, void* ws,
+                             size_t ws_bytes, mxfp4_stream_t stream) {
+  mxfp4_status st = validate_gemm(aq, asf, bq, bsf, M, N, K, y, ydt, ldy);
+  if (st != MXFP4_OK) return st;
+  if (!ws || !bias) return MXFP4_ERR_INVALID_ARG;
+  if (!aligned16(ws) || !aligned16(bias)) return MXFP4_ERR_ALIGN;
+  if (ws_bytes < mxfp4_workspace_bytes(MXFP4_OP_GEMM, M, N, K)) return MXFP4_ERR_WORKSPACE;
+  if (M == 0) return MXFP4_OK;
+  Epilogue ep;
+  ep.out = ydt == MXFP4_DT_F32 ? kOutF32 : kOutBf16;
+  ep.bias = bias;
+  return from_cuda(launch_gemm(aq, asf, bq, bsf, M, N, K, y, ep, ldy, static_cast<int*>(ws),
+                               static_cast<uint8_t*>(ws) + kStatusBytes, ws_bytes - kStatusBytes,
+                               false, static_cast<cudaStream_t>(stream)));
+}
+
+mxfp4_status mxfp4_gemm_quantize(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq,
+                                 const uint8_t* bsf, int64_t M, int64_t N, int64_t K,
+                                 const float* bias, mxfp4_rotation mode, const float* kron_a,
+                                 const float* kron_b, uint8_t* yq, uint8_t* ysf, void* ws,
+                                 size_t ws_bytes, mxfp4_stream_t stream) {
+  if (!aq || !asf || !bq || !bsf || !yq || !ysf || !ws) return MXFP4_ERR_INVALID_ARG;
+  if (mode != MXFP4_ROT_NONE && mode != MXFP4_ROT_HADAMARD32 && mode != MXFP4_ROT_KRON_4x8)
+    return MXFP4_ERR_UNSUPPORTED;
+  if (!shape_ok(M, K) || N < 32 || N % 32 != 0 || !within_limits(M, K) || !within_limits(N, K) ||
+      !within_limits(M, N))
+    return MXFP4_ERR_SHAPE;
+  if (!aligned16(aq) || !aligned16(asf) || !aligned16(bq) || !aligned16(bsf) || !aligned16(yq) ||
+      !aligned16(ysf) || !aligned16(ws) || (bias && !aligned16(bias)))
+    return MXFP4_ERR_ALIGN;
+  if (ws_bytes < mxfp4_workspace_bytes(MXFP4_OP_GEMM, M, N, K)) return MXFP4_ERR_WORKSPACE;
+  Epilogue ep;
+  ep.out = kOutMxfp4;
+  ep.bias = bias;
+  ep.mode = (int)mode;
+  ep.ysf = ysf;
+  if (mode == MXFP4_ROT_KRON_4x8 && !kron_from_host(kron_a, kron_b, &ep.kc))
+    return MXFP4_ERR_INVALID_ARG;
+  if (M == 0) return MXFP4_OK;
+  return from_cuda(launch_gemm(aq, asf, bq, bsf, M, N, K, yq, ep, N / 2, static_cast<int*>(ws),
+                               static_cast<uint8_t*>(ws) + kStatusBytes, ws_bytes - kStatusBytes,
+                               false, static_cast<cudaStream_t>(stream)));
 }
 
 mxfp4_status mxfp4_linear(const void* x, int64_t M, int64_t K, mxfp4_rotation mode,
@@ -187,7 +235,7 @@ mxfp4_status mxfp4_linear(const void* x, int64_t M, int64_t K, mxfp4_rotation mo
       launch_rotate_quantize(x, false, M, K, K, (int)mode, &kc, xq, xsf, static_cast<int*>(ws), s);
   if (e != cudaSuccess) return MXFP4_ERR_CUDA;
   // The kernel just before the GEMM is the quantiser above, which does not write W.
-  return from_cuda(launch_gemm(xq, xsf, wq, wsf, M, N, K, y, false, N, static_cast<int*>(ws),
+  return from_cuda(launch_gemm(xq, xsf, wq, wsf, M, N, K, y, Epilogue{}, N, static_cast<int*>(ws),
                                base + w.g_off, ws_bytes - w.g_off, true, s));
 }
 

@@ -64,6 +64,11 @@ struct Params {
   uint32_t full_units, units, split_g, kt_per_chunk;
   unsigned int* flags;     // [2 * split tiles]: partials stored, owner warps done
   float* part;             // [split tile][chunk 1..g-1][CTA rank] x 128 x 256 fp32
+  const float* bias;       // [N] or null
+  uint8_t* yq;             // MXFP4 output: codes [M, ldy bytes per row]
+  uint8_t* ysf;            // MXFP4 output: scales, tensor-core layout of an [M, N] operand
+  uint32_t qmode;          // MXFP4 output: rotation of each 32-column block
+  uint32_t rows_pad, n_katoms_y;
 };
 
 struct Unit {
@@ -175,13 +180,15 @@ struct PairConfig {
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
-template <uint32_t STAGES, bool Y_F32>
+template <uint32_t STAGES, int OUT>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     mxf4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a,
                           const __grid_constant__ CUtensorMap tmap_b,
                           const __grid_constant__ CUtensorMap tmap_sfa,
                           const __grid_constant__ CUtensorMap tmap_sfb,
-                          const __grid_constant__ CUtensorMap tmap_y, const Params p) {
+                          const __grid_constant__ CUtensorMap tmap_y, const Params p,
+                          const __grid_constant__ KronCoeffs kc) {
+  constexpr bool Y_F32 = OUT == kOutF32;
   using C = PairConfig<STAGES>;
   constexpr uint32_t BN = C::BN;
   extern __shared__ uint8_t smem_raw[];
@@ -218,7 +225,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     prefetch_tmap(&tmap_b);
     prefetch_tmap(&tmap_sfa);
     prefetch_tmap(&tmap_sfb);
-    prefetch_tmap(&tmap_y);
+    if constexpr (OUT != kOutMxfp4) prefetch_tmap(&tmap_y);  // unused (zero) map otherwise
   }
   if (warp == kMmaWarp) {
     tmem_alloc_pair(smem_addr(tmem_slot), C::TMEM_COLS);
@@ -379,6 +386,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
       const uint32_t taddr = tmem_base + ((quad * 32u) << 16) + acc_col;
       const int32_t row0 = (int32_t)(mt * 256u + rank * 128u + quad * 32u);
+      uint32_t sfw = 0;  // MXFP4 output: this row's 4 scale bytes of the warp's 128 columns
 #pragma unroll
       for (uint32_t r = 0; r < 2; ++r) {
         uint32_t v[2][32];
@@ -417,31 +425,78 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             }
           }
         }
+        const uint32_t col_base = nt * BN + ch[r] * 64u;  // first column of this chunk
+        if (p.bias != nullptr) {
 #pragma unroll
-        for (uint32_t c = 0; c < 64 / CCOLS; ++c) {
-          const int32_t col0 = (int32_t)(nt * BN + ch[r] * 64u + c * CCOLS);
-          if (lane == 0) bulk_wait_read_all();  // the buffer's previous store has read it
-          __syncwarp();
+          for (uint32_t h = 0; h < 2; ++h) {
 #pragma unroll
-          for (uint32_t j = 0; j < 8; ++j) {
-            const uint32_t addr = rowoff + ((j ^ (lane & 7u)) << 4);
-            if constexpr (Y_F32) {
-              const uint32_t* src = &v[c][4 * j];
-              st_shared_v4(addr, src[0], src[1], src[2], src[3]);
-            } else {
-              const uint32_t* src = &v[j / 4][(8 * j) % 32];
-              st_shared_v4(addr, pack_bf16x2(__uint_as_float(src[0]), __uint_as_float(src[1])),
-                           pack_bf16x2(__uint_as_float(src[2]), __uint_as_float(src[3])),
-                           pack_bf16x2(__uint_as_float(src[4]), __uint_as_float(src[5])),
-                           pack_bf16x2(__uint_as_float(src[6]), __uint_as_float(src[7])));
+            for (uint32_t j = 0; j < 32; j += 4) {
+              const uint32_t col = col_base + h * 32u + j;  // N % 16 == 0: 4 in or 4 out
+              const float4 b = col < p.N ? __ldg(reinterpret_cast<const float4*>(p.bias + col))
+                                         : make_float4(0.f, 0.f, 0.f, 0.f);
+              v[h][j + 0] = __float_as_uint(__fadd_rn(__uint_as_float(v[h][j + 0]), b.x));
+              v[h][j + 1] = __float_as_uint(__fadd_rn(__uint_as_float(v[h][j + 1]), b.y));
+              v[h][j + 2] = __float_as_uint(__fadd_rn(__uint_as_float(v[h][j + 2]), b.z));
+              v[h][j + 3] = __float_as_uint(__fadd_rn(__uint_as_float(v[h][j + 3]), b.w));
             }
           }
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-            tma_store_2d(&tmap_y, buf, col0, row0);
-            bulk_commit_group();
+        }
+        if constexpr (OUT == kOutMxfp4) {
+          // Each 32 columns of this thread's row are one block of the next layer's
+          // operand: rotate, quantise, store 16 code bytes; collect the scale byte.
+          const uint32_t row = (uint32_t)row0 + lane;
+#pragma unroll
+          for (uint32_t h = 0; h < 2; ++h) {
+            float2 P[16];
+#pragma unroll
+            for (uint32_t j = 0; j < 16; ++j)
+              P[j] = make_float2(__uint_as_float(v[h][2 * j]), __uint_as_float(v[h][2 * j + 1]));
+            if (p.qmode == 1) blockq::hadamard32(P);
+            if (p.qmode == 2) blockq::kron32(P, kc);
+            uint4 codes;
+            const uint32_t byte = blockq::quantize_block(P, codes);
+            const uint32_t col = col_base + h * 32u;
+            const bool inside = row < p.M && col < p.N;
+            if (inside) blockq::st_v4(p.yq + (uint64_t)row * p.ldy + col / 2u, codes);
+            sfw |= (inside ? byte : 0u) << (((col / 32u) & 3u) * 8u);
           }
+        } else {
+#pragma unroll
+          for (uint32_t c = 0; c < 64 / CCOLS; ++c) {
+            const int32_t col0 = (int32_t)(nt * BN + ch[r] * 64u + c * CCOLS);
+            if (lane == 0) bulk_wait_read_all();  // the buffer's previous store has read it
+            __syncwarp();
+#pragma unroll
+            for (uint32_t j = 0; j < 8; ++j) {
+              const uint32_t addr = rowoff + ((j ^ (lane & 7u)) << 4);
+              if constexpr (Y_F32) {
+                const uint32_t* src = &v[c][4 * j];
+                st_shared_v4(addr, src[0], src[1], src[2], src[3]);
+              } else {
+                const uint32_t* src = &v[j / 4][(8 * j) % 32];
+                st_shared_v4(addr, pack_bf16x2(__uint_as_float(src[0]), __uint_as_float(src[1])),
+                             pack_bf16x2(__uint_as_float(src[2]), __uint_as_float(src[3])),
+                             pack_bf16x2(__uint_as_float(src[4]), __uint_as_float(src[5])),
+                             pack_bf16x2(__uint_as_float(src[6]), __uint_as_float(src[7])));
+              }
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(&tmap_y, buf, col0, row0);
+              bulk_commit_group();
+            }
+          }
+        }
+      }
+      if constexpr (OUT == kOutMxfp4) {
+        if (!(w.split && w.chunk != 0)) {
+          // The warp's two chunks are 128 aligned columns: one word of a scale atom per row.
+          const uint32_t row = (uint32_t)row0 + lane;
+          const uint32_t ka = nt * 2u + (ch[0] >= 2u ? 1u : 0u);
+          if (row < p.rows_pad && ka < p.n_katoms_y)
+            *reinterpret_cast<uint32_t*>(p.ysf + ((uint64_t)(row >> 7) * p.n_katoms_y + ka) * 512u +
+                                         (row & 31u) * 16u + ((row >> 5) & 3u) * 4u) = sfw;
         }
       }
       if (w.split) {
@@ -592,21 +647,22 @@ PairPlan pair_plan(int64_t M, int64_t N, int64_t K, uint32_t pairs) {
   return pl;
 }
 
-template <uint32_t STAGES, bool Y_F32>
+template <uint32_t STAGES, int OUT>
 cudaError_t launch_pair(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq,
-                        const uint8_t* bsf, int64_t M, int64_t N, int64_t K, void* y, int64_t ldy,
-                        int* status, uint8_t* scratch, size_t scratch_bytes,
-                        cudaStream_t stream) {
+                        const uint8_t* bsf, int64_t M, int64_t N, int64_t K, void* y,
+                        const Epilogue& ep, int64_t ldy, int* status, uint8_t* scratch,
+                        size_t scratch_bytes, cudaStream_t stream) {
   using C = PairConfig<STAGES>;
   const uint64_t k_atoms = (uint64_t)sf_katoms(K);
-  CUtensorMap ta, tb, tsa, tsb, ty;
+  CUtensorMap ta, tb, tsa, tsb, ty{};
   if (!make_operand_map(&ta, aq, (uint64_t)M, (uint64_t)(K / 2), 128) ||
       !make_operand_map(&tb, bq, (uint64_t)N, (uint64_t)(K / 2), 128) ||
       !make_scale_map(&tsa, asf, (uint64_t)sf_row_tiles(M), k_atoms, false) ||
       !make_scale_map(&tsb, bsf, (uint64_t)sf_row_tiles(N), k_atoms, true) ||
-      !make_output_map(&ty, y, (uint64_t)M, (uint64_t)N, (uint64_t)ldy, Y_F32))
+      (OUT != kOutMxfp4 &&
+       !make_output_map(&ty, y, (uint64_t)M, (uint64_t)N, (uint64_t)ldy, OUT == kOutF32)))
     return cudaErrorInvalidValue;
-  auto kern = mxf4_gemm_pair_kernel<STAGES, Y_F32>;
+  auto kern = mxf4_gemm_pair_kernel<STAGES, OUT>;
   int dev = 0;
   cudaGetDevice(&dev);
   static bool attr_done[64] = {};
@@ -653,6 +709,12 @@ cudaError_t launch_pair(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq
   p.kt_per_chunk = pl.kt_per_chunk;
   p.flags = pl.g > 1 ? reinterpret_cast<unsigned int*>(scratch) : nullptr;
   p.part = pl.g > 1 ? reinterpret_cast<float*>(scratch + pl.flag_bytes) : nullptr;
+  p.bias = ep.bias;
+  p.yq = OUT == kOutMxfp4 ? static_cast<uint8_t*>(y) : nullptr;
+  p.ysf = ep.ysf;
+  p.qmode = (uint32_t)ep.mode;
+  p.rows_pad = (uint32_t)(sf_row_tiles(M) * 128);
+  p.n_katoms_y = (uint32_t)sf_katoms(N);
   const uint32_t pairs =
       pl.units < (uint32_t)max_clusters[dev] ? pl.units : (uint32_t)max_clusters[dev];
 
@@ -666,25 +728,30 @@ cudaError_t launch_pair(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, ta, tb, tsa, tsb, ty, p);
+  return cudaLaunchKernelEx(&cfg, kern, ta, tb, tsa, tsb, ty, p, ep.kc);
 }
 
 }  // namespace
 
 cudaError_t launch_gemm(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq,
                         const uint8_t* bsf, int64_t M, int64_t N, int64_t K, void* y,
-                        bool y_is_f32, int64_t ldy, int* status, uint8_t* scratch,
+                        const Epilogue& ep, int64_t ldy, int* status, uint8_t* scratch,
                         size_t scratch_bytes, bool b_early, cudaStream_t stream) {
   // Few activation rows: stream the weights with the swap-AB split-K kernel.
   if (M <= 128)
-    return launch_gemm_smallm(aq, asf, bq, bsf, M, N, K, y, y_is_f32, ldy, status, b_early,
-                              stream);
+    return launch_gemm_smallm(aq, asf, bq, bsf, M, N, K, y, ep, ldy, status, b_early, stream);
   // Otherwise CTA pairs with 256 x 256 tiles.
-  if (y_is_f32)
-    return launch_pair<5, true>(aq, asf, bq, bsf, M, N, K, y, ldy, status, scratch,
-                                scratch_bytes, stream);
-  return launch_pair<5, false>(aq, asf, bq, bsf, M, N, K, y, ldy, status, scratch, scratch_bytes,
-                               stream);
+  switch (ep.out) {
+    case kOutF32:
+      return launch_pair<5, kOutF32>(aq, asf, bq, bsf, M, N, K, y, ep, ldy, status, scratch,
+                                     scratch_bytes, stream);
+    case kOutMxfp4:
+      return launch_pair<5, kOutMxfp4>(aq, asf, bq, bsf, M, N, K, y, ep, ldy, status, scratch,
+                                       scratch_bytes, stream);
+    default:
+      return launch_pair<5, kOutBf16>(aq, asf, bq, bsf, M, N, K, y, ep, ldy, status, scratch,
+                                      scratch_bytes, stream);
+  }
 }
 
 size_t gemm_scratch_bytes(int64_t M, int64_t N, int64_t K) {

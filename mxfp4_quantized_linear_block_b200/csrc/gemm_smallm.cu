@@ -24,6 +24,7 @@
 
 #include <cstdint>
 
+#include "block_quant.cuh"
 #include "internal.h"
 #include "sm100.cuh"
 
@@ -74,6 +75,10 @@ struct SmallParams {
   uint64_t ldy;
   uint32_t k_tiles, k_atoms, splits, kt_per_split;
   uint32_t w_early;     // W may be loaded before the previous kernel has finished
+  const float* bias;    // [N] or null
+  uint8_t* ysf;         // MXFP4 output: scales (tensor-core layout of an [M, N] operand)
+  uint32_t qmode;       // MXFP4 output: rotation of each 32-column block
+  uint32_t n_katoms_y;  // MXFP4 output: scale atoms per 128-row group of Y
 };
 
 __device__ __forceinline__ void record_timeout(int* status) {
@@ -91,7 +96,7 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 // item is one (token, group): 4 fp32 values in each split's shared memory. The 128
 // epilogue threads take items tid, tid + 128, ...; IB items at a time, whose loads from
 // all S splits are issued together, then added in split order 0, 1, ..., S-1.
-template <uint32_t NT, bool Y_F32, uint32_t S>
+template <uint32_t NT, int OUT, uint32_t S>
 __device__ __forceinline__ void reduce_store(const SmallParams& p, uint32_t sbase, uint32_t wt,
                                              uint32_t sp, uint32_t tid) {
   constexpr uint32_t IB = 16 / S;  // 16 loads in flight per thread
@@ -124,7 +129,14 @@ __device__ __forceinline__ void reduce_store(const SmallParams& p, uint32_t sbas
         acc.z += t[i][s].z;
         acc.w += t[i][s].w;
       }
-      if constexpr (Y_F32) {
+      if (p.bias != nullptr) {
+        const float4 b = __ldg(reinterpret_cast<const float4*>(p.bias + col[i]));
+        acc.x += b.x;
+        acc.y += b.y;
+        acc.z += b.z;
+        acc.w += b.w;
+      }
+      if constexpr (OUT == kOutF32) {
         *reinterpret_cast<float4*>(static_cast<float*>(p.y) + (uint64_t)tok[i] * p.ldy + col[i]) =
             acc;
       } else {
@@ -138,10 +150,66 @@ __device__ __forceinline__ void reduce_store(const SmallParams& p, uint32_t sbas
   }
 }
 
-template <uint32_t NT, bool Y_F32>
+// MXFP4 output: CTA sp owns the 32-column blocks b (0..3 of the tile) with b % S == sp;
+// an item is one (row, block) of the 128-row scale tile: for rows m < M the 32 values of
+// every split are added in split order (8 loads per split in flight), the bias added,
+// the block rotated and quantised like an activation block; rows m >= M only get their
+// zero scale byte (padding of the scale layout).
+template <uint32_t NT>
+__device__ __forceinline__ void reduce_store_mxfp4(const SmallParams& p, const KronCoeffs& kc,
+                                                   uint32_t sbase, uint32_t wt, uint32_t sp,
+                                                   uint32_t S, uint32_t tid) {
+  uint32_t own[4], n_own = 0;
+#pragma unroll
+  for (uint32_t b = 0; b < 4; ++b)
+    if (b % S == sp) own[n_own++] = b;
+  for (uint32_t it = tid; it < 128u * n_own; it += 128u) {
+    const uint32_t m = it / n_own;
+    const uint32_t b = own[it - m * n_own];
+    const uint32_t col = wt * 128u + b * 32u;
+    const uint32_t kb = col / 32u;
+    uint32_t byte = 0;
+    if (m < p.M && col < p.N) {  // N % 32 == 0: the block is all in or all out
+      const uint32_t off = sbase + (m * 128u + b * 32u) * 4u;
+      float2 P[16];
+      for (uint32_t s = 0; s < S; ++s) {  // split order 0, 1, ..., S-1
+        float4 t[8];
+#pragma unroll
+        for (uint32_t i = 0; i < 8; ++i) t[i] = ld_shared_cluster_v4(map_to_rank(off + 16u * i, s));
+#pragma unroll
+        for (uint32_t i = 0; i < 8; ++i) {
+          if (s == 0) {
+            P[2 * i] = make_float2(t[i].x, t[i].y);
+            P[2 * i + 1] = make_float2(t[i].z, t[i].w);
+          } else {
+            P[2 * i] = make_float2(P[2 * i].x + t[i].x, P[2 * i].y + t[i].y);
+            P[2 * i + 1] = make_float2(P[2 * i + 1].x + t[i].z, P[2 * i + 1].y + t[i].w);
+          }
+        }
+      }
+      if (p.bias != nullptr) {
+#pragma unroll
+        for (uint32_t i = 0; i < 8; ++i) {
+          const float4 bb = __ldg(reinterpret_cast<const float4*>(p.bias + col + 4u * i));
+          P[2 * i] = make_float2(__fadd_rn(P[2 * i].x, bb.x), __fadd_rn(P[2 * i].y, bb.y));
+          P[2 * i + 1] =
+              make_float2(__fadd_rn(P[2 * i + 1].x, bb.z), __fadd_rn(P[2 * i + 1].y, bb.w));
+        }
+      }
+      if (p.qmode == 1) blockq::hadamard32(P);
+      if (p.qmode == 2) blockq::kron32(P, kc);
+      uint4 codes;
+      byte = blockq::quantize_block(P, codes);
+      blockq::st_v4(static_cast<uint8_t*>(p.y) + (uint64_t)m * p.ldy + col / 2u, codes);
+    }
+    if (kb < p.n_katoms_y * 4u) p.ysf[blockq::sf_offset(m, kb, p.n_katoms_y)] = (uint8_t)byte;
+  }
+}
+
+template <uint32_t NT, int OUT>
 __global__ void __launch_bounds__(kThreads, 2) mxf4_gemm_smallm_kernel(
     const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
-    const SmallParams p) {
+    const SmallParams p, const __grid_constant__ KronCoeffs kc) {
   using C = SmallConfig<NT>;
   constexpr uint32_t STAGES = C::STAGES;
   extern __shared__ uint8_t smem_raw[];
@@ -332,15 +400,19 @@ __global__ void __launch_bounds__(kThreads, 2) mxf4_gemm_smallm_kernel(
     tmem_dealloc(tmem_base, C::TMEM_COLS);
   } else if (warp >= kFirstEpiWarp) {
     const uint32_t tid = threadIdx.x - kFirstEpiWarp * 32u;
-    switch (S) {
-      case 1: reduce_store<NT, Y_F32, 1>(p, sbase, wt, sp, tid); break;
-      case 2: reduce_store<NT, Y_F32, 2>(p, sbase, wt, sp, tid); break;
-      case 3: reduce_store<NT, Y_F32, 3>(p, sbase, wt, sp, tid); break;
-      case 4: reduce_store<NT, Y_F32, 4>(p, sbase, wt, sp, tid); break;
-      case 5: reduce_store<NT, Y_F32, 5>(p, sbase, wt, sp, tid); break;
-      case 6: reduce_store<NT, Y_F32, 6>(p, sbase, wt, sp, tid); break;
-      case 7: reduce_store<NT, Y_F32, 7>(p, sbase, wt, sp, tid); break;
-      default: reduce_store<NT, Y_F32, 8>(p, sbase, wt, sp, tid); break;
+    if constexpr (OUT == kOutMxfp4) {
+      reduce_store_mxfp4<NT>(p, kc, sbase, wt, sp, S, tid);
+    } else {
+      switch (S) {
+        case 1: reduce_store<NT, OUT, 1>(p, sbase, wt, sp, tid); break;
+        case 2: reduce_store<NT, OUT, 2>(p, sbase, wt, sp, tid); break;
+        case 3: reduce_store<NT, OUT, 3>(p, sbase, wt, sp, tid); break;
+        case 4: reduce_store<NT, OUT, 4>(p, sbase, wt, sp, tid); break;
+        case 5: reduce_store<NT, OUT, 5>(p, sbase, wt, sp, tid); break;
+        case 6: reduce_store<NT, OUT, 6>(p, sbase, wt, sp, tid); break;
+        case 7: reduce_store<NT, OUT, 7>(p, sbase, wt, sp, tid); break;
+        default: reduce_store<NT, OUT, 8>(p, sbase, wt, sp, tid); break;
+      }
     }
   }
   // No CTA leaves (and releases its shared memory) while a peer may still read it.
@@ -398,16 +470,17 @@ Plan make_plan(int64_t M, int64_t N, int64_t K) {
   return pl;
 }
 
-template <uint32_t NT, bool Y_F32>
+template <uint32_t NT, int OUT>
 cudaError_t launch_nt(const Plan& pl, const uint8_t* aq, const uint8_t* asf, const uint8_t* bq,
-                      const uint8_t* bsf, int64_t M, int64_t N, int64_t K, void* y, int64_t ldy,
-                      int* status, bool w_early, cudaStream_t stream) {
+                      const uint8_t* bsf, int64_t M, int64_t N, int64_t K, void* y,
+                      const Epilogue& ep, int64_t ldy, int* status, bool w_early,
+                      cudaStream_t stream) {
   using C = SmallConfig<NT>;
   CUtensorMap tw, tx;
   if (!operand_map(&tw, bq, (uint64_t)N, (uint64_t)(K / 2), 128) ||
       !operand_map(&tx, aq, (uint64_t)M, (uint64_t)(K / 2), NT))
     return cudaErrorInvalidValue;
-  auto kern = mxf4_gemm_smallm_kernel<NT, Y_F32>;
+  auto kern = mxf4_gemm_smallm_kernel<NT, OUT>;
   int dev = 0;
   cudaGetDevice(&dev);
   static bool attr_done[64] = {};
@@ -432,6 +505,10 @@ cudaError_t launch_nt(const Plan& pl, const uint8_t* aq, const uint8_t* asf, con
   p.splits = pl.splits;
   p.kt_per_split = pl.kt_per_split;
   p.w_early = w_early ? 1u : 0u;
+  p.bias = ep.bias;
+  p.ysf = ep.ysf;
+  p.qmode = (uint32_t)ep.mode;
+  p.n_katoms_y = (uint32_t)sf_katoms(N);
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(pl.units);
   cfg.blockDim = dim3(kThreads);
@@ -446,20 +523,28 @@ cudaError_t launch_nt(const Plan& pl, const uint8_t* aq, const uint8_t* asf, con
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, kern, tw, tx, p);
+  return cudaLaunchKernelEx(&cfg, kern, tw, tx, p, ep.kc);
 }
 
 }  // namespace
 
 cudaError_t launch_gemm_smallm(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq,
                                const uint8_t* bsf, int64_t M, int64_t N, int64_t K, void* y,
-                               bool y_is_f32, int64_t ldy, int* status, bool b_early,
+                               const Epilogue& ep, int64_t ldy, int* status, bool b_early,
                                cudaStream_t stream) {
   const Plan pl = make_plan(M, N, K);
-#define MXFP4_SMALLM(NTV)                                                                        \
-  return y_is_f32                                                                                \
-             ? launch_nt<NTV, true>(pl, aq, asf, bq, bsf, M, N, K, y, ldy, status, b_early, stream)  \
-             : launch_nt<NTV, false>(pl, aq, asf, bq, bsf, M, N, K, y, ldy, status, b_early, stream);
+#define MXFP4_SMALLM(NTV)                                                                       \
+  switch (ep.out) {                                                                             \
+    case kOutF32:                                                                               \
+      return launch_nt<NTV, kOutF32>(pl, aq, asf, bq, bsf, M, N, K, y, ep, ldy, status, b_early, \
+                                     stream);                                                   \
+    case kOutMxfp4:                                                                             \
+      return launch_nt<NTV, kOutMxfp4>(pl, aq, asf, bq, bsf, M, N, K, y, ep, ldy, status,       \
+                                       b_early, stream);                                        \
+    default:                                                                                    \
+      return launch_nt<NTV, kOutBf16>(pl, aq, asf, bq, bsf, M, N, K, y, ep, ldy, status,        \
+                                      b_early, stream);                                         \
+  }
   switch (pl.nt) {
     case 16: MXFP4_SMALLM(16)
     case 32: MXFP4_SMALLM(32)

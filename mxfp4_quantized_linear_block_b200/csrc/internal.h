@@ -20,6 +20,19 @@ cudaError_t launch_rotate_quantize(const void* x, bool x_is_f32, int64_t rows, i
                                    int64_t ldx, int mode, const KronCoeffs* kc, uint8_t* q,
                                    uint8_t* sf, int* status, cudaStream_t stream);
 
+// What the GEMM epilogue writes.
+enum OutKind { kOutBf16 = 0, kOutF32 = 1, kOutMxfp4 = 2 };
+struct Epilogue {
+  int out = kOutBf16;
+  const float* bias = nullptr;  // [N] fp32 added to every row before the output step
+  // kOutMxfp4 only: each 32-column block of a row is rotated (mode 0/1/2 with kc) and
+  // quantised; y holds the packed codes [M, N/2] (ldy bytes per row), ysf the scales in
+  // the tensor-core layout of an [M, N] operand.
+  int mode = 0;
+  KronCoeffs kc{};
+  uint8_t* ysf = nullptr;
+};
+
 // Block-scaled GEMM y[M, N] = A[M, K] . B[N, K]^T on tcgen05. Host-validated arguments.
 // status: device word set to the timeout code if a bounded wait gives up.
 // Every kernel of the library is launched with programmatic dependent launch: it waits
@@ -31,7 +44,7 @@ cudaError_t launch_rotate_quantize(const void* x, bool x_is_f32, int64_t rows, i
 // the few-row kernel may start streaming them before that kernel has finished.
 cudaError_t launch_gemm(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq,
                         const uint8_t* bsf, int64_t M, int64_t N, int64_t K, void* y,
-                        bool y_is_f32, int64_t ldy, int* status, uint8_t* scratch,
+                        const Epilogue& ep, int64_t ldy, int* status, uint8_t* scratch,
                         size_t scratch_bytes, bool b_early, cudaStream_t stream);
 
 // Scratch that launch_gemm can use for this problem.
@@ -40,7 +53,7 @@ size_t gemm_scratch_bytes(int64_t M, int64_t N, int64_t K);
 // Few-row path (M <= 128): swap-AB, K split across the CTAs of a cluster (gemm_smallm.cu).
 cudaError_t launch_gemm_smallm(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq,
                                const uint8_t* bsf, int64_t M, int64_t N, int64_t K, void* y,
-                               bool y_is_f32, int64_t ldy, int* status, bool b_early,
+                               const Epilogue& ep, int64_t ldy, int* status, bool b_early,
                                cudaStream_t stream);
 
 // Scale-factor layout helpers (host side).

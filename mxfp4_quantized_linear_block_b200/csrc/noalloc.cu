@@ -101,7 +101,7 @@ extern "C" mxfp4_status mxfp4_linear_noalloc(const void* x, int64_t M, int64_t K
     return MXFP4_ERR_CUDA;
   // The kernel just before the GEMM is the quantiser above, which does not write W.
   // GEMM scratch: what is left of the array (the GEMM splits no tile if it is too small).
-  if (launch_gemm(xq, xsf, wq, wsf, M, N, K, y, false, N, status_word, scratch + need,
+  if (launch_gemm(xq, xsf, wq, wsf, M, N, K, y, Epilogue{}, N, status_word, scratch + need,
                   kScratchBytes - need, true, s) != cudaSuccess)
     return MXFP4_ERR_CUDA;
   return MXFP4_OK;

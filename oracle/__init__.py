@@ -206,6 +206,18 @@ def linear(x_bf16: np.ndarray, wq, ws, mode: int, A=None, B=None):
     return ref, S, xq, xs
 
 
+def quantize_output(y_f32: np.ndarray, bias, mode: int, A=None, B=None):
+    """MXFP4 output of a layer (no bf16 round trip between layers, "AMD Quark delivers
+    MXFP4 quantization for FLUX.1-dev on Instinct MI350 with 1.92x speedup", opening
+    section): y + bias in fp32 (one rounding), then each 32-column block of every row
+    rotated and quantised exactly like activations. y_f32 is the fp32 accumulator the
+    quantisation decisions are taken from."""
+    y = _c(y_f32, np.float32)
+    if bias is not None:
+        y = (y + _c(bias, np.float32)[None, :]).astype(np.float32)
+    return rotate_quantize(y, mode, A, B, bf16=False)
+
+
 def prepare_weight(w_f32: np.ndarray, mode: int, A=None, B=None):
     """Offline weight preparation: rotate each 32-block of W (H, or T^-T for Kronecker), quantise."""
     if mode == ROT_KRON_4x8:

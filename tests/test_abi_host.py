@@ -109,3 +109,28 @@ def test_poll_status_null():
     import ctypes
     out = ctypes.c_int(0)
     assert mx.lib.mxfp4_poll_status(None, ctypes.byref(out)) == mx.ERR_INVALID_ARG
+
+
+def test_gemm_bias_and_quantize_argument_errors():
+    L = mx.lib
+    assert L.mxfp4_gemm_bias(P, P, P, P, 4, 16, 64, None, P, 0, 16, P, 256, None) == \
+        mx.ERR_INVALID_ARG  # bias is required
+    assert L.mxfp4_gemm_bias(P, P, P, P, 4, 16, 64, P + 4, P, 0, 16, P, 256, None) == mx.ERR_ALIGN
+    assert L.mxfp4_gemm_bias(P, P, P, P, 4, 24, 64, P, P, 0, 24, P, 256, None) == mx.ERR_SHAPE
+    assert L.mxfp4_gemm_bias(P, P, P, P, 0, 16, 64, P, P, 0, 16, P, 256, None) == mx.OK
+    ok = dict(M=4, N=64, K=64, bias=None, mode=1, a=None, b=None, yq=P, ysf=P, ws=P, wsb=256)
+
+    def q(**kw):
+        a = {**ok, **kw}
+        return L.mxfp4_gemm_quantize(P, P, P, P, a["M"], a["N"], a["K"], a["bias"], a["mode"],
+                                     a["a"], a["b"], a["yq"], a["ysf"], a["ws"], a["wsb"], None)
+
+    assert q(yq=None) == mx.ERR_INVALID_ARG
+    assert q(ysf=None) == mx.ERR_INVALID_ARG
+    assert q(N=48) == mx.ERR_SHAPE            # N % 32 != 0 (the output's 32-blocks)
+    assert q(mode=7) == mx.ERR_UNSUPPORTED
+    assert q(mode=2) == mx.ERR_INVALID_ARG    # Kronecker needs both factors
+    assert q(bias=P + 8) == mx.ERR_ALIGN
+    assert q(ysf=P + 1) == mx.ERR_ALIGN
+    assert q(wsb=16) == mx.ERR_WORKSPACE
+    assert q(M=0) == mx.OK

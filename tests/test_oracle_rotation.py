@@ -119,3 +119,34 @@ def test_rotate_quantize_composes_rotation_and_quantisation():
     codes, sc = oracle.quantize_blocks(y)
     assert np.array_equal(oracle.unpack_codes(q).reshape(-1, 32), codes)
     assert np.array_equal(s.reshape(-1), sc)
+
+
+def test_quantize_output_adds_bias_once_in_fp32_then_quantises():
+    """MXFP4 output: row r of y + bias lands exactly on the E2M1 grid times 2^3, so the
+    codes are the grid's codes and every scale byte is 127 + 3 (amax 48 = 6 * 2^3)."""
+    grid = np.array([0, 0.5, 1, 1.5, 2, 3, 4, 6], np.float64)
+    target = np.concatenate([grid, -grid[::-1], grid, -grid[::-1]]) * 8.0  # 32 values
+    target[target == 0] = 0.0  # (y - b) + b is +0 in IEEE arithmetic, never -0
+    bias = (np.arange(32) % 5 - 2).astype(np.float32) * np.float32(0.25)  # exact quarters
+    y = np.stack([target - bias.astype(np.float64)] * 3).astype(np.float32)  # exact in fp32
+    q, s = oracle.quantize_output(y, bias, oracle.ROT_NONE)
+    codes = oracle.unpack_codes(q)
+    want = np.array([oracle.e2m1_code(v / 8.0) for v in target], np.uint8)
+    assert np.array_equal(codes, np.stack([want] * 3))
+    assert np.all(s == 130)
+    # no bias: the same as quantising y itself
+    q0, s0 = oracle.quantize_output(y, None, oracle.ROT_HADAMARD32)
+    q1, s1 = oracle.rotate_quantize(y, oracle.ROT_HADAMARD32, bf16=False)
+    assert np.array_equal(q0, q1) and np.array_equal(s0, s1)
+
+
+def test_quantize_output_rounds_the_sum_once():
+    """y + bias is one fp32 rounding (ties to even): 1 + 2^-24 -> 1, 1 + 3 * 2^-24 -> 1 + 2^-22."""
+    y = np.ones((1, 32), np.float32)
+    b = np.zeros(32, np.float32)
+    b[0], b[1] = 2.0 ** -24, 3 * 2.0 ** -24
+    yb = (y + b[None, :]).astype(np.float32)
+    assert yb[0, 0] == np.float32(1.0) and yb[0, 1] == np.float32(1.0 + 2.0 ** -22)
+    q, s = oracle.quantize_output(y, b, oracle.ROT_NONE)
+    q2, s2 = oracle.rotate_quantize(yb, oracle.ROT_NONE, bf16=False)
+    assert np.array_equal(q, q2) and np.array_equal(s, s2)
