@@ -85,6 +85,14 @@ __device__ __forceinline__ void record_timeout(int* status) {
   if (status) atomicExch(status, kTimeoutCode);
 }
 
+// Byte offset of the 4 fp32 values of (token m, 4-column group g) in a CTA's partial
+// [NT][128]: groups are XOR-swizzled by m % 8 within each 32-column block, so the 16-byte
+// reads of consecutive tokens (same g) fall on different banks, and a warp's stores of
+// one token still cover 512 contiguous bytes.
+__device__ __forceinline__ uint32_t red_off(uint32_t m, uint32_t g) {
+  return (m * 128u + ((g ^ (m & 7u)) * 4u)) * 4u;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
@@ -113,7 +121,7 @@ __device__ __forceinline__ void reduce_store(const SmallParams& p, uint32_t sbas
       const uint32_t g = g0 + (it - tok[i] * width);
       col[i] = wt * 128u + g * 4u;  // N % 16 == 0: the 4 columns are all in or all out
       if (it < items) {
-        const uint32_t off = sbase + (tok[i] * 128u + g * 4u) * 4u;
+        const uint32_t off = sbase + red_off(tok[i], g);
 #pragma unroll
         for (uint32_t s = 0; s < S; ++s) t[i][s] = ld_shared_cluster_v4(map_to_rank(off, s));
       }
@@ -152,7 +160,7 @@ __device__ __forceinline__ void reduce_store(const SmallParams& p, uint32_t sbas
 
 // MXFP4 output: CTA sp owns the 32-column blocks b (0..3 of the tile) with b % S == sp;
 // an item is one (row, block) of the 128-row scale tile: for rows m < M the 32 values of
-// every split are added in split order (8 loads per split in flight), the bias added,
+// every split are added in split order (two splits' loads in flight), the bias added,
 // the block rotated and quantised like an activation block; rows m >= M only get their
 // zero scale byte (padding of the scale layout).
 template <uint32_t NT>
@@ -170,20 +178,27 @@ __device__ __forceinline__ void reduce_store_mxfp4(const SmallParams& p, const K
     const uint32_t kb = col / 32u;
     uint32_t byte = 0;
     if (m < p.M && col < p.N) {  // N % 32 == 0: the block is all in or all out
-      const uint32_t off = sbase + (m * 128u + b * 32u) * 4u;
       float2 P[16];
-      for (uint32_t s = 0; s < S; ++s) {  // split order 0, 1, ..., S-1
-        float4 t[8];
+      for (uint32_t s0 = 0; s0 < S; s0 += 2) {  // two splits' loads in flight, added in order
+        float4 t[2][8];
 #pragma unroll
-        for (uint32_t i = 0; i < 8; ++i) t[i] = ld_shared_cluster_v4(map_to_rank(off + 16u * i, s));
+        for (uint32_t h = 0; h < 2; ++h)
 #pragma unroll
-        for (uint32_t i = 0; i < 8; ++i) {
-          if (s == 0) {
-            P[2 * i] = make_float2(t[i].x, t[i].y);
-            P[2 * i + 1] = make_float2(t[i].z, t[i].w);
-          } else {
-            P[2 * i] = make_float2(P[2 * i].x + t[i].x, P[2 * i].y + t[i].y);
-            P[2 * i + 1] = make_float2(P[2 * i + 1].x + t[i].z, P[2 * i + 1].y + t[i].w);
+          for (uint32_t i = 0; i < 8; ++i)
+            if (s0 + h < S)
+              t[h][i] = ld_shared_cluster_v4(map_to_rank(sbase + red_off(m, b * 8u + i), s0 + h));
+#pragma unroll
+        for (uint32_t h = 0; h < 2; ++h) {
+          if (s0 + h >= S) break;
+#pragma unroll
+          for (uint32_t i = 0; i < 8; ++i) {
+            if (s0 + h == 0) {
+              P[2 * i] = make_float2(t[h][i].x, t[h][i].y);
+              P[2 * i + 1] = make_float2(t[h][i].z, t[h][i].w);
+            } else {
+              P[2 * i] = make_float2(P[2 * i].x + t[h][i].x, P[2 * i].y + t[h][i].y);
+              P[2 * i + 1] = make_float2(P[2 * i + 1].x + t[h][i].z, P[2 * i + 1].y + t[h][i].w);
+            }
           }
         }
       }
@@ -385,7 +400,8 @@ __global__ void __launch_bounds__(kThreads, 2) mxf4_gemm_smallm_kernel(
         tmem_ld_wait();
 #pragma unroll
         for (uint32_t j = 0; j < 32; ++j)
-          if (c0 + j < NT) red[(c0 + j) * 128u + c] = __uint_as_float(v[j]);
+          if (c0 + j < NT)
+            red[red_off(c0 + j, c >> 2) / 4u + (c & 3u)] = __uint_as_float(v[j]);
       }
     } else if (lane == 0) {
       record_timeout(p.status);
