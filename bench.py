@@ -91,6 +91,10 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="dit_b1", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--chain", action="store_true",
+                    help="run the workload's linears as consecutive layers: each GEMM but the "
+                         "last writes MXFP4 (mxfp4_gemm_quantize) that the next GEMM reads, "
+                         "so only the first input is quantised from bf16")
     ap.add_argument("--e2e-steps", type=int, default=5)
     return ap.parse_args()
 
@@ -541,6 +545,213 @@ def run_ours(args, rank, world, local_rank):
     return result
 
 
+# --------------------------------------------------------------------------- chained layers
+
+def run_chain(args, rank, world, local_rank):
+    """Consecutive layers with MXFP4 between them: rotate+quantise X0 once, then
+    mxfp4_gemm_quantize for every layer but the last (its output, rotated and quantised
+    in the epilogue, is the next layer's operand), then mxfp4_gemm (bf16 out)."""
+    import torch
+
+    import mxfp4_quantized_linear_block_b200 as mx
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    wl = synth.WORKLOADS[args.workload]
+    L = wl.linears
+    for a, b in zip(L, L[1:]):
+        if a.N != b.K or a.M != b.M:
+            raise SystemExit(f"--chain: {a.name} ({a.M}x{a.N}) does not feed {b.name} ({b.M}x{b.K})")
+    if wl.rotation == synth.ROT_KRON_4x8:
+        raise SystemExit("--chain: Kronecker workloads need one transform per layer")
+    peaks = load_peaks()
+    mode = wl.rotation
+    weights = []
+    for lin in L:
+        w = torch.from_numpy(synth.weight_f32(wl.seed, lin.N, lin.K, lin.layer)).to(dev)
+        weights.append(mx.rotate_quantize(w, mode))
+        del w
+    x_host = rank_inputs(wl, rank)[L[0].x_tensor]
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+
+    def make_set():
+        x = torch.from_numpy(x_host.view(np.int16)).view(torch.bfloat16).to(dev)
+        acts = [(torch.empty((l.M, l.K // 2), dtype=torch.uint8, device=dev),
+                 torch.empty(mx.sf_bytes(l.M, l.K), dtype=torch.uint8, device=dev)) for l in L]
+        y = torch.empty((L[-1].M, L[-1].N), dtype=torch.bfloat16, device=dev)
+        gws = [mx.new_workspace(mx.workspace_bytes(mx.OP_GEMM, l.M, l.N, l.K), dev) for l in L]
+        return x, acts, y, gws
+
+    def set_bytes(st):
+        x, acts, y, gws = st
+        return (x.numel() * 2 + sum(q.numel() + f.numel() for q, f in acts) + y.numel() * 2 +
+                sum(g.numel() for g in gws))
+
+    w_bytes = sum(q.numel() + f.numel() for q, f in weights)
+    sets = [make_set()]
+    wsets = [weights]
+    while len(sets) * set_bytes(sets[0]) + len(wsets) * w_bytes < 3 * l2:
+        if len(sets) < 8 and set_bytes(sets[0]) >= w_bytes:
+            sets.append(make_set())
+        else:
+            wsets.append([(q.clone(), f.clone()) for q, f in weights])
+    footprint = len(sets) * set_bytes(sets[0]) + len(wsets) * w_bytes
+    stream = torch.cuda.current_stream(dev)
+
+    def step(i, s=stream, ev=None):
+        x, acts, y, gws = sets[i % len(sets)]
+        W = wsets[i % len(wsets)]
+        if ev is not None:
+            ev[0].record(stream)
+        mx.rotate_quantize(x, mode, q=acts[0][0], sf=acts[0][1], stream=s)
+        for j, lin in enumerate(L):
+            if ev is not None:
+                ev[j + 1].record(stream)
+            if j + 1 < len(L):
+                mx.gemm_quantize(acts[j][0], acts[j][1], W[j][0], W[j][1], lin.M, lin.N, lin.K,
+                                 mode=mode, yq=acts[j + 1][0], ysf=acts[j + 1][1], ws=gws[j],
+                                 stream=s)
+            else:
+                mx.gemm(acts[j][0], acts[j][1], W[j][0], W[j][1], lin.M, lin.N, lin.K, y=y,
+                        ws=gws[j], stream=s)
+        if ev is not None:
+            ev[len(L) + 1].record(stream)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    period = len(sets) * len(wsets) // math.gcd(len(sets), len(wsets))
+    U = period * max(1, 64 // period)
+    U = min(U, max(args.steps, 1))
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for i in range(U):
+            step(i, None)
+    n_full, rest = divmod(args.steps, U)
+    g_rest = None
+    if rest:
+        g_rest = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_rest):
+            for i in range(rest):
+                step(i, None)
+    g.replay()
+    torch.cuda.synchronize()
+
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    time.sleep(0.3)
+    rank_barrier(world)
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda._sleep(int(2e7))
+    ev0.record(stream)
+    for _ in range(n_full):
+        g.replay()
+    if g_rest is not None:
+        g_rest.replay()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    rank_barrier(world)
+    clk = clocks.stop()
+    elapsed = rank_max(ev0.elapsed_time(ev1) * 1e-3, world, dev)
+    value = job_tflops(wl.flops, args.steps, world, elapsed)
+
+    # attribution: events around every kernel of the same steps (eager launches)
+    n_attr = max(1, min(args.steps, args.attr_steps))
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(L) + 2)]
+           for _ in range(n_attr)]
+    torch.cuda._sleep(int(2e7))
+    for i in range(n_attr):
+        step(i, stream, evs[i])
+    torch.cuda.synchronize()
+    t_q = np.mean([e[0].elapsed_time(e[1]) * 1e-3 for e in evs])
+    t_g = np.array([np.mean([e[j + 1].elapsed_time(e[j + 2]) * 1e-3 for e in evs])
+                    for j in range(len(L))])
+    flops = np.array([l.flops for l in L], np.float64)
+    fp4_peak = peaks["bf16_tflops_sustained"] * FP4_OVER_BF16
+    # algorithmic bytes of each GEMM: its MXFP4 input and weight, and its output (MXFP4
+    # codes + scales between layers, bf16 after the last)
+    g_bytes = np.array([l.M * l.K // 2 + mx.sf_bytes(l.M, l.K) + l.N * l.K // 2 +
+                        mx.sf_bytes(l.N, l.K) +
+                        ((l.M * l.N // 2 + mx.sf_bytes(l.M, l.N)) if j + 1 < len(L)
+                         else 2 * l.M * l.N) for j, l in enumerate(L)], np.float64)
+    ridge = fp4_peak * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    intensity = flops.sum() / g_bytes.sum()
+    if intensity >= ridge:
+        roof = {"bound": "tensor", "achieved": flops.sum() / t_g.sum() / 1e12, "peak": fp4_peak,
+                "unit": "TFLOP/s", "peak_source": f"4 x {peaks['source']} bf16 sustained "
+                                                  f"({peaks['bf16_tflops_sustained']} TFLOP/s)"}
+    else:
+        roof = {"bound": "hbm", "achieved": g_bytes.sum() / t_g.sum() / 1e9,
+                "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "peak_source": f"{peaks['source']} HBM copy bandwidth"}
+    roof.update({"frac": roof["achieved"] / roof["peak"],
+                 "kernel": ("mxf4_gemm_pair_kernel" if L[0].M > 128 else "mxf4_gemm_smallm_kernel")
+                 + " (MXFP4 out between layers, bf16 out of the last)",
+                 "intensity_flop_per_byte": intensity, "ridge_flop_per_byte": ridge,
+                 "per_launch": [{"linear": l.name, "us": t_g[j] * 1e6,
+                                 "tflops": flops[j] / t_g[j] / 1e12,
+                                 "gbs": g_bytes[j] / t_g[j] / 1e9, "alg_bytes": int(g_bytes[j])}
+                                for j, l in enumerate(L)],
+                 "traffic": None})
+    x0 = L[0]
+    q_bytes = 2 * x0.M * x0.K + x0.M * x0.K // 2 + mx.sf_bytes(x0.M, x0.K)
+
+    # end to end: pinned X0 in, Y out, eager calls
+    x_pin = torch.from_numpy(x_host.view(np.int16)).view(torch.bfloat16).pin_memory()
+    y_pin = torch.empty((L[-1].M, L[-1].N), dtype=torch.bfloat16).pin_memory()
+    e2e = None
+    if args.e2e_steps > 0:
+        def e2e_step(i):
+            sets[0][0].copy_(x_pin, non_blocking=True)
+            step(0)
+            y_pin.copy_(sets[0][2], non_blocking=True)
+        e2e_step(0)
+        torch.cuda.synchronize()
+        rank_barrier(world)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda._sleep(int(2e7))
+        a.record(stream)
+        for i in range(args.e2e_steps):
+            e2e_step(i)
+        b.record(stream)
+        torch.cuda.synchronize()
+        rank_barrier(world)
+        t_e2e = rank_max(a.elapsed_time(b) * 1e-3, world, dev)
+        e2e = {"value": job_tflops(wl.flops, args.e2e_steps, world, t_e2e), "unit": UNIT,
+               "h2d_bytes_per_step": int(x_pin.numel() * 2),
+               "d2h_bytes_per_step": int(y_pin.numel() * 2),
+               "ms_per_step": t_e2e / args.e2e_steps * 1e3, "steps": args.e2e_steps,
+               "gpu_launches": (1 + len(L)) * args.e2e_steps}
+    for st in sets:
+        for gw in st[3]:
+            if mx.poll_status(gw) != mx.OK:
+                raise RuntimeError("a kernel reported a bounded-wait timeout")
+    return {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": elapsed / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "mxfp4",
+        "dtype_detail": "E2M1 x E2M1 with E8M0 block-32 scales, fp32 accumulate; MXFP4 "
+                        "between layers, bf16 out of the last",
+        "data": "synthetic (seeded N(0,1) activations with outlier channels, N(0,0.02^2) weights)",
+        "config": {"workload": workload_desc(wl) + "; chained: MXFP4 between layers",
+                   "tokens_per_gpu": L[0].M, "gflop_per_step_per_gpu": wl.flops / 1e9,
+                   "parallelism": f"replicas x{world} (token-parallel, no collective)",
+                   "launch": f"timed steps replayed from CUDA graphs of {U} steps",
+                   "l2": f"{len(sets)} rotating sets and {len(wsets)} weight copies, footprint "
+                         f"{footprint / 2**20:.0f} MiB >= 3 x L2 ({l2 / 2**20:.0f} MiB)"},
+        "roofline": roof,
+        "quantize_roofline": {"bound": "hbm", "kernel": "rotate_quantize_kernel (X0 only)",
+                              "achieved": q_bytes / t_q / 1e9, "peak": peaks["hbm_gbs"],
+                              "unit": "GB/s", "frac": q_bytes / t_q / 1e9 / peaks["hbm_gbs"],
+                              "per_launch_us": [t_q * 1e6], "traffic": None},
+        "e2e": e2e,
+        "gpu_launches": (1 + len(L)) * args.steps,
+        "attribution": {"steps": n_attr, "gpu_launches": (1 + len(L)) * n_attr},
+        "clocks": clk,
+    }
+
+
 # --------------------------------------------------------------------------- reference arm
 
 def run_reference(args):
@@ -583,7 +794,7 @@ def main():
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     try:
-        res = run_ours(args, rank, world, local_rank)
+        res = (run_chain if args.chain else run_ours)(args, rank, world, local_rank)
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
             v, sample = oracle_sample_time(synth.WORKLOADS[args.workload])
             res["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cpu_cores(),

@@ -200,6 +200,11 @@ WORKLOADS = {
     "llm_small_m128": Workload("llm_small_m128", ROT_HADAMARD32, (
         Linear("up", 128, 4096, 14336, 0, TID_X, 0.005, 50.0),
         Linear("down", 128, 14336, 4096, 1, TID_X + 1, 0.005, 50.0))),
+    # the DiT block's MLP alone (3584 tokens): up 3072 -> 12288, down 12288 -> 3072; run as
+    # a chain, the down layer's input is the up layer's output
+    "dit_mlp": Workload("dit_mlp", ROT_HADAMARD32, (
+        Linear("mlp_up", 3584, 3072, 12288, 1, TID_X, 0.01, 30.0),
+        Linear("mlp_down", 3584, 12288, 3072, 2, TID_X + 1, 0.01, 30.0))),
     "kron": Workload("kron", ROT_KRON_4x8, (
         Linear("kron", 3584, 3072, 3072, 0, TID_X, 0.01, 30.0),)),
     "dit_b16": Workload("dit_b16", ROT_HADAMARD32, (
