@@ -22,7 +22,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _SO = os.path.join(_HERE, "_oracle.so")
 _lib = None
 
-ROT_NONE, ROT_HADAMARD32, ROT_KRON_4x8 = 0, 1, 2
+ROT_NONE, ROT_HADAMARD32, ROT_KRON_4x8, ROT_HADAMARD64, ROT_HADAMARD128 = 0, 1, 2, 3, 4
 
 
 def build(force: bool = False) -> str:
@@ -55,6 +55,9 @@ def _load():
             "oracle_rotate_blocks": ([vp, i64, i32, vp, vp, vp], None),
             "oracle_quantize_blocks": ([vp, i64, vp, vp], None),
             "oracle_rotate_quantize": ([vp, i32, i64, i64, i64, i32, vp, vp, vp, vp], None),
+            "oracle_fwht_unnormalised": ([vp, i32, vp], None),
+            "oracle_hadamard_n": ([vp, i32, vp], None),
+            "oracle_rotation_span": ([i32], i32),
             "oracle_dequantize": ([vp, vp, i64, i64, vp], None),
             "oracle_gemm_pairs": ([vp, vp, vp, vp, i64, vp, vp, i64, vp, vp], None),
             "oracle_gemm": ([vp, vp, vp, vp, i64, i64, i64, vp, vp], None),
@@ -150,13 +153,40 @@ def rotate_blocks(x: np.ndarray, mode: int, A=None, B=None) -> np.ndarray:
 
 # ---------------------------------------------------------------- matrices
 
+def rotation_span(mode: int) -> int:
+    """Elements per rotation group: 32, or 64 / 128 for the larger Hadamard modes."""
+    return _load().oracle_rotation_span(int(mode))
+
+
+def fwht_unnormalised(x: np.ndarray) -> np.ndarray:
+    """Unnormalised fp32 Walsh-Hadamard butterfly over the last axis (n = 32, 64 or 128)."""
+    x = _c(x, np.float32)
+    n = x.shape[-1]
+    flat = x.reshape(-1, n)
+    out = np.empty_like(flat)
+    for i in range(flat.shape[0]):
+        _load().oracle_fwht_unnormalised(_p(flat[i]), n, _p(out[i]))
+    return out.reshape(x.shape)
+
+
+def hadamard_n(x: np.ndarray) -> np.ndarray:
+    """Normalised Sylvester Hadamard H_n (n = 32, 64 or 128) of every row, in fp32."""
+    x = _c(x, np.float32)
+    n = x.shape[-1]
+    flat = x.reshape(-1, n)
+    out = np.empty_like(flat)
+    for i in range(flat.shape[0]):
+        _load().oracle_hadamard_n(_p(flat[i]), n, _p(out[i]))
+    return out.reshape(x.shape)
+
+
 def rotate_quantize(x: np.ndarray, mode: int, A=None, B=None, bf16: bool | None = None):
     """x[rows, K] (uint16 bf16 bits or float32) -> (q[rows, K/2], s[rows, K/32]) logical layout."""
     if bf16 is None:
         bf16 = x.dtype == np.uint16
     x = _c(x, np.uint16 if bf16 else np.float32)
     rows, K = x.shape
-    assert K % 32 == 0
+    assert K % rotation_span(mode) == 0
     A = _c(A if A is not None else np.eye(4), np.float32)
     B = _c(B if B is not None else np.eye(8), np.float32)
     q = np.empty((rows, K // 2), dtype=np.uint8)

@@ -172,6 +172,33 @@ void oracle_hadamard32(const float* x, float* y) {
   for (int i = 0; i < 32; ++i) y[i] = y[i] * INV_SQRT32;
 }
 
+/* Larger rotation blocks (n = 64 or 128 elements, i.e. 2 or 4 MX blocks), the contrast
+ * "KroQuant..." ("Hintergrund") draws with block-wise Hadamard of larger blocks: Sylvester
+ * H_n = H2^(x log2 n) / sqrt(n), butterfly strides 1, 2, ..., n/2 in fp32, then one
+ * multiply by the fp32 nearest 1/sqrt(n). The scales stay per 32 elements. */
+static const float INV_SQRT64 = 0.125f;          /* exact */
+static const float INV_SQRT128 = 0x1.6a09e6p-4f; /* = fp32(1/sqrt(32)) / 2, exact halving */
+
+void oracle_fwht_unnormalised(const float* x, int n, float* v) {
+  for (int i = 0; i < n; ++i) v[i] = x[i];
+  for (int h = 1; h < n; h <<= 1)
+    for (int i = 0; i < n; ++i) {
+      if (i & h) continue;
+      float a = v[i], b = v[i + h];
+      v[i] = a + b;
+      v[i + h] = a - b;
+    }
+}
+
+void oracle_hadamard_n(const float* x, int n, float* y) {
+  const float c = n == 32 ? INV_SQRT32 : n == 64 ? INV_SQRT64 : INV_SQRT128;
+  oracle_fwht_unnormalised(x, n, y);
+  for (int i = 0; i < n; ++i) y[i] = y[i] * c;
+}
+
+/* Elements per rotation group of a mode: 32, or 64 / 128 for modes 3 / 4. */
+int oracle_rotation_span(int mode) { return mode == 3 ? 64 : mode == 4 ? 128 : 32; }
+
 /* y = (A (x) B) x for one 32-block; A 4x4, B 8x8 row-major fp32. */
 void oracle_kron32(const float* A, const float* B, const float* x, float* y) {
   float z[32];
@@ -218,20 +245,25 @@ static float bf16_to_f32(uint16_t b) {
  */
 void oracle_rotate_quantize(const void* x, int xdt, int64_t rows, int64_t K, int64_t ldx, int mode,
                             const float* A, const float* B, uint8_t* q, uint8_t* s) {
-  int64_t nb = K / 32;
+  const int64_t nb = K / 32;
+  const int span = oracle_rotation_span(mode); /* K % span == 0 */
 #pragma omp parallel for schedule(static)
   for (int64_t r = 0; r < rows; ++r) {
-    float xin[32], y[32];
+    float xin[128], y[128];
     uint8_t codes[32];
-    for (int64_t b = 0; b < nb; ++b) {
-      for (int i = 0; i < 32; ++i) {
-        int64_t idx = r * ldx + 32 * b + i;
+    for (int64_t g = 0; g < K / span; ++g) {
+      for (int i = 0; i < span; ++i) {
+        int64_t idx = r * ldx + (int64_t)span * g + i;
         xin[i] = xdt == 0 ? bf16_to_f32(((const uint16_t*)x)[idx]) : ((const float*)x)[idx];
       }
-      oracle_rotate_blocks(xin, 1, mode, A, B, y);
-      oracle_quantize_block(y, codes, s + r * nb + b);
-      for (int j = 0; j < 16; ++j)
-        q[r * (K / 2) + 16 * b + j] = (uint8_t)(codes[2 * j] | (codes[2 * j + 1] << 4));
+      if (mode == 3 || mode == 4) oracle_hadamard_n(xin, span, y);
+      else oracle_rotate_blocks(xin, 1, mode, A, B, y);
+      for (int c = 0; c < span / 32; ++c) {
+        const int64_t b = (int64_t)(span / 32) * g + c;
+        oracle_quantize_block(y + 32 * c, codes, s + r * nb + b);
+        for (int j = 0; j < 16; ++j)
+          q[r * (K / 2) + 16 * b + j] = (uint8_t)(codes[2 * j] | (codes[2 * j + 1] << 4));
+      }
     }
   }
 }

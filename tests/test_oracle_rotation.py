@@ -9,6 +9,7 @@ import math
 from decimal import Decimal, getcontext
 
 import numpy as np
+import pytest
 
 import oracle
 import synth
@@ -150,3 +151,57 @@ def test_quantize_output_rounds_the_sum_once():
     q, s = oracle.quantize_output(y, b, oracle.ROT_NONE)
     q2, s2 = oracle.rotate_quantize(yb, oracle.ROT_NONE, bf16=False)
     assert np.array_equal(q, q2) and np.array_equal(s, s2)
+
+
+# ---- larger Hadamard blocks (n = 64, 128 elements = 2, 4 MX blocks)
+
+@pytest.mark.parametrize("n", [64, 128])
+def test_larger_butterfly_is_sylvester_integer_exact(n):
+    H = _sylvester(n)
+    cols = oracle.fwht_unnormalised(np.eye(n, dtype=np.float32)).T  # column j = H e_j
+    assert np.array_equal(cols, H)
+    assert np.array_equal(cols @ cols.T, n * np.eye(n))
+
+
+def test_larger_normalisers_are_nearest_fp32():
+    getcontext().prec = 60
+    for n in (64, 128):
+        e = np.zeros((1, n), np.float32)
+        e[0, 0] = 1.0
+        c = oracle.hadamard_n(e)[0, 0]  # (H_n e_0)_0 = the normaliser itself
+        exact = Decimal(1) / Decimal(n).sqrt()
+        for nb in (np.nextafter(c, np.float32(0)), np.nextafter(c, np.float32(1))):
+            assert abs(Decimal(float(c)) - exact) <= abs(Decimal(float(nb)) - exact)
+    assert oracle.hadamard_n(np.eye(64, dtype=np.float32)[:1])[0, 0] == np.float32(0.125)
+
+
+@pytest.mark.parametrize("n", [64, 128])
+def test_larger_hadamard_matches_explicit_matrix_and_is_an_involution(n):
+    H = _sylvester(n) / math.sqrt(n)
+    x = synth.normal_f32(1, 998, (100, n))
+    x[:, 5] *= 40.0
+    y = oracle.hadamard_n(x).astype(np.float64)
+    ref = x.astype(np.float64) @ H.T
+    stages = int(math.log2(n))
+    bound = (stages + 3) * 2.0 ** -24 * (np.abs(x).astype(np.float64).sum(axis=1, keepdims=True)
+                                         / math.sqrt(n))
+    assert np.all(np.abs(y - ref) <= bound + 1e-30)
+    yy = oracle.hadamard_n(y.astype(np.float32)).astype(np.float64)
+    assert np.max(np.abs(yy - x) / np.abs(x).max(axis=1, keepdims=True)) < 2e-5
+
+
+@pytest.mark.parametrize("mode,n", [(oracle.ROT_HADAMARD64, 64), (oracle.ROT_HADAMARD128, 128)])
+def test_larger_block_modes_rotate_groups_then_quantise_per_32(mode, n):
+    xb, _ = synth.activation_bf16(2, 6, 512, 0.02, 20.0)
+    x32 = synth.bf16_bits_to_f32(xb)
+    q, s = oracle.rotate_quantize(xb, mode)
+    y = oracle.hadamard_n(x32.reshape(-1, n)).reshape(-1, 32)
+    codes, sc = oracle.quantize_blocks(y)
+    assert np.array_equal(oracle.unpack_codes(q).reshape(-1, 32), codes)
+    assert np.array_equal(s.reshape(-1), sc)
+    # weights rotated the same way: the layer's dot products are preserved (H_n orthonormal)
+    w = synth.weight_f32(2, 4, 512, 3)
+    yw = oracle.hadamard_n(w.reshape(-1, n)).reshape(4, 512).astype(np.float64)
+    ref = x32.astype(np.float64) @ w.astype(np.float64).T
+    got = oracle.hadamard_n(x32.reshape(-1, n)).reshape(6, 512).astype(np.float64) @ yw.T
+    assert np.max(np.abs(got - ref)) < 1e-4 * np.abs(ref).max()
