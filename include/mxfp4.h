@@ -77,7 +77,9 @@ typedef enum {
 typedef enum {
   MXFP4_ROT_NONE = 0,       /* plain MXFP4 quantisation */
   MXFP4_ROT_HADAMARD32 = 1, /* y = H32 x, H32 = H2^(x5) / sqrt(32) (Sylvester order) */
-  MXFP4_ROT_KRON_4x8 = 2    /* y = (A (x) B) x, A 4x4, B 8x8 */
+  MXFP4_ROT_KRON_4x8 = 2,   /* y = (A (x) B) x, A 4x4, B 8x8 */
+  MXFP4_ROT_HADAMARD64 = 3, /* y = H64 x over 64-element groups (2 blocks), K % 64 == 0 */
+  MXFP4_ROT_HADAMARD128 = 4 /* y = H128 x over 128-element groups (4 blocks), K % 128 == 0 */
 } mxfp4_rotation;
 
 typedef enum { MXFP4_DT_BF16 = 0, MXFP4_DT_F32 = 1 } mxfp4_dtype;
@@ -132,6 +134,13 @@ mxfp4_status mxfp4_quantize(const void* x, mxfp4_dtype xdt, int64_t rows, int64_
  * prepare weights for the Kronecker mode pass A^-T and B^-T here
  * (T^-T = A^-T (x) B^-T, "KroQuant...", "Hintergrund": the inverse goes on
  * the weights).
+ * Larger Hadamard blocks (modes HADAMARD64 / HADAMARD128; "KroQuant...",
+ * "Hintergrund", on the cost of larger Hadamard blocks): each 64- or
+ * 128-element group of a row is rotated by the butterfly with strides 1, 2,
+ * ..., n/2 and one multiply by the fp32 nearest 1/sqrt(n) (1/8, and half of
+ * the 1/sqrt(32) constant); the scales stay per 32 elements. K must be a
+ * multiple of the group; weights take the same mode (H_n is symmetric and
+ * orthonormal). These two modes have no bounded waits.
  */
 mxfp4_status mxfp4_rotate_quantize(const void* x, mxfp4_dtype xdt, int64_t rows, int64_t K,
                                    int64_t ldx, mxfp4_rotation mode, const float* kron_a,

@@ -20,7 +20,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libmxfp4.so")
 
 OK, ERR_INVALID_ARG, ERR_SHAPE, ERR_ALIGN, ERR_WORKSPACE, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT = range(8)
-ROT_NONE, ROT_HADAMARD32, ROT_KRON_4x8 = 0, 1, 2
+ROT_NONE, ROT_HADAMARD32, ROT_KRON_4x8, ROT_HADAMARD64, ROT_HADAMARD128 = 0, 1, 2, 3, 4
 DT_BF16, DT_F32 = 0, 1
 OP_QUANTIZE, OP_GEMM, OP_LINEAR = 0, 1, 2
 

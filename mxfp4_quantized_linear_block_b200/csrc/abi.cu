@@ -56,6 +56,8 @@ mxfp4_status validate_gemm(const uint8_t* aq, const uint8_t* asf, const uint8_t*
   return MXFP4_OK;
 }
 
+bool mode_ok(int mode) { return mode >= MXFP4_ROT_NONE && mode <= MXFP4_ROT_HADAMARD128; }
+
 bool kron_from_host(const float* a, const float* b, KronCoeffs* out) {
   if (!a || !b) return false;
   std::memcpy(out->a, a, sizeof(out->a));
@@ -135,8 +137,8 @@ mxfp4_status mxfp4_rotate_quantize(const void* x, mxfp4_dtype xdt, int64_t rows,
                                    mxfp4_stream_t stream) {
   mxfp4_status st = validate_quantize(x, xdt, rows, K, ldx, q, sf);
   if (st != MXFP4_OK) return st;
-  if (mode != MXFP4_ROT_NONE && mode != MXFP4_ROT_HADAMARD32 && mode != MXFP4_ROT_KRON_4x8)
-    return MXFP4_ERR_UNSUPPORTED;
+  if (!mode_ok(mode)) return MXFP4_ERR_UNSUPPORTED;
+  if (K % rotation_span(mode) != 0) return MXFP4_ERR_SHAPE;
   KronCoeffs kc{};
   if (mode == MXFP4_ROT_KRON_4x8 && !kron_from_host(kron_a, kron_b, &kc))
     return MXFP4_ERR_INVALID_ARG;
@@ -187,6 +189,7 @@ mxfp4_status mxfp4_gemm_quantize(const uint8_t* aq, const uint8_t* asf, const ui
                                  const float* kron_b, uint8_t* yq, uint8_t* ysf, void* ws,
                                  size_t ws_bytes, mxfp4_stream_t stream) {
   if (!aq || !asf || !bq || !bsf || !yq || !ysf || !ws) return MXFP4_ERR_INVALID_ARG;
+  // the epilogue rotates within one 32-column block: no larger Hadamard groups here
   if (mode != MXFP4_ROT_NONE && mode != MXFP4_ROT_HADAMARD32 && mode != MXFP4_ROT_KRON_4x8)
     return MXFP4_ERR_UNSUPPORTED;
   if (!shape_ok(M, K) || N < 32 || N % 32 != 0 || !within_limits(M, K) || !within_limits(N, K) ||
@@ -214,9 +217,9 @@ mxfp4_status mxfp4_linear(const void* x, int64_t M, int64_t K, mxfp4_rotation mo
                           const uint8_t* wsf, int64_t N, void* y, void* ws, size_t ws_bytes,
                           mxfp4_stream_t stream) {
   if (!x || !wq || !wsf || !y || !ws) return MXFP4_ERR_INVALID_ARG;
-  if (mode != MXFP4_ROT_NONE && mode != MXFP4_ROT_HADAMARD32 && mode != MXFP4_ROT_KRON_4x8)
-    return MXFP4_ERR_UNSUPPORTED;
-  if (!shape_ok(M, K) || N < 16 || N % 16 != 0 || !within_limits(M, K) || !within_limits(N, K))
+  if (!mode_ok(mode)) return MXFP4_ERR_UNSUPPORTED;
+  if (!shape_ok(M, K) || K % rotation_span(mode) != 0 || N < 16 || N % 16 != 0 ||
+      !within_limits(M, K) || !within_limits(N, K))
     return MXFP4_ERR_SHAPE;
   if (!aligned16(x) || !aligned16(wq) || !aligned16(wsf) || !aligned16(y) || !aligned16(ws) ||
       (K * 2) % 16 != 0 || (N * 2) % 16 != 0)

@@ -20,6 +20,14 @@ cudaError_t launch_rotate_quantize(const void* x, bool x_is_f32, int64_t rows, i
                                    int64_t ldx, int mode, const KronCoeffs* kc, uint8_t* q,
                                    uint8_t* sf, int* status, cudaStream_t stream);
 
+// Rotation over 64- or 128-element groups (span) + quantisation (quantize_wide.cu).
+cudaError_t launch_rotate_quantize_wide(const void* x, bool x_is_f32, int64_t rows, int64_t K,
+                                        int64_t ldx, int span, uint8_t* q, uint8_t* sf,
+                                        cudaStream_t stream);
+
+// Elements per rotation group of a mode (0, 1, 2: 32; 3: 64; 4: 128).
+inline int64_t rotation_span(int mode) { return mode == 3 ? 64 : mode == 4 ? 128 : 32; }
+
 // What the GEMM epilogue writes.
 enum OutKind { kOutBf16 = 0, kOutF32 = 1, kOutMxfp4 = 2 };
 struct Epilogue {

@@ -64,9 +64,9 @@ extern "C" mxfp4_status mxfp4_linear_noalloc(const void* x, int64_t M, int64_t K
                                               mxfp4_stream_t stream) {
   using namespace mxfp4;
   if (!x || !wq || !wsf || !y) return MXFP4_ERR_INVALID_ARG;
-  if (mode != MXFP4_ROT_NONE && mode != MXFP4_ROT_HADAMARD32 && mode != MXFP4_ROT_KRON_4x8)
-    return MXFP4_ERR_UNSUPPORTED;
-  if (M < 0 || K < 32 || K % 32 != 0 || N < 16 || N % 16 != 0 || M >= (1ll << 31) ||
+  if (mode < MXFP4_ROT_NONE || mode > MXFP4_ROT_HADAMARD128) return MXFP4_ERR_UNSUPPORTED;
+  if (M < 0 || K < 32 || K % rotation_span(mode) != 0 || N < 16 || N % 16 != 0 ||
+      M >= (1ll << 31) ||
       K >= (1ll << 31) || N >= (1ll << 31))
     return MXFP4_ERR_SHAPE;
   if (!aligned16(x) || !aligned16(wq) || !aligned16(wsf) || !aligned16(y) ||

@@ -241,6 +241,9 @@ cudaError_t launch_mode(const void* x, int64_t rows, int64_t K, int64_t ldx, con
 cudaError_t launch_rotate_quantize(const void* x, bool x_is_f32, int64_t rows, int64_t K,
                                    int64_t ldx, int mode, const KronCoeffs* kc, uint8_t* q,
                                    uint8_t* sf, int* status, cudaStream_t stream) {
+  if (mode == 3 || mode == 4)
+    return launch_rotate_quantize_wide(x, x_is_f32, rows, K, ldx, (int)rotation_span(mode), q, sf,
+                                       stream);
   KronCoeffs k{};
   if (kc) k = *kc;
   if (x_is_f32) {

@@ -86,3 +86,22 @@ def test_status_word_clear_after_runs():
               wl.rotation, ws=wsp)
     torch.cuda.synchronize()
     assert mx.poll_status(wsp) == mx.OK
+
+
+@pytest.mark.parametrize("mode", [oracle.ROT_HADAMARD64, oracle.ROT_HADAMARD128])
+@pytest.mark.parametrize("M", [16, 300])
+def test_linear_wide_hadamard(mode, M):
+    """The layer with a larger rotation group: weights rotated by the same H_n on the GPU
+    (fp32 input), activations online; compared with the oracle's layer."""
+    import torch
+    import mxfp4_quantized_linear_block_b200 as mx
+    K, N = 1024, 768
+    x, _ = synth.activation_bf16(M, M, K, 0.01, 30.0)
+    w = synth.weight_f32(2, N, K, 5)
+    wq_d, wsf_d = mx.rotate_quantize(torch.from_numpy(w).cuda(), mode)
+    y = mx.linear(to_dev_bf16(x), wq_d, wsf_d, N, mode)
+    torch.cuda.synchronize()
+    wq, ws = oracle.prepare_weight(w, mode)
+    assert np.array_equal(wq_d.cpu().numpy(), wq)
+    ref, S, _, _ = oracle.linear(x, wq, ws, mode)
+    check_gemm_values(bf16_dev_to_f64(y), ref, S, "bf16", f"H{oracle.rotation_span(mode)} M{M}")

@@ -129,3 +129,53 @@ def test_weight_preparation(mode):
     if mode != oracle.ROT_KRON_4x8:
         eq, es = oracle.prepare_weight(w, mode)
         assert np.array_equal(q, eq) and np.array_equal(s, es)
+
+
+# ---- larger Hadamard blocks: 64- and 128-element rotation groups, scales per 32
+
+WIDE = [oracle.ROT_HADAMARD64, oracle.ROT_HADAMARD128]
+
+
+def _rows_of(x: np.ndarray, span: int) -> np.ndarray:
+    """Adversarial 32-blocks regrouped into rows of `span` elements (zero blocks appended)."""
+    per = span // 32
+    n = -(-x.shape[0] // per) * per
+    pad = np.zeros((n - x.shape[0], 32), x.dtype)
+    return np.concatenate([x, pad]).reshape(-1, span)
+
+
+@pytest.mark.parametrize("mode", WIDE)
+def test_wide_adversarial_fp32_and_bf16(mode):
+    span = oracle.rotation_span(mode)
+    x = _rows_of(_adversarial_f32(), span)
+    x = np.concatenate([x, x[::-1], -x], axis=1)  # 3 groups per row
+    quantize_parity(x, mode)
+    quantize_parity(synth.f32_to_bf16_bits(x), mode)
+
+
+@pytest.mark.parametrize("mode", WIDE)
+@pytest.mark.parametrize("rows", [1, 127, 129, 300])
+@pytest.mark.parametrize("groups", [1, 3, 8])
+def test_wide_ragged_shapes(mode, rows, groups):
+    K = oracle.rotation_span(mode) * groups
+    x, _ = synth.activation_bf16(rows + K, rows, K, 0.02, 20.0)
+    quantize_parity(x, mode)
+
+
+@pytest.mark.parametrize("mode", WIDE)
+def test_wide_strided_rows_and_weights(mode):
+    x, _ = synth.activation_bf16(4, 200, 1024, 0.02, 20.0)
+    quantize_parity(x, mode, ld_pad=64)
+    w = synth.weight_f32(1, 256, 3072)
+    q, s = quantize_parity(w, mode, ld_pad=32)
+    eq, es = oracle.prepare_weight(w, mode)
+    assert np.array_equal(q, eq) and np.array_equal(s, es)
+
+
+@pytest.mark.parametrize("mode", WIDE)
+def test_wide_mode_rejects_k_not_a_multiple_of_the_group(mode):
+    import torch
+    import mxfp4_quantized_linear_block_b200 as mx
+    x = torch.zeros((4, 96), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(mx.MXFP4Error):
+        mx.rotate_quantize(x, mode)
