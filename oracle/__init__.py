@@ -58,6 +58,13 @@ def _load():
             "oracle_fwht_unnormalised": ([vp, i32, vp], None),
             "oracle_hadamard_n": ([vp, i32, vp], None),
             "oracle_rotation_span": ([i32], i32),
+            "oracle_e4m3_value": ([i32], dbl),
+            "oracle_e4m3_code": ([dbl], i32),
+            "oracle_nvfp4_quantize_group": ([vp, ctypes.c_float, vp, vp], None),
+            "oracle_nvfp4_tensor_scale": ([vp, i32, i64, i64, i64, i32], ctypes.c_float),
+            "oracle_nvfp4_rotate_quantize": ([vp, i32, i64, i64, i64, i32, ctypes.c_float, vp,
+                                              vp], None),
+            "oracle_nvfp4_gemm": ([vp, vp, vp, vp, i64, i64, i64, dbl, vp, vp], None),
             "oracle_dequantize": ([vp, vp, i64, i64, vp], None),
             "oracle_gemm_pairs": ([vp, vp, vp, vp, i64, vp, vp, i64, vp, vp], None),
             "oracle_gemm": ([vp, vp, vp, vp, i64, i64, i64, vp, vp], None),
@@ -254,6 +261,83 @@ def prepare_weight(w_f32: np.ndarray, mode: int, A=None, B=None):
         At, Bt = kron_weight_factors(A, B)
         return rotate_quantize(w_f32, mode, At, Bt, bf16=False)
     return rotate_quantize(w_f32, mode, None, None, bf16=False)
+
+
+# ---------------------------------------------------------------- NVFP4
+
+def e4m3_value(byte: int) -> float:
+    """Unsigned E4M3 group-scale byte (0..126) -> value."""
+    return _load().oracle_e4m3_value(int(byte))
+
+
+def e4m3_code(v: float) -> int:
+    """Nearest finite E4M3 code to v >= 0 (ties to even, above 448 -> 448)."""
+    return _load().oracle_e4m3_code(float(v))
+
+
+def nvfp4_quantize_group(y: np.ndarray, st: float):
+    """16 fp32 values, fp32 tensor scale -> (16 unpacked codes, E4M3 group byte)."""
+    y = _c(y, np.float32)
+    assert y.shape == (16,)
+    codes = np.empty(16, np.uint8)
+    sb = np.empty(1, np.uint8)
+    _load().oracle_nvfp4_quantize_group(_p(y), float(np.float32(st)), _p(codes), _p(sb))
+    return codes, int(sb[0])
+
+
+def nvfp4_tensor_scale(x: np.ndarray, mode: int, bf16: bool | None = None) -> np.float32:
+    """amax of x rotated by mode (0 or 1) / (6 * 448), fp32."""
+    if bf16 is None:
+        bf16 = x.dtype == np.uint16
+    x = _c(x, np.uint16 if bf16 else np.float32)
+    rows, K = x.shape
+    return np.float32(_load().oracle_nvfp4_tensor_scale(_p(x), 0 if bf16 else 1, rows, K, K,
+                                                        int(mode)))
+
+
+def nvfp4_rotate_quantize(x: np.ndarray, mode: int, st, bf16: bool | None = None):
+    """x[rows, K] -> (q[rows, K/2] packed codes, s[rows, K/16] E4M3 group bytes)."""
+    if bf16 is None:
+        bf16 = x.dtype == np.uint16
+    x = _c(x, np.uint16 if bf16 else np.float32)
+    rows, K = x.shape
+    assert K % 32 == 0 and mode in (ROT_NONE, ROT_HADAMARD32)
+    q = np.empty((rows, K // 2), np.uint8)
+    s = np.empty((rows, K // 16), np.uint8)
+    _load().oracle_nvfp4_rotate_quantize(_p(x), 0 if bf16 else 1, rows, K, K, int(mode),
+                                         float(np.float32(st)), _p(q), _p(s))
+    return q, s
+
+
+def nvfp4_gemm(aq, as_, bq, bs, alpha: float):
+    """Exact NVFP4 product times alpha (the product of the two tensor scales) -> (ref, S)."""
+    aq, as_, bq, bs = (_c(a, np.uint8) for a in (aq, as_, bq, bs))
+    M, N, K = aq.shape[0], bq.shape[0], aq.shape[1] * 2
+    ref = np.empty((M, N), np.float64)
+    S = np.empty((M, N), np.float64)
+    _load().oracle_nvfp4_gemm(_p(aq), _p(as_), _p(bq), _p(bs), M, N, K, float(alpha), _p(ref),
+                              _p(S))
+    return ref, S
+
+
+def nvfp4_dequantize(q: np.ndarray, s: np.ndarray, st) -> np.ndarray:
+    """NVFP4 matrix back to double: code value * E4M3(group byte) * st."""
+    codes = unpack_codes(q).astype(np.int64)
+    mag = np.array([0, 0.5, 1, 1.5, 2, 3, 4, 6], np.float64)[codes & 7]
+    val = np.where(codes & 8, -mag, mag)
+    sc = np.vectorize(e4m3_value)(s.astype(np.int64))
+    return val * np.repeat(sc, 16, axis=1) * float(st)
+
+
+def nvfp4_sf_to_physical(s: np.ndarray, K: int) -> np.ndarray:
+    """Logical [rows, K/16] E4M3 bytes -> the tensor-core layout: the same 512-byte atoms
+    as the MXFP4 scales with 16-element groups in place of 32-element blocks (so the map
+    of an operand with 2K elements per row)."""
+    return sf_to_physical(s, 2 * K)
+
+
+def nvfp4_sf_bytes(rows: int, K: int) -> int:
+    return sf_bytes(rows, 2 * K)
 
 
 # ---------------------------------------------------------------- helpers

@@ -426,3 +426,132 @@ void oracle_sf_from_physical(const uint8_t* phys, int64_t rows, int64_t K, uint8
   for (int64_t r = 0; r < rows; ++r)
     for (int64_t b = 0; b < K / 32; ++b) s[r * (K / 32) + b] = phys[oracle_sf_offset(r, b, K)];
 }
+
+/* ------------------------------------------------------------------ NVFP4
+ *
+ * The other FP4 format the pages compare ("Bridging the Gap Between Promise and
+ * Performance for Microscaling FP4 Quantization", "Probleemstelling" item 1 and
+ * "Format-specifieke Schaaloptimalisatie"): E2M1 elements in groups of 16, each group
+ * with its own scale, plus one scale for the whole tensor. Read as NVIDIA's NVFP4: the
+ * group scale is an unsigned E4M3 byte (4 exponent bits, bias 7, 3 mantissa bits, no
+ * infinities; finite codes 0..126, largest 448), the tensor scale an fp32 number.
+ */
+double oracle_e4m3_value(int b) {
+  int e = (b >> 3) & 15, m = b & 7;
+  if (e == 0) return ldexp((double)m, -9); /* subnormal: m/8 * 2^(1-7) */
+  return ldexp(1.0 + m / 8.0, e - 7);
+}
+
+/* Nearest finite E4M3 code to v >= 0, ties to the even code, above 448 -> 448. */
+int oracle_e4m3_code(double v) {
+  int best = 0;
+  double bd = fabs(v - oracle_e4m3_value(0));
+  for (int c = 1; c <= 126; ++c) {
+    double d = fabs(v - oracle_e4m3_value(c));
+    if (d < bd || (d == bd && (c & 1) == 0 && (best & 1) == 1)) {
+      best = c;
+      bd = d;
+    }
+  }
+  return best;
+}
+
+/* One group of 16 fp32 values with tensor scale st (> 0, or 0 for an all-zero tensor):
+ * g = amax / (6 st) in two fp32 roundings, group byte = nearest E4M3 of g, element scale
+ * S = E4M3(byte) * st (one fp32 rounding), r = 1 / S (one rounding), code_i = nearest
+ * E2M1 of y_i * r (one rounding; ties to even, saturating at 6, sign kept). */
+void oracle_nvfp4_quantize_group(const float* y, float st, uint8_t* codes, uint8_t* sbyte) {
+  float amax = 0.0f;
+  for (int i = 0; i < 16; ++i) {
+    float a = fabsf(y[i]);
+    if (a > amax) amax = a;
+  }
+  if (!(st > 0.0f)) {
+    *sbyte = 0;
+    memset(codes, 0, 16);
+    return;
+  }
+  float den = 6.0f * st;
+  float g = amax / den;
+  int sb = oracle_e4m3_code((double)g);
+  *sbyte = (uint8_t)sb;
+  float S = (float)oracle_e4m3_value(sb) * st;
+  if (S == 0.0f) {
+    memset(codes, 0, 16);
+    return;
+  }
+  float r = 1.0f / S;
+  for (int i = 0; i < 16; ++i) {
+    float v = y[i] * r;
+    codes[i] = (uint8_t)oracle_e2m1_code((double)v);
+  }
+}
+
+static void load_block(const void* x, int xdt, int64_t idx, float* out) {
+  for (int i = 0; i < 32; ++i)
+    out[i] = xdt == 0 ? bf16_to_f32(((const uint16_t*)x)[idx + i]) : ((const float*)x)[idx + i];
+}
+
+/* Tensor scale of x rotated by mode (0 none, 1 Hadamard-32): amax / (6 * 448), one
+ * fp32 rounding; 0 for an all-zero tensor. K % 32 == 0. */
+float oracle_nvfp4_tensor_scale(const void* x, int xdt, int64_t rows, int64_t K, int64_t ldx,
+                                int mode) {
+  float amax = 0.0f;
+  for (int64_t r = 0; r < rows; ++r)
+    for (int64_t b = 0; b < K / 32; ++b) {
+      float xin[32], y[32];
+      load_block(x, xdt, r * ldx + 32 * b, xin);
+      if (mode == 1) oracle_hadamard32(xin, y);
+      else memcpy(y, xin, sizeof(y));
+      for (int i = 0; i < 32; ++i)
+        if (fabsf(y[i]) > amax) amax = fabsf(y[i]);
+    }
+  return amax / 2688.0f;
+}
+
+/* Rotate (mode 0 / 1) and quantise x[rows, K] to NVFP4 with tensor scale st: q[rows, K/2]
+ * packed codes (element 2j low nibble of byte j), s[rows, K/16] E4M3 group bytes. */
+void oracle_nvfp4_rotate_quantize(const void* x, int xdt, int64_t rows, int64_t K, int64_t ldx,
+                                  int mode, float st, uint8_t* q, uint8_t* s) {
+#pragma omp parallel for schedule(static)
+  for (int64_t r = 0; r < rows; ++r) {
+    for (int64_t b = 0; b < K / 32; ++b) {
+      float xin[32], y[32];
+      uint8_t codes[32];
+      load_block(x, xdt, r * ldx + 32 * b, xin);
+      if (mode == 1) oracle_hadamard32(xin, y);
+      else memcpy(y, xin, sizeof(y));
+      oracle_nvfp4_quantize_group(y, st, codes, s + r * (K / 16) + 2 * b);
+      oracle_nvfp4_quantize_group(y + 16, st, codes + 16, s + r * (K / 16) + 2 * b + 1);
+      for (int j = 0; j < 16; ++j)
+        q[r * (K / 2) + 16 * b + j] = (uint8_t)(codes[2 * j] | (codes[2 * j + 1] << 4));
+    }
+  }
+}
+
+/* Exact NVFP4 product: ref[m][n] = alpha * sum_g E4M3(as[m,g]) E4M3(bs[n,g])
+ * sum_{i in g} v(a_i) v(b_i) (per-group integer sums in units of 1/4, then double),
+ * S[m][n] = |alpha| * sum_i |a_i b_i| with the group scales. */
+void oracle_nvfp4_gemm(const uint8_t* aq, const uint8_t* as, const uint8_t* bq,
+                       const uint8_t* bs, int64_t M, int64_t N, int64_t K, double alpha,
+                       double* ref, double* S) {
+  const int64_t ng = K / 16;
+#pragma omp parallel for schedule(static)
+  for (int64_t m = 0; m < M; ++m)
+    for (int64_t n = 0; n < N; ++n) {
+      double acc = 0.0, mag = 0.0;
+      for (int64_t g = 0; g < ng; ++g) {
+        int64_t isum = 0, iabs = 0;
+        for (int64_t i = 16 * g; i < 16 * g + 16; ++i) {
+          int64_t p = (int64_t)e2m1_twice(code_at(aq, K, m, i)) * e2m1_twice(code_at(bq, K, n, i));
+          isum += p;
+          iabs += p < 0 ? -p : p;
+        }
+        const double sc = oracle_e4m3_value(as[m * ng + g]) * oracle_e4m3_value(bs[n * ng + g]);
+        acc += (double)isum * 0.25 * sc;
+        mag += (double)iabs * 0.25 * sc;
+      }
+      ref[m * N + n] = alpha * acc;
+      S[m * N + n] = fabs(alpha) * mag;
+    }
+}
