@@ -84,7 +84,12 @@ typedef enum {
 
 typedef enum { MXFP4_DT_BF16 = 0, MXFP4_DT_F32 = 1 } mxfp4_dtype;
 
-typedef enum { MXFP4_OP_QUANTIZE = 0, MXFP4_OP_GEMM = 1, MXFP4_OP_LINEAR = 2 } mxfp4_op;
+typedef enum {
+  MXFP4_OP_QUANTIZE = 0,
+  MXFP4_OP_GEMM = 1, /* also mxfp4_gemm_bias, mxfp4_gemm_quantize, mxfp4_nvfp4_gemm */
+  MXFP4_OP_LINEAR = 2,
+  MXFP4_OP_NVFP4_LINEAR = 3
+} mxfp4_op;
 
 /* A cudaStream_t, passed as an opaque handle so this header needs no CUDA headers. */
 typedef void* mxfp4_stream_t;
@@ -212,6 +217,57 @@ mxfp4_status mxfp4_linear(const void* x, int64_t M, int64_t K, mxfp4_rotation mo
                           const float* kron_a, const float* kron_b, const uint8_t* wq,
                           const uint8_t* wsf, int64_t N, void* y, void* ws, size_t ws_bytes,
                           mxfp4_stream_t stream);
+
+/*
+ * NVFP4, the other FP4 format the pages compare ("Bridging the Gap Between
+ * Promise and Performance for Microscaling FP4 Quantization", "Probleemstelling"
+ * item 1: 16-element groups; "Format-specifieke Schaaloptimalisatie": tensor and
+ * group scales). Codes are packed E2M1 as above; every 16 elements of a row
+ * share an unsigned E4M3 scale byte (bias 7, 3 mantissa bits, largest 448) and
+ * the tensor has one fp32 scale st. Quantisation of a group of (rotated)
+ * values y: g = amax / (6 st), byte = nearest E4M3 of g (ties to even,
+ * saturating), S = E4M3(byte) * st, code_i = nearest E2M1 of y_i * (1 / S),
+ * each step one fp32 rounding; st = 0 or S = 0 gives byte and codes 0.
+ * Scale bytes use the 512-byte atoms of the MXFP4 layout with 16-element groups
+ * in place of 32-element blocks: mxfp4_nvfp4_sf_bytes(rows, K) =
+ * mxfp4_sf_bytes(rows, 2 K), byte of (row, group g) at mxfp4_sf_offset(row, g,
+ * 2 K). Rotation modes: NONE and HADAMARD32 only. K % 32 == 0.
+ */
+size_t mxfp4_nvfp4_sf_bytes(int64_t rows, int64_t K);
+
+/* Tensor scale st = amax(rotated x) / (6 * 448) (fp32, one rounding) into
+ * scale2[0]; scale2: DEVICE pointer to 2 floats, 8-byte aligned, [1] is scratch.
+ * Stream-ordered (a memset and two small kernels). */
+mxfp4_status mxfp4_nvfp4_tensor_scale(const void* x, mxfp4_dtype xdt, int64_t rows, int64_t K,
+                                      int64_t ldx, mxfp4_rotation mode, float* scale2,
+                                      mxfp4_stream_t stream);
+
+/* Rotate (mode) and quantise x to NVFP4 with the DEVICE fp32 tensor scale
+ * *tensor_scale: q [rows, K/2], sf mxfp4_nvfp4_sf_bytes(rows, K) bytes (padding
+ * 0). Requirements as mxfp4_quantize. Weights: quantise them with their own
+ * tensor scale (mxfp4_nvfp4_tensor_scale on W). */
+mxfp4_status mxfp4_nvfp4_quantize(const void* x, mxfp4_dtype xdt, int64_t rows, int64_t K,
+                                  int64_t ldx, mxfp4_rotation mode, const float* tensor_scale,
+                                  uint8_t* q, uint8_t* sf, mxfp4_stream_t stream);
+
+/* NVFP4 GEMM on the tcgen05 tensor cores (kind::mxf4nvf4, 16-element UE4M3
+ * block scales): y = (*a_scale) (*b_scale) sum_g E4M3(asf) E4M3(bsf) sum v(a) v(b),
+ * fp32 accumulation, the tensor scales applied once in fp32 to the sum.
+ * a_scale / b_scale: DEVICE fp32 tensor scales. Everything else as mxfp4_gemm
+ * (bf16 or fp32 output; workspace mxfp4_workspace_bytes(MXFP4_OP_GEMM, ...)). */
+mxfp4_status mxfp4_nvfp4_gemm(const uint8_t* aq, const uint8_t* asf, const float* a_scale,
+                              const uint8_t* bq, const uint8_t* bsf, const float* b_scale,
+                              int64_t M, int64_t N, int64_t K, void* y, mxfp4_dtype ydt,
+                              int64_t ldy, void* ws, size_t ws_bytes, mxfp4_stream_t stream);
+
+/* The NVFP4 layer: tensor scale of the rotated x, quantise x, GEMM with the
+ * pre-quantised weights (wq / wsf / *w_scale, from mxfp4_nvfp4_quantize with the
+ * same mode), bf16 y [M, N]. ws: mxfp4_workspace_bytes(MXFP4_OP_NVFP4_LINEAR,
+ * M, N, K) bytes, zeroed at allocation (status word as for mxfp4_linear). */
+mxfp4_status mxfp4_nvfp4_linear(const void* x, int64_t M, int64_t K, mxfp4_rotation mode,
+                                const uint8_t* wq, const uint8_t* wsf, const float* w_scale,
+                                int64_t N, void* y, void* ws, size_t ws_bytes,
+                                mxfp4_stream_t stream);
 
 /* Size in bytes of the device scratch array that mxfp4_linear_noalloc uses (per GPU). */
 #define MXFP4_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)

@@ -22,12 +22,14 @@ LIB_PATH = os.path.join(_HERE, "libmxfp4.so")
 OK, ERR_INVALID_ARG, ERR_SHAPE, ERR_ALIGN, ERR_WORKSPACE, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT = range(8)
 ROT_NONE, ROT_HADAMARD32, ROT_KRON_4x8, ROT_HADAMARD64, ROT_HADAMARD128 = 0, 1, 2, 3, 4
 DT_BF16, DT_F32 = 0, 1
-OP_QUANTIZE, OP_GEMM, OP_LINEAR = 0, 1, 2
+OP_QUANTIZE, OP_GEMM, OP_LINEAR, OP_NVFP4_LINEAR = 0, 1, 2, 3
 
 EXPORTS = (
     "mxfp4_sf_bytes", "mxfp4_sf_offset", "mxfp4_workspace_bytes", "mxfp4_status_string",
     "mxfp4_quantize", "mxfp4_rotate_quantize", "mxfp4_gemm", "mxfp4_linear",
     "mxfp4_poll_status", "mxfp4_linear_noalloc", "mxfp4_gemm_bias", "mxfp4_gemm_quantize",
+    "mxfp4_nvfp4_sf_bytes", "mxfp4_nvfp4_tensor_scale", "mxfp4_nvfp4_quantize",
+    "mxfp4_nvfp4_gemm", "mxfp4_nvfp4_linear",
 )
 
 
@@ -41,7 +43,7 @@ def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError(
             f"libmxfp4.so not found at {LIB_PATH}; build it with "
-            "`python -m mxfp4_quantized_linear_block_b200.build` (nvcc, sm_100a)")
+            "`python mxfp4_quantized_linear_block_b200/build.py` (nvcc, sm_100a)")
     lib = ctypes.CDLL(LIB_PATH)
     vp, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
     sig = {
@@ -58,6 +60,12 @@ def _load() -> ctypes.CDLL:
         "mxfp4_gemm_bias": ([vp, vp, vp, vp, i64, i64, i64, vp, vp, i32, i64, vp, sz, vp], i32),
         "mxfp4_gemm_quantize": ([vp, vp, vp, vp, i64, i64, i64, vp, i32, vp, vp, vp, vp, vp, sz,
                                  vp], i32),
+        "mxfp4_nvfp4_sf_bytes": ([i64, i64], sz),
+        "mxfp4_nvfp4_tensor_scale": ([vp, i32, i64, i64, i64, i32, vp, vp], i32),
+        "mxfp4_nvfp4_quantize": ([vp, i32, i64, i64, i64, i32, vp, vp, vp, vp], i32),
+        "mxfp4_nvfp4_gemm": ([vp, vp, vp, vp, vp, vp, i64, i64, i64, vp, i32, i64, vp, sz, vp],
+                             i32),
+        "mxfp4_nvfp4_linear": ([vp, i64, i64, i32, vp, vp, vp, i64, vp, vp, sz, vp], i32),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -213,6 +221,77 @@ def gemm_quantize(aq, asf, bq, bsf, M: int, N: int, K: int, bias=None,
                                  _stream_handle(stream))
     _check(st, "mxfp4_gemm_quantize")
     return yq, ysf
+
+
+# ---------------------------------------------------------------- NVFP4
+
+def nvfp4_sf_bytes(rows: int, K: int) -> int:
+    return lib.mxfp4_nvfp4_sf_bytes(rows, K)
+
+
+def nvfp4_tensor_scale(x, mode: int = ROT_NONE, scale2=None, stream=None):
+    """Device fp32 tensor scale amax(rotated x) / 2688; returns a 2-float CUDA tensor whose
+    element 0 is the scale."""
+    torch = _torch()
+    assert x.dim() == 2 and x.stride(1) == 1
+    rows, K = x.shape
+    if scale2 is None:
+        scale2 = torch.zeros(2, dtype=torch.float32, device=x.device)
+    st = lib.mxfp4_nvfp4_tensor_scale(x.data_ptr(), _dtype_code(x), rows, K, x.stride(0), mode,
+                                      scale2.data_ptr(), _stream_handle(stream))
+    _check(st, "mxfp4_nvfp4_tensor_scale")
+    return scale2
+
+
+def nvfp4_quantize(x, tensor_scale, mode: int = ROT_NONE, q=None, sf=None, stream=None):
+    """x [rows, K] bf16/fp32 -> (q [rows, K/2], sf [nvfp4_sf_bytes]) with the device fp32
+    tensor scale (a CUDA tensor whose first element is the scale)."""
+    torch = _torch()
+    assert x.dim() == 2 and x.stride(1) == 1
+    rows, K = x.shape
+    if q is None:
+        q = torch.empty((rows, K // 2), dtype=torch.uint8, device=x.device)
+    if sf is None:
+        sf = torch.empty(max(nvfp4_sf_bytes(rows, K), 16), dtype=torch.uint8, device=x.device)
+    st = lib.mxfp4_nvfp4_quantize(x.data_ptr(), _dtype_code(x), rows, K, x.stride(0), mode,
+                                  tensor_scale.data_ptr(), q.data_ptr(), sf.data_ptr(),
+                                  _stream_handle(stream))
+    _check(st, "mxfp4_nvfp4_quantize")
+    return q, sf
+
+
+def nvfp4_gemm(aq, asf, a_scale, bq, bsf, b_scale, M: int, N: int, K: int, y=None,
+               out_dtype=None, ws=None, stream=None):
+    """NVFP4 GEMM y = a_scale * b_scale * A . B^T (scales: device fp32 tensors)."""
+    torch = _torch()
+    out_dtype = out_dtype or torch.bfloat16
+    if y is None:
+        y = torch.empty((M, N), dtype=out_dtype, device=aq.device)
+    if ws is None:
+        ws = new_workspace(workspace_bytes(OP_GEMM, M, N, K), aq.device)
+    st = lib.mxfp4_nvfp4_gemm(aq.data_ptr(), asf.data_ptr(), a_scale.data_ptr(), bq.data_ptr(),
+                              bsf.data_ptr(), b_scale.data_ptr(), M, N, K, y.data_ptr(),
+                              _dtype_code(y), y.stride(0), ws.data_ptr(), ws.numel(),
+                              _stream_handle(stream))
+    _check(st, "mxfp4_nvfp4_gemm")
+    return y
+
+
+def nvfp4_linear(x, wq, wsf, w_scale, N: int, mode: int = ROT_NONE, y=None, ws=None,
+                 stream=None):
+    """The NVFP4 layer: tensor scale + quantise x, GEMM with NVFP4 weights (bf16 out)."""
+    torch = _torch()
+    assert x.dim() == 2 and x.is_contiguous() and x.dtype == torch.bfloat16
+    M, K = x.shape
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    if ws is None:
+        ws = new_workspace(workspace_bytes(OP_NVFP4_LINEAR, M, N, K), x.device)
+    st = lib.mxfp4_nvfp4_linear(x.data_ptr(), M, K, mode, wq.data_ptr(), wsf.data_ptr(),
+                                w_scale.data_ptr(), N, y.data_ptr(), ws.data_ptr(), ws.numel(),
+                                _stream_handle(stream))
+    _check(st, "mxfp4_nvfp4_linear")
+    return y
 
 
 def linear(x, wq, wsf, N: int, mode: int = ROT_HADAMARD32, kron_a=None, kron_b=None, y=None,

@@ -71,6 +71,19 @@ struct LinearWorkspace {
   size_t q_off, sf_off, g_off, total;
 };
 
+// Workspace of mxfp4_nvfp4_linear: [status | X tensor scale (2 floats at 64) | Xq | Xsf |
+// GEMM scratch].
+constexpr size_t kScaleOff = 64;
+
+LinearWorkspace nvfp4_linear_workspace(int64_t M, int64_t N, int64_t K) {
+  LinearWorkspace w;
+  w.q_off = kStatusBytes;
+  w.sf_off = round_up(w.q_off + (size_t)M * (size_t)(K / 2), 256);
+  w.g_off = round_up(w.sf_off + mxfp4_sf_bytes(M, 2 * K), 256);
+  w.total = round_up(w.g_off + gemm_scratch_bytes(M, N, K), 256);
+  return w;
+}
+
 LinearWorkspace linear_workspace(int64_t M, int64_t N, int64_t K) {
   LinearWorkspace w;
   w.q_off = kStatusBytes;
@@ -106,6 +119,9 @@ size_t mxfp4_workspace_bytes(int op, int64_t M, int64_t N, int64_t K) {
     case MXFP4_OP_LINEAR:
       if (!shape_ok(M, K) || N < 0) return 0;
       return linear_workspace(M, N, K).total;
+    case MXFP4_OP_NVFP4_LINEAR:
+      if (!shape_ok(M, K) || N < 0) return 0;
+      return nvfp4_linear_workspace(M, N, K).total;
     default:
       return 0;
   }
@@ -240,6 +256,95 @@ mxfp4_status mxfp4_linear(const void* x, int64_t M, int64_t K, mxfp4_rotation mo
   // The kernel just before the GEMM is the quantiser above, which does not write W.
   return from_cuda(launch_gemm(xq, xsf, wq, wsf, M, N, K, y, Epilogue{}, N, static_cast<int*>(ws),
                                base + w.g_off, ws_bytes - w.g_off, true, s));
+}
+
+size_t mxfp4_nvfp4_sf_bytes(int64_t rows, int64_t K) {
+  if (!shape_ok(rows, K)) return 0;
+  return mxfp4_sf_bytes(rows, 2 * K);  // atoms of 4 scales per 128 rows, 16-element groups
+}
+
+mxfp4_status mxfp4_nvfp4_tensor_scale(const void* x, mxfp4_dtype xdt, int64_t rows, int64_t K,
+                                      int64_t ldx, mxfp4_rotation mode, float* scale2,
+                                      mxfp4_stream_t stream) {
+  if (!x || !scale2) return MXFP4_ERR_INVALID_ARG;
+  if (xdt != MXFP4_DT_BF16 && xdt != MXFP4_DT_F32) return MXFP4_ERR_UNSUPPORTED;
+  if (mode != MXFP4_ROT_NONE && mode != MXFP4_ROT_HADAMARD32) return MXFP4_ERR_UNSUPPORTED;
+  if (!shape_ok(rows, K) || ldx < K || !within_limits(rows, K)) return MXFP4_ERR_SHAPE;
+  const int64_t esize = xdt == MXFP4_DT_F32 ? 4 : 2;
+  if (!aligned16(x) || (ldx * esize) % 16 != 0 || (reinterpret_cast<uintptr_t>(scale2) & 7u))
+    return MXFP4_ERR_ALIGN;
+  return from_cuda(launch_nvfp4_tensor_scale(x, xdt == MXFP4_DT_F32, rows, K, ldx, (int)mode,
+                                             scale2, static_cast<cudaStream_t>(stream)));
+}
+
+mxfp4_status mxfp4_nvfp4_quantize(const void* x, mxfp4_dtype xdt, int64_t rows, int64_t K,
+                                  int64_t ldx, mxfp4_rotation mode, const float* tensor_scale,
+                                  uint8_t* q, uint8_t* sf, mxfp4_stream_t stream) {
+  mxfp4_status st = validate_quantize(x, xdt, rows, K, ldx, q, sf);
+  if (st != MXFP4_OK) return st;
+  if (!tensor_scale) return MXFP4_ERR_INVALID_ARG;
+  if (mode != MXFP4_ROT_NONE && mode != MXFP4_ROT_HADAMARD32) return MXFP4_ERR_UNSUPPORTED;
+  if (!within_limits(rows, 2 * K)) return MXFP4_ERR_SHAPE;
+  if (rows == 0) return MXFP4_OK;
+  return from_cuda(launch_nvfp4_quantize(x, xdt == MXFP4_DT_F32, rows, K, ldx, (int)mode,
+                                         tensor_scale, q, sf, nullptr,
+                                         static_cast<cudaStream_t>(stream)));
+}
+
+mxfp4_status mxfp4_nvfp4_gemm(const uint8_t* aq, const uint8_t* asf, const float* a_scale,
+                              const uint8_t* bq, const uint8_t* bsf, const float* b_scale,
+                              int64_t M, int64_t N, int64_t K, void* y, mxfp4_dtype ydt,
+                              int64_t ldy, void* ws, size_t ws_bytes, mxfp4_stream_t stream) {
+  mxfp4_status st = validate_gemm(aq, asf, bq, bsf, M, N, K, y, ydt, ldy);
+  if (st != MXFP4_OK) return st;
+  if (!ws || !a_scale || !b_scale) return MXFP4_ERR_INVALID_ARG;
+  if (!within_limits(M, 2 * K) || !within_limits(N, 2 * K)) return MXFP4_ERR_SHAPE;
+  if (!aligned16(ws) || (reinterpret_cast<uintptr_t>(a_scale) & 3u) ||
+      (reinterpret_cast<uintptr_t>(b_scale) & 3u))
+    return MXFP4_ERR_ALIGN;
+  if (ws_bytes < mxfp4_workspace_bytes(MXFP4_OP_GEMM, M, N, K)) return MXFP4_ERR_WORKSPACE;
+  if (M == 0) return MXFP4_OK;
+  Epilogue ep;
+  ep.out = ydt == MXFP4_DT_F32 ? kOutF32 : kOutBf16;
+  ep.nvfp4 = true;
+  ep.a_scale = a_scale;
+  ep.b_scale = b_scale;
+  return from_cuda(launch_gemm(aq, asf, bq, bsf, M, N, K, y, ep, ldy, static_cast<int*>(ws),
+                               static_cast<uint8_t*>(ws) + kStatusBytes, ws_bytes - kStatusBytes,
+                               false, static_cast<cudaStream_t>(stream)));
+}
+
+mxfp4_status mxfp4_nvfp4_linear(const void* x, int64_t M, int64_t K, mxfp4_rotation mode,
+                                const uint8_t* wq, const uint8_t* wsf, const float* w_scale,
+                                int64_t N, void* y, void* ws, size_t ws_bytes,
+                                mxfp4_stream_t stream) {
+  if (!x || !wq || !wsf || !w_scale || !y || !ws) return MXFP4_ERR_INVALID_ARG;
+  if (mode != MXFP4_ROT_NONE && mode != MXFP4_ROT_HADAMARD32) return MXFP4_ERR_UNSUPPORTED;
+  if (!shape_ok(M, K) || N < 16 || N % 16 != 0 || !within_limits(M, 2 * K) ||
+      !within_limits(N, 2 * K))
+    return MXFP4_ERR_SHAPE;
+  if (!aligned16(x) || !aligned16(wq) || !aligned16(wsf) || !aligned16(y) || !aligned16(ws) ||
+      (K * 2) % 16 != 0 || (N * 2) % 16 != 0 || (reinterpret_cast<uintptr_t>(w_scale) & 3u))
+    return MXFP4_ERR_ALIGN;
+  const LinearWorkspace w = nvfp4_linear_workspace(M, N, K);
+  if (ws_bytes < w.total) return MXFP4_ERR_WORKSPACE;
+  if (M == 0) return MXFP4_OK;
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  float* xs = reinterpret_cast<float*>(base + kScaleOff);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_nvfp4_tensor_scale(x, false, M, K, K, (int)mode, xs, s);
+  if (e != cudaSuccess) return MXFP4_ERR_CUDA;
+  e = launch_nvfp4_quantize(x, false, M, K, K, (int)mode, xs, base + w.q_off, base + w.sf_off,
+                            static_cast<int*>(ws), s);
+  if (e != cudaSuccess) return MXFP4_ERR_CUDA;
+  Epilogue ep;
+  ep.nvfp4 = true;
+  ep.a_scale = xs;
+  ep.b_scale = w_scale;
+  // The kernel just before the GEMM is the quantiser above, which does not write W.
+  return from_cuda(launch_gemm(base + w.q_off, base + w.sf_off, wq, wsf, M, N, K, y, ep, N,
+                               static_cast<int*>(ws), base + w.g_off, ws_bytes - w.g_off, true,
+                               s));
 }
 
 mxfp4_status mxfp4_poll_status(void* ws, mxfp4_status* out) {

@@ -13,6 +13,7 @@
 // evaluation.
 #pragma once
 
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -177,6 +178,47 @@ __device__ __forceinline__ uint32_t quantize_block(const float2 (&P)[16], uint4&
     w[q] = e2m1x8(S[4 * q].x, S[4 * q].y, S[4 * q + 1].x, S[4 * q + 1].y, S[4 * q + 2].x,
                   S[4 * q + 2].y, S[4 * q + 3].x, S[4 * q + 3].y);
   codes = make_uint4(w[0], w[1], w[2], w[3]);
+  return byte;
+}
+
+// ---------------------------------------------------------------- NVFP4 groups
+//
+// NVFP4 ("Bridging the Gap...", "Probleemstelling" item 1): 16-element groups with an
+// unsigned E4M3 scale each and an fp32 tensor scale st. Per group: g = amax / (6 st)
+// (two roundings), byte = nearest E4M3 of g (ties to even, saturating at 448),
+// S = E4M3(byte) * st, r = 1 / S, code_i = nearest E2M1 of y_i * r; each step one
+// IEEE fp32 rounding. st <= 0 (all-zero tensor) or S == 0 gives byte / codes 0.
+
+__device__ __forceinline__ uint32_t e4m3_rn(float g) {
+  uint16_t h;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(h) : "f"(0.0f), "f"(g));
+  return h & 0xFFu;  // the second source goes to the low byte
+}
+
+__device__ __forceinline__ float e4m3_to_f32(uint32_t byte) {
+  uint32_t hh;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(hh) : "h"((uint16_t)byte));
+  return __half2float(__ushort_as_half((unsigned short)(hh & 0xFFFFu)));
+}
+
+// 8 packed pairs (16 rotated values) -> E4M3 byte, and 8 code bytes in w[0..1].
+__device__ __forceinline__ uint32_t quantize_group16(const float2* P, float st, uint32_t (&w)[2]) {
+  float m = fabsf(P[0].x);
+#pragma unroll
+  for (int j = 0; j < 8; ++j) m = fmaxf(m, fmaxf(fabsf(P[j].x), fabsf(P[j].y)));
+  w[0] = w[1] = 0u;
+  if (!(st > 0.0f)) return 0u;
+  const float g = __fdiv_rn(m, __fmul_rn(6.0f, st));
+  const uint32_t byte = e4m3_rn(g);
+  const float S = __fmul_rn(e4m3_to_f32(byte), st);
+  if (S == 0.0f) return byte;
+  const float r = __frcp_rn(S);
+  const float2 rr = make_float2(r, r);
+  float2 v[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) v[j] = __fmul2_rn(P[j], rr);
+  w[0] = e2m1x8(v[0].x, v[0].y, v[1].x, v[1].y, v[2].x, v[2].y, v[3].x, v[3].y);
+  w[1] = e2m1x8(v[4].x, v[4].y, v[5].x, v[5].y, v[6].x, v[6].y, v[7].x, v[7].y);
   return byte;
 }
 

@@ -56,7 +56,7 @@ struct Params {
   uint32_t M, N, K;
   uint32_t m_tiles, n_tiles;
   uint32_t k_tiles;        // ceil(K / 256)
-  uint32_t k_atoms;        // ceil(K / 128): scale atoms per 128-row group
+  uint32_t k_atoms;        // scale atoms per 128-row group: ceil(K / 128), NVFP4 ceil(K / 64)
   uint32_t b_row_tiles;    // ceil(N / 128)
   uint64_t ldy;            // elements
   // Work units: tiles [0, full_units) whole; each later tile split into split_g K chunks
@@ -69,6 +69,8 @@ struct Params {
   uint8_t* ysf;            // MXFP4 output: scales, tensor-core layout of an [M, N] operand
   uint32_t qmode;          // MXFP4 output: rotation of each 32-column block
   uint32_t rows_pad, n_katoms_y;
+  const float* a_scale;    // NVFP4: tensor scales of A and B (device fp32)
+  const float* b_scale;
 };
 
 struct Unit {
@@ -150,13 +152,16 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 // the leader's commits arrive on both CTAs' barriers. No load is multicast.
 
 
-template <uint32_t STAGES>
+template <uint32_t STAGES, bool NV = false>
 struct PairConfig {
+  // scale atoms (128 rows x 4 scales) per stage of 256 K-elements and 128 rows: 2 for
+  // MXFP4 (32-element blocks), 4 for NVFP4 (16-element groups)
+  static constexpr uint32_t AT = NV ? 4 : 2;
   static constexpr uint32_t BN = 256;                 // N per pair tile
   static constexpr uint32_t A_STAGE = 128 * BK_BYTES;  // own 128 rows of A
   static constexpr uint32_t B_STAGE = 128 * BK_BYTES;  // own 128 rows of B
-  static constexpr uint32_t SFA_STAGE = 1024;          // own rows: 2 scale atoms
-  static constexpr uint32_t SFB_STAGE = 2048;          // all 256 rows of B: 2 groups x 2 atoms
+  static constexpr uint32_t SFA_STAGE = AT * 512;      // own rows: AT scale atoms
+  static constexpr uint32_t SFB_STAGE = 2 * AT * 512;  // all 256 rows of B: 2 groups x AT atoms
   static constexpr uint32_t STAGE_TX = A_STAGE + B_STAGE + SFA_STAGE + SFB_STAGE;
   static constexpr uint32_t OFF_A = 0;
   static constexpr uint32_t OFF_B = OFF_A + STAGES * A_STAGE;
@@ -174,13 +179,13 @@ struct PairConfig {
   // overlap the rest of the drain.
   static constexpr uint32_t ACC1_COL = 192;
   static constexpr uint32_t SFA_COL = ACC1_COL + BN;  // 448
-  static constexpr uint32_t SFB_COL = SFA_COL + 8;
+  static constexpr uint32_t SFB_COL = SFA_COL + 4 * AT;
   static constexpr uint32_t TMEM_COLS = 512;
-  static_assert(SFB_COL + 16 <= TMEM_COLS, "tensor memory budget");
+  static_assert(SFB_COL + 8 * AT <= TMEM_COLS, "tensor memory budget");
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
-template <uint32_t STAGES, int OUT>
+template <uint32_t STAGES, int OUT, bool NV>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     mxf4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a,
                           const __grid_constant__ CUtensorMap tmap_b,
@@ -189,7 +194,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                           const __grid_constant__ CUtensorMap tmap_y, const Params p,
                           const __grid_constant__ KronCoeffs kc) {
   constexpr bool Y_F32 = OUT == kOutF32;
-  using C = PairConfig<STAGES>;
+  using C = PairConfig<STAGES, NV>;
   constexpr uint32_t BN = C::BN;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_addr(smem_raw);
@@ -266,9 +271,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           // scale atoms: A's are rows of a [row_tiles * k_atoms, 128-word] view, B's a
           // [row_tiles, k_atoms, 128-word] view (both 128-row groups of the tile)
           tma_load_2d_pair(sbase + C::OFF_SFA + stage * C::SFA_STAGE, &tmap_sfa, fb, 0,
-                           (int32_t)((uint32_t)(m_cta / 128) * p.k_atoms + 2 * kt));
+                           (int32_t)((uint32_t)(m_cta / 128) * p.k_atoms + C::AT * kt));
           tma_load_3d_pair(sbase + C::OFF_SFB + stage * C::SFB_STAGE, &tmap_sfb, fb, 0,
-                           (int32_t)(2 * kt), (int32_t)(nt * 2u));
+                           (int32_t)(C::AT * kt), (int32_t)(nt * 2u));
           ++issued;
           if (++stage == STAGES) {
             stage = 0;
@@ -312,22 +317,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           tc_fence_after();
           const uint32_t sfa_s = sbase + C::OFF_SFA + stage * C::SFA_STAGE;
           const uint32_t sfb_s = sbase + C::OFF_SFB + stage * C::SFB_STAGE;
-          for (uint32_t a = 0; a < 2; ++a) {
+          for (uint32_t a = 0; a < C::AT; ++a) {
             tmem_cp_32x128b_warpx4_pair(tmem_base + C::SFA_COL + 4 * a, smem_desc_sf(sfa_s + a * 512));
             for (uint32_t g = 0; g < 2; ++g)
               tmem_cp_32x128b_warpx4_pair(tmem_base + C::SFB_COL + 4 * (2 * a + g),
-                                          smem_desc_sf(sfb_s + (g * 2 + a) * 512));
+                                          smem_desc_sf(sfb_s + (g * C::AT + a) * 512));
           }
           const uint32_t k_left = p.K - kt * 256u;
           const uint32_t steps = k_left >= 256u ? 4u : (k_left + 63u) / 64u;
           const uint32_t a_tile = sbase + C::OFF_A + stage * C::A_STAGE;
           const uint32_t b_tile = sbase + C::OFF_B + stage * C::B_STAGE;
           for (uint32_t k = 0; k < steps; ++k) {
-            const uint32_t sf_id = (k & 1u) * 2u;
-            mma_mxf4_pair(d_tmem, smem_desc_sw128(a_tile + k * MMA_K_BYTES),
-                          smem_desc_sw128(b_tile + k * MMA_K_BYTES), idesc_mxf4(256, BN, sf_id, sf_id),
-                          tmem_base + C::SFA_COL + 4 * (k >> 1), tmem_base + C::SFB_COL + 8 * (k >> 1),
-                          (kt != w.kt0 || k != 0u) ? 1u : 0u);
+            const uint32_t acc_in = (kt != w.kt0 || k != 0u) ? 1u : 0u;
+            if constexpr (NV) {
+              // NVFP4: one atom (4 scales of 16 per row) per K = 64 step
+              mma_nvf4_pair(d_tmem, smem_desc_sw128(a_tile + k * MMA_K_BYTES),
+                            smem_desc_sw128(b_tile + k * MMA_K_BYTES), idesc_nvf4(256, BN),
+                            tmem_base + C::SFA_COL + 4 * k, tmem_base + C::SFB_COL + 8 * k, acc_in);
+            } else {
+              // MXFP4: an atom (4 scales of 32 per row) serves two K = 64 steps
+              const uint32_t sf_id = (k & 1u) * 2u;
+              mma_mxf4_pair(d_tmem, smem_desc_sw128(a_tile + k * MMA_K_BYTES),
+                            smem_desc_sw128(b_tile + k * MMA_K_BYTES),
+                            idesc_mxf4(256, BN, sf_id, sf_id), tmem_base + C::SFA_COL + 4 * (k >> 1),
+                            tmem_base + C::SFB_COL + 8 * (k >> 1), acc_in);
+            }
           }
           mma_commit_pair_both(bar_empty + 8 * stage);  // frees the stage in both CTAs
           if (++stage == STAGES) {
@@ -353,6 +367,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const uint32_t quad = warp & 3u;
     const uint32_t half = (warp - kFirstEpiWarp) / 4u;
     const uint32_t tempty_at_leader = map_to_rank(bar_tempty, 0);
+    // NVFP4: y = alpha * sum, alpha = product of the tensor scales (written by earlier
+    // kernels; this grid has waited for its predecessor above)
+    float alpha = 1.0f;
+    if constexpr (NV) alpha = __fmul_rn(__ldg(p.a_scale), __ldg(p.b_scale));
     const uint32_t buf = sbase + C::OFF_EPI + (warp - kFirstEpiWarp) * C::EPI_BUF;
     const uint32_t rowoff = buf + lane * 128u;
     constexpr uint32_t CCOLS = Y_F32 ? 32 : 64;  // columns per 128-byte staged row
@@ -426,6 +444,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           }
         }
         const uint32_t col_base = nt * BN + ch[r] * 64u;  // first column of this chunk
+        if constexpr (NV) {  // the two tensor scales, once, on the full sum
+#pragma unroll
+          for (uint32_t h = 0; h < 2; ++h)
+#pragma unroll
+            for (uint32_t j = 0; j < 32; ++j)
+              v[h][j] = __float_as_uint(__fmul_rn(__uint_as_float(v[h][j]), alpha));
+        }
         if (p.bias != nullptr) {
 #pragma unroll
           for (uint32_t h = 0; h < 2; ++h) {
@@ -565,9 +590,10 @@ bool make_operand_map(CUtensorMap* map, const uint8_t* base, uint64_t rows, uint
 }
 
 // Scale atoms of an operand as 128-word (512-byte) rows: 2-D [row_tiles * k_atoms, 128]
-// (box: 2 consecutive atoms) or 3-D [row_tiles, k_atoms, 128] (box: 2 atoms x 2 row tiles).
+// (box: `at` consecutive atoms) or 3-D [row_tiles, k_atoms, 128] (box: `at` atoms x 2 row
+// tiles).
 bool make_scale_map(CUtensorMap* map, const uint8_t* sf, uint64_t row_tiles, uint64_t k_atoms,
-                    bool three_d) {
+                    bool three_d, uint32_t at) {
   auto fn = get_encode_fn();
   if (!fn) return false;
   cuuint32_t estr[3] = {1, 1, 1};
@@ -575,14 +601,14 @@ bool make_scale_map(CUtensorMap* map, const uint8_t* sf, uint64_t row_tiles, uin
   if (three_d) {
     cuuint64_t dims[3] = {128, k_atoms, row_tiles};
     cuuint64_t strides[2] = {512, k_atoms * 512};
-    cuuint32_t box[3] = {128, 2, 2};
+    cuuint32_t box[3] = {128, at, 2};
     r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<uint8_t*>(sf), dims, strides, box,
            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   } else {
     cuuint64_t dims[2] = {128, row_tiles * k_atoms};
     cuuint64_t strides[1] = {512};
-    cuuint32_t box[2] = {128, 2};
+    cuuint32_t box[2] = {128, at};
     r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint8_t*>(sf), dims, strides, box,
            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -647,22 +673,23 @@ PairPlan pair_plan(int64_t M, int64_t N, int64_t K, uint32_t pairs) {
   return pl;
 }
 
-template <uint32_t STAGES, int OUT>
+template <uint32_t STAGES, int OUT, bool NV>
 cudaError_t launch_pair(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq,
                         const uint8_t* bsf, int64_t M, int64_t N, int64_t K, void* y,
                         const Epilogue& ep, int64_t ldy, int* status, uint8_t* scratch,
                         size_t scratch_bytes, cudaStream_t stream) {
-  using C = PairConfig<STAGES>;
-  const uint64_t k_atoms = (uint64_t)sf_katoms(K);
+  using C = PairConfig<STAGES, NV>;
+  // scale atoms per 128-row group: one per 4 scales, i.e. per 128 (MXFP4) or 64 (NVFP4) K
+  const uint64_t k_atoms = (uint64_t)sf_katoms(NV ? 2 * K : K);
   CUtensorMap ta, tb, tsa, tsb, ty{};
   if (!make_operand_map(&ta, aq, (uint64_t)M, (uint64_t)(K / 2), 128) ||
       !make_operand_map(&tb, bq, (uint64_t)N, (uint64_t)(K / 2), 128) ||
-      !make_scale_map(&tsa, asf, (uint64_t)sf_row_tiles(M), k_atoms, false) ||
-      !make_scale_map(&tsb, bsf, (uint64_t)sf_row_tiles(N), k_atoms, true) ||
+      !make_scale_map(&tsa, asf, (uint64_t)sf_row_tiles(M), k_atoms, false, C::AT) ||
+      !make_scale_map(&tsb, bsf, (uint64_t)sf_row_tiles(N), k_atoms, true, C::AT) ||
       (OUT != kOutMxfp4 &&
        !make_output_map(&ty, y, (uint64_t)M, (uint64_t)N, (uint64_t)ldy, OUT == kOutF32)))
     return cudaErrorInvalidValue;
-  auto kern = mxf4_gemm_pair_kernel<STAGES, OUT>;
+  auto kern = mxf4_gemm_pair_kernel<STAGES, OUT, NV>;
   int dev = 0;
   cudaGetDevice(&dev);
   static bool attr_done[64] = {};
@@ -715,6 +742,8 @@ cudaError_t launch_pair(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq
   p.qmode = (uint32_t)ep.mode;
   p.rows_pad = (uint32_t)(sf_row_tiles(M) * 128);
   p.n_katoms_y = (uint32_t)sf_katoms(N);
+  p.a_scale = ep.a_scale;
+  p.b_scale = ep.b_scale;
   const uint32_t pairs =
       pl.units < (uint32_t)max_clusters[dev] ? pl.units : (uint32_t)max_clusters[dev];
 
@@ -741,16 +770,23 @@ cudaError_t launch_gemm(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq
   if (M <= 128)
     return launch_gemm_smallm(aq, asf, bq, bsf, M, N, K, y, ep, ldy, status, b_early, stream);
   // Otherwise CTA pairs with 256 x 256 tiles.
+  if (ep.nvfp4) {
+    if (ep.out == kOutF32)
+      return launch_pair<5, kOutF32, true>(aq, asf, bq, bsf, M, N, K, y, ep, ldy, status,
+                                           scratch, scratch_bytes, stream);
+    return launch_pair<5, kOutBf16, true>(aq, asf, bq, bsf, M, N, K, y, ep, ldy, status, scratch,
+                                          scratch_bytes, stream);
+  }
   switch (ep.out) {
     case kOutF32:
-      return launch_pair<5, kOutF32>(aq, asf, bq, bsf, M, N, K, y, ep, ldy, status, scratch,
-                                     scratch_bytes, stream);
+      return launch_pair<5, kOutF32, false>(aq, asf, bq, bsf, M, N, K, y, ep, ldy, status,
+                                            scratch, scratch_bytes, stream);
     case kOutMxfp4:
-      return launch_pair<5, kOutMxfp4>(aq, asf, bq, bsf, M, N, K, y, ep, ldy, status, scratch,
-                                       scratch_bytes, stream);
+      return launch_pair<5, kOutMxfp4, false>(aq, asf, bq, bsf, M, N, K, y, ep, ldy, status,
+                                              scratch, scratch_bytes, stream);
     default:
-      return launch_pair<5, kOutBf16>(aq, asf, bq, bsf, M, N, K, y, ep, ldy, status, scratch,
-                                      scratch_bytes, stream);
+      return launch_pair<5, kOutBf16, false>(aq, asf, bq, bsf, M, N, K, y, ep, ldy, status,
+                                             scratch, scratch_bytes, stream);
   }
 }
 

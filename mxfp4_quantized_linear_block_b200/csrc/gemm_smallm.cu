@@ -39,13 +39,19 @@ constexpr uint32_t kMaxSplits = 8;  // portable cluster size
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr int kTimeoutCode = 7;
 
-template <uint32_t NT>
+template <uint32_t NT, bool NV = false>
 struct SmallConfig {
-  // Two CTAs per SM: stages sized so that 2 x SMEM_BYTES fits an SM's shared memory.
-  static constexpr uint32_t STAGES = NT <= 16 ? 5 : NT <= 64 ? 4 : 3;
+  // scale atoms (128 rows x 4 scales) per k-tile of 256 elements: 2 for MXFP4, 4 for NVFP4
+  static constexpr uint32_t AT = NV ? 4 : 2;
+  // Two CTAs per SM: as many stages (at most 5) as let 2 x SMEM_BYTES fit an SM's
+  // shared memory (233472 bytes, 1 KB of it reserved per CTA).
+  static constexpr uint32_t STAGE_BYTES = 128 * 128 + NT * 128 + 2 * AT * 512;
+  static constexpr uint32_t STAGES = (116736 - 1024 - 1024 - 512) / STAGE_BYTES < 5
+                                         ? (116736 - 1024 - 1024 - 512) / STAGE_BYTES
+                                         : 5;
   static constexpr uint32_t A_STAGE = 128 * 128;  // 128 rows of W x 256 elements
   static constexpr uint32_t B_STAGE = NT * 128;   // NT token rows x 256 elements
-  static constexpr uint32_t SF_STAGE = 1024;      // 2 scale atoms
+  static constexpr uint32_t SF_STAGE = AT * 512;  // AT scale atoms
   static constexpr uint32_t OFF_A = 0;
   static constexpr uint32_t OFF_B = OFF_A + STAGES * A_STAGE;
   static constexpr uint32_t OFF_SFA = OFF_B + STAGES * B_STAGE;
@@ -57,8 +63,8 @@ struct SmallConfig {
   // fp32 partial [NT][128] at offset 0, over the A/B stages once every MMA has completed
   static constexpr uint32_t RED_BYTES = NT * 128 * 4;
   static constexpr uint32_t SFA_COL = NT;
-  static constexpr uint32_t SFB_COL = NT + 8;
-  static constexpr uint32_t COLS_USED = NT + 16;
+  static constexpr uint32_t SFB_COL = NT + 4 * AT;
+  static constexpr uint32_t COLS_USED = NT + 8 * AT;
   static constexpr uint32_t TMEM_COLS = COLS_USED <= 32 ? 32 : COLS_USED <= 64 ? 64
                                         : COLS_USED <= 128 ? 128 : 256;
   static_assert(NT % 16 == 0 && NT >= 16 && NT <= 128, "token tile");
@@ -79,6 +85,8 @@ struct SmallParams {
   uint8_t* ysf;         // MXFP4 output: scales (tensor-core layout of an [M, N] operand)
   uint32_t qmode;       // MXFP4 output: rotation of each 32-column block
   uint32_t n_katoms_y;  // MXFP4 output: scale atoms per 128-row group of Y
+  const float* a_scale; // NVFP4: tensor scales (device fp32) of X and W
+  const float* b_scale;
 };
 
 __device__ __forceinline__ void record_timeout(int* status) {
@@ -106,7 +114,7 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 // all S splits are issued together, then added in split order 0, 1, ..., S-1.
 template <uint32_t NT, int OUT, uint32_t S>
 __device__ __forceinline__ void reduce_store(const SmallParams& p, uint32_t sbase, uint32_t wt,
-                                             uint32_t sp, uint32_t tid) {
+                                             uint32_t sp, uint32_t tid, float alpha) {
   constexpr uint32_t IB = 16 / S;  // 16 loads in flight per thread
   const uint32_t g0 = sp * 32u / S, g1 = (sp + 1u) * 32u / S, width = g1 - g0;
   const uint32_t rows = p.M < NT ? p.M : NT;
@@ -136,6 +144,12 @@ __device__ __forceinline__ void reduce_store(const SmallParams& p, uint32_t sbas
         acc.y += t[i][s].y;
         acc.z += t[i][s].z;
         acc.w += t[i][s].w;
+      }
+      if (alpha != 1.0f) {  // NVFP4: the product of the tensor scales, on the full sum
+        acc.x = __fmul_rn(acc.x, alpha);
+        acc.y = __fmul_rn(acc.y, alpha);
+        acc.z = __fmul_rn(acc.z, alpha);
+        acc.w = __fmul_rn(acc.w, alpha);
       }
       if (p.bias != nullptr) {
         const float4 b = __ldg(reinterpret_cast<const float4*>(p.bias + col[i]));
@@ -221,12 +235,13 @@ __device__ __forceinline__ void reduce_store_mxfp4(const SmallParams& p, const K
   }
 }
 
-template <uint32_t NT, int OUT>
+template <uint32_t NT, int OUT, bool NV>
 __global__ void __launch_bounds__(kThreads, 2) mxf4_gemm_smallm_kernel(
     const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
     const SmallParams p, const __grid_constant__ KronCoeffs kc) {
-  using C = SmallConfig<NT>;
+  using C = SmallConfig<NT, NV>;
   constexpr uint32_t STAGES = C::STAGES;
+  constexpr uint32_t AT = C::AT;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_addr(smem_raw);
   const uint32_t pad = ((raw_addr + 1023u) & ~1023u) - raw_addr;
@@ -267,13 +282,13 @@ __global__ void __launch_bounds__(kThreads, 2) mxf4_gemm_smallm_kernel(
     // and of the wait for that kernel. Each stage's barrier expects its X bytes too.
     for (uint32_t i = 0; i < (p.w_early ? pre : 0u); ++i) {
       const uint32_t kt = kt0 + i;
-      const uint32_t atoms = (p.k_atoms - 2 * kt) >= 2 ? 2u : 1u;
+      const uint32_t atoms = (p.k_atoms - AT * kt) >= AT ? AT : p.k_atoms - AT * kt;
       const uint32_t fb = bar_full + 8 * i;
       mbar_arrive_expect_tx(fb, C::A_STAGE + C::B_STAGE + 2u * atoms * 512u);
       tma_load_2d(sbase + C::OFF_A + i * C::A_STAGE, &tmap_w, fb, (int32_t)(kt * 128u),
                   (int32_t)(wt * 128u));
       bulk_load(sbase + C::OFF_SFA + i * C::SF_STAGE,
-                p.wsf + ((uint64_t)wt * p.k_atoms + 2 * kt) * 512u, atoms * 512u, fb);
+                p.wsf + ((uint64_t)wt * p.k_atoms + AT * kt) * 512u, atoms * 512u, fb);
     }
   }
   if (warp == 1) {
@@ -293,17 +308,17 @@ __global__ void __launch_bounds__(kThreads, 2) mxf4_gemm_smallm_kernel(
       asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
       for (uint32_t i = 0; i < pre; ++i) {
         const uint32_t kt = kt0 + i;
-        const uint32_t atoms = (p.k_atoms - 2 * kt) >= 2 ? 2u : 1u;
+        const uint32_t atoms = (p.k_atoms - AT * kt) >= AT ? AT : p.k_atoms - AT * kt;
         const uint32_t fb = bar_full + 8 * i;
         if (!p.w_early) {
           mbar_arrive_expect_tx(fb, C::A_STAGE + C::B_STAGE + 2u * atoms * 512u);
           tma_load_2d(sbase + C::OFF_A + i * C::A_STAGE, &tmap_w, fb, (int32_t)(kt * 128u),
                       (int32_t)(wt * 128u));
           bulk_load(sbase + C::OFF_SFA + i * C::SF_STAGE,
-                    p.wsf + ((uint64_t)wt * p.k_atoms + 2 * kt) * 512u, atoms * 512u, fb);
+                    p.wsf + ((uint64_t)wt * p.k_atoms + AT * kt) * 512u, atoms * 512u, fb);
         }
         tma_load_2d(sbase + C::OFF_B + i * C::B_STAGE, &tmap_x, fb, (int32_t)(kt * 128u), 0);
-        bulk_load(sbase + C::OFF_SFB + i * C::SF_STAGE, p.xsf + (uint64_t)(2 * kt) * 512u,
+        bulk_load(sbase + C::OFF_SFB + i * C::SF_STAGE, p.xsf + (uint64_t)(AT * kt) * 512u,
                   atoms * 512u, fb);
       }
       uint32_t stage = pre % STAGES, phase = pre == STAGES ? 1u : 0u, issued = pre;
@@ -313,15 +328,15 @@ __global__ void __launch_bounds__(kThreads, 2) mxf4_gemm_smallm_kernel(
           ok = false;
           break;
         }
-        const uint32_t atoms = (p.k_atoms - 2 * kt) >= 2 ? 2u : 1u;
+        const uint32_t atoms = (p.k_atoms - AT * kt) >= AT ? AT : p.k_atoms - AT * kt;
         const uint32_t fb = bar_full + 8 * stage;
         mbar_arrive_expect_tx(fb, C::A_STAGE + C::B_STAGE + 2u * atoms * 512u);
         tma_load_2d(sbase + C::OFF_A + stage * C::A_STAGE, &tmap_w, fb, (int32_t)(kt * 128u),
                     (int32_t)(wt * 128u));
         tma_load_2d(sbase + C::OFF_B + stage * C::B_STAGE, &tmap_x, fb, (int32_t)(kt * 128u), 0);
         bulk_load(sbase + C::OFF_SFA + stage * C::SF_STAGE,
-                  p.wsf + ((uint64_t)wt * p.k_atoms + 2 * kt) * 512u, atoms * 512u, fb);
-        bulk_load(sbase + C::OFF_SFB + stage * C::SF_STAGE, p.xsf + (uint64_t)(2 * kt) * 512u,
+                  p.wsf + ((uint64_t)wt * p.k_atoms + AT * kt) * 512u, atoms * 512u, fb);
+        bulk_load(sbase + C::OFF_SFB + stage * C::SF_STAGE, p.xsf + (uint64_t)(AT * kt) * 512u,
                   atoms * 512u, fb);
         ++issued;
         if (++stage == STAGES) {
@@ -353,7 +368,7 @@ __global__ void __launch_bounds__(kThreads, 2) mxf4_gemm_smallm_kernel(
           break;
         }
         tc_fence_after();
-        const uint32_t atoms = (p.k_atoms - 2 * kt) >= 2 ? 2u : 1u;
+        const uint32_t atoms = (p.k_atoms - AT * kt) >= AT ? AT : p.k_atoms - AT * kt;
         for (uint32_t a = 0; a < atoms; ++a) {
           tmem_cp_32x128b_warpx4(tmem_base + C::SFA_COL + 4 * a,
                                  smem_desc_sf(sbase + C::OFF_SFA + stage * C::SF_STAGE + a * 512));
@@ -366,9 +381,15 @@ __global__ void __launch_bounds__(kThreads, 2) mxf4_gemm_smallm_kernel(
         const uint32_t b_tile = sbase + C::OFF_B + stage * C::B_STAGE;
         for (uint32_t k = 0; k < steps; ++k) {
           const uint32_t sf_id = (k & 1u) * 2u;
-          mma_mxf4(tmem_base, smem_desc_sw128(a_tile + k * 32u), smem_desc_sw128(b_tile + k * 32u),
-                   idesc_mxf4(128, NT, sf_id, sf_id), tmem_base + C::SFA_COL + 4 * (k >> 1),
-                   tmem_base + C::SFB_COL + 4 * (k >> 1), (kt != kt0 || k != 0) ? 1u : 0u);
+          const uint32_t acc_in = (kt != kt0 || k != 0) ? 1u : 0u;
+          if constexpr (NV)  // one atom (4 scales of 16) per K = 64 step
+            mma_nvf4(tmem_base, smem_desc_sw128(a_tile + k * 32u), smem_desc_sw128(b_tile + k * 32u),
+                     idesc_nvf4(128, NT), tmem_base + C::SFA_COL + 4 * k,
+                     tmem_base + C::SFB_COL + 4 * k, acc_in);
+          else  // an atom (4 scales of 32) per two K = 64 steps
+            mma_mxf4(tmem_base, smem_desc_sw128(a_tile + k * 32u), smem_desc_sw128(b_tile + k * 32u),
+                     idesc_mxf4(128, NT, sf_id, sf_id), tmem_base + C::SFA_COL + 4 * (k >> 1),
+                     tmem_base + C::SFB_COL + 4 * (k >> 1), acc_in);
         }
         mma_commit(bar_empty + 8 * stage);
         if (++stage == STAGES) {
@@ -416,18 +437,20 @@ __global__ void __launch_bounds__(kThreads, 2) mxf4_gemm_smallm_kernel(
     tmem_dealloc(tmem_base, C::TMEM_COLS);
   } else if (warp >= kFirstEpiWarp) {
     const uint32_t tid = threadIdx.x - kFirstEpiWarp * 32u;
+    float alpha = 1.0f;  // scales written by earlier kernels: this grid has waited for them
+    if constexpr (NV) alpha = __fmul_rn(__ldg(p.a_scale), __ldg(p.b_scale));
     if constexpr (OUT == kOutMxfp4) {
       reduce_store_mxfp4<NT>(p, kc, sbase, wt, sp, S, tid);
     } else {
       switch (S) {
-        case 1: reduce_store<NT, OUT, 1>(p, sbase, wt, sp, tid); break;
-        case 2: reduce_store<NT, OUT, 2>(p, sbase, wt, sp, tid); break;
-        case 3: reduce_store<NT, OUT, 3>(p, sbase, wt, sp, tid); break;
-        case 4: reduce_store<NT, OUT, 4>(p, sbase, wt, sp, tid); break;
-        case 5: reduce_store<NT, OUT, 5>(p, sbase, wt, sp, tid); break;
-        case 6: reduce_store<NT, OUT, 6>(p, sbase, wt, sp, tid); break;
-        case 7: reduce_store<NT, OUT, 7>(p, sbase, wt, sp, tid); break;
-        default: reduce_store<NT, OUT, 8>(p, sbase, wt, sp, tid); break;
+        case 1: reduce_store<NT, OUT, 1>(p, sbase, wt, sp, tid, alpha); break;
+        case 2: reduce_store<NT, OUT, 2>(p, sbase, wt, sp, tid, alpha); break;
+        case 3: reduce_store<NT, OUT, 3>(p, sbase, wt, sp, tid, alpha); break;
+        case 4: reduce_store<NT, OUT, 4>(p, sbase, wt, sp, tid, alpha); break;
+        case 5: reduce_store<NT, OUT, 5>(p, sbase, wt, sp, tid, alpha); break;
+        case 6: reduce_store<NT, OUT, 6>(p, sbase, wt, sp, tid, alpha); break;
+        case 7: reduce_store<NT, OUT, 7>(p, sbase, wt, sp, tid, alpha); break;
+        default: reduce_store<NT, OUT, 8>(p, sbase, wt, sp, tid, alpha); break;
       }
     }
   }
@@ -486,17 +509,17 @@ Plan make_plan(int64_t M, int64_t N, int64_t K) {
   return pl;
 }
 
-template <uint32_t NT, int OUT>
+template <uint32_t NT, int OUT, bool NV>
 cudaError_t launch_nt(const Plan& pl, const uint8_t* aq, const uint8_t* asf, const uint8_t* bq,
                       const uint8_t* bsf, int64_t M, int64_t N, int64_t K, void* y,
                       const Epilogue& ep, int64_t ldy, int* status, bool w_early,
                       cudaStream_t stream) {
-  using C = SmallConfig<NT>;
+  using C = SmallConfig<NT, NV>;
   CUtensorMap tw, tx;
   if (!operand_map(&tw, bq, (uint64_t)N, (uint64_t)(K / 2), 128) ||
       !operand_map(&tx, aq, (uint64_t)M, (uint64_t)(K / 2), NT))
     return cudaErrorInvalidValue;
-  auto kern = mxf4_gemm_smallm_kernel<NT, OUT>;
+  auto kern = mxf4_gemm_smallm_kernel<NT, OUT, NV>;
   int dev = 0;
   cudaGetDevice(&dev);
   static bool attr_done[64] = {};
@@ -517,7 +540,7 @@ cudaError_t launch_nt(const Plan& pl, const uint8_t* aq, const uint8_t* asf, con
   p.K = (uint32_t)K;
   p.ldy = (uint64_t)ldy;
   p.k_tiles = pl.k_tiles;
-  p.k_atoms = (uint32_t)sf_katoms(K);
+  p.k_atoms = (uint32_t)sf_katoms(NV ? 2 * K : K);  // atoms of 4 scales per 128-row group
   p.splits = pl.splits;
   p.kt_per_split = pl.kt_per_split;
   p.w_early = w_early ? 1u : 0u;
@@ -525,6 +548,8 @@ cudaError_t launch_nt(const Plan& pl, const uint8_t* aq, const uint8_t* asf, con
   p.ysf = ep.ysf;
   p.qmode = (uint32_t)ep.mode;
   p.n_katoms_y = (uint32_t)sf_katoms(N);
+  p.a_scale = ep.a_scale;
+  p.b_scale = ep.b_scale;
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(pl.units);
   cfg.blockDim = dim3(kThreads);
@@ -550,16 +575,23 @@ cudaError_t launch_gemm_smallm(const uint8_t* aq, const uint8_t* asf, const uint
                                cudaStream_t stream) {
   const Plan pl = make_plan(M, N, K);
 #define MXFP4_SMALLM(NTV)                                                                       \
+  if (ep.nvfp4) {                                                                               \
+    if (ep.out == kOutF32)                                                                      \
+      return launch_nt<NTV, kOutF32, true>(pl, aq, asf, bq, bsf, M, N, K, y, ep, ldy, status,   \
+                                           b_early, stream);                                    \
+    return launch_nt<NTV, kOutBf16, true>(pl, aq, asf, bq, bsf, M, N, K, y, ep, ldy, status,    \
+                                          b_early, stream);                                     \
+  }                                                                                             \
   switch (ep.out) {                                                                             \
     case kOutF32:                                                                               \
-      return launch_nt<NTV, kOutF32>(pl, aq, asf, bq, bsf, M, N, K, y, ep, ldy, status, b_early, \
-                                     stream);                                                   \
+      return launch_nt<NTV, kOutF32, false>(pl, aq, asf, bq, bsf, M, N, K, y, ep, ldy, status,  \
+                                            b_early, stream);                                   \
     case kOutMxfp4:                                                                             \
-      return launch_nt<NTV, kOutMxfp4>(pl, aq, asf, bq, bsf, M, N, K, y, ep, ldy, status,       \
-                                       b_early, stream);                                        \
+      return launch_nt<NTV, kOutMxfp4, false>(pl, aq, asf, bq, bsf, M, N, K, y, ep, ldy,        \
+                                              status, b_early, stream);                         \
     default:                                                                                    \
-      return launch_nt<NTV, kOutBf16>(pl, aq, asf, bq, bsf, M, N, K, y, ep, ldy, status,        \
-                                      b_early, stream);                                         \
+      return launch_nt<NTV, kOutBf16, false>(pl, aq, asf, bq, bsf, M, N, K, y, ep, ldy, status, \
+                                             b_early, stream);                                  \
   }
   switch (pl.nt) {
     case 16: MXFP4_SMALLM(16)

@@ -20,6 +20,15 @@ cudaError_t launch_rotate_quantize(const void* x, bool x_is_f32, int64_t rows, i
                                    int64_t ldx, int mode, const KronCoeffs* kc, uint8_t* q,
                                    uint8_t* sf, int* status, cudaStream_t stream);
 
+// NVFP4 (quantize.cu): tensor scale of x rotated by mode (0 / 1) into scale2[0] (scale2[1]
+// is scratch; a memset and two small kernels), and the quantiser with that scale: codes
+// as for MXFP4, E4M3 group bytes in atoms of 4 groups of 16 (sf_katoms(2K) per row tile).
+cudaError_t launch_nvfp4_tensor_scale(const void* x, bool x_is_f32, int64_t rows, int64_t K,
+                                     int64_t ldx, int mode, float* scale2, cudaStream_t stream);
+cudaError_t launch_nvfp4_quantize(const void* x, bool x_is_f32, int64_t rows, int64_t K,
+                                  int64_t ldx, int mode, const float* tensor_scale, uint8_t* q,
+                                  uint8_t* sf, int* status, cudaStream_t stream);
+
 // Rotation over 64- or 128-element groups (span) + quantisation (quantize_wide.cu).
 cudaError_t launch_rotate_quantize_wide(const void* x, bool x_is_f32, int64_t rows, int64_t K,
                                         int64_t ldx, int span, uint8_t* q, uint8_t* sf,
@@ -39,6 +48,12 @@ struct Epilogue {
   int mode = 0;
   KronCoeffs kc{};
   uint8_t* ysf = nullptr;
+  // NVFP4 operands (16-element groups, E4M3 group scales in atoms of 4 per 64 K): the
+  // result is multiplied by *a_scale * *b_scale (device fp32 tensor scales); bf16 / fp32
+  // output only.
+  bool nvfp4 = false;
+  const float* a_scale = nullptr;
+  const float* b_scale = nullptr;
 };
 
 // Block-scaled GEMM y[M, N] = A[M, K] . B[N, K]^T on tcgen05. Host-validated arguments.

@@ -52,12 +52,12 @@ struct TileShape {
   static constexpr uint32_t SMEM = kStages * STAGE + 64 + 1024;
 };
 
-template <int MODE, bool F32_IN>
+template <int MODE, bool F32_IN, bool NV>
 __global__ void __launch_bounds__(kThreads) rotate_quantize_kernel(
     const __grid_constant__ CUtensorMap tmap_x, uint32_t rows, uint32_t rows_pad, uint32_t kb_real,
     uint32_t k_boxes, uint32_t tiles, uint32_t n_katoms, uint64_t q_row_bytes,
     const __grid_constant__ KronCoeffs kc, uint8_t* __restrict__ q, uint8_t* __restrict__ sf,
-    int* status) {
+    int* status, const float* __restrict__ tensor_scale) {
   using namespace sm100;
   using T = TileShape<F32_IN>;
   constexpr int CH = F32_IN ? 8 : 4;  // 16-byte chunks per 32-element block
@@ -85,6 +85,9 @@ __global__ void __launch_bounds__(kThreads) rotate_quantize_kernel(
   // then let the next kernel start its own set-up.
   asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  // NVFP4: the fp32 tensor scale (written by an earlier kernel; waited for above)
+  float st = 0.0f;
+  if constexpr (NV) st = __ldg(tensor_scale);
 
   auto issue = [&](uint32_t tile, uint32_t s) {
     const uint32_t rt = tile / k_boxes, kx = tile - rt * k_boxes;
@@ -142,15 +145,31 @@ __global__ void __launch_bounds__(kThreads) rotate_quantize_kernel(
     }
 
     if (row < rows_pad) {
-      uint32_t byte = 0;
-      if (row < rows && kb < kb_real) {
-        if constexpr (MODE == 1) hadamard32(P);
-        if constexpr (MODE == 2) kron32(P, kc);
-        uint4 codes;
-        byte = quantize_block(P, codes);
-        st_v4(q + (uint64_t)row * q_row_bytes + (uint64_t)kb * 16u, codes);
+      if constexpr (NV) {
+        // two 16-element groups: scale bytes 2 kb and 2 kb + 1 are adjacent in an atom
+        uint32_t b2 = 0;
+        if (row < rows && kb < kb_real) {
+          if constexpr (MODE == 1) hadamard32(P);
+          uint32_t w0[2], w1[2];
+          const uint32_t b0 = quantize_group16(&P[0], st, w0);
+          const uint32_t b1 = quantize_group16(&P[8], st, w1);
+          st_v4(q + (uint64_t)row * q_row_bytes + (uint64_t)kb * 16u,
+                make_uint4(w0[0], w0[1], w1[0], w1[1]));
+          b2 = b0 | (b1 << 8);
+        }
+        if (2u * kb < 4u * n_katoms)
+          *reinterpret_cast<uint16_t*>(sf + sf_offset(row, 2u * kb, n_katoms)) = (uint16_t)b2;
+      } else {
+        uint32_t byte = 0;
+        if (row < rows && kb < kb_real) {
+          if constexpr (MODE == 1) hadamard32(P);
+          if constexpr (MODE == 2) kron32(P, kc);
+          uint4 codes;
+          byte = quantize_block(P, codes);
+          st_v4(q + (uint64_t)row * q_row_bytes + (uint64_t)kb * 16u, codes);
+        }
+        sf[sf_offset(row, kb, n_katoms)] = static_cast<uint8_t>(byte);
       }
-      sf[sf_offset(row, kb, n_katoms)] = static_cast<uint8_t>(byte);
     }
     kx += step_kx;
     rt += step_rt;
@@ -180,9 +199,10 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-template <int MODE, bool F32_IN>
+template <int MODE, bool F32_IN, bool NV = false>
 cudaError_t launch_mode(const void* x, int64_t rows, int64_t K, int64_t ldx, const KronCoeffs& kc,
-                        uint8_t* q, uint8_t* sf, int* status, cudaStream_t stream) {
+                        uint8_t* q, uint8_t* sf, int* status, cudaStream_t stream,
+                        const float* tensor_scale = nullptr) {
   using T = TileShape<F32_IN>;
   auto fn = encode_fn();
   if (!fn) return cudaErrorNotSupported;
@@ -197,7 +217,7 @@ cudaError_t launch_mode(const void* x, int64_t rows, int64_t K, int64_t ldx, con
          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
 
-  auto kern = rotate_quantize_kernel<MODE, F32_IN>;
+  auto kern = rotate_quantize_kernel<MODE, F32_IN, NV>;
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
@@ -231,12 +251,105 @@ cudaError_t launch_mode(const void* x, int64_t rows, int64_t K, int64_t ldx, con
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  // scale atoms per 128-row group: 4 scales each, of 32 (MXFP4) or 16 (NVFP4) elements
+  const uint32_t n_katoms = (uint32_t)sf_katoms(NV ? 2 * K : K);
   return cudaLaunchKernelEx(&cfg, kern, map, (uint32_t)rows, (uint32_t)rows_pad,
-                            (uint32_t)kb_real, (uint32_t)k_boxes, (uint32_t)tiles,
-                            (uint32_t)sf_katoms(K), (uint64_t)(K / 2), kc, q, sf, status);
+                            (uint32_t)kb_real, (uint32_t)k_boxes, (uint32_t)tiles, n_katoms,
+                            (uint64_t)(K / 2), kc, q, sf, status, tensor_scale);
+}
+
+// NVFP4 tensor scale: amax of the (rotated) tensor by a grid-stride pass with one
+// atomicMax per warp on the fp32 bits (non-negative floats order like their bits, and
+// max is order-free, so the result is deterministic), then st = amax / (6 * 448).
+template <int MODE, bool F32_IN>
+__global__ void __launch_bounds__(256) nvfp4_amax_kernel(const void* __restrict__ x, uint64_t ldx,
+                                                         uint32_t rows, uint32_t kb_real,
+                                                         unsigned int* __restrict__ amax_bits) {
+  const uint64_t n = (uint64_t)rows * kb_real;
+  float m = 0.0f;
+  for (uint64_t b = blockIdx.x * (uint64_t)blockDim.x + threadIdx.x; b < n;
+       b += (uint64_t)gridDim.x * blockDim.x) {
+    const uint64_t row = b / kb_real, kb = b - row * kb_real;
+    float2 P[16];
+    if constexpr (F32_IN) {
+      const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(x) +
+                                                          row * ldx + kb * 32u);
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const float4 w = __ldcs(src + c);
+        P[2 * c] = make_float2(w.x, w.y);
+        P[2 * c + 1] = make_float2(w.z, w.w);
+      }
+    } else {
+      const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(x) +
+                                                        row * ldx + kb * 32u);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const uint4 w = __ldcs(src + c);
+        P[4 * c + 0] = make_float2(bf16_lo(w.x), bf16_hi(w.x));
+        P[4 * c + 1] = make_float2(bf16_lo(w.y), bf16_hi(w.y));
+        P[4 * c + 2] = make_float2(bf16_lo(w.z), bf16_hi(w.z));
+        P[4 * c + 3] = make_float2(bf16_lo(w.w), bf16_hi(w.w));
+      }
+    }
+    if constexpr (MODE == 1) hadamard32(P);
+#pragma unroll
+    for (int j = 0; j < 16; ++j) m = fmaxf(m, fmaxf(fabsf(P[j].x), fabsf(P[j].y)));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((threadIdx.x & 31u) == 0) atomicMax(amax_bits, __float_as_uint(m));
+}
+
+__global__ void nvfp4_scale_finalize_kernel(float* __restrict__ scale2) {
+  const float amax = __uint_as_float(reinterpret_cast<unsigned int*>(scale2)[1]);
+  scale2[0] = __fdiv_rn(amax, 2688.0f);
 }
 
 }  // namespace
+
+cudaError_t launch_nvfp4_tensor_scale(const void* x, bool x_is_f32, int64_t rows, int64_t K,
+                                     int64_t ldx, int mode, float* scale2, cudaStream_t stream) {
+  // scale2[1] holds the amax bits during the pass, scale2[0] receives the scale
+  cudaError_t e = cudaMemsetAsync(scale2 + 1, 0, sizeof(float), stream);
+  if (e != cudaSuccess) return e;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const uint64_t blocks = (uint64_t)rows * (uint64_t)(K / 32);
+  uint64_t grid = (blocks + 255) / 256;
+  if (grid > (uint64_t)sms * 8) grid = (uint64_t)sms * 8;
+  if (grid == 0) grid = 1;
+  unsigned int* bits = reinterpret_cast<unsigned int*>(scale2 + 1);
+  if (x_is_f32) {
+    if (mode == 1)
+      nvfp4_amax_kernel<1, true><<<(unsigned)grid, 256, 0, stream>>>(x, ldx, rows, K / 32, bits);
+    else
+      nvfp4_amax_kernel<0, true><<<(unsigned)grid, 256, 0, stream>>>(x, ldx, rows, K / 32, bits);
+  } else {
+    if (mode == 1)
+      nvfp4_amax_kernel<1, false><<<(unsigned)grid, 256, 0, stream>>>(x, ldx, rows, K / 32, bits);
+    else
+      nvfp4_amax_kernel<0, false><<<(unsigned)grid, 256, 0, stream>>>(x, ldx, rows, K / 32, bits);
+  }
+  nvfp4_scale_finalize_kernel<<<1, 1, 0, stream>>>(scale2);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_nvfp4_quantize(const void* x, bool x_is_f32, int64_t rows, int64_t K,
+                                  int64_t ldx, int mode, const float* tensor_scale, uint8_t* q,
+                                  uint8_t* sf, int* status, cudaStream_t stream) {
+  const KronCoeffs k{};
+  if (x_is_f32)
+    return mode == 1 ? launch_mode<1, true, true>(x, rows, K, ldx, k, q, sf, status, stream,
+                                                  tensor_scale)
+                     : launch_mode<0, true, true>(x, rows, K, ldx, k, q, sf, status, stream,
+                                                  tensor_scale);
+  return mode == 1 ? launch_mode<1, false, true>(x, rows, K, ldx, k, q, sf, status, stream,
+                                                 tensor_scale)
+                   : launch_mode<0, false, true>(x, rows, K, ldx, k, q, sf, status, stream,
+                                                 tensor_scale);
+}
 
 cudaError_t launch_rotate_quantize(const void* x, bool x_is_f32, int64_t rows, int64_t K,
                                    int64_t ldx, int mode, const KronCoeffs* kc, uint8_t* q,
