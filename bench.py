@@ -91,6 +91,10 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="dit_b1", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--format", default="mxfp4", choices=["mxfp4", "nvfp4"],
+                    help="nvfp4: 16-element groups with E4M3 scales and a dynamic fp32 tensor "
+                         "scale per activation (mxfp4_nvfp4_linear); rotation none or "
+                         "Hadamard-32 only")
     ap.add_argument("--chain", action="store_true",
                     help="run the workload's linears as consecutive layers: each GEMM but the "
                          "last writes MXFP4 (mxfp4_gemm_quantize) that the next GEMM reads, "
@@ -283,13 +287,23 @@ def run_ours(args, rank, world, local_rank):
         A, B = synth.kron_factors(wl.seed)
     Aw, Bw = (mx.kron_weight_factors(A, B) if A is not None else (None, None))
 
+    nv = args.format == "nvfp4"
+    if nv and wl.rotation not in (synth.ROT_NONE, synth.ROT_HADAMARD32):
+        raise SystemExit("--format nvfp4: rotation none or Hadamard-32 only")
+    op_linear = mx.OP_NVFP4_LINEAR if nv else mx.OP_LINEAR
+
     # ---- inputs: weights prepared on the GPU (offline step, untimed)
     weights = []
     for lin in wl.linears:
         w = torch.from_numpy(synth.weight_f32(wl.seed, lin.N, lin.K, lin.layer)).to(dev)
-        wq, wsf = mx.rotate_quantize(w, wl.rotation, Aw, Bw)
+        if nv:
+            w_sc = mx.nvfp4_tensor_scale(w, wl.rotation)
+            wq, wsf = mx.nvfp4_quantize(w, w_sc, wl.rotation)
+            weights.append((wq, wsf, w_sc))
+        else:
+            wq, wsf = mx.rotate_quantize(w, wl.rotation, Aw, Bw)
+            weights.append((wq, wsf, None))
         del w
-        weights.append((wq, wsf))
     xs_host = rank_inputs(wl, rank)
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
 
@@ -297,7 +311,7 @@ def run_ours(args, rank, world, local_rank):
         xs = {k: torch.from_numpy(v.view(np.int16)).view(torch.bfloat16).to(dev)
               for k, v in xs_host.items()}
         ys = [torch.empty((l.M, l.N), dtype=torch.bfloat16, device=dev) for l in wl.linears]
-        wss = [mx.new_workspace(mx.workspace_bytes(mx.OP_LINEAR, l.M, l.N, l.K), dev)
+        wss = [mx.new_workspace(mx.workspace_bytes(op_linear, l.M, l.N, l.K), dev)
                for l in wl.linears]
         return xs, ys, wss
 
@@ -308,14 +322,14 @@ def run_ours(args, rank, world, local_rank):
 
     # Rotate through input/output sets and, when those are small (few tokens), through
     # copies of the weights too, so that no step finds its operands in L2.
-    w_bytes = sum(wq.numel() + wsf.numel() for wq, wsf in weights)
+    w_bytes = sum(wq.numel() + wsf.numel() for wq, wsf, _ in weights)
     sets = [make_set()]
     wsets = [weights]
     while len(sets) * set_bytes(sets[0]) + len(wsets) * w_bytes < 3 * l2:
         if len(sets) < 8 and set_bytes(sets[0]) >= w_bytes:
             sets.append(make_set())
         else:
-            wsets.append([(wq.clone(), wsf.clone()) for wq, wsf in weights])
+            wsets.append([(wq.clone(), wsf.clone(), sc) for wq, wsf, sc in weights])
     footprint = len(sets) * set_bytes(sets[0]) + len(wsets) * w_bytes
 
     stream = torch.cuda.current_stream(dev)
@@ -323,9 +337,13 @@ def run_ours(args, rank, world, local_rank):
     def step(i, s=stream):
         xs, ys, wss = sets[i % len(sets)]
         for j, lin in enumerate(wl.linears):
-            wq, wsf = wsets[i % len(wsets)][j]
-            mx.linear(xs[lin.x_tensor], wq, wsf, lin.N, wl.rotation, A, B, y=ys[j], ws=wss[j],
-                      stream=s)
+            wq, wsf, wsc = wsets[i % len(wsets)][j]
+            if nv:
+                mx.nvfp4_linear(xs[lin.x_tensor], wq, wsf, wsc, lin.N, wl.rotation, y=ys[j],
+                                ws=wss[j], stream=s)
+            else:
+                mx.linear(xs[lin.x_tensor], wq, wsf, lin.N, wl.rotation, A, B, y=ys[j],
+                          ws=wss[j], stream=s)
 
     def barrier():
         rank_barrier(world)
@@ -387,7 +405,9 @@ def run_ours(args, rank, world, local_rank):
     flops_step = wl.flops
     value = job_tflops(flops_step, args.steps, world, elapsed)
     ms_per_step = elapsed / args.steps * 1e3
-    launches = 2 * len(wl.linears) * args.steps
+    # kernels per linear: quantise + GEMM; NVFP4 adds the tensor-scale pass (2 kernels)
+    k_per_linear = 4 if nv else 2
+    launches = k_per_linear * len(wl.linears) * args.steps
 
     # status words: no bounded wait expired
     for s in sets:
@@ -398,7 +418,9 @@ def run_ours(args, rank, world, local_rank):
     # ---- attribution pass: the same steps as separate quantise / GEMM launches with
     # CUDA events around each kernel (on the launching stream)
     qbufs = [(torch.empty((l.M, l.K // 2), dtype=torch.uint8, device=dev),
-              torch.empty(mx.sf_bytes(l.M, l.K), dtype=torch.uint8, device=dev)) for l in wl.linears]
+              torch.empty(mx.nvfp4_sf_bytes(l.M, l.K) if nv else mx.sf_bytes(l.M, l.K),
+                          dtype=torch.uint8, device=dev),
+              torch.zeros(2, dtype=torch.float32, device=dev)) for l in wl.linears]
     gws = [mx.new_workspace(mx.workspace_bytes(mx.OP_GEMM, l.M, l.N, l.K), dev)
            for l in wl.linears]
     n_lin = len(wl.linears)
@@ -409,14 +431,23 @@ def run_ours(args, rank, world, local_rank):
     def step_split(i, rec):
         xs, ys, _ = sets[i % len(sets)]
         for j, lin in enumerate(wl.linears):
-            wq, wsf = wsets[i % len(wsets)][j]
-            q, sf = qbufs[j]
+            wq, wsf, wsc = wsets[i % len(wsets)][j]
+            q, sf, xsc = qbufs[j]
             if rec:
                 evs[i][j][0].record(stream)
-            mx.rotate_quantize(xs[lin.x_tensor], wl.rotation, A, B, q=q, sf=sf, stream=stream)
+            if nv:
+                mx.nvfp4_tensor_scale(xs[lin.x_tensor], wl.rotation, scale2=xsc, stream=stream)
+                mx.nvfp4_quantize(xs[lin.x_tensor], xsc, wl.rotation, q=q, sf=sf, stream=stream)
+            else:
+                mx.rotate_quantize(xs[lin.x_tensor], wl.rotation, A, B, q=q, sf=sf,
+                                   stream=stream)
             if rec:
                 evs[i][j][1].record(stream)
-            mx.gemm(q, sf, wq, wsf, lin.M, lin.N, lin.K, y=ys[j], ws=gws[j], stream=stream)
+            if nv:
+                mx.nvfp4_gemm(q, sf, xsc, wq, wsf, wsc, lin.M, lin.N, lin.K, y=ys[j], ws=gws[j],
+                              stream=stream)
+            else:
+                mx.gemm(q, sf, wq, wsf, lin.M, lin.N, lin.K, y=ys[j], ws=gws[j], stream=stream)
             if rec:
                 evs[i][j][2].record(stream)
 
@@ -437,9 +468,11 @@ def run_ours(args, rank, world, local_rank):
     t_q /= n_attr
     t_g /= n_attr
     gemm_flops = np.array([l.flops for l in wl.linears], dtype=np.float64)
-    gemm_bytes = np.array([l.M * l.K // 2 + mx.sf_bytes(l.M, l.K) + l.N * l.K // 2 +
-                           mx.sf_bytes(l.N, l.K) + 2 * l.M * l.N for l in wl.linears], np.float64)
-    q_bytes = np.array([2 * l.M * l.K + l.M * l.K // 2 + mx.sf_bytes(l.M, l.K)
+    sfb = mx.nvfp4_sf_bytes if nv else mx.sf_bytes
+    gemm_bytes = np.array([l.M * l.K // 2 + sfb(l.M, l.K) + l.N * l.K // 2 +
+                           sfb(l.N, l.K) + 2 * l.M * l.N for l in wl.linears], np.float64)
+    # NVFP4's dynamic tensor scale needs a full pass over X before the quantiser reads it
+    q_bytes = np.array([(4 if nv else 2) * l.M * l.K + l.M * l.K // 2 + sfb(l.M, l.K)
                         for l in wl.linears], np.float64)
     fp4_peak = peaks["bf16_tflops_sustained"] * FP4_OVER_BF16
     q_ach = q_bytes.sum() / t_q.sum() / 1e9
@@ -451,8 +484,9 @@ def run_ours(args, rank, world, local_rank):
     g_src = f"{PKG}/csrc/gemm_smallm.cu" if few_rows else f"{PKG}/csrc/gemm.cu"
     ridge = fp4_peak * 1e12 / (peaks["hbm_gbs"] * 1e9)
     intensity = gemm_flops.sum() / gemm_bytes.sum()
-    traffic = ncu_traffic(wl.name, g_src)
-    q_traffic = ncu_traffic(wl.name, f"{PKG}/csrc/quantize.cu", NCU_TRAFFIC_QUANTIZE)
+    traffic = None if nv else ncu_traffic(wl.name, g_src)
+    q_traffic = None if nv else ncu_traffic(wl.name, f"{PKG}/csrc/quantize.cu",
+                                            NCU_TRAFFIC_QUANTIZE)
     if intensity >= ridge:
         roofline = {"bound": "tensor", "achieved": gemm_flops.sum() / t_g.sum() / 1e12,
                     "peak": fp4_peak, "unit": "TFLOP/s",
@@ -488,9 +522,13 @@ def run_ours(args, rank, world, local_rank):
             for k, t in xs_pin.items():
                 xs_d[k].copy_(t, non_blocking=True)
             for j, lin in enumerate(wl.linears):
-                wq, wsf = wsets[i % len(wsets)][j]
-                mx.linear(xs_d[lin.x_tensor], wq, wsf, lin.N, wl.rotation, A, B, y=ys_d[j],
-                          ws=wss_d[j], stream=stream)
+                wq, wsf, wsc = wsets[i % len(wsets)][j]
+                if nv:
+                    mx.nvfp4_linear(xs_d[lin.x_tensor], wq, wsf, wsc, lin.N, wl.rotation,
+                                    y=ys_d[j], ws=wss_d[j], stream=stream)
+                else:
+                    mx.linear(xs_d[lin.x_tensor], wq, wsf, lin.N, wl.rotation, A, B, y=ys_d[j],
+                              ws=wss_d[j], stream=stream)
                 ys_pin[j].copy_(ys_d[j], non_blocking=True)
 
         e2e_step(0)
@@ -508,14 +546,16 @@ def run_ours(args, rank, world, local_rank):
         e2e = {"value": job_tflops(flops_step, args.e2e_steps, world, t_e2e), "unit": UNIT,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "ms_per_step": t_e2e / args.e2e_steps * 1e3, "steps": args.e2e_steps,
-               "gpu_launches": 2 * len(wl.linears) * args.e2e_steps}
+               "gpu_launches": k_per_linear * len(wl.linears) * args.e2e_steps}
 
     result = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "mxfp4",
-        "dtype_detail": "E2M1 x E2M1 with E8M0 block-32 scales, fp32 accumulate, bf16 out; "
-                        "rotation in fp32",
+        "scaling": "weak", "vs_baseline": None, "dtype": args.format,
+        "dtype_detail": ("E2M1 x E2M1 with E4M3 group-16 scales and fp32 tensor scales (dynamic "
+                         "for X), fp32 accumulate, bf16 out; rotation in fp32" if nv else
+                         "E2M1 x E2M1 with E8M0 block-32 scales, fp32 accumulate, bf16 out; "
+                         "rotation in fp32"),
         "data": "synthetic (seeded N(0,1) activations with outlier channels, N(0,0.02^2) weights)",
         "config": {"workload": workload_desc(wl), "tokens_per_gpu": wl.linears[0].M,
                    "gflop_per_step_per_gpu": flops_step / 1e9, "parallelism": f"replicas x{world} "
@@ -526,7 +566,8 @@ def run_ours(args, rank, world, local_rank):
                          f"copies, footprint {footprint / 2**20:.0f} MiB >= 3 x L2 "
                          f"({l2 / 2**20:.0f} MiB)"},
         "roofline": roofline,
-        "quantize_roofline": {"bound": "hbm", "kernel": "rotate_quantize_kernel",
+        "quantize_roofline": {"bound": "hbm", "kernel": "nvfp4_amax_kernel + rotate_quantize_kernel"
+                              if nv else "rotate_quantize_kernel",
                               "achieved": q_ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                               "frac": q_ach / peaks["hbm_gbs"],
                               "per_launch_us": [t * 1e6 for t in t_q],
@@ -537,7 +578,7 @@ def run_ours(args, rank, world, local_rank):
                                                      if q_traffic else None)},
         "e2e": e2e,
         "gpu_launches": launches,
-        "attribution": {"steps": n_attr, "gpu_launches": 2 * n_lin * n_attr,
+        "attribution": {"steps": n_attr, "gpu_launches": k_per_linear * n_lin * n_attr,
                         "note": "quantise and GEMM launched separately with CUDA events "
                                 "around each kernel; source of both roofline objects"},
         "clocks": clk,
