@@ -65,6 +65,9 @@ def _load():
             "oracle_nvfp4_rotate_quantize": ([vp, i32, i64, i64, i64, i32, ctypes.c_float, vp,
                                               vp], None),
             "oracle_nvfp4_gemm": ([vp, vp, vp, vp, i64, i64, i64, dbl, vp, vp], None),
+            "oracle_row_stats": ([vp, i32, i64, i64, i64, i32, dbl, vp, vp], None),
+            "oracle_norm_rotate_quantize": ([vp, i32, i64, i64, i64, vp, vp, vp, vp, i32, vp,
+                                             vp, vp, vp], None),
             "oracle_dequantize": ([vp, vp, i64, i64, vp], None),
             "oracle_gemm_pairs": ([vp, vp, vp, vp, i64, vp, vp, i64, vp, vp], None),
             "oracle_gemm": ([vp, vp, vp, vp, i64, i64, i64, vp, vp], None),
@@ -261,6 +264,48 @@ def prepare_weight(w_f32: np.ndarray, mode: int, A=None, B=None):
         At, Bt = kron_weight_factors(A, B)
         return rotate_quantize(w_f32, mode, At, Bt, bf16=False)
     return rotate_quantize(w_f32, mode, None, None, bf16=False)
+
+
+# ---------------------------------------------------------------- norm prologue
+
+NORM_LAYER, NORM_RMS = 0, 1
+
+
+def row_stats(x: np.ndarray, kind: int, eps: float, bf16: bool | None = None):
+    """Exact-arithmetic row statistics in double: (mu, rstd) per row (LayerNorm: mean and
+    1 / sqrt(var + eps); RMSNorm: 0 and 1 / sqrt(mean(x^2) + eps))."""
+    if bf16 is None:
+        bf16 = x.dtype == np.uint16
+    x = _c(x, np.uint16 if bf16 else np.float32)
+    rows, K = x.shape
+    mu = np.empty(rows, np.float64)
+    rstd = np.empty(rows, np.float64)
+    _load().oracle_row_stats(_p(x), 0 if bf16 else 1, rows, K, K, int(kind), float(eps), _p(mu),
+                             _p(rstd))
+    return mu, rstd
+
+
+def norm_rotate_quantize(x: np.ndarray, mu_f32, rstd_f32, g, b, mode: int, A=None, B=None,
+                         bf16: bool | None = None):
+    """v = ((x - mu) * rstd) * g + b in fp32 with the given fp32 statistics, then
+    rotate-quantise like rotate_quantize (modes 0, 1, 2)."""
+    if bf16 is None:
+        bf16 = x.dtype == np.uint16
+    x = _c(x, np.uint16 if bf16 else np.float32)
+    rows, K = x.shape
+    mu = _c(mu_f32, np.float32)
+    rs = _c(rstd_f32, np.float32)
+    gg = _c(g, np.float32) if g is not None else None
+    bb = _c(b, np.float32) if b is not None else None
+    A = _c(A if A is not None else np.eye(4), np.float32)
+    B = _c(B if B is not None else np.eye(8), np.float32)
+    q = np.empty((rows, K // 2), np.uint8)
+    s = np.empty((rows, K // 32), np.uint8)
+    _load().oracle_norm_rotate_quantize(_p(x), 0 if bf16 else 1, rows, K, K, _p(mu), _p(rs),
+                                        _p(gg) if gg is not None else None,
+                                        _p(bb) if bb is not None else None, int(mode), _p(A),
+                                        _p(B), _p(q), _p(s))
+    return q, s
 
 
 # ---------------------------------------------------------------- NVFP4

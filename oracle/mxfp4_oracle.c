@@ -555,3 +555,63 @@ void oracle_nvfp4_gemm(const uint8_t* aq, const uint8_t* as, const uint8_t* bq,
       S[m * N + n] = fabs(alpha) * mag;
     }
 }
+
+/* ------------------------------------------------------- norm prologue (row f3)
+ *
+ * The step right before the rotation ("KroQuant: Effiziente Post-Training-Quantisierung
+ * fuer Diffusion Transformers mittels Kronecker-Produkt-Struktur", "Hintergrund": the
+ * normalisation layers are why the transform has to run online). Two norms:
+ *   kind 0 (LayerNorm): mu = mean(x), var = mean((x - mu)^2), rstd = 1 / sqrt(var + eps);
+ *   kind 1 (RMSNorm):   mu = 0, rstd = 1 / sqrt(mean(x^2) + eps);
+ * then, per element, v = ((x - mu) * rstd) * g[c] + b[c] (g = 1 and b = 0 when absent),
+ * before the rotation and quantisation. The statistics are defined in exact arithmetic
+ * and computed here in double; the per-element steps are fp32 operations in the order
+ * written (sub, mul, mul, add), so that given the fp32 statistics a GPU used, the codes
+ * follow bit for bit. */
+void oracle_row_stats(const void* x, int xdt, int64_t rows, int64_t K, int64_t ldx, int kind,
+                      double eps, double* mu, double* rstd) {
+  for (int64_t r = 0; r < rows; ++r) {
+    double s = 0.0, m = 0.0, v = 0.0;
+    for (int64_t k = 0; k < K; ++k) {
+      const int64_t idx = r * ldx + k;
+      s += xdt == 0 ? bf16_to_f32(((const uint16_t*)x)[idx]) : ((const float*)x)[idx];
+    }
+    if (kind == 0) m = s / (double)K;
+    for (int64_t k = 0; k < K; ++k) {
+      const int64_t idx = r * ldx + k;
+      const double d = (xdt == 0 ? bf16_to_f32(((const uint16_t*)x)[idx])
+                                 : ((const float*)x)[idx]) - m;
+      v += d * d;
+    }
+    mu[r] = m;
+    rstd[r] = 1.0 / sqrt(v / (double)K + eps);
+  }
+}
+
+/* Normalise with the given fp32 statistics (mu_f, rstd_f per row), then rotate-quantise
+ * (modes 0, 1, 2) into q[rows, K/2], s[rows, K/32] (logical layout). */
+void oracle_norm_rotate_quantize(const void* x, int xdt, int64_t rows, int64_t K, int64_t ldx,
+                                 const float* mu_f, const float* rstd_f, const float* g,
+                                 const float* bvec, int mode, const float* A, const float* B,
+                                 uint8_t* q, uint8_t* s) {
+  const int64_t nb = K / 32;
+#pragma omp parallel for schedule(static)
+  for (int64_t r = 0; r < rows; ++r) {
+    float xin[32], y[32];
+    uint8_t codes[32];
+    for (int64_t b = 0; b < nb; ++b) {
+      for (int i = 0; i < 32; ++i) {
+        const int64_t c = 32 * b + i, idx = r * ldx + c;
+        const float xv = xdt == 0 ? bf16_to_f32(((const uint16_t*)x)[idx]) : ((const float*)x)[idx];
+        float v = (xv - mu_f[r]) * rstd_f[r];
+        if (g) v = v * g[c];
+        if (bvec) v = v + bvec[c];
+        xin[i] = v;
+      }
+      oracle_rotate_blocks(xin, 1, mode, A, B, y);
+      oracle_quantize_block(y, codes, s + r * nb + b);
+      for (int j = 0; j < 16; ++j)
+        q[r * (K / 2) + 16 * b + j] = (uint8_t)(codes[2 * j] | (codes[2 * j + 1] << 4));
+    }
+  }
+}
