@@ -88,8 +88,11 @@ typedef enum {
   MXFP4_OP_QUANTIZE = 0,
   MXFP4_OP_GEMM = 1, /* also mxfp4_gemm_bias, mxfp4_gemm_quantize, mxfp4_nvfp4_gemm */
   MXFP4_OP_LINEAR = 2,
-  MXFP4_OP_NVFP4_LINEAR = 3
+  MXFP4_OP_NVFP4_LINEAR = 3,
+  MXFP4_OP_NORM_LINEAR = 4
 } mxfp4_op;
+
+typedef enum { MXFP4_NORM_LAYER = 0, MXFP4_NORM_RMS = 1 } mxfp4_norm;
 
 /* A cudaStream_t, passed as an opaque handle so this header needs no CUDA headers. */
 typedef void* mxfp4_stream_t;
@@ -217,6 +220,34 @@ mxfp4_status mxfp4_linear(const void* x, int64_t M, int64_t K, mxfp4_rotation mo
                           const float* kron_a, const float* kron_b, const uint8_t* wq,
                           const uint8_t* wsf, int64_t N, void* y, void* ws, size_t ws_bytes,
                           mxfp4_stream_t stream);
+
+/*
+ * Norm prologue: the normalisation that precedes the layer, applied inside the
+ * quantiser instead of as a separate pass that writes a normalised bf16 copy
+ * of x ("KroQuant...", "Hintergrund": the norms are why the transform runs
+ * online). A first kernel computes per-row statistics into stats (DEVICE,
+ * [rows][2] fp32, 8-byte aligned; also an output): LayerNorm mu = mean,
+ * rstd = 1 / sqrt(var + eps); RMSNorm mu = 0, rstd = 1 / sqrt(mean(x^2) + eps)
+ * (fp32 sums over the row). The quantiser then rotates and quantises
+ * v = ((x - mu) * rstd) * g[c] + b[c] (fp32, in that order; g / b: DEVICE fp32
+ * [K], 16-byte aligned, NULL for 1 / 0 -- for adaLN modulation pass
+ * g = 1 + scale and b = shift). x is bf16; modes NONE / HADAMARD32 / KRON_4x8;
+ * otherwise as mxfp4_rotate_quantize.
+ */
+mxfp4_status mxfp4_norm_rotate_quantize(const void* x, int64_t rows, int64_t K, int64_t ldx,
+                                        mxfp4_norm kind, float eps, const float* g,
+                                        const float* b, mxfp4_rotation mode, const float* kron_a,
+                                        const float* kron_b, uint8_t* q, uint8_t* sf,
+                                        float* stats, mxfp4_stream_t stream);
+
+/* The layer with the norm prologue: mxfp4_norm_rotate_quantize into the
+ * workspace, then the GEMM as in mxfp4_linear. ws: mxfp4_workspace_bytes(
+ * MXFP4_OP_NORM_LINEAR, M, N, K) bytes, zeroed at allocation. */
+mxfp4_status mxfp4_norm_linear(const void* x, int64_t M, int64_t K, mxfp4_norm kind, float eps,
+                               const float* g, const float* b, mxfp4_rotation mode,
+                               const float* kron_a, const float* kron_b, const uint8_t* wq,
+                               const uint8_t* wsf, int64_t N, void* y, void* ws,
+                               size_t ws_bytes, mxfp4_stream_t stream);
 
 /*
  * NVFP4, the other FP4 format the pages compare ("Bridging the Gap Between

@@ -22,14 +22,15 @@ LIB_PATH = os.path.join(_HERE, "libmxfp4.so")
 OK, ERR_INVALID_ARG, ERR_SHAPE, ERR_ALIGN, ERR_WORKSPACE, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT = range(8)
 ROT_NONE, ROT_HADAMARD32, ROT_KRON_4x8, ROT_HADAMARD64, ROT_HADAMARD128 = 0, 1, 2, 3, 4
 DT_BF16, DT_F32 = 0, 1
-OP_QUANTIZE, OP_GEMM, OP_LINEAR, OP_NVFP4_LINEAR = 0, 1, 2, 3
+OP_QUANTIZE, OP_GEMM, OP_LINEAR, OP_NVFP4_LINEAR, OP_NORM_LINEAR = 0, 1, 2, 3, 4
+NORM_LAYER, NORM_RMS = 0, 1
 
 EXPORTS = (
     "mxfp4_sf_bytes", "mxfp4_sf_offset", "mxfp4_workspace_bytes", "mxfp4_status_string",
     "mxfp4_quantize", "mxfp4_rotate_quantize", "mxfp4_gemm", "mxfp4_linear",
     "mxfp4_poll_status", "mxfp4_linear_noalloc", "mxfp4_gemm_bias", "mxfp4_gemm_quantize",
     "mxfp4_nvfp4_sf_bytes", "mxfp4_nvfp4_tensor_scale", "mxfp4_nvfp4_quantize",
-    "mxfp4_nvfp4_gemm", "mxfp4_nvfp4_linear",
+    "mxfp4_nvfp4_gemm", "mxfp4_nvfp4_linear", "mxfp4_norm_rotate_quantize", "mxfp4_norm_linear",
 )
 
 
@@ -66,6 +67,10 @@ def _load() -> ctypes.CDLL:
         "mxfp4_nvfp4_gemm": ([vp, vp, vp, vp, vp, vp, i64, i64, i64, vp, i32, i64, vp, sz, vp],
                              i32),
         "mxfp4_nvfp4_linear": ([vp, i64, i64, i32, vp, vp, vp, i64, vp, vp, sz, vp], i32),
+        "mxfp4_norm_rotate_quantize": ([vp, i64, i64, i64, i32, ctypes.c_float, vp, vp, i32, vp,
+                                        vp, vp, vp, vp, vp], i32),
+        "mxfp4_norm_linear": ([vp, i64, i64, i32, ctypes.c_float, vp, vp, i32, vp, vp, vp, vp,
+                               i64, vp, vp, sz, vp], i32),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -221,6 +226,55 @@ def gemm_quantize(aq, asf, bq, bsf, M: int, N: int, K: int, bias=None,
                                  _stream_handle(stream))
     _check(st, "mxfp4_gemm_quantize")
     return yq, ysf
+
+
+# ---------------------------------------------------------------- norm prologue
+
+def norm_rotate_quantize(x, kind: int = NORM_LAYER, eps: float = 1e-6, g=None, b=None,
+                         mode: int = ROT_HADAMARD32, kron_a=None, kron_b=None, q=None, sf=None,
+                         stats=None, stream=None):
+    """Normalise each bf16 row (LayerNorm / RMSNorm statistics, then * g + b), rotate and
+    quantise. Returns (q, sf, stats [rows, 2] fp32: mu, rstd)."""
+    torch = _torch()
+    assert x.dim() == 2 and x.stride(1) == 1 and x.dtype == torch.bfloat16
+    rows, K = x.shape
+    if q is None:
+        q = torch.empty((rows, K // 2), dtype=torch.uint8, device=x.device)
+    if sf is None:
+        sf = torch.empty(max(sf_bytes(rows, K), 16), dtype=torch.uint8, device=x.device)
+    if stats is None:
+        stats = torch.empty((rows, 2), dtype=torch.float32, device=x.device)
+    a = _host_f32(kron_a, 16) if mode == ROT_KRON_4x8 else None
+    bb = _host_f32(kron_b, 64) if mode == ROT_KRON_4x8 else None
+    st = lib.mxfp4_norm_rotate_quantize(x.data_ptr(), rows, K, x.stride(0), kind, eps,
+                                        g.data_ptr() if g is not None else None,
+                                        b.data_ptr() if b is not None else None, mode, a, bb,
+                                        q.data_ptr(), sf.data_ptr(), stats.data_ptr(),
+                                        _stream_handle(stream))
+    _check(st, "mxfp4_norm_rotate_quantize")
+    return q, sf, stats
+
+
+def norm_linear(x, wq, wsf, N: int, kind: int = NORM_LAYER, eps: float = 1e-6, g=None, b=None,
+                mode: int = ROT_HADAMARD32, kron_a=None, kron_b=None, y=None, ws=None,
+                stream=None):
+    """The layer with the norm prologue (bf16 x in, bf16 y out)."""
+    torch = _torch()
+    assert x.dim() == 2 and x.is_contiguous() and x.dtype == torch.bfloat16
+    M, K = x.shape
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    if ws is None:
+        ws = new_workspace(workspace_bytes(OP_NORM_LINEAR, M, N, K), x.device)
+    a = _host_f32(kron_a, 16) if mode == ROT_KRON_4x8 else None
+    bb = _host_f32(kron_b, 64) if mode == ROT_KRON_4x8 else None
+    st = lib.mxfp4_norm_linear(x.data_ptr(), M, K, kind, eps,
+                               g.data_ptr() if g is not None else None,
+                               b.data_ptr() if b is not None else None, mode, a, bb,
+                               wq.data_ptr(), wsf.data_ptr(), N, y.data_ptr(), ws.data_ptr(),
+                               ws.numel(), _stream_handle(stream))
+    _check(st, "mxfp4_norm_linear")
+    return y
 
 
 # ---------------------------------------------------------------- NVFP4

@@ -84,6 +84,22 @@ LinearWorkspace nvfp4_linear_workspace(int64_t M, int64_t N, int64_t K) {
   return w;
 }
 
+// Workspace of mxfp4_norm_linear: [status | Xq | Xsf | row statistics (M x 8 bytes) |
+// GEMM scratch]; g_off of the returned value is the GEMM scratch, stats sit before it.
+struct NormWorkspace {
+  size_t q_off, sf_off, st_off, g_off, total;
+};
+
+NormWorkspace norm_linear_workspace(int64_t M, int64_t N, int64_t K) {
+  NormWorkspace w;
+  w.q_off = kStatusBytes;
+  w.sf_off = round_up(w.q_off + (size_t)M * (size_t)(K / 2), 256);
+  w.st_off = round_up(w.sf_off + mxfp4_sf_bytes(M, K), 256);
+  w.g_off = round_up(w.st_off + (size_t)M * 2 * sizeof(float), 256);
+  w.total = round_up(w.g_off + gemm_scratch_bytes(M, N, K), 256);
+  return w;
+}
+
 LinearWorkspace linear_workspace(int64_t M, int64_t N, int64_t K) {
   LinearWorkspace w;
   w.q_off = kStatusBytes;
@@ -122,6 +138,9 @@ size_t mxfp4_workspace_bytes(int op, int64_t M, int64_t N, int64_t K) {
     case MXFP4_OP_NVFP4_LINEAR:
       if (!shape_ok(M, K) || N < 0) return 0;
       return nvfp4_linear_workspace(M, N, K).total;
+    case MXFP4_OP_NORM_LINEAR:
+      if (!shape_ok(M, K) || N < 0) return 0;
+      return norm_linear_workspace(M, N, K).total;
     default:
       return 0;
   }
@@ -256,6 +275,62 @@ mxfp4_status mxfp4_linear(const void* x, int64_t M, int64_t K, mxfp4_rotation mo
   // The kernel just before the GEMM is the quantiser above, which does not write W.
   return from_cuda(launch_gemm(xq, xsf, wq, wsf, M, N, K, y, Epilogue{}, N, static_cast<int*>(ws),
                                base + w.g_off, ws_bytes - w.g_off, true, s));
+}
+
+mxfp4_status mxfp4_norm_rotate_quantize(const void* x, int64_t rows, int64_t K, int64_t ldx,
+                                        mxfp4_norm kind, float eps, const float* g,
+                                        const float* b, mxfp4_rotation mode, const float* kron_a,
+                                        const float* kron_b, uint8_t* q, uint8_t* sf,
+                                        float* stats, mxfp4_stream_t stream) {
+  mxfp4_status st = validate_quantize(x, MXFP4_DT_BF16, rows, K, ldx, q, sf);
+  if (st != MXFP4_OK) return st;
+  if (!stats) return MXFP4_ERR_INVALID_ARG;
+  if (kind != MXFP4_NORM_LAYER && kind != MXFP4_NORM_RMS) return MXFP4_ERR_UNSUPPORTED;
+  if (mode != MXFP4_ROT_NONE && mode != MXFP4_ROT_HADAMARD32 && mode != MXFP4_ROT_KRON_4x8)
+    return MXFP4_ERR_UNSUPPORTED;
+  if (!(eps >= 0.0f)) return MXFP4_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(stats) & 7u) || (g && !aligned16(g)) || (b && !aligned16(b)))
+    return MXFP4_ERR_ALIGN;
+  KronCoeffs kc{};
+  if (mode == MXFP4_ROT_KRON_4x8 && !kron_from_host(kron_a, kron_b, &kc))
+    return MXFP4_ERR_INVALID_ARG;
+  if (rows == 0) return MXFP4_OK;
+  return from_cuda(launch_norm_rotate_quantize(x, rows, K, ldx, (int)kind, eps, g, b, (int)mode,
+                                               &kc, q, sf, stats, nullptr,
+                                               static_cast<cudaStream_t>(stream)));
+}
+
+mxfp4_status mxfp4_norm_linear(const void* x, int64_t M, int64_t K, mxfp4_norm kind, float eps,
+                               const float* g, const float* b, mxfp4_rotation mode,
+                               const float* kron_a, const float* kron_b, const uint8_t* wq,
+                               const uint8_t* wsf, int64_t N, void* y, void* ws,
+                               size_t ws_bytes, mxfp4_stream_t stream) {
+  if (!x || !wq || !wsf || !y || !ws) return MXFP4_ERR_INVALID_ARG;
+  if (kind != MXFP4_NORM_LAYER && kind != MXFP4_NORM_RMS) return MXFP4_ERR_UNSUPPORTED;
+  if (mode != MXFP4_ROT_NONE && mode != MXFP4_ROT_HADAMARD32 && mode != MXFP4_ROT_KRON_4x8)
+    return MXFP4_ERR_UNSUPPORTED;
+  if (!(eps >= 0.0f)) return MXFP4_ERR_INVALID_ARG;
+  if (!shape_ok(M, K) || N < 16 || N % 16 != 0 || !within_limits(M, K) || !within_limits(N, K))
+    return MXFP4_ERR_SHAPE;
+  if (!aligned16(x) || !aligned16(wq) || !aligned16(wsf) || !aligned16(y) || !aligned16(ws) ||
+      (g && !aligned16(g)) || (b && !aligned16(b)) || (K * 2) % 16 != 0 || (N * 2) % 16 != 0)
+    return MXFP4_ERR_ALIGN;
+  const NormWorkspace w = norm_linear_workspace(M, N, K);
+  if (ws_bytes < w.total) return MXFP4_ERR_WORKSPACE;
+  KronCoeffs kc{};
+  if (mode == MXFP4_ROT_KRON_4x8 && !kron_from_host(kron_a, kron_b, &kc))
+    return MXFP4_ERR_INVALID_ARG;
+  if (M == 0) return MXFP4_OK;
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_norm_rotate_quantize(
+      x, M, K, K, (int)kind, eps, g, b, (int)mode, &kc, base + w.q_off, base + w.sf_off,
+      reinterpret_cast<float*>(base + w.st_off), static_cast<int*>(ws), s);
+  if (e != cudaSuccess) return MXFP4_ERR_CUDA;
+  // The kernel just before the GEMM is the quantiser above, which does not write W.
+  return from_cuda(launch_gemm(base + w.q_off, base + w.sf_off, wq, wsf, M, N, K, y, Epilogue{},
+                               N, static_cast<int*>(ws), base + w.g_off, ws_bytes - w.g_off, true,
+                               s));
 }
 
 size_t mxfp4_nvfp4_sf_bytes(int64_t rows, int64_t K) {

@@ -52,12 +52,19 @@ struct TileShape {
   static constexpr uint32_t SMEM = kStages * STAGE + 64 + 1024;
 };
 
-template <int MODE, bool F32_IN, bool NV>
+// Norm prologue (per-row statistics from row_stats_kernel, optional g / b of length K).
+struct NormArgs {
+  const float* stats;  // [rows][2]: mu, rstd
+  const float* g;      // or null (1)
+  const float* b;      // or null (0)
+};
+
+template <int MODE, bool F32_IN, bool NV, bool NORM = false>
 __global__ void __launch_bounds__(kThreads) rotate_quantize_kernel(
     const __grid_constant__ CUtensorMap tmap_x, uint32_t rows, uint32_t rows_pad, uint32_t kb_real,
     uint32_t k_boxes, uint32_t tiles, uint32_t n_katoms, uint64_t q_row_bytes,
     const __grid_constant__ KronCoeffs kc, uint8_t* __restrict__ q, uint8_t* __restrict__ sf,
-    int* status, const float* __restrict__ tensor_scale) {
+    int* status, const float* __restrict__ tensor_scale, const NormArgs norm) {
   using namespace sm100;
   using T = TileShape<F32_IN>;
   constexpr int CH = F32_IN ? 8 : 4;  // 16-byte chunks per 32-element block
@@ -162,6 +169,23 @@ __global__ void __launch_bounds__(kThreads) rotate_quantize_kernel(
       } else {
         uint32_t byte = 0;
         if (row < rows && kb < kb_real) {
+          if constexpr (NORM) {
+            // v = ((x - mu) * rstd) * g + b, each an fp32 operation in that order
+            const float2 st = __ldg(reinterpret_cast<const float2*>(norm.stats) + row);
+            const float2 nmu = make_float2(-st.x, -st.x), rs = make_float2(st.y, st.y);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) P[j] = __fmul2_rn(__fadd2_rn(P[j], nmu), rs);
+            if (norm.g != nullptr) {
+              const float2* gv = reinterpret_cast<const float2*>(norm.g + kb * 32u);
+#pragma unroll
+              for (int j = 0; j < 16; ++j) P[j] = __fmul2_rn(P[j], __ldg(gv + j));
+            }
+            if (norm.b != nullptr) {
+              const float2* bv = reinterpret_cast<const float2*>(norm.b + kb * 32u);
+#pragma unroll
+              for (int j = 0; j < 16; ++j) P[j] = __fadd2_rn(P[j], __ldg(bv + j));
+            }
+          }
           if constexpr (MODE == 1) hadamard32(P);
           if constexpr (MODE == 2) kron32(P, kc);
           uint4 codes;
@@ -199,10 +223,10 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-template <int MODE, bool F32_IN, bool NV = false>
+template <int MODE, bool F32_IN, bool NV = false, bool NORM = false>
 cudaError_t launch_mode(const void* x, int64_t rows, int64_t K, int64_t ldx, const KronCoeffs& kc,
                         uint8_t* q, uint8_t* sf, int* status, cudaStream_t stream,
-                        const float* tensor_scale = nullptr) {
+                        const float* tensor_scale = nullptr, NormArgs norm = NormArgs{}) {
   using T = TileShape<F32_IN>;
   auto fn = encode_fn();
   if (!fn) return cudaErrorNotSupported;
@@ -217,7 +241,7 @@ cudaError_t launch_mode(const void* x, int64_t rows, int64_t K, int64_t ldx, con
          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
 
-  auto kern = rotate_quantize_kernel<MODE, F32_IN, NV>;
+  auto kern = rotate_quantize_kernel<MODE, F32_IN, NV, NORM>;
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
@@ -255,7 +279,7 @@ cudaError_t launch_mode(const void* x, int64_t rows, int64_t K, int64_t ldx, con
   const uint32_t n_katoms = (uint32_t)sf_katoms(NV ? 2 * K : K);
   return cudaLaunchKernelEx(&cfg, kern, map, (uint32_t)rows, (uint32_t)rows_pad,
                             (uint32_t)kb_real, (uint32_t)k_boxes, (uint32_t)tiles, n_katoms,
-                            (uint64_t)(K / 2), kc, q, sf, status, tensor_scale);
+                            (uint64_t)(K / 2), kc, q, sf, status, tensor_scale, norm);
 }
 
 // NVFP4 tensor scale: amax of the (rotated) tensor by a grid-stride pass with one
@@ -301,12 +325,90 @@ __global__ void __launch_bounds__(256) nvfp4_amax_kernel(const void* __restrict_
   if ((threadIdx.x & 31u) == 0) atomicMax(amax_bits, __float_as_uint(m));
 }
 
+// Norm prologue statistics: one warp per bf16 row, two passes (sum, then squared
+// deviations; RMSNorm: squares), fp32 sums, mu = sum / K, rstd = 1 / sqrt(var + eps)
+// correctly rounded. The quantiser applies them; the oracle checks them against exact
+// arithmetic and repeats the per-element steps with these fp32 values.
+template <int KIND>
+__global__ void __launch_bounds__(256) row_stats_kernel(const uint16_t* __restrict__ x,
+                                                        uint64_t ldx, uint32_t rows, uint32_t K,
+                                                        float eps, float* __restrict__ stats) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  const uint32_t lane = threadIdx.x & 31u;
+  const uint32_t row = blockIdx.x * 8u + (threadIdx.x >> 5);
+  if (row >= rows) return;
+  const uint16_t* xr = x + (uint64_t)row * ldx;
+  float mu = 0.0f;
+  if constexpr (KIND == 0) {
+    float s = 0.0f;
+    for (uint32_t k = lane * 8u; k < K; k += 256u) {
+      const uint4 w = __ldg(reinterpret_cast<const uint4*>(xr + k));
+      s += bf16_lo(w.x) + bf16_hi(w.x) + bf16_lo(w.y) + bf16_hi(w.y) + bf16_lo(w.z) +
+           bf16_hi(w.z) + bf16_lo(w.w) + bf16_hi(w.w);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    mu = __fdiv_rn(s, (float)K);
+  }
+  float v = 0.0f;
+  for (uint32_t k = lane * 8u; k < K; k += 256u) {
+    const uint4 w = __ldg(reinterpret_cast<const uint4*>(xr + k));
+    const float e[8] = {bf16_lo(w.x), bf16_hi(w.x), bf16_lo(w.y), bf16_hi(w.y),
+                        bf16_lo(w.z), bf16_hi(w.z), bf16_lo(w.w), bf16_hi(w.w)};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float d = e[i] - mu;
+      v = __fmaf_rn(d, d, v);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  if (lane == 0) {
+    stats[2u * row] = mu;
+    stats[2u * row + 1u] = __frsqrt_rn(__fadd_rn(__fdiv_rn(v, (float)K), eps));
+  }
+}
+
 __global__ void nvfp4_scale_finalize_kernel(float* __restrict__ scale2) {
   const float amax = __uint_as_float(reinterpret_cast<unsigned int*>(scale2)[1]);
   scale2[0] = __fdiv_rn(amax, 2688.0f);
 }
 
 }  // namespace
+
+cudaError_t launch_norm_rotate_quantize(const void* x, int64_t rows, int64_t K, int64_t ldx,
+                                       int kind, float eps, const float* g, const float* b,
+                                       int mode, const KronCoeffs* kc, uint8_t* q, uint8_t* sf,
+                                       float* stats, int* status, cudaStream_t stream) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3((unsigned)((rows + 7) / 8));
+  cfg.blockDim = dim3(256);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const uint16_t* xb = static_cast<const uint16_t*>(x);
+  cudaError_t e =
+      kind == 1 ? cudaLaunchKernelEx(&cfg, row_stats_kernel<1>, xb, (uint64_t)ldx, (uint32_t)rows,
+                                     (uint32_t)K, eps, stats)
+                : cudaLaunchKernelEx(&cfg, row_stats_kernel<0>, xb, (uint64_t)ldx, (uint32_t)rows,
+                                     (uint32_t)K, eps, stats);
+  if (e != cudaSuccess) return e;
+  KronCoeffs k{};
+  if (kc) k = *kc;
+  const NormArgs na{stats, g, b};
+  if (mode == 1)
+    return launch_mode<1, false, false, true>(x, rows, K, ldx, k, q, sf, status, stream, nullptr,
+                                              na);
+  if (mode == 2)
+    return launch_mode<2, false, false, true>(x, rows, K, ldx, k, q, sf, status, stream, nullptr,
+                                              na);
+  return launch_mode<0, false, false, true>(x, rows, K, ldx, k, q, sf, status, stream, nullptr,
+                                            na);
+}
 
 cudaError_t launch_nvfp4_tensor_scale(const void* x, bool x_is_f32, int64_t rows, int64_t K,
                                      int64_t ldx, int mode, float* scale2, cudaStream_t stream) {
