@@ -95,6 +95,9 @@ def parse():
                     help="nvfp4: 16-element groups with E4M3 scales and a dynamic fp32 tensor "
                          "scale per activation (mxfp4_nvfp4_linear); rotation none or "
                          "Hadamard-32 only")
+    ap.add_argument("--norm", default="none", choices=["none", "layer", "rms"],
+                    help="apply a LayerNorm / RMSNorm prologue (with per-channel g and b) "
+                         "inside the quantiser: mxfp4_norm_linear")
     ap.add_argument("--chain", action="store_true",
                     help="run the workload's linears as consecutive layers: each GEMM but the "
                          "last writes MXFP4 (mxfp4_gemm_quantize) that the next GEMM reads, "
@@ -290,7 +293,17 @@ def run_ours(args, rank, world, local_rank):
     nv = args.format == "nvfp4"
     if nv and wl.rotation not in (synth.ROT_NONE, synth.ROT_HADAMARD32):
         raise SystemExit("--format nvfp4: rotation none or Hadamard-32 only")
-    op_linear = mx.OP_NVFP4_LINEAR if nv else mx.OP_LINEAR
+    norm = {"none": None, "layer": mx.NORM_LAYER, "rms": mx.NORM_RMS}[args.norm]
+    if norm is not None and nv:
+        raise SystemExit("--norm: MXFP4 format only")
+    op_linear = (mx.OP_NVFP4_LINEAR if nv else
+                 mx.OP_NORM_LINEAR if norm is not None else mx.OP_LINEAR)
+    # norm prologue: per-channel g (around 1) and b (around 0) of every linear's input
+    norm_gb = [(torch.from_numpy((1.0 + 0.1 * synth.normal_f32(wl.seed, 90 + j, (l.K,)))
+                                 .astype(np.float32)).to(dev),
+                torch.from_numpy((0.1 * synth.normal_f32(wl.seed, 95 + j, (l.K,)))
+                                 .astype(np.float32)).to(dev))
+               for j, l in enumerate(wl.linears)] if norm is not None else None
 
     # ---- inputs: weights prepared on the GPU (offline step, untimed)
     weights = []
@@ -341,6 +354,9 @@ def run_ours(args, rank, world, local_rank):
             if nv:
                 mx.nvfp4_linear(xs[lin.x_tensor], wq, wsf, wsc, lin.N, wl.rotation, y=ys[j],
                                 ws=wss[j], stream=s)
+            elif norm is not None:
+                mx.norm_linear(xs[lin.x_tensor], wq, wsf, lin.N, norm, 1e-6, norm_gb[j][0],
+                               norm_gb[j][1], wl.rotation, A, B, y=ys[j], ws=wss[j], stream=s)
             else:
                 mx.linear(xs[lin.x_tensor], wq, wsf, lin.N, wl.rotation, A, B, y=ys[j],
                           ws=wss[j], stream=s)
@@ -405,8 +421,9 @@ def run_ours(args, rank, world, local_rank):
     flops_step = wl.flops
     value = job_tflops(flops_step, args.steps, world, elapsed)
     ms_per_step = elapsed / args.steps * 1e3
-    # kernels per linear: quantise + GEMM; NVFP4 adds the tensor-scale pass (2 kernels)
-    k_per_linear = 4 if nv else 2
+    # kernels per linear: quantise + GEMM; NVFP4 adds the tensor-scale pass (2 kernels),
+    # the norm prologue the row-statistics kernel
+    k_per_linear = 4 if nv else 3 if norm is not None else 2
     launches = k_per_linear * len(wl.linears) * args.steps
 
     # status words: no bounded wait expired
@@ -420,7 +437,8 @@ def run_ours(args, rank, world, local_rank):
     qbufs = [(torch.empty((l.M, l.K // 2), dtype=torch.uint8, device=dev),
               torch.empty(mx.nvfp4_sf_bytes(l.M, l.K) if nv else mx.sf_bytes(l.M, l.K),
                           dtype=torch.uint8, device=dev),
-              torch.zeros(2, dtype=torch.float32, device=dev)) for l in wl.linears]
+              torch.zeros(2, dtype=torch.float32, device=dev),
+              torch.empty((l.M, 2), dtype=torch.float32, device=dev)) for l in wl.linears]
     gws = [mx.new_workspace(mx.workspace_bytes(mx.OP_GEMM, l.M, l.N, l.K), dev)
            for l in wl.linears]
     n_lin = len(wl.linears)
@@ -432,12 +450,16 @@ def run_ours(args, rank, world, local_rank):
         xs, ys, _ = sets[i % len(sets)]
         for j, lin in enumerate(wl.linears):
             wq, wsf, wsc = wsets[i % len(wsets)][j]
-            q, sf, xsc = qbufs[j]
+            q, sf, xsc, stt = qbufs[j]
             if rec:
                 evs[i][j][0].record(stream)
             if nv:
                 mx.nvfp4_tensor_scale(xs[lin.x_tensor], wl.rotation, scale2=xsc, stream=stream)
                 mx.nvfp4_quantize(xs[lin.x_tensor], xsc, wl.rotation, q=q, sf=sf, stream=stream)
+            elif norm is not None:
+                mx.norm_rotate_quantize(xs[lin.x_tensor], norm, 1e-6, norm_gb[j][0],
+                                        norm_gb[j][1], wl.rotation, A, B, q=q, sf=sf, stats=stt,
+                                        stream=stream)
             else:
                 mx.rotate_quantize(xs[lin.x_tensor], wl.rotation, A, B, q=q, sf=sf,
                                    stream=stream)
@@ -471,9 +493,10 @@ def run_ours(args, rank, world, local_rank):
     sfb = mx.nvfp4_sf_bytes if nv else mx.sf_bytes
     gemm_bytes = np.array([l.M * l.K // 2 + sfb(l.M, l.K) + l.N * l.K // 2 +
                            sfb(l.N, l.K) + 2 * l.M * l.N for l in wl.linears], np.float64)
-    # NVFP4's dynamic tensor scale needs a full pass over X before the quantiser reads it
-    q_bytes = np.array([(4 if nv else 2) * l.M * l.K + l.M * l.K // 2 + sfb(l.M, l.K)
-                        for l in wl.linears], np.float64)
+    # NVFP4's dynamic tensor scale, and the norm's row statistics, need a full pass over X
+    # before the quantiser reads it
+    q_bytes = np.array([(4 if nv or norm is not None else 2) * l.M * l.K + l.M * l.K // 2 +
+                        sfb(l.M, l.K) for l in wl.linears], np.float64)
     fp4_peak = peaks["bf16_tflops_sustained"] * FP4_OVER_BF16
     q_ach = q_bytes.sum() / t_q.sum() / 1e9
     # The GEMM dominates every workload's step. It is tensor-bound when its arithmetic
@@ -484,9 +507,10 @@ def run_ours(args, rank, world, local_rank):
     g_src = f"{PKG}/csrc/gemm_smallm.cu" if few_rows else f"{PKG}/csrc/gemm.cu"
     ridge = fp4_peak * 1e12 / (peaks["hbm_gbs"] * 1e9)
     intensity = gemm_flops.sum() / gemm_bytes.sum()
-    traffic = None if nv else ncu_traffic(wl.name, g_src)
-    q_traffic = None if nv else ncu_traffic(wl.name, f"{PKG}/csrc/quantize.cu",
-                                            NCU_TRAFFIC_QUANTIZE)
+    plain = not nv and norm is None  # the configuration the recorded counters are of
+    traffic = ncu_traffic(wl.name, g_src) if plain else None
+    q_traffic = (ncu_traffic(wl.name, f"{PKG}/csrc/quantize.cu", NCU_TRAFFIC_QUANTIZE)
+                 if plain else None)
     if intensity >= ridge:
         roofline = {"bound": "tensor", "achieved": gemm_flops.sum() / t_g.sum() / 1e12,
                     "peak": fp4_peak, "unit": "TFLOP/s",
@@ -526,6 +550,10 @@ def run_ours(args, rank, world, local_rank):
                 if nv:
                     mx.nvfp4_linear(xs_d[lin.x_tensor], wq, wsf, wsc, lin.N, wl.rotation,
                                     y=ys_d[j], ws=wss_d[j], stream=stream)
+                elif norm is not None:
+                    mx.norm_linear(xs_d[lin.x_tensor], wq, wsf, lin.N, norm, 1e-6,
+                                   norm_gb[j][0], norm_gb[j][1], wl.rotation, A, B, y=ys_d[j],
+                                   ws=wss_d[j], stream=stream)
                 else:
                     mx.linear(xs_d[lin.x_tensor], wq, wsf, lin.N, wl.rotation, A, B, y=ys_d[j],
                               ws=wss_d[j], stream=stream)
@@ -557,7 +585,9 @@ def run_ours(args, rank, world, local_rank):
                          "E2M1 x E2M1 with E8M0 block-32 scales, fp32 accumulate, bf16 out; "
                          "rotation in fp32"),
         "data": "synthetic (seeded N(0,1) activations with outlier channels, N(0,0.02^2) weights)",
-        "config": {"workload": workload_desc(wl), "tokens_per_gpu": wl.linears[0].M,
+        "config": {"workload": workload_desc(wl) + ("" if norm is None else
+                                                    f"; {args.norm} norm prologue"),
+                   "tokens_per_gpu": wl.linears[0].M,
                    "gflop_per_step_per_gpu": flops_step / 1e9, "parallelism": f"replicas x{world} "
                    "(token-parallel, no collective)",
                    "launch": f"timed steps replayed from CUDA graphs of {U} steps captured from "
@@ -566,8 +596,10 @@ def run_ours(args, rank, world, local_rank):
                          f"copies, footprint {footprint / 2**20:.0f} MiB >= 3 x L2 "
                          f"({l2 / 2**20:.0f} MiB)"},
         "roofline": roofline,
-        "quantize_roofline": {"bound": "hbm", "kernel": "nvfp4_amax_kernel + rotate_quantize_kernel"
-                              if nv else "rotate_quantize_kernel",
+        "quantize_roofline": {"bound": "hbm",
+                              "kernel": ("nvfp4_amax_kernel + rotate_quantize_kernel" if nv else
+                                         "row_stats_kernel + rotate_quantize_kernel"
+                                         if norm is not None else "rotate_quantize_kernel"),
                               "achieved": q_ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                               "frac": q_ach / peaks["hbm_gbs"],
                               "per_launch_us": [t * 1e6 for t in t_q],

@@ -339,29 +339,46 @@ __global__ void __launch_bounds__(256) row_stats_kernel(const uint16_t* __restri
   const uint32_t row = blockIdx.x * 8u + (threadIdx.x >> 5);
   if (row >= rows) return;
   const uint16_t* xr = x + (uint64_t)row * ldx;
+  // Each lane reads 8 elements at k, k + 256, k + 512, k + 768 per step (4 loads in flight)
+  // into 4 independent partial sums, added in a fixed order at the end.
   float mu = 0.0f;
   if constexpr (KIND == 0) {
-    float s = 0.0f;
-    for (uint32_t k = lane * 8u; k < K; k += 256u) {
-      const uint4 w = __ldg(reinterpret_cast<const uint4*>(xr + k));
-      s += bf16_lo(w.x) + bf16_hi(w.x) + bf16_lo(w.y) + bf16_hi(w.y) + bf16_lo(w.z) +
-           bf16_hi(w.z) + bf16_lo(w.w) + bf16_hi(w.w);
+    float s4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    for (uint32_t k0 = lane * 8u; k0 < K; k0 += 1024u) {
+      uint4 w[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        if (k0 + 256u * j < K) w[j] = __ldg(reinterpret_cast<const uint4*>(xr + k0 + 256u * j));
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        if (k0 + 256u * j < K)
+          s4[j] += bf16_lo(w[j].x) + bf16_hi(w[j].x) + bf16_lo(w[j].y) + bf16_hi(w[j].y) +
+                   bf16_lo(w[j].z) + bf16_hi(w[j].z) + bf16_lo(w[j].w) + bf16_hi(w[j].w);
     }
+    float s = (s4[0] + s4[1]) + (s4[2] + s4[3]);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
     mu = __fdiv_rn(s, (float)K);
   }
-  float v = 0.0f;
-  for (uint32_t k = lane * 8u; k < K; k += 256u) {
-    const uint4 w = __ldg(reinterpret_cast<const uint4*>(xr + k));
-    const float e[8] = {bf16_lo(w.x), bf16_hi(w.x), bf16_lo(w.y), bf16_hi(w.y),
-                        bf16_lo(w.z), bf16_hi(w.z), bf16_lo(w.w), bf16_hi(w.w)};
+  float v4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+  for (uint32_t k0 = lane * 8u; k0 < K; k0 += 1024u) {
+    uint4 w[4];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const float d = e[i] - mu;
-      v = __fmaf_rn(d, d, v);
+    for (int j = 0; j < 4; ++j)
+      if (k0 + 256u * j < K) w[j] = __ldg(reinterpret_cast<const uint4*>(xr + k0 + 256u * j));
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      if (k0 + 256u * j >= K) continue;
+      const float e[8] = {bf16_lo(w[j].x), bf16_hi(w[j].x), bf16_lo(w[j].y), bf16_hi(w[j].y),
+                          bf16_lo(w[j].z), bf16_hi(w[j].z), bf16_lo(w[j].w), bf16_hi(w[j].w)};
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float d = e[i] - mu;
+        v4[j] = __fmaf_rn(d, d, v4[j]);
+      }
     }
   }
+  float v = (v4[0] + v4[1]) + (v4[2] + v4[3]);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
   if (lane == 0) {
