@@ -55,17 +55,17 @@ PKG = "mxfp4_quantized_linear_block_b200"
 # kernel ends is written back later and is not counted (hence writes < Y bytes).
 NCU_TRAFFIC = {
     "dit_b1": {"source": f"{PKG}/csrc/gemm.cu",
-               "sha256": "3375dd2225b170c8bea10ae09bd5825cfe726ef7fc4d86f46d2390450dc9ce4d",
-               "bytes_per_launch": [20924160 + 12758016, 26232064 + 37004032,
-                                    43504896 + 2775552]},
+               "sha256": "ce8e9516555dcfd97b35b07bdfb668fd861f456dfe64b4a097ae55ed6b6ef456",
+               "bytes_per_launch": [20933888 + 12544000, 26112768 + 37123840,
+                                    43493120 + 4070144]},
     "llm_small_m1": {"source": f"{PKG}/csrc/gemm_smallm.cu",
-                     "sha256": "4e2cb66424a7f58bbb686dd0ed5bba39f74382b140c3a691d6a293916c0fb05c",
-                     "bytes_per_launch": [31234304 + 0, 31282944 + 256]},
+                     "sha256": "acf6c8b08bbaeeded821351219e7d760f8aa8060096b2255cc347a0619361b05",
+                     "bytes_per_launch": [31272448 + 0, 31320576 + 0]},
 }
 NCU_TRAFFIC_QUANTIZE = {
     "dit_b1": {"source": f"{PKG}/csrc/quantize.cu",
-               "sha256": "daead7a2fa978630267d30cd9dbbba56138ee8ba9de661d3e1cbad8f0f053f49",
-               "bytes_per_launch": [22033920 + 1280, 22033664 + 0, 88095744 + 4947200]},
+               "sha256": "07f72460d21f61c42649b20e4cb913f50a43b32a3400be2da00f8e645ead3913",
+               "bytes_per_launch": [22033664 + 0, 22033920 + 0, 88096000 + 4988160]},
 }
 
 
