@@ -189,3 +189,41 @@ def test_gemm_full_size_sampled(M, N, K):
     mi, ni = _sample_pairs(M, N)
     ref, S = oracle.gemm_pairs(aq, as_, bq, bs, mi, ni)
     check_gemm_values(y[mi, ni], ref, S, "bf16", f"gemm {M}x{N}x{K} sampled")
+
+
+@pytest.mark.parametrize("M,N,K", [(5, 144, 512), (300, 272, 768)])
+@pytest.mark.parametrize("out", ["bf16", "f32"])
+def test_gemm_padded_output_rows(M, N, K, out):
+    """y with a row stride larger than N (both kernels): the N columns of every row are
+    the product, the padding between rows is never written."""
+    import torch
+    import mxfp4_quantized_linear_block_b200 as mx
+    aq, as_ = _operand(M + N, M, K, 14)
+    bq, bs = _operand(M + N, N, K, 15)
+    dt = torch.float32 if out == "f32" else torch.bfloat16
+    pad = 24 if out == "bf16" else 12  # row stride stays a multiple of 16 bytes
+    big = torch.full((M, N + pad), 7.0, dtype=dt, device="cuda")
+    y = big[:, :N]
+    mx.gemm(to_dev(aq), to_dev(oracle.sf_to_physical(as_, K)), to_dev(bq),
+            to_dev(oracle.sf_to_physical(bs, K)), M, N, K, y=y)
+    torch.cuda.synchronize()
+    assert torch.all(big[:, N:] == 7.0)
+    got = y.float().cpu().numpy().astype(np.float64)
+    ref, S = oracle.gemm(aq, as_, bq, bs)
+    check_gemm_values(got, ref, S, out, f"padded rows {M}x{N}x{K} {out}")
+
+
+def test_gemm_and_linear_with_no_rows_write_nothing():
+    import torch
+    import mxfp4_quantized_linear_block_b200 as mx
+    K, N = 256, 128
+    y = torch.full((1, N), 3.0, dtype=torch.bfloat16, device="cuda")
+    x = torch.zeros((1, K), dtype=torch.bfloat16, device="cuda")[:0]  # M = 0, non-null
+    wq = torch.zeros((N, K // 2), dtype=torch.uint8, device="cuda")
+    wsf = torch.zeros(mx.sf_bytes(N, K), dtype=torch.uint8, device="cuda")
+    mx.gemm(torch.zeros((1, K // 2), dtype=torch.uint8, device="cuda"),
+            torch.zeros(mx.sf_bytes(1, K), dtype=torch.uint8, device="cuda"), wq, wsf, 0, N, K,
+            y=y)
+    mx.linear(x, wq, wsf, N, y=y[:0])
+    torch.cuda.synchronize()
+    assert torch.all(y == 3.0)
