@@ -35,7 +35,9 @@
  *    MXFP4_ERR_SHAPE; misaligned pointer or row stride -> MXFP4_ERR_ALIGN;
  *    workspace too small -> MXFP4_ERR_WORKSPACE; unknown mode / dtype ->
  *    MXFP4_ERR_UNSUPPORTED. A failed launch returns MXFP4_ERR_CUDA.
- *    rows == 0 (or M == 0) is a valid empty call: nothing is launched.
+ *    rows == 0 (or M == 0) is a valid empty call: nothing is launched (the
+ *    NVFP4 tensor-scale pass still writes its scale), and the pointers to
+ *    row operands (x, the activation codes and scales, y) may then be NULL.
  *  - Packed E2M1 codes ("q" operands): row-major [rows, K/2] bytes; byte j of a
  *    row holds element 2j in bits 0-3 and element 2j+1 in bits 4-7; bit 3 of a
  *    code is the sign, codes 0..7 are 0, 0.5, 1, 1.5, 2, 3, 4, 6.

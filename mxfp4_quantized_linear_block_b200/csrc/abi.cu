@@ -30,9 +30,14 @@ bool within_limits(int64_t rows, int64_t K) {
 
 mxfp4_status from_cuda(cudaError_t e) { return e == cudaSuccess ? MXFP4_OK : MXFP4_ERR_CUDA; }
 
+// A row operand (activations, their codes and scales, the output) may be NULL when it has
+// no rows: torch and other frameworks hand out NULL for empty tensors.
+bool rows_ptr_ok(const void* p, int64_t rows) { return p != nullptr || rows == 0; }
+
 mxfp4_status validate_quantize(const void* x, mxfp4_dtype xdt, int64_t rows, int64_t K,
                                int64_t ldx, const uint8_t* q, const uint8_t* sf) {
-  if (!x || !q || !sf) return MXFP4_ERR_INVALID_ARG;
+  if (!rows_ptr_ok(x, rows) || !rows_ptr_ok(q, rows) || !rows_ptr_ok(sf, rows))
+    return MXFP4_ERR_INVALID_ARG;
   if (xdt != MXFP4_DT_BF16 && xdt != MXFP4_DT_F32) return MXFP4_ERR_UNSUPPORTED;
   if (!shape_ok(rows, K) || ldx < K || !within_limits(rows, K)) return MXFP4_ERR_SHAPE;
   const int64_t esize = xdt == MXFP4_DT_F32 ? 4 : 2;
@@ -44,7 +49,8 @@ mxfp4_status validate_quantize(const void* x, mxfp4_dtype xdt, int64_t rows, int
 mxfp4_status validate_gemm(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq,
                            const uint8_t* bsf, int64_t M, int64_t N, int64_t K, const void* y,
                            mxfp4_dtype ydt, int64_t ldy) {
-  if (!aq || !asf || !bq || !bsf || !y) return MXFP4_ERR_INVALID_ARG;
+  if (!rows_ptr_ok(aq, M) || !rows_ptr_ok(asf, M) || !bq || !bsf || !rows_ptr_ok(y, M))
+    return MXFP4_ERR_INVALID_ARG;
   if (ydt != MXFP4_DT_BF16 && ydt != MXFP4_DT_F32) return MXFP4_ERR_UNSUPPORTED;
   if (!shape_ok(M, K) || N < 16 || N % 16 != 0 || ldy < N || !within_limits(M, K) ||
       !within_limits(N, K))
@@ -223,7 +229,9 @@ mxfp4_status mxfp4_gemm_quantize(const uint8_t* aq, const uint8_t* asf, const ui
                                  const float* bias, mxfp4_rotation mode, const float* kron_a,
                                  const float* kron_b, uint8_t* yq, uint8_t* ysf, void* ws,
                                  size_t ws_bytes, mxfp4_stream_t stream) {
-  if (!aq || !asf || !bq || !bsf || !yq || !ysf || !ws) return MXFP4_ERR_INVALID_ARG;
+  if (!rows_ptr_ok(aq, M) || !rows_ptr_ok(asf, M) || !bq || !bsf || !rows_ptr_ok(yq, M) ||
+      !rows_ptr_ok(ysf, M) || !ws)
+    return MXFP4_ERR_INVALID_ARG;
   // the epilogue rotates within one 32-column block: no larger Hadamard groups here
   if (mode != MXFP4_ROT_NONE && mode != MXFP4_ROT_HADAMARD32 && mode != MXFP4_ROT_KRON_4x8)
     return MXFP4_ERR_UNSUPPORTED;
@@ -251,7 +259,8 @@ mxfp4_status mxfp4_linear(const void* x, int64_t M, int64_t K, mxfp4_rotation mo
                           const float* kron_a, const float* kron_b, const uint8_t* wq,
                           const uint8_t* wsf, int64_t N, void* y, void* ws, size_t ws_bytes,
                           mxfp4_stream_t stream) {
-  if (!x || !wq || !wsf || !y || !ws) return MXFP4_ERR_INVALID_ARG;
+  if (!rows_ptr_ok(x, M) || !wq || !wsf || !rows_ptr_ok(y, M) || !ws)
+    return MXFP4_ERR_INVALID_ARG;
   if (!mode_ok(mode)) return MXFP4_ERR_UNSUPPORTED;
   if (!shape_ok(M, K) || K % rotation_span(mode) != 0 || N < 16 || N % 16 != 0 ||
       !within_limits(M, K) || !within_limits(N, K))
@@ -305,7 +314,8 @@ mxfp4_status mxfp4_norm_linear(const void* x, int64_t M, int64_t K, mxfp4_norm k
                                const float* kron_a, const float* kron_b, const uint8_t* wq,
                                const uint8_t* wsf, int64_t N, void* y, void* ws,
                                size_t ws_bytes, mxfp4_stream_t stream) {
-  if (!x || !wq || !wsf || !y || !ws) return MXFP4_ERR_INVALID_ARG;
+  if (!rows_ptr_ok(x, M) || !wq || !wsf || !rows_ptr_ok(y, M) || !ws)
+    return MXFP4_ERR_INVALID_ARG;
   if (kind != MXFP4_NORM_LAYER && kind != MXFP4_NORM_RMS) return MXFP4_ERR_UNSUPPORTED;
   if (mode != MXFP4_ROT_NONE && mode != MXFP4_ROT_HADAMARD32 && mode != MXFP4_ROT_KRON_4x8)
     return MXFP4_ERR_UNSUPPORTED;
@@ -341,7 +351,7 @@ size_t mxfp4_nvfp4_sf_bytes(int64_t rows, int64_t K) {
 mxfp4_status mxfp4_nvfp4_tensor_scale(const void* x, mxfp4_dtype xdt, int64_t rows, int64_t K,
                                       int64_t ldx, mxfp4_rotation mode, float* scale2,
                                       mxfp4_stream_t stream) {
-  if (!x || !scale2) return MXFP4_ERR_INVALID_ARG;
+  if (!rows_ptr_ok(x, rows) || !scale2) return MXFP4_ERR_INVALID_ARG;
   if (xdt != MXFP4_DT_BF16 && xdt != MXFP4_DT_F32) return MXFP4_ERR_UNSUPPORTED;
   if (mode != MXFP4_ROT_NONE && mode != MXFP4_ROT_HADAMARD32) return MXFP4_ERR_UNSUPPORTED;
   if (!shape_ok(rows, K) || ldx < K || !within_limits(rows, K)) return MXFP4_ERR_SHAPE;
@@ -393,7 +403,8 @@ mxfp4_status mxfp4_nvfp4_linear(const void* x, int64_t M, int64_t K, mxfp4_rotat
                                 const uint8_t* wq, const uint8_t* wsf, const float* w_scale,
                                 int64_t N, void* y, void* ws, size_t ws_bytes,
                                 mxfp4_stream_t stream) {
-  if (!x || !wq || !wsf || !w_scale || !y || !ws) return MXFP4_ERR_INVALID_ARG;
+  if (!rows_ptr_ok(x, M) || !wq || !wsf || !w_scale || !rows_ptr_ok(y, M) || !ws)
+    return MXFP4_ERR_INVALID_ARG;
   if (mode != MXFP4_ROT_NONE && mode != MXFP4_ROT_HADAMARD32) return MXFP4_ERR_UNSUPPORTED;
   if (!shape_ok(M, K) || N < 16 || N % 16 != 0 || !within_limits(M, 2 * K) ||
       !within_limits(N, 2 * K))

@@ -63,7 +63,7 @@ extern "C" mxfp4_status mxfp4_linear_noalloc(const void* x, int64_t M, int64_t K
                                               const uint8_t* wsf, int64_t N, void* y, int* status,
                                               mxfp4_stream_t stream) {
   using namespace mxfp4;
-  if (!x || !wq || !wsf || !y) return MXFP4_ERR_INVALID_ARG;
+  if ((!x && M != 0) || !wq || !wsf || (!y && M != 0)) return MXFP4_ERR_INVALID_ARG;
   if (mode < MXFP4_ROT_NONE || mode > MXFP4_ROT_HADAMARD128) return MXFP4_ERR_UNSUPPORTED;
   if (M < 0 || K < 32 || K % rotation_span(mode) != 0 || N < 16 || N % 16 != 0 ||
       M >= (1ll << 31) ||

@@ -134,3 +134,21 @@ def test_gemm_bias_and_quantize_argument_errors():
     assert q(ysf=P + 1) == mx.ERR_ALIGN
     assert q(wsb=16) == mx.ERR_WORKSPACE
     assert q(M=0) == mx.OK
+
+
+def test_empty_calls_accept_null_row_operands():
+    """With no rows, x / the activation codes and scales / y may be NULL (frameworks hand out
+    NULL for empty tensors); the weight operands and the workspace stay required."""
+    L = mx.lib
+    assert L.mxfp4_rotate_quantize(None, 0, 0, 64, 64, 1, None, None, None, None, None) == mx.OK
+    assert L.mxfp4_gemm(None, None, P, P, 0, 16, 64, None, 0, 16, P, 256, None) == mx.OK
+    assert L.mxfp4_gemm(None, None, None, P, 0, 16, 64, None, 0, 16, P, 256, None) == \
+        mx.ERR_INVALID_ARG
+    assert L.mxfp4_gemm(None, P, P, P, 4, 16, 64, P, 0, 16, P, 256, None) == mx.ERR_INVALID_ARG
+    need = mx.workspace_bytes(mx.OP_LINEAR, 0, 32, 64)
+    assert L.mxfp4_linear(None, 0, 64, 1, None, None, P, P, 32, None, P, need, None) == mx.OK
+    assert L.mxfp4_linear(None, 0, 64, 1, None, None, P, P, 32, None, None, need, None) == \
+        mx.ERR_INVALID_ARG
+    assert L.mxfp4_linear(P, 4, 64, 1, None, None, P, P, 32, None, P, 1 << 20, None) == \
+        mx.ERR_INVALID_ARG
+    assert L.mxfp4_linear_noalloc(None, 0, 64, 1, None, None, P, P, 32, None, None, None) == mx.OK
