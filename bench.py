@@ -59,8 +59,8 @@ NCU_TRAFFIC = {
                "bytes_per_launch": [20933888 + 12544000, 26112768 + 37123840,
                                     43493120 + 4070144]},
     "llm_small_m1": {"source": f"{PKG}/csrc/gemm_smallm.cu",
-                     "sha256": "acf6c8b08bbaeeded821351219e7d760f8aa8060096b2255cc347a0619361b05",
-                     "bytes_per_launch": [31272448 + 0, 31320576 + 0]},
+                     "sha256": "17c99c26969ae4178694fdbd5d747735da958b59a157ff608b180262894be314",
+                     "bytes_per_launch": [31281920 + 0, 31299840 + 0]},
 }
 NCU_TRAFFIC_QUANTIZE = {
     "dit_b1": {"source": f"{PKG}/csrc/quantize.cu",
@@ -421,10 +421,13 @@ def run_ours(args, rank, world, local_rank):
     flops_step = wl.flops
     value = job_tflops(flops_step, args.steps, world, elapsed)
     ms_per_step = elapsed / args.steps * 1e3
-    # kernels per linear: quantise + GEMM; NVFP4 adds the tensor-scale pass (2 kernels),
-    # the norm prologue the row-statistics kernel
-    k_per_linear = 4 if nv else 3 if norm is not None else 2
-    launches = k_per_linear * len(wl.linears) * args.steps
+    # kernels per linear: quantise + GEMM, or one kernel when the layer quantises x inside
+    # the GEMM's CTAs (1..8 rows); NVFP4 adds the tensor-scale pass (2 kernels), the norm
+    # prologue the row-statistics kernel
+    kcount = [4 if nv else 3 if norm is not None else
+              mx.linear_kernel_count(l.M, l.N, l.K, wl.rotation) for l in wl.linears]
+    fused = [k == 1 for k in kcount]
+    launches = sum(kcount) * args.steps
 
     # status words: no bounded wait expired
     for s in sets:
@@ -433,14 +436,16 @@ def run_ours(args, rank, world, local_rank):
                 raise RuntimeError("a kernel reported a bounded-wait timeout")
 
     # ---- attribution pass: the same steps as separate quantise / GEMM launches with
-    # CUDA events around each kernel (on the launching stream)
+    # CUDA events around each kernel (on the launching stream); a layer that is one
+    # kernel is timed as that kernel
     qbufs = [(torch.empty((l.M, l.K // 2), dtype=torch.uint8, device=dev),
               torch.empty(mx.nvfp4_sf_bytes(l.M, l.K) if nv else mx.sf_bytes(l.M, l.K),
                           dtype=torch.uint8, device=dev),
               torch.zeros(2, dtype=torch.float32, device=dev),
               torch.empty((l.M, 2), dtype=torch.float32, device=dev)) for l in wl.linears]
-    gws = [mx.new_workspace(mx.workspace_bytes(mx.OP_GEMM, l.M, l.N, l.K), dev)
-           for l in wl.linears]
+    gws = [mx.new_workspace(mx.workspace_bytes(mx.OP_LINEAR if fused[j] else mx.OP_GEMM,
+                                               l.M, l.N, l.K), dev)
+           for j, l in enumerate(wl.linears)]
     n_lin = len(wl.linears)
     n_attr = max(1, min(args.steps, args.attr_steps))
     evs = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
@@ -453,6 +458,14 @@ def run_ours(args, rank, world, local_rank):
             q, sf, xsc, stt = qbufs[j]
             if rec:
                 evs[i][j][0].record(stream)
+            if fused[j]:
+                if rec:
+                    evs[i][j][1].record(stream)
+                mx.linear(xs[lin.x_tensor], wq, wsf, lin.N, wl.rotation, A, B, y=ys[j],
+                          ws=gws[j], stream=stream)
+                if rec:
+                    evs[i][j][2].record(stream)
+                continue
             if nv:
                 mx.nvfp4_tensor_scale(xs[lin.x_tensor], wl.rotation, scale2=xsc, stream=stream)
                 mx.nvfp4_quantize(xs[lin.x_tensor], xsc, wl.rotation, q=q, sf=sf, stream=stream)
@@ -491,19 +504,25 @@ def run_ours(args, rank, world, local_rank):
     t_g /= n_attr
     gemm_flops = np.array([l.flops for l in wl.linears], dtype=np.float64)
     sfb = mx.nvfp4_sf_bytes if nv else mx.sf_bytes
-    gemm_bytes = np.array([l.M * l.K // 2 + sfb(l.M, l.K) + l.N * l.K // 2 +
-                           sfb(l.N, l.K) + 2 * l.M * l.N for l in wl.linears], np.float64)
+    # a fused layer reads x in bf16 instead of its codes and scales
+    gemm_bytes = np.array([(2 * l.M * l.K if fused[j] else l.M * l.K // 2 + sfb(l.M, l.K)) +
+                           l.N * l.K // 2 + sfb(l.N, l.K) + 2 * l.M * l.N
+                           for j, l in enumerate(wl.linears)], np.float64)
     # NVFP4's dynamic tensor scale, and the norm's row statistics, need a full pass over X
     # before the quantiser reads it
-    q_bytes = np.array([(4 if nv or norm is not None else 2) * l.M * l.K + l.M * l.K // 2 +
-                        sfb(l.M, l.K) for l in wl.linears], np.float64)
+    q_bytes = np.array([0.0 if fused[j] else
+                        (4 if nv or norm is not None else 2) * l.M * l.K + l.M * l.K // 2 +
+                        sfb(l.M, l.K) for j, l in enumerate(wl.linears)], np.float64)
     fp4_peak = peaks["bf16_tflops_sustained"] * FP4_OVER_BF16
-    q_ach = q_bytes.sum() / t_q.sum() / 1e9
+    q_sel = [j for j in range(n_lin) if not fused[j]]
+    q_ach = q_bytes[q_sel].sum() / t_q[q_sel].sum() / 1e9 if q_sel else None
     # The GEMM dominates every workload's step. It is tensor-bound when its arithmetic
     # intensity (2MNK over its algorithmic bytes) is above the ridge of the two peaks,
     # HBM-bound otherwise (few tokens).
     few_rows = all(l.M <= 128 for l in wl.linears)
-    g_kernel = "mxf4_gemm_smallm_kernel" if few_rows else "mxf4_gemm_pair_kernel"
+    g_kernel = ("mxf4_gemm_smallm_kernel (whole layer: x rotated and quantised in the kernel)"
+                if all(fused) else "mxf4_gemm_smallm_kernel" if few_rows
+                else "mxf4_gemm_pair_kernel")
     g_src = f"{PKG}/csrc/gemm_smallm.cu" if few_rows else f"{PKG}/csrc/gemm.cu"
     ridge = fp4_peak * 1e12 / (peaks["hbm_gbs"] * 1e9)
     intensity = gemm_flops.sum() / gemm_bytes.sum()
@@ -511,17 +530,24 @@ def run_ours(args, rank, world, local_rank):
     traffic = ncu_traffic(wl.name, g_src) if plain else None
     q_traffic = (ncu_traffic(wl.name, f"{PKG}/csrc/quantize.cu", NCU_TRAFFIC_QUANTIZE)
                  if plain else None)
+    # When every layer of the step is one kernel, the timed region (graph replay, CUDA
+    # events on the launching stream) holds only those launches: their average duration
+    # is the step time over the launches. Otherwise the attribution pass splits the step.
+    t_dom = elapsed / args.steps if all(fused) else t_g.sum()
     if intensity >= ridge:
-        roofline = {"bound": "tensor", "achieved": gemm_flops.sum() / t_g.sum() / 1e12,
+        roofline = {"bound": "tensor", "achieved": gemm_flops.sum() / t_dom / 1e12,
                     "peak": fp4_peak, "unit": "TFLOP/s",
                     "peak_source": f"4 x {peaks['source']} bf16 sustained "
                                    f"({peaks['bf16_tflops_sustained']} TFLOP/s)"}
     else:
-        roofline = {"bound": "hbm", "achieved": gemm_bytes.sum() / t_g.sum() / 1e9,
+        roofline = {"bound": "hbm", "achieved": gemm_bytes.sum() / t_dom / 1e9,
                     "peak": peaks["hbm_gbs"], "unit": "GB/s",
                     "peak_source": f"{peaks['source']} HBM copy bandwidth"}
     roofline.update({
         "frac": roofline["achieved"] / roofline["peak"], "kernel": g_kernel,
+        "timing": ("timed region: every launch of the step is this kernel; per_launch: "
+                   "attribution pass (eager, events around each launch)" if all(fused) else
+                   "attribution pass: CUDA events around each launch (eager)"),
         "intensity_flop_per_byte": intensity, "ridge_flop_per_byte": ridge,
         "per_launch": [{"linear": l.name, "us": t_g[j] * 1e6,
                         "tflops": gemm_flops[j] / t_g[j] / 1e12,
@@ -574,7 +600,7 @@ def run_ours(args, rank, world, local_rank):
         e2e = {"value": job_tflops(flops_step, args.e2e_steps, world, t_e2e), "unit": UNIT,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "ms_per_step": t_e2e / args.e2e_steps * 1e3, "steps": args.e2e_steps,
-               "gpu_launches": k_per_linear * len(wl.linears) * args.e2e_steps}
+               "gpu_launches": sum(kcount) * args.e2e_steps}
 
     result = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -596,23 +622,27 @@ def run_ours(args, rank, world, local_rank):
                          f"copies, footprint {footprint / 2**20:.0f} MiB >= 3 x L2 "
                          f"({l2 / 2**20:.0f} MiB)"},
         "roofline": roofline,
-        "quantize_roofline": {"bound": "hbm",
-                              "kernel": ("nvfp4_amax_kernel + rotate_quantize_kernel" if nv else
-                                         "row_stats_kernel + rotate_quantize_kernel"
-                                         if norm is not None else "rotate_quantize_kernel"),
-                              "achieved": q_ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                              "frac": q_ach / peaks["hbm_gbs"],
-                              "per_launch_us": [t * 1e6 for t in t_q],
-                              "alg_bytes_per_launch": [int(b) for b in q_bytes],
-                              "traffic": (float(np.mean(q_traffic["bytes_per_launch"]))
-                                          if q_traffic else None),
-                              "traffic_per_launch": (q_traffic["bytes_per_launch"]
-                                                     if q_traffic else None)},
+        "quantize_roofline": ({"bound": "hbm",
+                               "kernel": ("nvfp4_amax_kernel + rotate_quantize_kernel" if nv else
+                                          "row_stats_kernel + rotate_quantize_kernel"
+                                          if norm is not None else "rotate_quantize_kernel"),
+                               "achieved": q_ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                               "frac": q_ach / peaks["hbm_gbs"],
+                               "per_launch_us": [t_q[j] * 1e6 for j in q_sel],
+                               "alg_bytes_per_launch": [int(q_bytes[j]) for j in q_sel],
+                               "traffic": (float(np.mean(q_traffic["bytes_per_launch"]))
+                                           if q_traffic else None),
+                               "traffic_per_launch": (q_traffic["bytes_per_launch"]
+                                                      if q_traffic else None)}
+                              if q_sel else
+                              {"fused": True, "note": "x is rotated and quantised inside the "
+                               "layer's one kernel (1..8 rows): no quantiser launch"}),
         "e2e": e2e,
         "gpu_launches": launches,
-        "attribution": {"steps": n_attr, "gpu_launches": k_per_linear * n_lin * n_attr,
+        "attribution": {"steps": n_attr, "gpu_launches": sum(kcount) * n_attr,
                         "note": "quantise and GEMM launched separately with CUDA events "
-                                "around each kernel; source of both roofline objects"},
+                                "around each kernel (a one-kernel layer as that kernel); "
+                                "source of both roofline objects"},
         "clocks": clk,
     }
     return result

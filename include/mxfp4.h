@@ -217,11 +217,26 @@ mxfp4_status mxfp4_gemm_quantize(const uint8_t* aq, const uint8_t* asf, const ui
  * mxfp4_workspace_bytes(MXFP4_OP_LINEAR, M, N, K) bytes. The two kernels run
  * back to back on `stream`; the GEMM may start loading wq / wsf while the
  * quantiser is still running, so wq / wsf must not overlap the workspace.
+ * For 1..8 rows (rotation none, Hadamard-32 or Kronecker, and K splits of at
+ * most 12 x 256 elements; see mxfp4_linear_kernel_count) the layer is one
+ * kernel: each CTA rotates and quantises its own K range of x into shared
+ * memory while it streams the weights. Codes, scales and the result are the
+ * same as with the two kernels.
  */
 mxfp4_status mxfp4_linear(const void* x, int64_t M, int64_t K, mxfp4_rotation mode,
                           const float* kron_a, const float* kron_b, const uint8_t* wq,
                           const uint8_t* wsf, int64_t N, void* y, void* ws, size_t ws_bytes,
                           mxfp4_stream_t stream);
+
+/*
+ * How many kernels mxfp4_linear (and mxfp4_linear_noalloc) launch for these
+ * sizes and rotation: 1 when the layer runs as one kernel (1..8 rows, mode
+ * none / Hadamard-32 / Kronecker, at most 12 k-tiles of 256 elements per K
+ * split of the few-row GEMM), 2 otherwise (quantiser, then GEMM), 0 for
+ * M == 0, -1 for sizes or a mode that mxfp4_linear rejects. Host only; no
+ * GPU is touched.
+ */
+int mxfp4_linear_kernel_count(int64_t M, int64_t N, int64_t K, mxfp4_rotation mode);
 
 /*
  * Norm prologue: the normalisation that precedes the layer, applied inside the

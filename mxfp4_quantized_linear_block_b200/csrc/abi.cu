@@ -278,12 +278,24 @@ mxfp4_status mxfp4_linear(const void* x, int64_t M, int64_t K, mxfp4_rotation mo
   uint8_t* xq = base + w.q_off;
   uint8_t* xsf = base + w.sf_off;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  cudaError_t e =
-      launch_rotate_quantize(x, false, M, K, K, (int)mode, &kc, xq, xsf, static_cast<int*>(ws), s);
+  // Up to 16 rows: one kernel quantises x inside the GEMM's CTAs.
+  cudaError_t e = launch_linear_smallm(x, K, (int)mode, &kc, wq, wsf, M, N, K, y, N,
+                                       static_cast<int*>(ws), s);
+  if (e != cudaErrorNotSupported) return from_cuda(e);
+  e = launch_rotate_quantize(x, false, M, K, K, (int)mode, &kc, xq, xsf, static_cast<int*>(ws), s);
   if (e != cudaSuccess) return MXFP4_ERR_CUDA;
   // The kernel just before the GEMM is the quantiser above, which does not write W.
   return from_cuda(launch_gemm(xq, xsf, wq, wsf, M, N, K, y, Epilogue{}, N, static_cast<int*>(ws),
                                base + w.g_off, ws_bytes - w.g_off, true, s));
+}
+
+int mxfp4_linear_kernel_count(int64_t M, int64_t N, int64_t K, mxfp4_rotation mode) {
+  if (!mode_ok(mode)) return -1;
+  if (!shape_ok(M, K) || K % rotation_span(mode) != 0 || N < 16 || N % 16 != 0 ||
+      !within_limits(M, K) || !within_limits(N, K))
+    return -1;
+  if (M == 0) return 0;
+  return linear_smallm_fits(M, N, K, (int)mode) ? 1 : 2;
 }
 
 mxfp4_status mxfp4_norm_rotate_quantize(const void* x, int64_t rows, int64_t K, int64_t ldx,

@@ -14,6 +14,13 @@
 // and writes that part of Y with coalesced row stores. No global scratch, no
 // atomics, no second kernel.
 //
+// The whole layer for up to 8 tokens (FX variant): the CTA's epilogue warps
+// rotate and quantise the CTA's K range of the bf16 activations themselves,
+// straight into the B-operand layout in shared memory, while the weight stream
+// is in flight -- no separate quantiser kernel, no activation round trip
+// through global memory, and the weight stream starts as soon as the kernel
+// before the layer has finished.
+//
 // ("AMD Quark delivers MXFP4 quantization for FLUX.1-dev on Instinct MI350
 // with 1.92x speedup", opening section: MXFP4 GEMM without dequantisation;
 // "Bridging the Gap Between Promise and Performance for Microscaling FP4
@@ -38,26 +45,39 @@ constexpr uint32_t kFirstEpiWarp = 2;
 constexpr uint32_t kMaxSplits = 8;  // portable cluster size
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr int kTimeoutCode = 7;
+// Fused layer: at most this many k-tiles (256 elements) of activations per CTA, all
+// resident in shared memory at once, and at most this many rows. Every CTA of a K split
+// reads the same slice of x, so the reads grow with the rows times the W tiles; beyond 8
+// rows (B200, 4096 <-> 14336) they slow the weight stream more than the separate
+// quantiser launch costs.
+constexpr uint32_t kFxMaxKt = 12;
+constexpr int64_t kFxMaxRows = 8;
 
-template <uint32_t NT, bool NV = false>
+template <uint32_t NT, bool NV = false, bool FX = false>
 struct SmallConfig {
   // scale atoms (128 rows x 4 scales) per k-tile of 256 elements: 2 for MXFP4, 4 for NVFP4
   static constexpr uint32_t AT = NV ? 4 : 2;
+  static constexpr uint32_t A_STAGE = 128 * 128;          // 128 rows of W x 256 elements
+  static constexpr uint32_t B_STAGE = FX ? 0 : NT * 128;  // NT token rows x 256 elements
+  static constexpr uint32_t SF_STAGE = AT * 512;          // AT scale atoms
+  // FX: the quantised activations of the CTA's whole K range (B-operand tiles and their
+  // scale atoms, one of each per k-tile), written by the CTA itself.
+  static constexpr uint32_t XQ_KT = NT * 128;
+  static constexpr uint32_t XQ_BYTES = FX ? kFxMaxKt * XQ_KT : 0;
+  static constexpr uint32_t XSF_BYTES = FX ? kFxMaxKt * SF_STAGE : 0;
   // Two CTAs per SM: as many stages (at most 5) as let 2 x SMEM_BYTES fit an SM's
   // shared memory (233472 bytes, 1 KB of it reserved per CTA).
-  static constexpr uint32_t STAGE_BYTES = 128 * 128 + NT * 128 + 2 * AT * 512;
-  static constexpr uint32_t STAGES = (116736 - 1024 - 1024 - 512) / STAGE_BYTES < 5
-                                         ? (116736 - 1024 - 1024 - 512) / STAGE_BYTES
-                                         : 5;
-  static constexpr uint32_t A_STAGE = 128 * 128;  // 128 rows of W x 256 elements
-  static constexpr uint32_t B_STAGE = NT * 128;   // NT token rows x 256 elements
-  static constexpr uint32_t SF_STAGE = AT * 512;  // AT scale atoms
+  static constexpr uint32_t STAGE_BYTES = A_STAGE + B_STAGE + (FX ? 1 : 2) * SF_STAGE;
+  static constexpr uint32_t BUDGET = 116736 - 1024 - 1024 - 512 - XQ_BYTES - XSF_BYTES;
+  static constexpr uint32_t STAGES = BUDGET / STAGE_BYTES < 5 ? BUDGET / STAGE_BYTES : 5;
   static constexpr uint32_t OFF_A = 0;
   static constexpr uint32_t OFF_B = OFF_A + STAGES * A_STAGE;
-  static constexpr uint32_t OFF_SFA = OFF_B + STAGES * B_STAGE;
+  static constexpr uint32_t OFF_XQ = OFF_B + STAGES * B_STAGE;
+  static constexpr uint32_t OFF_SFA = OFF_XQ + XQ_BYTES;
   static constexpr uint32_t OFF_SFB = OFF_SFA + STAGES * SF_STAGE;
-  static constexpr uint32_t OFF_BAR = OFF_SFB + STAGES * SF_STAGE;
-  static constexpr uint32_t NUM_BARS = 2 * STAGES + 2;
+  static constexpr uint32_t OFF_XSF = OFF_SFB + (FX ? 0 : STAGES * SF_STAGE);
+  static constexpr uint32_t OFF_BAR = OFF_XSF + XSF_BYTES;
+  static constexpr uint32_t NUM_BARS = 2 * STAGES + 2 + (FX ? kFxMaxKt : 0);
   static constexpr uint32_t OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr uint32_t SMEM_BYTES = OFF_MISC + 16 + 1024;
   // fp32 partial [NT][128] at offset 0, over the A/B stages once every MMA has completed
@@ -69,6 +89,8 @@ struct SmallConfig {
                                         : COLS_USED <= 128 ? 128 : 256;
   static_assert(NT % 16 == 0 && NT >= 16 && NT <= 128, "token tile");
   static_assert(RED_BYTES <= OFF_SFA, "partial fits over the operand stages");
+  static_assert(!FX || (!NV && STAGES >= 3), "fused layer: MXFP4, a ring of 3 or more");
+  static_assert(OFF_XQ % 1024 == 0 && XQ_KT % 1024 == 0, "128-byte swizzle atoms");
   static_assert(2 * (SMEM_BYTES + 1024) <= 233472, "two CTAs per SM");
 };
 
@@ -87,6 +109,9 @@ struct SmallParams {
   uint32_t n_katoms_y;  // MXFP4 output: scale atoms per 128-row group of Y
   const float* a_scale; // NVFP4: tensor scales (device fp32) of X and W
   const float* b_scale;
+  const void* x;        // FX: bf16 activations [M, K], row stride ldx elements
+  uint64_t ldx;
+  uint32_t xmode;       // FX: rotation of each 32-element block of X (0, 1, 2)
 };
 
 __device__ __forceinline__ void record_timeout(int* status) {
@@ -235,11 +260,82 @@ __device__ __forceinline__ void reduce_store_mxfp4(const SmallParams& p, const K
   }
 }
 
-template <uint32_t NT, int OUT, bool NV>
+// FX: the 128 epilogue threads rotate and quantise X[m, 256 kt0 .. 256 kt1) for the 16
+// token rows of the tile (rows >= M and blocks past K give zero codes and scales) into
+// the CTA's activation tiles, one k-tile at a time: thread (m, j) = (tid / 8, tid % 8)
+// does block j of row m in every k-tile, keeping the loads of the next four k-tiles in
+// flight, and releases the k-tile's barrier once it is written, so the MMAs of k-tile t
+// wait only for k-tile t. Codes of k-tile t, row m, block j (16 bytes) go to
+// XQ + t 2048 + m 128 + ((j ^ (m % 8)) 16) -- the K-major, 128-byte-swizzled operand
+// layout the tensor core reads -- and the scale byte to the k-tile's scale atoms, laid out
+// as in a global scale tensor. X comes from the kernel before this one: it is read only
+// after waiting for it.
+template <uint32_t NT>
+__device__ __forceinline__ void quantize_x_slice(const SmallParams& p, const KronCoeffs& kc,
+                                                 uint32_t sbase, uint32_t kt0, uint32_t kt1,
+                                                 uint32_t bar_x) {
+  using C = SmallConfig<NT, false, true>;
+  static_assert(NT * 8 == 128, "one block per epilogue thread and k-tile");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const uint32_t tid = threadIdx.x - kFirstEpiWarp * 32u;
+  const uint32_t nkt = kt1 - kt0;
+  for (uint32_t i = tid; i < nkt * C::SF_STAGE / 16u; i += 128u)
+    st_shared_v4(sbase + C::OFF_XSF + i * 16u, 0u, 0u, 0u, 0u);
+  asm volatile("bar.sync 1, 128;" ::: "memory");  // the four epilogue warps
+  const uint32_t kb_real = p.K / 32u;
+  const uint32_t m = tid >> 3, j = tid & 7u;
+  const bool row_ok = m < p.M;
+  const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.x) +
+                                                    (uint64_t)(row_ok ? m : 0u) * p.ldx);
+  // Four k-tiles of loads in flight per thread (a ring of registers, slot t % 4).
+  uint4 buf[4][4];
+  auto load = [&](uint32_t t, uint4 (&w)[4]) {
+    const uint32_t kb = (kt0 + t) * 8u + j;
+    if (t < nkt && row_ok && kb < kb_real) {
+#pragma unroll
+      for (int c = 0; c < 4; ++c) w[c] = __ldg(src + kb * 4u + c);
+    }
+  };
+#pragma unroll
+  for (uint32_t u = 0; u < 4; ++u) load(u, buf[u]);
+  for (uint32_t t0 = 0; t0 < nkt; t0 += 4) {
+#pragma unroll
+    for (uint32_t u = 0; u < 4; ++u) {
+      const uint32_t t = t0 + u;
+      if (t >= nkt) break;
+      const uint32_t kb = (kt0 + t) * 8u + j;
+      uint4 codes = make_uint4(0u, 0u, 0u, 0u);
+      if (row_ok && kb < kb_real) {
+        float2 P[16];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const uint4 w = buf[u][c];
+          P[4 * c + 0] = make_float2(blockq::bf16_lo(w.x), blockq::bf16_hi(w.x));
+          P[4 * c + 1] = make_float2(blockq::bf16_lo(w.y), blockq::bf16_hi(w.y));
+          P[4 * c + 2] = make_float2(blockq::bf16_lo(w.z), blockq::bf16_hi(w.z));
+          P[4 * c + 3] = make_float2(blockq::bf16_lo(w.w), blockq::bf16_hi(w.w));
+        }
+        load(t + 4, buf[u]);  // the slot is free again: refill it four k-tiles ahead
+        if (p.xmode == 1) blockq::hadamard32(P);
+        if (p.xmode == 2) blockq::kron32(P, kc);
+        const uint32_t byte = blockq::quantize_block(P, codes);
+        const uint32_t sf_addr = sbase + C::OFF_XSF + (t * C::AT + (j >> 2)) * 512u +
+                                 (m & 31u) * 16u + (m >> 5) * 4u + (j & 3u);
+        asm volatile("st.shared.u8 [%0], %1;" ::"r"(sf_addr), "r"(byte) : "memory");
+      }
+      st_shared_v4(sbase + C::OFF_XQ + t * C::XQ_KT + m * 128u + ((j ^ (m & 7u)) << 4),
+                   codes.x, codes.y, codes.z, codes.w);
+      fence_proxy_async_smem();  // the tensor core reads these tiles through the async proxy
+      mbar_arrive(bar_x + 8u * t);
+    }
+  }
+}
+
+template <uint32_t NT, int OUT, bool NV, bool FX>
 __global__ void __launch_bounds__(kThreads, 2) mxf4_gemm_smallm_kernel(
     const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
     const SmallParams p, const __grid_constant__ KronCoeffs kc) {
-  using C = SmallConfig<NT, NV>;
+  using C = SmallConfig<NT, NV, FX>;
   constexpr uint32_t STAGES = C::STAGES;
   constexpr uint32_t AT = C::AT;
   extern __shared__ uint8_t smem_raw[];
@@ -262,6 +358,7 @@ __global__ void __launch_bounds__(kThreads, 2) mxf4_gemm_smallm_kernel(
   const uint32_t bar_empty = bar_full + 8 * STAGES;
   const uint32_t bar_tfull = bar_empty + 8 * STAGES;
   const uint32_t bar_mma_done = bar_tfull + 8;
+  const uint32_t bar_xready = bar_mma_done + 8;  // FX: one per k-tile of activations
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
 
@@ -272,23 +369,26 @@ __global__ void __launch_bounds__(kThreads, 2) mxf4_gemm_smallm_kernel(
     }
     mbar_init(bar_tfull, 1);
     mbar_init(bar_mma_done, 1);
+    if constexpr (FX)
+      for (uint32_t t = 0; t < kFxMaxKt; ++t) mbar_init(bar_xready + 8 * t, 128);
     *abort_flag = 0;
     fence_mbar_init();
     fence_proxy_async_smem();
     prefetch_tmap(&tmap_w);
-    prefetch_tmap(&tmap_x);
+    if constexpr (!FX) prefetch_tmap(&tmap_x);
     // When the kernel just before this one does not write W (the layer's own
     // quantiser), the first stages' W loads go out now, ahead of the set-up below
     // and of the wait for that kernel. Each stage's barrier expects its X bytes too.
+    const uint64_t pol_w = l2_policy_evict_first();  // W is read once per call
     for (uint32_t i = 0; i < (p.w_early ? pre : 0u); ++i) {
       const uint32_t kt = kt0 + i;
       const uint32_t atoms = (p.k_atoms - AT * kt) >= AT ? AT : p.k_atoms - AT * kt;
       const uint32_t fb = bar_full + 8 * i;
-      mbar_arrive_expect_tx(fb, C::A_STAGE + C::B_STAGE + 2u * atoms * 512u);
-      tma_load_2d(sbase + C::OFF_A + i * C::A_STAGE, &tmap_w, fb, (int32_t)(kt * 128u),
-                  (int32_t)(wt * 128u));
-      bulk_load(sbase + C::OFF_SFA + i * C::SF_STAGE,
-                p.wsf + ((uint64_t)wt * p.k_atoms + AT * kt) * 512u, atoms * 512u, fb);
+      mbar_arrive_expect_tx(fb, C::A_STAGE + C::B_STAGE + (FX ? 1u : 2u) * atoms * 512u);
+      tma_load_2d_hint(sbase + C::OFF_A + i * C::A_STAGE, &tmap_w, fb, (int32_t)(kt * 128u),
+                       (int32_t)(wt * 128u), pol_w);
+      bulk_load_hint(sbase + C::OFF_SFA + i * C::SF_STAGE,
+                     p.wsf + ((uint64_t)wt * p.k_atoms + AT * kt) * 512u, atoms * 512u, fb, pol_w);
     }
   }
   if (warp == 1) {
@@ -306,20 +406,24 @@ __global__ void __launch_bounds__(kThreads, 2) mxf4_gemm_smallm_kernel(
       // let the next kernel start its set-up.
       asm volatile("griddepcontrol.wait;" ::: "memory");
       asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+      const uint64_t pol_w = l2_policy_evict_first();
       for (uint32_t i = 0; i < pre; ++i) {
         const uint32_t kt = kt0 + i;
         const uint32_t atoms = (p.k_atoms - AT * kt) >= AT ? AT : p.k_atoms - AT * kt;
         const uint32_t fb = bar_full + 8 * i;
         if (!p.w_early) {
-          mbar_arrive_expect_tx(fb, C::A_STAGE + C::B_STAGE + 2u * atoms * 512u);
-          tma_load_2d(sbase + C::OFF_A + i * C::A_STAGE, &tmap_w, fb, (int32_t)(kt * 128u),
-                      (int32_t)(wt * 128u));
-          bulk_load(sbase + C::OFF_SFA + i * C::SF_STAGE,
-                    p.wsf + ((uint64_t)wt * p.k_atoms + AT * kt) * 512u, atoms * 512u, fb);
+          mbar_arrive_expect_tx(fb, C::A_STAGE + C::B_STAGE + (FX ? 1u : 2u) * atoms * 512u);
+          tma_load_2d_hint(sbase + C::OFF_A + i * C::A_STAGE, &tmap_w, fb, (int32_t)(kt * 128u),
+                           (int32_t)(wt * 128u), pol_w);
+          bulk_load_hint(sbase + C::OFF_SFA + i * C::SF_STAGE,
+                         p.wsf + ((uint64_t)wt * p.k_atoms + AT * kt) * 512u, atoms * 512u, fb,
+                         pol_w);
         }
-        tma_load_2d(sbase + C::OFF_B + i * C::B_STAGE, &tmap_x, fb, (int32_t)(kt * 128u), 0);
-        bulk_load(sbase + C::OFF_SFB + i * C::SF_STAGE, p.xsf + (uint64_t)(AT * kt) * 512u,
-                  atoms * 512u, fb);
+        if constexpr (!FX) {
+          tma_load_2d(sbase + C::OFF_B + i * C::B_STAGE, &tmap_x, fb, (int32_t)(kt * 128u), 0);
+          bulk_load(sbase + C::OFF_SFB + i * C::SF_STAGE, p.xsf + (uint64_t)(AT * kt) * 512u,
+                    atoms * 512u, fb);
+        }
       }
       uint32_t stage = pre % STAGES, phase = pre == STAGES ? 1u : 0u, issued = pre;
       bool ok = true;
@@ -330,14 +434,18 @@ __global__ void __launch_bounds__(kThreads, 2) mxf4_gemm_smallm_kernel(
         }
         const uint32_t atoms = (p.k_atoms - AT * kt) >= AT ? AT : p.k_atoms - AT * kt;
         const uint32_t fb = bar_full + 8 * stage;
-        mbar_arrive_expect_tx(fb, C::A_STAGE + C::B_STAGE + 2u * atoms * 512u);
-        tma_load_2d(sbase + C::OFF_A + stage * C::A_STAGE, &tmap_w, fb, (int32_t)(kt * 128u),
-                    (int32_t)(wt * 128u));
-        tma_load_2d(sbase + C::OFF_B + stage * C::B_STAGE, &tmap_x, fb, (int32_t)(kt * 128u), 0);
-        bulk_load(sbase + C::OFF_SFA + stage * C::SF_STAGE,
-                  p.wsf + ((uint64_t)wt * p.k_atoms + AT * kt) * 512u, atoms * 512u, fb);
-        bulk_load(sbase + C::OFF_SFB + stage * C::SF_STAGE, p.xsf + (uint64_t)(AT * kt) * 512u,
-                  atoms * 512u, fb);
+        mbar_arrive_expect_tx(fb, C::A_STAGE + C::B_STAGE + (FX ? 1u : 2u) * atoms * 512u);
+        tma_load_2d_hint(sbase + C::OFF_A + stage * C::A_STAGE, &tmap_w, fb, (int32_t)(kt * 128u),
+                         (int32_t)(wt * 128u), pol_w);
+        bulk_load_hint(sbase + C::OFF_SFA + stage * C::SF_STAGE,
+                       p.wsf + ((uint64_t)wt * p.k_atoms + AT * kt) * 512u, atoms * 512u, fb,
+                       pol_w);
+        if constexpr (!FX) {
+          tma_load_2d(sbase + C::OFF_B + stage * C::B_STAGE, &tmap_x, fb, (int32_t)(kt * 128u),
+                      0);
+          bulk_load(sbase + C::OFF_SFB + stage * C::SF_STAGE, p.xsf + (uint64_t)(AT * kt) * 512u,
+                    atoms * 512u, fb);
+        }
         ++issued;
         if (++stage == STAGES) {
           stage = 0;
@@ -363,22 +471,25 @@ __global__ void __launch_bounds__(kThreads, 2) mxf4_gemm_smallm_kernel(
       uint32_t stage = 0, phase = 0;
       bool ok = true;
       for (uint32_t kt = kt0; kt < kt1; ++kt) {
-        if (!mbar_wait_bounded(bar_full + 8 * stage, phase, abort_flag, kWaitLimitNs)) {
+        if (!mbar_wait_bounded(bar_full + 8 * stage, phase, abort_flag, kWaitLimitNs) ||
+            (FX && !mbar_wait_bounded(bar_xready + 8 * (kt - kt0), 0, abort_flag, kWaitLimitNs))) {
           ok = false;
           break;
         }
         tc_fence_after();
         const uint32_t atoms = (p.k_atoms - AT * kt) >= AT ? AT : p.k_atoms - AT * kt;
+        const uint32_t sfb_src = FX ? sbase + C::OFF_XSF + (kt - kt0) * C::SF_STAGE
+                                    : sbase + C::OFF_SFB + stage * C::SF_STAGE;
         for (uint32_t a = 0; a < atoms; ++a) {
           tmem_cp_32x128b_warpx4(tmem_base + C::SFA_COL + 4 * a,
                                  smem_desc_sf(sbase + C::OFF_SFA + stage * C::SF_STAGE + a * 512));
-          tmem_cp_32x128b_warpx4(tmem_base + C::SFB_COL + 4 * a,
-                                 smem_desc_sf(sbase + C::OFF_SFB + stage * C::SF_STAGE + a * 512));
+          tmem_cp_32x128b_warpx4(tmem_base + C::SFB_COL + 4 * a, smem_desc_sf(sfb_src + a * 512));
         }
         const uint32_t k_left = p.K - kt * 256u;
         const uint32_t steps = k_left >= 256u ? 4u : (k_left + 63u) / 64u;
         const uint32_t a_tile = sbase + C::OFF_A + stage * C::A_STAGE;
-        const uint32_t b_tile = sbase + C::OFF_B + stage * C::B_STAGE;
+        const uint32_t b_tile = FX ? sbase + C::OFF_XQ + (kt - kt0) * C::XQ_KT
+                                   : sbase + C::OFF_B + stage * C::B_STAGE;
         for (uint32_t k = 0; k < steps; ++k) {
           const uint32_t sf_id = (k & 1u) * 2u;
           const uint32_t acc_in = (kt != kt0 || k != 0) ? 1u : 0u;
@@ -407,6 +518,7 @@ __global__ void __launch_bounds__(kThreads, 2) mxf4_gemm_smallm_kernel(
     // TMEM lane = W row = output column c of the tile, TMEM column = token m. The
     // accumulator goes to shared memory as red[m][c] (fp32): a warp's stores for one
     // token are 128 consecutive bytes.
+    if constexpr (FX) quantize_x_slice<NT>(p, kc, sbase, kt0, kt1, bar_xready);
     const uint32_t c = (warp & 3u) * 32u + lane;
     const bool ok = mbar_wait_bounded(bar_tfull, 0, abort_flag, kWaitLimitNs);
     if (__all_sync(0xffffffffu, ok)) {
@@ -509,17 +621,19 @@ Plan make_plan(int64_t M, int64_t N, int64_t K) {
   return pl;
 }
 
-template <uint32_t NT, int OUT, bool NV>
+// FX: aq / asf unused; x (bf16, row stride ldx) is rotated by xmode and quantised inside.
+template <uint32_t NT, int OUT, bool NV, bool FX = false>
 cudaError_t launch_nt(const Plan& pl, const uint8_t* aq, const uint8_t* asf, const uint8_t* bq,
                       const uint8_t* bsf, int64_t M, int64_t N, int64_t K, void* y,
                       const Epilogue& ep, int64_t ldy, int* status, bool w_early,
-                      cudaStream_t stream) {
-  using C = SmallConfig<NT, NV>;
-  CUtensorMap tw, tx;
+                      cudaStream_t stream, const void* x = nullptr, int64_t ldx = 0,
+                      int xmode = 0, const KronCoeffs* xkc = nullptr) {
+  using C = SmallConfig<NT, NV, FX>;
+  CUtensorMap tw, tx{};
   if (!operand_map(&tw, bq, (uint64_t)N, (uint64_t)(K / 2), 128) ||
-      !operand_map(&tx, aq, (uint64_t)M, (uint64_t)(K / 2), NT))
+      (!FX && !operand_map(&tx, aq, (uint64_t)M, (uint64_t)(K / 2), NT)))
     return cudaErrorInvalidValue;
-  auto kern = mxf4_gemm_smallm_kernel<NT, OUT, NV>;
+  auto kern = mxf4_gemm_smallm_kernel<NT, OUT, NV, FX>;
   int dev = 0;
   cudaGetDevice(&dev);
   static bool attr_done[64] = {};
@@ -550,6 +664,9 @@ cudaError_t launch_nt(const Plan& pl, const uint8_t* aq, const uint8_t* asf, con
   p.n_katoms_y = (uint32_t)sf_katoms(N);
   p.a_scale = ep.a_scale;
   p.b_scale = ep.b_scale;
+  p.x = x;
+  p.ldx = (uint64_t)ldx;
+  p.xmode = (uint32_t)xmode;
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(pl.units);
   cfg.blockDim = dim3(kThreads);
@@ -564,10 +681,27 @@ cudaError_t launch_nt(const Plan& pl, const uint8_t* aq, const uint8_t* asf, con
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, kern, tw, tx, p, ep.kc);
+  return cudaLaunchKernelEx(&cfg, kern, tw, tx, p, FX ? *xkc : ep.kc);
 }
 
 }  // namespace
+
+bool linear_smallm_fits(int64_t M, int64_t N, int64_t K, int mode) {
+  if (M < 1 || M > kFxMaxRows || mode < 0 || mode > 2) return false;
+  const Plan pl = make_plan(M, N, K);
+  return pl.nt == 16 && pl.kt_per_split <= kFxMaxKt;
+}
+
+cudaError_t launch_linear_smallm(const void* x, int64_t ldx, int mode, const KronCoeffs* kc,
+                                 const uint8_t* wq, const uint8_t* wsf, int64_t M, int64_t N,
+                                 int64_t K, void* y, int64_t ldy, int* status,
+                                 cudaStream_t stream) {
+  if (!linear_smallm_fits(M, N, K, mode)) return cudaErrorNotSupported;
+  const Plan pl = make_plan(M, N, K);
+  return launch_nt<16, kOutBf16, false, true>(pl, nullptr, nullptr, wq, wsf, M, N, K, y,
+                                              Epilogue{}, ldy, status, false, stream, x, ldx,
+                                              mode, kc);
+}
 
 cudaError_t launch_gemm_smallm(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq,
                                const uint8_t* bsf, int64_t M, int64_t N, int64_t K, void* y,

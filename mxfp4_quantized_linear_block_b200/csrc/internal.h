@@ -87,6 +87,17 @@ cudaError_t launch_gemm_smallm(const uint8_t* aq, const uint8_t* asf, const uint
                                const Epilogue& ep, int64_t ldy, int* status, bool b_early,
                                cudaStream_t stream);
 
+// The whole layer for 1..8 bf16 activation rows in one launch (gemm_smallm.cu): each
+// CTA rotates (mode 0/1/2) and quantises its own K range of x into shared memory while
+// it streams W. Returns cudaErrorNotSupported (launching nothing) when the problem is
+// outside that kernel's limits (linear_smallm_fits false); the caller then quantises
+// and multiplies separately.
+bool linear_smallm_fits(int64_t M, int64_t N, int64_t K, int mode);
+cudaError_t launch_linear_smallm(const void* x, int64_t ldx, int mode, const KronCoeffs* kc,
+                                 const uint8_t* wq, const uint8_t* wsf, int64_t M, int64_t N,
+                                 int64_t K, void* y, int64_t ldy, int* status,
+                                 cudaStream_t stream);
+
 // Scale-factor layout helpers (host side).
 inline int64_t sf_katoms(int64_t K) { return (K / 32 + 3) / 4; }
 inline int64_t sf_row_tiles(int64_t rows) { return (rows + 127) / 128; }

@@ -96,6 +96,10 @@ extern "C" mxfp4_status mxfp4_linear_noalloc(const void* x, int64_t M, int64_t K
   }
   uint8_t* xq = scratch + q_off;
   uint8_t* xsf = scratch + sf_off;
+  // Up to 16 rows: one kernel quantises x inside the GEMM's CTAs.
+  const cudaError_t fe = launch_linear_smallm(x, K, (int)mode, &kc, wq, wsf, M, N, K, y, N,
+                                              status_word, s);
+  if (fe != cudaErrorNotSupported) return fe == cudaSuccess ? MXFP4_OK : MXFP4_ERR_CUDA;
   if (launch_rotate_quantize(x, false, M, K, K, (int)mode, &kc, xq, xsf, status_word, s) !=
       cudaSuccess)
     return MXFP4_ERR_CUDA;

@@ -152,3 +152,19 @@ def test_empty_calls_accept_null_row_operands():
     assert L.mxfp4_linear(P, 4, 64, 1, None, None, P, P, 32, None, P, 1 << 20, None) == \
         mx.ERR_INVALID_ARG
     assert L.mxfp4_linear_noalloc(None, 0, 64, 1, None, None, P, P, 32, None, None, None) == mx.OK
+
+
+def test_linear_kernel_count():
+    """One kernel for 1..8 rows with rotation 0/1/2 and short K splits, two otherwise."""
+    kc = mx.linear_kernel_count
+    assert kc(1, 14336, 4096, mx.ROT_HADAMARD32) == 1
+    assert kc(8, 4096, 14336, mx.ROT_KRON_4x8) == 1
+    assert kc(4, 128, 256, mx.ROT_NONE) == 1
+    assert kc(9, 4096, 14336, mx.ROT_HADAMARD32) == 2
+    assert kc(128, 4096, 14336, mx.ROT_HADAMARD32) == 2
+    assert kc(1, 4096, 4096, mx.ROT_HADAMARD64) == 2
+    assert kc(5, 150 * 128, 3584, mx.ROT_HADAMARD32) == 2  # one split of 14 k-tiles
+    assert kc(0, 128, 256, mx.ROT_HADAMARD32) == 0
+    assert kc(1, 128, 48, mx.ROT_HADAMARD32) == -1
+    assert kc(1, 24, 256, mx.ROT_HADAMARD32) == -1
+    assert kc(1, 128, 256, 9) == -1
