@@ -108,9 +108,12 @@ int64_t mxfp4_sf_offset(int64_t row, int64_t kblock, int64_t K);
 
 /* Device workspace that `op` needs for this problem (0 if none). It starts with
  * a status word; for MXFP4_OP_LINEAR it also holds the quantised activations;
- * for both GEMM-running ops it ends with the GEMM's scratch (K-split partials
+ * for both GEMM-running ops it ends with the GEMM's scratch (K-split partials,
  * and counters for the last round of output tiles; sized for a 148-SM B200).
- * Allocate it zeroed: every call that completes leaves the scratch zeroed. */
+ * Allocate it zeroed: every call that completes leaves the counters zero (the
+ * partials are rewritten before they are read, so their contents do not
+ * matter). With a smaller scratch than this size, the few-row GEMM (M <= 128)
+ * sums its K splits on chip instead (same bits, slower for 33..128 rows). */
 size_t mxfp4_workspace_bytes(int op, int64_t M, int64_t N, int64_t K);
 
 /* Static description of a status code. Never NULL. */
@@ -165,11 +168,13 @@ mxfp4_status mxfp4_rotate_quantize(const void* x, mxfp4_dtype xdt, int64_t rows,
  * both in the formats above. y: row-major [M, N] with leading dimension ldy
  * elements. Requirements: K % 32 == 0, N % 16 == 0, ldy >= N, y 16-byte aligned
  * and ldy * elemsize a multiple of 16; aq, bq, asf, bsf 16-byte aligned.
- * ws must hold mxfp4_workspace_bytes(MXFP4_OP_GEMM, M, N, K) bytes (at least
- * 256), zeroed when allocated; its first 16 bytes are the device status word
- * (see mxfp4_poll_status). On a GPU whose SM count needs more scratch than
- * that, the last round of tiles is not split along K (slower; the result
- * still meets the stated tolerance).
+ * ws: at least 256 bytes, zeroed when allocated; its first 16 bytes are the
+ * device status word (see mxfp4_poll_status). mxfp4_workspace_bytes(
+ * MXFP4_OP_GEMM, M, N, K) bytes give the fastest form; with less scratch (or
+ * on a GPU whose SM count needs more), the last round of tiles is not split
+ * along K and the few-row kernel sums its K splits on chip (slower; the
+ * result still meets the stated tolerance, and the few-row sums are the same
+ * bits). Fewer than 256 bytes -> MXFP4_ERR_WORKSPACE.
  * ("AMD Quark...", opening section: MXFP4 GEMM with no dequantisation;
  * "Bridging the Gap...", "GPU Kernel Ondersteuning (QuTLASS)".)
  */

@@ -196,7 +196,7 @@ mxfp4_status mxfp4_gemm(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq
   if (st != MXFP4_OK) return st;
   if (!ws) return MXFP4_ERR_INVALID_ARG;
   if (!aligned16(ws)) return MXFP4_ERR_ALIGN;
-  if (ws_bytes < mxfp4_workspace_bytes(MXFP4_OP_GEMM, M, N, K)) return MXFP4_ERR_WORKSPACE;
+  if (ws_bytes < kStatusBytes) return MXFP4_ERR_WORKSPACE;  // scratch: optional, see header
   if (M == 0) return MXFP4_OK;
   // The caller's previous kernel may have written bq / bsf: no early weight loads.
   Epilogue ep;
@@ -214,7 +214,7 @@ mxfp4_status mxfp4_gemm_bias(const uint8_t* aq, const uint8_t* asf, const uint8_
   if (st != MXFP4_OK) return st;
   if (!ws || !bias) return MXFP4_ERR_INVALID_ARG;
   if (!aligned16(ws) || !aligned16(bias)) return MXFP4_ERR_ALIGN;
-  if (ws_bytes < mxfp4_workspace_bytes(MXFP4_OP_GEMM, M, N, K)) return MXFP4_ERR_WORKSPACE;
+  if (ws_bytes < kStatusBytes) return MXFP4_ERR_WORKSPACE;  // scratch: optional, see header
   if (M == 0) return MXFP4_OK;
   Epilogue ep;
   ep.out = ydt == MXFP4_DT_F32 ? kOutF32 : kOutBf16;
@@ -241,7 +241,7 @@ mxfp4_status mxfp4_gemm_quantize(const uint8_t* aq, const uint8_t* asf, const ui
   if (!aligned16(aq) || !aligned16(asf) || !aligned16(bq) || !aligned16(bsf) || !aligned16(yq) ||
       !aligned16(ysf) || !aligned16(ws) || (bias && !aligned16(bias)))
     return MXFP4_ERR_ALIGN;
-  if (ws_bytes < mxfp4_workspace_bytes(MXFP4_OP_GEMM, M, N, K)) return MXFP4_ERR_WORKSPACE;
+  if (ws_bytes < kStatusBytes) return MXFP4_ERR_WORKSPACE;  // scratch: optional, see header
   Epilogue ep;
   ep.out = kOutMxfp4;
   ep.bias = bias;
@@ -399,7 +399,7 @@ mxfp4_status mxfp4_nvfp4_gemm(const uint8_t* aq, const uint8_t* asf, const float
   if (!aligned16(ws) || (reinterpret_cast<uintptr_t>(a_scale) & 3u) ||
       (reinterpret_cast<uintptr_t>(b_scale) & 3u))
     return MXFP4_ERR_ALIGN;
-  if (ws_bytes < mxfp4_workspace_bytes(MXFP4_OP_GEMM, M, N, K)) return MXFP4_ERR_WORKSPACE;
+  if (ws_bytes < kStatusBytes) return MXFP4_ERR_WORKSPACE;  // scratch: optional, see header
   if (M == 0) return MXFP4_OK;
   Epilogue ep;
   ep.out = ydt == MXFP4_DT_F32 ? kOutF32 : kOutBf16;

@@ -768,7 +768,8 @@ cudaError_t launch_gemm(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq
                         size_t scratch_bytes, bool b_early, cudaStream_t stream) {
   // Few activation rows: stream the weights with the swap-AB split-K kernel.
   if (M <= 128)
-    return launch_gemm_smallm(aq, asf, bq, bsf, M, N, K, y, ep, ldy, status, b_early, stream);
+    return launch_gemm_smallm(aq, asf, bq, bsf, M, N, K, y, ep, ldy, status, scratch,
+                              scratch_bytes, b_early, stream);
   // Otherwise CTA pairs with 256 x 256 tiles.
   if (ep.nvfp4) {
     if (ep.out == kOutF32)
@@ -791,7 +792,7 @@ cudaError_t launch_gemm(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq
 }
 
 size_t gemm_scratch_bytes(int64_t M, int64_t N, int64_t K) {
-  if (M <= 128) return 0;
+  if (M <= 128) return gemm_smallm_scratch_bytes(M, N, K);
   return pair_plan(M, N, K, kPlanPairs).scratch_bytes;
 }
 

@@ -11,8 +11,13 @@
 // in its own shared memory (over the drained operand stages). After a cluster
 // barrier, CTA r adds the S partials of its share of the 128 columns through
 // distributed shared memory, in split order 0, 1, ..., S-1 (deterministic),
-// and writes that part of Y with coalesced row stores. No global scratch, no
-// atomics, no second kernel.
+// and writes that part of Y with coalesced row stores. No atomics, no second
+// kernel. For more than 32 tokens and 4 or more splits the partials are large
+// (up to 64 KB per CTA, mostly remote) and distributed shared memory moves them
+// at only a few tens of GB/s per SM, so they go through L2 instead: each CTA
+// writes its partial rows to a global scratch, and after the cluster barrier
+// (release / acquire at cluster scope) CTA r reads its share of all S partials
+// from L2 and adds them in the same order, so both forms give the same bits.
 //
 // The whole layer for up to 8 tokens (FX variant): the CTA's epilogue warps
 // rotate and quantise the CTA's K range of the bf16 activations themselves,
@@ -109,6 +114,7 @@ struct SmallParams {
   uint32_t n_katoms_y;  // MXFP4 output: scale atoms per 128-row group of Y
   const float* a_scale; // NVFP4: tensor scales (device fp32) of X and W
   const float* b_scale;
+  float* red_g;         // K-split partials [unit][min(M, NT)][128] fp32 in L2, or null
   const void* x;        // FX: bf16 activations [M, K], row stride ldx elements
   uint64_t ldx;
   uint32_t xmode;       // FX: rotation of each 32-element block of X (0, 1, 2)
@@ -137,13 +143,16 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 // item is one (token, group): 4 fp32 values in each split's shared memory. The 128
 // epilogue threads take items tid, tid + 128, ...; IB items at a time, whose loads from
 // all S splits are issued together, then added in split order 0, 1, ..., S-1.
-template <uint32_t NT, int OUT, uint32_t S>
+// L2: the partials come from p.red_g (written by the cluster's CTAs in this launch, so
+// read at L2, not through the incoherent L1 path) instead of distributed shared memory.
+template <uint32_t NT, int OUT, uint32_t S, bool L2 = false>
 __device__ __forceinline__ void reduce_store(const SmallParams& p, uint32_t sbase, uint32_t wt,
                                              uint32_t sp, uint32_t tid, float alpha) {
   constexpr uint32_t IB = 16 / S;  // 16 loads in flight per thread
   const uint32_t g0 = sp * 32u / S, g1 = (sp + 1u) * 32u / S, width = g1 - g0;
   const uint32_t rows = p.M < NT ? p.M : NT;
   const uint32_t items = rows * width;
+  const float* red_tile = L2 ? p.red_g + (uint64_t)wt * S * rows * 128u : nullptr;
   for (uint32_t it0 = tid; it0 < items; it0 += 128u * IB) {
     float4 t[IB][S];
     uint32_t tok[IB], col[IB];
@@ -154,9 +163,16 @@ __device__ __forceinline__ void reduce_store(const SmallParams& p, uint32_t sbas
       const uint32_t g = g0 + (it - tok[i] * width);
       col[i] = wt * 128u + g * 4u;  // N % 16 == 0: the 4 columns are all in or all out
       if (it < items) {
-        const uint32_t off = sbase + red_off(tok[i], g);
+        if constexpr (L2) {
 #pragma unroll
-        for (uint32_t s = 0; s < S; ++s) t[i][s] = ld_shared_cluster_v4(map_to_rank(off, s));
+          for (uint32_t s = 0; s < S; ++s)
+            t[i][s] = __ldcg(reinterpret_cast<const float4*>(
+                red_tile + ((uint64_t)s * rows + tok[i]) * 128u + g * 4u));
+        } else {
+          const uint32_t off = sbase + red_off(tok[i], g);
+#pragma unroll
+          for (uint32_t s = 0; s < S; ++s) t[i][s] = ld_shared_cluster_v4(map_to_rank(off, s));
+        }
       }
     }
 #pragma unroll
@@ -525,16 +541,26 @@ __global__ void __launch_bounds__(kThreads, 2) mxf4_gemm_smallm_kernel(
       tc_fence_after();
       float* red = reinterpret_cast<float*>(smem);
       const uint32_t taddr = tmem_base + (((warp & 3u) * 32u) << 16);
+      // L2 form: this CTA's partial rows m < min(M, NT) at red_g[unit][m][c]; a warp's
+      // stores for one token are 128 consecutive bytes.
+      const uint32_t rows = p.M < NT ? p.M : NT;
+      float* red_g = p.red_g ? p.red_g + (uint64_t)blockIdx.x * rows * 128u + c : nullptr;
 #pragma unroll
       for (uint32_t c0 = 0; c0 < NT; c0 += 32) {
         uint32_t v[32];
         tmem_ld_32x32b_x16(taddr + c0, &v[0]);
         if (c0 + 16 < NT) tmem_ld_32x32b_x16(taddr + c0 + 16, &v[16]);
         tmem_ld_wait();
+        if (red_g != nullptr) {
 #pragma unroll
-        for (uint32_t j = 0; j < 32; ++j)
-          if (c0 + j < NT)
-            red[red_off(c0 + j, c >> 2) / 4u + (c & 3u)] = __uint_as_float(v[j]);
+          for (uint32_t j = 0; j < 32; ++j)
+            if (c0 + j < NT && c0 + j < rows) __stcg(red_g + (c0 + j) * 128u, __uint_as_float(v[j]));
+        } else {
+#pragma unroll
+          for (uint32_t j = 0; j < 32; ++j)
+            if (c0 + j < NT)
+              red[red_off(c0 + j, c >> 2) / 4u + (c & 3u)] = __uint_as_float(v[j]);
+        }
       }
     } else if (lane == 0) {
       record_timeout(p.status);
@@ -553,6 +579,16 @@ __global__ void __launch_bounds__(kThreads, 2) mxf4_gemm_smallm_kernel(
     if constexpr (NV) alpha = __fmul_rn(__ldg(p.a_scale), __ldg(p.b_scale));
     if constexpr (OUT == kOutMxfp4) {
       reduce_store_mxfp4<NT>(p, kc, sbase, wt, sp, S, tid);
+    } else if (p.red_g != nullptr) {
+      switch (S) {
+        case 2: reduce_store<NT, OUT, 2, true>(p, sbase, wt, sp, tid, alpha); break;
+        case 3: reduce_store<NT, OUT, 3, true>(p, sbase, wt, sp, tid, alpha); break;
+        case 4: reduce_store<NT, OUT, 4, true>(p, sbase, wt, sp, tid, alpha); break;
+        case 5: reduce_store<NT, OUT, 5, true>(p, sbase, wt, sp, tid, alpha); break;
+        case 6: reduce_store<NT, OUT, 6, true>(p, sbase, wt, sp, tid, alpha); break;
+        case 7: reduce_store<NT, OUT, 7, true>(p, sbase, wt, sp, tid, alpha); break;
+        default: reduce_store<NT, OUT, 8, true>(p, sbase, wt, sp, tid, alpha); break;
+      }
     } else {
       switch (S) {
         case 1: reduce_store<NT, OUT, 1>(p, sbase, wt, sp, tid, alpha); break;
@@ -567,7 +603,7 @@ __global__ void __launch_bounds__(kThreads, 2) mxf4_gemm_smallm_kernel(
     }
   }
   // No CTA leaves (and releases its shared memory) while a peer may still read it.
-  cluster_sync();
+  if (p.red_g == nullptr) cluster_sync();
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -621,13 +657,23 @@ Plan make_plan(int64_t M, int64_t N, int64_t K) {
   return pl;
 }
 
+// L2 bytes of the K-split partials (after kSmallRedOffset in the GEMM scratch): for more
+// than 32 tokens split 4 or more ways; 0 means the sum goes through distributed shared
+// memory. (B200, 128 tokens: 8 splits 15.0 -> 13.2 us through L2; 2 splits, where half
+// of the reads are the CTA's own shared memory, 13.1 -> 13.9 us, so they stay on chip.)
+size_t red_bytes(const Plan& pl, int64_t M) {
+  if (pl.splits < 4 || pl.nt < 64) return 0;
+  const int64_t rows = M < (int64_t)pl.nt ? M : (int64_t)pl.nt;
+  return (size_t)pl.units * (size_t)rows * 128u * sizeof(float);
+}
+
 // FX: aq / asf unused; x (bf16, row stride ldx) is rotated by xmode and quantised inside.
 template <uint32_t NT, int OUT, bool NV, bool FX = false>
 cudaError_t launch_nt(const Plan& pl, const uint8_t* aq, const uint8_t* asf, const uint8_t* bq,
                       const uint8_t* bsf, int64_t M, int64_t N, int64_t K, void* y,
                       const Epilogue& ep, int64_t ldy, int* status, bool w_early,
                       cudaStream_t stream, const void* x = nullptr, int64_t ldx = 0,
-                      int xmode = 0, const KronCoeffs* xkc = nullptr) {
+                      int xmode = 0, const KronCoeffs* xkc = nullptr, float* red_g = nullptr) {
   using C = SmallConfig<NT, NV, FX>;
   CUtensorMap tw, tx{};
   if (!operand_map(&tw, bq, (uint64_t)N, (uint64_t)(K / 2), 128) ||
@@ -667,6 +713,7 @@ cudaError_t launch_nt(const Plan& pl, const uint8_t* aq, const uint8_t* asf, con
   p.x = x;
   p.ldx = (uint64_t)ldx;
   p.xmode = (uint32_t)xmode;
+  p.red_g = OUT == kOutMxfp4 ? nullptr : red_g;  // the MXFP4 epilogue sums on chip
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(pl.units);
   cfg.blockDim = dim3(kThreads);
@@ -703,29 +750,33 @@ cudaError_t launch_linear_smallm(const void* x, int64_t ldx, int mode, const Kro
                                               mode, kc);
 }
 
+size_t gemm_smallm_scratch_bytes(int64_t M, int64_t N, int64_t K) {
+  const size_t r = red_bytes(make_plan(M, N, K), M);
+  return r ? kSmallRedOffset + r : 0;
+}
+
 cudaError_t launch_gemm_smallm(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq,
                                const uint8_t* bsf, int64_t M, int64_t N, int64_t K, void* y,
-                               const Epilogue& ep, int64_t ldy, int* status, bool b_early,
-                               cudaStream_t stream) {
+                               const Epilogue& ep, int64_t ldy, int* status, uint8_t* scratch,
+                               size_t scratch_bytes, bool b_early, cudaStream_t stream) {
   const Plan pl = make_plan(M, N, K);
-#define MXFP4_SMALLM(NTV)                                                                       \
-  if (ep.nvfp4) {                                                                               \
-    if (ep.out == kOutF32)                                                                      \
-      return launch_nt<NTV, kOutF32, true>(pl, aq, asf, bq, bsf, M, N, K, y, ep, ldy, status,   \
-                                           b_early, stream);                                    \
-    return launch_nt<NTV, kOutBf16, true>(pl, aq, asf, bq, bsf, M, N, K, y, ep, ldy, status,    \
-                                          b_early, stream);                                     \
-  }                                                                                             \
-  switch (ep.out) {                                                                             \
-    case kOutF32:                                                                               \
-      return launch_nt<NTV, kOutF32, false>(pl, aq, asf, bq, bsf, M, N, K, y, ep, ldy, status,  \
-                                            b_early, stream);                                   \
-    case kOutMxfp4:                                                                             \
-      return launch_nt<NTV, kOutMxfp4, false>(pl, aq, asf, bq, bsf, M, N, K, y, ep, ldy,        \
-                                              status, b_early, stream);                         \
-    default:                                                                                    \
-      return launch_nt<NTV, kOutBf16, false>(pl, aq, asf, bq, bsf, M, N, K, y, ep, ldy, status, \
-                                             b_early, stream);                                  \
+  // K-split partials through L2 when the caller's scratch holds them, else on chip
+  const size_t rb = red_bytes(pl, M);
+  float* red = rb && scratch && scratch_bytes >= kSmallRedOffset + rb
+                   ? reinterpret_cast<float*>(scratch + kSmallRedOffset)
+                   : nullptr;
+#define MXFP4_SMALLM_LAUNCH(NTV, OUTV, NVV)                                           \
+  return launch_nt<NTV, OUTV, NVV>(pl, aq, asf, bq, bsf, M, N, K, y, ep, ldy, status, \
+                                   b_early, stream, nullptr, 0, 0, nullptr, red)
+#define MXFP4_SMALLM(NTV)                                                             \
+  if (ep.nvfp4) {                                                                     \
+    if (ep.out == kOutF32) MXFP4_SMALLM_LAUNCH(NTV, kOutF32, true);                   \
+    MXFP4_SMALLM_LAUNCH(NTV, kOutBf16, true);                                         \
+  }                                                                                   \
+  switch (ep.out) {                                                                   \
+    case kOutF32: MXFP4_SMALLM_LAUNCH(NTV, kOutF32, false);                           \
+    case kOutMxfp4: MXFP4_SMALLM_LAUNCH(NTV, kOutMxfp4, false);                       \
+    default: MXFP4_SMALLM_LAUNCH(NTV, kOutBf16, false);                               \
   }
   switch (pl.nt) {
     case 16: MXFP4_SMALLM(16)
@@ -734,6 +785,7 @@ cudaError_t launch_gemm_smallm(const uint8_t* aq, const uint8_t* asf, const uint
     default: MXFP4_SMALLM(128)
   }
 #undef MXFP4_SMALLM
+#undef MXFP4_SMALLM_LAUNCH
 }
 
 }  // namespace mxfp4

@@ -82,10 +82,19 @@ cudaError_t launch_gemm(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq
 size_t gemm_scratch_bytes(int64_t M, int64_t N, int64_t K);
 
 // Few-row path (M <= 128): swap-AB, K split across the CTAs of a cluster (gemm_smallm.cu).
+// scratch: the GEMM scratch; for 33..128 rows split 4 or more ways the K-split partials
+// go through it (from kSmallRedOffset on, gemm_smallm_scratch_bytes in all) when it is
+// large enough, else they are summed through distributed shared memory. Either way the
+// bits are the same.
 cudaError_t launch_gemm_smallm(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq,
                                const uint8_t* bsf, int64_t M, int64_t N, int64_t K, void* y,
-                               const Epilogue& ep, int64_t ldy, int* status, bool b_early,
-                               cudaStream_t stream);
+                               const Epilogue& ep, int64_t ldy, int* status, uint8_t* scratch,
+                               size_t scratch_bytes, bool b_early, cudaStream_t stream);
+size_t gemm_smallm_scratch_bytes(int64_t M, int64_t N, int64_t K);
+// The few-row partials start here, past the counters at the start of the scratch that the
+// CTA-pair kernel needs zero (2 x 4 bytes per split tile, fewer than 512 tiles), so a
+// workspace shared by both kernels keeps its counters zero.
+constexpr size_t kSmallRedOffset = 4096;
 
 // The whole layer for 1..8 bf16 activation rows in one launch (gemm_smallm.cu): each
 // CTA rotates (mode 0/1/2) and quantises its own K range of x into shared memory while

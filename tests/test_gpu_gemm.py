@@ -62,7 +62,8 @@ def test_gemm_zero_and_single_pair():
 
 # Few activation rows (M <= 128): the weight-streaming kernel splits K over the
 # CTAs of a thread-block cluster and adds the partials through distributed shared
-# memory. (M, N, K) -> W tiles x K splits: (1,16,4096) 1x8; (5,400,2080) 4x5 with a
+# memory (up to 32 rows, or fewer than 4 splits) or through L2 (33..128 rows split 4 or
+# more ways, with the workspace's scratch). (M, N, K) -> W tiles x K splits: (1,16,4096) 1x8; (5,400,2080) 4x5 with a
 # 32-element K tail; (16,256,8192) 2x8; (17,12288,1024) 96x2; (33,9216,1536) 72x3;
 # (64,2048,3104) 16x7 with a K tail; (100,1024,7168) 8x7; (65,14336,4096) 112x2;
 # (128,4096,14336) 32x8.
@@ -227,3 +228,50 @@ def test_gemm_and_linear_with_no_rows_write_nothing():
     mx.linear(x, wq, wsf, N, y=y[:0])
     torch.cuda.synchronize()
     assert torch.all(y == 3.0)
+
+
+@pytest.mark.parametrize("M,N,K", [(33, 4608, 1536), (100, 1024, 7168), (128, 4096, 14336)])
+@pytest.mark.parametrize("out", ["bf16", "f32"])
+def test_few_rows_l2_and_on_chip_sums_agree(M, N, K, out):
+    """33..128 rows split 6 or 8 ways (36 W tiles x 6, 8 x 8, 32 x 8) sum their K splits
+    through L2 when the workspace has the scratch and
+    through distributed shared memory when it has only the status word: same order of
+    additions, so the same bits; both match the oracle."""
+    import torch
+    import mxfp4_quantized_linear_block_b200 as mx
+    aq, as_ = _operand(M + N + K, M, K, 12)
+    bq, bs = _operand(M + N + K, N, K, 13)
+    args = (to_dev(aq), to_dev(oracle.sf_to_physical(as_, K)), to_dev(bq),
+            to_dev(oracle.sf_to_physical(bs, K)), M, N, K)
+    dt = torch.float32 if out == "f32" else torch.bfloat16
+    full = mx.new_workspace(mx.workspace_bytes(mx.OP_GEMM, M, N, K))
+    assert full.numel() > 4096  # this size uses the L2 form
+    y_l2 = mx.gemm(*args, out_dtype=dt, ws=full)
+    y_chip = mx.gemm(*args, out_dtype=dt, ws=mx.new_workspace(256))
+    torch.cuda.synchronize()
+    assert torch.equal(y_l2, y_chip)
+    y = y_l2.cpu().numpy().astype(np.float64) if out == "f32" else bf16_dev_to_f64(y_l2)
+    ref, S = oracle.gemm(aq, as_, bq, bs)
+    check_gemm_values(y, ref, S, out, f"few-row L2 sum {M}x{N}x{K} {out}")
+    assert mx.poll_status(full) == mx.OK
+
+
+def test_workspace_shared_by_few_row_and_pair_kernels():
+    """The few-row kernel's L2 partials leave the pair kernel's split counters (the first
+    bytes of the scratch) zero: one workspace serves a 128-row call, then a split call."""
+    import torch
+    import mxfp4_quantized_linear_block_b200 as mx
+    shapes = [(128, 4096, 14336), (512, 512, 4096)]
+    ws = mx.new_workspace(max(mx.workspace_bytes(mx.OP_GEMM, *sh) for sh in shapes))
+    for rep in range(2):
+        for (M, N, K) in shapes:
+            aq, as_ = _operand(M + N, M, K, 14)
+            bq, bs = _operand(M + N, N, K, 15)
+            y = mx.gemm(to_dev(aq), to_dev(oracle.sf_to_physical(as_, K)), to_dev(bq),
+                        to_dev(oracle.sf_to_physical(bs, K)), M, N, K, out_dtype=torch.float32,
+                        ws=ws)
+            torch.cuda.synchronize()
+            ref, S = oracle.gemm(aq, as_, bq, bs)
+            check_gemm_values(y.cpu().numpy().astype(np.float64), ref, S, "f32",
+                              f"shared workspace {M}x{N}x{K} pass {rep}")
+            assert mx.poll_status(ws) == mx.OK
