@@ -422,9 +422,11 @@ def run_ours(args, rank, world, local_rank):
     value = job_tflops(flops_step, args.steps, world, elapsed)
     ms_per_step = elapsed / args.steps * 1e3
     # kernels per linear: quantise + GEMM, or one kernel when the layer quantises x inside
-    # the GEMM's CTAs (1..8 rows); NVFP4 adds the tensor-scale pass (2 kernels), the norm
-    # prologue the row-statistics kernel
-    kcount = [4 if nv else 3 if norm is not None else
+    # the GEMM's CTAs (1..8 rows); NVFP4 adds the tensor-scale pass (2 kernels); the norm
+    # prologue is one kernel with the quantiser while a row fits in shared memory, else it
+    # adds the row-statistics kernel
+    kcount = [4 if nv else
+              mx.norm_linear_kernel_count(l.M, l.N, l.K, wl.rotation) if norm is not None else
               mx.linear_kernel_count(l.M, l.N, l.K, wl.rotation) for l in wl.linears]
     fused = [k == 1 for k in kcount]
     launches = sum(kcount) * args.steps
@@ -508,11 +510,12 @@ def run_ours(args, rank, world, local_rank):
     gemm_bytes = np.array([(2 * l.M * l.K if fused[j] else l.M * l.K // 2 + sfb(l.M, l.K)) +
                            l.N * l.K // 2 + sfb(l.N, l.K) + 2 * l.M * l.N
                            for j, l in enumerate(wl.linears)], np.float64)
-    # NVFP4's dynamic tensor scale, and the norm's row statistics, need a full pass over X
-    # before the quantiser reads it
+    # NVFP4's dynamic tensor scale, and the norm's row statistics when they are a kernel of
+    # their own, need a full pass over X before the quantiser reads it
     q_bytes = np.array([0.0 if fused[j] else
-                        (4 if nv or norm is not None else 2) * l.M * l.K + l.M * l.K // 2 +
-                        sfb(l.M, l.K) for j, l in enumerate(wl.linears)], np.float64)
+                        (4 if nv or (norm is not None and kcount[j] == 3) else 2) * l.M * l.K +
+                        l.M * l.K // 2 + sfb(l.M, l.K) for j, l in enumerate(wl.linears)],
+                       np.float64)
     fp4_peak = peaks["bf16_tflops_sustained"] * FP4_OVER_BF16
     q_sel = [j for j in range(n_lin) if not fused[j]]
     q_ach = q_bytes[q_sel].sum() / t_q[q_sel].sum() / 1e9 if q_sel else None
@@ -624,7 +627,9 @@ def run_ours(args, rank, world, local_rank):
         "roofline": roofline,
         "quantize_roofline": ({"bound": "hbm",
                                "kernel": ("nvfp4_amax_kernel + rotate_quantize_kernel" if nv else
-                                          "row_stats_kernel + rotate_quantize_kernel"
+                                          ("norm_rows_kernel (one pass)"
+                                           if all(k == 2 for k in kcount) else
+                                           "row_stats_kernel + rotate_quantize_kernel")
                                           if norm is not None else "rotate_quantize_kernel"),
                                "achieved": q_ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                                "frac": q_ach / peaks["hbm_gbs"],

@@ -247,13 +247,15 @@ int mxfp4_linear_kernel_count(int64_t M, int64_t N, int64_t K, mxfp4_rotation mo
  * Norm prologue: the normalisation that precedes the layer, applied inside the
  * quantiser instead of as a separate pass that writes a normalised bf16 copy
  * of x ("KroQuant...", "Hintergrund": the norms are why the transform runs
- * online). A first kernel computes per-row statistics into stats (DEVICE,
- * [rows][2] fp32, 8-byte aligned; also an output): LayerNorm mu = mean,
- * rstd = 1 / sqrt(var + eps); RMSNorm mu = 0, rstd = 1 / sqrt(mean(x^2) + eps)
- * (fp32 sums over the row). The quantiser then rotates and quantises
- * v = ((x - mu) * rstd) * g[c] + b[c] (fp32, in that order; g / b: DEVICE fp32
- * [K], 16-byte aligned, NULL for 1 / 0 -- for adaLN modulation pass
- * g = 1 + scale and b = shift). x is bf16; modes NONE / HADAMARD32 / KRON_4x8;
+ * online). Per-row statistics go to stats (DEVICE, [rows][2] fp32, 8-byte
+ * aligned; also an output): LayerNorm mu = mean, rstd = 1 / sqrt(var + eps);
+ * RMSNorm mu = 0, rstd = 1 / sqrt(mean(x^2) + eps) (fp32 sums over the row,
+ * in an order the library chooses). Then v = ((x - mu) * rstd) * g[c] + b[c]
+ * (fp32, in that order; g / b: DEVICE fp32 [K], 16-byte aligned, NULL for
+ * 1 / 0 -- for adaLN modulation pass g = 1 + scale and b = shift) is rotated
+ * and quantised. For K <= 6144 one kernel does both from whole rows copied
+ * into shared memory (x read once); longer rows take a statistics kernel and
+ * then the quantiser. x is bf16; modes NONE / HADAMARD32 / KRON_4x8;
  * otherwise as mxfp4_rotate_quantize.
  */
 mxfp4_status mxfp4_norm_rotate_quantize(const void* x, int64_t rows, int64_t K, int64_t ldx,
@@ -270,6 +272,15 @@ mxfp4_status mxfp4_norm_linear(const void* x, int64_t M, int64_t K, mxfp4_norm k
                                const float* kron_a, const float* kron_b, const uint8_t* wq,
                                const uint8_t* wsf, int64_t N, void* y, void* ws,
                                size_t ws_bytes, mxfp4_stream_t stream);
+
+/*
+ * How many kernels mxfp4_norm_linear launches for these sizes: 2 when the
+ * norm, rotation and quantisation run as one kernel that copies whole rows
+ * into shared memory (K <= 6144), then the GEMM; 3 otherwise (row
+ * statistics, quantiser, GEMM); 0 for M == 0; -1 for arguments it rejects.
+ * mxfp4_norm_rotate_quantize launches one kernel fewer. Host only.
+ */
+int mxfp4_norm_linear_kernel_count(int64_t M, int64_t N, int64_t K, mxfp4_rotation mode);
 
 /*
  * NVFP4, the other FP4 format the pages compare ("Bridging the Gap Between

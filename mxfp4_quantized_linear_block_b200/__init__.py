@@ -31,7 +31,7 @@ EXPORTS = (
     "mxfp4_poll_status", "mxfp4_linear_noalloc", "mxfp4_gemm_bias", "mxfp4_gemm_quantize",
     "mxfp4_nvfp4_sf_bytes", "mxfp4_nvfp4_tensor_scale", "mxfp4_nvfp4_quantize",
     "mxfp4_nvfp4_gemm", "mxfp4_nvfp4_linear", "mxfp4_norm_rotate_quantize", "mxfp4_norm_linear",
-    "mxfp4_linear_kernel_count",
+    "mxfp4_linear_kernel_count", "mxfp4_norm_linear_kernel_count",
 )
 
 
@@ -73,6 +73,7 @@ def _load() -> ctypes.CDLL:
         "mxfp4_norm_linear": ([vp, i64, i64, i32, ctypes.c_float, vp, vp, i32, vp, vp, vp, vp,
                                i64, vp, vp, sz, vp], i32),
         "mxfp4_linear_kernel_count": ([i64, i64, i64, i32], i32),
+        "mxfp4_norm_linear_kernel_count": ([i64, i64, i64, i32], i32),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -392,6 +393,12 @@ def linear_kernel_count(M: int, N: int, K: int, mode: int = ROT_HADAMARD32) -> i
     """Kernels that linear() launches for these sizes: 1 (x quantised inside the GEMM's
     CTAs), 2 (quantiser + GEMM), 0 (M == 0); -1 for arguments linear() rejects."""
     return int(lib.mxfp4_linear_kernel_count(M, N, K, mode))
+
+
+def norm_linear_kernel_count(M: int, N: int, K: int, mode: int = ROT_HADAMARD32) -> int:
+    """Kernels that norm_linear() launches: 2 (one-pass norm quantiser + GEMM, K <= 6144),
+    3 (row statistics + quantiser + GEMM), 0 (M == 0); -1 for arguments it rejects."""
+    return int(lib.mxfp4_norm_linear_kernel_count(M, N, K, mode))
 
 
 def poll_status(ws) -> int:

@@ -298,6 +298,15 @@ int mxfp4_linear_kernel_count(int64_t M, int64_t N, int64_t K, mxfp4_rotation mo
   return linear_smallm_fits(M, N, K, (int)mode) ? 1 : 2;
 }
 
+int mxfp4_norm_linear_kernel_count(int64_t M, int64_t N, int64_t K, mxfp4_rotation mode) {
+  if (mode != MXFP4_ROT_NONE && mode != MXFP4_ROT_HADAMARD32 && mode != MXFP4_ROT_KRON_4x8)
+    return -1;
+  if (!shape_ok(M, K) || N < 16 || N % 16 != 0 || !within_limits(M, K) || !within_limits(N, K))
+    return -1;
+  if (M == 0) return 0;
+  return norm_one_pass(K) ? 2 : 3;
+}
+
 mxfp4_status mxfp4_norm_rotate_quantize(const void* x, int64_t rows, int64_t K, int64_t ldx,
                                         mxfp4_norm kind, float eps, const float* g,
                                         const float* b, mxfp4_rotation mode, const float* kron_a,

@@ -16,7 +16,10 @@ def _vec(seed, K, mean, std):
 
 
 @pytest.mark.parametrize("kind", [oracle.NORM_LAYER, oracle.NORM_RMS])
-@pytest.mark.parametrize("rows,K", [(1, 64), (5, 3072), (129, 1024), (300, 12288)])
+# K <= 6144 (8 or 16 rows per CTA) takes the one-pass kernel; K = 6176 and 12288 the
+# statistics kernel + norm quantiser.
+@pytest.mark.parametrize("rows,K", [(1, 64), (5, 3072), (129, 1024), (17, 6144), (9, 6176),
+                                    (300, 12288)])
 @pytest.mark.parametrize("affine", [False, True])
 def test_norm_rotate_quantize(kind, rows, K, affine):
     import torch
