@@ -554,7 +554,8 @@ __global__ void __launch_bounds__(kThreads, 2) mxf4_gemm_smallm_kernel(
         if (red_g != nullptr) {
 #pragma unroll
           for (uint32_t j = 0; j < 32; ++j)
-            if (c0 + j < NT && c0 + j < rows) __stcg(red_g + (c0 + j) * 128u, __uint_as_float(v[j]));
+            if (c0 + j < NT && c0 + j < rows)
+              __stcg(red_g + (c0 + j) * 128u, __uint_as_float(v[j]));
         } else {
 #pragma unroll
           for (uint32_t j = 0; j < 32; ++j)
