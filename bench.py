@@ -55,17 +55,17 @@ PKG = "mxfp4_quantized_linear_block_b200"
 # kernel ends is written back later and is not counted (hence writes < Y bytes).
 NCU_TRAFFIC = {
     "dit_b1": {"source": f"{PKG}/csrc/gemm.cu",
-               "sha256": "ce8e9516555dcfd97b35b07bdfb668fd861f456dfe64b4a097ae55ed6b6ef456",
-               "bytes_per_launch": [20933888 + 12544000, 26112768 + 37123840,
-                                    43493120 + 4070144]},
+               "sha256": "2c72c144e76ac116fcb8b15e0baa3282996a0905199fe131db814be17a28a7d7",
+               "bytes_per_launch": [20943104 + 15270400, 26347520 + 38186496,
+                                    43526656 + 6366976]},
     "llm_small_m1": {"source": f"{PKG}/csrc/gemm_smallm.cu",
-                     "sha256": "17c99c26969ae4178694fdbd5d747735da958b59a157ff608b180262894be314",
-                     "bytes_per_launch": [31281920 + 0, 31299840 + 0]},
+                     "sha256": "908f4b942417d3a74078820ae1ab25ec583f1c82cf7514773a8c7c84ee7fc6ac",
+                     "bytes_per_launch": [31283456 + 0, 31301376 + 0]},
 }
 NCU_TRAFFIC_QUANTIZE = {
     "dit_b1": {"source": f"{PKG}/csrc/quantize.cu",
-               "sha256": "07f72460d21f61c42649b20e4cb913f50a43b32a3400be2da00f8e645ead3913",
-               "bytes_per_launch": [22033664 + 0, 22033920 + 0, 88096000 + 4988160]},
+               "sha256": "41177f864f0c9cd1568db157a6f61f1db0b2fda040ccb3c5481d3767108415dc",
+               "bytes_per_launch": [22033664 + 0, 22033408 + 0, 88096256 + 4231936]},
 }
 
 
@@ -627,9 +627,12 @@ def run_ours(args, rank, world, local_rank):
         "roofline": roofline,
         "quantize_roofline": ({"bound": "hbm",
                                "kernel": ("nvfp4_amax_kernel + rotate_quantize_kernel" if nv else
-                                          ("norm_rows_kernel (one pass)"
-                                           if all(k == 2 for k in kcount) else
-                                           "row_stats_kernel + rotate_quantize_kernel")
+                                          "; ".join(
+                                              f"{l.name}: " + ("norm_rows_kernel (one pass)"
+                                                               if kcount[j] == 2 else
+                                                               "row_stats_kernel + "
+                                                               "rotate_quantize_kernel")
+                                              for j, l in enumerate(wl.linears))
                                           if norm is not None else "rotate_quantize_kernel"),
                                "achieved": q_ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                                "frac": q_ach / peaks["hbm_gbs"],
