@@ -64,8 +64,8 @@ NCU_TRAFFIC = {
 }
 NCU_TRAFFIC_QUANTIZE = {
     "dit_b1": {"source": f"{PKG}/csrc/quantize.cu",
-               "sha256": "41177f864f0c9cd1568db157a6f61f1db0b2fda040ccb3c5481d3767108415dc",
-               "bytes_per_launch": [22033664 + 0, 22033408 + 0, 88096256 + 4231936]},
+               "sha256": "0bc4e6bbf44f13a10a5fca392f9bc3a7a4a2e20e9f8d1d362cfe5b1b167b7261",
+               "bytes_per_launch": [22033408 + 0, 22033920 + 0, 88103168 + 4817664]},
 }
 
 

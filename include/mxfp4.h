@@ -253,7 +253,7 @@ int mxfp4_linear_kernel_count(int64_t M, int64_t N, int64_t K, mxfp4_rotation mo
  * in an order the library chooses). Then v = ((x - mu) * rstd) * g[c] + b[c]
  * (fp32, in that order; g / b: DEVICE fp32 [K], 16-byte aligned, NULL for
  * 1 / 0 -- for adaLN modulation pass g = 1 + scale and b = shift) is rotated
- * and quantised. For K <= 6144 one kernel does both from whole rows copied
+ * and quantised. For K <= 51168 one kernel does both from whole rows copied
  * into shared memory (x read once); longer rows take a statistics kernel and
  * then the quantiser. x is bf16; modes NONE / HADAMARD32 / KRON_4x8;
  * otherwise as mxfp4_rotate_quantize.
@@ -276,7 +276,7 @@ mxfp4_status mxfp4_norm_linear(const void* x, int64_t M, int64_t K, mxfp4_norm k
 /*
  * How many kernels mxfp4_norm_linear launches for these sizes: 2 when the
  * norm, rotation and quantisation run as one kernel that copies whole rows
- * into shared memory (K <= 6144), then the GEMM; 3 otherwise (row
+ * into shared memory (K <= 51168), then the GEMM; 3 otherwise (row
  * statistics, quantiser, GEMM); 0 for M == 0; -1 for arguments it rejects.
  * mxfp4_norm_rotate_quantize launches one kernel fewer. Host only.
  */

@@ -396,7 +396,7 @@ def linear_kernel_count(M: int, N: int, K: int, mode: int = ROT_HADAMARD32) -> i
 
 
 def norm_linear_kernel_count(M: int, N: int, K: int, mode: int = ROT_HADAMARD32) -> int:
-    """Kernels that norm_linear() launches: 2 (one-pass norm quantiser + GEMM, K <= 6144),
+    """Kernels that norm_linear() launches: 2 (one-pass norm quantiser + GEMM, K <= 51168),
     3 (row statistics + quantiser + GEMM), 0 (M == 0); -1 for arguments it rejects."""
     return int(lib.mxfp4_norm_linear_kernel_count(M, N, K, mode))
 

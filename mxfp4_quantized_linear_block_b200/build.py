@@ -8,8 +8,8 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libmxfp4.so")
-SOURCES = ["csrc/abi.cu", "csrc/quantize.cu", "csrc/quantize_wide.cu", "csrc/gemm.cu",
-           "csrc/gemm_smallm.cu", "csrc/noalloc.cu"]
+SOURCES = ["csrc/abi.cu", "csrc/quantize.cu", "csrc/quantize_wide.cu", "csrc/quantize_norm.cu",
+           "csrc/gemm.cu", "csrc/gemm_smallm.cu", "csrc/noalloc.cu"]
 DEPS = SOURCES + ["csrc/internal.h", "csrc/sm100.cuh", "csrc/block_quant.cuh",
                   "../include/mxfp4.h"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")

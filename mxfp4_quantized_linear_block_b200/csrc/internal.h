@@ -32,9 +32,14 @@ cudaError_t launch_nvfp4_quantize(const void* x, bool x_is_f32, int64_t rows, in
 // Norm prologue (quantize.cu): per-row statistics of bf16 x into stats [rows][2] (kind 0
 // LayerNorm: mean, 1/sqrt(var + eps); kind 1 RMSNorm: 0, 1/sqrt(mean(x^2) + eps)), then
 // the quantiser applies v = ((x - mu) * rstd) * g + b before rotating (modes 0, 1, 2).
-// One kernel when norm_one_pass(K) (rows copied whole into shared memory: K <= 6144),
-// else a statistics kernel and the quantiser.
+// One kernel when norm_one_pass(K) (quantize_norm.cu: rows copied whole into shared memory,
+// two buffers of at least one row in 200 KB: K <= 51168), else a statistics kernel and
+// the quantiser.
 bool norm_one_pass(int64_t K);
+cudaError_t launch_norm_one_pass(const void* x, int64_t rows, int64_t K, int64_t ldx, int kind,
+                                 float eps, const float* g, const float* b, int mode,
+                                 const KronCoeffs* kc, uint8_t* q, uint8_t* sf, float* stats,
+                                 int* status, cudaStream_t stream);
 cudaError_t launch_norm_rotate_quantize(const void* x, int64_t rows, int64_t K, int64_t ldx,
                                        int kind, float eps, const float* g, const float* b,
                                        int mode, const KronCoeffs* kc, uint8_t* q, uint8_t* sf,

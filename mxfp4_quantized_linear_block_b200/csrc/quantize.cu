@@ -387,163 +387,6 @@ __global__ void __launch_bounds__(256) row_stats_kernel(const uint16_t* __restri
   }
 }
 
-// Norm prologue in one pass over x: a CTA copies R whole bf16 rows into shared memory
-// (one bulk copy per row), a warp per row takes the row's statistics from that copy (sum,
-// then squared deviations; RMSNorm: squares; fp32, each lane's share in order, then a
-// butterfly across the warp; mu = sum / K, rstd = 1 / sqrt(var + eps) correctly rounded),
-// and the 256 threads then normalise, rotate and quantise the R x K/32 blocks from the
-// same copy: v = ((x - mu) * rstd) * g + b, each an fp32 operation in that order, as in the
-// quantiser's norm form. x is read from HBM once, where the statistics kernel + norm
-// quantiser read it twice. R = 16 or 8 rows of 2K bytes (plus a 16-byte pad each) in
-// 96 KB + 256 bytes (two CTAs per SM). Rows sit 2K + 16 bytes apart in shared memory and thread i takes
-// block (row i % R, kb i / R), so the 16-byte reads of a warp spread over all 8 bank
-// groups.
-constexpr uint32_t kRowsSmemBudget = 98304 + 16 * 16;  // 96 KB of rows + their 16-byte pads
-
-template <int KIND, int MODE>
-__global__ void __launch_bounds__(256) norm_rows_kernel(
-    const uint16_t* __restrict__ x, uint64_t ldx, uint32_t rows, uint32_t rows_pad, uint32_t K,
-    uint32_t R, uint32_t n_katoms, float eps, const __grid_constant__ KronCoeffs kc,
-    const float* __restrict__ g, const float* __restrict__ b, uint8_t* __restrict__ q,
-    uint8_t* __restrict__ sf, float* __restrict__ stats, int* status) {
-  using namespace sm100;
-  extern __shared__ uint8_t smem_raw[];
-  const uint32_t sbase = (smem_addr(smem_raw) + 127u) & ~127u;
-  uint8_t* sptr = smem_raw + (sbase - smem_addr(smem_raw));
-  const uint32_t row_bytes = K * 2u;          // a multiple of 64 (K % 32 == 0)
-  const uint32_t row_stride = row_bytes + 16u;  // shared-memory row pitch
-  const uint32_t bar = sbase + R * row_stride;
-  float2* st_s = reinterpret_cast<float2*>(sptr + R * row_stride + 16u);  // R x (mu, rstd)
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(sptr + R * row_stride + 8u);
-  const uint32_t lane = threadIdx.x & 31u, warp = threadIdx.x >> 5;
-  const uint32_t kb_real = K / 32u, kb_pad = n_katoms * 4u;
-  const uint32_t n_groups = rows_pad / R;
-
-  if (threadIdx.x == 0) {
-    mbar_init(bar, 1);
-    *abort_flag = 0;
-    fence_mbar_init();
-  }
-  __syncthreads();
-  // Launched with programmatic dependent launch: the kernel before this one may still be
-  // writing x or reading q / sf / stats. Wait for it before the first access.
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-
-  uint32_t phase = 0;
-  bool aborted = false;
-  for (uint32_t grp = blockIdx.x; grp < n_groups; grp += gridDim.x) {
-    const uint32_t row0 = grp * R;
-    const uint32_t nreal = row0 >= rows ? 0u : (rows - row0 < R ? rows - row0 : R);
-    if (nreal > 0) {
-      if (threadIdx.x == 0) {
-        mbar_arrive_expect_tx(bar, nreal * row_bytes);
-        for (uint32_t r = 0; r < nreal; ++r)
-          bulk_load(sbase + r * row_stride, x + (uint64_t)(row0 + r) * ldx, row_bytes, bar);
-      }
-      const bool ok = mbar_wait_bounded(bar, phase, abort_flag, kWaitLimitNs);
-      if (__syncthreads_or(!ok)) {
-        if (threadIdx.x == 0 && status) atomicExch(status, kTimeoutCode);
-        aborted = true;
-        break;
-      }
-      phase ^= 1u;
-      // Row statistics: warp w takes rows w, w + 8, ...; lane l adds the 8 elements of
-      // each 16-byte chunk l, l + 32, ... of the row in order.
-      for (uint32_t r = warp; r < nreal; r += 8u) {
-        const uint32_t rbase = sbase + r * row_stride;
-        float mu = 0.0f;
-        if constexpr (KIND == 0) {
-          float s = 0.0f;
-          for (uint32_t c = lane; c < row_bytes / 16u; c += 32u) {
-            const uint4 w = ld_shared_v4(rbase + c * 16u);
-            s += bf16_lo(w.x) + bf16_hi(w.x) + bf16_lo(w.y) + bf16_hi(w.y) + bf16_lo(w.z) +
-                 bf16_hi(w.z) + bf16_lo(w.w) + bf16_hi(w.w);
-          }
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-          mu = __fdiv_rn(s, (float)K);
-        }
-        float v = 0.0f;
-        for (uint32_t c = lane; c < row_bytes / 16u; c += 32u) {
-          const uint4 w = ld_shared_v4(rbase + c * 16u);
-          const float e[8] = {bf16_lo(w.x), bf16_hi(w.x), bf16_lo(w.y), bf16_hi(w.y),
-                              bf16_lo(w.z), bf16_hi(w.z), bf16_lo(w.w), bf16_hi(w.w)};
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const float d = e[i] - mu;
-            v = __fmaf_rn(d, d, v);
-          }
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-        if (lane == 0) {
-          const float rstd = __frsqrt_rn(__fadd_rn(__fdiv_rn(v, (float)K), eps));
-          st_s[r] = make_float2(mu, rstd);
-          stats[2u * (row0 + r)] = mu;
-          stats[2u * (row0 + r) + 1u] = rstd;
-        }
-      }
-      __syncthreads();
-      // Blocks: thread i takes blocks i, i + 256, ... of the group, row index fastest.
-      for (uint32_t blk = threadIdx.x; blk < nreal * kb_real; blk += 256u) {
-        const uint32_t kb = blk / nreal, r = blk - kb * nreal;
-        const uint32_t baddr = sbase + r * row_stride + kb * 64u;
-        float2 P[16];
-#pragma unroll
-        for (uint32_t c = 0; c < 4; ++c) {
-          const uint4 w = ld_shared_v4(baddr + c * 16u);
-          P[4 * c + 0] = make_float2(bf16_lo(w.x), bf16_hi(w.x));
-          P[4 * c + 1] = make_float2(bf16_lo(w.y), bf16_hi(w.y));
-          P[4 * c + 2] = make_float2(bf16_lo(w.z), bf16_hi(w.z));
-          P[4 * c + 3] = make_float2(bf16_lo(w.w), bf16_hi(w.w));
-        }
-        const float2 stv = st_s[r];
-        const float2 nmu = make_float2(-stv.x, -stv.x), rs = make_float2(stv.y, stv.y);
-#pragma unroll
-        for (int j = 0; j < 16; ++j) P[j] = __fmul2_rn(__fadd2_rn(P[j], nmu), rs);
-        if (g != nullptr) {
-          const float2* gv = reinterpret_cast<const float2*>(g + kb * 32u);
-#pragma unroll
-          for (int j = 0; j < 16; ++j) P[j] = __fmul2_rn(P[j], __ldg(gv + j));
-        }
-        if (b != nullptr) {
-          const float2* bv = reinterpret_cast<const float2*>(b + kb * 32u);
-#pragma unroll
-          for (int j = 0; j < 16; ++j) P[j] = __fadd2_rn(P[j], __ldg(bv + j));
-        }
-        if constexpr (MODE == 1) hadamard32(P);
-        if constexpr (MODE == 2) kron32(P, kc);
-        uint4 codes;
-        const uint32_t byte = quantize_block(P, codes);
-        st_v4(q + (uint64_t)(row0 + r) * (K / 2u) + (uint64_t)kb * 16u, codes);
-        sf[sf_offset(row0 + r, kb, n_katoms)] = static_cast<uint8_t>(byte);
-      }
-    }
-    // Padding of the scale layout: blocks kb_real..kb_pad of real rows, every block of
-    // the padding rows (>= rows) of this group.
-    const uint32_t pad_real = kb_pad - kb_real;
-    for (uint32_t i = threadIdx.x; i < nreal * pad_real + (R - nreal) * kb_pad; i += 256u) {
-      uint32_t r, kb;
-      if (i < nreal * pad_real) {
-        r = i / pad_real;
-        kb = kb_real + (i - r * pad_real);
-      } else {
-        const uint32_t j = i - nreal * pad_real;
-        r = nreal + j / kb_pad;
-        kb = j - (r - nreal) * kb_pad;
-      }
-      sf[sf_offset(row0 + r, kb, n_katoms)] = 0;
-    }
-    __syncthreads();  // the row copies are read: the buffer may be refilled
-  }
-  // After an early stop the row copies in flight still land in this CTA's shared memory.
-  if (aborted && threadIdx.x == 0) {
-    volatile int never = 0;
-    mbar_wait_bounded(bar, phase, &never, kWaitLimitNs);
-  }
-}
-
 __global__ void nvfp4_scale_finalize_kernel(float* __restrict__ scale2) {
   const float amax = __uint_as_float(reinterpret_cast<unsigned int*>(scale2)[1]);
   scale2[0] = __fdiv_rn(amax, 2688.0f);
@@ -551,87 +394,14 @@ __global__ void nvfp4_scale_finalize_kernel(float* __restrict__ scale2) {
 
 }  // namespace
 
-namespace {
-
-template <int KIND, int MODE>
-cudaError_t launch_norm_rows(const uint16_t* x, int64_t rows, int64_t K, int64_t ldx, float eps,
-                             const KronCoeffs& kc, const float* g, const float* b, uint8_t* q,
-                             uint8_t* sf, float* stats, int* status, uint32_t R,
-                             cudaStream_t stream) {
-  auto kern = norm_rows_kernel<KIND, MODE>;
-  const size_t smem = 128 + (size_t)R * ((size_t)K * 2 + 16) + 16 + 16 * 8;
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  static size_t smem_set[64] = {};
-  if (smem_set[dev] < smem) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
-    if (e != cudaSuccess) return e;
-    smem_set[dev] = smem;
-  }
-  int per_sm = 0, sms = 148;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 256, smem) != cudaSuccess ||
-      per_sm <= 0)
-    per_sm = 1;
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int64_t rows_pad = sf_row_tiles(rows) * 128;
-  const int64_t groups = rows_pad / R;
-  const int64_t cap = (int64_t)sms * per_sm;
-  cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3((unsigned)(groups < cap ? groups : cap));
-  cfg.blockDim = dim3(256);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, x, (uint64_t)ldx, (uint32_t)rows, (uint32_t)rows_pad,
-                            (uint32_t)K, R, (uint32_t)sf_katoms(K), eps, kc, g, b, q, sf, stats,
-                            status);
-}
-
-}  // namespace
-
-// Rows per CTA of the one-pass norm kernel, 0 when it is not used: it needs 8 or more rows
-// in its budget (K <= 6144). With fewer, a CTA holds so few rows that its copy and its
-// arithmetic no longer overlap across the CTAs of an SM; B200, 3584 rows: K = 3072 one
-// pass 18.2 us against 27 us for two kernels, K = 12288 (4 rows per CTA) 85.6 us against
-// 78 us, so long rows keep the statistics kernel + quantiser.
-uint32_t norm_rows_per_cta(int64_t K) {
-  uint32_t R = 16;
-  while (R > 8 && (uint64_t)R * ((uint64_t)K * 2 + 16) > kRowsSmemBudget) R >>= 1;
-  return (uint64_t)R * ((uint64_t)K * 2 + 16) <= kRowsSmemBudget ? R : 0;
-}
-
-bool norm_one_pass(int64_t K) { return norm_rows_per_cta(K) != 0; }
-
 cudaError_t launch_norm_rotate_quantize(const void* x, int64_t rows, int64_t K, int64_t ldx,
                                        int kind, float eps, const float* g, const float* b,
                                        int mode, const KronCoeffs* kc, uint8_t* q, uint8_t* sf,
                                        float* stats, int* status, cudaStream_t stream) {
-  // One pass when 8 rows fit the shared-memory budget (K <= 6144): rows copied whole
-  // into shared memory, statistics and quantisation from that copy.
-  const uint32_t R = norm_rows_per_cta(K);
-  if (R != 0) {
-    KronCoeffs k{};
-    if (kc) k = *kc;
-    const uint16_t* xb = static_cast<const uint16_t*>(x);
-#define MXFP4_NORM_ROWS(KINDV, MODEV)                                                  \
-  return launch_norm_rows<KINDV, MODEV>(xb, rows, K, ldx, eps, k, g, b, q, sf, stats, \
-                                        status, R, stream)
-    if (kind == 1) {
-      if (mode == 1) MXFP4_NORM_ROWS(1, 1);
-      if (mode == 2) MXFP4_NORM_ROWS(1, 2);
-      MXFP4_NORM_ROWS(1, 0);
-    }
-    if (mode == 1) MXFP4_NORM_ROWS(0, 1);
-    if (mode == 2) MXFP4_NORM_ROWS(0, 2);
-    MXFP4_NORM_ROWS(0, 0);
-#undef MXFP4_NORM_ROWS
-  }
+  // One pass (quantize_norm.cu) while two buffers of a row fit one SM's shared memory.
+  if (norm_one_pass(K))
+    return launch_norm_one_pass(x, rows, K, ldx, kind, eps, g, b, mode, kc, q, sf, stats, status,
+                                stream);
   // Longer rows: statistics kernel, then the quantiser in its norm form.
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3((unsigned)((rows + 7) / 8));

@@ -171,12 +171,12 @@ def test_linear_kernel_count():
 
 
 def test_norm_linear_kernel_count():
-    """The norm prologue is one kernel while 8 rows fit the one-pass kernel (K <= 6144)."""
+    """The norm prologue is one kernel while two row buffers fit one SM (K <= 51168)."""
     kc = mx.norm_linear_kernel_count
     assert kc(3584, 9216, 3072, mx.ROT_HADAMARD32) == 2
-    assert kc(3, 256, 6144, mx.ROT_KRON_4x8) == 2
-    assert kc(3, 256, 6176, mx.ROT_HADAMARD32) == 3
-    assert kc(3584, 3072, 12288, mx.ROT_HADAMARD32) == 3
+    assert kc(3584, 3072, 12288, mx.ROT_HADAMARD32) == 2
+    assert kc(3, 256, 51168, mx.ROT_KRON_4x8) == 2
+    assert kc(3, 256, 51200, mx.ROT_HADAMARD32) == 3
     assert kc(0, 256, 1024, mx.ROT_NONE) == 0
     assert kc(4, 256, 1024, mx.ROT_HADAMARD64) == -1
     assert kc(4, 24, 1024, mx.ROT_HADAMARD32) == -1

@@ -16,10 +16,11 @@ def _vec(seed, K, mean, std):
 
 
 @pytest.mark.parametrize("kind", [oracle.NORM_LAYER, oracle.NORM_RMS])
-# K <= 6144 (8 or 16 rows per CTA) takes the one-pass kernel; K = 6176 and 12288 the
+# K <= 51168 takes the one-pass kernel (groups of 16 / 8 / 4 / 2 / 1 rows per CTA for
+# K = 3072 / 6144 / 12288 / 24576 / 51168, with a partial last group); K = 51200 the
 # statistics kernel + norm quantiser.
-@pytest.mark.parametrize("rows,K", [(1, 64), (5, 3072), (129, 1024), (17, 6144), (9, 6176),
-                                    (300, 12288)])
+@pytest.mark.parametrize("rows,K", [(1, 64), (5, 3072), (129, 1024), (17, 6144),
+                                    (300, 12288), (7, 24576), (3, 51168), (3, 51200)])
 @pytest.mark.parametrize("affine", [False, True])
 def test_norm_rotate_quantize(kind, rows, K, affine):
     import torch
