@@ -136,20 +136,29 @@ __global__ void __launch_bounds__(kNormThreads, 1) norm_rows_kernel(
       phase ^= 1u << bi;
       if (tid == 0) pending &= ~(1u << bi);
 
-      // Statistics: warp w takes slice w % W of row w / W; lane l adds the 8 elements of
-      // each 16-byte chunk (w % W) 32 + l + 32 W i in order; the W slices of a row are
-      // then added in slice order.
+      // Statistics: warp w takes slice w % W of row w / W; lane l takes the 16-byte chunks
+      // (w % W) 32 + l + 32 W i, i = 0, 1, ..., into four partial sums by i mod 4 (each
+      // adds a chunk's 8 elements in order), added as (p0 + p1) + (p2 + p3); the warp's
+      // lanes are then added by a butterfly and the W slices of a row in slice order.
       const uint32_t r = warp / W, sl = warp - r * W;
       const uint32_t rbase = buf + r * L.pitch;
+      const uint32_t cstep = 32u * W;
       float mu = 0.0f;
       if constexpr (KIND == 0) {
-        float s = 0.0f;
+        float p4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
         if (r < nreal)
-          for (uint32_t c = sl * 32u + lane; c < chunks; c += 32u * W) {
-            const uint4 w = ld_shared_v4(rbase + c * 16u);
-            s += bf16_lo(w.x) + bf16_hi(w.x) + bf16_lo(w.y) + bf16_hi(w.y) + bf16_lo(w.z) +
-                 bf16_hi(w.z) + bf16_lo(w.w) + bf16_hi(w.w);
+          for (uint32_t c0 = sl * 32u + lane; c0 < chunks; c0 += 4u * cstep) {
+#pragma unroll
+            for (uint32_t j = 0; j < 4; ++j) {
+              const uint32_t c = c0 + j * cstep;
+              if (c < chunks) {
+                const uint4 w = ld_shared_v4(rbase + c * 16u);
+                p4[j] += bf16_lo(w.x) + bf16_hi(w.x) + bf16_lo(w.y) + bf16_hi(w.y) +
+                         bf16_lo(w.z) + bf16_hi(w.z) + bf16_lo(w.w) + bf16_hi(w.w);
+              }
+            }
           }
+        float s = (p4[0] + p4[1]) + (p4[2] + p4[3]);
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
         if (lane == 0) part[warp] = s;
@@ -162,18 +171,25 @@ __global__ void __launch_bounds__(kNormThreads, 1) norm_rows_kernel(
         __syncthreads();
         if (r < nreal) mu = st_s[r].x;
       }
-      float v = 0.0f;
+      float q4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
       if (r < nreal)
-        for (uint32_t c = sl * 32u + lane; c < chunks; c += 32u * W) {
-          const uint4 w = ld_shared_v4(rbase + c * 16u);
-          const float e[8] = {bf16_lo(w.x), bf16_hi(w.x), bf16_lo(w.y), bf16_hi(w.y),
-                              bf16_lo(w.z), bf16_hi(w.z), bf16_lo(w.w), bf16_hi(w.w)};
+        for (uint32_t c0 = sl * 32u + lane; c0 < chunks; c0 += 4u * cstep) {
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const float d = e[i] - mu;
-            v = __fmaf_rn(d, d, v);
+          for (uint32_t j = 0; j < 4; ++j) {
+            const uint32_t c = c0 + j * cstep;
+            if (c < chunks) {
+              const uint4 w = ld_shared_v4(rbase + c * 16u);
+              const float e[8] = {bf16_lo(w.x), bf16_hi(w.x), bf16_lo(w.y), bf16_hi(w.y),
+                                  bf16_lo(w.z), bf16_hi(w.z), bf16_lo(w.w), bf16_hi(w.w)};
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                const float d = e[i] - mu;
+                q4[j] = __fmaf_rn(d, d, q4[j]);
+              }
+            }
           }
         }
+      float v = (q4[0] + q4[1]) + (q4[2] + q4[3]);
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
       if (lane == 0) part[warp] = v;
@@ -207,15 +223,23 @@ __global__ void __launch_bounds__(kNormThreads, 1) norm_rows_kernel(
         const float2 nmu = make_float2(-stv.x, -stv.x), rs = make_float2(stv.y, stv.y);
 #pragma unroll
         for (int j = 0; j < 16; ++j) P[j] = __fmul2_rn(__fadd2_rn(P[j], nmu), rs);
-        if (g != nullptr) {
-          const float2* gv = reinterpret_cast<const float2*>(g + kb * 32u);
+        if (g != nullptr) {  // 16-byte loads: g and b are 16-byte aligned, kb 32 floats apart
+          const float4* gv = reinterpret_cast<const float4*>(g + kb * 32u);
 #pragma unroll
-          for (int j = 0; j < 16; ++j) P[j] = __fmul2_rn(P[j], __ldg(gv + j));
+          for (int j = 0; j < 8; ++j) {
+            const float4 t = __ldg(gv + j);
+            P[2 * j] = __fmul2_rn(P[2 * j], make_float2(t.x, t.y));
+            P[2 * j + 1] = __fmul2_rn(P[2 * j + 1], make_float2(t.z, t.w));
+          }
         }
         if (b != nullptr) {
-          const float2* bv = reinterpret_cast<const float2*>(b + kb * 32u);
+          const float4* bv = reinterpret_cast<const float4*>(b + kb * 32u);
 #pragma unroll
-          for (int j = 0; j < 16; ++j) P[j] = __fadd2_rn(P[j], __ldg(bv + j));
+          for (int j = 0; j < 8; ++j) {
+            const float4 t = __ldg(bv + j);
+            P[2 * j] = __fadd2_rn(P[2 * j], make_float2(t.x, t.y));
+            P[2 * j + 1] = __fadd2_rn(P[2 * j + 1], make_float2(t.z, t.w));
+          }
         }
         if constexpr (MODE == 1) hadamard32(P);
         if constexpr (MODE == 2) kron32(P, kc);
