@@ -300,8 +300,9 @@ int mxfp4_norm_linear_kernel_count(int64_t M, int64_t N, int64_t K, mxfp4_rotati
 size_t mxfp4_nvfp4_sf_bytes(int64_t rows, int64_t K);
 
 /* Tensor scale st = amax(rotated x) / (6 * 448) (fp32, one rounding) into
- * scale2[0]; scale2: DEVICE pointer to 2 floats, 8-byte aligned, [1] is scratch.
- * Stream-ordered (a memset and two small kernels). */
+ * scale2[0]; scale2: DEVICE pointer to 2 floats, 8-byte aligned, both
+ * overwritten ([1] is scratch). Stream-ordered (a memset and one kernel, whose
+ * last block to finish writes the scale). */
 mxfp4_status mxfp4_nvfp4_tensor_scale(const void* x, mxfp4_dtype xdt, int64_t rows, int64_t K,
                                       int64_t ldx, mxfp4_rotation mode, float* scale2,
                                       mxfp4_stream_t stream);

@@ -77,8 +77,8 @@ struct LinearWorkspace {
   size_t q_off, sf_off, g_off, total;
 };
 
-// Workspace of mxfp4_nvfp4_linear: [status | X tensor scale (2 floats at 64) | Xq | Xsf |
-// GEMM scratch].
+// Workspace of mxfp4_nvfp4_linear: [status (X tensor scale at 64, the scale pass's
+// running maximum and block counter at 72 and 76) | Xq | Xsf | GEMM scratch].
 constexpr size_t kScaleOff = 64;
 
 LinearWorkspace nvfp4_linear_workspace(int64_t M, int64_t N, int64_t K) {
@@ -439,7 +439,10 @@ mxfp4_status mxfp4_nvfp4_linear(const void* x, int64_t M, int64_t K, mxfp4_rotat
   uint8_t* base = static_cast<uint8_t*>(ws);
   float* xs = reinterpret_cast<float*>(base + kScaleOff);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  cudaError_t e = launch_nvfp4_tensor_scale(x, false, M, K, K, (int)mode, xs, s);
+  // the pass's running maximum and block counter: two words after the scale, zero at
+  // allocation and left zero by every pass that completes
+  cudaError_t e = launch_nvfp4_tensor_scale(x, false, M, K, K, (int)mode, xs, s,
+                                            reinterpret_cast<unsigned int*>(xs + 2));
   if (e != cudaSuccess) return MXFP4_ERR_CUDA;
   e = launch_nvfp4_quantize(x, false, M, K, K, (int)mode, xs, base + w.q_off, base + w.sf_off,
                             static_cast<int*>(ws), s);

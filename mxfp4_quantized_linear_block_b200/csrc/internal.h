@@ -20,11 +20,14 @@ cudaError_t launch_rotate_quantize(const void* x, bool x_is_f32, int64_t rows, i
                                    int64_t ldx, int mode, const KronCoeffs* kc, uint8_t* q,
                                    uint8_t* sf, int* status, cudaStream_t stream);
 
-// NVFP4 (quantize.cu): tensor scale of x rotated by mode (0 / 1) into scale2[0] (scale2[1]
-// is scratch; a memset and two small kernels), and the quantiser with that scale: codes
-// as for MXFP4, E4M3 group bytes in atoms of 4 groups of 16 (sf_katoms(2K) per row tile).
+// NVFP4 (quantize.cu): tensor scale of x rotated by mode (0 / 1) into scale2[0], and the
+// quantiser with that scale: codes as for MXFP4, E4M3 group bytes in atoms of 4 groups of
+// 16 (sf_katoms(2K) per row tile). The scale pass is one kernel whose last block writes
+// the scale; state: two device words that are zero and that it leaves zero (running
+// maximum, block counter), or null: scale2[0..1] are zeroed by a memset and used instead.
 cudaError_t launch_nvfp4_tensor_scale(const void* x, bool x_is_f32, int64_t rows, int64_t K,
-                                     int64_t ldx, int mode, float* scale2, cudaStream_t stream);
+                                     int64_t ldx, int mode, float* scale2, cudaStream_t stream,
+                                     unsigned int* state = nullptr);
 cudaError_t launch_nvfp4_quantize(const void* x, bool x_is_f32, int64_t rows, int64_t K,
                                   int64_t ldx, int mode, const float* tensor_scale, uint8_t* q,
                                   uint8_t* sf, int* status, cudaStream_t stream);

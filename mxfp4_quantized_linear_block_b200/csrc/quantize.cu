@@ -288,7 +288,8 @@ cudaError_t launch_mode(const void* x, int64_t rows, int64_t K, int64_t ldx, con
 template <int MODE, bool F32_IN>
 __global__ void __launch_bounds__(256) nvfp4_amax_kernel(const void* __restrict__ x, uint64_t ldx,
                                                          uint32_t rows, uint32_t kb_real,
-                                                         unsigned int* __restrict__ amax_bits) {
+                                                         unsigned int* __restrict__ amax_bits,
+                                                         unsigned int* done, float* scale_out) {
   const uint64_t n = (uint64_t)rows * kb_real;
   float m = 0.0f;
   for (uint64_t b = blockIdx.x * (uint64_t)blockDim.x + threadIdx.x; b < n;
@@ -323,6 +324,19 @@ __global__ void __launch_bounds__(256) nvfp4_amax_kernel(const void* __restrict_
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
   if ((threadIdx.x & 31u) == 0) atomicMax(amax_bits, __float_as_uint(m));
+  // The last block to finish turns the maximum into the scale and leaves the maximum (and
+  // a separate counter) zero for the next pass. `done` may be scale_out itself, which
+  // the caller zeroed; the scale then simply replaces it.
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    if (atomicAdd(done, 1u) == gridDim.x - 1u) {
+      __threadfence();
+      const unsigned int bits = atomicExch(amax_bits, 0u);
+      if (done != reinterpret_cast<unsigned int*>(scale_out)) atomicExch(done, 0u);
+      scale_out[0] = __fdiv_rn(__uint_as_float(bits), 2688.0f);
+    }
+  }
 }
 
 // Norm prologue statistics: one warp per bf16 row, two passes (sum, then squared
@@ -387,11 +401,6 @@ __global__ void __launch_bounds__(256) row_stats_kernel(const uint16_t* __restri
   }
 }
 
-__global__ void nvfp4_scale_finalize_kernel(float* __restrict__ scale2) {
-  const float amax = __uint_as_float(reinterpret_cast<unsigned int*>(scale2)[1]);
-  scale2[0] = __fdiv_rn(amax, 2688.0f);
-}
-
 }  // namespace
 
 cudaError_t launch_norm_rotate_quantize(const void* x, int64_t rows, int64_t K, int64_t ldx,
@@ -433,10 +442,21 @@ cudaError_t launch_norm_rotate_quantize(const void* x, int64_t rows, int64_t K, 
 }
 
 cudaError_t launch_nvfp4_tensor_scale(const void* x, bool x_is_f32, int64_t rows, int64_t K,
-                                     int64_t ldx, int mode, float* scale2, cudaStream_t stream) {
-  // scale2[1] holds the amax bits during the pass, scale2[0] receives the scale
-  cudaError_t e = cudaMemsetAsync(scale2 + 1, 0, sizeof(float), stream);
-  if (e != cudaSuccess) return e;
+                                     int64_t ldx, int mode, float* scale2, cudaStream_t stream,
+                                     unsigned int* state) {
+  // With `state` (two words, zero, left zero): one kernel. Without: scale2[0] serves as
+  // the block counter and scale2[1] as the running maximum, zeroed first.
+  unsigned int* bits;
+  unsigned int* done;
+  if (state != nullptr) {
+    bits = state;
+    done = state + 1;
+  } else {
+    cudaError_t e = cudaMemsetAsync(scale2, 0, 2 * sizeof(float), stream);
+    if (e != cudaSuccess) return e;
+    done = reinterpret_cast<unsigned int*>(scale2);
+    bits = reinterpret_cast<unsigned int*>(scale2 + 1);
+  }
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -444,19 +464,18 @@ cudaError_t launch_nvfp4_tensor_scale(const void* x, bool x_is_f32, int64_t rows
   uint64_t grid = (blocks + 255) / 256;
   if (grid > (uint64_t)sms * 8) grid = (uint64_t)sms * 8;
   if (grid == 0) grid = 1;
-  unsigned int* bits = reinterpret_cast<unsigned int*>(scale2 + 1);
+  const unsigned g = (unsigned)grid;
   if (x_is_f32) {
     if (mode == 1)
-      nvfp4_amax_kernel<1, true><<<(unsigned)grid, 256, 0, stream>>>(x, ldx, rows, K / 32, bits);
+      nvfp4_amax_kernel<1, true><<<g, 256, 0, stream>>>(x, ldx, rows, K / 32, bits, done, scale2);
     else
-      nvfp4_amax_kernel<0, true><<<(unsigned)grid, 256, 0, stream>>>(x, ldx, rows, K / 32, bits);
+      nvfp4_amax_kernel<0, true><<<g, 256, 0, stream>>>(x, ldx, rows, K / 32, bits, done, scale2);
   } else {
     if (mode == 1)
-      nvfp4_amax_kernel<1, false><<<(unsigned)grid, 256, 0, stream>>>(x, ldx, rows, K / 32, bits);
+      nvfp4_amax_kernel<1, false><<<g, 256, 0, stream>>>(x, ldx, rows, K / 32, bits, done, scale2);
     else
-      nvfp4_amax_kernel<0, false><<<(unsigned)grid, 256, 0, stream>>>(x, ldx, rows, K / 32, bits);
+      nvfp4_amax_kernel<0, false><<<g, 256, 0, stream>>>(x, ldx, rows, K / 32, bits, done, scale2);
   }
-  nvfp4_scale_finalize_kernel<<<1, 1, 0, stream>>>(scale2);
   return cudaGetLastError();
 }
 

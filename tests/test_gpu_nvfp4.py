@@ -123,3 +123,30 @@ def test_nvfp4_linear(mode, M):
     alpha = float(np.float32(st_x) * np.float32(st_w))
     ref, S = oracle.nvfp4_gemm(xq_r, xs_r, wq_r, ws_r, alpha)
     check_gemm_values(bf16_dev_to_f64(y), ref, S, "bf16", f"nvfp4 linear M{M} mode {mode}")
+
+
+def test_nvfp4_linear_repeated_on_one_workspace():
+    """The layer's tensor-scale pass keeps its running maximum and block counter in the
+    workspace and leaves them zero: a call whose x has a smaller amax than the one before
+    on the same workspace gets its own scale (a leftover maximum would inflate it)."""
+    import torch
+    import mxfp4_quantized_linear_block_b200 as mx
+    M, K, N, mode = 300, 1024, 512, oracle.ROT_HADAMARD32
+    w = synth.weight_f32(4, N, K, 6)
+    w_d = torch.from_numpy(w).cuda()
+    w_sc = mx.nvfp4_tensor_scale(w_d, mode)
+    wq, wsf = mx.nvfp4_quantize(w_d, w_sc, mode)
+    st_w = oracle.nvfp4_tensor_scale(w, mode)
+    wq_r, ws_r = oracle.nvfp4_rotate_quantize(w, mode, st_w)
+    ws = mx.new_workspace(mx.workspace_bytes(mx.OP_NVFP4_LINEAR, M, N, K))
+    big, _ = synth.activation_bf16(7, M, K, 0.01, 30.0)
+    small = synth.f32_to_bf16_bits(synth.bf16_bits_to_f32(big) * np.float32(0.125))
+    for x in (big, small, big):
+        y = mx.nvfp4_linear(to_dev_bf16(x), wq, wsf, w_sc, N, mode, ws=ws)
+        torch.cuda.synchronize()
+        st_x = oracle.nvfp4_tensor_scale(x, mode)
+        xq_r, xs_r = oracle.nvfp4_rotate_quantize(x, mode, st_x)
+        alpha = float(np.float32(st_x) * np.float32(st_w))
+        ref, S = oracle.nvfp4_gemm(xq_r, xs_r, wq_r, ws_r, alpha)
+        check_gemm_values(bf16_dev_to_f64(y), ref, S, "bf16", "nvfp4 linear, shared workspace")
+    assert mx.poll_status(ws) == mx.OK
