@@ -64,8 +64,8 @@ NCU_TRAFFIC = {
 }
 NCU_TRAFFIC_QUANTIZE = {
     "dit_b1": {"source": f"{PKG}/csrc/quantize.cu",
-               "sha256": "62bd6238066e555dfaf650df4336b627c46bf3e229c004ad212f185f0b332193",
-               "bytes_per_launch": [22033408 + 0, 22033664 + 0, 88095488 + 4247040]},
+               "sha256": "b82e8111e1747408436756885476a13ce6d552bb7750be06d1f89bda66f8e4b5",
+               "bytes_per_launch": [22033920 + 0, 22033664 + 0, 88094976 + 4763904]},
 }
 
 

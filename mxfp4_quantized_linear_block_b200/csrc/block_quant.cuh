@@ -96,11 +96,11 @@ __device__ __forceinline__ uint64_t sf_offset(uint32_t row, uint32_t kb, uint32_
 
 #define BLK(P, i) (((i) & 1) ? (P)[(i) >> 1].y : (P)[(i) >> 1].x)
 
-// Normalised Sylvester Hadamard of one block: butterfly stages with strides
-// 1, 2, 4, 8, 16 ((a, b) -> (a + b, a - b)), then one multiply by kInvSqrt32.
-// Stride 1 pairs the two halves of each packed value; strides 2..16 pair whole
-// packed values lane by lane (a - b as the exact fma b * -1 + a).
-__device__ __forceinline__ void hadamard32(float2 (&P)[16]) {
+// Unnormalised Sylvester butterfly of one block: stages with strides 1, 2, 4, 8, 16
+// ((a, b) -> (a + b, a - b)). Stride 1 pairs the two halves of each packed value;
+// strides 2..16 pair whole packed values lane by lane (a - b as the exact fma
+// b * -1 + a).
+__device__ __forceinline__ void fwht32(float2 (&P)[16]) {
 #pragma unroll
   for (int j = 0; j < 16; ++j) {
     const float a = P[j].x, b = P[j].y;
@@ -117,6 +117,12 @@ __device__ __forceinline__ void hadamard32(float2 (&P)[16]) {
       P[j + h] = __ffma2_rn(b, m1, a);
     }
   }
+}
+
+// Normalised Sylvester Hadamard of one block: the butterfly, then one multiply by
+// kInvSqrt32.
+__device__ __forceinline__ void hadamard32(float2 (&P)[16]) {
+  fwht32(P);
   const float2 c = make_float2(kInvSqrt32, kInvSqrt32);
 #pragma unroll
   for (int j = 0; j < 16; ++j) P[j] = __fmul2_rn(P[j], c);

@@ -59,6 +59,8 @@ struct NormArgs {
   const float* b;      // or null (0)
 };
 
+// MODE 3 (64-element Hadamard groups) takes bf16 input without norm or NVFP4: a group is
+// one 128-byte row chunk of a tile, held by a lane pair.
 template <int MODE, bool F32_IN, bool NV, bool NORM = false>
 __global__ void __launch_bounds__(kThreads) rotate_quantize_kernel(
     const __grid_constant__ CUtensorMap tmap_x, uint32_t rows, uint32_t rows_pad, uint32_t kb_real,
@@ -67,6 +69,7 @@ __global__ void __launch_bounds__(kThreads) rotate_quantize_kernel(
     int* status, const float* __restrict__ tensor_scale, const NormArgs norm) {
   using namespace sm100;
   using T = TileShape<F32_IN>;
+  static_assert(MODE != 3 || (!F32_IN && !NV && !NORM), "64-element groups: bf16, MXFP4");
   constexpr int CH = F32_IN ? 8 : 4;  // 16-byte chunks per 32-element block
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_addr(smem_raw);
@@ -148,6 +151,22 @@ __global__ void __launch_bounds__(kThreads) rotate_quantize_kernel(
       if (next < tiles) {
         issue(next, s);
         ++issued;
+      }
+    }
+    if constexpr (MODE == 3) {
+      // 64-element Hadamard: the two blocks of a row chunk sit in lanes 2i and 2i + 1.
+      // Butterfly strides 1..16 inside each block, stride 32 across the lane pair (lower
+      // lane a + b, upper lane a - b, each as one fma with +-1), then the multiply by
+      // 1/8. Every lane takes part (the shuffles need the whole warp); rows and blocks
+      // past the input only carry zeros and are not stored.
+      fwht32(P);
+      const float2 sg = b_loc ? make_float2(-1.0f, -1.0f) : make_float2(1.0f, 1.0f);
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        float2 o;
+        o.x = __shfl_xor_sync(0xffffffffu, P[j].x, 1);
+        o.y = __shfl_xor_sync(0xffffffffu, P[j].y, 1);
+        P[j] = __fmul2_rn(__ffma2_rn(P[j], sg, o), make_float2(0.125f, 0.125f));
       }
     }
 
@@ -497,11 +516,15 @@ cudaError_t launch_nvfp4_quantize(const void* x, bool x_is_f32, int64_t rows, in
 cudaError_t launch_rotate_quantize(const void* x, bool x_is_f32, int64_t rows, int64_t K,
                                    int64_t ldx, int mode, const KronCoeffs* kc, uint8_t* q,
                                    uint8_t* sf, int* status, cudaStream_t stream) {
+  KronCoeffs k{};
+  if (kc) k = *kc;
+  // 64-element groups of bf16 rows: the tile kernel (a group is one row chunk of a tile);
+  // fp32 input (weight preparation) and 128-element groups: the warp-shuffle kernel.
+  if (mode == 3 && !x_is_f32)
+    return launch_mode<3, false>(x, rows, K, ldx, k, q, sf, status, stream);
   if (mode == 3 || mode == 4)
     return launch_rotate_quantize_wide(x, x_is_f32, rows, K, ldx, (int)rotation_span(mode), q, sf,
                                        stream);
-  KronCoeffs k{};
-  if (kc) k = *kc;
   if (x_is_f32) {
     if (mode == 1) return launch_mode<1, true>(x, rows, K, ldx, k, q, sf, status, stream);
     if (mode == 2) return launch_mode<2, true>(x, rows, K, ldx, k, q, sf, status, stream);
