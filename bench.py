@@ -64,8 +64,8 @@ NCU_TRAFFIC = {
 }
 NCU_TRAFFIC_QUANTIZE = {
     "dit_b1": {"source": f"{PKG}/csrc/quantize.cu",
-               "sha256": "b82e8111e1747408436756885476a13ce6d552bb7750be06d1f89bda66f8e4b5",
-               "bytes_per_launch": [22033920 + 0, 22033664 + 0, 88094976 + 4763904]},
+               "sha256": "46f5986c60972c28299ff9b4b5c39c6e71e8f5a6ef8b8ca9680a20c9eccb0215",
+               "bytes_per_launch": [22033664 + 0, 22033408 + 0, 88095488 + 4093952]},
 }
 
 

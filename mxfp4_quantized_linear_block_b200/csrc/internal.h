@@ -48,7 +48,8 @@ cudaError_t launch_norm_rotate_quantize(const void* x, int64_t rows, int64_t K, 
                                        int mode, const KronCoeffs* kc, uint8_t* q, uint8_t* sf,
                                        float* stats, int* status, cudaStream_t stream);
 
-// Rotation over 64- or 128-element groups (span) + quantisation (quantize_wide.cu).
+// Rotation over 64- or 128-element groups (span) + quantisation of fp32 rows
+// (quantize_wide.cu); cudaErrorNotSupported for bf16, which the tile quantiser handles.
 cudaError_t launch_rotate_quantize_wide(const void* x, bool x_is_f32, int64_t rows, int64_t K,
                                         int64_t ldx, int span, uint8_t* q, uint8_t* sf,
                                         cudaStream_t stream);

@@ -44,12 +44,18 @@ constexpr uint32_t kStages = 4;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 constexpr int kTimeoutCode = 7;                  // MXFP4_ERR_TIMEOUT
 
-template <bool F32_IN>
+// A stage is BOXES TMA boxes of ROWS rows x 128 bytes, side by side along K (two for
+// 128-element Hadamard groups, so that a group is in one stage).
+template <bool F32_IN, int MODE = 0>
 struct TileShape {
-  static constexpr uint32_t ROWS = F32_IN ? 256 : 128;  // rows per TMA box
-  static constexpr uint32_t BPR = F32_IN ? 1 : 2;       // 32-element blocks per row per box
-  static constexpr uint32_t STAGE = ROWS * 128;         // bytes per stage (128 bytes per row)
-  static constexpr uint32_t SMEM = kStages * STAGE + 64 + 1024;
+  static constexpr uint32_t BOXES = MODE == 4 ? 2 : 1;
+  static constexpr uint32_t ROWS = F32_IN ? 256 : 128;       // rows per TMA box
+  static constexpr uint32_t BPR = F32_IN ? 1 : 2 * BOXES;    // 32-element blocks per row per stage
+  static constexpr uint32_t BOX_BYTES = ROWS * 128;          // 128 bytes per row
+  static constexpr uint32_t STAGE = BOXES * BOX_BYTES;       // bytes per stage
+  static constexpr uint32_t STAGES = MODE == 4 ? 3 : kStages;
+  static constexpr uint32_t THREADS = MODE == 4 ? 512 : kThreads;  // one per block of a stage
+  static constexpr uint32_t SMEM = STAGES * STAGE + 64 + 1024;
 };
 
 // Norm prologue (per-row statistics from row_stats_kernel, optional g / b of length K).
@@ -59,17 +65,18 @@ struct NormArgs {
   const float* b;      // or null (0)
 };
 
-// MODE 3 (64-element Hadamard groups) takes bf16 input without norm or NVFP4: a group is
-// one 128-byte row chunk of a tile, held by a lane pair.
+// MODE 3 / 4 (64- / 128-element Hadamard groups) take bf16 input without norm or NVFP4: a
+// group is one (two) 128-byte row chunks of a stage, held by 2 (4) consecutive lanes.
 template <int MODE, bool F32_IN, bool NV, bool NORM = false>
-__global__ void __launch_bounds__(kThreads) rotate_quantize_kernel(
+__global__ void __launch_bounds__(TileShape<F32_IN, MODE>::THREADS) rotate_quantize_kernel(
     const __grid_constant__ CUtensorMap tmap_x, uint32_t rows, uint32_t rows_pad, uint32_t kb_real,
     uint32_t k_boxes, uint32_t tiles, uint32_t n_katoms, uint64_t q_row_bytes,
     const __grid_constant__ KronCoeffs kc, uint8_t* __restrict__ q, uint8_t* __restrict__ sf,
     int* status, const float* __restrict__ tensor_scale, const NormArgs norm) {
   using namespace sm100;
-  using T = TileShape<F32_IN>;
-  static_assert(MODE != 3 || (!F32_IN && !NV && !NORM), "64-element groups: bf16, MXFP4");
+  using T = TileShape<F32_IN, MODE>;
+  constexpr uint32_t kStages = T::STAGES;
+  static_assert(MODE < 3 || (!F32_IN && !NV && !NORM), "wide groups: bf16, MXFP4");
   constexpr int CH = F32_IN ? 8 : 4;  // 16-byte chunks per 32-element block
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_addr(smem_raw);
@@ -79,9 +86,12 @@ __global__ void __launch_bounds__(kThreads) rotate_quantize_kernel(
       reinterpret_cast<volatile int*>(smem_raw + (bar_full - raw_addr) + 8 * kStages);
 
   const uint32_t lane = threadIdx.x & 31u, warp = threadIdx.x >> 5;
-  // thread -> (row inside the tile, block inside the row)
-  const uint32_t r_loc = F32_IN ? warp * 32u + lane : warp * 16u + (lane >> 1);
-  const uint32_t b_loc = F32_IN ? 0u : (lane & 1u);
+  // thread -> (row inside the tile, block inside the row's part of the stage)
+  const uint32_t r_loc = F32_IN ? warp * 32u + lane
+                                : (MODE == 4 ? warp * 8u + (lane >> 2) : warp * 16u + (lane >> 1));
+  const uint32_t b_loc = F32_IN ? 0u : (MODE == 4 ? (lane & 3u) : (lane & 1u));
+  const uint32_t box = MODE == 4 ? b_loc >> 1 : 0u;     // TMA box of the block
+  const uint32_t b_box = MODE == 4 ? b_loc & 1u : b_loc;  // block inside the box row
 
   if (threadIdx.x == 0) {
     for (uint32_t s = 0; s < kStages; ++s) mbar_init(bar_full + 8 * s, 1);
@@ -102,8 +112,10 @@ __global__ void __launch_bounds__(kThreads) rotate_quantize_kernel(
   auto issue = [&](uint32_t tile, uint32_t s) {
     const uint32_t rt = tile / k_boxes, kx = tile - rt * k_boxes;
     mbar_arrive_expect_tx(bar_full + 8 * s, T::STAGE);
-    tma_load_2d(sbase + s * T::STAGE, &tmap_x, bar_full + 8 * s, (int32_t)(kx * (F32_IN ? 32 : 64)),
-                (int32_t)(rt * T::ROWS));
+#pragma unroll
+    for (uint32_t bx = 0; bx < T::BOXES; ++bx)
+      tma_load_2d(sbase + s * T::STAGE + bx * T::BOX_BYTES, &tmap_x, bar_full + 8 * s,
+                  (int32_t)((kx * T::BOXES + bx) * (F32_IN ? 32 : 64)), (int32_t)(rt * T::ROWS));
   };
   uint32_t issued = 0;
   if (threadIdx.x == 0)
@@ -130,10 +142,10 @@ __global__ void __launch_bounds__(kThreads) rotate_quantize_kernel(
     const uint32_t kb = kx * T::BPR + b_loc;
 
     float2 P[16];
-    const uint32_t rbase = sbase + s * T::STAGE + r_loc * 128u;
+    const uint32_t rbase = sbase + s * T::STAGE + box * T::BOX_BYTES + r_loc * 128u;
 #pragma unroll
     for (int c = 0; c < CH; ++c) {
-      const uint32_t chunk = ((b_loc * CH + (uint32_t)c) ^ (r_loc & 7u)) << 4;
+      const uint32_t chunk = ((b_box * CH + (uint32_t)c) ^ (r_loc & 7u)) << 4;
       const uint4 w = ld_shared_v4(rbase + chunk);
       if constexpr (F32_IN) {
         P[2 * c + 0] = make_float2(__uint_as_float(w.x), __uint_as_float(w.y));
@@ -168,6 +180,27 @@ __global__ void __launch_bounds__(kThreads) rotate_quantize_kernel(
         o.y = __shfl_xor_sync(0xffffffffu, P[j].y, 1);
         P[j] = __fmul2_rn(__ffma2_rn(P[j], sg, o), make_float2(0.125f, 0.125f));
       }
+    }
+    if constexpr (MODE == 4) {
+      // 128-element Hadamard: the four blocks of a group sit in lanes 4i .. 4i + 3.
+      // Strides 1..16 inside each block, then stride 32 (lanes l, l ^ 1) and stride 64
+      // (lanes l, l ^ 2) across lanes as for 64-element groups, then the multiply by the
+      // fp32 nearest 1/sqrt(128) (half the fp32 nearest 1/sqrt(32), exactly).
+      fwht32(P);
+#pragma unroll
+      for (uint32_t m = 1; m <= 2; m <<= 1) {
+        const float2 sg = (b_loc & m) ? make_float2(-1.0f, -1.0f) : make_float2(1.0f, 1.0f);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          float2 o;
+          o.x = __shfl_xor_sync(0xffffffffu, P[j].x, m);
+          o.y = __shfl_xor_sync(0xffffffffu, P[j].y, m);
+          P[j] = __ffma2_rn(P[j], sg, o);
+        }
+      }
+      const float2 c128 = make_float2(0x1.6a09e6p-4f, 0x1.6a09e6p-4f);
+#pragma unroll
+      for (int j = 0; j < 16; ++j) P[j] = __fmul2_rn(P[j], c128);
     }
 
     if (row < rows_pad) {
@@ -246,7 +279,7 @@ template <int MODE, bool F32_IN, bool NV = false, bool NORM = false>
 cudaError_t launch_mode(const void* x, int64_t rows, int64_t K, int64_t ldx, const KronCoeffs& kc,
                         uint8_t* q, uint8_t* sf, int* status, cudaStream_t stream,
                         const float* tensor_scale = nullptr, NormArgs norm = NormArgs{}) {
-  using T = TileShape<F32_IN>;
+  using T = TileShape<F32_IN, MODE>;
   auto fn = encode_fn();
   if (!fn) return cudaErrorNotSupported;
   CUtensorMap map;
@@ -270,7 +303,8 @@ cudaError_t launch_mode(const void* x, int64_t rows, int64_t K, int64_t ldx, con
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, T::SMEM);
     if (e != cudaSuccess) return e;
     int n = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kThreads, T::SMEM) != cudaSuccess ||
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, T::THREADS, T::SMEM) !=
+            cudaSuccess ||
         n <= 0)
       n = 1;
     cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev);
@@ -286,7 +320,7 @@ cudaError_t launch_mode(const void* x, int64_t rows, int64_t K, int64_t ldx, con
   const int grid = (int)(tiles < cap ? tiles : cap);
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(kThreads);
+  cfg.blockDim = dim3(T::THREADS);
   cfg.dynamicSmemBytes = T::SMEM;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
@@ -518,10 +552,12 @@ cudaError_t launch_rotate_quantize(const void* x, bool x_is_f32, int64_t rows, i
                                    uint8_t* sf, int* status, cudaStream_t stream) {
   KronCoeffs k{};
   if (kc) k = *kc;
-  // 64-element groups of bf16 rows: the tile kernel (a group is one row chunk of a tile);
-  // fp32 input (weight preparation) and 128-element groups: the warp-shuffle kernel.
+  // 64- / 128-element groups of bf16 rows: the tile kernel (a group is one or two row
+  // chunks of a stage); fp32 input (weight preparation): the warp-shuffle kernel.
   if (mode == 3 && !x_is_f32)
     return launch_mode<3, false>(x, rows, K, ldx, k, q, sf, status, stream);
+  if (mode == 4 && !x_is_f32)
+    return launch_mode<4, false>(x, rows, K, ldx, k, q, sf, status, stream);
   if (mode == 3 || mode == 4)
     return launch_rotate_quantize_wide(x, x_is_f32, rows, K, ldx, (int)rotation_span(mode), q, sf,
                                        stream);

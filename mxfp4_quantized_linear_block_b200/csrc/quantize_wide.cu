@@ -6,9 +6,10 @@
 // Hadamard rotations of larger blocks; the E8M0 scale stays per 32 elements. Butterfly
 // strides 1, 2, ..., n/2 in fp32, then one multiply by the fp32 nearest 1/sqrt(n).
 //
+// fp32 input (the offline weight preparation; bf16 activations take the tile quantiser).
 // A rotation group is spread over the lanes of a warp: each lane holds EPL consecutive
-// elements (8 for bf16 input: one 16-byte load; 4 for fp32), so a warp covers 32 * EPL
-// consecutive elements of a row. Butterfly strides below EPL run inside a lane, the
+// elements (4 fp32: one 16-byte load; the kernel is written for 8 bf16 as well), so a
+// warp covers 32 * EPL consecutive elements of a row. Butterfly strides below EPL run inside a lane, the
 // others pair lane l with l ^ (stride / EPL) through shuffles: the lower lane computes
 // a + b, the upper a - b as fma(b, -1, a), i.e. every element sees the fp32 operations
 // of a sequential evaluation, in the same order. amax and the scale are reduced over
@@ -211,11 +212,10 @@ cudaError_t launch_wide(const void* x, int64_t rows, int64_t K, int64_t ldx, uin
 cudaError_t launch_rotate_quantize_wide(const void* x, bool x_is_f32, int64_t rows, int64_t K,
                                         int64_t ldx, int span, uint8_t* q, uint8_t* sf,
                                         cudaStream_t stream) {
-  if (x_is_f32)
-    return span == 64 ? launch_wide<4, 64>(x, rows, K, ldx, q, sf, stream)
-                      : launch_wide<4, 128>(x, rows, K, ldx, q, sf, stream);
-  return span == 64 ? launch_wide<8, 64>(x, rows, K, ldx, q, sf, stream)
-                    : launch_wide<8, 128>(x, rows, K, ldx, q, sf, stream);
+  // bf16 rows take the tile quantiser (quantize.cu, modes 3 and 4)
+  if (!x_is_f32) return cudaErrorNotSupported;
+  return span == 64 ? launch_wide<4, 64>(x, rows, K, ldx, q, sf, stream)
+                    : launch_wide<4, 128>(x, rows, K, ldx, q, sf, stream);
 }
 
 }  // namespace mxfp4
