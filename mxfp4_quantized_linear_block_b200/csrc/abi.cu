@@ -68,6 +68,7 @@ bool kron_from_host(const float* a, const float* b, KronCoeffs* out) {
   if (!a || !b) return false;
   std::memcpy(out->a, a, sizeof(out->a));
   std::memcpy(out->b, b, sizeof(out->b));
+  kron_derive(out);
   return true;
 }
 

@@ -130,31 +130,33 @@ __device__ __forceinline__ void hadamard32(float2 (&P)[16]) {
 
 // y = (A (x) B) x: z[8j+k] = sum_l B[k][l] x[8j+l], y[8i+k] = sum_j A[i][j] z[8j+k],
 // each sum a chain that starts with the first product and adds the rest by fma
-// in ascending index order.
+// in ascending index order. Two outputs per packed fp32 operation, each lane doing that
+// chain: z[8j+k], z[8j+k+1] with the coefficient pair (B[k][l], B[k+1][l]) and x[8j+l]
+// in both lanes; y[8i+k], y[8i+k+1] with A[i][j] in both lanes.
 __device__ __forceinline__ void kron32(float2 (&P)[16], const KronCoeffs& kc) {
-  float z[32];
+  const float2* bt = reinterpret_cast<const float2*>(kc.bt);  // bt[4 l + kp]: k = 2 kp, 2 kp + 1
+  const float2* a2 = reinterpret_cast<const float2*>(kc.a2);  // a2[4 i + j]: A[i][j] twice
+  float2 zp[4][4];  // zp[j][kp] = (z[8j + 2kp], z[8j + 2kp + 1])
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      float acc = __fmul_rn(kc.b[k * 8 + 0], BLK(P, 8 * j + 0));
+    for (int l = 0; l < 8; ++l) {
+      const float xv = BLK(P, 8 * j + l);
+      const float2 xd = make_float2(xv, xv);
 #pragma unroll
-      for (int l = 1; l < 8; ++l) acc = __fmaf_rn(kc.b[k * 8 + l], BLK(P, 8 * j + l), acc);
-      z[8 * j + k] = acc;
+      for (int kp = 0; kp < 4; ++kp)
+        zp[j][kp] = l == 0 ? __fmul2_rn(bt[4 * l + kp], xd)
+                           : __ffma2_rn(bt[4 * l + kp], xd, zp[j][kp]);
     }
   }
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
 #pragma unroll
-    for (int k = 0; k < 8; k += 2) {
-      float y0 = __fmul_rn(kc.a[i * 4 + 0], z[k]);
-      float y1 = __fmul_rn(kc.a[i * 4 + 0], z[k + 1]);
+    for (int kp = 0; kp < 4; ++kp) {
+      float2 y = __fmul2_rn(a2[4 * i + 0], zp[0][kp]);
 #pragma unroll
-      for (int j = 1; j < 4; ++j) {
-        y0 = __fmaf_rn(kc.a[i * 4 + j], z[8 * j + k], y0);
-        y1 = __fmaf_rn(kc.a[i * 4 + j], z[8 * j + k + 1], y1);
-      }
-      P[(8 * i + k) >> 1] = make_float2(y0, y1);
+      for (int j = 1; j < 4; ++j) y = __ffma2_rn(a2[4 * i + j], zp[j][kp], y);
+      P[4 * i + kp] = y;
     }
   }
 }

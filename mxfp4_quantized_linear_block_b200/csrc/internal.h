@@ -11,7 +11,17 @@ namespace mxfp4 {
 struct KronCoeffs {
   float a[16];  // A, 4x4 row-major
   float b[64];  // B, 8x8 row-major
+  // The same numbers laid out for packed (two-lane) FMAs, filled by kron_derive:
+  // bt[8 l + k] = B[k][l] (two outputs k, k + 1 per pair), a2[2 q] = a2[2 q + 1] = a[q].
+  alignas(8) float bt[64];
+  alignas(8) float a2[32];
 };
+
+inline void kron_derive(KronCoeffs* kc) {
+  for (int k = 0; k < 8; ++k)
+    for (int l = 0; l < 8; ++l) kc->bt[8 * l + k] = kc->b[8 * k + l];
+  for (int q = 0; q < 16; ++q) kc->a2[2 * q] = kc->a2[2 * q + 1] = kc->a[q];
+}
 
 // Rotate (mode 0/1/2) + quantise x[rows, K] (bf16 or fp32) into packed codes q and
 // scale bytes sf (tensor-core layout, padding zeroed). Host-validated arguments.

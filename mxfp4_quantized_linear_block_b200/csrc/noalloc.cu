@@ -77,6 +77,7 @@ extern "C" mxfp4_status mxfp4_linear_noalloc(const void* x, int64_t M, int64_t K
     if (!kron_a || !kron_b) return MXFP4_ERR_INVALID_ARG;
     for (int i = 0; i < 16; ++i) kc.a[i] = kron_a[i];
     for (int i = 0; i < 64; ++i) kc.b[i] = kron_b[i];
+    kron_derive(&kc);
   }
   const size_t q_off = kStatusBytes;
   const size_t sf_off = round_up(q_off + (size_t)M * (size_t)(K / 2), 256);
