@@ -180,3 +180,18 @@ def test_norm_linear_kernel_count():
     assert kc(0, 256, 1024, mx.ROT_NONE) == 0
     assert kc(4, 256, 1024, mx.ROT_HADAMARD64) == -1
     assert kc(4, 24, 1024, mx.ROT_HADAMARD32) == -1
+
+
+def test_gemm_scratch_for_few_rows():
+    """The few-row GEMM's K-split partials go through the workspace's scratch for 33..128
+    rows split 4 or more ways: 4096 bytes past the pair kernel's counters, then
+    units x rows x 128 columns x 4 bytes; fewer splits or rows need no scratch."""
+    def gemm_ws(M, N, K):
+        return mx.workspace_bytes(mx.OP_GEMM, M, N, K)
+    # 4096 -> 14336 weights transposed: 32 W tiles x 8 splits = 256 units, 128 rows
+    assert gemm_ws(128, 4096, 14336) == 256 + 4096 + 256 * 128 * 128 * 4
+    # 100 rows, 8 W tiles x 7 splits (28 k-tiles in splits of 4)
+    assert gemm_ws(100, 1024, 7168) == 256 + 4096 + 56 * 100 * 128 * 4
+    assert gemm_ws(128, 14336, 4096) == 256  # 112 W tiles x 2 splits: on-chip sum
+    assert gemm_ws(32, 4096, 14336) == 256   # 32 rows: on-chip sum
+    assert gemm_ws(1, 14336, 4096) == 256
