@@ -233,7 +233,7 @@ def test_gemm_and_linear_with_no_rows_write_nothing():
 @pytest.mark.parametrize("M,N,K", [(33, 4608, 1536), (100, 1024, 7168), (128, 4096, 14336)])
 @pytest.mark.parametrize("out", ["bf16", "f32"])
 def test_few_rows_l2_and_on_chip_sums_agree(M, N, K, out):
-    """33..128 rows split 6 or 8 ways (36 W tiles x 6, 8 x 8, 32 x 8) sum their K splits
+    """33..128 rows split 6 to 8 ways (36 W tiles x 6, 8 x 7, 32 x 8) sum their K splits
     through L2 when the workspace has the scratch and
     through distributed shared memory when it has only the status word: same order of
     additions, so the same bits; both match the oracle."""
