@@ -62,11 +62,11 @@ def test_gemm_zero_and_single_pair():
 
 # Few activation rows (M <= 128): the weight-streaming kernel splits K over the
 # CTAs of a thread-block cluster and adds the partials through distributed shared
-# memory (up to 32 rows, or fewer than 4 splits) or through L2 (33..128 rows split 4 or
-# more ways, with the workspace's scratch). (M, N, K) -> W tiles x K splits: (1,16,4096) 1x8; (5,400,2080) 4x5 with a
-# 32-element K tail; (16,256,8192) 2x8; (17,12288,1024) 96x2; (33,9216,1536) 72x3;
-# (64,2048,3104) 16x7 with a K tail; (100,1024,7168) 8x7; (65,14336,4096) 112x2;
-# (128,4096,14336) 32x8.
+# memory (up to 32 rows, or fewer than 4 splits) or through L2 (33..128 rows split 4
+# or more ways, with the workspace's scratch). (M, N, K) -> W tiles x K splits:
+# (1,16,4096) 1x8; (5,400,2080) 4x5 with a 32-element K tail; (16,256,8192) 2x8;
+# (17,12288,1024) 96x2; (33,9216,1536) 72x3; (64,2048,3104) 16x7 with a K tail (L2);
+# (100,1024,7168) 8x7 (L2); (65,14336,4096) 112x2; (128,4096,14336) 32x8 (L2).
 SMALLM_SHAPES = [
     (1, 16, 4096), (5, 400, 2080), (16, 256, 8192), (17, 12288, 1024), (33, 9216, 1536),
     (64, 2048, 3104), (100, 1024, 7168), (65, 14336, 4096), (128, 4096, 14336),
