@@ -327,8 +327,10 @@ mxfp4_status mxfp4_nvfp4_gemm(const uint8_t* aq, const uint8_t* asf, const float
 
 /* The NVFP4 layer: tensor scale of the rotated x, quantise x, GEMM with the
  * pre-quantised weights (wq / wsf / *w_scale, from mxfp4_nvfp4_quantize with the
- * same mode), bf16 y [M, N]. ws: mxfp4_workspace_bytes(MXFP4_OP_NVFP4_LINEAR,
- * M, N, K) bytes, zeroed at allocation (status word as for mxfp4_linear). */
+ * same mode), bf16 y [M, N]: three kernels. ws: mxfp4_workspace_bytes(
+ * MXFP4_OP_NVFP4_LINEAR, M, N, K) bytes, zeroed at allocation (status word as
+ * for mxfp4_linear; the tensor-scale pass keeps two words of its own there and
+ * leaves them zero, so zero the workspace again after a timeout). */
 mxfp4_status mxfp4_nvfp4_linear(const void* x, int64_t M, int64_t K, mxfp4_rotation mode,
                                 const uint8_t* wq, const uint8_t* wsf, const float* w_scale,
                                 int64_t N, void* y, void* ws, size_t ws_bytes,
