@@ -106,14 +106,18 @@ size_t mxfp4_sf_bytes(int64_t rows, int64_t K);
 /* Byte offset of the scale of (row, 32-element block kblock) in that buffer, or -1 if out of range. */
 int64_t mxfp4_sf_offset(int64_t row, int64_t kblock, int64_t K);
 
-/* Device workspace that `op` needs for this problem (0 if none). It starts with
- * a status word; for MXFP4_OP_LINEAR it also holds the quantised activations;
- * for both GEMM-running ops it ends with the GEMM's scratch (K-split partials,
- * and counters for the last round of output tiles; sized for a 148-SM B200).
- * Allocate it zeroed: every call that completes leaves the counters zero (the
- * partials are rewritten before they are read, so their contents do not
- * matter). With a smaller scratch than this size, the few-row GEMM (M <= 128)
- * sums its K splits on chip instead (same bits, slower for 33..128 rows). */
+/* Device workspace that `op` needs for this problem (0 if none). Every
+ * workspace starts with the same 4352-byte head: a 256-byte status region (the
+ * status word at byte 0) and a 4096-byte block of GEMM counters (per-tile
+ * counters of a last round of output tiles split along K). The head sits at the
+ * same offsets whatever the op and sizes, so one workspace can serve calls of
+ * different sizes. After it come, for the layer ops, the quantised activations
+ * (and the NORM_LINEAR row statistics), then the GEMM's K-split partials (sized
+ * for a 148-SM B200). Allocate it zeroed: every call that completes leaves the
+ * counters zero, and the other parts are written before they are read. With a
+ * smaller partial area than this size, the CTA-pair GEMM does not split its
+ * last round and the few-row GEMM (M <= 128) sums its K splits on chip instead
+ * (slower; the few-row sums are the same bits). */
 size_t mxfp4_workspace_bytes(int op, int64_t M, int64_t N, int64_t K);
 
 /* Static description of a status code. Never NULL. */
@@ -170,11 +174,12 @@ mxfp4_status mxfp4_rotate_quantize(const void* x, mxfp4_dtype xdt, int64_t rows,
  * and ldy * elemsize a multiple of 16; aq, bq, asf, bsf 16-byte aligned.
  * ws: at least 256 bytes, zeroed when allocated; its first 16 bytes are the
  * device status word (see mxfp4_poll_status). mxfp4_workspace_bytes(
- * MXFP4_OP_GEMM, M, N, K) bytes give the fastest form; with less scratch (or
- * on a GPU whose SM count needs more), the last round of tiles is not split
- * along K and the few-row kernel sums its K splits on chip (slower; the
- * result still meets the stated tolerance, and the few-row sums are the same
- * bits). Fewer than 256 bytes -> MXFP4_ERR_WORKSPACE.
+ * MXFP4_OP_GEMM, M, N, K) bytes give the fastest form; with less (fewer than
+ * the 4352-byte head, too little room for the partials, or a GPU whose SM
+ * count needs more), the last round of tiles is not split along K and the
+ * few-row kernel sums its K splits on chip (slower; the result still meets
+ * the stated tolerance, and the few-row sums are the same bits). Fewer than
+ * 256 bytes -> MXFP4_ERR_WORKSPACE.
  * ("AMD Quark...", opening section: MXFP4 GEMM with no dequantisation;
  * "Bridging the Gap...", "GPU Kernel Ondersteuning (QuTLASS)".)
  */
@@ -182,6 +187,20 @@ mxfp4_status mxfp4_gemm(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq
                         const uint8_t* bsf, int64_t M, int64_t N, int64_t K, void* y,
                         mxfp4_dtype ydt, int64_t ldy, void* ws, size_t ws_bytes,
                         mxfp4_stream_t stream);
+
+/*
+ * Offline weight preparation for the Kronecker mode ("KroQuant...",
+ * "Hintergrund": the transform is invertible and its inverse goes on the
+ * weights). With activations rotated by T = A (x) B, weights are rotated by
+ * T^-T = A^-T (x) B^-T so that (T x) . (T^-T w) = x . w. This computes
+ * At_inv = (A^-1)^T (4x4) and Bt_inv = (B^-1)^T (8x8), all row-major HOST
+ * float arrays: each inverse by Gauss-Jordan elimination with partial pivoting
+ * in double, then every entry rounded once to fp32. Pass them as kron_a /
+ * kron_b of mxfp4_rotate_quantize on the fp32 weights. Host only, no GPU.
+ * NULL pointer, or a singular or non-finite factor -> MXFP4_ERR_INVALID_ARG.
+ */
+mxfp4_status mxfp4_kron_weight_factors(const float* A, const float* B, float* At_inv,
+                                       float* Bt_inv);
 
 /*
  * mxfp4_gemm with a bias: y[m][n] = (fp32 accumulator) + bias[n], one fp32
@@ -352,18 +371,26 @@ mxfp4_status mxfp4_nvfp4_linear(const void* x, int64_t M, int64_t K, mxfp4_rotat
  * MXFP4_NOALLOC_SCRATCH_BYTES (32 MiB) inside the library, which every GPU
  * that loads the library keeps until the process exits. Nothing is allocated
  * per call (no cudaMalloc / cudaFree, no allocating library routine).
- *  - Limit: 256 + round256(M * K / 2) + round256(mxfp4_sf_bytes(M, K)) must
+ *  - Arguments are checked exactly as mxfp4_linear checks them.
+ *  - Limit: 4352 + round256(M * K / 2) + round256(mxfp4_sf_bytes(M, K)) must
  *    not exceed the array (about 62 million activation elements); larger
- *    problems return MXFP4_ERR_WORKSPACE and launch nothing.
+ *    problems return MXFP4_ERR_WORKSPACE and launch nothing. The rest of the
+ *    array holds the GEMM's K-split partials when they fit (else the GEMM
+ *    runs without them: slower, same tolerance).
  *  - status: optional DEVICE pointer to a caller-owned, 4-byte aligned int
  *    that the caller zeroes; a bounded-wait timeout sets it to
  *    MXFP4_ERR_TIMEOUT. With NULL the library keeps a status word in its array
- *    and clears it at the start of each call (the caller cannot read it).
+ *    (the caller cannot read it).
+ *  - Each call first clears the array's status region and GEMM counter block
+ *    (one cudaMemsetAsync of 4352 bytes on `stream`), so nothing that an
+ *    earlier call left there -- a timed-out call's counters included -- is
+ *    seen; every other part it reads it writes first. A call after a timeout
+ *    needs no reset.
  *  - The first call on each device looks up the array's device address
  *    (cudaGetSymbolAddress) with that device current; make that first call
  *    before any stream capture.
  *  - Every call shares the one array, which keeps the previous call's
- *    contents (each call rewrites all of the part it reads). Calls whose
+ *    contents (see the clearing above). Calls whose
  *    kernels can overlap on the GPU -- different streams, or host threads
  *    without ordering between them -- race on the array and corrupt each
  *    other's results; keep them on one stream or otherwise ordered.
@@ -374,13 +401,38 @@ mxfp4_status mxfp4_linear_noalloc(const void* x, int64_t M, int64_t K, mxfp4_rot
                                   mxfp4_stream_t stream);
 
 /*
+ * Testing only: the faults that mxfp4_test_set_fault can make the GEMM simulate.
+ * MXFP4_TEST_FAULT_SKIP_SPLIT_PUBLISH: when the CTA-pair GEMM (M > 128) splits the
+ * tiles of its last round along K, chunk 1 of each split tile stores its partial
+ * but never publishes it; the chunk that owns the tile waits for it at most 1 ms
+ * (instead of 2 s), records MXFP4_ERR_TIMEOUT in the status word and finishes the
+ * tile without it (those output tiles are wrong). The kernel returns normally.
+ */
+typedef enum {
+  MXFP4_TEST_FAULT_NONE = 0,
+  MXFP4_TEST_FAULT_SKIP_SPLIT_PUBLISH = 1
+} mxfp4_test_fault;
+
+/*
+ * Testing only: make the GEMM launches set up after this call simulate `fault`
+ * (MXFP4_TEST_FAULT_NONE restores normal operation, the state at load time).
+ * It lets a test drive a bounded device wait to its limit -- the path that
+ * reports MXFP4_ERR_TIMEOUT -- with no GPU fault and no hang. Process-wide
+ * and read when a launch is set up; never call it in production code. After
+ * a simulated fault, zero the workspace before its next use (the counter
+ * block may be left set). Unknown values -> MXFP4_ERR_UNSUPPORTED.
+ */
+mxfp4_status mxfp4_test_set_fault(int fault);
+
+/*
  * Read the device status word at the start of a workspace (synchronises with
  * the device): MXFP4_OK, or MXFP4_ERR_TIMEOUT if a kernel's bounded wait on a
  * pipeline barrier ran out (the kernel then stopped early, released its
  * tensor memory and returned; its output is incomplete). The word is sticky:
  * kernels only ever set it, this call clears it. Zero the whole workspace once
  * when it is allocated, and again after a timeout (a kernel that stopped early
- * can leave GEMM scratch counters set).
+ * can leave GEMM counters, or the NVFP4 tensor-scale pass's words, set).
+ * mxfp4_linear_noalloc needs no such reset: it clears its own at each call.
  */
 mxfp4_status mxfp4_poll_status(void* ws, mxfp4_status* out);
 

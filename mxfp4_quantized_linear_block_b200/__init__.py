@@ -24,6 +24,7 @@ ROT_NONE, ROT_HADAMARD32, ROT_KRON_4x8, ROT_HADAMARD64, ROT_HADAMARD128 = 0, 1, 
 DT_BF16, DT_F32 = 0, 1
 OP_QUANTIZE, OP_GEMM, OP_LINEAR, OP_NVFP4_LINEAR, OP_NORM_LINEAR = 0, 1, 2, 3, 4
 NORM_LAYER, NORM_RMS = 0, 1
+TEST_FAULT_NONE, TEST_FAULT_SKIP_SPLIT_PUBLISH = 0, 1
 
 EXPORTS = (
     "mxfp4_sf_bytes", "mxfp4_sf_offset", "mxfp4_workspace_bytes", "mxfp4_status_string",
@@ -32,6 +33,7 @@ EXPORTS = (
     "mxfp4_nvfp4_sf_bytes", "mxfp4_nvfp4_tensor_scale", "mxfp4_nvfp4_quantize",
     "mxfp4_nvfp4_gemm", "mxfp4_nvfp4_linear", "mxfp4_norm_rotate_quantize", "mxfp4_norm_linear",
     "mxfp4_linear_kernel_count", "mxfp4_norm_linear_kernel_count",
+    "mxfp4_kron_weight_factors", "mxfp4_test_set_fault",
 )
 
 
@@ -74,6 +76,8 @@ def _load() -> ctypes.CDLL:
                                i64, vp, vp, sz, vp], i32),
         "mxfp4_linear_kernel_count": ([i64, i64, i64, i32], i32),
         "mxfp4_norm_linear_kernel_count": ([i64, i64, i64, i32], i32),
+        "mxfp4_kron_weight_factors": ([vp, vp, vp, vp], i32),
+        "mxfp4_test_set_fault": ([i32], i32),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -408,10 +412,20 @@ def poll_status(ws) -> int:
 
 
 def kron_weight_factors(A, B):
-    """Weight-side factors of the Kronecker mode: (A^-T, B^-T), inverted in float64 on the host
-    (a 4x4 and an 8x8 matrix) and rounded to float32."""
+    """Weight-side factors of the Kronecker mode, (A^-T, B^-T) as float32 arrays, from
+    mxfp4_kron_weight_factors (double Gauss-Jordan inverses, rounded once to fp32)."""
     import numpy as np
-    A = np.asarray(A, dtype=np.float64)
-    B = np.asarray(B, dtype=np.float64)
-    return (np.linalg.inv(A).T.astype(np.float32).copy(),
-            np.linalg.inv(B).T.astype(np.float32).copy())
+    A = np.ascontiguousarray(A, dtype=np.float32)
+    B = np.ascontiguousarray(B, dtype=np.float32)
+    assert A.shape == (4, 4) and B.shape == (8, 8)
+    At = np.empty((4, 4), dtype=np.float32)
+    Bt = np.empty((8, 8), dtype=np.float32)
+    _check(lib.mxfp4_kron_weight_factors(A.ctypes.data, B.ctypes.data, At.ctypes.data,
+                                         Bt.ctypes.data), "mxfp4_kron_weight_factors")
+    return At, Bt
+
+
+def test_set_fault(fault: int) -> None:
+    """Testing only: make later GEMM launches simulate `fault` (TEST_FAULT_*); see
+    mxfp4_test_set_fault in include/mxfp4.h."""
+    _check(lib.mxfp4_test_set_fault(fault), "mxfp4_test_set_fault")

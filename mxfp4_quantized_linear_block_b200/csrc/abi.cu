@@ -3,36 +3,17 @@
 // is allocated here; every launch is ordered on the caller's stream.
 #include <cuda_runtime.h>
 
+#include <cmath>
 #include <cstdint>
-#include <cstring>
+#include <utility>
 
-#include "../../include/mxfp4.h"
 #include "internal.h"
 
 using namespace mxfp4;
 
 namespace {
 
-constexpr size_t kStatusBytes = 256;  // status word region at the start of a workspace
-
-bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
-size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
-
-// Valid [rows, K] operand description for the scale layout.
-bool shape_ok(int64_t rows, int64_t K) { return rows >= 0 && K >= 32 && K % 32 == 0; }
-
-// Limits of the kernels' 32-bit index arithmetic.
-bool within_limits(int64_t rows, int64_t K) {
-  const int64_t units = sf_row_tiles(rows) * 128 * sf_katoms(K) * 4;
-  return rows < (1ll << 31) && K < (1ll << 31) && units < (1ll << 32);
-}
-
 mxfp4_status from_cuda(cudaError_t e) { return e == cudaSuccess ? MXFP4_OK : MXFP4_ERR_CUDA; }
-
-// A row operand (activations, their codes and scales, the output) may be NULL when it has
-// no rows: torch and other frameworks hand out NULL for empty tensors.
-bool rows_ptr_ok(const void* p, int64_t rows) { return p != nullptr || rows == 0; }
 
 mxfp4_status validate_quantize(const void* x, mxfp4_dtype xdt, int64_t rows, int64_t K,
                                int64_t ldx, const uint8_t* q, const uint8_t* sf) {
@@ -62,61 +43,97 @@ mxfp4_status validate_gemm(const uint8_t* aq, const uint8_t* asf, const uint8_t*
   return MXFP4_OK;
 }
 
-bool mode_ok(int mode) { return mode >= MXFP4_ROT_NONE && mode <= MXFP4_ROT_HADAMARD128; }
-
-bool kron_from_host(const float* a, const float* b, KronCoeffs* out) {
-  if (!a || !b) return false;
-  std::memcpy(out->a, a, sizeof(out->a));
-  std::memcpy(out->b, b, sizeof(out->b));
-  kron_derive(out);
-  return true;
+// The GEMM scratch of a GEMM-only workspace: [status | counters | data]. A workspace of
+// fewer than kHeadBytes has no counter block (the last round is then not split).
+GemmScratch gemm_workspace_scratch(void* ws, size_t ws_bytes) {
+  if (ws_bytes < kHeadBytes) return GemmScratch{};
+  return workspace_scratch(static_cast<uint8_t*>(ws), kHeadBytes, ws_bytes);
 }
 
-// Workspace of mxfp4_linear: [status | Xq (M x K/2) | Xsf | GEMM scratch], each part
-// 256-byte aligned.
-struct LinearWorkspace {
-  size_t q_off, sf_off, g_off, total;
-};
-
-// Workspace of mxfp4_nvfp4_linear: [status (X tensor scale at 64, the scale pass's
-// running maximum and block counter at 72 and 76) | Xq | Xsf | GEMM scratch].
+// Workspace of mxfp4_nvfp4_linear: the layer layout with NVFP4 scale bytes; the status
+// region holds the X tensor scale at 64 and the scale pass's running maximum and block
+// counter at 72 and 76.
 constexpr size_t kScaleOff = 64;
 
-LinearWorkspace nvfp4_linear_workspace(int64_t M, int64_t N, int64_t K) {
-  LinearWorkspace w;
-  w.q_off = kStatusBytes;
-  w.sf_off = round_up(w.q_off + (size_t)M * (size_t)(K / 2), 256);
-  w.g_off = round_up(w.sf_off + mxfp4_sf_bytes(M, 2 * K), 256);
-  w.total = round_up(w.g_off + gemm_scratch_bytes(M, N, K), 256);
-  return w;
-}
-
-// Workspace of mxfp4_norm_linear: [status | Xq | Xsf | row statistics (M x 8 bytes) |
-// GEMM scratch]; g_off of the returned value is the GEMM scratch, stats sit before it.
+// Workspace of mxfp4_norm_linear: [status | counters | Xq | Xsf | row statistics (M x 8
+// bytes) | GEMM data].
 struct NormWorkspace {
   size_t q_off, sf_off, st_off, g_off, total;
 };
 
 NormWorkspace norm_linear_workspace(int64_t M, int64_t N, int64_t K) {
+  const LinearLayout l = linear_layout(M, N, K, K);
   NormWorkspace w;
-  w.q_off = kStatusBytes;
-  w.sf_off = round_up(w.q_off + (size_t)M * (size_t)(K / 2), 256);
-  w.st_off = round_up(w.sf_off + mxfp4_sf_bytes(M, K), 256);
+  w.q_off = l.q_off;
+  w.sf_off = l.sf_off;
+  w.st_off = l.g_off;
   w.g_off = round_up(w.st_off + (size_t)M * 2 * sizeof(float), 256);
   w.total = round_up(w.g_off + gemm_scratch_bytes(M, N, K), 256);
   return w;
 }
 
-LinearWorkspace linear_workspace(int64_t M, int64_t N, int64_t K) {
-  LinearWorkspace w;
-  w.q_off = kStatusBytes;
+// Inverse of the n x n row-major matrix a (n <= 8) in double by Gauss-Jordan elimination
+// on [a | I], choosing as pivot the largest magnitude in the column at or below the
+// diagonal; false if a pivot is zero or a value is not finite.
+bool invert_small(const float* a, int n, double* inv) {
+  double m[8][16];
+  for (int r = 0; r < n; ++r)
+    for (int c = 0; c < 2 * n; ++c)
+      m[r][c] = c < n ? (double)a[r * n + c] : (c - n == r ? 1.0 : 0.0);
+  for (int col = 0; col < n; ++col) {
+    int piv = col;
+    for (int r = col + 1; r < n; ++r)
+      if (std::fabs(m[r][col]) > std::fabs(m[piv][col])) piv = r;
+    if (!(std::fabs(m[piv][col]) > 0.0) || !std::isfinite(m[piv][col])) return false;
+    if (piv != col)
+      for (int c = 0; c < 2 * n; ++c) std::swap(m[piv][c], m[col][c]);
+    const double d = m[col][col];
+    for (int c = 0; c < 2 * n; ++c) m[col][c] /= d;
+    for (int r = 0; r < n; ++r) {
+      if (r == col) continue;
+      const double f = m[r][col];
+      if (f == 0.0) continue;
+      for (int c = 0; c < 2 * n; ++c) m[r][c] -= f * m[col][c];
+    }
+  }
+  for (int r = 0; r < n; ++r)
+    for (int c = 0; c < n; ++c) {
+      inv[r * n + c] = m[r][n + c];
+      if (!std::isfinite(inv[r * n + c])) return false;
+    }
+  return true;
+}
+
+}  // namespace
+
+namespace mxfp4 {
+
+LinearLayout linear_layout(int64_t M, int64_t N, int64_t K, int64_t sf_k) {
+  LinearLayout w;
+  w.q_off = kHeadBytes;
   w.sf_off = round_up(w.q_off + (size_t)M * (size_t)(K / 2), 256);
-  w.g_off = round_up(w.sf_off + mxfp4_sf_bytes(M, K), 256);
+  w.g_off = round_up(w.sf_off + mxfp4_sf_bytes(M, sf_k), 256);
   w.total = round_up(w.g_off + gemm_scratch_bytes(M, N, K), 256);
   return w;
 }
 
-}  // namespace
+mxfp4_status validate_linear(const void* x, int64_t M, int64_t K, mxfp4_rotation mode,
+                             const float* kron_a, const float* kron_b, const uint8_t* wq,
+                             const uint8_t* wsf, int64_t N, const void* y, KronCoeffs* kc) {
+  if (!rows_ptr_ok(x, M) || !wq || !wsf || !rows_ptr_ok(y, M)) return MXFP4_ERR_INVALID_ARG;
+  if (!mode_ok(mode)) return MXFP4_ERR_UNSUPPORTED;
+  if (!shape_ok(M, K) || K % rotation_span(mode) != 0 || N < 16 || N % 16 != 0 ||
+      !within_limits(M, K) || !within_limits(N, K))
+    return MXFP4_ERR_SHAPE;
+  if (!aligned16(x) || !aligned16(wq) || !aligned16(wsf) || !aligned16(y) ||
+      (K * 2) % 16 != 0 || (N * 2) % 16 != 0)
+    return MXFP4_ERR_ALIGN;
+  if (mode == MXFP4_ROT_KRON_4x8 && !kron_from_host(kron_a, kron_b, kc))
+    return MXFP4_ERR_INVALID_ARG;
+  return MXFP4_OK;
+}
+
+}  // namespace mxfp4
 
 extern "C" {
 
@@ -137,14 +154,14 @@ size_t mxfp4_workspace_bytes(int op, int64_t M, int64_t N, int64_t K) {
     case MXFP4_OP_QUANTIZE:
       return 0;
     case MXFP4_OP_GEMM:
-      if (!shape_ok(M, K) || N < 0) return kStatusBytes;
-      return kStatusBytes + round_up(gemm_scratch_bytes(M, N, K), 256);
+      if (!shape_ok(M, K) || N < 0) return kHeadBytes;
+      return kHeadBytes + round_up(gemm_scratch_bytes(M, N, K), 256);
     case MXFP4_OP_LINEAR:
       if (!shape_ok(M, K) || N < 0) return 0;
-      return linear_workspace(M, N, K).total;
+      return linear_layout(M, N, K, K).total;
     case MXFP4_OP_NVFP4_LINEAR:
       if (!shape_ok(M, K) || N < 0) return 0;
-      return nvfp4_linear_workspace(M, N, K).total;
+      return linear_layout(M, N, K, 2 * K).total;
     case MXFP4_OP_NORM_LINEAR:
       if (!shape_ok(M, K) || N < 0) return 0;
       return norm_linear_workspace(M, N, K).total;
@@ -202,9 +219,9 @@ mxfp4_status mxfp4_gemm(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq
   // The caller's previous kernel may have written bq / bsf: no early weight loads.
   Epilogue ep;
   ep.out = ydt == MXFP4_DT_F32 ? kOutF32 : kOutBf16;
-  return from_cuda(launch_gemm(aq, asf, bq, bsf, M, N, K, y, ep, ldy,
-                               static_cast<int*>(ws), static_cast<uint8_t*>(ws) + kStatusBytes,
-                               ws_bytes - kStatusBytes, false, static_cast<cudaStream_t>(stream)));
+  return from_cuda(launch_gemm(aq, asf, bq, bsf, M, N, K, y, ep, ldy, static_cast<int*>(ws),
+                               gemm_workspace_scratch(ws, ws_bytes), false,
+                               static_cast<cudaStream_t>(stream)));
 }
 
 mxfp4_status mxfp4_gemm_bias(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq,
@@ -221,8 +238,8 @@ mxfp4_status mxfp4_gemm_bias(const uint8_t* aq, const uint8_t* asf, const uint8_
   ep.out = ydt == MXFP4_DT_F32 ? kOutF32 : kOutBf16;
   ep.bias = bias;
   return from_cuda(launch_gemm(aq, asf, bq, bsf, M, N, K, y, ep, ldy, static_cast<int*>(ws),
-                               static_cast<uint8_t*>(ws) + kStatusBytes, ws_bytes - kStatusBytes,
-                               false, static_cast<cudaStream_t>(stream)));
+                               gemm_workspace_scratch(ws, ws_bytes), false,
+                               static_cast<cudaStream_t>(stream)));
 }
 
 mxfp4_status mxfp4_gemm_quantize(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq,
@@ -252,34 +269,27 @@ mxfp4_status mxfp4_gemm_quantize(const uint8_t* aq, const uint8_t* asf, const ui
     return MXFP4_ERR_INVALID_ARG;
   if (M == 0) return MXFP4_OK;
   return from_cuda(launch_gemm(aq, asf, bq, bsf, M, N, K, yq, ep, N / 2, static_cast<int*>(ws),
-                               static_cast<uint8_t*>(ws) + kStatusBytes, ws_bytes - kStatusBytes,
-                               false, static_cast<cudaStream_t>(stream)));
+                               gemm_workspace_scratch(ws, ws_bytes), false,
+                               static_cast<cudaStream_t>(stream)));
 }
 
 mxfp4_status mxfp4_linear(const void* x, int64_t M, int64_t K, mxfp4_rotation mode,
                           const float* kron_a, const float* kron_b, const uint8_t* wq,
                           const uint8_t* wsf, int64_t N, void* y, void* ws, size_t ws_bytes,
                           mxfp4_stream_t stream) {
-  if (!rows_ptr_ok(x, M) || !wq || !wsf || !rows_ptr_ok(y, M) || !ws)
-    return MXFP4_ERR_INVALID_ARG;
-  if (!mode_ok(mode)) return MXFP4_ERR_UNSUPPORTED;
-  if (!shape_ok(M, K) || K % rotation_span(mode) != 0 || N < 16 || N % 16 != 0 ||
-      !within_limits(M, K) || !within_limits(N, K))
-    return MXFP4_ERR_SHAPE;
-  if (!aligned16(x) || !aligned16(wq) || !aligned16(wsf) || !aligned16(y) || !aligned16(ws) ||
-      (K * 2) % 16 != 0 || (N * 2) % 16 != 0)
-    return MXFP4_ERR_ALIGN;
-  const LinearWorkspace w = linear_workspace(M, N, K);
-  if (ws_bytes < w.total) return MXFP4_ERR_WORKSPACE;
   KronCoeffs kc{};
-  if (mode == MXFP4_ROT_KRON_4x8 && !kron_from_host(kron_a, kron_b, &kc))
-    return MXFP4_ERR_INVALID_ARG;
+  const mxfp4_status st = validate_linear(x, M, K, mode, kron_a, kron_b, wq, wsf, N, y, &kc);
+  if (st != MXFP4_OK) return st;
+  if (!ws) return MXFP4_ERR_INVALID_ARG;
+  if (!aligned16(ws)) return MXFP4_ERR_ALIGN;
+  const LinearLayout w = linear_layout(M, N, K, K);
+  if (ws_bytes < w.total) return MXFP4_ERR_WORKSPACE;
   if (M == 0) return MXFP4_OK;
   uint8_t* base = static_cast<uint8_t*>(ws);
   uint8_t* xq = base + w.q_off;
   uint8_t* xsf = base + w.sf_off;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  // Up to 16 rows: one kernel quantises x inside the GEMM's CTAs.
+  // 1..8 rows: one kernel quantises x inside the GEMM's CTAs.
   cudaError_t e = launch_linear_smallm(x, K, (int)mode, &kc, wq, wsf, M, N, K, y, N,
                                        static_cast<int*>(ws), s);
   if (e != cudaErrorNotSupported) return from_cuda(e);
@@ -287,7 +297,7 @@ mxfp4_status mxfp4_linear(const void* x, int64_t M, int64_t K, mxfp4_rotation mo
   if (e != cudaSuccess) return MXFP4_ERR_CUDA;
   // The kernel just before the GEMM is the quantiser above, which does not write W.
   return from_cuda(launch_gemm(xq, xsf, wq, wsf, M, N, K, y, Epilogue{}, N, static_cast<int*>(ws),
-                               base + w.g_off, ws_bytes - w.g_off, true, s));
+                               workspace_scratch(base, w.g_off, ws_bytes), true, s));
 }
 
 int mxfp4_linear_kernel_count(int64_t M, int64_t N, int64_t K, mxfp4_rotation mode) {
@@ -361,8 +371,8 @@ mxfp4_status mxfp4_norm_linear(const void* x, int64_t M, int64_t K, mxfp4_norm k
   if (e != cudaSuccess) return MXFP4_ERR_CUDA;
   // The kernel just before the GEMM is the quantiser above, which does not write W.
   return from_cuda(launch_gemm(base + w.q_off, base + w.sf_off, wq, wsf, M, N, K, y, Epilogue{},
-                               N, static_cast<int*>(ws), base + w.g_off, ws_bytes - w.g_off, true,
-                               s));
+                               N, static_cast<int*>(ws), workspace_scratch(base, w.g_off, ws_bytes),
+                               true, s));
 }
 
 size_t mxfp4_nvfp4_sf_bytes(int64_t rows, int64_t K) {
@@ -417,8 +427,8 @@ mxfp4_status mxfp4_nvfp4_gemm(const uint8_t* aq, const uint8_t* asf, const float
   ep.a_scale = a_scale;
   ep.b_scale = b_scale;
   return from_cuda(launch_gemm(aq, asf, bq, bsf, M, N, K, y, ep, ldy, static_cast<int*>(ws),
-                               static_cast<uint8_t*>(ws) + kStatusBytes, ws_bytes - kStatusBytes,
-                               false, static_cast<cudaStream_t>(stream)));
+                               gemm_workspace_scratch(ws, ws_bytes), false,
+                               static_cast<cudaStream_t>(stream)));
 }
 
 mxfp4_status mxfp4_nvfp4_linear(const void* x, int64_t M, int64_t K, mxfp4_rotation mode,
@@ -434,7 +444,7 @@ mxfp4_status mxfp4_nvfp4_linear(const void* x, int64_t M, int64_t K, mxfp4_rotat
   if (!aligned16(x) || !aligned16(wq) || !aligned16(wsf) || !aligned16(y) || !aligned16(ws) ||
       (K * 2) % 16 != 0 || (N * 2) % 16 != 0 || (reinterpret_cast<uintptr_t>(w_scale) & 3u))
     return MXFP4_ERR_ALIGN;
-  const LinearWorkspace w = nvfp4_linear_workspace(M, N, K);
+  const LinearLayout w = linear_layout(M, N, K, 2 * K);
   if (ws_bytes < w.total) return MXFP4_ERR_WORKSPACE;
   if (M == 0) return MXFP4_OK;
   uint8_t* base = static_cast<uint8_t*>(ws);
@@ -454,8 +464,28 @@ mxfp4_status mxfp4_nvfp4_linear(const void* x, int64_t M, int64_t K, mxfp4_rotat
   ep.b_scale = w_scale;
   // The kernel just before the GEMM is the quantiser above, which does not write W.
   return from_cuda(launch_gemm(base + w.q_off, base + w.sf_off, wq, wsf, M, N, K, y, ep, N,
-                               static_cast<int*>(ws), base + w.g_off, ws_bytes - w.g_off, true,
-                               s));
+                               static_cast<int*>(ws), workspace_scratch(base, w.g_off, ws_bytes),
+                               true, s));
+}
+
+mxfp4_status mxfp4_kron_weight_factors(const float* A, const float* B, float* At_inv,
+                                       float* Bt_inv) {
+  if (!A || !B || !At_inv || !Bt_inv) return MXFP4_ERR_INVALID_ARG;
+  double ai[16], bi[64];
+  if (!invert_small(A, 4, ai) || !invert_small(B, 8, bi)) return MXFP4_ERR_INVALID_ARG;
+  // (A^-1)^T and (B^-1)^T, each entry rounded once to fp32
+  for (int r = 0; r < 4; ++r)
+    for (int c = 0; c < 4; ++c) At_inv[r * 4 + c] = (float)ai[c * 4 + r];
+  for (int r = 0; r < 8; ++r)
+    for (int c = 0; c < 8; ++c) Bt_inv[r * 8 + c] = (float)bi[c * 8 + r];
+  return MXFP4_OK;
+}
+
+mxfp4_status mxfp4_test_set_fault(int fault) {
+  if (fault != MXFP4_TEST_FAULT_NONE && fault != MXFP4_TEST_FAULT_SKIP_SPLIT_PUBLISH)
+    return MXFP4_ERR_UNSUPPORTED;
+  g_test_fault.store(fault);
+  return MXFP4_OK;
 }
 
 mxfp4_status mxfp4_poll_status(void* ws, mxfp4_status* out) {

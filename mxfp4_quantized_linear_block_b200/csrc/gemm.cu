@@ -27,6 +27,7 @@
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdint>
 
 #include "block_quant.cuh"
@@ -62,7 +63,8 @@ struct Params {
   // Work units: tiles [0, full_units) whole; each later tile split into split_g K chunks
   // of kt_per_chunk k-tiles (units full_units + t * split_g + c). Chunk 0 owns the tile.
   uint32_t full_units, units, split_g, kt_per_chunk;
-  unsigned int* flags;     // [2 * split tiles]: partials stored, owner warps done
+  unsigned int* flags;     // [2 * split tiles] in the fixed counter block: partials stored,
+                           // owner warps done
   float* part;             // [split tile][chunk 1..g-1][CTA rank] x 128 x 256 fp32
   const float* bias;       // [N] or null
   uint8_t* yq;             // MXFP4 output: codes [M, ldy bytes per row]
@@ -71,6 +73,9 @@ struct Params {
   uint32_t rows_pad, n_katoms_y;
   const float* a_scale;    // NVFP4: tensor scales of A and B (device fp32)
   const float* b_scale;
+  uint64_t count_wait_ns;  // bound of the owner's wait for the other chunks' partials
+  uint32_t skip_publish;   // testing only: chunk that stores its partial but never
+                           // publishes it (0: none, every chunk publishes)
 };
 
 struct Unit {
@@ -120,10 +125,11 @@ __device__ __forceinline__ uint64_t global_ns() {
 }
 
 // Bounded wait until *ptr >= target (stores of the other chunks of a split tile).
-__device__ __forceinline__ bool wait_count(const unsigned int* ptr, uint32_t target) {
+__device__ __forceinline__ bool wait_count(const unsigned int* ptr, uint32_t target,
+                                           uint64_t limit_ns) {
   const uint64_t t0 = global_ns();
   while (ld_acquire_u32(ptr) < target) {
-    if (global_ns() - t0 > kWaitLimitNs) return false;
+    if (global_ns() - t0 > limit_ns) return false;
     __nanosleep(100);
   }
   return true;
@@ -388,7 +394,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       // Split tile, chunk 0: the other chunks' partials must be stored before they are added.
       if (w.split && w.chunk == 0) {
         bool got = true;
-        if (lane == 0) got = wait_count(p.flags + st, (p.split_g - 1) * 2u * kEpiWarps);
+        if (lane == 0)
+          got = wait_count(p.flags + st, (p.split_g - 1) * 2u * kEpiWarps, p.count_wait_ns);
         got = __shfl_sync(0xffffffffu, got ? 1 : 0, 0) != 0;
         if (!got && lane == 0) record_timeout(p.status);
       }
@@ -529,7 +536,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           // Publish this warp's part of the partial to the owner.
           __threadfence();
           __syncwarp();
-          if (lane == 0) atomicAdd(p.flags + st, 1u);
+          if (lane == 0 && w.chunk != p.skip_publish) atomicAdd(p.flags + st, 1u);
         } else {
           // Owner warps done reading: the last one clears both counters for the next launch.
           __syncwarp();
@@ -642,10 +649,8 @@ constexpr uint32_t kMaxSplit = 4;
 
 struct PairPlan {
   uint32_t tiles, full_units, units, g, kt_per_chunk, n_split;
-  size_t flag_bytes, scratch_bytes;
+  size_t scratch_bytes;  // fp32 partials (the data part of the scratch)
 };
-
-size_t round256(size_t v) { return (v + 255) / 256 * 256; }
 
 PairPlan pair_plan(int64_t M, int64_t N, int64_t K, uint32_t pairs) {
   PairPlan pl{};
@@ -660,6 +665,8 @@ PairPlan pair_plan(int64_t M, int64_t N, int64_t K, uint32_t pairs) {
   if (g > k_tiles / kMinChunkKt) g = k_tiles / kMinChunkKt;
   if (g > kMaxSplit) g = kMaxSplit;
   if (g < 2) return pl;
+  // two counters per split tile, all inside the fixed counter block
+  if ((size_t)2 * tail * sizeof(unsigned int) > kCounterBytes) return pl;
   const uint32_t kt = (k_tiles + g - 1) / g;
   g = (k_tiles + kt - 1) / kt;
   if (g < 2) return pl;
@@ -668,16 +675,15 @@ PairPlan pair_plan(int64_t M, int64_t N, int64_t K, uint32_t pairs) {
   pl.n_split = tail;
   pl.full_units = pl.tiles - tail;
   pl.units = pl.full_units + tail * g;
-  pl.flag_bytes = round256((size_t)2 * tail * sizeof(unsigned int));
-  pl.scratch_bytes = pl.flag_bytes + (size_t)tail * (g - 1) * 2 * 128 * 256 * sizeof(float);
+  pl.scratch_bytes = (size_t)tail * (g - 1) * 2 * 128 * 256 * sizeof(float);
   return pl;
 }
 
 template <uint32_t STAGES, int OUT, bool NV>
 cudaError_t launch_pair(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq,
                         const uint8_t* bsf, int64_t M, int64_t N, int64_t K, void* y,
-                        const Epilogue& ep, int64_t ldy, int* status, uint8_t* scratch,
-                        size_t scratch_bytes, cudaStream_t stream) {
+                        const Epilogue& ep, int64_t ldy, int* status,
+                        const GemmScratch& scratch, cudaStream_t stream) {
   using C = PairConfig<STAGES, NV>;
   // scale atoms per 128-row group: one per 4 scales, i.e. per 128 (MXFP4) or 64 (NVFP4) K
   const uint64_t k_atoms = (uint64_t)sf_katoms(NV ? 2 * K : K);
@@ -728,14 +734,15 @@ cudaError_t launch_pair(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq
   p.b_row_tiles = (uint32_t)sf_row_tiles(N);
   p.ldy = (uint64_t)ldy;
   PairPlan pl = pair_plan(M, N, K, (uint32_t)max_clusters[dev]);
-  if (pl.g > 1 && (scratch == nullptr || pl.scratch_bytes > scratch_bytes))
-    pl = pair_plan(M, N, K, 0);  // no room for partials: whole tiles only
+  if (pl.g > 1 && (scratch.counters == nullptr || scratch.data == nullptr ||
+                   pl.scratch_bytes > scratch.data_bytes))
+    pl = pair_plan(M, N, K, 0);  // no counters or no room for partials: whole tiles only
   p.full_units = pl.full_units;
   p.units = pl.units;
   p.split_g = pl.g;
   p.kt_per_chunk = pl.kt_per_chunk;
-  p.flags = pl.g > 1 ? reinterpret_cast<unsigned int*>(scratch) : nullptr;
-  p.part = pl.g > 1 ? reinterpret_cast<float*>(scratch + pl.flag_bytes) : nullptr;
+  p.flags = pl.g > 1 ? scratch.counters : nullptr;
+  p.part = pl.g > 1 ? reinterpret_cast<float*>(scratch.data) : nullptr;
   p.bias = ep.bias;
   p.yq = OUT == kOutMxfp4 ? static_cast<uint8_t*>(y) : nullptr;
   p.ysf = ep.ysf;
@@ -744,6 +751,12 @@ cudaError_t launch_pair(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq
   p.n_katoms_y = (uint32_t)sf_katoms(N);
   p.a_scale = ep.a_scale;
   p.b_scale = ep.b_scale;
+  p.count_wait_ns = kWaitLimitNs;
+  p.skip_publish = 0;
+  if (g_test_fault.load(std::memory_order_relaxed) == MXFP4_TEST_FAULT_SKIP_SPLIT_PUBLISH) {
+    p.skip_publish = 1;             // chunk 1 of every split tile
+    p.count_wait_ns = 1000000ull;   // 1 ms
+  }
   const uint32_t pairs =
       pl.units < (uint32_t)max_clusters[dev] ? pl.units : (uint32_t)max_clusters[dev];
 
@@ -762,32 +775,34 @@ cudaError_t launch_pair(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq
 
 }  // namespace
 
+std::atomic<int> g_test_fault{MXFP4_TEST_FAULT_NONE};
+
 cudaError_t launch_gemm(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq,
                         const uint8_t* bsf, int64_t M, int64_t N, int64_t K, void* y,
-                        const Epilogue& ep, int64_t ldy, int* status, uint8_t* scratch,
-                        size_t scratch_bytes, bool b_early, cudaStream_t stream) {
+                        const Epilogue& ep, int64_t ldy, int* status, const GemmScratch& scratch,
+                        bool b_early, cudaStream_t stream) {
   // Few activation rows: stream the weights with the swap-AB split-K kernel.
   if (M <= 128)
-    return launch_gemm_smallm(aq, asf, bq, bsf, M, N, K, y, ep, ldy, status, scratch,
-                              scratch_bytes, b_early, stream);
+    return launch_gemm_smallm(aq, asf, bq, bsf, M, N, K, y, ep, ldy, status, scratch, b_early,
+                              stream);
   // Otherwise CTA pairs with 256 x 256 tiles.
   if (ep.nvfp4) {
     if (ep.out == kOutF32)
       return launch_pair<5, kOutF32, true>(aq, asf, bq, bsf, M, N, K, y, ep, ldy, status,
-                                           scratch, scratch_bytes, stream);
+                                           scratch, stream);
     return launch_pair<5, kOutBf16, true>(aq, asf, bq, bsf, M, N, K, y, ep, ldy, status, scratch,
-                                          scratch_bytes, stream);
+                                          stream);
   }
   switch (ep.out) {
     case kOutF32:
       return launch_pair<5, kOutF32, false>(aq, asf, bq, bsf, M, N, K, y, ep, ldy, status,
-                                            scratch, scratch_bytes, stream);
+                                            scratch, stream);
     case kOutMxfp4:
       return launch_pair<5, kOutMxfp4, false>(aq, asf, bq, bsf, M, N, K, y, ep, ldy, status,
-                                              scratch, scratch_bytes, stream);
+                                              scratch, stream);
     default:
       return launch_pair<5, kOutBf16, false>(aq, asf, bq, bsf, M, N, K, y, ep, ldy, status,
-                                             scratch, scratch_bytes, stream);
+                                             scratch, stream);
   }
 }
 

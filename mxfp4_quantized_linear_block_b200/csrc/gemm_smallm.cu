@@ -658,7 +658,7 @@ Plan make_plan(int64_t M, int64_t N, int64_t K) {
   return pl;
 }
 
-// L2 bytes of the K-split partials (after kSmallRedOffset in the GEMM scratch): for more
+// L2 bytes of the K-split partials (the data part of the GEMM scratch): for more
 // than 32 tokens split 4 or more ways; 0 means the sum goes through distributed shared
 // memory. (B200, 128 tokens: 8 splits 15.0 -> 13.2 us through L2; 2 splits, where half
 // of the reads are the CTA's own shared memory, 13.1 -> 13.9 us, so they stay on chip.)
@@ -752,19 +752,18 @@ cudaError_t launch_linear_smallm(const void* x, int64_t ldx, int mode, const Kro
 }
 
 size_t gemm_smallm_scratch_bytes(int64_t M, int64_t N, int64_t K) {
-  const size_t r = red_bytes(make_plan(M, N, K), M);
-  return r ? kSmallRedOffset + r : 0;
+  return red_bytes(make_plan(M, N, K), M);
 }
 
 cudaError_t launch_gemm_smallm(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq,
                                const uint8_t* bsf, int64_t M, int64_t N, int64_t K, void* y,
-                               const Epilogue& ep, int64_t ldy, int* status, uint8_t* scratch,
-                               size_t scratch_bytes, bool b_early, cudaStream_t stream) {
+                               const Epilogue& ep, int64_t ldy, int* status,
+                               const GemmScratch& scratch, bool b_early, cudaStream_t stream) {
   const Plan pl = make_plan(M, N, K);
   // K-split partials through L2 when the caller's scratch holds them, else on chip
   const size_t rb = red_bytes(pl, M);
-  float* red = rb && scratch && scratch_bytes >= kSmallRedOffset + rb
-                   ? reinterpret_cast<float*>(scratch + kSmallRedOffset)
+  float* red = rb && scratch.data && scratch.data_bytes >= rb
+                   ? reinterpret_cast<float*>(scratch.data)
                    : nullptr;
 #define MXFP4_SMALLM_LAUNCH(NTV, OUTV, NVV)                                           \
   return launch_nt<NTV, OUTV, NVV>(pl, aq, asf, bq, bsf, M, N, K, y, ep, ldy, status, \

@@ -3,7 +3,11 @@
 
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdint>
+#include <cstring>
+
+#include "../../include/mxfp4.h"
 
 namespace mxfp4 {
 
@@ -86,37 +90,51 @@ struct Epilogue {
   const float* b_scale = nullptr;
 };
 
+// Scratch of the GEMM launchers, in two parts.
+//  - counters: kCounterBytes at a place of the caller's memory that does not move with the
+//    problem size (right after the status region of every workspace layout). The CTA-pair
+//    kernel's per-tile counters for a split last round live here; they must read zero when
+//    a launch starts, and every launch that completes leaves them zero. Because the block
+//    never moves, no launch can find bytes of another part of a workspace (codes, scales,
+//    partials of an earlier call with other sizes) where it expects its counters.
+//  - data: data_bytes for K-split partials (fp32), which every launch writes before it
+//    reads them, so their previous contents do not matter.
+// Either part may be absent (null): the pair kernel then splits no tile and the few-row
+// kernel sums its K splits on chip (same bits).
+constexpr size_t kCounterBytes = 4096;
+struct GemmScratch {
+  unsigned int* counters = nullptr;
+  uint8_t* data = nullptr;
+  size_t data_bytes = 0;
+};
+
 // Block-scaled GEMM y[M, N] = A[M, K] . B[N, K]^T on tcgen05. Host-validated arguments.
 // status: device word set to the timeout code if a bounded wait gives up.
 // Every kernel of the library is launched with programmatic dependent launch: it waits
 // for the previous kernel on the stream before touching memory that kernel may share.
-// scratch: scratch_bytes of device memory, zero before its first use and left zero by
-// every launch that completes (K-split partials and counters of the last round's tiles;
-// with less than gemm_scratch_bytes(M, N, K) the tiles are not split).
 // b_early: the kernel just before this launch on the stream does not write bq / bsf, so
 // the few-row kernel may start streaming them before that kernel has finished.
 cudaError_t launch_gemm(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq,
                         const uint8_t* bsf, int64_t M, int64_t N, int64_t K, void* y,
-                        const Epilogue& ep, int64_t ldy, int* status, uint8_t* scratch,
-                        size_t scratch_bytes, bool b_early, cudaStream_t stream);
+                        const Epilogue& ep, int64_t ldy, int* status, const GemmScratch& scratch,
+                        bool b_early, cudaStream_t stream);
 
-// Scratch that launch_gemm can use for this problem.
+// Bytes of the data part of the scratch that launch_gemm can use for this problem.
 size_t gemm_scratch_bytes(int64_t M, int64_t N, int64_t K);
 
 // Few-row path (M <= 128): swap-AB, K split across the CTAs of a cluster (gemm_smallm.cu).
-// scratch: the GEMM scratch; for 33..128 rows split 4 or more ways the K-split partials
-// go through it (from kSmallRedOffset on, gemm_smallm_scratch_bytes in all) when it is
-// large enough, else they are summed through distributed shared memory. Either way the
-// bits are the same.
+// For 33..128 rows split 4 or more ways the K-split partials go through the data part of
+// the scratch (gemm_smallm_scratch_bytes) when it is large enough, else they are summed
+// through distributed shared memory. Either way the bits are the same.
 cudaError_t launch_gemm_smallm(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq,
                                const uint8_t* bsf, int64_t M, int64_t N, int64_t K, void* y,
-                               const Epilogue& ep, int64_t ldy, int* status, uint8_t* scratch,
-                               size_t scratch_bytes, bool b_early, cudaStream_t stream);
+                               const Epilogue& ep, int64_t ldy, int* status,
+                               const GemmScratch& scratch, bool b_early, cudaStream_t stream);
 size_t gemm_smallm_scratch_bytes(int64_t M, int64_t N, int64_t K);
-// The few-row partials start here, past the counters at the start of the scratch that the
-// CTA-pair kernel needs zero (2 x 4 bytes per split tile, fewer than 512 tiles), so a
-// workspace shared by both kernels keeps its counters zero.
-constexpr size_t kSmallRedOffset = 4096;
+
+// Testing only (mxfp4_test_set_fault): a fault the next GEMM launches simulate, read on
+// the host when a launch is set up. MXFP4_TEST_FAULT_NONE in every product path.
+extern std::atomic<int> g_test_fault;
 
 // The whole layer for 1..8 bf16 activation rows in one launch (gemm_smallm.cu): each
 // CTA rotates (mode 0/1/2) and quantises its own K range of x into shared memory while
@@ -132,5 +150,62 @@ cudaError_t launch_linear_smallm(const void* x, int64_t ldx, int mode, const Kro
 // Scale-factor layout helpers (host side).
 inline int64_t sf_katoms(int64_t K) { return (K / 32 + 3) / 4; }
 inline int64_t sf_row_tiles(int64_t rows) { return (rows + 127) / 128; }
+
+// ---- argument checks and workspace layouts shared by the entry points (abi.cu, noalloc.cu)
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Valid [rows, K] operand description for the scale layout.
+inline bool shape_ok(int64_t rows, int64_t K) { return rows >= 0 && K >= 32 && K % 32 == 0; }
+
+// Limits of the kernels' 32-bit index arithmetic.
+inline bool within_limits(int64_t rows, int64_t K) {
+  const int64_t units = sf_row_tiles(rows) * 128 * sf_katoms(K) * 4;
+  return rows < (1ll << 31) && K < (1ll << 31) && units < (1ll << 32);
+}
+
+inline bool mode_ok(int mode) { return mode >= MXFP4_ROT_NONE && mode <= MXFP4_ROT_HADAMARD128; }
+
+// A row operand (activations, their codes and scales, the output) may be NULL when it has
+// no rows: torch and other frameworks hand out NULL for empty tensors.
+inline bool rows_ptr_ok(const void* p, int64_t rows) { return p != nullptr || rows == 0; }
+
+// Kronecker factors from host memory into the kernel-parameter form; false if one is NULL.
+inline bool kron_from_host(const float* a, const float* b, KronCoeffs* out) {
+  if (!a || !b) return false;
+  std::memcpy(out->a, a, sizeof(out->a));
+  std::memcpy(out->b, b, sizeof(out->b));
+  kron_derive(out);
+  return true;
+}
+
+// Checks of the layer's arguments (mxfp4_linear and mxfp4_linear_noalloc reject exactly
+// the same calls), and the Kronecker coefficients when mode needs them.
+mxfp4_status validate_linear(const void* x, int64_t M, int64_t K, mxfp4_rotation mode,
+                             const float* kron_a, const float* kron_b, const uint8_t* wq,
+                             const uint8_t* wsf, int64_t N, const void* y, KronCoeffs* kc);
+
+// Every workspace starts with the status region (the status word at byte 0; the NVFP4
+// layer's tensor scale and its pass's state at 64..79) and then the GEMM counter block, so
+// that block sits at the same place whatever the sizes of the call.
+constexpr size_t kStatusBytes = 256;
+constexpr size_t kHeadBytes = kStatusBytes + kCounterBytes;
+
+// Layout of the layer's workspace: [status | counters | Xq (M x K/2) | Xsf (sf_k-element
+// operand scales) | GEMM data], parts 256-byte aligned. sf_k = K for MXFP4, 2 K for NVFP4.
+struct LinearLayout {
+  size_t q_off, sf_off, g_off, total;
+};
+LinearLayout linear_layout(int64_t M, int64_t N, int64_t K, int64_t sf_k);
+
+// The GEMM scratch of a workspace laid out as above (data part: from g_off to ws_bytes).
+inline GemmScratch workspace_scratch(uint8_t* ws, size_t g_off, size_t ws_bytes) {
+  GemmScratch g;
+  g.counters = reinterpret_cast<unsigned int*>(ws + kStatusBytes);
+  g.data = ws_bytes > g_off ? ws + g_off : nullptr;
+  g.data_bytes = ws_bytes > g_off ? ws_bytes - g_off : 0;
+  return g;
+}
 
 }  // namespace mxfp4

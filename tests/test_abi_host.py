@@ -45,10 +45,10 @@ def test_status_strings():
 
 def test_workspace_sizes():
     assert mx.workspace_bytes(mx.OP_QUANTIZE, 10, 16, 64) == 0
-    assert mx.workspace_bytes(mx.OP_GEMM, 10, 16, 64) >= 256
+    assert mx.workspace_bytes(mx.OP_GEMM, 10, 16, 64) == 4352
     M, K = 3584, 3072
     ws = mx.workspace_bytes(mx.OP_LINEAR, M, 9216, K)
-    assert ws >= 256 + M * K // 2 + mx.sf_bytes(M, K)
+    assert ws >= 4352 + M * K // 2 + mx.sf_bytes(M, K)
 
 
 # Fake device addresses: validation rejects these calls on the host, so nothing is dereferenced.
@@ -183,15 +183,86 @@ def test_norm_linear_kernel_count():
 
 
 def test_gemm_scratch_for_few_rows():
-    """The few-row GEMM's K-split partials go through the workspace's scratch for 33..128
-    rows split 4 or more ways: 4096 bytes past the pair kernel's counters, then
-    units x rows x 128 columns x 4 bytes; fewer splits or rows need no scratch."""
+    """Every workspace starts with a 4352-byte head (256-byte status region, then the
+    4096-byte counter block of the CTA-pair kernel). The few-row GEMM's K-split partials
+    follow it for 33..128 rows split 4 or more ways: units x rows x 128 columns x 4 bytes;
+    fewer splits or rows need nothing past the head."""
     def gemm_ws(M, N, K):
         return mx.workspace_bytes(mx.OP_GEMM, M, N, K)
     # 4096 -> 14336 weights transposed: 32 W tiles x 8 splits = 256 units, 128 rows
     assert gemm_ws(128, 4096, 14336) == 256 + 4096 + 256 * 128 * 128 * 4
     # 100 rows, 8 W tiles x 7 splits (28 k-tiles in splits of 4)
     assert gemm_ws(100, 1024, 7168) == 256 + 4096 + 56 * 100 * 128 * 4
-    assert gemm_ws(128, 14336, 4096) == 256  # 112 W tiles x 2 splits: on-chip sum
-    assert gemm_ws(32, 4096, 14336) == 256   # 32 rows: on-chip sum
-    assert gemm_ws(1, 14336, 4096) == 256
+    assert gemm_ws(128, 14336, 4096) == 4352  # 112 W tiles x 2 splits: on-chip sum
+    assert gemm_ws(32, 4096, 14336) == 4352   # 32 rows: on-chip sum
+    assert gemm_ws(1, 14336, 4096) == 4352
+
+
+def test_gemm_scratch_for_a_split_last_round():
+    """CTA-pair plan on 74 pairs: 2560 x 2048 gives 10 x 8 = 80 tiles of 256 x 256, so the
+    last round has 6 tiles; each is split into g = min(74 / 6, 24 k-tiles / 8, 4) = 3 K
+    chunks, and chunks 1 and 2 leave one 128 x 256 fp32 partial per CTA of the pair.
+    The counters stay in the head; the partials follow it."""
+    part = 6 * (3 - 1) * 2 * 128 * 256 * 4
+    assert mx.workspace_bytes(mx.OP_GEMM, 2560, 2048, 6144) == 4352 + part
+    # the layer adds the activation codes and scales between the head and the partials
+    M, K = 2560, 6144
+    codes = M * K // 2
+    assert mx.workspace_bytes(mx.OP_LINEAR, M, 2048, K) == 4352 + codes + mx.sf_bytes(M, K) + part
+    # 4096 x 2048 x 8192: 16 x 8 = 128 tiles, 54 left for a second round: g = 1, no split
+    assert mx.workspace_bytes(mx.OP_GEMM, 4096, 2048, 8192) == 4352
+
+
+def test_kron_weight_factors_match_oracle():
+    """mxfp4_kron_weight_factors (the library's own double Gauss-Jordan) against the
+    oracle's: within 1 fp32 ulp everywhere, and identical on the seeded workload factors,
+    so weights prepared through the library and through the oracle are the same bytes."""
+    import synth
+    for seed in range(12):
+        A, B = synth.kron_factors(seed)
+        At, Bt = mx.kron_weight_factors(A, B)
+        oAt, oBt = oracle.kron_weight_factors(A, B)
+        for got, exp in ((At, oAt), (Bt, oBt)):
+            ulp = np.spacing(np.abs(exp).astype(np.float32))
+            assert np.all(np.abs(got.astype(np.float64) - exp) <= ulp)
+        # inverse and transpose: A^T At = I (A^-T = (A^T)^-1)
+        assert np.allclose(A.astype(np.float64).T @ At.astype(np.float64), np.eye(4), atol=1e-6)
+        assert np.allclose(B.astype(np.float64).T @ Bt.astype(np.float64), np.eye(8), atol=1e-6)
+    A, B = synth.kron_factors(0)
+    At, Bt = mx.kron_weight_factors(A, B)
+    oAt, oBt = oracle.kron_weight_factors(A, B)
+    assert np.array_equal(At, oAt) and np.array_equal(Bt, oBt)
+    w = synth.weight_f32(0, 64, 256, 3)
+    assert all(np.array_equal(p, q) for p, q in zip(
+        oracle.rotate_quantize(w, oracle.ROT_KRON_4x8, At, Bt),
+        oracle.rotate_quantize(w, oracle.ROT_KRON_4x8, oAt, oBt)))
+
+
+def test_kron_weight_factors_closed_forms_and_errors():
+    # a permutation with scaling: inverse known exactly (powers of two)
+    A = np.zeros((4, 4), np.float32)
+    for i, j, v in ((0, 2, 2.0), (1, 0, -0.5), (2, 3, 4.0), (3, 1, 0.25)):
+        A[i, j] = v
+    B = np.diag(np.arange(1, 9, dtype=np.float32) * 2.0)
+    At, Bt = mx.kron_weight_factors(A, B)
+    assert np.array_equal(At, np.linalg.inv(A.astype(np.float64)).T.astype(np.float32))
+    assert np.array_equal(np.diag(Bt), (1.0 / (np.arange(1, 9) * 2.0)).astype(np.float32))
+    L = mx.lib
+    buf4 = np.zeros((4, 4), np.float32)
+    buf8 = np.zeros((8, 8), np.float32)
+    eye4, eye8 = np.eye(4, dtype=np.float32), np.eye(8, dtype=np.float32)
+    assert L.mxfp4_kron_weight_factors(None, eye8.ctypes.data, buf4.ctypes.data,
+                                       buf8.ctypes.data) == mx.ERR_INVALID_ARG
+    sing = eye4.copy()
+    sing[2] = sing[1]
+    assert L.mxfp4_kron_weight_factors(sing.ctypes.data, eye8.ctypes.data, buf4.ctypes.data,
+                                       buf8.ctypes.data) == mx.ERR_INVALID_ARG
+    nan8 = eye8.copy()
+    nan8[3, 3] = np.nan
+    assert L.mxfp4_kron_weight_factors(eye4.ctypes.data, nan8.ctypes.data, buf4.ctypes.data,
+                                       buf8.ctypes.data) == mx.ERR_INVALID_ARG
+
+
+def test_test_fault_hook_arguments():
+    assert mx.lib.mxfp4_test_set_fault(7) == mx.ERR_UNSUPPORTED
+    assert mx.lib.mxfp4_test_set_fault(mx.TEST_FAULT_NONE) == mx.OK
