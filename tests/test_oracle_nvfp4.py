@@ -105,3 +105,54 @@ def test_nvfp4_scale_layout_is_the_atom_map_with_16_element_groups():
         for g in range(K // 16):
             off = (g // 4) * 512 + (r % 32) * 16 + ((r // 32) % 4) * 4 + g % 4
             assert phys[off] == s[r, g]
+
+
+def _f32_inv_sqrt32():
+    """fp32 nearest 1/sqrt(32), from 60-digit decimals (independent of the oracle)."""
+    from decimal import Decimal, getcontext
+    getcontext().prec = 60
+    return np.float32(float(Decimal(1) / Decimal(32).sqrt()))
+
+
+def _bf16(v):
+    return synth.f32_to_bf16_bits(np.asarray(v, np.float32))
+
+
+def test_tensor_scale_closed_form_unrotated():
+    """No rotation: st = amax / (6 * 448) in one fp32 rounding. With amax = 2688 * 2^k
+    (a bf16 value) st is exactly 2^k, wherever the largest magnitude sits and whatever
+    its sign; a wrong divisor (448 or 6 alone) or a signed maximum fails."""
+    for k in (-20, -3, 0, 5):
+        x = np.zeros((7, 96), np.float32)
+        x[0, :] = 0.25 * 2688 * 2.0 ** k          # smaller entries everywhere in row 0
+        x[6, 95] = -2688 * 2.0 ** k                # the largest magnitude: last element, negative
+        st = oracle.nvfp4_tensor_scale(_bf16(x), oracle.ROT_NONE)
+        assert st == np.float32(2.0 ** k)
+    # a value that is not a power of two: one fp32 division
+    x = np.zeros((2, 32), np.float32)
+    x[1, 7] = 3.0
+    st = oracle.nvfp4_tensor_scale(_bf16(x), oracle.ROT_NONE)
+    assert st == np.float32(np.float32(3.0) / np.float32(2688.0))
+
+
+def test_tensor_scale_closed_form_after_hadamard():
+    """Hadamard mode: the amax is taken after the rotation. A block c * e_0 rotates to 32
+    equal values fl(c * fl(1/sqrt(32))) (the butterfly only adds zeros), so st is that value
+    / 2688 in one fp32 rounding. A second block with a larger raw maximum b e_0 + ... but a
+    smaller rotated one shows that the maximum is not taken before the rotation."""
+    c32 = _f32_inv_sqrt32()
+    for c in (1.0, 3.0, 448.0, 1.5 * 2.0 ** -10):
+        x = np.zeros((3, 128), np.float32)
+        x[2, 64] = c                               # block 2 of row 2 is c * e_0
+        st = oracle.nvfp4_tensor_scale(_bf16(x), oracle.ROT_HADAMARD32)
+        assert st == np.float32(np.float32(np.float32(c) * c32) / np.float32(2688.0))
+    # block A = a (e_0 + e_1): rotated even entries fl(2a * c32), odd ones 0;
+    # block B = 1.5 a e_0: raw maximum 1.5 a > a, rotated maximum fl(1.5 a * c32) < 2a c32
+    a = 8.0
+    x = np.zeros((1, 64), np.float32)
+    x[0, 0] = x[0, 1] = a
+    x[0, 32] = 1.5 * a
+    st = oracle.nvfp4_tensor_scale(_bf16(x), oracle.ROT_HADAMARD32)
+    want = np.float32(np.float32(np.float32(2 * a) * c32) / np.float32(2688.0))
+    assert st == want
+    assert st != np.float32(np.float32(1.5 * a) / np.float32(2688.0))
