@@ -323,10 +323,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           tc_fence_after();
           const uint32_t sfa_s = sbase + C::OFF_SFA + stage * C::SFA_STAGE;
           const uint32_t sfb_s = sbase + C::OFF_SFB + stage * C::SFB_STAGE;
+          const uint32_t sfa_t = tmem_base + C::SFA_COL;
+          const uint32_t sfb_t = tmem_base + C::SFB_COL;
           for (uint32_t a = 0; a < C::AT; ++a) {
-            tmem_cp_32x128b_warpx4_pair(tmem_base + C::SFA_COL + 4 * a, smem_desc_sf(sfa_s + a * 512));
+            tmem_cp_32x128b_warpx4_pair(sfa_t + 4 * a, smem_desc_sf(sfa_s + a * 512));
             for (uint32_t g = 0; g < 2; ++g)
-              tmem_cp_32x128b_warpx4_pair(tmem_base + C::SFB_COL + 4 * (2 * a + g),
+              tmem_cp_32x128b_warpx4_pair(sfb_t + 4 * (2 * a + g),
                                           smem_desc_sf(sfb_s + (g * C::AT + a) * 512));
           }
           const uint32_t k_left = p.K - kt * 256u;
@@ -339,14 +341,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
               // NVFP4: one atom (4 scales of 16 per row) per K = 64 step
               mma_nvf4_pair(d_tmem, smem_desc_sw128(a_tile + k * MMA_K_BYTES),
                             smem_desc_sw128(b_tile + k * MMA_K_BYTES), idesc_nvf4(256, BN),
-                            tmem_base + C::SFA_COL + 4 * k, tmem_base + C::SFB_COL + 8 * k, acc_in);
+                            sfa_t + 4 * k, sfb_t + 8 * k, acc_in);
             } else {
               // MXFP4: an atom (4 scales of 32 per row) serves two K = 64 steps
               const uint32_t sf_id = (k & 1u) * 2u;
               mma_mxf4_pair(d_tmem, smem_desc_sw128(a_tile + k * MMA_K_BYTES),
                             smem_desc_sw128(b_tile + k * MMA_K_BYTES),
-                            idesc_mxf4(256, BN, sf_id, sf_id), tmem_base + C::SFA_COL + 4 * (k >> 1),
-                            tmem_base + C::SFB_COL + 8 * (k >> 1), acc_in);
+                            idesc_mxf4(256, BN, sf_id, sf_id), sfa_t + 4 * (k >> 1),
+                            sfb_t + 8 * (k >> 1), acc_in);
             }
           }
           mma_commit_pair_both(bar_empty + 8 * stage);  // frees the stage in both CTAs
@@ -640,11 +642,12 @@ bool make_output_map(CUtensorMap* map, void* y, uint64_t M, uint64_t N, uint64_t
 
 // Work plan of the persistent pair kernel. Whole 256 x 256 tiles go round-robin over the
 // CTA pairs; when the last round would leave pairs idle, its tiles are split into K
-// chunks (at most 4) so that it finishes in a fraction of a round. Chunk c > 0 leaves an
-// fp32 partial in the scratch; chunk 0 adds them in order. Handing a partial over costs
-// about as long as 4 k-tiles of MMAs, so a chunk gets at least 8 (2048 elements of K).
+// chunks (at most 4, at most as many as pairs per tile of that round) so that it finishes
+// in a fraction of a round. Chunk c > 0 leaves an fp32 partial in the scratch; chunk 0
+// adds them in order. Handing a partial over costs about as long as 4 k-tiles of MMAs,
+// so a split is taken only when a chunk plus that cost is clearly shorter than the tile.
 constexpr uint32_t kPlanPairs = 74;  // CTA-pair slots of a B200 (148 SMs), for scratch sizing
-constexpr uint32_t kMinChunkKt = 8;
+constexpr uint32_t kHandoffKt = 4;
 constexpr uint32_t kMaxSplit = 4;
 
 struct PairPlan {
@@ -662,9 +665,10 @@ PairPlan pair_plan(int64_t M, int64_t N, int64_t K, uint32_t pairs) {
   const uint32_t tail = pairs ? pl.tiles % pairs : 0;
   if (tail == 0) return pl;
   uint32_t g = pairs / tail;
-  if (g > k_tiles / kMinChunkKt) g = k_tiles / kMinChunkKt;
   if (g > kMaxSplit) g = kMaxSplit;
   if (g < 2) return pl;
+  // worth it: chunk + hand-off below 85 % of the whole tile
+  if (20u * ((k_tiles + g - 1) / g + kHandoffKt) >= 17u * k_tiles) return pl;
   // two counters per split tile, all inside the fixed counter block
   if ((size_t)2 * tail * sizeof(unsigned int) > kCounterBytes) return pl;
   const uint32_t kt = (k_tiles + g - 1) / g;

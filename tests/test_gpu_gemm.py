@@ -101,9 +101,10 @@ def test_gemm_few_rows_single_pair_in_last_split():
 
 
 # Large-M shapes whose last round of 256x256 tiles is split along K over several CTA
-# pairs (74 pairs on a B200; chunks of at least 8 k-tiles): tiles -> split tiles x K
-# chunks. (512,512,4096) 4 -> 4x2; (768,1024,8192) 12 -> 12x4; (700,784,6176) 12 ragged
-# tiles -> 12x3, chunks of 9, 9 and 7 k-tiles with a 32-element K tail.
+# pairs (74 pairs on a B200; up to 4 chunks, when a chunk plus the 4-k-tile hand-off is
+# under 85 % of the tile): tiles -> split tiles x K chunks. (512,512,4096) 4 -> 4x4;
+# (768,1024,8192) 12 -> 12x4; (700,784,6176) 12 ragged tiles -> 12x4, chunks of 7, 7, 7
+# and 4 k-tiles with a 32-element K tail.
 SPLIT_SHAPES = [(512, 512, 4096), (768, 1024, 8192), (700, 784, 6176)]
 
 
@@ -118,7 +119,7 @@ def test_gemm_split_last_round(M, N, K, out):
 
 
 def test_gemm_split_full_rounds_then_tail():
-    """80 tiles on 74 pairs: one round of whole tiles, then 6 tiles in 3 K chunks each.
+    """80 tiles on 74 pairs: one round of whole tiles, then 6 tiles in 4 K chunks each.
     Every element of the last 256-row band (which holds the 6 split tiles) is checked,
     plus sampled pairs elsewhere."""
     M, N, K = 2560, 2048, 6144
@@ -139,7 +140,7 @@ def test_gemm_split_repeat_and_scratch_reset():
     import mxfp4_quantized_linear_block_b200 as mx
     M, N, K = 768, 1024, 8192
     ws = mx.new_workspace(mx.workspace_bytes(mx.OP_GEMM, M, N, K))
-    assert ws.numel() > 256 + 12 * 3 * 2 * 128 * 256 * 4  # partials of 12 tiles x 3 chunks
+    assert ws.numel() >= 4352 + 12 * 3 * 2 * 128 * 256 * 4  # 12 tiles x chunks 1..3
     outs = []
     for seed in (21, 22, 21):
         aq, as_ = _operand(seed, M, K, 12)
@@ -153,7 +154,7 @@ def test_gemm_split_repeat_and_scratch_reset():
         check_gemm_values(outs[-1].astype(np.float64), ref, S, "f32", f"seed {seed}")
     assert np.array_equal(outs[0].view(np.uint32), outs[2].view(np.uint32))
     assert mx.poll_status(ws) == mx.OK
-    assert not ws[256:512].cpu().numpy().any()  # both counter arrays (2 x 12 words)
+    assert not ws[256:4352].cpu().numpy().any()  # the counter block
 
 
 def test_gemm_wide_scale_range_fp32():
@@ -234,9 +235,9 @@ def test_gemm_and_linear_with_no_rows_write_nothing():
 @pytest.mark.parametrize("out", ["bf16", "f32"])
 def test_few_rows_l2_and_on_chip_sums_agree(M, N, K, out):
     """33..128 rows split 6 to 8 ways (36 W tiles x 6, 8 x 7, 32 x 8) sum their K splits
-    through L2 when the workspace has the scratch and
-    through distributed shared memory when it has only the status word: same order of
-    additions, so the same bits; both match the oracle."""
+    through L2 when the workspace has room for the partials past its 4352-byte head,
+    and through distributed shared memory when it has only the status region: same order
+    of additions, so the same bits; both match the oracle."""
     import torch
     import mxfp4_quantized_linear_block_b200 as mx
     aq, as_ = _operand(M + N + K, M, K, 12)
@@ -245,7 +246,7 @@ def test_few_rows_l2_and_on_chip_sums_agree(M, N, K, out):
             to_dev(oracle.sf_to_physical(bs, K)), M, N, K)
     dt = torch.float32 if out == "f32" else torch.bfloat16
     full = mx.new_workspace(mx.workspace_bytes(mx.OP_GEMM, M, N, K))
-    assert full.numel() > 4096  # this size uses the L2 form
+    assert full.numel() > 4352  # this size uses the L2 form
     y_l2 = mx.gemm(*args, out_dtype=dt, ws=full)
     y_chip = mx.gemm(*args, out_dtype=dt, ws=mx.new_workspace(256))
     torch.cuda.synchronize()
@@ -257,8 +258,9 @@ def test_few_rows_l2_and_on_chip_sums_agree(M, N, K, out):
 
 
 def test_workspace_shared_by_few_row_and_pair_kernels():
-    """The few-row kernel's L2 partials leave the pair kernel's split counters (the first
-    bytes of the scratch) zero: one workspace serves a 128-row call, then a split call."""
+    """The few-row kernel's L2 partials lie past the workspace's counter block, so they
+    leave the pair kernel's split counters zero: one workspace serves a 128-row call, then
+    a split call."""
     import torch
     import mxfp4_quantized_linear_block_b200 as mx
     shapes = [(128, 4096, 14336), (512, 512, 4096)]

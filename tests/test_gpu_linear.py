@@ -54,15 +54,19 @@ def test_linear_workloads_sampled(name):
         check_gemm_values(y[mi, ni], ref, S, "bf16", f"{name}/{lin.name}")
 
 
-def test_linear_batch16_sampled():
+@pytest.mark.parametrize("j", [0, 1])
+def test_linear_batch16_sampled(j):
+    """Both layers of the batch-16 DiT MLP at full size (57344 tokens): 3072 -> 12288 and
+    12288 -> 3072, sampled outputs (first and last tiles, edge rows and columns, 8192
+    random) against the oracle's exact products of its own quantisation."""
     wl = synth.WORKLOADS["dit_b16"]
-    lin = wl.linears[0]
+    lin = wl.linears[j]
     x, wq, ws, A, B = _layer_inputs(wl, lin)
     y = _run_linear(x, wq, ws, lin.N, wl.rotation, A, B)
     xq, xs = oracle.rotate_quantize(x, wl.rotation)
-    mi, ni = _sample_pairs(lin.M, lin.N, n_random=8192, seed=3)
+    mi, ni = _sample_pairs(lin.M, lin.N, n_random=8192, seed=3 + j)
     ref, S = oracle.gemm_pairs(xq, xs, wq, ws, mi, ni)
-    check_gemm_values(y[mi, ni], ref, S, "bf16", "dit_b16/mlp_up")
+    check_gemm_values(y[mi, ni], ref, S, "bf16", f"dit_b16/{lin.name}")
 
 
 def test_linear_repeatable():

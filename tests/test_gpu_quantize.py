@@ -108,10 +108,12 @@ def test_workload_activations(name):
         quantize_parity(x, wl.rotation, A, B)
 
 
-def test_large_batch_activation_rows():
-    """The 57344 x 3072 activation of the batch-16 DiT layer: the whole tensor on
-    the GPU, every row compared (rows are independent)."""
-    lin = synth.WORKLOADS["dit_b16"].linears[0]
+@pytest.mark.parametrize("j", [0, 1])
+def test_large_batch_activation_rows(j):
+    """The two activations of the batch-16 DiT MLP, whole, on the GPU: 57344 x 3072
+    (MLP-up input) and 57344 x 12288 (MLP-down input, 1.41 GB of bf16); every code and
+    scale byte compared with the oracle's."""
+    lin = synth.WORKLOADS["dit_b16"].linears[j]
     x, _ = synth.activation_bf16(0, lin.M, lin.K, lin.outlier_frac, lin.outlier_factor, lin.x_tensor)
     quantize_parity(x, oracle.ROT_HADAMARD32)
 

@@ -6,7 +6,7 @@ right after the status region of every workspace, so a call never finds codes, s
 or partials of an earlier call with other sizes where it expects zero counters. The
 sequence below is the one that would expose such stale counters: a large call fills
 the workspace with codes, then a call whose last round is split (2560 x 6144 -> 2048:
-80 tiles of 256 x 256 on 74 CTA pairs, the last 6 tiles split in 3 K chunks) runs on
+80 tiles of 256 x 256 on 74 CTA pairs, the last 6 tiles split in 4 K chunks) runs on
 the same workspace. Its outputs, the split tiles included, are checked against the
 oracle's exact products.
 """
@@ -21,7 +21,7 @@ from test_gpu_gemm import _sample_pairs
 pytestmark = pytest.mark.gpu
 
 LARGE = (4096, 8192, 2048)  # M, K, N: 128 tiles, no split
-SPLIT = (2560, 6144, 2048)  # 80 tiles: the last 6 (rows 2304.., columns 512..) split 3 ways
+SPLIT = (2560, 6144, 2048)  # 80 tiles: the last 6 (rows 2304.., columns 512..) split 4 ways
 
 
 def _problem(seed, M, K, N):
@@ -54,7 +54,7 @@ def test_split_plan_of_the_second_call():
     """The second shape really splits its last round (host-side plan)."""
     import mxfp4_quantized_linear_block_b200 as mx
     M, K, N = SPLIT
-    part = 6 * 2 * 2 * 128 * 256 * 4
+    part = 6 * 3 * 2 * 128 * 256 * 4
     assert mx.workspace_bytes(mx.OP_GEMM, M, N, K) == 4352 + part
     M, K, N = LARGE
     assert mx.workspace_bytes(mx.OP_GEMM, M, N, K) == 4352
