@@ -56,15 +56,24 @@ PKG = "mxfp4_quantized_linear_block_b200"
 # ncu flushes L2 before every pass, so reads are cold; output still dirty in L2 when the
 # kernel ends is written back later and is not counted (hence writes < Y bytes).
 NCU_TRAFFIC = {
+    "dit_b16": {"source": f"{PKG}/csrc/gemm.cu",
+                "sha256": "1c5542388a3740ee08690759276d2c9c6fbad750f41a0da5e6a21bf9f77e1f84",
+                "bytes_per_launch": [151046000 + 1367771000, 396393000 + 332764000]},
     "dit_b1": {"source": f"{PKG}/csrc/gemm.cu",
-               "sha256": "2c72c144e76ac116fcb8b15e0baa3282996a0905199fe131db814be17a28a7d7",
-               "bytes_per_launch": [20943104 + 15270400, 26347520 + 38186496,
-                                    43526656 + 6366976]},
-    "llm_small_m1": {"source": f"{PKG}/csrc/gemm_smallm.cu",
-                     "sha256": "908f4b942417d3a74078820ae1ab25ec583f1c82cf7514773a8c7c84ee7fc6ac",
-                     "bytes_per_launch": [31283456 + 0, 31301376 + 0]},
+               "sha256": "1c5542388a3740ee08690759276d2c9c6fbad750f41a0da5e6a21bf9f77e1f84",
+               "bytes_per_launch": [20934400 + 12165888, 26183424 + 41680384,
+                                    43516160 + 5652736]},
+    "llm_small_m16": {"source": f"{PKG}/csrc/gemm_smallm.cu",
+                      "sha256": "00d1f124ffd446fabf7e60419776340596702696091ba863f76e04ae84a7db68",
+                      "bytes_per_launch": [31321856 + 0, 31442944 + 0]},
+    "llm_small_m128": {"source": f"{PKG}/csrc/gemm_smallm.cu",
+                       "sha256": "00d1f124ffd446fabf7e60419776340596702696091ba863f76e04ae84a7db68",
+                       "bytes_per_launch": [31553536 + 0, 32242432 + 96256]},
 }
 NCU_TRAFFIC_QUANTIZE = {
+    "dit_b16": {"source": f"{PKG}/csrc/quantize.cu",
+                "sha256": "46f5986c60972c28299ff9b4b5c39c6e71e8f5a6ef8b8ca9680a20c9eccb0215",
+                "bytes_per_launch": [352345000 + 70407000, 1409518000 + 354194000]},
     "dit_b1": {"source": f"{PKG}/csrc/quantize.cu",
                "sha256": "46f5986c60972c28299ff9b4b5c39c6e71e8f5a6ef8b8ca9680a20c9eccb0215",
                "bytes_per_launch": [22033664 + 0, 22033408 + 0, 88095488 + 4093952]},
