@@ -107,17 +107,13 @@ size_t mxfp4_sf_bytes(int64_t rows, int64_t K);
 int64_t mxfp4_sf_offset(int64_t row, int64_t kblock, int64_t K);
 
 /* Device workspace that `op` needs for this problem (0 if none). Every
- * workspace starts with the same 4352-byte head: a 256-byte status region (the
- * status word at byte 0) and a 4096-byte block of GEMM counters (per-tile
- * counters of a last round of output tiles split along K). The head sits at the
- * same offsets whatever the op and sizes, so one workspace can serve calls of
- * different sizes. After it come, for the layer ops, the quantised activations
- * (and the NORM_LINEAR row statistics), then the GEMM's K-split partials (sized
- * for a 148-SM B200). Allocate it zeroed: every call that completes leaves the
- * counters zero, and the other parts are written before they are read. With a
- * smaller partial area than this size, the CTA-pair GEMM does not split its
- * last round and the few-row GEMM (M <= 128) sums its K splits on chip instead
- * (slower; the few-row sums are the same bits). */
+ * workspace starts with the same 256-byte status region (the status word at
+ * byte 0), so one workspace can serve calls of different sizes. After it come,
+ * for the layer ops, the quantised activations (and the NORM_LINEAR row
+ * statistics), then, for 33..128 activation rows, the few-row GEMM's K-split
+ * partials (sized for a 148-SM B200). Allocate it zeroed; every other part is
+ * written before it is read. With a smaller partial area than this size the
+ * few-row GEMM sums its K splits on chip instead (slower, the same bits). */
 size_t mxfp4_workspace_bytes(int op, int64_t M, int64_t N, int64_t K);
 
 /* Static description of a status code. Never NULL. */
@@ -174,12 +170,10 @@ mxfp4_status mxfp4_rotate_quantize(const void* x, mxfp4_dtype xdt, int64_t rows,
  * and ldy * elemsize a multiple of 16; aq, bq, asf, bsf 16-byte aligned.
  * ws: at least 256 bytes, zeroed when allocated; its first 16 bytes are the
  * device status word (see mxfp4_poll_status). mxfp4_workspace_bytes(
- * MXFP4_OP_GEMM, M, N, K) bytes give the fastest form; with less (fewer than
- * the 4352-byte head, too little room for the partials, or a GPU whose SM
- * count needs more), the last round of tiles is not split along K and the
- * few-row kernel sums its K splits on chip (slower; the result still meets
- * the stated tolerance, and the few-row sums are the same bits). Fewer than
- * 256 bytes -> MXFP4_ERR_WORKSPACE.
+ * MXFP4_OP_GEMM, M, N, K) bytes give the fastest form; with less (too little
+ * room for the few-row K-split partials, or a GPU whose SM count needs more)
+ * the few-row kernel sums its K splits on chip (slower, the same bits). Fewer
+ * than 256 bytes -> MXFP4_ERR_WORKSPACE.
  * ("AMD Quark...", opening section: MXFP4 GEMM with no dequantisation;
  * "Bridging the Gap...", "GPU Kernel Ondersteuning (QuTLASS)".)
  */
@@ -372,20 +366,19 @@ mxfp4_status mxfp4_nvfp4_linear(const void* x, int64_t M, int64_t K, mxfp4_rotat
  * that loads the library keeps until the process exits. Nothing is allocated
  * per call (no cudaMalloc / cudaFree, no allocating library routine).
  *  - Arguments are checked exactly as mxfp4_linear checks them.
- *  - Limit: 4352 + round256(M * K / 2) + round256(mxfp4_sf_bytes(M, K)) must
+ *  - Limit: 256 + round256(M * K / 2) + round256(mxfp4_sf_bytes(M, K)) must
  *    not exceed the array (about 62 million activation elements); larger
  *    problems return MXFP4_ERR_WORKSPACE and launch nothing. The rest of the
- *    array holds the GEMM's K-split partials when they fit (else the GEMM
- *    runs without them: slower, same tolerance).
+ *    array holds the few-row GEMM's K-split partials when they fit (else it
+ *    sums them on chip: slower, the same bits).
  *  - status: optional DEVICE pointer to a caller-owned, 4-byte aligned int
  *    that the caller zeroes; a bounded-wait timeout sets it to
  *    MXFP4_ERR_TIMEOUT. With NULL the library keeps a status word in its array
  *    (the caller cannot read it).
- *  - Each call first clears the array's status region and GEMM counter block
- *    (one cudaMemsetAsync of 4352 bytes on `stream`), so nothing that an
- *    earlier call left there -- a timed-out call's counters included -- is
- *    seen; every other part it reads it writes first. A call after a timeout
- *    needs no reset.
+ *  - Each call first clears the array's status region (one cudaMemsetAsync
+ *    of 256 bytes on `stream`), so a status that an earlier call left there
+ *    is not seen; every other part it reads it writes first. A call after a
+ *    timeout needs no reset.
  *  - The first call on each device looks up the array's device address
  *    (cudaGetSymbolAddress) with that device current; make that first call
  *    before any stream capture.
@@ -402,15 +395,17 @@ mxfp4_status mxfp4_linear_noalloc(const void* x, int64_t M, int64_t K, mxfp4_rot
 
 /*
  * Testing only: the faults that mxfp4_test_set_fault can make the GEMM simulate.
- * MXFP4_TEST_FAULT_SKIP_SPLIT_PUBLISH: when the CTA-pair GEMM (M > 128) splits the
- * tiles of its last round along K, chunk 1 of each split tile stores its partial
- * but never publishes it; the chunk that owns the tile waits for it at most 1 ms
- * (instead of 2 s), records MXFP4_ERR_TIMEOUT in the status word and finishes the
- * tile without it (those output tiles are wrong). The kernel returns normally.
+ * MXFP4_TEST_FAULT_WITHHOLD_ACCUMULATOR: in the CTA-pair GEMM (M > 128), the first
+ * CTA pair never signals that its first accumulator is complete. Its epilogue
+ * waits for that signal at most 1 ms (instead of 2 s), records MXFP4_ERR_TIMEOUT
+ * in the status word and stops; the pair's other roles see the stop at their
+ * next bounded wait, drain their copies, release tensor memory and return, so
+ * the kernel ends normally. The tiles of that pair are not written; every other
+ * pair's tiles are right.
  */
 typedef enum {
   MXFP4_TEST_FAULT_NONE = 0,
-  MXFP4_TEST_FAULT_SKIP_SPLIT_PUBLISH = 1
+  MXFP4_TEST_FAULT_WITHHOLD_ACCUMULATOR = 1
 } mxfp4_test_fault;
 
 /*
@@ -418,9 +413,8 @@ typedef enum {
  * (MXFP4_TEST_FAULT_NONE restores normal operation, the state at load time).
  * It lets a test drive a bounded device wait to its limit -- the path that
  * reports MXFP4_ERR_TIMEOUT -- with no GPU fault and no hang. Process-wide
- * and read when a launch is set up; never call it in production code. After
- * a simulated fault, zero the workspace before its next use (the counter
- * block may be left set). Unknown values -> MXFP4_ERR_UNSUPPORTED.
+ * and read when a launch is set up; never call it in production code.
+ * Unknown values -> MXFP4_ERR_UNSUPPORTED.
  */
 mxfp4_status mxfp4_test_set_fault(int fault);
 
@@ -431,8 +425,8 @@ mxfp4_status mxfp4_test_set_fault(int fault);
  * tensor memory and returned; its output is incomplete). The word is sticky:
  * kernels only ever set it, this call clears it. Zero the whole workspace once
  * when it is allocated, and again after a timeout (a kernel that stopped early
- * can leave GEMM counters, or the NVFP4 tensor-scale pass's words, set).
- * mxfp4_linear_noalloc needs no such reset: it clears its own at each call.
+ * can leave the NVFP4 tensor-scale pass's words set). mxfp4_linear_noalloc
+ * needs no such reset: it clears its own at each call.
  */
 mxfp4_status mxfp4_poll_status(void* ws, mxfp4_status* out);
 

@@ -24,7 +24,7 @@ ROT_NONE, ROT_HADAMARD32, ROT_KRON_4x8, ROT_HADAMARD64, ROT_HADAMARD128 = 0, 1, 
 DT_BF16, DT_F32 = 0, 1
 OP_QUANTIZE, OP_GEMM, OP_LINEAR, OP_NVFP4_LINEAR, OP_NORM_LINEAR = 0, 1, 2, 3, 4
 NORM_LAYER, NORM_RMS = 0, 1
-TEST_FAULT_NONE, TEST_FAULT_SKIP_SPLIT_PUBLISH = 0, 1
+TEST_FAULT_NONE, TEST_FAULT_WITHHOLD_ACCUMULATOR = 0, 1
 
 EXPORTS = (
     "mxfp4_sf_bytes", "mxfp4_sf_offset", "mxfp4_workspace_bytes", "mxfp4_status_string",

@@ -43,8 +43,7 @@ mxfp4_status validate_gemm(const uint8_t* aq, const uint8_t* asf, const uint8_t*
   return MXFP4_OK;
 }
 
-// The GEMM scratch of a GEMM-only workspace: [status | counters | data]. A workspace of
-// fewer than kHeadBytes has no counter block (the last round is then not split).
+// The GEMM scratch of a GEMM-only workspace: [status | data].
 GemmScratch gemm_workspace_scratch(void* ws, size_t ws_bytes) {
   if (ws_bytes < kHeadBytes) return GemmScratch{};
   return workspace_scratch(static_cast<uint8_t*>(ws), kHeadBytes, ws_bytes);
@@ -55,7 +54,7 @@ GemmScratch gemm_workspace_scratch(void* ws, size_t ws_bytes) {
 // counter at 72 and 76.
 constexpr size_t kScaleOff = 64;
 
-// Workspace of mxfp4_norm_linear: [status | counters | Xq | Xsf | row statistics (M x 8
+// Workspace of mxfp4_norm_linear: [status | Xq | Xsf | row statistics (M x 8
 // bytes) | GEMM data].
 struct NormWorkspace {
   size_t q_off, sf_off, st_off, g_off, total;
@@ -214,7 +213,7 @@ mxfp4_status mxfp4_gemm(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq
   if (st != MXFP4_OK) return st;
   if (!ws) return MXFP4_ERR_INVALID_ARG;
   if (!aligned16(ws)) return MXFP4_ERR_ALIGN;
-  if (ws_bytes < kStatusBytes) return MXFP4_ERR_WORKSPACE;  // scratch: optional, see header
+  if (ws_bytes < kHeadBytes) return MXFP4_ERR_WORKSPACE;  // scratch: optional, see header
   if (M == 0) return MXFP4_OK;
   // The caller's previous kernel may have written bq / bsf: no early weight loads.
   Epilogue ep;
@@ -232,7 +231,7 @@ mxfp4_status mxfp4_gemm_bias(const uint8_t* aq, const uint8_t* asf, const uint8_
   if (st != MXFP4_OK) return st;
   if (!ws || !bias) return MXFP4_ERR_INVALID_ARG;
   if (!aligned16(ws) || !aligned16(bias)) return MXFP4_ERR_ALIGN;
-  if (ws_bytes < kStatusBytes) return MXFP4_ERR_WORKSPACE;  // scratch: optional, see header
+  if (ws_bytes < kHeadBytes) return MXFP4_ERR_WORKSPACE;  // scratch: optional, see header
   if (M == 0) return MXFP4_OK;
   Epilogue ep;
   ep.out = ydt == MXFP4_DT_F32 ? kOutF32 : kOutBf16;
@@ -259,7 +258,7 @@ mxfp4_status mxfp4_gemm_quantize(const uint8_t* aq, const uint8_t* asf, const ui
   if (!aligned16(aq) || !aligned16(asf) || !aligned16(bq) || !aligned16(bsf) || !aligned16(yq) ||
       !aligned16(ysf) || !aligned16(ws) || (bias && !aligned16(bias)))
     return MXFP4_ERR_ALIGN;
-  if (ws_bytes < kStatusBytes) return MXFP4_ERR_WORKSPACE;  // scratch: optional, see header
+  if (ws_bytes < kHeadBytes) return MXFP4_ERR_WORKSPACE;  // scratch: optional, see header
   Epilogue ep;
   ep.out = kOutMxfp4;
   ep.bias = bias;
@@ -419,7 +418,7 @@ mxfp4_status mxfp4_nvfp4_gemm(const uint8_t* aq, const uint8_t* asf, const float
   if (!aligned16(ws) || (reinterpret_cast<uintptr_t>(a_scale) & 3u) ||
       (reinterpret_cast<uintptr_t>(b_scale) & 3u))
     return MXFP4_ERR_ALIGN;
-  if (ws_bytes < kStatusBytes) return MXFP4_ERR_WORKSPACE;  // scratch: optional, see header
+  if (ws_bytes < kHeadBytes) return MXFP4_ERR_WORKSPACE;  // scratch: optional, see header
   if (M == 0) return MXFP4_OK;
   Epilogue ep;
   ep.out = ydt == MXFP4_DT_F32 ? kOutF32 : kOutBf16;
@@ -482,7 +481,7 @@ mxfp4_status mxfp4_kron_weight_factors(const float* A, const float* B, float* At
 }
 
 mxfp4_status mxfp4_test_set_fault(int fault) {
-  if (fault != MXFP4_TEST_FAULT_NONE && fault != MXFP4_TEST_FAULT_SKIP_SPLIT_PUBLISH)
+  if (fault != MXFP4_TEST_FAULT_NONE && fault != MXFP4_TEST_FAULT_WITHHOLD_ACCUMULATOR)
     return MXFP4_ERR_UNSUPPORTED;
   g_test_fault.store(fault);
   return MXFP4_OK;

@@ -9,7 +9,8 @@
 // FP4 Quantization", "GPU Kernel Ondersteuning (QuTLASS)").
 //
 // Structure: persistent clusters of two CTAs (one CTA per SM, 320 threads each)
-// share 256 x 256 output tiles through tcgen05.mma.cta_group::2:
+// share 256 x 256 output tiles through tcgen05.mma.cta_group::2 (a last round that
+// would leave half of the pairs idle runs as 256 x 128 units instead):
 //   warp 0      TMA producer: this CTA's 128 rows of A and 128 rows of B per
 //               stage (128-byte swizzled tiles) and the scale atoms, into a
 //               ring of shared-memory stages;
@@ -60,12 +61,9 @@ struct Params {
   uint32_t k_atoms;        // scale atoms per 128-row group: ceil(K / 128), NVFP4 ceil(K / 64)
   uint32_t b_row_tiles;    // ceil(N / 128)
   uint64_t ldy;            // elements
-  // Work units: tiles [0, full_units) whole; each later tile split into split_g K chunks
-  // of kt_per_chunk k-tiles (units full_units + t * split_g + c). Chunk 0 owns the tile.
-  uint32_t full_units, units, split_g, kt_per_chunk;
-  unsigned int* flags;     // [2 * split tiles] in the fixed counter block: partials stored,
-                           // owner warps done
-  float* part;             // [split tile][chunk 1..g-1][CTA rank] x 128 x 256 fp32
+  // Work units: tiles [0, full_units) whole (256 x 256); each later tile is two units of
+  // 256 x 128 (unit full_units + 2 t + h: column half h of tile full_units + t).
+  uint32_t full_units, units;
   const float* bias;       // [N] or null
   uint8_t* yq;             // MXFP4 output: codes [M, ldy bytes per row]
   uint8_t* ysf;            // MXFP4 output: scales, tensor-core layout of an [M, N] operand
@@ -73,66 +71,29 @@ struct Params {
   uint32_t rows_pad, n_katoms_y;
   const float* a_scale;    // NVFP4: tensor scales of A and B (device fp32)
   const float* b_scale;
-  uint64_t count_wait_ns;  // bound of the owner's wait for the other chunks' partials
-  uint32_t skip_publish;   // testing only: chunk that stores its partial but never
-                           // publishes it (0: none, every chunk publishes)
+  uint64_t tfull_wait_ns;  // bound of the epilogue's wait for an accumulator
+  uint32_t skip_commit;    // testing only: 1 = pair 0 never signals its first accumulator
 };
 
 struct Unit {
-  uint32_t tile, kt0, kt1, chunk;
-  bool split;
+  uint32_t tile;
+  uint32_t half;  // 128-column unit: which half of the tile's 256 columns
+  bool n128;      // a 256 x 128 unit (the last round's tiles, two units each)
 };
 
 __device__ __forceinline__ Unit unit_at(uint32_t u, const Params& p) {
   Unit w;
   if (u < p.full_units) {
     w.tile = u;
-    w.kt0 = 0;
-    w.kt1 = p.k_tiles;
-    w.chunk = 0;
-    w.split = false;
+    w.half = 0;
+    w.n128 = false;
   } else {
     const uint32_t v = u - p.full_units;
-    const uint32_t t = v / p.split_g;
-    w.chunk = v - t * p.split_g;
-    w.tile = p.full_units + t;
-    w.kt0 = w.chunk * p.kt_per_chunk;
-    w.kt1 = w.kt0 + p.kt_per_chunk < p.k_tiles ? w.kt0 + p.kt_per_chunk : p.k_tiles;
-    w.split = true;
+    w.tile = p.full_units + (v >> 1);
+    w.half = v & 1u;
+    w.n128 = true;
   }
   return w;
-}
-
-// Partial of K chunk c (>= 1) of split tile t for this CTA's 128 rows, at the slot of
-// (32-row quarter `quad`, 4-column group g4, lane): lane-fastest, so a warp's 16-byte
-// accesses for one column group cover 512 consecutive bytes.
-__device__ __forceinline__ float* part_at(const Params& p, uint32_t t, uint32_t c, uint32_t rank,
-                                          uint32_t quad, uint32_t g4, uint32_t lane) {
-  const uint64_t base = ((uint64_t)(t * (p.split_g - 1) + (c - 1)) * 2 + rank) * (128u * 256u);
-  return p.part + base + ((uint64_t)(quad * 64u + g4) * 32u + lane) * 4u;
-}
-
-__device__ __forceinline__ uint32_t ld_acquire_u32(const unsigned int* ptr) {
-  uint32_t v;
-  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ptr) : "memory");
-  return v;
-}
-
-__device__ __forceinline__ uint64_t global_ns() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-
-// Bounded wait until *ptr >= target (stores of the other chunks of a split tile).
-__device__ __forceinline__ bool wait_count(const unsigned int* ptr, uint32_t target,
-                                           uint64_t limit_ns) {
-  const uint64_t t0 = global_ns();
-  while (ld_acquire_u32(ptr) < target) {
-    if (global_ns() - t0 > limit_ns) return false;
-    __nanosleep(100);
-  }
-  return true;
 }
 
 __device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
@@ -195,6 +156,7 @@ template <uint32_t STAGES, int OUT, bool NV>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     mxf4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a,
                           const __grid_constant__ CUtensorMap tmap_b,
+                          const __grid_constant__ CUtensorMap tmap_b64,
                           const __grid_constant__ CUtensorMap tmap_sfa,
                           const __grid_constant__ CUtensorMap tmap_sfb,
                           const __grid_constant__ CUtensorMap tmap_y, const Params p,
@@ -234,6 +196,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     fence_mbar_init();
     prefetch_tmap(&tmap_a);
     prefetch_tmap(&tmap_b);
+    prefetch_tmap(&tmap_b64);
     prefetch_tmap(&tmap_sfa);
     prefetch_tmap(&tmap_sfb);
     if constexpr (OUT != kOutMxfp4) prefetch_tmap(&tmap_y);  // unused (zero) map otherwise
@@ -262,18 +225,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const Unit w = unit_at(u, p);
         const uint32_t mt = w.tile / p.n_tiles, nt = w.tile % p.n_tiles;  // 256-row m tiles
         const int32_t m_cta = (int32_t)(mt * 256u + rank * 128u);
-        const int32_t n_cta = (int32_t)(nt * BN + rank * 128u);
-        for (uint32_t kt = w.kt0; kt < w.kt1; ++kt) {
+        // B rows of this CTA: 128 of the tile's 256, or 64 of a 128-column unit's 128
+        const int32_t n_cta =
+            (int32_t)(nt * BN + (w.n128 ? w.half * 128u + rank * 64u : rank * 128u));
+        const uint32_t tx = 2u * (w.n128 ? C::STAGE_TX - C::B_STAGE / 2u : C::STAGE_TX);
+        for (uint32_t kt = 0; kt < p.k_tiles; ++kt) {
           if (!mbar_wait_bounded(bar_empty + 8 * stage, phase ^ 1u, abort_flag, kWaitLimitNs)) {
             ok = false;
             break;
           }
-          if (rank == 0) mbar_arrive_expect_tx(bar_full + 8 * stage, 2u * C::STAGE_TX);
+          if (rank == 0) mbar_arrive_expect_tx(bar_full + 8 * stage, tx);
           const uint32_t fb = full_at_leader + 8 * stage;
           tma_load_2d_pair(sbase + C::OFF_A + stage * C::A_STAGE, &tmap_a, fb,
                            (int32_t)(kt * BK_BYTES), m_cta);
-          tma_load_2d_pair(sbase + C::OFF_B + stage * C::B_STAGE, &tmap_b, fb,
-                           (int32_t)(kt * BK_BYTES), n_cta);
+          tma_load_2d_pair(sbase + C::OFF_B + stage * C::B_STAGE, w.n128 ? &tmap_b64 : &tmap_b,
+                           fb, (int32_t)(kt * BK_BYTES), n_cta);
           // scale atoms: A's are rows of a [row_tiles * k_atoms, 128-word] view, B's a
           // [row_tiles, k_atoms, 128-word] view (both 128-row groups of the tile)
           tma_load_2d_pair(sbase + C::OFF_SFA + stage * C::SFA_STAGE, &tmap_sfa, fb, 0,
@@ -315,7 +281,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (acc_phase ? C::ACC1_COL : 0u);
-        for (uint32_t kt = w.kt0; kt < w.kt1; ++kt) {
+        // A 128-column unit: N = 128, and its B rows are the scale group of its half.
+        const uint32_t n_mma = w.n128 ? 128u : BN;
+        const uint32_t sfb_half = w.n128 ? 4u * w.half : 0u;
+        for (uint32_t kt = 0; kt < p.k_tiles; ++kt) {
           if (!mbar_wait_bounded(bar_full + 8 * stage, phase, abort_flag, kWaitLimitNs)) {
             ok = false;
             break;
@@ -336,19 +305,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           const uint32_t a_tile = sbase + C::OFF_A + stage * C::A_STAGE;
           const uint32_t b_tile = sbase + C::OFF_B + stage * C::B_STAGE;
           for (uint32_t k = 0; k < steps; ++k) {
-            const uint32_t acc_in = (kt != w.kt0 || k != 0u) ? 1u : 0u;
+            const uint32_t acc_in = (kt != 0u || k != 0u) ? 1u : 0u;
             if constexpr (NV) {
               // NVFP4: one atom (4 scales of 16 per row) per K = 64 step
               mma_nvf4_pair(d_tmem, smem_desc_sw128(a_tile + k * MMA_K_BYTES),
-                            smem_desc_sw128(b_tile + k * MMA_K_BYTES), idesc_nvf4(256, BN),
-                            sfa_t + 4 * k, sfb_t + 8 * k, acc_in);
+                            smem_desc_sw128(b_tile + k * MMA_K_BYTES), idesc_nvf4(256, n_mma),
+                            sfa_t + 4 * k, sfb_t + 8 * k + sfb_half, acc_in);
             } else {
               // MXFP4: an atom (4 scales of 32 per row) serves two K = 64 steps
               const uint32_t sf_id = (k & 1u) * 2u;
               mma_mxf4_pair(d_tmem, smem_desc_sw128(a_tile + k * MMA_K_BYTES),
                             smem_desc_sw128(b_tile + k * MMA_K_BYTES),
-                            idesc_mxf4(256, BN, sf_id, sf_id), sfa_t + 4 * (k >> 1),
-                            sfb_t + 8 * (k >> 1), acc_in);
+                            idesc_mxf4(256, n_mma, sf_id, sf_id), sfa_t + 4 * (k >> 1),
+                            sfb_t + 8 * (k >> 1) + sfb_half, acc_in);
             }
           }
           mma_commit_pair_both(bar_empty + 8 * stage);  // frees the stage in both CTAs
@@ -358,7 +327,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           }
         }
         if (!ok) break;
-        mma_commit_pair_both(bar_tfull);  // both halves of the accumulator are ready
+        // both halves of the accumulator are ready (the test hook withholds pair 0's first)
+        if (!(p.skip_commit && u == 0u)) mma_commit_pair_both(bar_tfull);
         acc_phase ^= 1u;
       }
       if (!ok) record_timeout(p.status);
@@ -370,6 +340,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // Epilogue. Warp w owns TMEM lanes 32 * (w % 4) .. +31 and two of the tile's
     // four 64-column chunks; the half-0 warps take the chunk the other
     // accumulator overlaps first and release the accumulator after reading it.
+    // A 128-column unit has two chunks, both drained by the half-0 warps.
     // Each chunk goes TMEM -> registers -> bf16/fp32 -> the warp's swizzled
     // shared buffer -> TMA store (which clips rows >= M and columns >= N).
     const uint32_t quad = warp & 3u;
@@ -386,25 +357,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     for (uint32_t u = pair; u < p.units; u += num_pairs) {
       const Unit w = unit_at(u, p);
       const uint32_t mt = w.tile / p.n_tiles, nt = w.tile % p.n_tiles;
-      const uint32_t st = w.tile - p.full_units;  // index among split tiles (if split)
-      const bool ok = mbar_wait_bounded(bar_tfull, acc_phase, abort_flag, kWaitLimitNs);
+      if (w.n128 && half == 1) {  // the half-0 warps drain a 128-column unit
+        acc_phase ^= 1u;
+        continue;
+      }
+      const bool ok = mbar_wait_bounded(bar_tfull, acc_phase, abort_flag, p.tfull_wait_ns);
       if (!__all_sync(0xffffffffu, ok)) {  // leave together so .aligned ops stay convergent
         if (lane == 0) record_timeout(p.status);
         break;
       }
       tc_fence_after();
-      // Split tile, chunk 0: the other chunks' partials must be stored before they are added.
-      if (w.split && w.chunk == 0) {
-        bool got = true;
-        if (lane == 0)
-          got = wait_count(p.flags + st, (p.split_g - 1) * 2u * kEpiWarps, p.count_wait_ns);
-        got = __shfl_sync(0xffffffffu, got ? 1 : 0, 0) != 0;
-        if (!got && lane == 0) record_timeout(p.status);
-      }
       const uint32_t acc_col = acc_phase ? C::ACC1_COL : 0u;
       const uint32_t shared_chunk = acc_phase ? 0u : 3u;
+      const uint32_t col_tile = nt * BN + (w.n128 ? w.half * 128u : 0u);  // first column
       uint32_t ch[2];
-      if (half == 0) {
+      if (w.n128) {
+        ch[0] = 0;
+        ch[1] = 1;
+      } else if (half == 0) {
         ch[0] = shared_chunk;
         ch[1] = acc_phase ? 1u : 2u;
       } else {
@@ -425,34 +395,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           __syncwarp();
           if (lane == 0) mbar_arrive_cluster(tempty_at_leader);
         }
-        if (w.split && w.chunk != 0) {
-          // Another CTA pair owns this tile: store the fp32 partial for it.
-          float* dst = part_at(p, st, w.chunk, rank, quad, ch[r] * 16u, lane);
-#pragma unroll
-          for (uint32_t j = 0; j < 16; ++j) {
-            const uint32_t* src = &v[j / 8][(j % 8) * 4];
-            *reinterpret_cast<float4*>(dst + j * 128u) =
-                make_float4(__uint_as_float(src[0]), __uint_as_float(src[1]),
-                            __uint_as_float(src[2]), __uint_as_float(src[3]));
-          }
-          continue;
-        }
-        if (w.split) {
-          // Owner: add chunks 1, 2, ... in that order to its own chunk-0 sum.
-          for (uint32_t c = 1; c < p.split_g; ++c) {
-            const float* srcp = part_at(p, st, c, rank, quad, ch[r] * 16u, lane);
-#pragma unroll
-            for (uint32_t j = 0; j < 16; ++j) {
-              const float4 q = __ldcg(reinterpret_cast<const float4*>(srcp + j * 128u));
-              uint32_t* d = &v[j / 8][(j % 8) * 4];
-              d[0] = __float_as_uint(__uint_as_float(d[0]) + q.x);
-              d[1] = __float_as_uint(__uint_as_float(d[1]) + q.y);
-              d[2] = __float_as_uint(__uint_as_float(d[2]) + q.z);
-              d[3] = __float_as_uint(__uint_as_float(d[3]) + q.w);
-            }
-          }
-        }
-        const uint32_t col_base = nt * BN + ch[r] * 64u;  // first column of this chunk
+        const uint32_t col_base = col_tile + ch[r] * 64u;  // first column of this chunk
         if constexpr (NV) {  // the two tensor scales, once, on the full sum
 #pragma unroll
           for (uint32_t h = 0; h < 2; ++h)
@@ -497,7 +440,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         } else {
 #pragma unroll
           for (uint32_t c = 0; c < 64 / CCOLS; ++c) {
-            const int32_t col0 = (int32_t)(nt * BN + ch[r] * 64u + c * CCOLS);
+            const int32_t col0 = (int32_t)(col_base + c * CCOLS);
             if (lane == 0) bulk_wait_read_all();  // the buffer's previous store has read it
             __syncwarp();
 #pragma unroll
@@ -524,33 +467,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
       }
       if constexpr (OUT == kOutMxfp4) {
-        if (!(w.split && w.chunk != 0)) {
-          // The warp's two chunks are 128 aligned columns: one word of a scale atom per row.
-          const uint32_t row = (uint32_t)row0 + lane;
-          const uint32_t ka = nt * 2u + (ch[0] >= 2u ? 1u : 0u);
-          if (row < p.rows_pad && ka < p.n_katoms_y)
-            *reinterpret_cast<uint32_t*>(p.ysf + ((uint64_t)(row >> 7) * p.n_katoms_y + ka) * 512u +
-                                         (row & 31u) * 16u + ((row >> 5) & 3u) * 4u) = sfw;
-        }
-      }
-      if (w.split) {
-        if (w.chunk != 0) {
-          // Publish this warp's part of the partial to the owner.
-          __threadfence();
-          __syncwarp();
-          if (lane == 0 && w.chunk != p.skip_publish) atomicAdd(p.flags + st, 1u);
-        } else {
-          // Owner warps done reading: the last one clears both counters for the next launch.
-          __syncwarp();
-          if (lane == 0) {
-            const uint32_t n_split = (p.units - p.full_units) / p.split_g;
-            unsigned int* done = p.flags + n_split + st;
-            if (atomicAdd(done, 1u) == 2u * kEpiWarps - 1u) {
-              atomicExch(p.flags + st, 0u);
-              atomicExch(done, 0u);
-            }
-          }
-        }
+        // The warp's two chunks are 128 aligned columns: one word of a scale atom per row.
+        const uint32_t row = (uint32_t)row0 + lane;
+        const uint32_t ka = (col_tile + (ch[0] >= 2u ? 128u : 0u)) / 128u;
+        if (row < p.rows_pad && ka < p.n_katoms_y)
+          *reinterpret_cast<uint32_t*>(p.ysf + ((uint64_t)(row >> 7) * p.n_katoms_y + ka) * 512u +
+                                       (row & 31u) * 16u + ((row >> 5) & 3u) * 4u) = sfw;
       }
       acc_phase ^= 1u;
     }
@@ -641,59 +563,38 @@ bool make_output_map(CUtensorMap* map, void* y, uint64_t M, uint64_t N, uint64_t
 }
 
 // Work plan of the persistent pair kernel. Whole 256 x 256 tiles go round-robin over the
-// CTA pairs; when the last round would leave pairs idle, its tiles are split into K
-// chunks (at most 4, at most as many as pairs per tile of that round) so that it finishes
-// in a fraction of a round. Chunk c > 0 leaves an fp32 partial in the scratch; chunk 0
-// adds them in order. Handing a partial over costs about as long as 4 k-tiles of MMAs,
-// so a split is taken only when a chunk plus that cost is clearly shorter than the tile.
-constexpr uint32_t kPlanPairs = 74;  // CTA-pair slots of a B200 (148 SMs), for scratch sizing
-constexpr uint32_t kHandoffKt = 4;
-constexpr uint32_t kMaxSplit = 4;
-
+// CTA pairs. When the last round would leave at least half of the pairs idle, each of its
+// tiles becomes two 256 x 128 units (N = 128 MMAs on the tile's column halves), so that
+// round takes about half as long and needs no exchange between pairs. (The earlier form
+// split those tiles along K and added fp32 partials through L2: at 3584 x 3072 -> 3072
+// the hand-over took about 8 us against 1.3 us of MMAs.)
 struct PairPlan {
-  uint32_t tiles, full_units, units, g, kt_per_chunk, n_split;
-  size_t scratch_bytes;  // fp32 partials (the data part of the scratch)
+  uint32_t tiles, full_units, units;
 };
 
-PairPlan pair_plan(int64_t M, int64_t N, int64_t K, uint32_t pairs) {
+PairPlan pair_plan(int64_t M, int64_t N, uint32_t pairs) {
   PairPlan pl{};
-  const uint32_t k_tiles = (uint32_t)((K + 255) / 256);
   pl.tiles = (uint32_t)(((M + 255) / 256) * ((N + 255) / 256));
   pl.full_units = pl.units = pl.tiles;
-  pl.g = 1;
-  pl.kt_per_chunk = k_tiles;
   const uint32_t tail = pairs ? pl.tiles % pairs : 0;
-  if (tail == 0) return pl;
-  uint32_t g = pairs / tail;
-  if (g > kMaxSplit) g = kMaxSplit;
-  if (g < 2) return pl;
-  // worth it: chunk + hand-off below 85 % of the whole tile
-  if (20u * ((k_tiles + g - 1) / g + kHandoffKt) >= 17u * k_tiles) return pl;
-  // two counters per split tile, all inside the fixed counter block
-  if ((size_t)2 * tail * sizeof(unsigned int) > kCounterBytes) return pl;
-  const uint32_t kt = (k_tiles + g - 1) / g;
-  g = (k_tiles + kt - 1) / kt;
-  if (g < 2) return pl;
-  pl.g = g;
-  pl.kt_per_chunk = kt;
-  pl.n_split = tail;
-  pl.full_units = pl.tiles - tail;
-  pl.units = pl.full_units + tail * g;
-  pl.scratch_bytes = (size_t)tail * (g - 1) * 2 * 128 * 256 * sizeof(float);
+  if (tail != 0 && 2u * tail <= pairs) {
+    pl.full_units = pl.tiles - tail;
+    pl.units = pl.full_units + 2u * tail;
+  }
   return pl;
 }
 
 template <uint32_t STAGES, int OUT, bool NV>
 cudaError_t launch_pair(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq,
                         const uint8_t* bsf, int64_t M, int64_t N, int64_t K, void* y,
-                        const Epilogue& ep, int64_t ldy, int* status,
-                        const GemmScratch& scratch, cudaStream_t stream) {
+                        const Epilogue& ep, int64_t ldy, int* status, cudaStream_t stream) {
   using C = PairConfig<STAGES, NV>;
   // scale atoms per 128-row group: one per 4 scales, i.e. per 128 (MXFP4) or 64 (NVFP4) K
   const uint64_t k_atoms = (uint64_t)sf_katoms(NV ? 2 * K : K);
-  CUtensorMap ta, tb, tsa, tsb, ty{};
+  CUtensorMap ta, tb, tb64, tsa, tsb, ty{};
   if (!make_operand_map(&ta, aq, (uint64_t)M, (uint64_t)(K / 2), 128) ||
       !make_operand_map(&tb, bq, (uint64_t)N, (uint64_t)(K / 2), 128) ||
+      !make_operand_map(&tb64, bq, (uint64_t)N, (uint64_t)(K / 2), 64) ||
       !make_scale_map(&tsa, asf, (uint64_t)sf_row_tiles(M), k_atoms, false, C::AT) ||
       !make_scale_map(&tsb, bsf, (uint64_t)sf_row_tiles(N), k_atoms, true, C::AT) ||
       (OUT != kOutMxfp4 &&
@@ -737,16 +638,9 @@ cudaError_t launch_pair(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq
   p.k_atoms = (uint32_t)k_atoms;
   p.b_row_tiles = (uint32_t)sf_row_tiles(N);
   p.ldy = (uint64_t)ldy;
-  PairPlan pl = pair_plan(M, N, K, (uint32_t)max_clusters[dev]);
-  if (pl.g > 1 && (scratch.counters == nullptr || scratch.data == nullptr ||
-                   pl.scratch_bytes > scratch.data_bytes))
-    pl = pair_plan(M, N, K, 0);  // no counters or no room for partials: whole tiles only
+  const PairPlan pl = pair_plan(M, N, (uint32_t)max_clusters[dev]);
   p.full_units = pl.full_units;
   p.units = pl.units;
-  p.split_g = pl.g;
-  p.kt_per_chunk = pl.kt_per_chunk;
-  p.flags = pl.g > 1 ? scratch.counters : nullptr;
-  p.part = pl.g > 1 ? reinterpret_cast<float*>(scratch.data) : nullptr;
   p.bias = ep.bias;
   p.yq = OUT == kOutMxfp4 ? static_cast<uint8_t*>(y) : nullptr;
   p.ysf = ep.ysf;
@@ -755,11 +649,11 @@ cudaError_t launch_pair(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq
   p.n_katoms_y = (uint32_t)sf_katoms(N);
   p.a_scale = ep.a_scale;
   p.b_scale = ep.b_scale;
-  p.count_wait_ns = kWaitLimitNs;
-  p.skip_publish = 0;
-  if (g_test_fault.load(std::memory_order_relaxed) == MXFP4_TEST_FAULT_SKIP_SPLIT_PUBLISH) {
-    p.skip_publish = 1;             // chunk 1 of every split tile
-    p.count_wait_ns = 1000000ull;   // 1 ms
+  p.tfull_wait_ns = kWaitLimitNs;
+  p.skip_commit = 0;
+  if (g_test_fault.load(std::memory_order_relaxed) == MXFP4_TEST_FAULT_WITHHOLD_ACCUMULATOR) {
+    p.skip_commit = 1;             // pair 0, first unit
+    p.tfull_wait_ns = 1000000ull;  // 1 ms
   }
   const uint32_t pairs =
       pl.units < (uint32_t)max_clusters[dev] ? pl.units : (uint32_t)max_clusters[dev];
@@ -774,7 +668,7 @@ cudaError_t launch_pair(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, ta, tb, tsa, tsb, ty, p, ep.kc);
+  return cudaLaunchKernelEx(&cfg, kern, ta, tb, tb64, tsa, tsb, ty, p, ep.kc);
 }
 
 }  // namespace
@@ -793,26 +687,23 @@ cudaError_t launch_gemm(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq
   if (ep.nvfp4) {
     if (ep.out == kOutF32)
       return launch_pair<5, kOutF32, true>(aq, asf, bq, bsf, M, N, K, y, ep, ldy, status,
-                                           scratch, stream);
-    return launch_pair<5, kOutBf16, true>(aq, asf, bq, bsf, M, N, K, y, ep, ldy, status, scratch,
-                                          stream);
+                                           stream);
+    return launch_pair<5, kOutBf16, true>(aq, asf, bq, bsf, M, N, K, y, ep, ldy, status, stream);
   }
   switch (ep.out) {
     case kOutF32:
-      return launch_pair<5, kOutF32, false>(aq, asf, bq, bsf, M, N, K, y, ep, ldy, status,
-                                            scratch, stream);
+      return launch_pair<5, kOutF32, false>(aq, asf, bq, bsf, M, N, K, y, ep, ldy, status, stream);
     case kOutMxfp4:
       return launch_pair<5, kOutMxfp4, false>(aq, asf, bq, bsf, M, N, K, y, ep, ldy, status,
-                                              scratch, stream);
+                                              stream);
     default:
-      return launch_pair<5, kOutBf16, false>(aq, asf, bq, bsf, M, N, K, y, ep, ldy, status,
-                                             scratch, stream);
+      return launch_pair<5, kOutBf16, false>(aq, asf, bq, bsf, M, N, K, y, ep, ldy, status, stream);
   }
 }
 
 size_t gemm_scratch_bytes(int64_t M, int64_t N, int64_t K) {
-  if (M <= 128) return gemm_smallm_scratch_bytes(M, N, K);
-  return pair_plan(M, N, K, kPlanPairs).scratch_bytes;
+  // the CTA-pair kernel needs no scratch
+  return M <= 128 ? gemm_smallm_scratch_bytes(M, N, K) : 0;
 }
 
 }  // namespace mxfp4

@@ -90,20 +90,11 @@ struct Epilogue {
   const float* b_scale = nullptr;
 };
 
-// Scratch of the GEMM launchers, in two parts.
-//  - counters: kCounterBytes at a place of the caller's memory that does not move with the
-//    problem size (right after the status region of every workspace layout). The CTA-pair
-//    kernel's per-tile counters for a split last round live here; they must read zero when
-//    a launch starts, and every launch that completes leaves them zero. Because the block
-//    never moves, no launch can find bytes of another part of a workspace (codes, scales,
-//    partials of an earlier call with other sizes) where it expects its counters.
-//  - data: data_bytes for K-split partials (fp32), which every launch writes before it
-//    reads them, so their previous contents do not matter.
-// Either part may be absent (null): the pair kernel then splits no tile and the few-row
-// kernel sums its K splits on chip (same bits).
-constexpr size_t kCounterBytes = 4096;
+// Scratch of the GEMM launchers: data_bytes for the few-row kernel's K-split partials
+// (fp32), which every launch writes before it reads them, so their previous contents do
+// not matter. It may be absent (null): the few-row kernel then sums its K splits on chip
+// (same bits). The CTA-pair kernel needs none.
 struct GemmScratch {
-  unsigned int* counters = nullptr;
   uint8_t* data = nullptr;
   size_t data_bytes = 0;
 };
@@ -186,14 +177,12 @@ mxfp4_status validate_linear(const void* x, int64_t M, int64_t K, mxfp4_rotation
                              const float* kron_a, const float* kron_b, const uint8_t* wq,
                              const uint8_t* wsf, int64_t N, const void* y, KronCoeffs* kc);
 
-// Every workspace starts with the status region (the status word at byte 0; the NVFP4
-// layer's tensor scale and its pass's state at 64..79) and then the GEMM counter block, so
-// that block sits at the same place whatever the sizes of the call.
-constexpr size_t kStatusBytes = 256;
-constexpr size_t kHeadBytes = kStatusBytes + kCounterBytes;
+// Every workspace starts with the status region: the status word at byte 0, the NVFP4
+// layer's tensor scale and its pass's state at 64..79.
+constexpr size_t kHeadBytes = 256;
 
-// Layout of the layer's workspace: [status | counters | Xq (M x K/2) | Xsf (sf_k-element
-// operand scales) | GEMM data], parts 256-byte aligned. sf_k = K for MXFP4, 2 K for NVFP4.
+// Layout of the layer's workspace: [status | Xq (M x K/2) | Xsf (sf_k-element operand
+// scales) | GEMM data], parts 256-byte aligned. sf_k = K for MXFP4, 2 K for NVFP4.
 struct LinearLayout {
   size_t q_off, sf_off, g_off, total;
 };
@@ -202,7 +191,6 @@ LinearLayout linear_layout(int64_t M, int64_t N, int64_t K, int64_t sf_k);
 // The GEMM scratch of a workspace laid out as above (data part: from g_off to ws_bytes).
 inline GemmScratch workspace_scratch(uint8_t* ws, size_t g_off, size_t ws_bytes) {
   GemmScratch g;
-  g.counters = reinterpret_cast<unsigned int*>(ws + kStatusBytes);
   g.data = ws_bytes > g_off ? ws + g_off : nullptr;
   g.data_bytes = ws_bytes > g_off ? ws_bytes - g_off : 0;
   return g;

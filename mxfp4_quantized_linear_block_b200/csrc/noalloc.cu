@@ -11,8 +11,8 @@
 //
 // The array is a file-scope __device__ variable, so every GPU that loads this
 // part of the library holds it until the process exits. Its size caps the
-// problem: 4352 bytes (status region and GEMM counters) + round256(M * K / 2) +
-// round256(the scale bytes of X) must fit in it.
+// problem: 256 bytes (status region) + round256(M * K / 2) + round256(the scale bytes of
+// X) must fit in it.
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -24,11 +24,10 @@ namespace {
 
 constexpr size_t kScratchBytes = MXFP4_NOALLOC_SCRATCH_BYTES;
 
-// Layout: the layer workspace's (status region | GEMM counter block | Xq | X scales |
-// GEMM data = the rest of the array), parts 256-byte aligned. Each call clears the status
-// region and the counter block before its first launch, so nothing an earlier call left
-// there (a timed-out call's counters included) reaches it; the other parts are written
-// before they are read.
+// Layout: the layer workspace's (status region | Xq | X scales | GEMM data = the rest of
+// the array), parts 256-byte aligned. Each call clears the status region before its first
+// launch, so a status an earlier call left there does not reach it; the other parts are
+// written before they are read.
 static __device__ __align__(256) unsigned char g_linear_scratch[kScratchBytes];
 
 std::mutex g_scratch_mutex;
@@ -72,7 +71,7 @@ extern "C" mxfp4_status mxfp4_linear_noalloc(const void* x, int64_t M, int64_t K
   mxfp4_status st = scratch_on_current_device(&scratch);
   if (st != MXFP4_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  // Status word (used when the caller passes none) and GEMM counters start at zero.
+  // The status word (used when the caller passes none) starts at zero.
   if (cudaMemsetAsync(scratch, 0, kHeadBytes, s) != cudaSuccess) return MXFP4_ERR_CUDA;
   int* status_word = status ? status : reinterpret_cast<int*>(scratch);
   uint8_t* xq = scratch + w.q_off;

@@ -45,10 +45,10 @@ def test_status_strings():
 
 def test_workspace_sizes():
     assert mx.workspace_bytes(mx.OP_QUANTIZE, 10, 16, 64) == 0
-    assert mx.workspace_bytes(mx.OP_GEMM, 10, 16, 64) == 4352
+    assert mx.workspace_bytes(mx.OP_GEMM, 10, 16, 64) == 256
     M, K = 3584, 3072
     ws = mx.workspace_bytes(mx.OP_LINEAR, M, 9216, K)
-    assert ws >= 4352 + M * K // 2 + mx.sf_bytes(M, K)
+    assert ws == 256 + M * K // 2 + mx.sf_bytes(M, K)
 
 
 # Fake device addresses: validation rejects these calls on the host, so nothing is dereferenced.
@@ -183,40 +183,29 @@ def test_norm_linear_kernel_count():
 
 
 def test_gemm_scratch_for_few_rows():
-    """Every workspace starts with a 4352-byte head (256-byte status region, then the
-    4096-byte counter block). The few-row GEMM's K-split partials follow it for 33..128
-    rows split 4 or more ways: units x rows x 128 columns x 4 bytes; fewer splits or rows
-    need nothing past the head."""
+    """Every workspace starts with the 256-byte status region. The few-row GEMM's K-split
+    partials follow it for 33..128 rows split 4 or more ways: units x rows x 128 columns
+    x 4 bytes; fewer splits or rows need nothing past the head."""
     def gemm_ws(M, N, K):
         return mx.workspace_bytes(mx.OP_GEMM, M, N, K)
     # 4096 -> 14336 weights transposed: 32 W tiles x 8 splits = 256 units, 128 rows
-    assert gemm_ws(128, 4096, 14336) == 4352 + 256 * 128 * 128 * 4
+    assert gemm_ws(128, 4096, 14336) == 256 + 256 * 128 * 128 * 4
     # 100 rows, 8 W tiles x 7 splits (28 k-tiles in splits of 4)
-    assert gemm_ws(100, 1024, 7168) == 4352 + 56 * 100 * 128 * 4
-    assert gemm_ws(128, 14336, 4096) == 4352  # 112 W tiles x 2 splits: on-chip sum
-    assert gemm_ws(32, 4096, 14336) == 4352   # 32 rows: on-chip sum
-    assert gemm_ws(1, 14336, 4096) == 4352
+    assert gemm_ws(100, 1024, 7168) == 256 + 56 * 100 * 128 * 4
+    assert gemm_ws(128, 14336, 4096) == 256  # 112 W tiles x 2 splits: on-chip sum
+    assert gemm_ws(32, 4096, 14336) == 256   # 32 rows: on-chip sum
+    assert gemm_ws(1, 14336, 4096) == 256
 
 
-def test_gemm_scratch_for_a_split_last_round():
-    """CTA-pair plan on 74 pairs: 2560 x 2048 gives 10 x 8 = 80 tiles of 256 x 256, so the
-    last round has 6 tiles; each is split into g = min(74 / 6, 4) = 4 K chunks of 6
-    k-tiles (6 + a hand-off of about 4 is under 85 % of 24), and chunks 1..3 leave one
-    128 x 256 fp32 partial per CTA of the pair. The counters stay in the head; the
-    partials follow it."""
-    part = 6 * (4 - 1) * 2 * 128 * 256 * 4
-    assert mx.workspace_bytes(mx.OP_GEMM, 2560, 2048, 6144) == 4352 + part
-    # the layer adds the activation codes and scales between the head and the partials
-    M, K = 2560, 6144
-    codes = M * K // 2
-    assert mx.workspace_bytes(mx.OP_LINEAR, M, 2048, K) == 4352 + codes + mx.sf_bytes(M, K) + part
-    # 4096 x 2048 x 8192: 16 x 8 = 128 tiles, 54 left for a second round: g = 1, no split
-    assert mx.workspace_bytes(mx.OP_GEMM, 4096, 2048, 8192) == 4352
-    # the DiT MLP-up at batch 16: 224 x 48 = 10752 tiles, 22 in the last round, K = 3072
-    # (12 k-tiles) in 3 chunks of 4
-    assert mx.workspace_bytes(mx.OP_GEMM, 57344, 12288, 3072) == 4352 + 22 * 2 * 2 * 131072
-    # 4 k-tiles: a chunk of 1 plus the hand-off is no gain, no split
-    assert mx.workspace_bytes(mx.OP_GEMM, 2560, 2048, 1024) == 4352
+def test_pair_gemm_needs_no_scratch():
+    """The CTA-pair GEMM (more than 128 rows) exchanges nothing between pairs, whatever
+    its last round looks like: its workspace is the status region alone, and the layer's
+    adds only the activation codes and scales."""
+    for M, N, K in [(2560, 2048, 6144), (4096, 2048, 8192), (57344, 12288, 3072),
+                    (3584, 3072, 3072), (129, 16, 64)]:
+        assert mx.workspace_bytes(mx.OP_GEMM, M, N, K) == 256
+        assert mx.workspace_bytes(mx.OP_LINEAR, M, N, K) == (
+            256 + -(-M * K // 2 // 256) * 256 + -(-mx.sf_bytes(M, K) // 256) * 256)
 
 
 def test_kron_weight_factors_match_oracle():

@@ -100,28 +100,28 @@ def test_gemm_few_rows_single_pair_in_last_split():
     assert not y.any()
 
 
-# Large-M shapes whose last round of 256x256 tiles is split along K over several CTA
-# pairs (74 pairs on a B200; up to 4 chunks, when a chunk plus the 4-k-tile hand-off is
-# under 85 % of the tile): tiles -> split tiles x K chunks. (512,512,4096) 4 -> 4x4;
-# (768,1024,8192) 12 -> 12x4; (700,784,6176) 12 ragged tiles -> 12x4, chunks of 7, 7, 7
-# and 4 k-tiles with a 32-element K tail.
-SPLIT_SHAPES = [(512, 512, 4096), (768, 1024, 8192), (700, 784, 6176)]
+# Large-M shapes whose last round of 256x256 tiles leaves at least half of the 74 CTA
+# pairs of a B200 idle, so that its tiles run as two 256 x 128 units each (N = 128 MMAs,
+# the scale group of the column half): tiles -> units. (512,512,4096) 4 -> 8;
+# (768,1024,8192) 12 -> 24; (700,784,6176) 12 ragged tiles -> 24, a 32-element K tail,
+# and a last column tile of 16 columns (its second half lies wholly past N).
+HALF_SHAPES = [(512, 512, 4096), (768, 1024, 8192), (700, 784, 6176)]
 
 
-@pytest.mark.parametrize("M,N,K", SPLIT_SHAPES)
+@pytest.mark.parametrize("M,N,K", HALF_SHAPES)
 @pytest.mark.parametrize("out", ["bf16", "f32"])
-def test_gemm_split_last_round(M, N, K, out):
+def test_gemm_last_round_in_column_halves(M, N, K, out):
     aq, as_ = _operand(M + 3 * N + K, M, K, 8)
     bq, bs = _operand(M + 3 * N + K, N, K, 9)
     y = _run(aq, as_, bq, bs, out)
     ref, S = oracle.gemm(aq, as_, bq, bs)
-    check_gemm_values(y, ref, S, out, f"split gemm {M}x{N}x{K} {out}")
+    check_gemm_values(y, ref, S, out, f"column-half gemm {M}x{N}x{K} {out}")
 
 
-def test_gemm_split_full_rounds_then_tail():
-    """80 tiles on 74 pairs: one round of whole tiles, then 6 tiles in 4 K chunks each.
-    Every element of the last 256-row band (which holds the 6 split tiles) is checked,
-    plus sampled pairs elsewhere."""
+def test_gemm_full_rounds_then_column_halves():
+    """80 tiles on 74 pairs: one round of whole tiles, then 6 tiles as 12 column-half
+    units. Every element of the last 256-row band (which holds the 6 tiles of the last
+    round) is checked, plus sampled pairs elsewhere."""
     M, N, K = 2560, 2048, 6144
     aq, as_ = _operand(5, M, K, 10)
     bq, bs = _operand(5, N, K, 11)
@@ -133,14 +133,14 @@ def test_gemm_split_full_rounds_then_tail():
     check_gemm_values(y[mi, ni], ref, S, "f32", "sampled")
 
 
-def test_gemm_split_repeat_and_scratch_reset():
-    """Back-to-back launches on different inputs through one workspace: each result is
-    right, repeated inputs give identical bits, and the split counters are zero after."""
+def test_gemm_column_halves_repeat():
+    """Back-to-back launches on different inputs through one workspace (the status
+    region alone): each result is right and repeated inputs give identical bits."""
     import torch
     import mxfp4_quantized_linear_block_b200 as mx
     M, N, K = 768, 1024, 8192
     ws = mx.new_workspace(mx.workspace_bytes(mx.OP_GEMM, M, N, K))
-    assert ws.numel() >= 4352 + 12 * 3 * 2 * 128 * 256 * 4  # 12 tiles x chunks 1..3
+    assert ws.numel() == 256
     outs = []
     for seed in (21, 22, 21):
         aq, as_ = _operand(seed, M, K, 12)
@@ -154,7 +154,6 @@ def test_gemm_split_repeat_and_scratch_reset():
         check_gemm_values(outs[-1].astype(np.float64), ref, S, "f32", f"seed {seed}")
     assert np.array_equal(outs[0].view(np.uint32), outs[2].view(np.uint32))
     assert mx.poll_status(ws) == mx.OK
-    assert not ws[256:4352].cpu().numpy().any()  # the counter block
 
 
 def test_gemm_wide_scale_range_fp32():
@@ -235,7 +234,7 @@ def test_gemm_and_linear_with_no_rows_write_nothing():
 @pytest.mark.parametrize("out", ["bf16", "f32"])
 def test_few_rows_l2_and_on_chip_sums_agree(M, N, K, out):
     """33..128 rows split 6 to 8 ways (36 W tiles x 6, 8 x 7, 32 x 8) sum their K splits
-    through L2 when the workspace has room for the partials past its 4352-byte head,
+    through L2 when the workspace has room for the partials past its 256-byte head,
     and through distributed shared memory when it has only the status region: same order
     of additions, so the same bits; both match the oracle."""
     import torch
@@ -246,7 +245,7 @@ def test_few_rows_l2_and_on_chip_sums_agree(M, N, K, out):
             to_dev(oracle.sf_to_physical(bs, K)), M, N, K)
     dt = torch.float32 if out == "f32" else torch.bfloat16
     full = mx.new_workspace(mx.workspace_bytes(mx.OP_GEMM, M, N, K))
-    assert full.numel() > 4352  # this size uses the L2 form
+    assert full.numel() > 256  # this size uses the L2 form
     y_l2 = mx.gemm(*args, out_dtype=dt, ws=full)
     y_chip = mx.gemm(*args, out_dtype=dt, ws=mx.new_workspace(256))
     torch.cuda.synchronize()
@@ -258,9 +257,8 @@ def test_few_rows_l2_and_on_chip_sums_agree(M, N, K, out):
 
 
 def test_workspace_shared_by_few_row_and_pair_kernels():
-    """The few-row kernel's L2 partials lie past the workspace's counter block, so they
-    leave the pair kernel's split counters zero: one workspace serves a 128-row call, then
-    a split call."""
+    """One workspace serves a 128-row call (its L2 partials past the status region),
+    then a pair call whose last round runs in column halves, and again."""
     import torch
     import mxfp4_quantized_linear_block_b200 as mx
     shapes = [(128, 4096, 14336), (512, 512, 4096)]

@@ -1,14 +1,12 @@
 """One workspace serving layer calls of different sizes.
 
-The CTA-pair GEMM splits the tiles of a short last round along K; chunk 0 of a split
-tile waits on a counter for the other chunks' partials. Those counters live in a block
-right after the status region of every workspace, so a call never finds codes, scales
-or partials of an earlier call with other sizes where it expects zero counters. The
-sequence below is the one that would expose such stale counters: a large call fills
-the workspace with codes, then a call whose last round is split (2560 x 6144 -> 2048:
-80 tiles of 256 x 256 on 74 CTA pairs, the last 6 tiles split in 4 K chunks) runs on
-the same workspace. Its outputs, the split tiles included, are checked against the
-oracle's exact products.
+Every part of a layer workspace past its status region is written before it is read, so
+what an earlier call with other sizes left there never reaches a later call. The sequence
+below checks that: a large call fills the workspace with codes and scales, then a call
+whose last round runs in column halves (2560 x 6144 -> 2048: 80 tiles of 256 x 256 on 74
+CTA pairs, the last 6 tiles as twelve 256 x 128 units) runs on the same workspace, and
+both again. Its outputs, the tiles of the last round included, are checked against the
+oracle's exact products, and repeated calls give the same bits.
 """
 import numpy as np
 import pytest
@@ -20,8 +18,8 @@ from test_gpu_gemm import _sample_pairs
 
 pytestmark = pytest.mark.gpu
 
-LARGE = (4096, 8192, 2048)  # M, K, N: 128 tiles, no split
-SPLIT = (2560, 6144, 2048)  # 80 tiles: the last 6 (rows 2304.., columns 512..) split 4 ways
+LARGE = (4096, 8192, 2048)  # M, K, N: 128 tiles: a full round, then 54 whole tiles
+SPLIT = (2560, 6144, 2048)  # 80 tiles: the last 6 (rows 2304.., columns 512..) in halves
 
 
 def _problem(seed, M, K, N):
@@ -32,8 +30,8 @@ def _problem(seed, M, K, N):
 
 
 def _split_tile_pairs(M, N, seed):
-    """Every (m, n) of 64 random columns of the split tiles (the last row tile of 256,
-    columns 512..N-1), plus the usual edge and random samples."""
+    """Every (m, n) of 64 random columns of the last round's tiles (the last row tile of
+    256, columns 512..N-1), plus the usual edge and random samples."""
     rng = np.random.default_rng(seed)
     rows = np.arange(M - 256, M)
     cols = rng.choice(np.arange(512, N), 64, replace=False)
@@ -50,14 +48,13 @@ def _check(y, x, wq, ws, what, seed):
     check_gemm_values(y[mi, ni], ref, S, "bf16", what)
 
 
-def test_split_plan_of_the_second_call():
-    """The second shape really splits its last round (host-side plan)."""
+def test_workspace_sizes_of_the_two_calls():
+    """The layer workspace is the status region, the codes and the scales (no GEMM
+    scratch for more than 128 rows)."""
     import mxfp4_quantized_linear_block_b200 as mx
-    M, K, N = SPLIT
-    part = 6 * 3 * 2 * 128 * 256 * 4
-    assert mx.workspace_bytes(mx.OP_GEMM, M, N, K) == 4352 + part
-    M, K, N = LARGE
-    assert mx.workspace_bytes(mx.OP_GEMM, M, N, K) == 4352
+    for M, K, N in (LARGE, SPLIT):
+        assert mx.workspace_bytes(mx.OP_GEMM, M, N, K) == 256
+        assert mx.workspace_bytes(mx.OP_LINEAR, M, N, K) == 256 + M * K // 2 + mx.sf_bytes(M, K)
 
 
 def test_linear_workspace_large_then_split_call():
@@ -80,5 +77,3 @@ def test_linear_workspace_large_then_split_call():
     # the same calls again on the same workspace give the same bits
     assert np.array_equal(results[0], results[2])
     assert np.array_equal(results[1], results[3])
-    # the counter block (bytes 256 .. 4351) is zero after calls that completed
-    assert not ws[256:4352].cpu().numpy().any()

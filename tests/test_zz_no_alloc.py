@@ -78,8 +78,9 @@ def test_noalloc_matches_linear_on_two_calls_in_a_row():
 
 
 def test_noalloc_call_after_a_timeout_needs_no_reset():
-    """A call whose split wait ran out (the library's test hook) may leave GEMM counters
-    set in the shared array; the next call clears them itself and is right."""
+    """A call whose accumulator wait ran out (the library's test hook) leaves the timeout
+    in the caller's status word and part of Y unwritten; the next calls on the shared
+    array need no reset and are right."""
     import torch
     import mxfp4_quantized_linear_block_b200 as mx
 
@@ -89,7 +90,7 @@ def test_noalloc_call_after_a_timeout_needs_no_reset():
     y_ref = mx.linear(xd, wqd, wsfd, N, mx.ROT_HADAMARD32)
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     y_na = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
-    mx.test_set_fault(mx.TEST_FAULT_SKIP_SPLIT_PUBLISH)
+    mx.test_set_fault(mx.TEST_FAULT_WITHHOLD_ACCUMULATOR)
     try:
         st = _call_noalloc(mx, xd, wqd, wsfd, M, K, N, y_na, status, mx.ROT_HADAMARD32)
     finally:
