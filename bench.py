@@ -57,18 +57,18 @@ PKG = "mxfp4_quantized_linear_block_b200"
 # kernel ends is written back later and is not counted (hence writes < Y bytes).
 NCU_TRAFFIC = {
     "dit_b16": {"source": f"{PKG}/csrc/gemm.cu",
-                "sha256": "1c5542388a3740ee08690759276d2c9c6fbad750f41a0da5e6a21bf9f77e1f84",
-                "bytes_per_launch": [151046000 + 1367771000, 396393000 + 332764000]},
+                "sha256": "c85828eea8edddc5ded4db226d7ba778ad3a0bfce965270c0a53781d6f5af657",
+                "bytes_per_launch": [143816210 + 1354265618, 401536420 + 325861138]},
     "dit_b1": {"source": f"{PKG}/csrc/gemm.cu",
-               "sha256": "1c5542388a3740ee08690759276d2c9c6fbad750f41a0da5e6a21bf9f77e1f84",
-               "bytes_per_launch": [20934400 + 12165888, 26183424 + 41680384,
-                                    43516160 + 5652736]},
+               "sha256": "c85828eea8edddc5ded4db226d7ba778ad3a0bfce965270c0a53781d6f5af657",
+               "bytes_per_launch": [20928512 + 12389632, 26400256 + 37001984,
+                                    43516160 + 2887424]},
     "llm_small_m16": {"source": f"{PKG}/csrc/gemm_smallm.cu",
-                      "sha256": "00d1f124ffd446fabf7e60419776340596702696091ba863f76e04ae84a7db68",
+                      "sha256": "bbb88d371a5c74f77f3a387bb3678bf27b061d3e357a23d24451cf9914d26966",
                       "bytes_per_launch": [31321856 + 0, 31442944 + 0]},
     "llm_small_m128": {"source": f"{PKG}/csrc/gemm_smallm.cu",
-                       "sha256": "00d1f124ffd446fabf7e60419776340596702696091ba863f76e04ae84a7db68",
-                       "bytes_per_launch": [31553536 + 0, 32242432 + 96256]},
+                       "sha256": "bbb88d371a5c74f77f3a387bb3678bf27b061d3e357a23d24451cf9914d26966",
+                       "bytes_per_launch": [31556864 + 0, 32239104 + 4608]},
 }
 NCU_TRAFFIC_QUANTIZE = {
     "dit_b16": {"source": f"{PKG}/csrc/quantize.cu",

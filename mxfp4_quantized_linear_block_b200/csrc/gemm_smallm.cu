@@ -70,11 +70,18 @@ struct SmallConfig {
   static constexpr uint32_t XQ_KT = NT * 128;
   static constexpr uint32_t XQ_BYTES = FX ? kFxMaxKt * XQ_KT : 0;
   static constexpr uint32_t XSF_BYTES = FX ? kFxMaxKt * SF_STAGE : 0;
-  // Two CTAs per SM: as many stages (at most 5) as let 2 x SMEM_BYTES fit an SM's
-  // shared memory (233472 bytes, 1 KB of it reserved per CTA).
+  // Up to 64 tokens two CTAs per SM: as many stages (at most 5) as let 2 x SMEM_BYTES fit
+  // an SM's shared memory (233472 bytes, 1 KB of it reserved per CTA). 128 tokens: one
+  // CTA per SM with up to 12 stages, so that half as many K splits keep the same bytes in
+  // flight (B200, 128 x 14336 <-> 4096: 12.4 / 12.6 -> 11.8 / 11.0 us; at 1 and 16 tokens
+  // the same change cost 0.2-0.8 us, the sums being small there).
+  static constexpr bool WIDE = NT == 128;
   static constexpr uint32_t STAGE_BYTES = A_STAGE + B_STAGE + (FX ? 1 : 2) * SF_STAGE;
-  static constexpr uint32_t BUDGET = 116736 - 1024 - 1024 - 512 - XQ_BYTES - XSF_BYTES;
-  static constexpr uint32_t STAGES = BUDGET / STAGE_BYTES < 5 ? BUDGET / STAGE_BYTES : 5;
+  static constexpr uint32_t BUDGET =
+      (WIDE ? 232448 : 116736) - 1024 - 1024 - 512 - XQ_BYTES - XSF_BYTES;
+  static constexpr uint32_t MAX_STAGES = WIDE ? 12 : 5;
+  static constexpr uint32_t STAGES =
+      BUDGET / STAGE_BYTES < MAX_STAGES ? BUDGET / STAGE_BYTES : MAX_STAGES;
   static constexpr uint32_t OFF_A = 0;
   static constexpr uint32_t OFF_B = OFF_A + STAGES * A_STAGE;
   static constexpr uint32_t OFF_XQ = OFF_B + STAGES * B_STAGE;
@@ -96,7 +103,8 @@ struct SmallConfig {
   static_assert(RED_BYTES <= OFF_SFA, "partial fits over the operand stages");
   static_assert(!FX || (!NV && STAGES >= 3), "fused layer: MXFP4, a ring of 3 or more");
   static_assert(OFF_XQ % 1024 == 0 && XQ_KT % 1024 == 0, "128-byte swizzle atoms");
-  static_assert(2 * (SMEM_BYTES + 1024) <= 233472, "two CTAs per SM");
+  static_assert(WIDE ? SMEM_BYTES <= 232448 : 2 * (SMEM_BYTES + 1024) <= 233472,
+                "one CTA per SM (128 tokens), else two");
 };
 
 struct SmallParams {
@@ -639,16 +647,16 @@ struct Plan {
 
 uint32_t token_tile(int64_t M) { return M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : 128; }
 
-// Units (W tile x K split) are sized so that all of them are resident at once:
-// two CTAs per SM on the 148 SMs of a B200.
-constexpr uint32_t kSlots = 148 * 2;
+// Units (W tile x K split) are sized so that all of them are resident at once on the
+// 148 SMs of a B200: two CTAs per SM, one for 128 tokens.
+constexpr uint32_t kSms = 148;
 
 Plan make_plan(int64_t M, int64_t N, int64_t K) {
   Plan pl{};
   pl.nt = token_tile(M);
   pl.w_tiles = (uint32_t)((N + 127) / 128);
   pl.k_tiles = (uint32_t)((K + 255) / 256);
-  uint32_t splits = kSlots / pl.w_tiles;
+  uint32_t splits = (pl.nt == 128 ? kSms : 2 * kSms) / pl.w_tiles;
   if (splits > kMaxSplits) splits = kMaxSplits;
   if (splits < 1) splits = 1;
   if (splits > pl.k_tiles) splits = pl.k_tiles;

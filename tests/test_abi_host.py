@@ -188,11 +188,12 @@ def test_gemm_scratch_for_few_rows():
     x 4 bytes; fewer splits or rows need nothing past the head."""
     def gemm_ws(M, N, K):
         return mx.workspace_bytes(mx.OP_GEMM, M, N, K)
-    # 4096 -> 14336 weights transposed: 32 W tiles x 8 splits = 256 units, 128 rows
-    assert gemm_ws(128, 4096, 14336) == 256 + 256 * 128 * 128 * 4
+    # 4096 -> 14336 weights transposed, 128 rows (one CTA per SM): 32 W tiles x 4 splits
+    # = 128 units
+    assert gemm_ws(128, 4096, 14336) == 256 + 128 * 128 * 128 * 4
     # 100 rows, 8 W tiles x 7 splits (28 k-tiles in splits of 4)
     assert gemm_ws(100, 1024, 7168) == 256 + 56 * 100 * 128 * 4
-    assert gemm_ws(128, 14336, 4096) == 256  # 112 W tiles x 2 splits: on-chip sum
+    assert gemm_ws(128, 14336, 4096) == 256  # 112 W tiles, one split: no sum
     assert gemm_ws(32, 4096, 14336) == 256   # 32 rows: on-chip sum
     assert gemm_ws(1, 14336, 4096) == 256
 

@@ -61,12 +61,13 @@ def test_gemm_zero_and_single_pair():
 
 
 # Few activation rows (M <= 128): the weight-streaming kernel splits K over the
-# CTAs of a thread-block cluster and adds the partials through distributed shared
-# memory (up to 32 rows, or fewer than 4 splits) or through L2 (33..128 rows split 4
-# or more ways, with the workspace's scratch). (M, N, K) -> W tiles x K splits:
-# (1,16,4096) 1x8; (5,400,2080) 4x5 with a 32-element K tail; (16,256,8192) 2x8;
-# (17,12288,1024) 96x2; (33,9216,1536) 72x3; (64,2048,3104) 16x7 with a K tail (L2);
-# (100,1024,7168) 8x7 (L2); (65,14336,4096) 112x2; (128,4096,14336) 32x8 (L2).
+# CTAs of a thread-block cluster (two CTAs per SM, one for 65..128 rows) and adds the
+# partials through distributed shared memory (up to 32 rows, or fewer than 4 splits) or
+# through L2 (33..128 rows split 4 or more ways, with the workspace's scratch).
+# (M, N, K) -> W tiles x K splits: (1,16,4096) 1x8; (5,400,2080) 4x5 with a 32-element
+# K tail; (16,256,8192) 2x8; (17,12288,1024) 96x2; (33,9216,1536) 72x3; (64,2048,3104)
+# 16x7 with a K tail (L2); (100,1024,7168) 8x7 (L2); (65,14336,4096) 112x1 (no sum);
+# (128,4096,14336) 32x4 (L2).
 SMALLM_SHAPES = [
     (1, 16, 4096), (5, 400, 2080), (16, 256, 8192), (17, 12288, 1024), (33, 9216, 1536),
     (64, 2048, 3104), (100, 1024, 7168), (65, 14336, 4096), (128, 4096, 14336),
@@ -233,7 +234,7 @@ def test_gemm_and_linear_with_no_rows_write_nothing():
 @pytest.mark.parametrize("M,N,K", [(33, 4608, 1536), (100, 1024, 7168), (128, 4096, 14336)])
 @pytest.mark.parametrize("out", ["bf16", "f32"])
 def test_few_rows_l2_and_on_chip_sums_agree(M, N, K, out):
-    """33..128 rows split 6 to 8 ways (36 W tiles x 6, 8 x 7, 32 x 8) sum their K splits
+    """33..128 rows split 4 to 7 ways (36 W tiles x 6, 8 x 7, 32 x 4) sum their K splits
     through L2 when the workspace has room for the partials past its 256-byte head,
     and through distributed shared memory when it has only the status region: same order
     of additions, so the same bits; both match the oracle."""
