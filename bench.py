@@ -114,6 +114,10 @@ def parse():
                          "last writes MXFP4 (mxfp4_gemm_quantize) that the next GEMM reads, "
                          "so only the first input is quantised from bf16")
     ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--library-baseline", action="store_true",
+                    help="also time the vendor library's MXFP4 GEMM (cuBLASLt through "
+                         "torch.nn.functional.scaled_mm) on the same quantised operands, as "
+                         "context for the GEMM row (MXFP4, no norm, not fused)")
     return ap.parse_args()
 
 
@@ -521,6 +525,10 @@ def run_ours(args, rank, world, local_rank):
         if not fused[j]:
             t_q[j] = time_graph(quant_launch, j)
         t_g[j] = time_graph(gemm_launch, j)
+    library = (library_gemm(mx, wl, sets, wsets, qbufs, nq, gws, quant_launch, time_graph,
+                            t_g, stream)
+               if args.library_baseline and not nv and norm is None and not any(fused)
+               else None)
     gemm_flops = np.array([l.flops for l in wl.linears], dtype=np.float64)
     sfb = mx.nvfp4_sf_bytes if nv else mx.sf_bytes
     # a fused layer reads x in bf16 instead of its codes and scales
@@ -701,6 +709,7 @@ def run_ours(args, rank, world, local_rank):
                                "layer's one kernel (1..8 rows): no quantiser launch"}),
         "e2e": e2e,
         "gpu_launches": launches,
+        **({"library_gemm": library} if library is not None else {}),
         "attribution": {"launches_per_graph": n_attr,
                         "note": "per linear, one CUDA graph of back-to-back quantiser launches "
                                 "and one of back-to-back GEMM launches (a one-kernel layer: "
@@ -709,6 +718,66 @@ def run_ours(args, rank, world, local_rank):
         "clocks": clk,
     }
     return result
+
+
+def library_gemm(mx, wl, sets, wsets, qbufs, nq, gws, quant_launch, time_graph, t_g, stream):
+    """The vendor library's MXFP4 GEMM (cuBLASLt, through torch.nn.functional.scaled_mm)
+    on the operands the step's quantiser wrote: E2M1 codes, E8M0 scales per 32 elements in
+    the 128 x 4 tensor-core atom layout (the library's 32_4_4 swizzle), bf16 out. Timed like
+    the attribution pass; its output is compared with this library's on the same operands
+    (both accumulate in fp32, in different orders: they should agree to about 1 bf16 ulp)."""
+    import torch
+    import torch.nn.functional as F
+    from torch.nn.functional import ScalingType, SwizzleType
+
+    def ru(a, b):
+        return -(-a // b) * b
+
+    def operands(i, j):
+        lin = wl.linears[j]
+        q, sf, _, _ = qbufs[i % nq][j]
+        wq, wsf, _ = wsets[i % len(wsets)][j]
+        a = q.view(torch.float4_e2m1fn_x2)
+        b = wq.view(torch.float4_e2m1fn_x2).t()
+        sa = sf[:ru(lin.M, 128) * ru(lin.K // 32, 4)].view(torch.float8_e8m0fnu).view(
+            ru(lin.M, 128), ru(lin.K // 32, 4))
+        sb = wsf[:ru(lin.N, 128) * ru(lin.K // 32, 4)].view(torch.float8_e8m0fnu).view(
+            ru(lin.N, 128), ru(lin.K // 32, 4))
+        return a, b, sa, sb
+
+    def lib_launch(i, j, s):
+        a, b, sa, sb = operands(i, j)
+        return F.scaled_mm(a, b, sa, ScalingType.BlockWise1x32, sb, ScalingType.BlockWise1x32,
+                           SwizzleType.SWIZZLE_32_4_4, SwizzleType.SWIZZLE_32_4_4,
+                           output_dtype=torch.bfloat16)
+
+    out = {"impl": "cuBLASLt MXFP4 GEMM through torch.nn.functional.scaled_mm "
+                   f"(torch {torch.__version__})", "per_launch": []}
+    for j, lin in enumerate(wl.linears):
+        try:
+            t = time_graph(lib_launch, j)
+            quant_launch(0, j, stream)
+            y_lib = lib_launch(0, j, stream)
+            q, sf, _, _ = qbufs[0][j]
+            wq, wsf, _ = wsets[0][j]
+            y_own = mx.gemm(q, sf, wq, wsf, lin.M, lin.N, lin.K, ws=gws[j], stream=stream)
+            torch.cuda.synchronize()
+            # difference in units of the bf16 spacing at each of our values: |y| = m 2^e
+            # with m in [0.5, 1) has spacing 2^(e - 8)
+            d = (y_lib.float() - y_own.float()).abs()
+            _, e = torch.frexp(y_own.float().abs().clamp(min=2.0 ** -126))
+            ulp = torch.ldexp(torch.ones_like(d), e - 8)
+            r = d / ulp
+            out["per_launch"].append({
+                "linear": lin.name, "us": t * 1e6, "tflops": lin.flops / t / 1e12,
+                "ours_us": t_g[j] * 1e6, "library_time_over_ours": t / t_g[j],
+                "outputs_within_1_ulp": float((r <= 1.0).float().mean()),
+                "outputs_within_2_ulp": float((r <= 2.0).float().mean())})
+            del y_lib, y_own, d, ulp, r
+        except Exception as e:  # the library may not offer this shape
+            out["per_launch"].append({"linear": lin.name,
+                                      "unavailable": str(e).splitlines()[0][:200]})
+    return out
 
 
 # --------------------------------------------------------------------------- chained layers
