@@ -26,7 +26,8 @@ from gpu_helpers import check_gemm_values, to_dev
 pytestmark = pytest.mark.gpu
 
 # few-row kernel (M <= 128, K split over 1-8 CTAs of a cluster) and CTA-pair kernel
-# (M > 128; (512, 512, 4096) splits its only round along K); N % 128 != 0 included.
+# (M > 128; every pair-kernel shape here runs its only round as 256 x 128 column-half
+# units, (129, 416, 512) with a last half of 32 columns); N % 128 != 0 included.
 SHAPES = [(1, 416, 1024), (5, 128, 4096), (17, 12288, 1024), (128, 4096, 2048),
           (129, 416, 512), (300, 1024, 768), (512, 512, 4096)]
 
