@@ -79,8 +79,8 @@ def _nv_operands(M, N, K, seed):
 
 
 # few-row kernel (M <= 128; clusters of 1-8 K splits) and CTA-pair kernel (M > 128;
-# every pair-kernel shape here runs its last round as 256 x 128 column-half units, the
-# N = 144 one with a last half wholly past N); K tails at 32 / 96 of 64
+# every pair-kernel shape here runs its last round as 256 x 128 column-half units: N = 144
+# ends in a half of 16 columns, N = 384 in a half wholly past N); K tails at 32 / 96 of 64
 NV_SHAPES = [(1, 16, 64), (5, 400, 2080), (16, 256, 8192), (128, 4096, 2048), (129, 144, 96),
              (300, 384, 1056), (512, 512, 4096), (768, 1024, 8192)]
 
