@@ -47,6 +47,9 @@ import synth  # noqa: E402
 METRIC = "MXFP4 W4A4 linear TFLOPS & % FP4 peak; quantize GB/s & % HBM peak"
 UNIT = "TFLOPS"
 FP4_OVER_BF16 = 4.0  # nominal dense FP4 : BF16 tensor throughput on B200 (9 : 2.25 PFLOP/s)
+# Nominal B200 figures, reported beside the measured-peak fractions: dense FP4 9 PFLOP/s,
+# HBM3e about 8 TB/s.
+NOMINAL = {"TFLOP/s": 9000.0, "GB/s": 8000.0}
 PKG = "mxfp4_quantized_linear_block_b200"
 
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the dominant GEMM kernel,
@@ -579,6 +582,7 @@ def run_ours(args, rank, world, local_rank):
                     "peak_source": f"{peaks['source']} HBM copy bandwidth"}
     roofline.update({
         "frac": roofline["achieved"] / roofline["peak"], "kernel": g_kernel,
+        "frac_of_nominal": roofline["achieved"] / NOMINAL[roofline["unit"]],
         "timing": ("timed region: every launch of the step is this kernel; per_launch: "
                    "attribution pass" if all(fused) else
                    "attribution pass: a CUDA graph of back-to-back launches of this kernel "
@@ -698,6 +702,7 @@ def run_ours(args, rank, world, local_rank):
                                           if norm is not None else "rotate_quantize_kernel"),
                                "achieved": q_ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                                "frac": q_ach / peaks["hbm_gbs"],
+                               "frac_of_nominal": q_ach / NOMINAL["GB/s"],
                                "per_launch_us": [t_q[j] * 1e6 for j in q_sel],
                                "alg_bytes_per_launch": [int(q_bytes[j]) for j in q_sel],
                                "traffic": (float(np.mean(q_traffic["bytes_per_launch"]))
@@ -926,6 +931,7 @@ def run_chain(args, rank, world, local_rank):
                 "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "peak_source": f"{peaks['source']} HBM copy bandwidth"}
     roof.update({"frac": roof["achieved"] / roof["peak"],
+                 "frac_of_nominal": roof["achieved"] / NOMINAL[roof["unit"]],
                  "kernel": ("mxf4_gemm_pair_kernel" if L[0].M > 128 else "mxf4_gemm_smallm_kernel")
                  + " (MXFP4 out between layers, bf16 out of the last)",
                  "intensity_flop_per_byte": intensity, "ridge_flop_per_byte": ridge,
@@ -984,6 +990,7 @@ def run_chain(args, rank, world, local_rank):
         "quantize_roofline": {"bound": "hbm", "kernel": "rotate_quantize_kernel (X0 only)",
                               "achieved": q_bytes / t_q / 1e9, "peak": peaks["hbm_gbs"],
                               "unit": "GB/s", "frac": q_bytes / t_q / 1e9 / peaks["hbm_gbs"],
+                              "frac_of_nominal": q_bytes / t_q / 1e9 / NOMINAL["GB/s"],
                               "per_launch_us": [t_q * 1e6], "traffic": None},
         "e2e": e2e,
         "gpu_launches": (1 + len(L)) * args.steps,
