@@ -556,9 +556,12 @@ def run_ours(args, rank, world, local_rank):
     # intensity (2MNK over its algorithmic bytes) is above the ridge of the two peaks,
     # HBM-bound otherwise (few tokens).
     few_rows = all(l.M <= 128 for l in wl.linears)
-    g_kernel = ("mxf4_gemm_smallm_kernel (whole layer: x rotated and quantised in the kernel)"
-                if all(fused) else "mxf4_gemm_smallm_kernel" if few_rows
-                else "mxf4_gemm_pair_kernel")
+    if few_rows:
+        g_kernel = ("mxf4_gemm_smallm_kernel (whole layer: x rotated and quantised in the kernel)"
+                    if all(fused) else "mxf4_gemm_smallm_kernel")
+    else:
+        g_kernel = ("mxf4_gemm_pair_kernel (whole layer: quantiser warps rotate and quantise x "
+                    "beside the GEMM)" if all(fused) else "mxf4_gemm_pair_kernel")
     g_src = f"{PKG}/csrc/gemm_smallm.cu" if few_rows else f"{PKG}/csrc/gemm.cu"
     ridge = fp4_peak * 1e12 / (peaks["hbm_gbs"] * 1e9)
     intensity = gemm_flops.sum() / gemm_bytes.sum()

@@ -111,9 +111,11 @@ int64_t mxfp4_sf_offset(int64_t row, int64_t kblock, int64_t K);
  * byte 0), so one workspace can serve calls of different sizes. After it come,
  * for the layer ops, the quantised activations (and the NORM_LINEAR row
  * statistics), then, for 33..128 activation rows, the few-row GEMM's K-split
- * partials (sized for a 148-SM B200). Allocate it zeroed; every other part is
- * written before it is read. With a smaller partial area than this size the
- * few-row GEMM sums its K splits on chip instead (slower, the same bits). */
+ * partials (sized for a 148-SM B200), or, for MXFP4_OP_LINEAR with more than
+ * 128 rows, one 4-byte row counter per 128 rows (the one-kernel layer's; each
+ * call clears them itself). Allocate it zeroed; every other part is written
+ * before it is read. With a smaller partial area than this size the few-row
+ * GEMM sums its K splits on chip instead (slower, the same bits). */
 size_t mxfp4_workspace_bytes(int op, int64_t M, int64_t N, int64_t K);
 
 /* Static description of a status code. Never NULL. */
@@ -235,11 +237,18 @@ mxfp4_status mxfp4_gemm_quantize(const uint8_t* aq, const uint8_t* asf, const ui
  * mxfp4_workspace_bytes(MXFP4_OP_LINEAR, M, N, K) bytes. The two kernels run
  * back to back on `stream`; the GEMM may start loading wq / wsf while the
  * quantiser is still running, so wq / wsf must not overlap the workspace.
- * For 1..8 rows (rotation none, Hadamard-32 or Kronecker, and K splits of at
- * most 12 x 256 elements; see mxfp4_linear_kernel_count) the layer is one
- * kernel: each CTA rotates and quantises its own K range of x into shared
- * memory while it streams the weights. Codes, scales and the result are the
- * same as with the two kernels.
+ * Two sizes run the layer as one kernel instead (rotation none, Hadamard-32 or
+ * Kronecker; see mxfp4_linear_kernel_count):
+ *  - 1..8 rows (K splits of at most 12 x 256 elements): each CTA rotates and
+ *    quantises its own K range of x into shared memory while it streams the
+ *    weights;
+ *  - large problems (more than 128 rows, at least 8 x 74 output tiles of
+ *    256 x 256, x at least 40 MiB): the CTA-pair GEMM with six more warps per
+ *    CTA that rotate and quantise x into the workspace while the other warps
+ *    multiply; each CTA's TMA producer waits, per 128-row group of x, for the
+ *    group's rows to be published (a GPU-scope release and a counter in the
+ *    workspace, cleared by one cudaMemsetAsync before the launch).
+ * Codes, scales and the result are the same in every form.
  */
 mxfp4_status mxfp4_linear(const void* x, int64_t M, int64_t K, mxfp4_rotation mode,
                           const float* kron_a, const float* kron_b, const uint8_t* wq,
@@ -248,13 +257,34 @@ mxfp4_status mxfp4_linear(const void* x, int64_t M, int64_t K, mxfp4_rotation mo
 
 /*
  * How many kernels mxfp4_linear (and mxfp4_linear_noalloc) launch for these
- * sizes and rotation: 1 when the layer runs as one kernel (1..8 rows, mode
- * none / Hadamard-32 / Kronecker, at most 12 k-tiles of 256 elements per K
- * split of the few-row GEMM), 2 otherwise (quantiser, then GEMM), 0 for
- * M == 0, -1 for sizes or a mode that mxfp4_linear rejects. Host only; no
- * GPU is touched.
+ * sizes and rotation: 1 when the layer runs as one kernel (mode none /
+ * Hadamard-32 / Kronecker, and either 1..8 rows with at most 12 k-tiles of
+ * 256 elements per K split of the few-row GEMM, or the large-problem form
+ * above), 2 otherwise (quantiser, then GEMM), 0 for M == 0, -1 for sizes or a
+ * mode that mxfp4_linear rejects. Follows mxfp4_set_linear_form. Host only;
+ * no GPU is touched.
  */
 int mxfp4_linear_kernel_count(int64_t M, int64_t N, int64_t K, mxfp4_rotation mode);
+
+/*
+ * Which form mxfp4_linear and mxfp4_linear_noalloc take where they have a
+ * choice (more than 128 rows, or 1..8 rows within the one-kernel limits; mode
+ * none / Hadamard-32 / Kronecker): MXFP4_LINEAR_AUTO (the state at load time)
+ * chooses by size as described above; MXFP4_LINEAR_ONE_KERNEL takes the
+ * one-kernel form for every problem of more than 128 rows (and keeps the
+ * few-row choice); MXFP4_LINEAR_TWO_KERNELS always quantises and multiplies
+ * in two kernels. Every form gives the same codes, scales and result; this is
+ * for tests that cover both and for measuring them against each other.
+ * Process-wide, read when a call is set up. Unknown values ->
+ * MXFP4_ERR_UNSUPPORTED.
+ */
+typedef enum {
+  MXFP4_LINEAR_AUTO = 0,
+  MXFP4_LINEAR_ONE_KERNEL = 1,
+  MXFP4_LINEAR_TWO_KERNELS = 2
+} mxfp4_linear_form;
+
+mxfp4_status mxfp4_set_linear_form(int form);
 
 /*
  * Norm prologue: the normalisation that precedes the layer, applied inside the
@@ -366,11 +396,12 @@ mxfp4_status mxfp4_nvfp4_linear(const void* x, int64_t M, int64_t K, mxfp4_rotat
  * that loads the library keeps until the process exits. Nothing is allocated
  * per call (no cudaMalloc / cudaFree, no allocating library routine).
  *  - Arguments are checked exactly as mxfp4_linear checks them.
- *  - Limit: 256 + round256(M * K / 2) + round256(mxfp4_sf_bytes(M, K)) must
- *    not exceed the array (about 62 million activation elements); larger
- *    problems return MXFP4_ERR_WORKSPACE and launch nothing. The rest of the
- *    array holds the few-row GEMM's K-split partials when they fit (else it
- *    sums them on chip: slower, the same bits).
+ *  - Limit: 256 + round256(M * K / 2) + round256(mxfp4_sf_bytes(M, K)), plus
+ *    4 bytes per 128 rows for more than 128 rows (the one-kernel form's row
+ *    counters), must not exceed the array (about 62 million activation
+ *    elements); larger problems return MXFP4_ERR_WORKSPACE and launch nothing.
+ *    The rest of the array holds the few-row GEMM's K-split partials when they
+ *    fit (else it sums them on chip: slower, the same bits).
  *  - status: optional DEVICE pointer to a caller-owned, 4-byte aligned int
  *    that the caller zeroes; a bounded-wait timeout sets it to
  *    MXFP4_ERR_TIMEOUT. With NULL the library keeps a status word in its array

@@ -25,6 +25,7 @@ DT_BF16, DT_F32 = 0, 1
 OP_QUANTIZE, OP_GEMM, OP_LINEAR, OP_NVFP4_LINEAR, OP_NORM_LINEAR = 0, 1, 2, 3, 4
 NORM_LAYER, NORM_RMS = 0, 1
 TEST_FAULT_NONE, TEST_FAULT_WITHHOLD_ACCUMULATOR = 0, 1
+LINEAR_AUTO, LINEAR_ONE_KERNEL, LINEAR_TWO_KERNELS = 0, 1, 2
 
 EXPORTS = (
     "mxfp4_sf_bytes", "mxfp4_sf_offset", "mxfp4_workspace_bytes", "mxfp4_status_string",
@@ -33,7 +34,7 @@ EXPORTS = (
     "mxfp4_nvfp4_sf_bytes", "mxfp4_nvfp4_tensor_scale", "mxfp4_nvfp4_quantize",
     "mxfp4_nvfp4_gemm", "mxfp4_nvfp4_linear", "mxfp4_norm_rotate_quantize", "mxfp4_norm_linear",
     "mxfp4_linear_kernel_count", "mxfp4_norm_linear_kernel_count",
-    "mxfp4_kron_weight_factors", "mxfp4_test_set_fault",
+    "mxfp4_kron_weight_factors", "mxfp4_test_set_fault", "mxfp4_set_linear_form",
 )
 
 
@@ -78,6 +79,7 @@ def _load() -> ctypes.CDLL:
         "mxfp4_norm_linear_kernel_count": ([i64, i64, i64, i32], i32),
         "mxfp4_kron_weight_factors": ([vp, vp, vp, vp], i32),
         "mxfp4_test_set_fault": ([i32], i32),
+        "mxfp4_set_linear_form": ([i32], i32),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -423,6 +425,12 @@ def kron_weight_factors(A, B):
     _check(lib.mxfp4_kron_weight_factors(A.ctypes.data, B.ctypes.data, At.ctypes.data,
                                          Bt.ctypes.data), "mxfp4_kron_weight_factors")
     return At, Bt
+
+
+def set_linear_form(form: int) -> None:
+    """Which form linear() / linear_noalloc() take where they have a choice (LINEAR_AUTO,
+    LINEAR_ONE_KERNEL, LINEAR_TWO_KERNELS); see mxfp4_set_linear_form in include/mxfp4.h."""
+    _check(lib.mxfp4_set_linear_form(form), "mxfp4_set_linear_form")
 
 
 def test_set_fault(fault: int) -> None:

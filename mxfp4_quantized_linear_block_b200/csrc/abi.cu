@@ -107,12 +107,14 @@ bool invert_small(const float* a, int n, double* inv) {
 
 namespace mxfp4 {
 
-LinearLayout linear_layout(int64_t M, int64_t N, int64_t K, int64_t sf_k) {
+LinearLayout linear_layout(int64_t M, int64_t N, int64_t K, int64_t sf_k, bool row_counters) {
   LinearLayout w;
   w.q_off = kHeadBytes;
   w.sf_off = round_up(w.q_off + (size_t)M * (size_t)(K / 2), 256);
   w.g_off = round_up(w.sf_off + mxfp4_sf_bytes(M, sf_k), 256);
-  w.total = round_up(w.g_off + gemm_scratch_bytes(M, N, K), 256);
+  size_t last = gemm_scratch_bytes(M, N, K);  // few-row GEMM data (M <= 128)
+  if (row_counters && linear_row_counter_bytes(M) > last) last = linear_row_counter_bytes(M);
+  w.total = round_up(w.g_off + last, 256);
   return w;
 }
 
@@ -157,7 +159,7 @@ size_t mxfp4_workspace_bytes(int op, int64_t M, int64_t N, int64_t K) {
       return kHeadBytes + round_up(gemm_scratch_bytes(M, N, K), 256);
     case MXFP4_OP_LINEAR:
       if (!shape_ok(M, K) || N < 0) return 0;
-      return linear_layout(M, N, K, K).total;
+      return linear_layout(M, N, K, K, true).total;
     case MXFP4_OP_NVFP4_LINEAR:
       if (!shape_ok(M, K) || N < 0) return 0;
       return linear_layout(M, N, K, 2 * K).total;
@@ -281,7 +283,7 @@ mxfp4_status mxfp4_linear(const void* x, int64_t M, int64_t K, mxfp4_rotation mo
   if (st != MXFP4_OK) return st;
   if (!ws) return MXFP4_ERR_INVALID_ARG;
   if (!aligned16(ws)) return MXFP4_ERR_ALIGN;
-  const LinearLayout w = linear_layout(M, N, K, K);
+  const LinearLayout w = linear_layout(M, N, K, K, true);
   if (ws_bytes < w.total) return MXFP4_ERR_WORKSPACE;
   if (M == 0) return MXFP4_OK;
   uint8_t* base = static_cast<uint8_t*>(ws);
@@ -291,6 +293,10 @@ mxfp4_status mxfp4_linear(const void* x, int64_t M, int64_t K, mxfp4_rotation mo
   // 1..8 rows: one kernel quantises x inside the GEMM's CTAs.
   cudaError_t e = launch_linear_smallm(x, K, (int)mode, &kc, wq, wsf, M, N, K, y, N,
                                        static_cast<int*>(ws), s);
+  if (e != cudaErrorNotSupported) return from_cuda(e);
+  // More than 128 rows: one kernel, quantiser warps beside the CTA-pair GEMM.
+  e = launch_linear_pair(x, (int)mode, &kc, xq, xsf, reinterpret_cast<uint32_t*>(base + w.g_off),
+                         wq, wsf, M, N, K, y, static_cast<int*>(ws), s);
   if (e != cudaErrorNotSupported) return from_cuda(e);
   e = launch_rotate_quantize(x, false, M, K, K, (int)mode, &kc, xq, xsf, static_cast<int*>(ws), s);
   if (e != cudaSuccess) return MXFP4_ERR_CUDA;
@@ -305,7 +311,7 @@ int mxfp4_linear_kernel_count(int64_t M, int64_t N, int64_t K, mxfp4_rotation mo
       !within_limits(M, K) || !within_limits(N, K))
     return -1;
   if (M == 0) return 0;
-  return linear_smallm_fits(M, N, K, (int)mode) ? 1 : 2;
+  return linear_smallm_fits(M, N, K, (int)mode) || linear_pair_fits(M, N, K, (int)mode) ? 1 : 2;
 }
 
 int mxfp4_norm_linear_kernel_count(int64_t M, int64_t N, int64_t K, mxfp4_rotation mode) {
@@ -477,6 +483,14 @@ mxfp4_status mxfp4_kron_weight_factors(const float* A, const float* B, float* At
     for (int c = 0; c < 4; ++c) At_inv[r * 4 + c] = (float)ai[c * 4 + r];
   for (int r = 0; r < 8; ++r)
     for (int c = 0; c < 8; ++c) Bt_inv[r * 8 + c] = (float)bi[c * 8 + r];
+  return MXFP4_OK;
+}
+
+mxfp4_status mxfp4_set_linear_form(int form) {
+  if (form != MXFP4_LINEAR_AUTO && form != MXFP4_LINEAR_ONE_KERNEL &&
+      form != MXFP4_LINEAR_TWO_KERNELS)
+    return MXFP4_ERR_UNSUPPORTED;
+  g_linear_form.store(form);
   return MXFP4_OK;
 }
 

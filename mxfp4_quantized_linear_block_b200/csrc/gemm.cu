@@ -47,6 +47,12 @@ constexpr uint32_t kMmaWarp = 1;
 constexpr uint32_t kFirstEpiWarp = 2;
 constexpr uint32_t kEpiWarps = 8;
 constexpr uint32_t kThreads = (kFirstEpiWarp + kEpiWarps) * 32;
+// The one-launch layer adds quantiser warps 10..15 (see fused_quantise_rows): 16 warps,
+// four per SM sub-partition, so every warp keeps up to 128 registers.
+constexpr uint32_t kQuantWarps = 6;
+constexpr uint32_t kFirstQuantWarp = kFirstEpiWarp + kEpiWarps;
+constexpr uint32_t kThreadsFused = (kFirstQuantWarp + kQuantWarps) * 32;
+constexpr uint32_t kQDepth = 3;  // steps of x loads in flight per quantiser lane
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 constexpr int kTimeoutCode = 7;                  // MXFP4_ERR_TIMEOUT
 
@@ -73,6 +79,13 @@ struct Params {
   const float* b_scale;
   uint64_t tfull_wait_ns;  // bound of the epilogue's wait for an accumulator
   uint32_t skip_commit;    // testing only: 1 = pair 0 never signals its first accumulator
+  // One-launch layer: A is quantised from x by the kernel's own quantiser warps.
+  const uint16_t* x;       // bf16 [M, K], row stride K
+  uint8_t* xq;             // A codes (what tmap_a reads)
+  uint8_t* xsf;            // A scales
+  uint32_t* rows_done;     // per 128-row group of A: rows published (zero at launch)
+  uint32_t xmode;          // rotation of x: 0 none, 1 Hadamard-32, 2 Kronecker
+  uint32_t rows_per_item;  // rows per quantiser work item (a power of two, <= 128)
 };
 
 struct Unit {
@@ -106,6 +119,103 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
+}
+
+// ---------------------------------------------------------------- fused quantiser warps
+//
+// The one-launch layer's quantiser: rotate (xmode) and quantise x into the A operand
+// (codes and scales in the tensor-core layout) while the other warps of the grid run
+// the GEMM on the rows already done. Rows go out in items of rows_per_item consecutive
+// rows (an item never crosses a 128-row group), item i to quantiser warp i mod (the
+// grid's quantiser warps), so all warps walk down the rows together, in the order the
+// persistent tile loop asks for them. Lane l handles the 32-element blocks l, l + 32, ...
+// of a row: one step is a 1024-element stretch of one row (the lanes past the row's
+// scale padding idle), and each lane keeps the x loads of the next kQDepth steps in
+// flight in registers. A finished item is published: every lane orders its stores
+// before the async proxy (the GEMM reads the codes with TMA) and fences at GPU scope,
+// then lane 0 adds the item's rows to its group's counter, which the TMA producers wait
+// on. Scale bytes of the K padding (blocks K/32 .. 4 ceil(K/128) - 1) are written 0.
+__device__ __forceinline__ void fused_quantise_rows(const Params& p, const KronCoeffs& kc,
+                                                    uint32_t qwarp, uint32_t n_qwarps,
+                                                    uint32_t lane) {
+  const uint32_t kb_real = p.K / 32u;        // blocks of a row
+  const uint32_t kb_pad = p.k_atoms * 4u;    // scale bytes of a row, K padding included
+  const uint32_t spr = (kb_pad + 31u) / 32u;  // steps per row
+  const uint32_t rpi = p.rows_per_item;
+  const uint32_t n_items = (p.M + rpi - 1u) / rpi;
+  const uint64_t pol = l2_policy_evict_first();  // x is read once
+  struct Cursor {
+    uint32_t item, r, j;  // work item, row within it, step within the row
+  };
+  auto advance = [&](Cursor& c) {
+    if (++c.j == spr) {
+      c.j = 0;
+      if (++c.r == rpi || c.item * rpi + c.r >= p.M) {
+        c.r = 0;
+        c.item += n_qwarps;
+      }
+    }
+  };
+  auto load = [&](const Cursor& c, uint4 (&w)[4]) {
+    const uint32_t kb = c.j * 32u + lane;
+    if (c.item < n_items && kb < kb_real) {
+      const uint4* src =
+          reinterpret_cast<const uint4*>(p.x + (uint64_t)(c.item * rpi + c.r) * p.K + kb * 32u);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) w[q] = ld_nc_v4_hint(src + q, pol);
+    }
+  };
+  Cursor ld{qwarp, 0u, 0u}, cp{qwarp, 0u, 0u};
+  uint4 buf[kQDepth][4];
+#pragma unroll
+  for (uint32_t d = 0; d < kQDepth; ++d) {
+    load(ld, buf[d]);
+    advance(ld);
+  }
+  while (cp.item < n_items) {
+#pragma unroll
+    for (uint32_t d = 0; d < kQDepth; ++d) {
+      if (cp.item >= n_items) break;
+      const uint32_t row = cp.item * rpi + cp.r;
+      const uint32_t kb = cp.j * 32u + lane;
+      const bool has = kb < kb_real;
+      float2 P[16];
+      if (has) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const uint4 w = buf[d][c];
+          P[4 * c + 0] = make_float2(blockq::bf16_lo(w.x), blockq::bf16_hi(w.x));
+          P[4 * c + 1] = make_float2(blockq::bf16_lo(w.y), blockq::bf16_hi(w.y));
+          P[4 * c + 2] = make_float2(blockq::bf16_lo(w.z), blockq::bf16_hi(w.z));
+          P[4 * c + 3] = make_float2(blockq::bf16_lo(w.w), blockq::bf16_hi(w.w));
+        }
+      }
+      load(ld, buf[d]);  // the slot is free again: refill it kQDepth steps ahead
+      advance(ld);
+      uint32_t byte = 0;
+      if (has) {
+        if (p.xmode == 1) blockq::hadamard32(P);
+        if (p.xmode == 2) blockq::kron32(P, kc);
+        uint4 codes;
+        byte = blockq::quantize_block(P, codes);
+        blockq::st_v4(p.xq + (uint64_t)row * (p.K / 2u) + kb * 16u, codes);
+      }
+      // lane 4i writes the scale word of blocks 4i .. 4i + 3 (one word of an atom row)
+      const uint32_t b1 = __shfl_down_sync(0xffffffffu, byte, 1);
+      const uint32_t b2 = __shfl_down_sync(0xffffffffu, byte, 2);
+      const uint32_t b3 = __shfl_down_sync(0xffffffffu, byte, 3);
+      if ((lane & 3u) == 0u && kb < kb_pad)
+        *reinterpret_cast<uint32_t*>(p.xsf + blockq::sf_offset(row, kb, p.k_atoms)) =
+            byte | (b1 << 8) | (b2 << 16) | (b3 << 24);
+      if (cp.j + 1u == spr && (cp.r + 1u == rpi || row + 1u >= p.M)) {  // item done
+        fence_proxy_async_global();
+        __threadfence();
+        __syncwarp();
+        if (lane == 0) atomicAdd(p.rows_done + (row >> 7), cp.r + 1u);
+      }
+      advance(cp);
+    }
+  }
 }
 
 // ---------------------------------------------------------------- CTA-pair kernel
@@ -152,8 +262,8 @@ struct PairConfig {
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
-template <uint32_t STAGES, int OUT, bool NV>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+template <uint32_t STAGES, int OUT, bool NV, bool FQ>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FQ ? kThreadsFused : kThreads, 1)
     mxf4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a,
                           const __grid_constant__ CUtensorMap tmap_b,
                           const __grid_constant__ CUtensorMap tmap_b64,
@@ -220,11 +330,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     if (elect_one()) {
       const uint32_t full_at_leader = map_to_rank(bar_full, 0);
       uint32_t stage = 0, phase = 0, issued = 0;
+      uint32_t ready_group = 0xffffffffu;  // one-launch layer: last A group seen complete
       bool ok = true;
       for (uint32_t u = pair; u < p.units && ok; u += num_pairs) {
         const Unit w = unit_at(u, p);
         const uint32_t mt = w.tile / p.n_tiles, nt = w.tile % p.n_tiles;  // 256-row m tiles
         const int32_t m_cta = (int32_t)(mt * 256u + rank * 128u);
+        if constexpr (FQ) {
+          // This CTA's 128 rows of A come from the grid's quantiser warps: wait until all
+          // of them are published (a group past M has none).
+          const uint32_t g = 2u * mt + rank;
+          const uint32_t left = p.M > 128u * g ? p.M - 128u * g : 0u;
+          if (g != ready_group && left != 0u) {
+            if (!wait_count_bounded(p.rows_done + g, left < 128u ? left : 128u, abort_flag,
+                                    kWaitLimitNs)) {
+              ok = false;
+              break;
+            }
+            fence_proxy_async_global();
+            ready_group = g;
+          }
+        }
         // B rows of this CTA: 128 of the tile's 256, or 64 of a 128-column unit's 128
         const int32_t n_cta =
             (int32_t)(nt * BN + (w.n128 ? w.half * 128u + rank * 64u : rank * 128u));
@@ -336,7 +462,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       volatile int never = 0;
       mbar_wait_bounded(bar_mma_done, 0, &never, kWaitLimitNs);
     }
-  } else {
+  } else if (warp < kFirstQuantWarp) {
     // Epilogue. Warp w owns TMEM lanes 32 * (w % 4) .. +31 and two of the tile's
     // four 64-column chunks; the half-0 warps take the chunk the other
     // accumulator overlaps first and release the accumulator after reading it.
@@ -478,6 +604,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
     if (lane == 0) bulk_wait_all();  // this warp's output stores are complete
     __syncwarp();
+  } else if constexpr (FQ) {
+    fused_quantise_rows(p, kc, blockIdx.x * kQuantWarps + (warp - kFirstQuantWarp),
+                        gridDim.x * kQuantWarps, lane);
   }
 
   tc_fence_before();
@@ -584,11 +713,20 @@ PairPlan pair_plan(int64_t M, int64_t N, uint32_t pairs) {
   return pl;
 }
 
-template <uint32_t STAGES, int OUT, bool NV>
+// The one-launch layer's x (quantised into aq / asf by the kernel itself).
+struct FusedX {
+  const void* x;
+  int mode;
+  uint32_t* rows_done;
+};
+
+template <uint32_t STAGES, int OUT, bool NV, bool FQ = false>
 cudaError_t launch_pair(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq,
                         const uint8_t* bsf, int64_t M, int64_t N, int64_t K, void* y,
-                        const Epilogue& ep, int64_t ldy, int* status, cudaStream_t stream) {
+                        const Epilogue& ep, int64_t ldy, int* status, cudaStream_t stream,
+                        const FusedX* fx = nullptr) {
   using C = PairConfig<STAGES, NV>;
+  constexpr uint32_t threads = FQ ? kThreadsFused : kThreads;
   // scale atoms per 128-row group: one per 4 scales, i.e. per 128 (MXFP4) or 64 (NVFP4) K
   const uint64_t k_atoms = (uint64_t)sf_katoms(NV ? 2 * K : K);
   CUtensorMap ta, tb, tb64, tsa, tsb, ty{};
@@ -600,7 +738,7 @@ cudaError_t launch_pair(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq
       (OUT != kOutMxfp4 &&
        !make_output_map(&ty, y, (uint64_t)M, (uint64_t)N, (uint64_t)ldy, OUT == kOutF32)))
     return cudaErrorInvalidValue;
-  auto kern = mxf4_gemm_pair_kernel<STAGES, OUT, NV>;
+  auto kern = mxf4_gemm_pair_kernel<STAGES, OUT, NV, FQ>;
   int dev = 0;
   cudaGetDevice(&dev);
   static bool attr_done[64] = {};
@@ -612,7 +750,7 @@ cudaError_t launch_pair(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t q{};
     q.gridDim = dim3(2);
-    q.blockDim = dim3(kThreads);
+    q.blockDim = dim3(threads);
     q.dynamicSmemBytes = C::SMEM_BYTES;
     int n = 0;
     if (cudaOccupancyMaxActiveClusters(&n, kern, &q) != cudaSuccess || n <= 0) {
@@ -655,12 +793,29 @@ cudaError_t launch_pair(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq
     p.skip_commit = 1;             // pair 0, first unit
     p.tfull_wait_ns = 1000000ull;  // 1 ms
   }
+  if constexpr (FQ) {
+    p.x = static_cast<const uint16_t*>(fx->x);
+    p.xq = const_cast<uint8_t*>(aq);
+    p.xsf = const_cast<uint8_t*>(asf);
+    p.rows_done = fx->rows_done;
+    p.xmode = (uint32_t)fx->mode;
+  }
   const uint32_t pairs =
       pl.units < (uint32_t)max_clusters[dev] ? pl.units : (uint32_t)max_clusters[dev];
+  if constexpr (FQ) {
+    // Work items of up to about 24 steps of 1024 elements (one publication per item), but
+    // at least four items per quantiser warp, so that the rows the first tiles need are
+    // spread over all the warps and published early.
+    const uint32_t spr = (uint32_t)((k_atoms * 4 + 31) / 32);
+    const uint64_t qwarps = 2ull * pairs * kQuantWarps;
+    uint32_t rpi = 1;
+    while (rpi < 16 && 2 * rpi * spr <= 24 && (uint64_t)M >= 2ull * rpi * 4 * qwarps) rpi *= 2;
+    p.rows_per_item = rpi;
+  }
 
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(2 * pairs);
-  cfg.blockDim = dim3(kThreads);
+  cfg.blockDim = dim3(threads);
   cfg.dynamicSmemBytes = C::SMEM_BYTES;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
@@ -674,6 +829,7 @@ cudaError_t launch_pair(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq
 }  // namespace
 
 std::atomic<int> g_test_fault{MXFP4_TEST_FAULT_NONE};
+std::atomic<int> g_linear_form{MXFP4_LINEAR_AUTO};
 
 cudaError_t launch_gemm(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq,
                         const uint8_t* bsf, int64_t M, int64_t N, int64_t K, void* y,
@@ -699,6 +855,37 @@ cudaError_t launch_gemm(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq
     default:
       return launch_pair<5, kOutBf16, false>(aq, asf, bq, bsf, M, N, K, y, ep, ldy, status, stream);
   }
+}
+
+size_t linear_row_counter_bytes(int64_t M) {
+  return M > 128 ? (size_t)((M + 127) / 128) * sizeof(uint32_t) : 0;
+}
+
+bool linear_pair_fits(int64_t M, int64_t N, int64_t K, int mode) {
+  if (M <= 128 || mode < MXFP4_ROT_NONE || mode > MXFP4_ROT_KRON_4x8) return false;
+  const int form = g_linear_form.load(std::memory_order_relaxed);
+  if (form != MXFP4_LINEAR_AUTO) return form == MXFP4_LINEAR_ONE_KERNEL;
+  // Measured on B200 (DiT-shaped layers, 3584..57344 rows): one kernel is faster once the
+  // tiles fill at least 8 rounds of the 74 CTA pairs and x is at least 40 MiB of bf16;
+  // below that, quantising the rows the first round needs before it can start costs
+  // more than running the quantiser beside the GEMM saves.
+  const int64_t tiles = ((M + 255) / 256) * ((N + 255) / 256);
+  return tiles >= 8 * 74 && 2 * M * K >= (40ll << 20);
+}
+
+cudaError_t launch_linear_pair(const void* x, int mode, const KronCoeffs* kc, uint8_t* xq,
+                               uint8_t* xsf, uint32_t* rows_done, const uint8_t* wq,
+                               const uint8_t* wsf, int64_t M, int64_t N, int64_t K, void* y,
+                               int* status, cudaStream_t stream) {
+  if (!linear_pair_fits(M, N, K, mode)) return cudaErrorNotSupported;
+  // The counters start at zero in every call (a timed-out call may have left them set).
+  cudaError_t e = cudaMemsetAsync(rows_done, 0, linear_row_counter_bytes(M), stream);
+  if (e != cudaSuccess) return e;
+  Epilogue ep{};
+  if (kc) ep.kc = *kc;
+  const FusedX fx{x, mode, rows_done};
+  return launch_pair<5, kOutBf16, false, true>(xq, xsf, wq, wsf, M, N, K, y, ep, N, status,
+                                               stream, &fx);
 }
 
 size_t gemm_scratch_bytes(int64_t M, int64_t N, int64_t K) {

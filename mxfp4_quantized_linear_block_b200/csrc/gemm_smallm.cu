@@ -744,6 +744,7 @@ cudaError_t launch_nt(const Plan& pl, const uint8_t* aq, const uint8_t* asf, con
 
 bool linear_smallm_fits(int64_t M, int64_t N, int64_t K, int mode) {
   if (M < 1 || M > kFxMaxRows || mode < 0 || mode > 2) return false;
+  if (g_linear_form.load(std::memory_order_relaxed) == MXFP4_LINEAR_TWO_KERNELS) return false;
   const Plan pl = make_plan(M, N, K);
   return pl.nt == 16 && pl.kt_per_split <= kFxMaxKt;
 }

@@ -138,6 +138,22 @@ cudaError_t launch_linear_smallm(const void* x, int64_t ldx, int mode, const Kro
                                  int64_t K, void* y, int64_t ldy, int* status,
                                  cudaStream_t stream);
 
+// The whole layer for more than 128 rows in one launch (gemm.cu): the CTA-pair GEMM with
+// six more warps per CTA that rotate (mode 0/1/2) and quantise x into xq / xsf while the
+// other warps multiply; the TMA producer of each CTA waits, per 128-row group of A, for
+// rows_done[group] to reach the group's row count. rows_done: linear_row_counter_bytes(M)
+// bytes, cleared here (one memset) before the launch. Returns cudaErrorNotSupported
+// (launching nothing) when linear_pair_fits is false.
+// linear_pair_fits: whether the layer takes this form (sizes and mode, or the form set by
+// mxfp4_set_linear_form). Host only.
+extern std::atomic<int> g_linear_form;
+bool linear_pair_fits(int64_t M, int64_t N, int64_t K, int mode);
+size_t linear_row_counter_bytes(int64_t M);
+cudaError_t launch_linear_pair(const void* x, int mode, const KronCoeffs* kc, uint8_t* xq,
+                               uint8_t* xsf, uint32_t* rows_done, const uint8_t* wq,
+                               const uint8_t* wsf, int64_t M, int64_t N, int64_t K, void* y,
+                               int* status, cudaStream_t stream);
+
 // Scale-factor layout helpers (host side).
 inline int64_t sf_katoms(int64_t K) { return (K / 32 + 3) / 4; }
 inline int64_t sf_row_tiles(int64_t rows) { return (rows + 127) / 128; }
@@ -182,11 +198,14 @@ mxfp4_status validate_linear(const void* x, int64_t M, int64_t K, mxfp4_rotation
 constexpr size_t kHeadBytes = 256;
 
 // Layout of the layer's workspace: [status | Xq (M x K/2) | Xsf (sf_k-element operand
-// scales) | GEMM data], parts 256-byte aligned. sf_k = K for MXFP4, 2 K for NVFP4.
+// scales) | GEMM data], parts 256-byte aligned. sf_k = K for MXFP4, 2 K for NVFP4. With
+// row_counters (the MXFP4 layer), the last part also holds the one-launch layer's row
+// counters for more than 128 rows (the pair GEMM needs no data there).
 struct LinearLayout {
   size_t q_off, sf_off, g_off, total;
 };
-LinearLayout linear_layout(int64_t M, int64_t N, int64_t K, int64_t sf_k);
+LinearLayout linear_layout(int64_t M, int64_t N, int64_t K, int64_t sf_k,
+                           bool row_counters = false);
 
 // The GEMM scratch of a workspace laid out as above (data part: from g_off to ws_bytes).
 inline GemmScratch workspace_scratch(uint8_t* ws, size_t g_off, size_t ws_bytes) {

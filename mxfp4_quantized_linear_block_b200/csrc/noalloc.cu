@@ -12,7 +12,7 @@
 // The array is a file-scope __device__ variable, so every GPU that loads this
 // part of the library holds it until the process exits. Its size caps the
 // problem: 256 bytes (status region) + round256(M * K / 2) + round256(the scale bytes of
-// X) must fit in it.
+// X), plus 4 bytes per 128 rows of row counters for more than 128 rows, must fit in it.
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -24,10 +24,11 @@ namespace {
 
 constexpr size_t kScratchBytes = MXFP4_NOALLOC_SCRATCH_BYTES;
 
-// Layout: the layer workspace's (status region | Xq | X scales | GEMM data = the rest of
-// the array), parts 256-byte aligned. Each call clears the status region before its first
-// launch, so a status an earlier call left there does not reach it; the other parts are
-// written before they are read.
+// Layout: the layer workspace's (status region | Xq | X scales | GEMM data or the
+// one-launch layer's row counters = the rest of the array), parts 256-byte aligned. Each
+// call clears the status region before its first launch, and the row counters before the
+// launch that uses them, so nothing an earlier call left there reaches it; the other parts
+// are written before they are read.
 static __device__ __align__(256) unsigned char g_linear_scratch[kScratchBytes];
 
 std::mutex g_scratch_mutex;
@@ -64,7 +65,8 @@ extern "C" mxfp4_status mxfp4_linear_noalloc(const void* x, int64_t M, int64_t K
   if (vs != MXFP4_OK) return vs;
   if (status && (reinterpret_cast<uintptr_t>(status) & 3u)) return MXFP4_ERR_ALIGN;
   const LinearLayout w = linear_layout(M, N, K, K);
-  if (w.g_off > kScratchBytes) return MXFP4_ERR_WORKSPACE;  // beyond the fixed capacity
+  if (w.g_off + linear_row_counter_bytes(M) > kScratchBytes)
+    return MXFP4_ERR_WORKSPACE;  // beyond the fixed capacity
   if (M == 0) return MXFP4_OK;
 
   unsigned char* scratch = nullptr;
@@ -80,6 +82,12 @@ extern "C" mxfp4_status mxfp4_linear_noalloc(const void* x, int64_t M, int64_t K
   const cudaError_t fe = launch_linear_smallm(x, K, (int)mode, &kc, wq, wsf, M, N, K, y, N,
                                               status_word, s);
   if (fe != cudaErrorNotSupported) return fe == cudaSuccess ? MXFP4_OK : MXFP4_ERR_CUDA;
+  // More than 128 rows: one kernel, quantiser warps beside the CTA-pair GEMM; its row
+  // counters follow the scales.
+  const cudaError_t pe =
+      launch_linear_pair(x, (int)mode, &kc, xq, xsf, reinterpret_cast<uint32_t*>(scratch + w.g_off),
+                         wq, wsf, M, N, K, y, status_word, s);
+  if (pe != cudaErrorNotSupported) return pe == cudaSuccess ? MXFP4_OK : MXFP4_ERR_CUDA;
   if (launch_rotate_quantize(x, false, M, K, K, (int)mode, &kc, xq, xsf, status_word, s) !=
       cudaSuccess)
     return MXFP4_ERR_CUDA;

@@ -128,6 +128,51 @@ __device__ __forceinline__ void bulk_load_hint(uint32_t dst, const void* src, ui
       : "memory");
 }
 
+// 16-byte global load of data read once (the activations a fused layer quantises): kept
+// out of L2's way with an eviction-priority policy.
+__device__ __forceinline__ uint4 ld_nc_v4_hint(const void* p, uint64_t policy) {
+  uint4 v;
+  asm volatile("ld.global.nc.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p), "l"(policy));
+  return v;
+}
+
+// ------------------------------------------------------------------ cross-CTA hand-over
+//
+// One CTA writes an operand with ordinary stores and another reads it with TMA: the
+// writer orders its stores before the async proxy and publishes with a GPU-scope fence
+// and an atomic add; the reader acquires the count and fences the async proxy before
+// its copies.
+
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Wait until *p >= target, giving up like mbar_wait_bounded.
+__device__ __forceinline__ bool wait_count_bounded(const uint32_t* p, uint32_t target,
+                                                   volatile int* abort_flag, uint64_t limit_ns) {
+  if (ld_acquire_gpu(p) >= target) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t i = 0;; ++i) {
+    __nanosleep(64);
+    if (ld_acquire_gpu(p) >= target) return true;
+    if ((i & 15u) == 15u) {
+      if (*abort_flag) return false;
+      if (global_timer_ns() - t0 > limit_ns) {
+        *abort_flag = 1;
+        return false;
+      }
+    }
+  }
+}
+
 __device__ __forceinline__ void prefetch_tmap(const void* tmap) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(tmap) : "memory");
 }

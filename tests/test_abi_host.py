@@ -48,7 +48,8 @@ def test_workspace_sizes():
     assert mx.workspace_bytes(mx.OP_GEMM, 10, 16, 64) == 256
     M, K = 3584, 3072
     ws = mx.workspace_bytes(mx.OP_LINEAR, M, 9216, K)
-    assert ws == 256 + M * K // 2 + mx.sf_bytes(M, K)
+    # status, codes, scales, and the one-launch layer's row counters (4 bytes per 128 rows)
+    assert ws == 256 + M * K // 2 + mx.sf_bytes(M, K) + 256
 
 
 # Fake device addresses: validation rejects these calls on the host, so nothing is dereferenced.
@@ -155,8 +156,16 @@ def test_empty_calls_accept_null_row_operands():
 
 
 def test_linear_kernel_count():
-    """One kernel for 1..8 rows with rotation 0/1/2 and short K splits, two otherwise."""
+    """One kernel for 1..8 rows with rotation 0/1/2 and short K splits, and for large
+    problems (8 rounds of 256 x 256 tiles on 74 CTA pairs, x of 40 MiB or more); two
+    otherwise."""
     kc = mx.linear_kernel_count
+    assert kc(57344, 12288, 3072, mx.ROT_HADAMARD32) == 1   # 10752 tiles, 336 MiB of x
+    assert kc(57344, 3072, 12288, mx.ROT_KRON_4x8) == 1
+    assert kc(7168, 12288, 3072, mx.ROT_NONE) == 1          # 1344 tiles, 42 MiB
+    assert kc(7168, 3072, 12288, mx.ROT_HADAMARD32) == 2    # 336 tiles: under 8 rounds
+    assert kc(3584, 12288, 3072, mx.ROT_HADAMARD32) == 2    # 21 MiB of x
+    assert kc(57344, 3072, 12288, mx.ROT_HADAMARD64) == 2   # wide groups: two kernels
     assert kc(1, 14336, 4096, mx.ROT_HADAMARD32) == 1
     assert kc(8, 4096, 14336, mx.ROT_KRON_4x8) == 1
     assert kc(4, 128, 256, mx.ROT_NONE) == 1
@@ -201,12 +210,13 @@ def test_gemm_scratch_for_few_rows():
 def test_pair_gemm_needs_no_scratch():
     """The CTA-pair GEMM (more than 128 rows) exchanges nothing between pairs, whatever
     its last round looks like: its workspace is the status region alone, and the layer's
-    adds only the activation codes and scales."""
+    adds the activation codes and scales and one row counter per 128-row group of them."""
+    r256 = lambda v: -(-v // 256) * 256
     for M, N, K in [(2560, 2048, 6144), (4096, 2048, 8192), (57344, 12288, 3072),
                     (3584, 3072, 3072), (129, 16, 64)]:
         assert mx.workspace_bytes(mx.OP_GEMM, M, N, K) == 256
         assert mx.workspace_bytes(mx.OP_LINEAR, M, N, K) == (
-            256 + -(-M * K // 2 // 256) * 256 + -(-mx.sf_bytes(M, K) // 256) * 256)
+            256 + r256(M * K // 2) + r256(mx.sf_bytes(M, K)) + r256(4 * -(-M // 128)))
 
 
 def test_kron_weight_factors_match_oracle():
@@ -262,3 +272,22 @@ def test_kron_weight_factors_closed_forms_and_errors():
 def test_test_fault_hook_arguments():
     assert mx.lib.mxfp4_test_set_fault(7) == mx.ERR_UNSUPPORTED
     assert mx.lib.mxfp4_test_set_fault(mx.TEST_FAULT_NONE) == mx.OK
+
+
+def test_linear_form_control():
+    """mxfp4_set_linear_form overrides the choice by size (host only), and the default is
+    restored."""
+    kc, H = mx.linear_kernel_count, mx.ROT_HADAMARD32
+    try:
+        mx.set_linear_form(mx.LINEAR_ONE_KERNEL)
+        assert kc(129, 16, 64, H) == 1 and kc(3584, 9216, 3072, mx.ROT_KRON_4x8) == 1
+        assert kc(9, 4096, 14336, H) == 2                  # 9..128 rows: no one-kernel form
+        assert kc(57344, 3072, 12288, mx.ROT_HADAMARD128) == 2
+        assert kc(4, 128, 256, mx.ROT_NONE) == 1
+        mx.set_linear_form(mx.LINEAR_TWO_KERNELS)
+        assert kc(57344, 12288, 3072, H) == 2 and kc(4, 128, 256, mx.ROT_NONE) == 2
+    finally:
+        mx.set_linear_form(mx.LINEAR_AUTO)
+    assert kc(57344, 12288, 3072, H) == 1 and kc(4, 128, 256, mx.ROT_NONE) == 1
+    assert mx.lib.mxfp4_set_linear_form(3) == mx.ERR_UNSUPPORTED
+    assert mx.lib.mxfp4_set_linear_form(-1) == mx.ERR_UNSUPPORTED

@@ -265,6 +265,31 @@ def test_linear_guard_cases_reach_both_launch_forms():
     assert counts == {1, 2}, counts
 
 
+@pytest.mark.parametrize("M,K,N,mode", [(129, 64, 16, oracle.ROT_NONE),
+                                        (300, 1024, 384, oracle.ROT_HADAMARD32),
+                                        (700, 160, 2496, oracle.ROT_KRON_4x8),
+                                        (2560, 6144, 2048, oracle.ROT_HADAMARD32)])
+def test_linear_one_kernel_guards(M, K, N, mode):
+    """The layer for more than 128 rows as one kernel (forced here for small sizes): its
+    row counters past the scales and everything around its buffers."""
+    import torch
+    import mxfp4_quantized_linear_block_b200 as mx
+    x = _x_bf16(M + 5 * K, M, K)
+    wq, wsf = _mx_operand(M + 5 * K, N, K, 10)
+    A, B = _kron(8) if mode == oracle.ROT_KRON_4x8 else (None, None)
+
+    def call(ar):
+        y = ar.out("y", M, N, torch.bfloat16)
+        ws = ar.workspace(mx.workspace_bytes(mx.OP_LINEAR, M, N, K))
+        mx.linear(x, wq, wsf, N, mode, A, B, y=y, ws=ws)
+
+    mx.set_linear_form(mx.LINEAR_ONE_KERNEL)
+    try:
+        run_twice(f"one-kernel linear {M}x{K}->{N} mode {mode}", [x, wq, wsf], call)
+    finally:
+        mx.set_linear_form(mx.LINEAR_AUTO)
+
+
 @pytest.mark.parametrize("M,K,N,kind", [(77, 224, 256, 0), (300, 1024, 384, 1),
                                         (3, 53248, 64, 1)])
 def test_norm_linear_guards(M, K, N, kind):

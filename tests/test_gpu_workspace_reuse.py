@@ -49,12 +49,13 @@ def _check(y, x, wq, ws, what, seed):
 
 
 def test_workspace_sizes_of_the_two_calls():
-    """The layer workspace is the status region, the codes and the scales (no GEMM
-    scratch for more than 128 rows)."""
+    """The layer workspace is the status region, the codes, the scales and the row
+    counters of the one-launch layer (no GEMM scratch for more than 128 rows)."""
     import mxfp4_quantized_linear_block_b200 as mx
     for M, K, N in (LARGE, SPLIT):
         assert mx.workspace_bytes(mx.OP_GEMM, M, N, K) == 256
-        assert mx.workspace_bytes(mx.OP_LINEAR, M, N, K) == 256 + M * K // 2 + mx.sf_bytes(M, K)
+        assert mx.workspace_bytes(mx.OP_LINEAR, M, N, K) == (
+            256 + M * K // 2 + mx.sf_bytes(M, K) + -(-4 * -(-M // 128) // 256) * 256)
 
 
 def test_linear_workspace_large_then_split_call():
