@@ -99,6 +99,9 @@ def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--linear-form", default="auto", choices=["auto", "one-kernel", "two-kernels"],
+                    help="form of each layer where the library has a choice (mxfp4_set_linear_"
+                         "form): by size, or forced")
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--attr-steps", type=int, default=200,
                     help="steps of the per-kernel attribution pass (capped at --steps)")
@@ -299,6 +302,8 @@ def run_ours(args, rank, world, local_rank):
 
     import mxfp4_quantized_linear_block_b200 as mx
 
+    mx.set_linear_form({"auto": mx.LINEAR_AUTO, "one-kernel": mx.LINEAR_ONE_KERNEL,
+                        "two-kernels": mx.LINEAR_TWO_KERNELS}[args.linear_form])
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     wl = synth.WORKLOADS[args.workload]
@@ -688,6 +693,8 @@ def run_ours(args, rank, world, local_rank):
                    "tokens_per_gpu": wl.linears[0].M,
                    "gflop_per_step_per_gpu": flops_step / 1e9, "parallelism": f"replicas x{world} "
                    "(token-parallel, no collective)",
+                   "layer_forms": [f"{l.name}: {'one kernel' if kcount[j] == 1 else f'{kcount[j]} kernels'}"
+                                   for j, l in enumerate(wl.linears)],
                    "launch": f"timed steps replayed from CUDA graphs of {U} steps captured from "
                              "mxfp4_linear calls (programmatic dependent launch between kernels)",
                    "l2": f"{len(sets)} rotating input/output sets and {len(wsets)} weight "
@@ -714,7 +721,9 @@ def run_ours(args, rank, world, local_rank):
                                                       if q_traffic else None)}
                               if q_sel else
                               {"fused": True, "note": "x is rotated and quantised inside the "
-                               "layer's one kernel (1..8 rows): no quantiser launch"}),
+                               "layer's one kernel (quantiser warps beside the CTA-pair GEMM "
+                               "for large problems, the few-row GEMM's own CTAs for 1..8 "
+                               "rows): no quantiser launch"}),
         "e2e": e2e,
         "gpu_launches": launches,
         **({"library_gemm": library} if library is not None else {}),

@@ -207,6 +207,11 @@ WORKLOADS = {
         Linear("mlp_down", 3584, 12288, 3072, 2, TID_X + 1, 0.01, 30.0))),
     "kron": Workload("kron", ROT_KRON_4x8, (
         Linear("kron", 3584, 3072, 3072, 0, TID_X, 0.01, 30.0),)),
+    # the DiT block's MLP at batch 4 (14336 tokens): a mid-size case between dit_mlp and
+    # dit_b16, small enough for full profiler captures
+    "dit_b4": Workload("dit_b4", ROT_HADAMARD32, (
+        Linear("mlp_up", 14336, 3072, 12288, 1, TID_X, 0.01, 30.0),
+        Linear("mlp_down", 14336, 12288, 3072, 2, TID_X + 1, 0.01, 30.0))),
     "dit_b16": Workload("dit_b16", ROT_HADAMARD32, (
         Linear("mlp_up", 57344, 3072, 12288, 1, TID_X, 0.01, 30.0),
         Linear("mlp_down", 57344, 12288, 3072, 2, TID_X + 1, 0.01, 30.0))),
