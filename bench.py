@@ -59,9 +59,14 @@ PKG = "mxfp4_quantized_linear_block_b200"
 # ncu flushes L2 before every pass, so reads are cold; output still dirty in L2 when the
 # kernel ends is written back later and is not counted (hence writes < Y bytes).
 NCU_TRAFFIC = {
+    # one-kernel layers (quantiser warps beside the GEMM): x bf16 in, codes written and
+    # read back, Y out
     "dit_b16": {"source": f"{PKG}/csrc/gemm.cu",
-                "sha256": "c85828eea8edddc5ded4db226d7ba778ad3a0bfce965270c0a53781d6f5af657",
-                "bytes_per_launch": [143816210 + 1354265618, 401536420 + 325861138]},
+                "sha256": "f6e74bf76858aa7f5e2a369cbcdefb2b504cb33fe9fbf69d516847d6a08a5755",
+                "bytes_per_launch": [495855616 + 1448034816, 1729230592 + 698682368]},
+    "dit_b4": {"source": f"{PKG}/csrc/gemm.cu",
+               "sha256": "f6e74bf76858aa7f5e2a369cbcdefb2b504cb33fe9fbf69d516847d6a08a5755",
+               "bytes_per_launch": [131513344 + 323793920, 407015424 + 146972928]},
     "dit_b1": {"source": f"{PKG}/csrc/gemm.cu",
                "sha256": "c85828eea8edddc5ded4db226d7ba778ad3a0bfce965270c0a53781d6f5af657",
                "bytes_per_launch": [20928512 + 12389632, 26400256 + 37001984,
