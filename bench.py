@@ -68,9 +68,9 @@ NCU_TRAFFIC = {
                "sha256": "f6e74bf76858aa7f5e2a369cbcdefb2b504cb33fe9fbf69d516847d6a08a5755",
                "bytes_per_launch": [131513344 + 323793920, 407015424 + 146972928]},
     "dit_b1": {"source": f"{PKG}/csrc/gemm.cu",
-               "sha256": "c85828eea8edddc5ded4db226d7ba778ad3a0bfce965270c0a53781d6f5af657",
-               "bytes_per_launch": [20928512 + 12389632, 26400256 + 37001984,
-                                    43516160 + 2887424]},
+               "sha256": "f6e74bf76858aa7f5e2a369cbcdefb2b504cb33fe9fbf69d516847d6a08a5755",
+               "bytes_per_launch": [20930816 + 7372544, 26255872 + 31961600,
+                                    43481600 + 51200]},
     "llm_small_m16": {"source": f"{PKG}/csrc/gemm_smallm.cu",
                       "sha256": "bbb88d371a5c74f77f3a387bb3678bf27b061d3e357a23d24451cf9914d26966",
                       "bytes_per_launch": [31321856 + 0, 31442944 + 0]},
