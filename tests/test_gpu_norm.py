@@ -80,9 +80,10 @@ def _oracle_stats_f32(x, kind, eps):
 
 @pytest.mark.parametrize("kind", [oracle.NORM_LAYER, oracle.NORM_RMS])
 # K <= 51168 takes the one-pass kernel (groups of 16 .. 1 rows per CTA, a partial last group
-# included); K = 65536 the statistics kernel + norm quantiser.
+# included; 16384 and 32768: groups of 2 and 1 rows); K = 65536 the statistics kernel +
+# norm quantiser.
 @pytest.mark.parametrize("rows,K", [(1, 64), (5, 1024), (129, 1024), (17, 4096), (300, 2048),
-                                    (3, 65536)])
+                                    (9, 16384), (3, 32768), (3, 65536)])
 @pytest.mark.parametrize("eps", [0.0, 2.0 ** -12])
 def test_norm_rotate_quantize_exact_rows(kind, rows, K, eps):
     import torch
