@@ -24,6 +24,12 @@
 // in the status word, drains its own copies, releases tensor memory and
 // returns. Problems of at most 128 activation rows go to the weight-streaming
 // kernel in gemm_smallm.cu instead.
+//
+// The same kernel runs a whole layer of more than 128 rows as one launch (FQ):
+//   warps 10..15 quantiser: rotate and quantise x into the A operand in global
+//               memory, publishing rows per 128-row group with a GPU-scope
+//               release and a counter; the producer of each CTA waits for its
+//               group before its first A load of a unit (fused_quantise_rows).
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
