@@ -62,15 +62,15 @@ NCU_TRAFFIC = {
     # one-kernel layers (quantiser warps beside the GEMM): x bf16 in, codes written and
     # read back, Y out
     "dit_b16": {"source": f"{PKG}/csrc/gemm.cu",
-                "sha256": "f6e74bf76858aa7f5e2a369cbcdefb2b504cb33fe9fbf69d516847d6a08a5755",
-                "bytes_per_launch": [495855616 + 1448034816, 1729230592 + 698682368]},
+                "sha256": "5a49545d3732a4c3f75a49a16f5523137cee8fbd1e0de38be05c37807a37ae66",
+                "bytes_per_launch": [510394880 + 1448633088, 1706296320 + 697629696]},
     "dit_b4": {"source": f"{PKG}/csrc/gemm.cu",
-               "sha256": "f6e74bf76858aa7f5e2a369cbcdefb2b504cb33fe9fbf69d516847d6a08a5755",
-               "bytes_per_launch": [131513344 + 323793920, 407015424 + 146972928]},
+               "sha256": "5a49545d3732a4c3f75a49a16f5523137cee8fbd1e0de38be05c37807a37ae66",
+               "bytes_per_launch": [132762112 + 323908608, 403864064 + 144591616]},
     "dit_b1": {"source": f"{PKG}/csrc/gemm.cu",
-               "sha256": "f6e74bf76858aa7f5e2a369cbcdefb2b504cb33fe9fbf69d516847d6a08a5755",
-               "bytes_per_launch": [20930816 + 7372544, 26255872 + 31961600,
-                                    43481600 + 51200]},
+               "sha256": "5a49545d3732a4c3f75a49a16f5523137cee8fbd1e0de38be05c37807a37ae66",
+               "bytes_per_launch": [20923648 + 7406592, 26151424 + 32315904,
+                                    43483136 + 49920]},
     "llm_small_m16": {"source": f"{PKG}/csrc/gemm_smallm.cu",
                       "sha256": "bbb88d371a5c74f77f3a387bb3678bf27b061d3e357a23d24451cf9914d26966",
                       "bytes_per_launch": [31321856 + 0, 31442944 + 0]},
