@@ -22,11 +22,12 @@ def _layer_inputs(wl, lin):
     return x, wq, ws, A, B
 
 
-def _run_linear(x, wq, ws, N, mode, A, B):
+def _run_linear(x, wq, ws, N, mode, A, B, workspace=None):
     import torch
     import mxfp4_quantized_linear_block_b200 as mx
     K = x.shape[1]
-    y = mx.linear(to_dev_bf16(x), to_dev(wq), to_dev(oracle.sf_to_physical(ws, K)), N, mode, A, B)
+    y = mx.linear(to_dev_bf16(x), to_dev(wq), to_dev(oracle.sf_to_physical(ws, K)), N, mode, A, B,
+                  ws=workspace)
     torch.cuda.synchronize()
     return bf16_dev_to_f64(y)
 
@@ -57,13 +58,25 @@ def test_linear_workloads_sampled(name):
 @pytest.mark.parametrize("j", [0, 1])
 def test_linear_batch16_sampled(j):
     """Both layers of the batch-16 DiT MLP at full size (57344 tokens): 3072 -> 12288 and
-    12288 -> 3072, sampled outputs (first and last tiles, edge rows and columns, 8192
-    random) against the oracle's exact products of its own quantisation."""
+    12288 -> 3072, each one kernel (quantiser warps beside the CTA-pair GEMM). Every code
+    and scale byte the quantiser warps leave in the workspace against the oracle's, and
+    sampled outputs (first and last tiles, edge rows and columns, 8192 random) against the
+    oracle's exact products of its own quantisation."""
+    import mxfp4_quantized_linear_block_b200 as mx
     wl = synth.WORKLOADS["dit_b16"]
     lin = wl.linears[j]
+    assert mx.linear_kernel_count(lin.M, lin.N, lin.K, wl.rotation) == 1
     x, wq, ws, A, B = _layer_inputs(wl, lin)
-    y = _run_linear(x, wq, ws, lin.N, wl.rotation, A, B)
+    wsd = mx.new_workspace(mx.workspace_bytes(mx.OP_LINEAR, lin.M, lin.N, lin.K))
+    y = _run_linear(x, wq, ws, lin.N, wl.rotation, A, B, workspace=wsd)
     xq, xs = oracle.rotate_quantize(x, wl.rotation)
+    # workspace: 256-byte status region, the codes, then the scales at the next 256 bytes
+    h = wsd.cpu().numpy()
+    M, K = lin.M, lin.K
+    sf_off = -(-(256 + M * K // 2) // 256) * 256
+    assert np.array_equal(h[256:256 + M * K // 2].reshape(M, K // 2), xq), "codes differ"
+    assert np.array_equal(h[sf_off:sf_off + oracle.sf_bytes(M, K)],
+                          oracle.sf_to_physical(xs, K)), "scale bytes differ"
     mi, ni = _sample_pairs(lin.M, lin.N, n_random=8192, seed=3 + j)
     ref, S = oracle.gemm_pairs(xq, xs, wq, ws, mi, ni)
     check_gemm_values(y[mi, ni], ref, S, "bf16", f"dit_b16/{lin.name}")
