@@ -112,8 +112,8 @@ int64_t mxfp4_sf_offset(int64_t row, int64_t kblock, int64_t K);
  * for the layer ops, the quantised activations (and the NORM_LINEAR row
  * statistics), then, for 33..128 activation rows, the few-row GEMM's K-split
  * partials (sized for a 148-SM B200), or, for MXFP4_OP_LINEAR with more than
- * 128 rows, one 4-byte row counter per 128 rows (the one-kernel layer's; each
- * call clears them itself). Allocate it zeroed; every other part is written
+ * 128 rows, one 4-byte row counter per 128 rows and a 4-byte work-item counter
+ * (the one-kernel layer's; each call clears them itself). Allocate it zeroed; every other part is written
  * before it is read. With a smaller partial area than this size the few-row
  * GEMM sums its K splits on chip instead (slower, the same bits). */
 size_t mxfp4_workspace_bytes(int op, int64_t M, int64_t N, int64_t K);
@@ -247,7 +247,9 @@ mxfp4_status mxfp4_gemm_quantize(const uint8_t* aq, const uint8_t* asf, const ui
  *    CTA that rotate and quantise x into the workspace while the other warps
  *    multiply; each CTA's TMA producer waits, per 128-row group of x, for the
  *    group's rows to be published (a GPU-scope release and a counter in the
- *    workspace, cleared by one cudaMemsetAsync before the launch).
+ *    workspace, cleared by one cudaMemsetAsync before the launch); the quantiser
+ *    warps take their rows from a work-item counter there, so whichever CTAs
+ *    are resident do all of the quantisation.
  * Codes, scales and the result are the same in every form.
  */
 mxfp4_status mxfp4_linear(const void* x, int64_t M, int64_t K, mxfp4_rotation mode,
@@ -397,8 +399,8 @@ mxfp4_status mxfp4_nvfp4_linear(const void* x, int64_t M, int64_t K, mxfp4_rotat
  * per call (no cudaMalloc / cudaFree, no allocating library routine).
  *  - Arguments are checked exactly as mxfp4_linear checks them.
  *  - Limit: 256 + round256(M * K / 2) + round256(mxfp4_sf_bytes(M, K)), plus
- *    4 bytes per 128 rows for more than 128 rows (the one-kernel form's row
- *    counters), must not exceed the array (about 62 million activation
+ *    4 bytes per 128 rows and 4 more for more than 128 rows (the one-kernel
+ *    form's counters), must not exceed the array (about 62 million activation
  *    elements); larger problems return MXFP4_ERR_WORKSPACE and launch nothing.
  *    The rest of the array holds the few-row GEMM's K-split partials when they
  *    fit (else it sums them on chip: slower, the same bits).

@@ -92,6 +92,7 @@ struct Params {
   uint32_t* rows_done;     // per 128-row group of A: rows published (zero at launch)
   uint32_t xmode;          // rotation of x: 0 none, 1 Hadamard-32, 2 Kronecker
   uint32_t rows_per_item;  // rows per quantiser work item (a power of two, <= 128)
+  uint32_t* next_item;     // the next work item to hand out (zero at launch)
 };
 
 struct Unit {
@@ -132,9 +133,10 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 // The one-launch layer's quantiser: rotate (xmode) and quantise x into the A operand
 // (codes and scales in the tensor-core layout) while the other warps of the grid run
 // the GEMM on the rows already done. Rows go out in items of rows_per_item consecutive
-// rows (an item never crosses a 128-row group), item i to quantiser warp i mod (the
-// grid's quantiser warps), so all warps walk down the rows together, in the order the
-// persistent tile loop asks for them. Lane l handles the 32-element blocks l, l + 32, ...
+// rows (an item never crosses a 128-row group), handed out in order by an atomic counter,
+// so the running quantiser warps walk down the rows together, in the order the persistent
+// tile loop asks for them, and do all of them whichever CTAs happen to be resident. Lane l
+// handles the 32-element blocks l, l + 32, ...
 // of a row: one step is a 1024-element stretch of one row (the lanes past the row's
 // scale padding idle), and each lane keeps the x loads of the next kQDepth steps in
 // flight in registers. A finished item is published: every lane orders its stores
@@ -142,7 +144,6 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 // then lane 0 adds the item's rows to its group's counter, which the TMA producers wait
 // on. Scale bytes of the K padding (blocks K/32 .. 4 ceil(K/128) - 1) are written 0.
 __device__ __forceinline__ void fused_quantise_rows(const Params& p, const KronCoeffs& kc,
-                                                    uint32_t qwarp, uint32_t n_qwarps,
                                                     uint32_t lane) {
   const uint32_t kb_real = p.K / 32u;        // blocks of a row
   const uint32_t kb_pad = p.k_atoms * 4u;    // scale bytes of a row, K padding included
@@ -150,15 +151,28 @@ __device__ __forceinline__ void fused_quantise_rows(const Params& p, const KronC
   const uint32_t rpi = p.rows_per_item;
   const uint32_t n_items = (p.M + rpi - 1u) / rpi;
   const uint64_t pol = l2_policy_evict_first();  // x is read once
-  struct Cursor {
-    uint32_t item, r, j;  // work item, row within it, step within the row
+  // The load cursor runs kQDepth steps ahead of the compute cursor, so it takes each item
+  // from the counter first; the items between the two wait in a 4-slot queue kept one per
+  // lane (slot s in lane s: at most kQDepth items lie between the cursors).
+  static_assert(kQDepth <= 3, "the item queue has 4 slots");
+  uint32_t queue = 0;
+  auto grab = [&](uint32_t seq) -> uint32_t {
+    uint32_t it = 0;
+    if (lane == 0) it = atomicAdd(p.next_item, 1u);
+    it = __shfl_sync(0xffffffffu, it, 0);
+    if (lane == (seq & 3u)) queue = it;
+    return it;
   };
-  auto advance = [&](Cursor& c) {
+  struct Cursor {
+    uint32_t item, r, j, seq;  // work item, row within it, step within the row, item number
+  };
+  auto advance = [&](Cursor& c, bool loads) {
     if (++c.j == spr) {
       c.j = 0;
       if (++c.r == rpi || c.item * rpi + c.r >= p.M) {
         c.r = 0;
-        c.item += n_qwarps;
+        ++c.seq;
+        c.item = loads ? grab(c.seq) : __shfl_sync(0xffffffffu, queue, c.seq & 3u);
       }
     }
   };
@@ -171,12 +185,13 @@ __device__ __forceinline__ void fused_quantise_rows(const Params& p, const KronC
       for (int q = 0; q < 4; ++q) w[q] = ld_nc_v4_hint(src + q, pol);
     }
   };
-  Cursor ld{qwarp, 0u, 0u}, cp{qwarp, 0u, 0u};
+  Cursor ld{grab(0u), 0u, 0u, 0u};
+  Cursor cp = ld;
   uint4 buf[kQDepth][4];
 #pragma unroll
   for (uint32_t d = 0; d < kQDepth; ++d) {
     load(ld, buf[d]);
-    advance(ld);
+    advance(ld, true);
   }
   while (cp.item < n_items) {
 #pragma unroll
@@ -197,7 +212,7 @@ __device__ __forceinline__ void fused_quantise_rows(const Params& p, const KronC
         }
       }
       load(ld, buf[d]);  // the slot is free again: refill it kQDepth steps ahead
-      advance(ld);
+      advance(ld, true);
       uint32_t byte = 0;
       if (has) {
         if (p.xmode == 1) blockq::hadamard32(P);
@@ -219,7 +234,7 @@ __device__ __forceinline__ void fused_quantise_rows(const Params& p, const KronC
         __syncwarp();
         if (lane == 0) atomicAdd(p.rows_done + (row >> 7), cp.r + 1u);
       }
-      advance(cp);
+      advance(cp, false);
     }
   }
 }
@@ -611,8 +626,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FQ ? kThreadsFused :
     if (lane == 0) bulk_wait_all();  // this warp's output stores are complete
     __syncwarp();
   } else if constexpr (FQ) {
-    fused_quantise_rows(p, kc, blockIdx.x * kQuantWarps + (warp - kFirstQuantWarp),
-                        gridDim.x * kQuantWarps, lane);
+    fused_quantise_rows(p, kc, lane);
   }
 
   tc_fence_before();
@@ -804,6 +818,7 @@ cudaError_t launch_pair(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq
     p.xq = const_cast<uint8_t*>(aq);
     p.xsf = const_cast<uint8_t*>(asf);
     p.rows_done = fx->rows_done;
+    p.next_item = fx->rows_done + (M + 127) / 128;  // the word after the row counters
     p.xmode = (uint32_t)fx->mode;
   }
   const uint32_t pairs =
@@ -864,7 +879,8 @@ cudaError_t launch_gemm(const uint8_t* aq, const uint8_t* asf, const uint8_t* bq
 }
 
 size_t linear_row_counter_bytes(int64_t M) {
-  return M > 128 ? (size_t)((M + 127) / 128) * sizeof(uint32_t) : 0;
+  // one counter per 128 rows, then the quantiser's next work item
+  return M > 128 ? (size_t)((M + 127) / 128 + 1) * sizeof(uint32_t) : 0;
 }
 
 bool linear_pair_fits(int64_t M, int64_t N, int64_t K, int mode) {

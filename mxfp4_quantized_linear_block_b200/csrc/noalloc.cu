@@ -12,7 +12,8 @@
 // The array is a file-scope __device__ variable, so every GPU that loads this
 // part of the library holds it until the process exits. Its size caps the
 // problem: 256 bytes (status region) + round256(M * K / 2) + round256(the scale bytes of
-// X), plus 4 bytes per 128 rows of row counters for more than 128 rows, must fit in it.
+// X), plus 4 bytes per 128 rows and 4 more (the one-kernel form's counters) for more than
+// 128 rows, must fit in it.
 #include <cuda_runtime.h>
 
 #include <cstdint>

@@ -210,13 +210,14 @@ def test_gemm_scratch_for_few_rows():
 def test_pair_gemm_needs_no_scratch():
     """The CTA-pair GEMM (more than 128 rows) exchanges nothing between pairs, whatever
     its last round looks like: its workspace is the status region alone, and the layer's
-    adds the activation codes and scales and one row counter per 128-row group of them."""
+    adds the activation codes and scales, one row counter per 128-row group of them and
+    the one-kernel form's work-item counter."""
     r256 = lambda v: -(-v // 256) * 256
     for M, N, K in [(2560, 2048, 6144), (4096, 2048, 8192), (57344, 12288, 3072),
                     (3584, 3072, 3072), (129, 16, 64)]:
         assert mx.workspace_bytes(mx.OP_GEMM, M, N, K) == 256
         assert mx.workspace_bytes(mx.OP_LINEAR, M, N, K) == (
-            256 + r256(M * K // 2) + r256(mx.sf_bytes(M, K)) + r256(4 * -(-M // 128)))
+            256 + r256(M * K // 2) + r256(mx.sf_bytes(M, K)) + r256(4 * (-(-M // 128) + 1)))
 
 
 def test_kron_weight_factors_match_oracle():

@@ -55,7 +55,7 @@ def test_workspace_sizes_of_the_two_calls():
     for M, K, N in (LARGE, SPLIT):
         assert mx.workspace_bytes(mx.OP_GEMM, M, N, K) == 256
         assert mx.workspace_bytes(mx.OP_LINEAR, M, N, K) == (
-            256 + M * K // 2 + mx.sf_bytes(M, K) + -(-4 * -(-M // 128) // 256) * 256)
+            256 + M * K // 2 + mx.sf_bytes(M, K) + -(-4 * (-(-M // 128) + 1) // 256) * 256)
 
 
 def test_linear_workspace_large_then_split_call():
