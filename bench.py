@@ -62,15 +62,15 @@ NCU_TRAFFIC = {
     # one-kernel layers (quantiser warps beside the GEMM): x bf16 in, codes written and
     # read back, Y out
     "dit_b16": {"source": f"{PKG}/csrc/gemm.cu",
-                "sha256": "5a49545d3732a4c3f75a49a16f5523137cee8fbd1e0de38be05c37807a37ae66",
-                "bytes_per_launch": [510394880 + 1448633088, 1706296320 + 697629696]},
+                "sha256": "12f8da48d77476a66b875dce8dfc816345624329cc29b5288a8939e5a09d053f",
+                "bytes_per_launch": [505209344 + 1448007936, 1741553152 + 700484864]},
     "dit_b4": {"source": f"{PKG}/csrc/gemm.cu",
-               "sha256": "5a49545d3732a4c3f75a49a16f5523137cee8fbd1e0de38be05c37807a37ae66",
-               "bytes_per_launch": [132762112 + 323908608, 403864064 + 144591616]},
+               "sha256": "12f8da48d77476a66b875dce8dfc816345624329cc29b5288a8939e5a09d053f",
+               "bytes_per_launch": [133406208 + 324511744, 400334848 + 142204672]},
     "dit_b1": {"source": f"{PKG}/csrc/gemm.cu",
-               "sha256": "5a49545d3732a4c3f75a49a16f5523137cee8fbd1e0de38be05c37807a37ae66",
-               "bytes_per_launch": [20923648 + 7406592, 26151424 + 32315904,
-                                    43483136 + 49920]},
+               "sha256": "12f8da48d77476a66b875dce8dfc816345624329cc29b5288a8939e5a09d053f",
+               "bytes_per_launch": [20935424 + 7750912, 26691072 + 32043008,
+                                    43485184 + 876288]},
     "llm_small_m16": {"source": f"{PKG}/csrc/gemm_smallm.cu",
                       "sha256": "bbb88d371a5c74f77f3a387bb3678bf27b061d3e357a23d24451cf9914d26966",
                       "bytes_per_launch": [31321856 + 0, 31442944 + 0]},
