@@ -292,3 +292,13 @@ def test_linear_form_control():
     assert kc(57344, 12288, 3072, H) == 1 and kc(4, 128, 256, mx.ROT_NONE) == 1
     assert mx.lib.mxfp4_set_linear_form(3) == mx.ERR_UNSUPPORTED
     assert mx.lib.mxfp4_set_linear_form(-1) == mx.ERR_UNSUPPORTED
+
+
+def test_one_kernel_size_rule_boundaries():
+    """The large-problem one-kernel form needs at least 8 x 74 = 592 output tiles of
+    256 x 256 and at least 40 MiB of bf16 x (M K >= 20971520): both edges exactly."""
+    kc, H = mx.linear_kernel_count, mx.ROT_HADAMARD32
+    assert kc(4096, 9472, 5120, H) == 1   # 16 x 37 = 592 tiles, M K = 20971520
+    assert kc(4096, 9472, 5088, H) == 2   # M K one 32-block column short
+    assert kc(4096, 9216, 5120, H) == 2   # 16 x 36 = 576 tiles
+    assert kc(4096, 9472, 5120, mx.ROT_HADAMARD64) == 2  # wide groups: two kernels
