@@ -437,8 +437,11 @@ def run_ours(args, rank, world, local_rank):
     # device, so the timed steps run back to back (the sleep itself is not timed).
     torch.cuda._sleep(int(2e7))
     ev0.record(stream)
-    for _ in range(n_main):
+    # an event after every graph of U steps as well: the spread of the step time
+    ev_graph = [torch.cuda.Event(enable_timing=True) for _ in range(n_main)]
+    for i in range(n_main):
         g_main.replay()
+        ev_graph[i].record(stream)
     if g_rest is not None:
         g_rest.replay()
     ev1.record(stream)
@@ -446,6 +449,11 @@ def run_ours(args, rank, world, local_rank):
     barrier()
     clk = clocks.stop()
     elapsed = max_over_ranks(ev0.elapsed_time(ev1) * 1e-3)
+    per_graph = [(ev_graph[i].elapsed_time(ev_graph[i + 1]) if i + 1 < n_main else None)
+                 for i in range(n_main)]
+    per_graph = [ev0.elapsed_time(ev_graph[0])] + [t for t in per_graph if t is not None] \
+        if n_main else []
+    step_ms = np.array(per_graph, np.float64) / min(U, args.steps)
     flops_step = wl.flops
     value = job_tflops(flops_step, args.steps, world, elapsed)
     ms_per_step = elapsed / args.steps * 1e3
@@ -734,6 +742,12 @@ def run_ours(args, rank, world, local_rank):
                                   if any(fused) else {})}),
         "e2e": e2e,
         "gpu_launches": launches,
+        "step_ms_spread": {"median": float(np.median(step_ms)),
+                           "p10": float(np.percentile(step_ms, 10)),
+                           "p90": float(np.percentile(step_ms, 90)),
+                           "graphs": int(step_ms.size), "steps_per_graph": int(min(U, args.steps)),
+                           "note": "per replayed graph of steps (rank 0), from CUDA events "
+                                   "between the replays inside the timed region"},
         **({"library_gemm": library} if library is not None else {}),
         "attribution": {"launches_per_graph": n_attr,
                         "note": "per linear, one CUDA graph of back-to-back quantiser launches "
