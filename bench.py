@@ -14,11 +14,14 @@ in HBM; the timed steps are replayed from CUDA graphs captured from the same
 ``mxfp4_linear`` calls. ``e2e`` = the same metric through the same public call from host
 buffers (pinned H2D of X and D2H of Y inside the timed region, each direction on a copy
 stream of its own, double-buffered so that copies overlap the layers of other steps). ``roofline`` =
-the GEMM kernel (the largest share of every step) against the FP4 tensor peak,
-or against HBM bandwidth when its arithmetic intensity is below the ridge (few
-tokens); ``quantize_roofline`` = the rotate+quantise kernel against HBM
-bandwidth; both from CUDA events around each kernel launch in an attribution
-pass over the same steps.
+the GEMM kernel (the largest share of every step; for layers that run as one kernel,
+that kernel, quantisation included) against the FP4 tensor peak, or against HBM
+bandwidth when its arithmetic intensity is below the ridge (few tokens);
+``quantize_roofline`` = the rotate+quantise kernel against HBM bandwidth (the
+standalone kernel on the same activations when the layers quantise inside their one
+kernel); both from CUDA events around each kernel launch in an attribution pass over
+the same steps. ``step_ms_spread`` = median / p10 / p90 of the step time over the
+replayed graphs of the timed region.
 
 --impl reference times the CPU oracle (the plain C implementation that
 defines the results) on a bounded row sample of the same workload.
