@@ -65,15 +65,15 @@ NCU_TRAFFIC = {
     # one-kernel layers (quantiser warps beside the GEMM): x bf16 in, codes written and
     # read back, Y out
     "dit_b16": {"source": f"{PKG}/csrc/gemm.cu",
-                "sha256": "12f8da48d77476a66b875dce8dfc816345624329cc29b5288a8939e5a09d053f",
-                "bytes_per_launch": [505209344 + 1448007936, 1741553152 + 700484864]},
+                "sha256": "a41af15780f8b18448d08bf791b9ca1b3d44b286808452e35d00e2d835e9df1a",
+                "bytes_per_launch": [486365440 + 1446813440, 1610452992 + 697108992]},
     "dit_b4": {"source": f"{PKG}/csrc/gemm.cu",
-               "sha256": "12f8da48d77476a66b875dce8dfc816345624329cc29b5288a8939e5a09d053f",
-               "bytes_per_launch": [133406208 + 324511744, 400334848 + 142204672]},
+               "sha256": "a41af15780f8b18448d08bf791b9ca1b3d44b286808452e35d00e2d835e9df1a",
+               "bytes_per_launch": [130578432 + 326460416, 391931904 + 142951424]},
     "dit_b1": {"source": f"{PKG}/csrc/gemm.cu",
-               "sha256": "12f8da48d77476a66b875dce8dfc816345624329cc29b5288a8939e5a09d053f",
-               "bytes_per_launch": [20935424 + 7750912, 26691072 + 32043008,
-                                    43485184 + 876288]},
+               "sha256": "a41af15780f8b18448d08bf791b9ca1b3d44b286808452e35d00e2d835e9df1a",
+               "bytes_per_launch": [20928768 + 8118528, 26286336 + 32677888,
+                                    43485184 + 938752]},
     "llm_small_m16": {"source": f"{PKG}/csrc/gemm_smallm.cu",
                       "sha256": "bbb88d371a5c74f77f3a387bb3678bf27b061d3e357a23d24451cf9914d26966",
                       "bytes_per_launch": [31321856 + 0, 31442944 + 0]},

@@ -58,7 +58,7 @@ constexpr uint32_t kThreads = (kFirstEpiWarp + kEpiWarps) * 32;
 constexpr uint32_t kQuantWarps = 6;
 constexpr uint32_t kFirstQuantWarp = kFirstEpiWarp + kEpiWarps;
 constexpr uint32_t kThreadsFused = (kFirstQuantWarp + kQuantWarps) * 32;
-constexpr uint32_t kQDepth = 3;  // steps of x loads in flight per quantiser lane
+constexpr uint32_t kQDepth = 2;  // steps of x loads in flight per quantiser lane
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 constexpr int kTimeoutCode = 7;                  // MXFP4_ERR_TIMEOUT
 
