@@ -120,6 +120,10 @@ def parse():
                     help="nvfp4: 16-element groups with E4M3 scales and a dynamic fp32 tensor "
                          "scale per activation (mxfp4_nvfp4_linear); rotation none or "
                          "Hadamard-32 only")
+    ap.add_argument("--nvfp4-scale", default="dynamic", choices=["dynamic", "static"],
+                    help="with --format nvfp4: the activation tensor scale from each x "
+                         "(dynamic: three kernels per layer) or one calibrated beforehand "
+                         "(static: mxfp4_nvfp4_linear_static, two kernels)")
     ap.add_argument("--norm", default="none", choices=["none", "layer", "rms"],
                     help="apply a LayerNorm / RMSNorm prologue (with per-channel g and b) "
                          "inside the quantiser: mxfp4_norm_linear")
@@ -377,14 +381,26 @@ def run_ours(args, rank, world, local_rank):
     footprint = len(sets) * set_bytes(sets[0]) + len(wsets) * w_bytes
 
     stream = torch.cuda.current_stream(dev)
+    # NVFP4 with a static activation scale: one scale per linear, calibrated once (untimed)
+    # on the first input set, as a deployment would calibrate it offline
+    static_nv = nv and args.nvfp4_scale == "static"
+    x_static = ([mx.nvfp4_tensor_scale(sets[0][0][l.x_tensor], wl.rotation) for l in wl.linears]
+                if static_nv else None)
+
+    def nv_layer(x, j, wq, wsf, wsc, y, ws, s):
+        lin = wl.linears[j]
+        if static_nv:
+            mx.nvfp4_linear_static(x, x_static[j], wq, wsf, wsc, lin.N, wl.rotation, y=y,
+                                   ws=ws, stream=s)
+        else:
+            mx.nvfp4_linear(x, wq, wsf, wsc, lin.N, wl.rotation, y=y, ws=ws, stream=s)
 
     def step(i, s=stream):
         xs, ys, wss = sets[i % len(sets)]
         for j, lin in enumerate(wl.linears):
             wq, wsf, wsc = wsets[i % len(wsets)][j]
             if nv:
-                mx.nvfp4_linear(xs[lin.x_tensor], wq, wsf, wsc, lin.N, wl.rotation, y=ys[j],
-                                ws=wss[j], stream=s)
+                nv_layer(xs[lin.x_tensor], j, wq, wsf, wsc, ys[j], wss[j], s)
             elif norm is not None:
                 mx.norm_linear(xs[lin.x_tensor], wq, wsf, lin.N, norm, 1e-6, norm_gb[j][0],
                                norm_gb[j][1], wl.rotation, A, B, y=ys[j], ws=wss[j], stream=s)
@@ -464,7 +480,7 @@ def run_ours(args, rank, world, local_rank):
     # the GEMM's CTAs (1..8 rows); NVFP4 adds the tensor-scale pass (1 kernel); the norm
     # prologue is one kernel with the quantiser while a row fits in shared memory, else it
     # adds the row-statistics kernel
-    kcount = [3 if nv else
+    kcount = [(2 if static_nv else 3) if nv else
               mx.norm_linear_kernel_count(l.M, l.N, l.K, wl.rotation) if norm is not None else
               mx.linear_kernel_count(l.M, l.N, l.K, wl.rotation) for l in wl.linears]
     fused = [k == 1 for k in kcount]
@@ -499,7 +515,10 @@ def run_ours(args, rank, world, local_rank):
         lin = wl.linears[j]
         q, sf, xsc, stt = qbufs[i % nq][j]
         if nv:
-            mx.nvfp4_tensor_scale(xs[lin.x_tensor], wl.rotation, scale2=xsc, stream=s)
+            if static_nv:
+                xsc = x_static[j]
+            else:
+                mx.nvfp4_tensor_scale(xs[lin.x_tensor], wl.rotation, scale2=xsc, stream=s)
             mx.nvfp4_quantize(xs[lin.x_tensor], xsc, wl.rotation, q=q, sf=sf, stream=s)
         elif norm is not None:
             mx.norm_rotate_quantize(xs[lin.x_tensor], norm, 1e-6, norm_gb[j][0], norm_gb[j][1],
@@ -517,8 +536,8 @@ def run_ours(args, rank, world, local_rank):
             return
         q, sf, xsc, _ = qbufs[i % nq][j]
         if nv:
-            mx.nvfp4_gemm(q, sf, xsc, wq, wsf, wsc, lin.M, lin.N, lin.K, y=ys[j], ws=gws[j],
-                          stream=s)
+            mx.nvfp4_gemm(q, sf, x_static[j] if static_nv else xsc, wq, wsf, wsc, lin.M, lin.N,
+                          lin.K, y=ys[j], ws=gws[j], stream=s)
         else:
             mx.gemm(q, sf, wq, wsf, lin.M, lin.N, lin.K, y=ys[j], ws=gws[j], stream=s)
 
@@ -562,7 +581,8 @@ def run_ours(args, rank, world, local_rank):
                            for j, l in enumerate(wl.linears)], np.float64)
     # NVFP4's dynamic tensor scale, and the norm's row statistics when they are a kernel of
     # their own, need a full pass over X before the quantiser reads it
-    q_bytes = np.array([(4 if nv or (norm is not None and kcount[j] == 3) else 2) * l.M * l.K +
+    q_bytes = np.array([(4 if (nv and not static_nv) or (norm is not None and kcount[j] == 3)
+                         else 2) * l.M * l.K +
                         l.M * l.K // 2 + sfb(l.M, l.K) for j, l in enumerate(wl.linears)],
                        np.float64)
     # The FP4 ceiling is derived from the measured bf16 one: its burst figure for a timed
@@ -653,8 +673,7 @@ def run_ours(args, rank, world, local_rank):
             for j, lin in enumerate(wl.linears):
                 wq, wsf, wsc = wsets[i % len(wsets)][j]
                 if nv:
-                    mx.nvfp4_linear(xs_d[lin.x_tensor], wq, wsf, wsc, lin.N, wl.rotation,
-                                    y=ys_d[j], ws=wss_d[j], stream=stream)
+                    nv_layer(xs_d[lin.x_tensor], j, wq, wsf, wsc, ys_d[j], wss_d[j], stream)
                 elif norm is not None:
                     mx.norm_linear(xs_d[lin.x_tensor], wq, wsf, lin.N, norm, 1e-6,
                                    norm_gb[j][0], norm_gb[j][1], wl.rotation, A, B, y=ys_d[j],
@@ -699,8 +718,9 @@ def run_ours(args, rank, world, local_rank):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": args.format,
-        "dtype_detail": ("E2M1 x E2M1 with E4M3 group-16 scales and fp32 tensor scales (dynamic "
-                         "for X), fp32 accumulate, bf16 out; rotation in fp32" if nv else
+        "dtype_detail": ("E2M1 x E2M1 with E4M3 group-16 scales and fp32 tensor scales ("
+                         + ("static, calibrated once," if static_nv else "dynamic") +
+                         " for X), fp32 accumulate, bf16 out; rotation in fp32" if nv else
                          "E2M1 x E2M1 with E8M0 block-32 scales, fp32 accumulate, bf16 out; "
                          "rotation in fp32"),
         "data": "synthetic (seeded N(0,1) activations with outlier channels, N(0,0.02^2) weights)",
@@ -718,7 +738,9 @@ def run_ours(args, rank, world, local_rank):
                          f"({l2 / 2**20:.0f} MiB)"},
         "roofline": roofline,
         "quantize_roofline": ({"bound": "hbm",
-                               "kernel": ("nvfp4_amax_kernel + rotate_quantize_kernel" if nv else
+                               "kernel": (("rotate_quantize_kernel (static tensor scale)"
+                                           if static_nv else
+                                           "nvfp4_amax_kernel + rotate_quantize_kernel") if nv else
                                           "; ".join(
                                               f"{l.name}: " + ("norm_rows_kernel (one pass)"
                                                                if kcount[j] == 2 else

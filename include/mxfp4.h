@@ -381,6 +381,20 @@ mxfp4_status mxfp4_nvfp4_linear(const void* x, int64_t M, int64_t K, mxfp4_rotat
                                 int64_t N, void* y, void* ws, size_t ws_bytes,
                                 mxfp4_stream_t stream);
 
+/* The NVFP4 layer with a static activation tensor scale (one calibrated offline, for
+ * instance): x is quantised with *x_scale (DEVICE fp32, 4-byte aligned; the
+ * quantisation rule of mxfp4_nvfp4_quantize with st = *x_scale) instead of a scale
+ * taken from x, so the layer is two kernels, the quantiser and the GEMM, and x is read
+ * once ("Bridging the Gap...", "Methodologie: MR-GPTQ" item 2: tensor and group
+ * scales). Groups whose amax / (6 st) exceeds 448 saturate at group scale 448; st = 0
+ * gives zero codes. Everything else as mxfp4_nvfp4_linear; x_scale must not be written
+ * by the layer's own workspace. */
+mxfp4_status mxfp4_nvfp4_linear_static(const void* x, int64_t M, int64_t K,
+                                       mxfp4_rotation mode, const float* x_scale,
+                                       const uint8_t* wq, const uint8_t* wsf,
+                                       const float* w_scale, int64_t N, void* y, void* ws,
+                                       size_t ws_bytes, mxfp4_stream_t stream);
+
 /* Size in bytes of the device scratch array that mxfp4_linear_noalloc uses (per GPU). */
 #define MXFP4_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
 

@@ -35,6 +35,7 @@ EXPORTS = (
     "mxfp4_nvfp4_gemm", "mxfp4_nvfp4_linear", "mxfp4_norm_rotate_quantize", "mxfp4_norm_linear",
     "mxfp4_linear_kernel_count", "mxfp4_norm_linear_kernel_count",
     "mxfp4_kron_weight_factors", "mxfp4_test_set_fault", "mxfp4_set_linear_form",
+    "mxfp4_nvfp4_linear_static",
 )
 
 
@@ -71,6 +72,8 @@ def _load() -> ctypes.CDLL:
         "mxfp4_nvfp4_gemm": ([vp, vp, vp, vp, vp, vp, i64, i64, i64, vp, i32, i64, vp, sz, vp],
                              i32),
         "mxfp4_nvfp4_linear": ([vp, i64, i64, i32, vp, vp, vp, i64, vp, vp, sz, vp], i32),
+        "mxfp4_nvfp4_linear_static": ([vp, i64, i64, i32, vp, vp, vp, vp, i64, vp, vp, sz, vp],
+                                      i32),
         "mxfp4_norm_rotate_quantize": ([vp, i64, i64, i64, i32, ctypes.c_float, vp, vp, i32, vp,
                                         vp, vp, vp, vp, vp], i32),
         "mxfp4_norm_linear": ([vp, i64, i64, i32, ctypes.c_float, vp, vp, i32, vp, vp, vp, vp,
@@ -354,6 +357,25 @@ def nvfp4_linear(x, wq, wsf, w_scale, N: int, mode: int = ROT_NONE, y=None, ws=N
                                 w_scale.data_ptr(), N, y.data_ptr(), ws.data_ptr(), ws.numel(),
                                 _stream_handle(stream))
     _check(st, "mxfp4_nvfp4_linear")
+    return y
+
+
+def nvfp4_linear_static(x, x_scale, wq, wsf, w_scale, N: int, mode: int = ROT_NONE, y=None,
+                        ws=None, stream=None):
+    """The NVFP4 layer with a static activation tensor scale (x_scale: a device fp32 tensor
+    whose first element is the scale): quantise x with it, GEMM (bf16 out); two kernels."""
+    torch = _torch()
+    assert x.dim() == 2 and x.is_contiguous() and x.dtype == torch.bfloat16
+    M, K = x.shape
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    if ws is None:
+        ws = new_workspace(workspace_bytes(OP_NVFP4_LINEAR, M, N, K), x.device)
+    st = lib.mxfp4_nvfp4_linear_static(x.data_ptr(), M, K, mode, x_scale.data_ptr(),
+                                       wq.data_ptr(), wsf.data_ptr(), w_scale.data_ptr(), N,
+                                       y.data_ptr(), ws.data_ptr(), ws.numel(),
+                                       _stream_handle(stream))
+    _check(st, "mxfp4_nvfp4_linear_static")
     return y
 
 

@@ -15,6 +15,23 @@ namespace {
 
 mxfp4_status from_cuda(cudaError_t e) { return e == cudaSuccess ? MXFP4_OK : MXFP4_ERR_CUDA; }
 
+// Checks shared by the two NVFP4 layer entry points.
+mxfp4_status validate_nvfp4_linear(const void* x, int64_t M, int64_t K, mxfp4_rotation mode,
+                                   const uint8_t* wq, const uint8_t* wsf, const float* w_scale,
+                                   int64_t N, const void* y, const void* ws, size_t ws_bytes) {
+  if (!rows_ptr_ok(x, M) || !wq || !wsf || !w_scale || !rows_ptr_ok(y, M) || !ws)
+    return MXFP4_ERR_INVALID_ARG;
+  if (mode != MXFP4_ROT_NONE && mode != MXFP4_ROT_HADAMARD32) return MXFP4_ERR_UNSUPPORTED;
+  if (!shape_ok(M, K) || N < 16 || N % 16 != 0 || !within_limits(M, 2 * K) ||
+      !within_limits(N, 2 * K))
+    return MXFP4_ERR_SHAPE;
+  if (!aligned16(x) || !aligned16(wq) || !aligned16(wsf) || !aligned16(y) || !aligned16(ws) ||
+      (K * 2) % 16 != 0 || (N * 2) % 16 != 0 || (reinterpret_cast<uintptr_t>(w_scale) & 3u))
+    return MXFP4_ERR_ALIGN;
+  if (ws_bytes < linear_layout(M, N, K, 2 * K).total) return MXFP4_ERR_WORKSPACE;
+  return MXFP4_OK;
+}
+
 mxfp4_status validate_quantize(const void* x, mxfp4_dtype xdt, int64_t rows, int64_t K,
                                int64_t ldx, const uint8_t* q, const uint8_t* sf) {
   if (!rows_ptr_ok(x, rows) || !rows_ptr_ok(q, rows) || !rows_ptr_ok(sf, rows))
@@ -436,21 +453,41 @@ mxfp4_status mxfp4_nvfp4_gemm(const uint8_t* aq, const uint8_t* asf, const float
                                static_cast<cudaStream_t>(stream)));
 }
 
+mxfp4_status mxfp4_nvfp4_linear_static(const void* x, int64_t M, int64_t K,
+                                       mxfp4_rotation mode, const float* x_scale,
+                                       const uint8_t* wq, const uint8_t* wsf,
+                                       const float* w_scale, int64_t N, void* y, void* ws,
+                                       size_t ws_bytes, mxfp4_stream_t stream) {
+  if (!x_scale) return MXFP4_ERR_INVALID_ARG;
+  const mxfp4_status vs = validate_nvfp4_linear(x, M, K, mode, wq, wsf, w_scale, N, y, ws,
+                                                ws_bytes);
+  if (vs != MXFP4_OK) return vs;
+  if (reinterpret_cast<uintptr_t>(x_scale) & 3u) return MXFP4_ERR_ALIGN;
+  if (M == 0) return MXFP4_OK;
+  const LinearLayout w = linear_layout(M, N, K, 2 * K);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_nvfp4_quantize(x, false, M, K, K, (int)mode, x_scale, base + w.q_off,
+                                        base + w.sf_off, static_cast<int*>(ws), s);
+  if (e != cudaSuccess) return MXFP4_ERR_CUDA;
+  Epilogue ep;
+  ep.nvfp4 = true;
+  ep.a_scale = x_scale;
+  ep.b_scale = w_scale;
+  // The kernel just before the GEMM is the quantiser above, which does not write W.
+  return from_cuda(launch_gemm(base + w.q_off, base + w.sf_off, wq, wsf, M, N, K, y, ep, N,
+                               static_cast<int*>(ws), workspace_scratch(base, w.g_off, ws_bytes),
+                               true, s));
+}
+
 mxfp4_status mxfp4_nvfp4_linear(const void* x, int64_t M, int64_t K, mxfp4_rotation mode,
                                 const uint8_t* wq, const uint8_t* wsf, const float* w_scale,
                                 int64_t N, void* y, void* ws, size_t ws_bytes,
                                 mxfp4_stream_t stream) {
-  if (!rows_ptr_ok(x, M) || !wq || !wsf || !w_scale || !rows_ptr_ok(y, M) || !ws)
-    return MXFP4_ERR_INVALID_ARG;
-  if (mode != MXFP4_ROT_NONE && mode != MXFP4_ROT_HADAMARD32) return MXFP4_ERR_UNSUPPORTED;
-  if (!shape_ok(M, K) || N < 16 || N % 16 != 0 || !within_limits(M, 2 * K) ||
-      !within_limits(N, 2 * K))
-    return MXFP4_ERR_SHAPE;
-  if (!aligned16(x) || !aligned16(wq) || !aligned16(wsf) || !aligned16(y) || !aligned16(ws) ||
-      (K * 2) % 16 != 0 || (N * 2) % 16 != 0 || (reinterpret_cast<uintptr_t>(w_scale) & 3u))
-    return MXFP4_ERR_ALIGN;
+  const mxfp4_status vs = validate_nvfp4_linear(x, M, K, mode, wq, wsf, w_scale, N, y, ws,
+                                                ws_bytes);
+  if (vs != MXFP4_OK) return vs;
   const LinearLayout w = linear_layout(M, N, K, 2 * K);
-  if (ws_bytes < w.total) return MXFP4_ERR_WORKSPACE;
   if (M == 0) return MXFP4_OK;
   uint8_t* base = static_cast<uint8_t*>(ws);
   float* xs = reinterpret_cast<float*>(base + kScaleOff);

@@ -302,3 +302,25 @@ def test_one_kernel_size_rule_boundaries():
     assert kc(4096, 9472, 5088, H) == 2   # M K one 32-block column short
     assert kc(4096, 9216, 5120, H) == 2   # 16 x 36 = 576 tiles
     assert kc(4096, 9472, 5120, mx.ROT_HADAMARD64) == 2  # wide groups: two kernels
+
+
+def test_nvfp4_static_scale_argument_errors():
+    """mxfp4_nvfp4_linear_static: the static activation scale must be given and 4-byte
+    aligned; the rest is checked as for mxfp4_nvfp4_linear (all on the host, nothing
+    launched); an empty call is valid."""
+    L = mx.lib
+    ws = mx.workspace_bytes(mx.OP_NVFP4_LINEAR, 4, 32, 64)
+    assert L.mxfp4_nvfp4_linear_static(P, 4, 64, 0, None, P, P, P, 32, P, P, ws, None) == \
+        mx.ERR_INVALID_ARG
+    assert L.mxfp4_nvfp4_linear_static(P, 4, 64, 0, P + 2, P, P, P, 32, P, P, ws, None) == \
+        mx.ERR_ALIGN
+    assert L.mxfp4_nvfp4_linear_static(P, 4, 64, 2, P, P, P, P, 32, P, P, ws, None) == \
+        mx.ERR_UNSUPPORTED
+    assert L.mxfp4_nvfp4_linear_static(P, 4, 48, 0, P, P, P, P, 32, P, P, ws, None) == \
+        mx.ERR_SHAPE
+    assert L.mxfp4_nvfp4_linear_static(P, 4, 64, 0, P, P, P, P, 32, P, P, ws - 16, None) == \
+        mx.ERR_WORKSPACE
+    assert L.mxfp4_nvfp4_linear_static(P, 4, 64, 0, P, P, P, None, 32, P, P, ws, None) == \
+        mx.ERR_INVALID_ARG
+    assert L.mxfp4_nvfp4_linear_static(None, 0, 64, 1, P, P, P, P, 32, None, P, ws, None) == \
+        mx.OK

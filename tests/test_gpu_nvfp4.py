@@ -126,6 +126,49 @@ def test_nvfp4_linear(mode, M):
     check_gemm_values(bf16_dev_to_f64(y), ref, S, "bf16", f"nvfp4 linear M{M} mode {mode}")
 
 
+@pytest.mark.parametrize("mode", MODES)
+@pytest.mark.parametrize("M", [16, 300])
+@pytest.mark.parametrize("factor", [0.25, 1.0, 4.0])
+def test_nvfp4_linear_static_scale(mode, M, factor):
+    """The NVFP4 layer with a static activation tensor scale: the dynamic scale of x times
+    `factor` (0.25: many groups saturate at group scale 448; 4: finer groups), given on
+    the device; against the oracle's quantisation with that same scale."""
+    import torch
+    import mxfp4_quantized_linear_block_b200 as mx
+    K, N = 1024, 512
+    x, _ = synth.activation_bf16(M + 2, M, K, 0.01, 30.0)
+    w = synth.weight_f32(4, N, K, 6)
+    w_d = torch.from_numpy(w).cuda()
+    w_sc = mx.nvfp4_tensor_scale(w_d, mode)
+    wq, wsf = mx.nvfp4_quantize(w_d, w_sc, mode)
+    st_x = np.float32(np.float32(oracle.nvfp4_tensor_scale(x, mode)) * np.float32(factor))
+    x_sc = torch.tensor([float(st_x), 0.0], dtype=torch.float32, device="cuda")
+    y = mx.nvfp4_linear_static(to_dev_bf16(x), x_sc, wq, wsf, w_sc, N, mode)
+    torch.cuda.synchronize()
+    st_w = oracle.nvfp4_tensor_scale(w, mode)
+    wq_r, ws_r = oracle.nvfp4_rotate_quantize(w, mode, st_w)
+    xq_r, xs_r = oracle.nvfp4_rotate_quantize(x, mode, st_x)
+    alpha = float(np.float32(st_x) * np.float32(st_w))
+    ref, S = oracle.nvfp4_gemm(xq_r, xs_r, wq_r, ws_r, alpha)
+    check_gemm_values(bf16_dev_to_f64(y), ref, S, "bf16",
+                      f"nvfp4 static-scale linear M{M} mode {mode} x{factor}")
+
+
+def test_nvfp4_linear_static_zero_scale():
+    """A static activation scale of 0 gives zero codes, so a zero output."""
+    import torch
+    import mxfp4_quantized_linear_block_b200 as mx
+    M, K, N = 40, 256, 128
+    x, _ = synth.activation_bf16(5, M, K, 0.01, 30.0)
+    w_d = torch.from_numpy(synth.weight_f32(5, N, K, 6)).cuda()
+    w_sc = mx.nvfp4_tensor_scale(w_d, oracle.ROT_NONE)
+    wq, wsf = mx.nvfp4_quantize(w_d, w_sc, oracle.ROT_NONE)
+    x_sc = torch.zeros(2, dtype=torch.float32, device="cuda")
+    y = mx.nvfp4_linear_static(to_dev_bf16(x), x_sc, wq, wsf, w_sc, N, oracle.ROT_NONE)
+    torch.cuda.synchronize()
+    assert not bool(y.float().abs().max() > 0)
+
+
 def test_nvfp4_linear_repeated_on_one_workspace():
     """The layer's tensor-scale pass keeps its running maximum and block counter in the
     workspace and leaves them zero: a call whose x has a smaller amax than the one before
