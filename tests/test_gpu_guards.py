@@ -328,6 +328,26 @@ def test_nvfp4_linear_guards(M, K, N):
     run_twice(f"nvfp4_linear {M}x{K}->{N}", [x, wq, wsf, wsc], call)
 
 
+@pytest.mark.parametrize("M,K,N", [(5, 256, 128), (300, 1024, 384)])
+def test_nvfp4_linear_static_guards(M, K, N):
+    """The NVFP4 layer with a static activation scale (two kernels)."""
+    import torch
+    import mxfp4_quantized_linear_block_b200 as mx
+    x = _x_bf16(M * 19 + K, M, K)
+    wq = _dev(synth.uniform_u8(M + K, synth.TID_CODES + 43, (N, K // 2), 0, 255))
+    wsf = _dev(oracle.nvfp4_sf_to_physical(
+        synth.uniform_u8(M + K, synth.TID_SCALES + 43, (N, K // 16), 24, 80), K))
+    wsc = torch.tensor([0.5, 0.0], dtype=torch.float32, device="cuda")
+    xsc = torch.tensor([0.125, 0.0], dtype=torch.float32, device="cuda")
+
+    def call(ar):
+        y = ar.out("y", M, N, torch.bfloat16)
+        ws = ar.workspace(mx.workspace_bytes(mx.OP_NVFP4_LINEAR, M, N, K))
+        mx.nvfp4_linear_static(x, xsc, wq, wsf, wsc, N, mx.ROT_HADAMARD32, y=y, ws=ws)
+
+    run_twice(f"nvfp4_linear_static {M}x{K}->{N}", [x, wq, wsf, wsc, xsc], call)
+
+
 @pytest.mark.parametrize("M,K,N", [(5, 512, 256), (300, 1024, 384)])
 def test_linear_noalloc_guards(M, K, N):
     import torch
