@@ -150,6 +150,18 @@ def load_peaks():
             "source": "fallback"}
 
 
+def fp4_ceiling(peaks: dict, elapsed: float):
+    """The dense FP4 ceiling for a timed region of `elapsed` seconds, derived from the
+    measured bf16 one (x FP4_OVER_BF16): its burst figure for a region shorter than a second
+    (clocks still at their boost), the figure sustained under the power cap for a longer
+    one. Returns (TFLOP/s, the line's peak_source text)."""
+    sustained = elapsed >= 1.0
+    bf16 = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
+    src = (f"4 x {peaks['source']} bf16 {'sustained' if sustained else 'burst'} "
+           f"({bf16} TFLOP/s); timed region {elapsed:.3f} s")
+    return bf16 * FP4_OVER_BF16, src
+
+
 def workload_desc(wl) -> str:
     parts = [f"{l.name} {l.M}x{l.K}->{l.N}" for l in wl.linears]
     rot = {0: "no rotation", 1: "Hadamard-32", 2: "Kronecker 4x8"}[wl.rotation]
@@ -585,12 +597,7 @@ def run_ours(args, rank, world, local_rank):
                          else 2) * l.M * l.K +
                         l.M * l.K // 2 + sfb(l.M, l.K) for j, l in enumerate(wl.linears)],
                        np.float64)
-    # The FP4 ceiling is derived from the measured bf16 one: its burst figure for a timed
-    # region shorter than a second (clocks still at their boost), the figure sustained
-    # under the power cap for a longer one.
-    sustained = elapsed >= 1.0
-    bf16_peak = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
-    fp4_peak = bf16_peak * FP4_OVER_BF16
+    fp4_peak, fp4_src = fp4_ceiling(peaks, elapsed)
     q_sel = list(range(n_lin))
     q_ach = q_bytes[q_sel].sum() / t_q[q_sel].sum() / 1e9 if q_sel else None
     # The GEMM dominates every workload's step. It is tensor-bound when its arithmetic
@@ -616,10 +623,7 @@ def run_ours(args, rank, world, local_rank):
     t_dom = elapsed / args.steps if all(fused) else t_g.sum()
     if intensity >= ridge:
         roofline = {"bound": "tensor", "achieved": gemm_flops.sum() / t_dom / 1e12,
-                    "peak": fp4_peak, "unit": "TFLOP/s",
-                    "peak_source": f"4 x {peaks['source']} bf16 "
-                                   f"{'sustained' if sustained else 'burst'} ({bf16_peak} "
-                                   f"TFLOP/s); timed region {elapsed:.3f} s"}
+                    "peak": fp4_peak, "unit": "TFLOP/s", "peak_source": fp4_src}
     else:
         roofline = {"bound": "hbm", "achieved": gemm_bytes.sum() / t_dom / 1e9,
                     "peak": peaks["hbm_gbs"], "unit": "GB/s",
@@ -967,12 +971,7 @@ def run_chain(args, rank, world, local_rank):
     t_g = np.array([np.mean([e[j + 1].elapsed_time(e[j + 2]) * 1e-3 for e in evs])
                     for j in range(len(L))])
     flops = np.array([l.flops for l in L], np.float64)
-    # The FP4 ceiling is derived from the measured bf16 one: its burst figure for a timed
-    # region shorter than a second (clocks still at their boost), the figure sustained
-    # under the power cap for a longer one.
-    sustained = elapsed >= 1.0
-    bf16_peak = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
-    fp4_peak = bf16_peak * FP4_OVER_BF16
+    fp4_peak, fp4_src = fp4_ceiling(peaks, elapsed)
     # algorithmic bytes of each GEMM: its MXFP4 input and weight, and its output (MXFP4
     # codes + scales between layers, bf16 after the last)
     g_bytes = np.array([l.M * l.K // 2 + mx.sf_bytes(l.M, l.K) + l.N * l.K // 2 +
@@ -983,8 +982,7 @@ def run_chain(args, rank, world, local_rank):
     intensity = flops.sum() / g_bytes.sum()
     if intensity >= ridge:
         roof = {"bound": "tensor", "achieved": flops.sum() / t_g.sum() / 1e12, "peak": fp4_peak,
-                "unit": "TFLOP/s", "peak_source": f"4 x {peaks['source']} bf16 sustained "
-                                                  f"({peaks['bf16_tflops_sustained']} TFLOP/s)"}
+                "unit": "TFLOP/s", "peak_source": fp4_src}
     else:
         roof = {"bound": "hbm", "achieved": g_bytes.sum() / t_g.sum() / 1e9,
                 "peak": peaks["hbm_gbs"], "unit": "GB/s",

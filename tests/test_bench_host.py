@@ -1,0 +1,62 @@
+"""Host arithmetic of bench.py that the JSON line's roofline rests on, on CPU: which FP4
+ceiling a timed region is held against, where the peaks come from, when recorded DRAM
+traffic is still valid, and the whole-job throughput formula."""
+import json
+import os
+
+import pytest
+
+import bench
+
+PEAKS = {"hbm_gbs": 6000.0, "bf16_tflops": 1600.0, "bf16_tflops_sustained": 1300.0,
+         "source": "measured"}
+
+
+@pytest.mark.parametrize("elapsed, bf16, word", [(0.04, 1600.0, "burst"),
+                                                 (0.999, 1600.0, "burst"),
+                                                 (1.0, 1300.0, "sustained"),
+                                                 (6.5, 1300.0, "sustained")])
+def test_fp4_ceiling_by_region_length(elapsed, bf16, word):
+    peak, src = bench.fp4_ceiling(PEAKS, elapsed)
+    assert peak == 4.0 * bf16  # dense FP4 : bf16 = 9 : 2.25 PFLOP/s
+    assert f"bf16 {word} ({bf16} TFLOP/s)" in src and src.startswith("4 x measured")
+    assert f"timed region {elapsed:.3f} s" in src
+
+
+def test_peaks_file_or_fallback():
+    p = bench.load_peaks()
+    path = os.path.join(bench.ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            m = json.load(f)
+        assert p["source"] == "measured"
+        assert (p["hbm_gbs"], p["bf16_tflops"], p["bf16_tflops_sustained"]) == \
+            (m["hbm_gbs"], m["bf16_tflops"], m["bf16_tflops_sustained"])
+    else:
+        assert p == {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                     "source": "fallback"}
+
+
+def test_traffic_only_for_the_source_it_was_taken_on():
+    src = "bench.py"
+    good = {"w": {"source": src, "sha256": bench.source_sha256(src), "bytes_per_launch": [7]}}
+    stale = {"w": {"source": src, "sha256": "0" * 64, "bytes_per_launch": [7]}}
+    assert bench.ncu_traffic("w", src, good)["bytes_per_launch"] == [7]
+    assert bench.ncu_traffic("w", src, stale) is None
+    assert bench.ncu_traffic("w", "oracle/__init__.py", good) is None  # another kernel's file
+    assert bench.ncu_traffic("other", src, good) is None
+
+
+def test_traffic_table_entries_are_well_formed():
+    for table in (bench.NCU_TRAFFIC, bench.NCU_TRAFFIC_QUANTIZE):
+        for name, e in table.items():
+            wl = bench.synth.WORKLOADS[name]
+            assert os.path.exists(os.path.join(bench.ROOT, e["source"]))
+            assert len(e["sha256"]) == 64
+            assert len(e["bytes_per_launch"]) == len(wl.linears)
+            assert all(b > 0 for b in e["bytes_per_launch"])
+
+
+def test_job_tflops():
+    # 2 ranks x 10 steps x 1e12 FLOP over the slowest rank's 4 s
+    assert bench.job_tflops(1e12, 10, 2, 4.0) == pytest.approx(5.0)
