@@ -72,9 +72,9 @@ struct SmallConfig {
   static constexpr uint32_t XSF_BYTES = FX ? kFxMaxKt * SF_STAGE : 0;
   // Up to 64 tokens two CTAs per SM: as many stages (at most 5) as let 2 x SMEM_BYTES fit
   // an SM's shared memory (233472 bytes, 1 KB of it reserved per CTA). 128 tokens: one
-  // CTA per SM with up to 12 stages, so that half as many K splits keep the same bytes in
-  // flight (B200, 128 x 14336 <-> 4096: 12.4 / 12.6 -> 11.8 / 11.0 us; at 1 and 16 tokens
-  // the same change cost 0.2-0.8 us, the sums being small there).
+  // CTA per SM with as many stages as fit (6 of the 12 allowed), so that half as many K
+  // splits keep the same bytes in flight (B200, 128 x 14336 <-> 4096: 12.4 / 12.6 -> 11.8 /
+  // 11.0 us; at 1 and 16 tokens the same change cost 0.2-0.8 us, the sums being small there).
   static constexpr bool WIDE = NT == 128;
   static constexpr uint32_t STAGE_BYTES = A_STAGE + B_STAGE + (FX ? 1 : 2) * SF_STAGE;
   static constexpr uint32_t BUDGET =
