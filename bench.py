@@ -74,12 +74,16 @@ NCU_TRAFFIC = {
                "sha256": "a41af15780f8b18448d08bf791b9ca1b3d44b286808452e35d00e2d835e9df1a",
                "bytes_per_launch": [20928768 + 8118528, 26286336 + 32677888,
                                     43485184 + 938752]},
+    # few-row layers: the weight stream (codes and scales) read once per launch
+    "llm_small_m1": {"source": f"{PKG}/csrc/gemm_smallm.cu",
+                     "sha256": "c1a5856ae3b89278695761ee6fea9183eaca35a89aa5ed2d29be07339156fcbd",
+                     "bytes_per_launch": [31289344 + 0, 31300864 + 0]},
     "llm_small_m16": {"source": f"{PKG}/csrc/gemm_smallm.cu",
-                      "sha256": "bbb88d371a5c74f77f3a387bb3678bf27b061d3e357a23d24451cf9914d26966",
-                      "bytes_per_launch": [31321856 + 0, 31442944 + 0]},
+                      "sha256": "c1a5856ae3b89278695761ee6fea9183eaca35a89aa5ed2d29be07339156fcbd",
+                      "bytes_per_launch": [31327488 + 0, 31444480 + 2560]},
     "llm_small_m128": {"source": f"{PKG}/csrc/gemm_smallm.cu",
-                       "sha256": "bbb88d371a5c74f77f3a387bb3678bf27b061d3e357a23d24451cf9914d26966",
-                       "bytes_per_launch": [31556864 + 0, 32239104 + 4608]},
+                       "sha256": "c1a5856ae3b89278695761ee6fea9183eaca35a89aa5ed2d29be07339156fcbd",
+                       "bytes_per_launch": [31561216 + 0, 32240128 + 0]},
 }
 NCU_TRAFFIC_QUANTIZE = {
     "dit_b16": {"source": f"{PKG}/csrc/quantize.cu",
