@@ -324,3 +324,36 @@ def test_nvfp4_static_scale_argument_errors():
         mx.ERR_INVALID_ARG
     assert L.mxfp4_nvfp4_linear_static(None, 0, 64, 1, P, P, P, P, 32, None, P, ws, None) == \
         mx.OK
+
+
+def test_empty_calls_of_the_epilogue_norm_and_nvfp4_layers():
+    """With no rows the remaining entry points validate their arguments and return OK
+    without launching anything (so no device is touched here); the row operands may be
+    NULL, the weight operands, scales and workspace stay required."""
+    L = mx.lib
+    ws = mx.workspace_bytes(mx.OP_GEMM, 0, 32, 64)
+    assert L.mxfp4_gemm_bias(None, None, P, P, 0, 32, 64, P, None, 0, 32, P, ws, None) == mx.OK
+    assert L.mxfp4_gemm_bias(None, None, P, P, 0, 32, 64, None, None, 0, 32, P, ws, None) == \
+        mx.ERR_INVALID_ARG  # the bias stays required
+    assert L.mxfp4_gemm_quantize(None, None, P, P, 0, 32, 64, None, 1, None, None, None, None, P,
+                                 ws, None) == mx.OK
+    assert L.mxfp4_gemm_quantize(None, None, None, P, 0, 32, 64, None, 1, None, None, None, None,
+                                 P, ws, None) == mx.ERR_INVALID_ARG
+    assert L.mxfp4_norm_rotate_quantize(None, 0, 64, 64, mx.NORM_LAYER, 1e-6, None, None, 1, None,
+                                        None, None, None, P, None) == mx.OK
+    assert L.mxfp4_norm_rotate_quantize(None, 0, 64, 64, mx.NORM_LAYER, 1e-6, None, None, 1, None,
+                                        None, None, None, None, None) == mx.ERR_INVALID_ARG
+    wsn = mx.workspace_bytes(mx.OP_NORM_LINEAR, 0, 32, 64)
+    assert L.mxfp4_norm_linear(None, 0, 64, mx.NORM_RMS, 1e-6, None, None, 1, None, None, P, P,
+                               32, None, P, wsn, None) == mx.OK
+    assert L.mxfp4_nvfp4_quantize(None, 0, 0, 64, 64, 1, P, None, None, None) == mx.OK
+    assert L.mxfp4_nvfp4_quantize(None, 0, 0, 64, 64, 1, None, None, None, None) == \
+        mx.ERR_INVALID_ARG  # the tensor scale stays required
+    assert L.mxfp4_nvfp4_gemm(None, None, P, P, P, P, 0, 32, 64, None, 0, 32, P, ws,
+                              None) == mx.OK
+    wsv = mx.workspace_bytes(mx.OP_NVFP4_LINEAR, 0, 32, 64)
+    assert L.mxfp4_nvfp4_linear(None, 0, 64, 1, P, P, P, 32, None, P, wsv, None) == mx.OK
+    assert L.mxfp4_nvfp4_linear_static(None, 0, 64, 1, P, P, P, P, 32, None, P, wsv,
+                                       None) == mx.OK
+    assert L.mxfp4_nvfp4_linear_static(None, 0, 64, 1, None, P, P, P, 32, None, P, wsv,
+                                       None) == mx.ERR_INVALID_ARG
