@@ -169,6 +169,21 @@ def test_nvfp4_linear_static_zero_scale():
     assert not bool(y.float().abs().max() > 0)
 
 
+def test_nvfp4_tensor_scale_of_empty_and_zero_tensors():
+    """amax of no elements, or of zeros only, is 0, so the tensor scale is 0 (written over
+    whatever the 2-float buffer held, by the pass's one block when there are no rows)."""
+    import torch
+    import mxfp4_quantized_linear_block_b200 as mx
+    for rows in (0, 3):
+        for mode in (oracle.ROT_NONE, oracle.ROT_HADAMARD32):
+            for dt in (torch.bfloat16, torch.float32):
+                x = torch.zeros((rows, 96), dtype=dt, device="cuda")
+                sc = torch.full((2,), 7.5, dtype=torch.float32, device="cuda")
+                mx.nvfp4_tensor_scale(x, mode, scale2=sc)
+                torch.cuda.synchronize()
+                assert float(sc[0]) == 0.0, (rows, mode, dt)
+
+
 def test_nvfp4_linear_repeated_on_one_workspace():
     """The layer's tensor-scale pass keeps its running maximum and block counter in the
     workspace and leaves them zero: a call whose x has a smaller amax than the one before
