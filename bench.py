@@ -238,16 +238,70 @@ def cpu_cores() -> int:
 # --------------------------------------------------------------------------- clocks
 
 class ClockSampler:
+    """SM clock and throttle reasons of this rank's GPU while the timed region runs.
+
+    NVML is polled every 5 ms from a thread, and only the samples taken between the
+    host-side start and end of the region are kept, so that a region of a few tens of
+    milliseconds still has samples of its own. Where NVML cannot be loaded, nvidia-smi's
+    200-ms loop is read instead (every sample it wrote). Only reads: nothing is set."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+    PERIOD_S = 0.005
 
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
         self.proc = None
         self.path = None
+        self.thread = None
+        self.samples = []  # NVML: (host time, sm MHz, reason names)
 
-    def start(self):
+    # -- NVML
+    def _nvml_handle(self, nv):
+        try:
+            import torch
+            pr = torch.cuda.get_device_properties(torch.cuda.current_device())
+            bus = f"{pr.pci_domain_id:08X}:{pr.pci_bus_id:02X}:{pr.pci_device_id:02X}.0"
+            return nv.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:
+            return nv.nvmlDeviceGetHandleByIndex(self.gpu)
+
+    def _start_nvml(self) -> bool:
+        import threading
+        try:
+            import pynvml as nv
+            nv.nvmlInit()
+        except Exception:
+            return False
+        try:
+            h = self._nvml_handle(nv)
+            self.sm_max = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+            masks = (nv.nvmlClocksEventReasonHwSlowdown, nv.nvmlClocksEventReasonHwThermalSlowdown,
+                     nv.nvmlClocksEventReasonSwThermalSlowdown, nv.nvmlClocksEventReasonSwPowerCap)
+        except Exception:
+            nv.nvmlShutdown()
+            return False
+        self.nv, self.stop_flag = nv, threading.Event()
+
+        def poll():
+            while not self.stop_flag.is_set():
+                try:
+                    t = time.perf_counter()
+                    mhz = float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+                    bits = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                    self.samples.append((t, mhz,
+                                         tuple(n for n, m in zip(self.NAMES, masks) if bits & m)))
+                except Exception:
+                    pass
+                self.stop_flag.wait(self.PERIOD_S)
+
+        self.thread = threading.Thread(target=poll, daemon=True)
+        self.thread.start()
+        return True
+
+    # -- nvidia-smi
+    def _start_smi(self):
         fd, self.path = tempfile.mkstemp(suffix=".csv")
         os.close(fd)
         try:
@@ -258,7 +312,27 @@ class ClockSampler:
         except Exception:
             self.proc = None
 
-    def stop(self):
+    def start(self):
+        if not self._start_nvml():
+            self._start_smi()
+
+    def stop(self, t0: float = None, t1: float = None):
+        """Summary of the samples; with NVML, of those taken between host times t0 and t1
+        (time.perf_counter) when given."""
+        if self.thread is not None:
+            self.stop_flag.set()
+            self.thread.join(timeout=5)
+            try:
+                self.nv.nvmlShutdown()
+            except Exception:
+                pass
+            rows = [r for r in self.samples
+                    if (t0 is None or r[0] >= t0) and (t1 is None or r[0] <= t1)]
+            if not rows:
+                return None
+            return {"sm_mhz": statistics.median(r[1] for r in rows), "sm_max_mhz": self.sm_max,
+                    "reasons": sorted({n for r in rows for n in r[2]}), "samples": len(rows),
+                    "source": "nvml, every 5 ms"}
         if self.proc is None:
             return None
         self.proc.terminate()
@@ -277,11 +351,11 @@ class ClockSampler:
             return None
         sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
         smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        reasons = sorted({self.NAMES[i] for r in rows for i in range(4)
+                          if r[5 + i].lower() == "active"})
         return {"sm_mhz": statistics.median(sm) if sm else None,
                 "sm_max_mhz": max(smax) if smax else None,
-                "reasons": reasons, "samples": len(rows)}
+                "reasons": reasons, "samples": len(rows), "source": "nvidia-smi, every 200 ms"}
 
 
 # --------------------------------------------------------------------------- GPU arm
@@ -470,6 +544,7 @@ def run_ours(args, rank, world, local_rank):
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     # A short GPU sleep ahead of the first event lets the host queue launches ahead of the
     # device, so the timed steps run back to back (the sleep itself is not timed).
+    t_host0 = time.perf_counter()
     torch.cuda._sleep(int(2e7))
     ev0.record(stream)
     # an event after every graph of U steps as well: the spread of the step time
@@ -481,8 +556,9 @@ def run_ours(args, rank, world, local_rank):
         g_rest.replay()
     ev1.record(stream)
     torch.cuda.synchronize()
+    t_host1 = time.perf_counter()
     barrier()
-    clk = clocks.stop()
+    clk = clocks.stop(t_host0, t_host1)
     elapsed = max_over_ranks(ev0.elapsed_time(ev1) * 1e-3)
     per_graph = [(ev_graph[i].elapsed_time(ev_graph[i + 1]) if i + 1 < n_main else None)
                  for i in range(n_main)]
@@ -950,6 +1026,7 @@ def run_chain(args, rank, world, local_rank):
     rank_barrier(world)
     torch.cuda.synchronize()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t_host0 = time.perf_counter()
     torch.cuda._sleep(int(2e7))
     ev0.record(stream)
     for _ in range(n_full):
@@ -958,8 +1035,9 @@ def run_chain(args, rank, world, local_rank):
         g_rest.replay()
     ev1.record(stream)
     torch.cuda.synchronize()
+    t_host1 = time.perf_counter()
     rank_barrier(world)
-    clk = clocks.stop()
+    clk = clocks.stop(t_host0, t_host1)
     elapsed = rank_max(ev0.elapsed_time(ev1) * 1e-3, world, dev)
     value = job_tflops(wl.flops, args.steps, world, elapsed)
 

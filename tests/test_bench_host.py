@@ -60,3 +60,72 @@ def test_traffic_table_entries_are_well_formed():
 def test_job_tflops():
     # 2 ranks x 10 steps x 1e12 FLOP over the slowest rank's 4 s
     assert bench.job_tflops(1e12, 10, 2, 4.0) == pytest.approx(5.0)
+
+
+class _FakeNvml:
+    """Stands in for pynvml: the clock and reasons it reports are those of the
+    phase the test sets (before, inside or after the timed region)."""
+    NVML_CLOCK_SM = 1
+    nvmlClocksEventReasonHwSlowdown = 0x8
+    nvmlClocksEventReasonHwThermalSlowdown = 0x40
+    nvmlClocksEventReasonSwThermalSlowdown = 0x20
+    nvmlClocksEventReasonSwPowerCap = 0x4
+    PHASES = {"before": (700.0, 0x0), "inside": (1900.0, 0x4), "after": (600.0, 0x8)}
+
+    def __init__(self):
+        self.phase = "before"
+        self.shut = False
+
+    def nvmlInit(self):
+        pass
+
+    def nvmlShutdown(self):
+        self.shut = True
+
+    def nvmlDeviceGetHandleByPciBusId(self, bus):
+        raise RuntimeError("no such bus here")
+
+    def nvmlDeviceGetHandleByIndex(self, i):
+        return ("gpu", i)
+
+    def nvmlDeviceGetMaxClockInfo(self, h, kind):
+        return 1965
+
+    def nvmlDeviceGetClockInfo(self, h, kind):
+        return self.PHASES[self.phase][0]
+
+    def nvmlDeviceGetCurrentClocksEventReasons(self, h):
+        return self.PHASES[self.phase][1]
+
+
+
+def test_clock_sampler_keeps_only_the_timed_region(monkeypatch):
+    import sys
+    import time
+    fake = _FakeNvml()
+    monkeypatch.setitem(sys.modules, "pynvml", fake)
+    c = bench.ClockSampler(0)
+    c.start()
+    time.sleep(0.05)
+    fake.phase = "inside"
+    time.sleep(0.01)  # let a sample of the old phase drain
+    t0 = time.perf_counter()
+    time.sleep(0.06)
+    t1 = time.perf_counter()
+    time.sleep(0.01)
+    fake.phase = "after"
+    time.sleep(0.05)
+    clk = c.stop(t0, t1)
+    assert fake.shut
+    assert clk["sm_mhz"] == 1900.0 and clk["sm_max_mhz"] == 1965.0
+    assert clk["reasons"] == ["sw_power_cap"]
+    assert clk["samples"] >= 3 and clk["source"].startswith("nvml")
+
+
+def test_clock_sampler_without_nvml_or_smi_reports_none(monkeypatch):
+    import sys
+    monkeypatch.setitem(sys.modules, "pynvml", None)  # import fails
+    monkeypatch.setenv("PATH", "/nonexistent")          # and nvidia-smi cannot start
+    c = bench.ClockSampler(0)
+    c.start()
+    assert c.stop() is None
