@@ -21,7 +21,8 @@ bandwidth when its arithmetic intensity is below the ridge (few tokens);
 standalone kernel on the same activations when the layers quantise inside their one
 kernel); both from CUDA events around each kernel launch in an attribution pass over
 the same steps. ``step_ms_spread`` = median / p10 / p90 of the step time over the
-replayed graphs of the timed region.
+replayed graphs of the timed region. ``clocks`` = the median SM clock and the
+throttle reasons seen inside the timed region (NVML read every 5 ms from a thread).
 
 --impl reference times the CPU oracle (the plain C implementation that
 defines the results) on a bounded row sample of the same workload.
