@@ -129,3 +129,39 @@ def test_clock_sampler_without_nvml_or_smi_reports_none(monkeypatch):
     c = bench.ClockSampler(0)
     c.start()
     assert c.stop() is None
+
+
+def _profile_bench_commands():
+    """Every `python bench.py ...` command quoted in the profile summaries, with shell line
+    continuations joined; W in the few-row summary stands for each workload named there."""
+    import glob
+    import re
+    import shlex
+    cmds = []
+    for path in sorted(glob.glob(os.path.join(bench.ROOT, "profiles", "*.md"))):
+        text = open(path).read().replace("\\\n", " ")
+        for line in text.splitlines():
+            for m in re.finditer(r"python bench\.py([^`\n]*)", line):
+                args = shlex.split(m.group(1).split(">")[0])
+                subs = ["llm_small_m1", "llm_small_m16", "llm_small_m128"] if "W" in args else [None]
+                for w in subs:
+                    cmds.append((os.path.basename(path),
+                                 [w if (a == "W" and w) else a for a in args]))
+    return cmds
+
+
+def test_profile_commands_parse_with_the_current_bench(monkeypatch):
+    import sys
+    cmds = _profile_bench_commands()
+    assert len(cmds) >= 10
+    for name, args in cmds:
+        monkeypatch.setattr(sys, "argv", ["bench.py"] + args)
+        try:
+            a = bench.parse()
+        except SystemExit:
+            raise AssertionError(f"{name}: bench.py {' '.join(args)} no longer parses")
+        assert a.workload in bench.synth.WORKLOADS
+        # a summary named for one workload quotes commands that run that workload
+        named = [w for w in bench.synth.WORKLOADS if w in name]
+        if named:
+            assert a.workload == max(named, key=len), f"{name}: runs {a.workload}"
